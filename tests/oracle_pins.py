@@ -1,0 +1,299 @@
+"""Pins of the CPU oracle to things other than itself.
+
+Each ``pin_*`` takes an ``oracle.Oracle`` and raises AssertionError when the
+oracle disagrees with a closed form, an invariant, a textbook routine or an
+independent brute-force formulation.  ``test_oracle_pins.py`` runs them on
+the real oracle; ``test_oracle_mutations.py`` runs them on copies of the
+oracle with planted mistakes and checks that every mistake is caught.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import qsa_inputs as Q
+
+SQRT_D = math.sqrt(128.0)
+
+
+def _bf(x):
+    """bf16 bits of values that are exactly representable."""
+    b = Q.f32_to_bf16(np.asarray(x, dtype=np.float32))
+    assert np.array_equal(Q.bf16_to_f32(b), np.asarray(x, dtype=np.float32)), "not bf16-exact"
+    return b
+
+
+def _rope_complex(x: np.ndarray, pos: int, theta=1e7, rope_dim=64) -> np.ndarray:
+    """RoPE as complex multiplication: z_i = x_i + i x_{i+32} times e^{i pos theta^(-i/32)}."""
+    half = rope_dim // 2
+    y = np.array(x, dtype=np.float64, copy=True)
+    z = x[..., :half] + 1j * x[..., half:rope_dim]
+    f = theta ** (-np.arange(half) / half)
+    z = z * np.exp(1j * pos * f)
+    y[..., :half] = z.real
+    y[..., half:rope_dim] = z.imag
+    return y
+
+
+# --------------------------------------------------------------------- RoPE
+def pin_rope_identity_at_zero(O):
+    x = np.random.default_rng(1).standard_normal(256)
+    assert np.array_equal(O.rope(x, 0), x)
+
+
+def pin_rope_norm_and_tail(O):
+    x = np.random.default_rng(2).standard_normal(256)
+    for pos in (1, 7, 4095, 262143, 1048575):
+        y = O.rope(x, pos)
+        assert abs(np.linalg.norm(y) - np.linalg.norm(x)) < 1e-12 * np.linalg.norm(x)
+        assert np.array_equal(y[64:], x[64:]), "dims beyond rope_dim must be untouched"
+        # each (i, i+32) pair keeps its own length
+        assert np.allclose(np.hypot(y[:32], y[32:64]), np.hypot(x[:32], x[32:64]), rtol=1e-13)
+
+
+def pin_rope_complex_form(O):
+    """Rotate-half pairs, frequency theta^(-2i/64), theta = 1e7: as complex rotations."""
+    rng = np.random.default_rng(3)
+    for pos in (1, 3, 1000, 262144, 1048575):
+        x = rng.standard_normal(256)
+        assert np.allclose(O.rope(x, pos), _rope_complex(x, pos), rtol=0, atol=1e-9), pos
+
+
+def pin_rope_relative(O):
+    """(R_m q).(R_n k) depends only on m - n."""
+    rng = np.random.default_rng(4)
+    q, k = rng.standard_normal(256), rng.standard_normal(256)
+    for m, n in ((5, 2), (1000, 10), (700000, 699990)):
+        a = O.rope(q, m) @ O.rope(k, n)
+        b = O.rope(q, m - n) @ k
+        assert abs(a - b) < 1e-8 * (abs(b) + 1), (m, n, a, b)
+
+
+# ------------------------------------------------------------------- scores
+def pin_token_score_closed_form(O):
+    """q_h = a_h e_0, k = b e_0: s = sum_h w_h max(0, a_h b) / sqrt(128)."""
+    a = np.array([2.0, -3.0, 0.5, 4.0])
+    b = 1.5
+    w = np.array([0.25, 0.5, 0.125, 0.125])
+    q = np.zeros((4, 128)); q[:, 0] = a
+    k = np.zeros(128); k[0] = b
+    want = sum(w[h] * max(0.0, a[h] * b) for h in range(4)) / SQRT_D
+    got = O.token_score(_bf(q), _bf(w), _bf(k))
+    assert abs(got - want) < 1e-15, (got, want)
+    # the key element other than dim 0 matters too (no dropped dims)
+    k2 = k.copy(); k2[127] = 2.0
+    q2 = q.copy(); q2[3, 127] = 1.0
+    want2 = sum(w[h] * max(0.0, a[h] * b + (2.0 if h == 3 else 0.0)) for h in range(4)) / SQRT_D
+    got2 = O.token_score(_bf(q2), _bf(w), _bf(k2))
+    assert abs(got2 - want2) < 1e-15, (got2, want2)
+
+
+def _matrix_scores(q_idx, w, k_idx, r=4):
+    """Brute force in matrix form: all token pairs at once, then block max."""
+    T = q_idx.shape[0]
+    qf, wf, kf = Q.bf16_to_f64(q_idx), Q.bf16_to_f64(w), Q.bf16_to_f64(k_idx)
+    dots = np.einsum("thc,jc->thj", qf, kf)                    # [T][4][T]
+    s = (wf[:, :, None] * np.maximum(dots, 0.0)).sum(1) / SQRT_D  # [T][T]
+    causal = np.tril(np.ones((T, T), dtype=bool))
+    s = np.where(causal, s, -np.inf)
+    nb = (T + r - 1) // r
+    pad = np.full((nb * r, nb * r), -np.inf)
+    pad[:T, :T] = s
+    S = pad.reshape(nb, r, nb, r).max(axis=(1, 3))
+    S[np.triu(np.ones((nb, nb), dtype=bool), 1)] = np.nan
+    return S
+
+
+def pin_block_scores_brute(O):
+    for T, seed in ((1, 0), (5, 1), (13, 2), (64, 3), (67, 4)):
+        P = Q.PrefillProblem(T=T, seed=seed, n_plant=2)
+        q_idx, w, k_idx = P.q_idx(), P.w(), P.k_idx()
+        want = _matrix_scores(q_idx, w, k_idx)
+        got = O.index_scores(T, q_idx, w, k_idx)
+        m = ~np.isnan(want)
+        assert np.array_equal(m, ~np.isnan(got)), T
+        assert np.allclose(got[m], want[m], rtol=1e-12, atol=1e-14), T
+
+
+def pin_block_scores_page_formula(O):
+    """Block size 1 and constant head weight c: S * sqrt(128) / c is the
+    indexer score I_ib = sum_h ReLU(<q_i^h, k_b>) with the block key = the key."""
+    import oracle as OR
+    P1 = OR.params(block=1, budget=O.P.budget)
+    O1 = type(O)(P1, O.L)
+    T = 23
+    P = Q.PrefillProblem(T=T, seed=5)
+    q_idx, k_idx = P.q_idx(), P.k_idx()
+    c = 8.0
+    w = _bf(np.full((T, 4), c))
+    S = O1.index_scores(T, q_idx, w, k_idx)
+    qf, kf = Q.bf16_to_f64(q_idx), Q.bf16_to_f64(k_idx)
+    I = np.maximum(np.einsum("thc,jc->thj", qf, kf), 0.0).sum(1)   # [T][T]
+    for i in range(T):
+        for b in range(i + 1):
+            assert abs(S[i, b] * SQRT_D / c - I[i, b]) < 1e-10 * (1 + abs(I[i, b])), (i, b)
+
+
+def pin_identical_keys_block(O):
+    """A key block of four identical keys scores the max over query tokens of
+    the score against that one key; a block after the query is never scored."""
+    T = 16
+    P = Q.PrefillProblem(T=T, seed=6)
+    q_idx, w, k_idx = P.q_idx(), P.w(), P.k_idx().copy()
+    k_idx[4:8] = k_idx[5]
+    S = O.index_scores(T, q_idx, w, k_idx)
+    for qb in (1, 2, 3):
+        want = max(O.token_score(q_idx[t], w[t], k_idx[5]) for t in range(4 * qb, 4 * qb + 4))
+        assert abs(S[qb, 1] - want) < 1e-14 * (1 + want)
+    # own block: token 4qb sees only key 4qb
+    for qb in range(4):
+        t0 = 4 * qb
+        want = max(O.token_score(q_idx[t], w[t], k_idx[j]) for t in range(t0, t0 + 4) for j in range(t0, t + 1))
+        assert abs(S[qb, qb] - want) < 1e-14 * (1 + want)
+
+
+# ---------------------------------------------------------------- selection
+def _select_lexsort(S_row, qb, budget):
+    if qb + 1 <= budget:
+        return np.arange(qb + 1)
+    cand = np.arange(qb - 1)
+    order = np.lexsort((cand, -S_row[:qb - 1]))      # score desc, index asc
+    top = cand[order[:budget - 2]]
+    return np.sort(np.concatenate([top, [qb - 1, qb]]))
+
+
+def pin_select_vs_lexsort(O):
+    rng = np.random.default_rng(7)
+    B = O.P.budget
+    for qb in (0, 1, B - 2, B - 1, B, B + 1, B + 5, 3 * B + 7):
+        S = rng.random(qb + 1).round(2)            # many ties
+        sel, cnt = O.select(qb, S)
+        want = _select_lexsort(S, qb, B)
+        assert cnt == len(want), (qb, cnt)
+        assert np.array_equal(sel[:cnt], want), qb
+        assert (sel[cnt:] == -1).all()
+
+
+def pin_select_invariants(O):
+    rng = np.random.default_rng(8)
+    B = O.P.budget
+    for qb in (B - 1, B, 2 * B + 3):
+        S = rng.random(qb + 1)
+        sel, cnt = O.select(qb, S)
+        s = sel[:cnt]
+        assert cnt == min(B, qb + 1)
+        assert np.all(np.diff(s) > 0)
+        assert qb in s and (qb - 1 in s or qb == 0)
+        if qb + 1 > B:
+            free_sel = [b for b in s if b < qb - 1]
+            unsel = np.setdiff1d(np.arange(qb - 1), s)
+            assert min(S[free_sel]) >= max(S[unsel])
+    # all scores equal: the lowest indices win
+    qb = 3 * B
+    sel, cnt = O.select(qb, np.zeros(qb + 1))
+    assert np.array_equal(sel[:cnt], np.concatenate([np.arange(B - 2), [qb - 1, qb]]))
+
+
+# ---------------------------------------------------------------- attention
+def _dense_causal_sdpa(q, k, v, pos0=0):
+    """Dense causal GQA attention via torch's SDPA in fp64 on complex-form RoPE."""
+    T = q.shape[0]
+    qf = np.stack([_rope_complex(Q.bf16_to_f64(q[t]), pos0 + t) for t in range(T)])   # [T][24][256]
+    kf = np.stack([_rope_complex(Q.bf16_to_f64(k[t]), pos0 + t) for t in range(T)])   # [T][2][256]
+    vf = Q.bf16_to_f64(v)
+    qt = torch.from_numpy(qf).permute(1, 0, 2)[None]
+    kt = torch.from_numpy(kf).permute(1, 0, 2).repeat_interleave(12, dim=0)[None]
+    vt = torch.from_numpy(vf).permute(1, 0, 2).repeat_interleave(12, dim=0)[None]
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True)
+    logits = torch.einsum("bhtc,bhjc->bhtj", qt, kt) / 16.0
+    logits = logits.masked_fill(~torch.tril(torch.ones(T, T, dtype=torch.bool)), float("-inf"))
+    lse = torch.logsumexp(logits, dim=-1)
+    return o[0].permute(1, 0, 2).numpy(), lse[0].permute(1, 0).numpy()
+
+
+def pin_attention_dense_when_budget_covers(O):
+    """Budget >= number of blocks: QSA is dense causal attention."""
+    import oracle as OR
+    for T, pos0 in ((37, 0), (64, 0), (21, 1000)):
+        Ob = type(O)(OR.params(budget=64), O.L)
+        P = Q.PrefillProblem(T=T, seed=9, n_plant=3)
+        h = P.host()
+        sel, cnt, out, lse = Ob.prefill_blocks(T, h["q"], h["k"], h["v"], h["q_idx"], h["w"], h["k_idx"], pos0=pos0)
+        want_o, want_l = _dense_causal_sdpa(h["q"], h["k"], h["v"], pos0)
+        assert np.allclose(out[:T], want_o, rtol=1e-10, atol=1e-12), T
+        assert np.allclose(lse[:T], want_l, rtol=1e-10, atol=1e-12), T
+
+
+def pin_attention_constant_v_and_single_key(O):
+    T = 12
+    P = Q.PrefillProblem(T=T, seed=10)
+    q, k = P.q(), P.k()
+    vv = np.zeros((T, 2, 256), dtype=np.float32)
+    vv[:, 0, :] = 0.75
+    vv[:, 1, :] = np.linspace(-2, 2, 256, dtype=np.float32).round(2)
+    v = Q.f32_to_bf16(vv)
+    sel = np.tile(np.arange(O.P.budget, dtype=np.int32), (3, 1))
+    sel[:, 3:] = -1
+    cnt = np.full(3, 3, np.int32)
+    out, lse = O.attend_blocks(T, q, k, v, np.arange(3), sel, cnt)
+    vf = Q.bf16_to_f64(v)
+    assert np.allclose(out[:, :12, :], vf[0, 0], atol=1e-12)
+    assert np.allclose(out[:, 12:, :], vf[0, 1], atol=1e-12)
+    # token 0 has a single key: out = v_0, lse = its logit
+    vr = P.v()
+    out, lse = O.attend_blocks(T, q, k, vr, np.arange(1), sel[:1], cnt[:1])
+    vf = Q.bf16_to_f64(vr)
+    for h in range(24):
+        assert np.allclose(out[0, h], vf[0, h // 12], atol=1e-13)
+        logit = (Q.bf16_to_f64(q[0, h]) @ Q.bf16_to_f64(k[0, h // 12])) / 16.0   # RoPE is the identity at 0
+        assert abs(lse[0, h] - logit) < 1e-12
+
+
+def pin_attention_respects_selection(O):
+    """Keys outside the selected blocks do not influence the output."""
+    T = 32
+    P = Q.PrefillProblem(T=T, seed=11)
+    q, k, v = P.q(), P.k(), P.v()
+    qb = 7
+    sel = np.full((1, O.P.budget), -1, np.int32)
+    sel[0, :3] = [1, 4, 7]
+    cnt = np.array([3], np.int32)
+    out1, _ = O.attend_blocks(T, q, k, v, [qb], sel, cnt)
+    k2, v2 = k.copy(), v.copy()
+    for b in (0, 2, 3, 5, 6):
+        k2[4 * b: 4 * b + 4] = 0x3F80
+        v2[4 * b: 4 * b + 4] = 0x4000
+    out2, _ = O.attend_blocks(T, q, k2, v2, [qb], sel, cnt)
+    assert np.array_equal(out1, out2)
+    # and the keys that are selected do
+    v3 = v.copy(); v3[4 * 4] = 0x4000
+    out3, _ = O.attend_blocks(T, q, k, v3, [qb], sel, cnt)
+    assert not np.array_equal(out1, out3)
+
+
+# ------------------------------------------------------------------- decode
+def pin_decode_equals_prefill_last(O):
+    """Decode of token L over caches (keys rotated then rounded to bf16) gives
+    prefill's token-L output, up to that rounding; the selection is exact."""
+    import oracle as OR
+    for L in (40, 41, 43, 70):
+        Ob = type(O)(OR.params(budget=8), O.L)
+        T = L + 1
+        P = Q.PrefillProblem(T=T, seed=12 + L, n_plant=2)
+        h = P.host()
+        qb = L // 4
+        sel, cnt, out, lse = Ob.prefill_blocks(T, h["q"], h["k"], h["v"], h["q_idx"], h["w"], h["k_idx"], [qb])
+        kf = np.stack([_rope_complex(Q.bf16_to_f64(h["k"][t]), t) for t in range(L)])
+        k_cache = Q.f32_to_bf16(kf.astype(np.float32))
+        t0 = qb * 4
+        dsel, dcnt, dout, dlse = Ob.decode(L, k_cache, h["v"][:L], h["k_idx"][:L], h["q_idx"][t0:L], h["w"][t0:L],
+                                           h["q"][L], h["k"][L], h["v"][L], h["q_idx"][L], h["k_idx"][L], h["w"][L])
+        assert dcnt == cnt[0] and np.array_equal(dsel, sel[0]), L
+        i = L - t0
+        assert np.abs(dout - out[i]).max() < 2e-2
+        assert np.linalg.norm(dout - out[i]) < 5e-3 * np.linalg.norm(out[i])
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -1,0 +1,56 @@
+"""Plant plausible mistakes in copies of the oracle (on the CPU) and check that
+the pins catch every one of them."""
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+import oracle
+from oracle_pins import ALL_PINS
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
+
+# (name, exact text in oracle.c, replacement)
+MUTANTS = [
+    ("relu_dropped", "double relu = dot > 0.0 ? dot : 0.0;", "double relu = dot;"),
+    ("head_weight_dropped", "s += bf16_to_f64(w_t[h]) * relu;", "s += relu;"),
+    ("score_scale_dropped", "return s / sqrt((double)p->idx_dim);", "return s;"),
+    ("causal_off_by_one", "if (j > t) continue;", "if (j > t + 1) continue;"),
+    ("block_sum_not_max", "if (s > best) best = s;", "best = (best < 0.0 ? 0.0 : best) + s;"),
+    ("key_dim_dropped", "for (int c = 0; c < p->idx_dim; ++c) dot +=", "for (int c = 1; c < p->idx_dim; ++c) dot +="),
+    ("rope_sign", "y[i] = x[i] * ca - x[i + half] * sa;", "y[i] = x[i] * ca + x[i + half] * sa;"),
+    ("rope_pairing", "y[i + half] = x[i + half] * ca + x[i] * sa;", "y[i + half] = x[i + half] * ca + x[(i + 1) % half] * sa;"),
+    ("rope_freq", "pow(p->rope_theta, -2.0 * (double)i / (double)p->rope_dim)", "pow(p->rope_theta, -1.0 * (double)i / (double)p->rope_dim)"),
+    ("tie_to_higher_index", "return (x->idx > y->idx) - (x->idx < y->idx);", "return (x->idx < y->idx) - (x->idx > y->idx);"),
+    ("prev_block_not_forced", "for (int i = 0; i < budget - 2; ++i) sel[n++] = (int32_t)c[i].idx;\n  sel[n++] = (int32_t)(qb - 1);",
+     "for (int i = 0; i < budget - 1; ++i) sel[n++] = (int32_t)c[i].idx;"),
+    ("select_ascending_score", "if (x->s > y->s) return -1;\n  if (x->s < y->s) return 1;", "if (x->s < y->s) return -1;\n  if (x->s > y->s) return 1;"),
+    ("attn_scale", "1.0 / sqrt((double)d)", "1.0 / (double)d"),
+    ("gqa_map", "int g = h / (H / G);", "int g = h % G;"),
+    ("lse_max_dropped", "lse[h] = m + log(z);", "lse[h] = log(z);"),
+    ("causal_attn_off_by_one", "if (j <= t) js[n++] = j;", "if (j <= t + 1) js[n++] = j;"),
+    ("value_head_swap", "vv[(e * G + g) * d + c] = bf16_to_f64(v[(js[e] * G + g) * d + c]);",
+     "vv[(e * G + g) * d + c] = bf16_to_f64(v[(js[e] * G + (G - 1 - g)) * d + c]);"),
+    ("decode_new_key_position", "oracle_rope(p, x, L, kr + (e * G + g) * d);", "oracle_rope(p, x, L - 1, kr + (e * G + g) * d);"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation anchor not found: {name}"
+    mutated = src.replace(old, new)
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "m.c")
+        so = os.path.join(d, "m.so")
+        open(c, "w").write(mutated)
+        subprocess.run(["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-std=c11", c, "-o", so, "-lm"], check=True)
+        O = oracle.Oracle(L=oracle.load_variant(so))
+        failed = []
+        for pin in ALL_PINS:
+            try:
+                pin(O)
+            except AssertionError:
+                failed.append(pin.__name__)
+        assert failed, f"mutant {name} passed every pin"
