@@ -1,0 +1,184 @@
+"""Python binding of libqsa.so, the C-ABI QSA hot path for B200 (sm_100a).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind ``include/qsa.h``.  PyTorch supplies device memory and the
+current stream.  The entry points keep the C names (``qsa_prefill`` ...)
+and take torch tensors; bf16 data may be ``torch.bfloat16`` or ``torch.uint16``
+(bit patterns).  If libqsa.so is missing this module raises on first use:
+there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqsa.so")
+
+QSA_OK = 0
+_STATUS = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_UNSUPPORTED", 3: "QSA_ERR_MISALIGNED",
+           4: "QSA_ERR_WORKSPACE_TOO_SMALL", 5: "QSA_ERR_CUDA", 6: "QSA_ERR_DEVICE_TIMEOUT",
+           7: "QSA_ERR_DEVICE_BOUNDS", 8: "QSA_ERR_ARCH"}
+
+EXPORTED = ["qsa_default_params", "qsa_status_string", "qsa_index_scores", "qsa_select_blocks",
+            "qsa_select_workspace_size", "qsa_prefill", "qsa_prefill_workspace_size", "qsa_decode",
+            "qsa_decode_workspace_size", "qsa_check_device_error"]
+
+
+class QSAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_STATUS.get(status, status)}")
+
+
+class qsa_params(ctypes.Structure):
+    _fields_ = [("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("rope_dim", ctypes.c_int32), ("rope_theta", ctypes.c_double), ("idx_heads", ctypes.c_int32),
+                ("idx_dim", ctypes.c_int32), ("block_size", ctypes.c_int32), ("budget_blocks", ctypes.c_int32),
+                ("softmax_scale", ctypes.c_float)]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libqsa.so and declare its signatures (raises if it is not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m block_sparse_long_qsa_b200._build` "
+                          "(the QSA path has no non-CUDA fallback)")
+    L = ctypes.CDLL(path)
+    P, vp, i64, i32, sz = ctypes.POINTER(qsa_params), ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+    psz = ctypes.POINTER(ctypes.c_size_t)
+    L.qsa_default_params.argtypes = [P]
+    L.qsa_default_params.restype = None
+    L.qsa_status_string.argtypes = [ctypes.c_int]
+    L.qsa_status_string.restype = ctypes.c_char_p
+    L.qsa_index_scores.argtypes = [P, i64, vp, vp, vp, i64, i64, vp, i64, vp, sz, vp]
+    L.qsa_select_blocks.argtypes = [P, vp, i64, i64, i64, vp, vp, vp, sz, vp]
+    L.qsa_select_workspace_size.argtypes = [P, psz]
+    L.qsa_prefill.argtypes = [P, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.qsa_prefill_workspace_size.argtypes = [P, i64, psz, psz]
+    L.qsa_decode.argtypes = [P, i32, i64, ctypes.POINTER(ctypes.c_int64), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                             vp, vp, vp, vp, sz, vp]
+    L.qsa_decode_workspace_size.argtypes = [P, i32, i64, psz]
+    L.qsa_check_device_error.argtypes = [vp, vp]
+    for f in EXPORTED:
+        if f not in ("qsa_default_params", "qsa_status_string"):
+            getattr(L, f).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def params(budget: int = 512, **kw) -> qsa_params:
+    p = qsa_params()
+    load().qsa_default_params(ctypes.byref(p))
+    p.budget_blocks = budget
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("QSA tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc: int, where: str):
+    if rc != QSA_OK:
+        raise QSAError(rc, where)
+
+
+# ------------------------------------------------------------ raw entry points
+def qsa_status_string(status: int) -> str:
+    return load().qsa_status_string(status).decode()
+
+
+def qsa_index_scores(p: qsa_params, T: int, q_idx, w, k_idx, qb_begin: int, qb_end: int, scores, ld: int,
+                     ws=None, stream=None):
+    _check(load().qsa_index_scores(ctypes.byref(p), T, _ptr(q_idx), _ptr(w), _ptr(k_idx), qb_begin, qb_end,
+                                   _ptr(scores), ld, _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                                   _stream(stream)), "qsa_index_scores")
+
+
+def qsa_select_workspace_size(p: qsa_params) -> int:
+    n = ctypes.c_size_t()
+    _check(load().qsa_select_workspace_size(ctypes.byref(p), ctypes.byref(n)), "qsa_select_workspace_size")
+    return n.value
+
+
+def qsa_select_blocks(p: qsa_params, scores, ld: int, qb_begin: int, qb_end: int, sel, cnt, ws, stream=None):
+    _check(load().qsa_select_blocks(ctypes.byref(p), _ptr(scores), ld, qb_begin, qb_end, _ptr(sel), _ptr(cnt),
+                                    _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "qsa_select_blocks")
+
+
+def qsa_prefill_workspace_size(p: qsa_params, T: int) -> tuple[int, int]:
+    a, b = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(load().qsa_prefill_workspace_size(ctypes.byref(p), T, ctypes.byref(a), ctypes.byref(b)),
+           "qsa_prefill_workspace_size")
+    return a.value, b.value
+
+
+def qsa_prefill(p: qsa_params, T: int, pos0: int, q, k, v, q_idx, w, k_idx, out, lse=None, sel_out=None,
+                cnt_out=None, k_rot_out=None, ws=None, stream=None):
+    _check(load().qsa_prefill(ctypes.byref(p), T, pos0, _ptr(q), _ptr(k), _ptr(v), _ptr(q_idx), _ptr(w), _ptr(k_idx),
+                              _ptr(out), _ptr(lse), _ptr(sel_out), _ptr(cnt_out), _ptr(k_rot_out), _ptr(ws),
+                              ws.numel() * ws.element_size(), _stream(stream)), "qsa_prefill")
+
+
+def qsa_decode_workspace_size(p: qsa_params, B: int, max_len: int) -> int:
+    n = ctypes.c_size_t()
+    _check(load().qsa_decode_workspace_size(ctypes.byref(p), B, max_len, ctypes.byref(n)), "qsa_decode_workspace_size")
+    return n.value
+
+
+def qsa_decode(p: qsa_params, B: int, max_len: int, cache_len, k_cache, v_cache, kidx_cache, qidx_ring, w_ring,
+               q_new, k_new, v_new, q_idx_new, k_idx_new, w_new, out, sel_out=None, lse_out=None, ws=None,
+               stream=None):
+    """``cache_len``: host sequence of B ints (lengths before this token)."""
+    lens = (ctypes.c_int64 * B)(*[int(x) for x in cache_len])
+    _check(load().qsa_decode(ctypes.byref(p), B, max_len, lens, _ptr(k_cache), _ptr(v_cache), _ptr(kidx_cache),
+                             _ptr(qidx_ring), _ptr(w_ring), _ptr(q_new), _ptr(k_new), _ptr(v_new), _ptr(q_idx_new),
+                             _ptr(k_idx_new), _ptr(w_new), _ptr(out), _ptr(sel_out), _ptr(lse_out), _ptr(ws),
+                             ws.numel() * ws.element_size(), _stream(stream)), "qsa_decode")
+
+
+def qsa_check_device_error(ws, stream=None) -> int:
+    return load().qsa_check_device_error(_ptr(ws), _stream(stream))
+
+
+# ----------------------------------------------------- allocating conveniences
+def workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def prefill(q, k, v, q_idx, w, k_idx, budget: int = 512, pos0: int = 0, want_lse=True, want_sel=True,
+            want_krot=False, ws_bytes: int | None = None, stream=None):
+    """Allocate outputs and a workspace, run qsa_prefill; returns a dict."""
+    T = q.shape[0]
+    dev = q.device
+    p = params(budget)
+    mn, pref = qsa_prefill_workspace_size(p, T)
+    ws = workspace(pref if ws_bytes is None else max(ws_bytes, mn), dev)
+    nqb = (T + 3) // 4
+    res = dict(out=torch.empty((T, 24, 256), dtype=torch.uint16, device=dev))
+    res["lse"] = torch.empty((T, 24), dtype=torch.float32, device=dev) if want_lse else None
+    res["sel"] = torch.empty((nqb, budget), dtype=torch.int32, device=dev) if want_sel else None
+    res["cnt"] = torch.empty((nqb,), dtype=torch.int32, device=dev) if want_sel else None
+    res["k_rot"] = torch.empty((T, 2, 256), dtype=torch.uint16, device=dev) if want_krot else None
+    qsa_prefill(p, T, pos0, q, k, v, q_idx, w, k_idx, res["out"], res["lse"], res["sel"], res["cnt"], res["k_rot"],
+                ws, stream)
+    res["ws"] = ws
+    return res

@@ -1,0 +1,414 @@
+// C ABI of the QSA hot path: argument validation, workspace planning, tensor
+// map encoding and kernel launches on the caller's stream.  Every entry point
+// validates on the host before launching anything and returns a qsa_status.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "qsa.h"
+#include "qsa_kernels.h"
+
+namespace {
+
+constexpr size_t HEADER_BYTES = 256;            // device error word + padding
+constexpr size_t ALIGN = 256;
+constexpr int DECODE_SPLIT = 16;
+constexpr int MAX_DEV = 64;
+
+size_t align_up(size_t x, size_t a = ALIGN) { return (x + a - 1) / a * a; }
+int64_t round4(int64_t x) { return (x + 3) / 4 * 4; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+qsa_status check_params(const qsa_params* p) {
+  if (!p) return QSA_ERR_INVALID_ARG;
+  if (p->n_q_heads != 24 || p->n_kv_heads != 2 || p->head_dim != 256 || p->rope_dim != 64 || p->idx_heads != 4 ||
+      p->idx_dim != 128 || p->block_size != 4)
+    return QSA_ERR_UNSUPPORTED;
+  if (!(p->rope_theta > 1.0) || !std::isfinite(p->rope_theta)) return QSA_ERR_INVALID_ARG;
+  if (p->budget_blocks < 2 || p->budget_blocks > 4096) return QSA_ERR_UNSUPPORTED;
+  if (!(p->softmax_scale >= 0.f) || !std::isfinite(p->softmax_scale)) return QSA_ERR_INVALID_ARG;
+  return QSA_OK;
+}
+
+float softmax_scale(const qsa_params* p) {
+  return p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt((float)p->head_dim);
+}
+
+void inv_freq(const qsa_params* p, double* f) {
+  const int half = p->rope_dim / 2;
+  for (int i = 0; i < half; ++i) f[i] = std::pow(p->rope_theta, -2.0 * (double)i / (double)p->rope_dim);
+}
+
+// --------------------------------------------------------------- device info
+struct DevInfo {
+  bool known = false;
+  bool sm100 = false;
+  int num_sms = 0;
+};
+DevInfo g_dev[MAX_DEV];
+std::mutex g_dev_mu;
+
+qsa_status device_info(DevInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QSA_ERR_CUDA;
+  if (dev < 0 || dev >= MAX_DEV) return QSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.known) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return QSA_ERR_CUDA;
+    d.sm100 = (major == 10 && minor == 0);
+    d.num_sms = sms;
+    d.known = true;
+  }
+  *out = d;
+  return d.sm100 ? QSA_OK : QSA_ERR_ARCH;
+}
+
+// ---------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2D bf16 tensor [rows][cols] (row-major), box [box_rows][box_cols], 128B swizzle.
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                 uint32_t box_cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// 1D bf16 array of n elements, box of `box` elements.
+bool make_map_1d(CUtensorMap* m, const void* base, uint64_t n, uint32_t box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[1] = {n};
+  cuuint32_t boxd[1] = {box};
+  cuuint32_t estr[1] = {1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 1, const_cast<void*>(base), dims, nullptr, boxd, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+qsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA; }
+
+// Indexer launch for query blocks [qb0, qb1) into S (ld), maps built here.
+qsa_status run_indexer(int64_t T, const uint16_t* q_idx, const uint16_t* w, const uint16_t* k_idx, int64_t qb0,
+                       int64_t qb1, float* S, int64_t ld, uint32_t* err, int num_sms, cudaStream_t st) {
+  if (qb1 <= qb0) return QSA_OK;
+  CUtensorMap tq, tk, tw;
+  if (!make_map_2d(&tq, q_idx, (uint64_t)T * 4, 128, 256, 64) || !make_map_2d(&tk, k_idx, (uint64_t)T, 128, 128, 64) ||
+      !make_map_1d(&tw, w, (uint64_t)T * 4, 256))
+    return QSA_ERR_CUDA;
+  const float scale = 1.0f / std::sqrt(128.0f);
+  return from_cuda(qsa::launch_indexer_prefill(tq, tk, tw, S, ld, T, qb0, qb1, scale, err, num_sms, st));
+}
+
+// ------------------------------------------------------------ prefill layout
+struct PrefillLayout {
+  size_t cs, k_rot, sel, cnt, slab, total_fixed;
+};
+PrefillLayout prefill_layout(int64_t T, int budget, bool need_krot, bool need_sel, bool need_cnt) {
+  const int64_t nqb = (T + 3) / 4;
+  PrefillLayout L;
+  size_t off = HEADER_BYTES;
+  L.cs = off; off = align_up(off + (size_t)T * 32 * sizeof(float2));
+  L.k_rot = off; off = align_up(off + (need_krot ? (size_t)T * 1024 : 0));
+  L.sel = off; off = align_up(off + (need_sel ? (size_t)nqb * budget * 4 : 0));
+  L.cnt = off; off = align_up(off + (need_cnt ? (size_t)nqb * 4 : 0));
+  L.slab = off;
+  L.total_fixed = off;
+  return L;
+}
+// largest qb1 in (qb0, nqb] whose slab (qb1-qb0) x round4(qb1) x 4 fits
+int64_t chunk_end(int64_t qb0, int64_t nqb, size_t slab_bytes) {
+  int64_t lo = qb0 + 1, hi = nqb;
+  if ((size_t)1 * round4(lo) * 4 > slab_bytes) return qb0;  // not even one row
+  while (lo < hi) {
+    const int64_t mid = (lo + hi + 1) / 2;
+    if ((size_t)(mid - qb0) * (size_t)round4(mid) * 4 <= slab_bytes) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+constexpr int64_t MIN_ROWS = 64;
+constexpr size_t PREF_CAP = (size_t)16 << 30;
+
+}  // namespace
+
+extern "C" {
+
+void qsa_default_params(qsa_params* p) {
+  if (!p) return;
+  p->n_q_heads = 24;
+  p->n_kv_heads = 2;
+  p->head_dim = 256;
+  p->rope_dim = 64;
+  p->rope_theta = 1e7;
+  p->idx_heads = 4;
+  p->idx_dim = 128;
+  p->block_size = 4;
+  p->budget_blocks = 512;
+  p->softmax_scale = 0.f;
+}
+
+const char* qsa_status_string(qsa_status s) {
+  switch (s) {
+    case QSA_OK: return "ok";
+    case QSA_ERR_INVALID_ARG: return "invalid argument";
+    case QSA_ERR_UNSUPPORTED: return "unsupported shape";
+    case QSA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case QSA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case QSA_ERR_CUDA: return "CUDA error";
+    case QSA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case QSA_ERR_DEVICE_BOUNDS: return "device-side check failed";
+    case QSA_ERR_ARCH: return "device is not sm_100";
+  }
+  return "unknown status";
+}
+
+qsa_status qsa_index_scores(const qsa_params* p, int64_t T, const uint16_t* q_idx, const uint16_t* w,
+                            const uint16_t* k_idx, int64_t qb_begin, int64_t qb_end, float* scores, int64_t ld,
+                            void* ws, size_t ws_bytes, void* stream) {
+  qsa_status st = check_params(p);
+  if (st != QSA_OK) return st;
+  if (T <= 0 || T > ((int64_t)1 << 24)) return T <= 0 ? QSA_ERR_INVALID_ARG : QSA_ERR_UNSUPPORTED;
+  const int64_t nqb = (T + 3) / 4;
+  if (qb_begin < 0 || qb_end < qb_begin || qb_end > nqb || ld < qb_end || ld % 4 != 0) return QSA_ERR_INVALID_ARG;
+  if (!q_idx || !w || !k_idx || !scores) return QSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(w) || !aligned16(k_idx) || !aligned16(scores)) return QSA_ERR_MISALIGNED;
+  if (ws && ws_bytes < HEADER_BYTES) return QSA_ERR_WORKSPACE_TOO_SMALL;
+  if (ws && !aligned16(ws)) return QSA_ERR_MISALIGNED;
+  DevInfo di;
+  if ((st = device_info(&di)) != QSA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* err = static_cast<uint32_t*>(ws);
+  if (err && cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return QSA_ERR_CUDA;
+  return run_indexer(T, q_idx, w, k_idx, qb_begin, qb_end, scores, ld, err, di.num_sms, s);
+}
+
+qsa_status qsa_select_workspace_size(const qsa_params* p, size_t* bytes) {
+  qsa_status st = check_params(p);
+  if (st != QSA_OK) return st;
+  if (!bytes) return QSA_ERR_INVALID_ARG;
+  *bytes = HEADER_BYTES;
+  return QSA_OK;
+}
+
+qsa_status qsa_select_blocks(const qsa_params* p, const float* scores, int64_t ld, int64_t qb_begin, int64_t qb_end,
+                             int32_t* sel, int32_t* cnt, void* ws, size_t ws_bytes, void* stream) {
+  qsa_status st = check_params(p);
+  if (st != QSA_OK) return st;
+  if (qb_begin < 0 || qb_end < qb_begin || ld < qb_end || ld % 4 != 0) return QSA_ERR_INVALID_ARG;
+  if (!scores || !sel || !cnt || !ws) return QSA_ERR_INVALID_ARG;
+  if (!aligned16(scores) || !aligned16(sel) || !aligned16(cnt) || !aligned16(ws)) return QSA_ERR_MISALIGNED;
+  if (ws_bytes < HEADER_BYTES) return QSA_ERR_WORKSPACE_TOO_SMALL;
+  DevInfo di;
+  if ((st = device_info(&di)) != QSA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* err = static_cast<uint32_t*>(ws);
+  if (cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return QSA_ERR_CUDA;
+  return from_cuda(qsa::launch_select(scores, ld, qb_begin, qb_end - qb_begin, nullptr, p->budget_blocks, sel, cnt,
+                                      err, s));
+}
+
+qsa_status qsa_prefill_workspace_size(const qsa_params* p, int64_t T, size_t* min_bytes, size_t* pref_bytes) {
+  qsa_status st = check_params(p);
+  if (st != QSA_OK) return st;
+  if (T <= 0) return QSA_ERR_INVALID_ARG;
+  if (T > ((int64_t)1 << 24)) return QSA_ERR_UNSUPPORTED;
+  const int64_t nqb = (T + 3) / 4;
+  // worst case: the library keeps k_rot, sel and cnt itself
+  PrefillLayout L = prefill_layout(T, p->budget_blocks, true, true, true);
+  const int64_t min_rows = nqb < MIN_ROWS ? nqb : MIN_ROWS;
+  const size_t row_bytes = (size_t)round4(nqb) * 4;
+  if (min_bytes) *min_bytes = L.total_fixed + (size_t)min_rows * row_bytes;
+  if (pref_bytes) {
+    // whole triangle in one pass is nqb rows of round4(nqb); cap it
+    size_t full = (size_t)nqb * row_bytes;
+    size_t cap = PREF_CAP > (size_t)min_rows * row_bytes ? PREF_CAP : (size_t)min_rows * row_bytes;
+    *pref_bytes = L.total_fixed + (full < cap ? full : cap);
+  }
+  return QSA_OK;
+}
+
+qsa_status qsa_prefill(const qsa_params* p, int64_t T, int64_t pos0, const uint16_t* q, const uint16_t* k,
+                       const uint16_t* v, const uint16_t* q_idx, const uint16_t* w, const uint16_t* k_idx,
+                       uint16_t* out, float* lse, int32_t* sel_out, int32_t* cnt_out, uint16_t* k_rot_out, void* ws,
+                       size_t ws_bytes, void* stream) {
+  qsa_status st = check_params(p);
+  if (st != QSA_OK) return st;
+  if (T <= 0 || pos0 < 0) return QSA_ERR_INVALID_ARG;
+  if (T > ((int64_t)1 << 24) || pos0 + T > ((int64_t)1 << 40)) return QSA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !q_idx || !w || !k_idx || !out || !ws) return QSA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, q_idx, w, k_idx, out, lse, sel_out, cnt_out, k_rot_out, ws};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return QSA_ERR_MISALIGNED;
+  const int budget = p->budget_blocks;
+  const int64_t nqb = (T + 3) / 4;
+  PrefillLayout L = prefill_layout(T, budget, k_rot_out == nullptr, sel_out == nullptr, cnt_out == nullptr);
+  if (ws_bytes < L.total_fixed) return QSA_ERR_WORKSPACE_TOO_SMALL;
+  const size_t slab_bytes = ws_bytes - L.total_fixed;
+  const int64_t min_rows = nqb < MIN_ROWS ? nqb : MIN_ROWS;
+  if (slab_bytes < (size_t)min_rows * (size_t)round4(nqb) * 4) return QSA_ERR_WORKSPACE_TOO_SMALL;
+  DevInfo di;
+  if ((st = device_info(&di)) != QSA_OK) return st;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint32_t* err = reinterpret_cast<uint32_t*>(base);
+  float2* cs = reinterpret_cast<float2*>(base + L.cs);
+  uint16_t* k_rot = k_rot_out ? k_rot_out : reinterpret_cast<uint16_t*>(base + L.k_rot);
+  int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(base + L.sel);
+  int32_t* cnt = cnt_out ? cnt_out : reinterpret_cast<int32_t*>(base + L.cnt);
+  float* slab = reinterpret_cast<float*>(base + L.slab);
+
+  if (cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return QSA_ERR_CUDA;
+  double f[32];
+  inv_freq(p, f);
+  if ((st = from_cuda(qsa::launch_rope_table(T, pos0, f, cs, s))) != QSA_OK) return st;
+  if ((st = from_cuda(qsa::launch_rope_k(T, k, cs, k_rot, s))) != QSA_OK) return st;
+  const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
+  for (int64_t qb0 = 0; qb0 < nqb;) {
+    const int64_t qb1 = chunk_end(qb0, nqb, slab_bytes);
+    if (qb1 <= qb0) return QSA_ERR_WORKSPACE_TOO_SMALL;
+    const int64_t ld = round4(qb1);
+    if ((st = run_indexer(T, q_idx, w, k_idx, qb0, qb1, slab, ld, err, di.num_sms, s)) != QSA_OK) return st;
+    if ((st = from_cuda(qsa::launch_select(slab, ld, qb0, qb1 - qb0, nullptr, budget, sel + qb0 * budget, cnt + qb0,
+                                           err, s))) != QSA_OK)
+      return st;
+    if ((st = from_cuda(qsa::launch_sparse_attn_prefill(T, q, k_rot, v, cs, sel + qb0 * budget, cnt + qb0, budget,
+                                                        qb0, qb1, scale_log2, out, lse, s))) != QSA_OK)
+      return st;
+    qb0 = qb1;
+  }
+  return QSA_OK;
+}
+
+// ------------------------------------------------------------------ decode
+namespace {
+struct DecodeLayout {
+  size_t Ls, qbs, S, sel, cnt, q_rot, part_o, part_lse, total;
+  int64_t ld;
+};
+DecodeLayout decode_layout(int B, int64_t max_len, int budget) {
+  DecodeLayout L;
+  L.ld = round4(max_len / 4 + 1);
+  size_t off = HEADER_BYTES;
+  L.Ls = off; off = align_up(off + (size_t)B * 8);
+  L.qbs = off; off = align_up(off + (size_t)B * 8);
+  L.S = off; off = align_up(off + (size_t)B * L.ld * 4);
+  L.sel = off; off = align_up(off + (size_t)B * budget * 4);
+  L.cnt = off; off = align_up(off + (size_t)B * 4);
+  L.q_rot = off; off = align_up(off + (size_t)B * 24 * 256 * 2);
+  L.part_o = off; off = align_up(off + (size_t)B * DECODE_SPLIT * 24 * 256 * 4);
+  L.part_lse = off; off = align_up(off + (size_t)B * DECODE_SPLIT * 24 * 4);
+  L.total = off;
+  return L;
+}
+}  // namespace
+
+qsa_status qsa_decode_workspace_size(const qsa_params* p, int32_t B, int64_t max_len, size_t* bytes) {
+  qsa_status st = check_params(p);
+  if (st != QSA_OK) return st;
+  if (B <= 0 || max_len <= 0 || !bytes) return QSA_ERR_INVALID_ARG;
+  if (B > 4096 || max_len > ((int64_t)1 << 24)) return QSA_ERR_UNSUPPORTED;
+  *bytes = decode_layout(B, max_len, p->budget_blocks).total;
+  return QSA_OK;
+}
+
+qsa_status qsa_decode(const qsa_params* p, int32_t B, int64_t max_len, const int64_t* cache_len, uint16_t* k_cache,
+                      uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* qidx_ring, uint16_t* w_ring,
+                      const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new, const uint16_t* q_idx_new,
+                      const uint16_t* k_idx_new, const uint16_t* w_new, uint16_t* out, int32_t* sel_out,
+                      float* lse_out, void* ws, size_t ws_bytes, void* stream) {
+  qsa_status st = check_params(p);
+  if (st != QSA_OK) return st;
+  if (B <= 0 || max_len <= 0 || !cache_len) return QSA_ERR_INVALID_ARG;
+  if (B > 4096 || max_len > ((int64_t)1 << 24)) return QSA_ERR_UNSUPPORTED;
+  const void* ptrs[] = {k_cache, v_cache, kidx_cache, qidx_ring, w_ring, q_new, k_new, v_new,
+                        q_idx_new, k_idx_new, w_new, out, ws};
+  for (const void* ptr : ptrs) {
+    if (!ptr) return QSA_ERR_INVALID_ARG;
+    if (!aligned16(ptr)) return QSA_ERR_MISALIGNED;
+  }
+  if ((sel_out && !aligned16(sel_out)) || (lse_out && !aligned16(lse_out))) return QSA_ERR_MISALIGNED;
+  int64_t max_L = 0;
+  for (int b = 0; b < B; ++b) {
+    if (cache_len[b] < 0 || cache_len[b] >= max_len) return QSA_ERR_INVALID_ARG;
+    if (cache_len[b] > max_L) max_L = cache_len[b];
+  }
+  const int budget = p->budget_blocks;
+  DecodeLayout L = decode_layout(B, max_len, budget);
+  if (ws_bytes < L.total) return QSA_ERR_WORKSPACE_TOO_SMALL;
+  DevInfo di;
+  if ((st = device_info(&di)) != QSA_OK) return st;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint32_t* err = reinterpret_cast<uint32_t*>(base);
+  int64_t* Ls = reinterpret_cast<int64_t*>(base + L.Ls);
+  int64_t* qbs = reinterpret_cast<int64_t*>(base + L.qbs);
+  float* S = reinterpret_cast<float*>(base + L.S);
+  int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(base + L.sel);
+  int32_t* cnt = reinterpret_cast<int32_t*>(base + L.cnt);
+  uint16_t* q_rot = reinterpret_cast<uint16_t*>(base + L.q_rot);
+  float* part_o = reinterpret_cast<float*>(base + L.part_o);
+  float* part_lse = reinterpret_cast<float*>(base + L.part_lse);
+
+  if (cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return QSA_ERR_CUDA;
+  double f[32];
+  inv_freq(p, f);
+  // the append kernel receives the lengths as launch parameters and stores
+  // them (and L/4) in the workspace for the later kernels
+  if ((st = from_cuda(qsa::launch_decode_append(B, max_len, cache_len, Ls, qbs, f, k_cache, v_cache, kidx_cache,
+                                                qidx_ring, w_ring, q_new, k_new, v_new, q_idx_new, k_idx_new, w_new,
+                                                q_rot, s))) != QSA_OK)
+    return st;
+  const float scale = 1.0f / std::sqrt(128.0f);
+  if ((st = from_cuda(qsa::launch_decode_indexer(B, max_len, max_L, Ls, kidx_cache, qidx_ring, w_ring, S, L.ld, scale,
+                                                 s))) != QSA_OK)
+    return st;
+  if ((st = from_cuda(qsa::launch_select(S, L.ld, 0, B, qbs, budget, sel, cnt, err, s))) != QSA_OK) return st;
+  const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
+  if ((st = from_cuda(qsa::launch_decode_attn(B, max_len, Ls, q_rot, k_cache, v_cache, sel, cnt, budget, DECODE_SPLIT,
+                                              scale_log2, part_o, part_lse, s))) != QSA_OK)
+    return st;
+  return from_cuda(qsa::launch_decode_combine(B, DECODE_SPLIT, part_o, part_lse, out, lse_out, s));
+}
+
+qsa_status qsa_check_device_error(void* ws, void* stream) {
+  if (!ws) return QSA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t h = 0;
+  if (cudaMemcpyAsync(&h, ws, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return QSA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return QSA_ERR_CUDA;
+  if (h != 0 && cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) return QSA_ERR_CUDA;
+  if (h == 0) return QSA_OK;
+  return (h == QSA_ERR_DEVICE_TIMEOUT || h == QSA_ERR_DEVICE_BOUNDS) ? static_cast<qsa_status>(h) : QSA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,142 @@
+// Decode: indexer block scores of the new token's query block over the whole
+// indexer-key cache (the decode step's dominant HBM stream).
+//
+// Same score as prefill (page "Qwen3.8-Flash-Next, 1/9의 학습 비용으로 Qwen3.7-
+// Plus(397B-A17B) 수준에 도달한 125B-A6B 모델", section "QSA: 인덱서 자체의 비용을
+// 줄이는 희소 어텐션", eq. I_ib with this library's head weights and causal
+// block max): for the block qb = L/4 of the new token at position L, the
+// query tokens are the present block-mates 4qb .. L (from the ring) and
+// S(qb, kb) = max over those tokens t and keys j of block kb, j <= t, of
+// sum_h w_h(t) ReLU(q_idx_h(t) . k_idx(j)) / sqrt(128).
+//
+// Kernel: 16 keys x 16 (token, head) columns per bf16 tensor-core MMA
+// (m16n8k16, two n-tiles).  The dot product is a sum over the 128 dims, so
+// the dims may be assigned to MMA k-slots in any order as long as A and B
+// agree: each thread loads 16 contiguous bytes (8 dims) of a key row straight
+// from global memory into its A fragment registers for two k-steps, and the
+// query fragments use the same assignment.  No shared memory; every load is a
+// full 32-byte sector.  Column n of n-tile nt is (token n/2, head 2*nt + n%2),
+// so a thread's accumulators hold all 4 heads of one token for two keys.
+#include "qsa_device.cuh"
+#include "qsa_kernels.h"
+
+namespace qsa {
+namespace {
+
+constexpr int THREADS = 128;
+constexpr int KEYS_PER_CTA = 2048;
+
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__global__ void __launch_bounds__(THREADS)
+decode_indexer_kernel(int64_t max_len, const int64_t* __restrict__ Ls, const uint16_t* __restrict__ kidx_cache,
+                      const uint16_t* __restrict__ qidx_ring, const uint16_t* __restrict__ w_ring,
+                      float* __restrict__ S, int64_t ld, float scale) {
+  const int64_t b = blockIdx.y;
+  const int64_t L = Ls[b];
+  const int64_t qb = L >> 2;
+  const int64_t j_begin = (int64_t)blockIdx.x * KEYS_PER_CTA;
+  if (j_begin > L) return;
+  int64_t j_end = j_begin + KEYS_PER_CTA;
+  if (j_end > 4 * qb + 4) j_end = 4 * qb + 4;
+  const int present = (int)(L - 4 * qb) + 1;        // block-mates 4qb .. L (ring slots 0 .. present-1)
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g8 = lane >> 2, q4 = lane & 3;
+
+  // B fragments: column g8 -> (token g8/2, head 2*nt + g8%2), dims 32*d + 8*q4 .. +7
+  uint4 qf[2][4];
+  {
+    const int tok = g8 >> 1;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const int head = 2 * nt + (g8 & 1);
+      const uint4* src = reinterpret_cast<const uint4*>(qidx_ring + ((b * 4 + tok) * 4 + head) * 128);
+#pragma unroll
+      for (int d = 0; d < 4; ++d) qf[nt][d] = tok < present ? src[4 * d + q4] : make_uint4(0, 0, 0, 0);
+    }
+  }
+  // head weights of this thread's token q4
+  float w[4];
+  {
+    const bool ok = q4 < present;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) w[h] = ok ? bf16_bits_to_f32(w_ring[(b * 4 + q4) * 4 + h]) : 0.f;
+  }
+  const int64_t t_tok = 4 * qb + q4;                 // this thread's query token
+  const bool tok_ok = q4 < present;
+  const uint16_t* kb_base = kidx_cache + b * max_len * 128;
+  float* Srow = S + b * ld;
+
+  for (int64_t jt = j_begin + 16 * warp; jt < j_end; jt += 16 * (THREADS / 32)) {
+    const int64_t j0 = jt + g8, j1 = jt + g8 + 8;
+    const int64_t r0 = j0 <= L ? j0 : L, r1 = j1 <= L ? j1 : L;
+    const uint4* k0p = reinterpret_cast<const uint4*>(kb_base + r0 * 128);
+    const uint4* k1p = reinterpret_cast<const uint4*>(kb_base + r1 * 128);
+    uint4 k0[4], k1[4];
+#pragma unroll
+    for (int d = 0; d < 4; ++d) { k0[d] = ldg_stream(k0p + 4 * d + q4); k1[d] = ldg_stream(k1p + 4 * d + q4); }
+    float acc[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+    for (int d = 0; d < 4; ++d) {
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        mma16816(acc[nt], k0[d].x, k1[d].x, k0[d].y, k1[d].y, qf[nt][d].x, qf[nt][d].y);
+        mma16816(acc[nt], k0[d].z, k1[d].z, k0[d].w, k1[d].w, qf[nt][d].z, qf[nt][d].w);
+      }
+    }
+    // acc[nt][0..1]: key j0, heads 2nt, 2nt+1 of token q4; acc[nt][2..3]: key j1
+    float s0 = w[0] * fmaxf(acc[0][0], 0.f);
+    s0 = fmaf(w[1], fmaxf(acc[0][1], 0.f), s0);
+    s0 = fmaf(w[2], fmaxf(acc[1][0], 0.f), s0);
+    s0 = fmaf(w[3], fmaxf(acc[1][1], 0.f), s0);
+    float s1 = w[0] * fmaxf(acc[0][2], 0.f);
+    s1 = fmaf(w[1], fmaxf(acc[0][3], 0.f), s1);
+    s1 = fmaf(w[2], fmaxf(acc[1][2], 0.f), s1);
+    s1 = fmaf(w[3], fmaxf(acc[1][3], 0.f), s1);
+    s0 = (tok_ok && j0 <= t_tok) ? s0 : 0.f;
+    s1 = (tok_ok && j1 <= t_tok) ? s1 : 0.f;
+    // max over the 4 tokens (lanes q4), then over the 4 keys of a block (g8 % 4)
+#pragma unroll
+    for (int off = 1; off <= 8; off <<= 1) {
+      s0 = fmaxf(s0, __shfl_xor_sync(0xffffffffu, s0, off));
+      s1 = fmaxf(s1, __shfl_xor_sync(0xffffffffu, s1, off));
+    }
+    if ((lane & 15) == 0) {
+      const int64_t kb0 = (jt >> 2) + (lane >> 4);     // lane 0: blocks +0 / +2, lane 16: +1 / +3
+      if (kb0 <= qb) Srow[kb0] = s0 * scale;
+      if (kb0 + 2 <= qb) Srow[kb0 + 2] = s1 * scale;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_decode_indexer(int B, int64_t max_len, int64_t max_L, const int64_t* L_dev,
+                                  const uint16_t* kidx_cache, const uint16_t* qidx_ring, const uint16_t* w_ring,
+                                  float* S, int64_t ld, float scale, cudaStream_t s) {
+  if (B <= 0) return cudaSuccess;
+  const int64_t nx = (max_L + 4 + KEYS_PER_CTA - 1) / KEYS_PER_CTA;
+  dim3 grid((unsigned)nx, (unsigned)B);
+  decode_indexer_kernel<<<grid, THREADS, 0, s>>>(max_len, L_dev, kidx_cache, qidx_ring, w_ring, S, ld, scale);
+  return cudaGetLastError();
+}
+
+}  // namespace qsa

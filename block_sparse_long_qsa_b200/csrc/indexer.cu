@@ -1,0 +1,339 @@
+// Stage 1, prefill: indexer block scores on the 5th-generation tensor cores.
+//
+//   s(t, j)   = sum_h w[t][h] * ReLU(q_idx[t][h] . k_idx[j]) / sqrt(128)
+//   S(qb, kb) = max over t in block qb, j in block kb, j <= t, of s(t, j)
+//
+// ([PT] = page "Qwen3.8-Flash-Next, 1/9의 학습 비용으로 Qwen3.7-Plus(397B-A17B)
+// 수준에 도달한 125B-A6B 모델", section "QSA: 인덱서 자체의 비용을 줄이는 희소
+// 어텐션", eq. I_ib: ReLU of the per-head similarity, summed over the 4
+// indexer heads; block-causal scoring of r = 4 token micro-blocks.)
+//
+// Design (one persistent CTA per SM, 320 threads):
+//   * A = 128 keys x 128 dims (K-major, TMA, 128B swizzle), B = 64 query tokens
+//     x 4 heads = 256 rows x 128 dims; D = A B^T is 128 x 256 fp32 in TMEM, so a
+//     TMEM lane is one key and the 4 head values of one token sit in 4
+//     consecutive columns of that lane.  The head-weighted ReLU sum and the max
+//     over the 4 tokens of a query block happen in one thread's registers; the
+//     max over the 4 keys of a key block is two warp shuffles.
+//   * A query tile is 128 tokens (two N = 256 halves, two TMEM accumulators of
+//     256 columns); each 32 KB key tile loaded from HBM feeds 2 x 8.4 MFLOP.
+//   * Work unit = (query tile, key tile).  The causal triangle's units are
+//     split evenly across CTAs in query-major order, so every CTA gets the
+//     same number of MMAs whatever the chunk shape.
+//   * warp 0: TMA producer (3-stage key ring, Q + w tile); warp 1: TMEM
+//     allocation and the single MMA-issuing thread; warps 2-9: epilogue
+//     (tcgen05.ld -> ReLU, head weights, block max -> fp32 scores).
+//   * Every mbarrier wait is bounded; on timeout the CTA records
+//     QSA_ERR_DEVICE_TIMEOUT, drains and exits.
+#include "qsa_device.cuh"
+#include "qsa_kernels.h"
+
+namespace qsa {
+namespace {
+
+constexpr int QT = 128;                 // query tokens per tile
+constexpr int KT = 128;                 // keys per tile
+constexpr int STAGES = 3;
+constexpr int THREADS = 320;
+constexpr uint32_t Q_SUB_BYTES = 256 * 128;              // 256 rows x 64 bf16
+constexpr uint32_t Q_BYTES = 4 * Q_SUB_BYTES;            // [half][k-chunk]
+constexpr uint32_t K_SUB_BYTES = 128 * 128;              // 128 rows x 64 bf16
+constexpr uint32_t K_STAGE_BYTES = 2 * K_SUB_BYTES;
+constexpr uint32_t W_BYTES = QT * 4 * 2;                 // bf16 [128][4]
+constexpr uint32_t OFF_K = Q_BYTES;
+constexpr uint32_t OFF_W = OFF_K + STAGES * K_STAGE_BYTES;
+constexpr uint32_t OFF_BAR = OFF_W + W_BYTES;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 128;
+static_assert(SMEM_BYTES <= 232448, "indexer smem");
+constexpr uint32_t TMEM_COLS = 512;
+
+struct Sched {
+  int64_t T0, Tend, n_tiles, c;   // c = nkt(0)
+  int64_t qb_begin;
+  __device__ __forceinline__ int64_t nkt(int64_t i) const {
+    int64_t tl = T0 + QT * i + (QT - 1);
+    if (tl > Tend - 1) tl = Tend - 1;
+    return tl / KT + 1;
+  }
+  // units before tile i (valid for i <= n_tiles - 1; tiles before the last are full)
+  __device__ __forceinline__ int64_t prefix(int64_t i) const { return c * i + i * (i - 1) / 2; }
+  __device__ __forceinline__ int64_t total() const { return prefix(n_tiles - 1) + nkt(n_tiles - 1); }
+  __device__ __forceinline__ void locate(int64_t u, int64_t& tile, int64_t& kt) const {
+    int64_t lo = 0, hi = n_tiles - 1;
+    while (lo < hi) {
+      int64_t mid = (lo + hi + 1) >> 1;
+      if (prefix(mid) <= u) lo = mid; else hi = mid - 1;
+    }
+    tile = lo;
+    kt = u - prefix(lo);
+  }
+};
+
+struct Iter {
+  const Sched* s;
+  int64_t u, u_end, tile, kt, nkt;
+  __device__ __forceinline__ void begin(const Sched* sch, int64_t u0, int64_t u1) {
+    s = sch; u = u0; u_end = u1;
+    if (u < u_end) { s->locate(u, tile, kt); nkt = s->nkt(tile); }
+  }
+  __device__ __forceinline__ bool valid() const { return u < u_end; }
+  __device__ __forceinline__ bool first_of_tile(int64_t u0) const { return kt == 0 || u == u0; }
+  // next unit in range belongs to another tile
+  __device__ __forceinline__ bool tile_ends_here() const { return kt == nkt - 1 && u + 1 < u_end; }
+  __device__ __forceinline__ void next() {
+    ++u; ++kt;
+    if (kt == nkt) { ++tile; kt = 0; if (u < u_end) nkt = s->nkt(tile); }
+  }
+};
+
+__global__ void __launch_bounds__(THREADS, 1)
+indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_w, float* __restrict__ S, int64_t ld, int64_t T,
+                       int64_t qb_begin, int64_t qb_end, float scale, uint32_t* err) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + OFF_K;
+  const uint16_t* sW = reinterpret_cast<const uint16_t*>(smem + OFF_W);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* full = bars;               // [STAGES]
+  uint64_t* empty = bars + STAGES;     // [STAGES]
+  uint64_t* qfull = bars + 2 * STAGES;
+  uint64_t* qempty = qfull + 1;
+  uint64_t* accfull = qfull + 2;       // [2]
+  uint64_t* accempty = qfull + 4;      // [2]
+  uint64_t* done = qfull + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qfull + 7);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if ((smem_u32(smem) & 1023u) != 0u) {  // the swizzled operand layout needs 1 KB alignment
+    if (threadIdx.x == 0) report_error(err, QSA_ERR_DEVICE_BOUNDS);
+    return;
+  }
+
+  Sched sch;
+  sch.qb_begin = qb_begin;
+  sch.T0 = qb_begin * 4;
+  sch.Tend = qb_end * 4 < T ? qb_end * 4 : T;
+  sch.n_tiles = (sch.Tend - sch.T0 + QT - 1) / QT;
+  sch.c = (sch.T0 + QT - 1) / KT + 1;
+  const int64_t W = sch.total();
+  const int64_t u0 = W * (int64_t)blockIdx.x / gridDim.x;
+  const int64_t u1 = W * (int64_t)(blockIdx.x + 1) / gridDim.x;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    mbar_init(qfull, 1);
+    mbar_init(qempty, 1 + 8);
+    for (int h = 0; h < 2; ++h) { mbar_init(&accfull[h], 1); mbar_init(&accempty[h], 8); }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) { tmem_alloc(tmem_slot, TMEM_COLS); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_w);
+      Iter it; it.begin(&sch, u0, u1);
+      int stage = 0; uint32_t ephase = 1; uint32_t qcount = 0;
+      for (; it.valid(); it.next()) {
+        if (it.first_of_tile(u0)) {
+          if (qcount > 0 && !mbar_wait(qempty, (qcount - 1) & 1, abort_flag, err)) break;
+          const int32_t t_first = (int32_t)(sch.T0 + QT * it.tile);
+          mbar_arrive_expect_tx(qfull, Q_BYTES + W_BYTES);
+          for (int hf = 0; hf < 2; ++hf)
+            for (int kc = 0; kc < 2; ++kc)
+              tma_load_2d(sQ + (hf * 2 + kc) * Q_SUB_BYTES, &tm_q, kc * 64, 4 * t_first + 256 * hf, qfull);
+          // w as a flat bf16 array of 4*T: two 256-element boxes (x * 2 bytes is a multiple of 16)
+          tma_load_1d(smem + OFF_W, &tm_w, 4 * t_first, qfull);
+          tma_load_1d(smem + OFF_W + W_BYTES / 2, &tm_w, 4 * t_first + 256, qfull);
+          ++qcount;
+        }
+        if (!mbar_wait(&empty[stage], ephase, abort_flag, err)) break;
+        mbar_arrive_expect_tx(&full[stage], K_STAGE_BYTES);
+        for (int kc = 0; kc < 2; ++kc)
+          tma_load_2d(sK + stage * K_STAGE_BYTES + kc * K_SUB_BYTES, &tm_k, kc * 64, (int32_t)(KT * it.kt),
+                      &full[stage]);
+        if (++stage == STAGES) { stage = 0; ephase ^= 1; }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16_f32(128, 256);
+      Iter it; it.begin(&sch, u0, u1);
+      int stage = 0; uint32_t fphase = 0; uint32_t qcount = 0;
+      uint32_t acc_use[2] = {0, 0};
+      bool ok = true;
+      for (; ok && it.valid(); it.next()) {
+        if (it.first_of_tile(u0)) {
+          if (!mbar_wait(qfull, qcount & 1, abort_flag, err)) break;
+          ++qcount;
+        }
+        if (!mbar_wait(&full[stage], fphase, abort_flag, err)) break;
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(sK + stage * K_STAGE_BYTES);
+        for (int hf = 0; hf < 2; ++hf) {
+          if (!mbar_wait(&accempty[hf], (acc_use[hf] & 1) ^ 1, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t b_base = smem_u32(sQ + hf * 2 * Q_SUB_BYTES);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t koff = (uint32_t)(k & 3) * 32;      // 16 bf16 = 32 bytes inside the swizzle atom
+            const uint64_t ad = umma_desc_k_sw128(a_base + (k >> 2) * K_SUB_BYTES + koff);
+            const uint64_t bd = umma_desc_k_sw128(b_base + (k >> 2) * Q_SUB_BYTES + koff);
+            umma_bf16(tmem + hf * 256, ad, bd, idesc, k > 0 ? 1u : 0u);
+          }
+          tc_commit(&accfull[hf]);
+          ++acc_use[hf];
+        }
+        if (!ok) break;
+        tc_commit(&empty[stage]);
+        if (it.tile_ends_here()) tc_commit(qempty);
+        if (++stage == STAGES) { stage = 0; fphase ^= 1; }
+      }
+      // all issued MMAs retired before TMEM is released
+      tc_commit(done);
+      mbar_wait(done, 0, abort_flag, err);
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue
+    const int e = warp - 2;                 // 0..7
+    const int quad = warp & 3;              // TMEM lanes 32*quad .. +31
+    const int cgrp = e >> 2;                // column group: tokens [32*cgrp, +32) of a half
+    const uint32_t lane_addr = (uint32_t)(32 * quad) << 16;
+    Iter it; it.begin(&sch, u0, u1);
+    uint32_t qcount = 0;
+    uint32_t acc_use[2] = {0, 0};
+    for (; it.valid(); it.next()) {
+      if (it.first_of_tile(u0)) {
+        if (!mbar_wait(qfull, qcount & 1, abort_flag, err)) break;
+        ++qcount;
+      }
+      const int64_t t_tile = sch.T0 + QT * it.tile;
+      const int64_t qb_tile = qb_begin + (QT / 4) * it.tile;
+      const int64_t j = KT * it.kt + 32 * quad + lane;       // this thread's key
+      const int64_t kb = j >> 2;
+      bool ok = true;
+      for (int hf = 0; hf < 2; ++hf) {
+        if (!mbar_wait(&accfull[hf], acc_use[hf] & 1, abort_flag, err)) { ok = false; break; }
+        ++acc_use[hf];
+        tc_fence_after();
+        const int64_t t_first = t_tile + 64 * hf + 32 * cgrp;  // first token of this thread's columns
+        const int64_t qb_first = qb_tile + 16 * hf + 8 * cgrp;
+        const int64_t kt_last_key = KT * it.kt + KT - 1;
+        // skip when every key block of this warp lies after every query block of its columns
+        const bool live = (KT * it.kt + 32 * quad) <= (t_first + 31) && qb_first < qb_end;
+        float m[8];
+        if (live) {
+          float v[4][32];
+          const uint32_t base = tmem + lane_addr + hf * 256 + 128 * cgrp;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld32(base + 32 * c, v[c]);
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&accempty[hf]);
+          const bool masked = kt_last_key > t_first;
+          const uint16_t* wrow = sW + (64 * hf + 32 * cgrp) * 4;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+#pragma unroll
+            for (int half_blk = 0; half_blk < 2; ++half_blk) {
+              float sc[4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const int tl = 8 * c + 4 * half_blk + u;    // token index within the 32 columns
+                const uint2 wv = *reinterpret_cast<const uint2*>(wrow + 4 * tl);
+                const float* x = &v[c][4 * (4 * half_blk + u)];
+                float s = bf16lo(wv.x) * fmaxf(x[0], 0.f);
+                s = fmaf(bf16hi(wv.x), fmaxf(x[1], 0.f), s);
+                s = fmaf(bf16lo(wv.y), fmaxf(x[2], 0.f), s);
+                s = fmaf(bf16hi(wv.y), fmaxf(x[3], 0.f), s);
+                if (masked) s = (j <= t_first + tl) ? s : 0.f;
+                sc[u] = s;
+              }
+              m[2 * c + half_blk] = fmaxf(max3f(sc[0], sc[1], sc[2]), sc[3]);
+            }
+          }
+        } else {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&accempty[hf]);
+#pragma unroll
+          for (int b = 0; b < 8; ++b) m[b] = 0.f;
+        }
+        if (live) {
+#pragma unroll
+          for (int b = 0; b < 8; ++b) {
+            m[b] = fmaxf(m[b], __shfl_xor_sync(0xffffffffu, m[b], 1));
+            m[b] = fmaxf(m[b], __shfl_xor_sync(0xffffffffu, m[b], 2));
+          }
+          const int r = lane & 3;
+#pragma unroll
+          for (int rr = 0; rr < 2; ++rr) {
+            const int b = r + 4 * rr;
+            const int64_t qb = qb_first + b;
+            // select m[b] without dynamic register indexing
+            float val = m[0];
+#pragma unroll
+            for (int bb = 1; bb < 8; ++bb) val = (bb == b) ? m[bb] : val;
+            if (qb < qb_end && kb <= qb) S[(qb - qb_begin) * ld + kb] = val * scale;
+          }
+        }
+      }
+      if (!ok) break;
+      if (it.tile_ends_here()) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(qempty);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_indexer_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_w,
+                                   float* S, int64_t ld, int64_t T, int64_t qb_begin, int64_t qb_end, float scale,
+                                   uint32_t* err, int num_sms, cudaStream_t stream) {
+  if (qb_end <= qb_begin) return cudaSuccess;
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(indexer_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = true;
+  }
+  // units in this call; never more CTAs than units
+  const int64_t T0 = qb_begin * 4;
+  const int64_t Tend = qb_end * 4 < T ? qb_end * 4 : T;
+  const int64_t n_tiles = (Tend - T0 + QT - 1) / QT;
+  int64_t units = 0;
+  for (int64_t i = 0; i < n_tiles && units < num_sms; ++i) {
+    int64_t tl = T0 + QT * i + QT - 1;
+    if (tl > Tend - 1) tl = Tend - 1;
+    units += tl / KT + 1;
+  }
+  const int grid = (int)(units < num_sms ? units : num_sms);
+  indexer_prefill_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tm_q, tm_k, tm_w, S, ld, T, qb_begin, qb_end, scale,
+                                                                 err);
+  return cudaGetLastError();
+}
+
+}  // namespace qsa

@@ -1,0 +1,50 @@
+// Internal launchers of the QSA kernels (not part of the C ABI).
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace qsa {
+
+// RoPE angles of positions pos0 .. pos0+T-1: cs[t][i] = (cos a, sin a),
+// a = (pos0 + t) * inv_freq[i], i < 32, angle formed in fp64.
+cudaError_t launch_rope_table(int64_t T, int64_t pos0, const double* inv_freq_host, float2* cs, cudaStream_t s);
+// k_rot[t][g] = RoPE(k[t][g]) on dims 0..63, dims 64..255 copied.
+cudaError_t launch_rope_k(int64_t T, const uint16_t* k, const float2* cs, uint16_t* k_rot, cudaStream_t s);
+
+cudaError_t launch_indexer_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_w,
+                                   float* S, int64_t ld, int64_t T, int64_t qb_begin, int64_t qb_end, float scale,
+                                   uint32_t* err, int num_sms, cudaStream_t stream);
+
+// Top-k block selection, one row per query block.  Row r covers query block
+// row_qb ? row_qb[r] : qb_begin + r, read from S + r * ld.
+size_t select_smem_bytes(int budget);
+cudaError_t launch_select(const float* S, int64_t ld, int64_t qb_begin, int64_t n_rows, const int64_t* row_qb,
+                          int budget, int32_t* sel, int32_t* cnt, uint32_t* err, cudaStream_t stream);
+
+// Sparse GQA attention for query blocks [qb_begin, qb_end) given their selections.
+cudaError_t launch_sparse_attn_prefill(int64_t T, const uint16_t* q, const uint16_t* k_rot, const uint16_t* v,
+                                       const float2* cs, const int32_t* sel, const int32_t* cnt, int budget,
+                                       int64_t qb_begin, int64_t qb_end, float scale_log2, uint16_t* out, float* lse,
+                                       cudaStream_t stream);
+
+// ---------------------------------------------------------------- decode
+// Lengths come from the host array L_host (passed to the kernel as launch
+// parameters) and are stored to L_dev / qb_dev for the later kernels.
+cudaError_t launch_decode_append(int B, int64_t max_len, const int64_t* L_host, int64_t* L_dev, int64_t* qb_dev,
+                                 const double* inv_freq_host,
+                                 uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* qidx_ring,
+                                 uint16_t* w_ring, const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
+                                 const uint16_t* q_idx_new, const uint16_t* k_idx_new, const uint16_t* w_new,
+                                 uint16_t* q_rot, cudaStream_t s);
+cudaError_t launch_decode_indexer(int B, int64_t max_len, int64_t max_L, const int64_t* L_dev,
+                                  const uint16_t* kidx_cache, const uint16_t* qidx_ring, const uint16_t* w_ring,
+                                  float* S, int64_t ld, float scale, cudaStream_t s);
+cudaError_t launch_decode_attn(int B, int64_t max_len, const int64_t* L_dev, const uint16_t* q_rot,
+                               const uint16_t* k_cache, const uint16_t* v_cache, const int32_t* sel,
+                               const int32_t* cnt, int budget, int n_split, float scale_log2, float* part_o,
+                               float* part_lse, cudaStream_t s);
+cudaError_t launch_decode_combine(int B, int n_split, const float* part_o, const float* part_lse, uint16_t* out,
+                                  float* lse, cudaStream_t s);
+
+}  // namespace qsa

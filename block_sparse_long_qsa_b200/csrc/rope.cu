@@ -1,0 +1,169 @@
+// RoPE on the keys (prefill) and the decode append.
+//
+// Rotary embedding with theta = 1e7 on dims 0..63 of every Q and K head
+// (rope_dim 64 = partial_rotary_factor 0.25 of head_dim 256; page "Qwen3.8-
+// Flash-Next, 1/9의 학습 비용으로 Qwen3.7-Plus(397B-A17B) 수준에 도달한 125B-A6B
+// 모델", spec table and section "100만 토큰까지 늘리기").  Pairs are
+// (i, i + 32); angle a = position * theta^(-i/32), formed in fp64 so that
+// positions near 2^20 keep their phase, then rotated in fp32.
+#include "qsa_device.cuh"
+#include "qsa_kernels.h"
+
+namespace qsa {
+namespace {
+
+struct InvFreq { double f[32]; };
+
+// cs[t][i] = (cos a, sin a) for a = (pos0 + t) * inv_freq[i]
+__global__ void rope_table_kernel(int64_t T, int64_t pos0, InvFreq inv, float2* __restrict__ cs) {
+  const int64_t n = T * 32;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = e >> 5;
+    const int i = (int)(e & 31);
+    double sa, ca;
+    sincos((double)(pos0 + t) * inv.f[i], &sa, &ca);
+    cs[e] = make_float2((float)ca, (float)sa);
+  }
+}
+
+__device__ __forceinline__ void rotate8(const uint4& lo, const uint4& hi, const float2* c8, uint4& olo, uint4& ohi) {
+  // lo holds dims i..i+7, hi holds dims i+32..i+39
+  const uint32_t* a = reinterpret_cast<const uint32_t*>(&lo);
+  const uint32_t* b = reinterpret_cast<const uint32_t*>(&hi);
+  uint32_t* oa = reinterpret_cast<uint32_t*>(&olo);
+  uint32_t* ob = reinterpret_cast<uint32_t*>(&ohi);
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const float x0 = bf16lo(a[p]), x1 = bf16hi(a[p]);
+    const float y0 = bf16lo(b[p]), y1 = bf16hi(b[p]);
+    const float2 c0 = c8[2 * p], c1 = c8[2 * p + 1];
+    oa[p] = pack_bf16x2(x0 * c0.x - y0 * c0.y, x1 * c1.x - y1 * c1.y);
+    ob[p] = pack_bf16x2(y0 * c0.x + x0 * c0.y, y1 * c1.x + x1 * c1.y);
+  }
+}
+
+// One thread per (token, kv head, 16-byte chunk slot): slots 0..3 rotate the
+// chunk pairs (s, s+4) of dims 0..63, slots 4..27 copy chunks 8..31.
+__global__ void rope_k_kernel(int64_t T, const uint4* __restrict__ k, const float2* __restrict__ cs,
+                              uint4* __restrict__ k_rot) {
+  const int64_t n = T * 2 * 28;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = e / 28;          // t * 2 + g
+    const int slot = (int)(e - row * 28);
+    const uint4* src = k + row * 32;
+    uint4* dst = k_rot + row * 32;
+    if (slot < 4) {
+      const int64_t t = row >> 1;
+      const uint4 lo = __ldg(src + slot), hi = __ldg(src + slot + 4);
+      uint4 olo, ohi;
+      rotate8(lo, hi, cs + t * 32 + 8 * slot, olo, ohi);
+      dst[slot] = olo;
+      dst[slot + 4] = ohi;
+    } else {
+      dst[slot + 4] = __ldg(src + slot + 4);
+    }
+  }
+}
+
+// Decode append: one CTA per sequence.
+//   k_cache[b][L] = RoPE(k_new[b], L); v_cache[b][L] = v_new[b];
+//   kidx_cache[b][L] = k_idx_new[b]; ring slot L % 4 <- (q_idx_new[b], w_new[b]);
+//   q_rot[b] = RoPE(q_new[b], L).
+constexpr int LEN_CHUNK = 1024;
+struct LenChunk { int64_t L[LEN_CHUNK]; int32_t b0; };
+
+__global__ void decode_append_kernel(int64_t max_len, LenChunk lens, int64_t* __restrict__ L_dev,
+                                     int64_t* __restrict__ qb_dev, InvFreq inv,
+                                     uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                                     uint4* __restrict__ kidx_cache, uint4* __restrict__ qidx_ring,
+                                     uint16_t* __restrict__ w_ring, const uint4* __restrict__ q_new,
+                                     const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+                                     const uint4* __restrict__ q_idx_new, const uint4* __restrict__ k_idx_new,
+                                     const uint16_t* __restrict__ w_new, uint4* __restrict__ q_rot) {
+  __shared__ float2 cs[32];
+  const int b = lens.b0 + blockIdx.x;
+  const int64_t L = lens.L[blockIdx.x];
+  if (threadIdx.x == 0) { L_dev[b] = L; qb_dev[b] = L >> 2; }
+  if (threadIdx.x < 32) {
+    double sa, ca;
+    sincos((double)L * inv.f[threadIdx.x], &sa, &ca);
+    cs[threadIdx.x] = make_float2((float)ca, (float)sa);
+  }
+  __syncthreads();
+  // rotated rows: 2 kv heads (k) + 24 q heads, 4 rotate slots each; copies of the rest
+  const int n_rows = 2 + 24;
+  for (int e = threadIdx.x; e < n_rows * 28; e += blockDim.x) {
+    const int row = e / 28, slot = e % 28;
+    const uint4* src = row < 2 ? k_new + ((int64_t)b * 2 + row) * 32 : q_new + ((int64_t)b * 24 + row - 2) * 32;
+    uint4* dst = row < 2 ? k_cache + (((int64_t)b * max_len + L) * 2 + row) * 32
+                         : q_rot + ((int64_t)b * 24 + row - 2) * 32;
+    if (slot < 4) {
+      uint4 olo, ohi;
+      rotate8(src[slot], src[slot + 4], cs + 8 * slot, olo, ohi);
+      dst[slot] = olo;
+      dst[slot + 4] = ohi;
+    } else {
+      dst[slot + 4] = src[slot + 4];
+    }
+  }
+  for (int e = threadIdx.x; e < 64; e += blockDim.x)            // v: 2 x 512 B
+    v_cache[((int64_t)b * max_len + L) * 64 + e] = v_new[(int64_t)b * 64 + e];
+  for (int e = threadIdx.x; e < 16; e += blockDim.x)            // k_idx: 256 B
+    kidx_cache[((int64_t)b * max_len + L) * 16 + e] = k_idx_new[(int64_t)b * 16 + e];
+  const int slot = (int)(L & 3);
+  for (int e = threadIdx.x; e < 64; e += blockDim.x)            // q_idx: 4 x 256 B
+    qidx_ring[((int64_t)b * 4 + slot) * 64 + e] = q_idx_new[(int64_t)b * 64 + e];
+  if (threadIdx.x < 4) w_ring[((int64_t)b * 4 + slot) * 4 + threadIdx.x] = w_new[(int64_t)b * 4 + threadIdx.x];
+}
+
+InvFreq to_struct(const double* f) {
+  InvFreq s;
+  for (int i = 0; i < 32; ++i) s.f[i] = f[i];
+  return s;
+}
+
+int grid_for(int64_t n, int threads) {
+  int64_t g = (n + threads - 1) / threads;
+  const int64_t cap = 148LL * 16;
+  return (int)(g < 1 ? 1 : (g > cap ? cap : g));
+}
+
+}  // namespace
+
+cudaError_t launch_rope_table(int64_t T, int64_t pos0, const double* inv_freq_host, float2* cs, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  rope_table_kernel<<<grid_for(T * 32, 256), 256, 0, s>>>(T, pos0, to_struct(inv_freq_host), cs);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_k(int64_t T, const uint16_t* k, const float2* cs, uint16_t* k_rot, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  rope_k_kernel<<<grid_for(T * 56, 256), 256, 0, s>>>(T, reinterpret_cast<const uint4*>(k), cs,
+                                                        reinterpret_cast<uint4*>(k_rot));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_append(int B, int64_t max_len, const int64_t* L_host, int64_t* L_dev, int64_t* qb_dev,
+                                 const double* inv_freq_host, uint16_t* k_cache, uint16_t* v_cache,
+                                 uint16_t* kidx_cache, uint16_t* qidx_ring, uint16_t* w_ring, const uint16_t* q_new,
+                                 const uint16_t* k_new, const uint16_t* v_new, const uint16_t* q_idx_new,
+                                 const uint16_t* k_idx_new, const uint16_t* w_new, uint16_t* q_rot, cudaStream_t s) {
+  const InvFreq inv = to_struct(inv_freq_host);
+  for (int b0 = 0; b0 < B; b0 += LEN_CHUNK) {
+    const int n = B - b0 < LEN_CHUNK ? B - b0 : LEN_CHUNK;
+    LenChunk lens;
+    lens.b0 = b0;
+    for (int i = 0; i < n; ++i) lens.L[i] = L_host[b0 + i];
+    decode_append_kernel<<<n, 256, 0, s>>>(
+        max_len, lens, L_dev, qb_dev, inv, reinterpret_cast<uint4*>(k_cache), reinterpret_cast<uint4*>(v_cache),
+        reinterpret_cast<uint4*>(kidx_cache), reinterpret_cast<uint4*>(qidx_ring), w_ring,
+        reinterpret_cast<const uint4*>(q_new), reinterpret_cast<const uint4*>(k_new),
+        reinterpret_cast<const uint4*>(v_new), reinterpret_cast<const uint4*>(q_idx_new),
+        reinterpret_cast<const uint4*>(k_idx_new), w_new, reinterpret_cast<uint4*>(q_rot));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace qsa

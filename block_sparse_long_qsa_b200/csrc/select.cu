@@ -1,0 +1,311 @@
+// Stage 2: per-query-block top-k block selection.
+//
+// Page "Qwen3.8-Flash-Next, 1/9의 학습 비용으로 Qwen3.7-Plus(397B-A17B) 수준에
+// 도달한 125B-A6B 모델", section "QSA: 인덱서 자체의 비용을 줄이는 희소 어텐션":
+// token budget K = 2048 with r = 4, i.e. 512 blocks per query; the tail
+// tokens of the own (incomplete) block are always included.  This library's
+// reading: block qb and qb-1 are forced; the other budget-2 slots go to the
+// blocks of [0, qb-2] with the highest score, ties to the lower index, -0.0
+// equal to +0.0; all blocks when qb+1 <= budget; output ascending.
+//
+// Scores are >= 0, so the IEEE bit pattern with the sign cleared orders them
+// as unsigned integers.  One CTA per row:
+//   1. rows with at most CAP candidates are loaded whole into shared memory;
+//      longer rows draw a strided sample of 2048 scores whose order statistic
+//      at a safely conservative rank gives a threshold, and one coalesced
+//      pass keeps the scores at or above it (ballot-compacted) -- a few
+//      thousand candidates out of up to 262,143;
+//   2. an exact MSB-first radix select (8-bit digits, shared histograms)
+//      finds the k-th largest key among the candidates; ties at the threshold
+//      are resolved by a second radix select on the block indices;
+//   3. if the sample's threshold left fewer than k or more than CAP
+//      candidates (rare), the same radix select runs over the whole row in
+//      global memory and an index-ordered pass collects the winners;
+//   4. the winners plus the two forced blocks are bitonic-sorted ascending.
+#include <climits>
+
+#include "qsa_device.cuh"
+#include "qsa_kernels.h"
+
+namespace qsa {
+namespace {
+
+constexpr int THREADS = 512;
+constexpr int NSAMPLE = 2048;
+
+__host__ __device__ inline int cap_for(int budget) {
+  int c = 3 * budget;
+  if (c < 6144) c = 6144;
+  if (c > 16384) c = 16384;
+  return c;
+}
+__host__ __device__ inline int pow2_at_least(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+struct SelSmem {
+  uint32_t* hist;   // [256]
+  uint32_t* misc;   // [16]
+  uint32_t* warp_tot;  // [32]
+  uint32_t* sample; // [NSAMPLE]
+  uint32_t* ckey;   // [cap]
+  int32_t* cidx;    // [cap]
+  int32_t* out;     // [pow2(budget)]
+};
+
+__device__ __forceinline__ uint32_t key_of(float x) { return __float_as_uint(x) & 0x7FFFFFFFu; }
+
+// k-th largest (1-based k, 1 <= k <= n) of get(0..n-1) by MSB-first radix
+// select.  Returns the key and the number of elements strictly greater.
+template <class Get>
+__device__ void radix_kth_largest(Get get, int64_t n, int64_t k, const SelSmem& sm, uint32_t& tau, int64_t& n_gt) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t prefix = 0, mask = 0;
+  int64_t kk = k;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tid; i < 256; i += blockDim.x) sm.hist[i] = 0;
+    __syncthreads();
+    for (int64_t i = tid; i < n; i += blockDim.x) {
+      const uint32_t key = get(i);
+      if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t c[8], s = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) { c[q] = sm.hist[255 - 8 * lane - q]; s += c[q]; }
+      uint32_t incl = s;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      const uint32_t excl = incl - s;
+      if ((int64_t)excl < kk && kk <= (int64_t)incl) {
+        uint32_t cum = excl;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (cum + c[q] >= kk) {
+            sm.misc[0] = (uint32_t)(255 - 8 * lane - q);
+            sm.misc[1] = (uint32_t)(kk - cum);
+            break;
+          }
+          cum += c[q];
+        }
+      }
+    }
+    __syncthreads();
+    const uint32_t bin = sm.misc[0];
+    kk = sm.misc[1];
+    prefix |= bin << shift;
+    mask |= 0xFFu << shift;
+    __syncthreads();
+  }
+  tau = prefix;
+  n_gt = k - kk;
+}
+
+// Block-wide exclusive prefix count of `flag` in thread order; returns the
+// block total through *total.
+__device__ __forceinline__ uint32_t block_excl_count(bool flag, const SelSmem& sm, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const uint32_t ball = __ballot_sync(0xffffffffu, flag);
+  const uint32_t in_warp = __popc(ball & ((1u << lane) - 1u));
+  if (lane == 0) sm.warp_tot[warp] = __popc(ball);
+  __syncthreads();
+  uint32_t before = 0, tot = 0;
+  for (int w = 0; w < nwarps; ++w) {
+    const uint32_t v = sm.warp_tot[w];
+    if (w < warp) before += v;
+    tot += v;
+  }
+  __syncthreads();
+  *total = tot;
+  return before + in_warp;
+}
+
+__global__ void __launch_bounds__(THREADS)
+select_kernel(const float* __restrict__ S, int64_t ld, int64_t qb_begin, int64_t n_rows,
+              const int64_t* __restrict__ row_qb, int budget, int32_t* __restrict__ sel, int32_t* __restrict__ cnt,
+              uint32_t* err) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const int cap = cap_for(budget);
+  const int P = pow2_at_least(budget);
+  SelSmem sm;
+  sm.hist = reinterpret_cast<uint32_t*>(smem_raw);
+  sm.misc = sm.hist + 256;
+  sm.warp_tot = sm.misc + 16;
+  sm.sample = sm.warp_tot + 32;
+  sm.ckey = sm.sample + NSAMPLE;
+  sm.cidx = reinterpret_cast<int32_t*>(sm.ckey + cap);
+  sm.out = sm.cidx + cap;
+  const int tid = threadIdx.x, lane = tid & 31;
+
+  for (int64_t r = blockIdx.x; r < n_rows; r += gridDim.x) {
+    const int64_t qb = row_qb ? row_qb[r] : qb_begin + r;
+    const float* row = S + r * ld;
+    int32_t* srow = sel + r * budget;
+    if (qb + 1 <= budget) {
+      for (int i = tid; i < budget; i += blockDim.x) srow[i] = i <= qb ? i : -1;
+      if (tid == 0) cnt[r] = (int32_t)(qb + 1);
+      continue;
+    }
+    const int64_t m = qb - 1;          // candidates 0 .. qb-2
+    const int64_t k = budget - 2;
+    if (tid == 0) { sm.misc[2] = 0; sm.misc[3] = 0; }
+    __syncthreads();
+
+    bool global_path = false;
+    int64_t nc = 0;
+    if (k == 0) {
+      // budget 2: only the forced blocks
+    } else if (m <= cap) {
+      for (int64_t i = tid; i < m; i += blockDim.x) {
+        sm.ckey[i] = key_of(row[i]);
+        sm.cidx[i] = (int32_t)i;
+      }
+      nc = m;
+    } else {
+      // 1. threshold from a strided sample
+      for (int i = tid; i < NSAMPLE; i += blockDim.x) sm.sample[i] = key_of(row[(int64_t)i * m / NSAMPLE]);
+      const float e = (float)NSAMPLE * (float)k / (float)m;
+      int64_t rs = (int64_t)ceilf(e + 4.f * sqrtf(e) + 8.f);
+      if (rs > NSAMPLE) rs = NSAMPLE;
+      __syncthreads();
+      uint32_t tau0;
+      int64_t dummy;
+      radix_kth_largest([&](int64_t i) { return sm.sample[i]; }, NSAMPLE, rs, sm, tau0, dummy);
+      // 2. filter pass: keep key >= tau0 (row start is 16-byte aligned: ld % 4 == 0)
+      const float4* row4 = reinterpret_cast<const float4*>(row);
+      const int64_t m4 = (m + 3) >> 2;
+      for (int64_t i4 = tid; i4 - tid < m4; i4 += blockDim.x) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i4 < m4) v = row4[i4];
+        const float vals[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int64_t idx = 4 * i4 + q;
+          const bool pass = idx < m && key_of(vals[q]) >= tau0;
+          const uint32_t ball = __ballot_sync(0xffffffffu, pass);
+          if (ball) {
+            uint32_t base = 0;
+            if (lane == 0) base = atomicAdd(&sm.misc[2], (uint32_t)__popc(ball));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            const uint32_t pos = base + __popc(ball & ((1u << lane) - 1u));
+            if (pass && pos < (uint32_t)cap) { sm.ckey[pos] = key_of(vals[q]); sm.cidx[pos] = (int32_t)idx; }
+          }
+        }
+      }
+      __syncthreads();
+      nc = sm.misc[2];
+      global_path = (nc < k || nc > cap);
+      __syncthreads();
+    }
+
+    if (k == 0) {
+      if (tid == 0) sm.misc[2] = 0;
+      __syncthreads();
+    } else if (!global_path) {
+      __syncthreads();
+      uint32_t tau;
+      int64_t n_gt;
+      radix_kth_largest([&](int64_t i) { return sm.ckey[i]; }, nc, k, sm, tau, n_gt);
+      const int64_t need = k - n_gt;
+      // count ties
+      if (tid == 0) { sm.misc[2] = 0; sm.misc[4] = 0; }
+      __syncthreads();
+      for (int64_t i = tid; i < nc; i += blockDim.x)
+        if (sm.ckey[i] == tau) atomicAdd(&sm.misc[4], 1u);
+      __syncthreads();
+      const int64_t n_eq = sm.misc[4];
+      uint32_t idx_cut = 0xFFFFFFFFu;   // take ties with index <= idx_cut
+      if (n_eq > need) {
+        uint32_t ntau;
+        int64_t d2;
+        radix_kth_largest([&](int64_t i) { return sm.ckey[i] == tau ? ~(uint32_t)sm.cidx[i] : 0u; }, nc, need, sm,
+                          ntau, d2);
+        idx_cut = ~ntau;
+      }
+      for (int64_t i = tid; i < nc; i += blockDim.x) {
+        const uint32_t key = sm.ckey[i];
+        const bool take = key > tau || (key == tau && (uint32_t)sm.cidx[i] <= idx_cut);
+        if (take) {
+          const uint32_t pos = atomicAdd(&sm.misc[2], 1u);
+          if (pos < (uint32_t)k) sm.out[pos] = sm.cidx[i];
+        }
+      }
+      __syncthreads();
+    } else {
+      // 3. exact selection over the row in global memory
+      uint32_t tau;
+      int64_t n_gt;
+      radix_kth_largest([&](int64_t i) { return key_of(row[i]); }, m, k, sm, tau, n_gt);
+      const int64_t need = k - n_gt;
+      if (tid == 0) sm.misc[2] = 0;
+      __syncthreads();
+      int64_t eq_taken = 0;
+      for (int64_t base = 0; base < m; base += blockDim.x) {
+        const int64_t i = base + tid;
+        const uint32_t key = i < m ? key_of(row[i]) : 0u;
+        const bool gt = i < m && key > tau;
+        const bool eq = i < m && key == tau;
+        uint32_t tot;
+        const uint32_t rank = block_excl_count(eq, sm, &tot);
+        if (gt || (eq && eq_taken + (int64_t)rank < need)) {
+          const uint32_t pos = atomicAdd(&sm.misc[2], 1u);
+          if (pos < (uint32_t)k) sm.out[pos] = (int32_t)i;
+        }
+        eq_taken += tot;
+      }
+      __syncthreads();
+    }
+    if (tid == 0 && sm.misc[2] != (uint32_t)k) report_error(err, QSA_ERR_DEVICE_BOUNDS);
+    // 4. forced blocks, then ascending sort of the budget entries
+    if (tid == 0) { sm.out[k] = (int32_t)(qb - 1); sm.out[k + 1] = (int32_t)qb; }
+    for (int i = budget + tid; i < P; i += blockDim.x) sm.out[i] = INT_MAX;
+    __syncthreads();
+    for (int size = 2; size <= P; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        for (int i = tid; i < P / 2; i += blockDim.x) {
+          const int lo = 2 * i - (i & (stride - 1));
+          const int hi = lo + stride;
+          const bool up = (lo & size) == 0;
+          const int32_t a = sm.out[lo], b = sm.out[hi];
+          if ((a > b) == up) { sm.out[lo] = b; sm.out[hi] = a; }
+        }
+        __syncthreads();
+      }
+    }
+    for (int i = tid; i < budget; i += blockDim.x) srow[i] = sm.out[i];
+    if (tid == 0) cnt[r] = budget;
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+size_t select_smem_bytes(int budget) {
+  const int cap = cap_for(budget);
+  return (size_t)(256 + 16 + 32 + NSAMPLE) * 4 + (size_t)cap * 8 + (size_t)pow2_at_least(budget) * 4;
+}
+
+cudaError_t launch_select(const float* S, int64_t ld, int64_t qb_begin, int64_t n_rows, const int64_t* row_qb,
+                          int budget, int32_t* sel, int32_t* cnt, uint32_t* err, cudaStream_t stream) {
+  if (n_rows <= 0) return cudaSuccess;
+  const size_t smem = select_smem_bytes(budget);
+  static size_t attr_set[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && attr_set[dev] < smem) {
+    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = smem;
+  }
+  const int64_t grid = n_rows < 148 * 64 ? n_rows : 148 * 64;
+  select_kernel<<<(unsigned)grid, THREADS, smem, stream>>>(S, ld, qb_begin, n_rows, row_qb, budget, sel, cnt, err);
+  return cudaGetLastError();
+}
+
+}  // namespace qsa

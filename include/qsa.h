@@ -1,0 +1,159 @@
+/*
+ * qsa.h -- C ABI of the QSA (Qwen Sparse Attention) hot path for NVIDIA B200 (sm_100a).
+ *
+ * QSA is the micro-block sparse global attention layer described on the page
+ * "Qwen3.8-Flash-Next, 1/9의 학습 비용으로 Qwen3.7-Plus(397B-A17B) 수준에 도달한
+ * 125B-A6B 모델" (discuss.pytorch.kr), cited below as [PT]; section
+ * "QSA: 인덱서 자체의 비용을 줄이는 희소 어텐션" ([PT §QSA]) and its spec table.
+ * It runs in three stages:
+ *   1. an MQA indexer (4 query heads, one shared 128-dim key head) scores the
+ *      causal key micro-blocks of r = 4 tokens for every query micro-block;
+ *   2. a top-k step keeps `budget_blocks` = 512 blocks (2048 tokens) per query
+ *      block, always including the query block itself and the one before it;
+ *   3. GQA softmax attention (24 Q heads, 2 KV heads, head dim 256, RoPE with
+ *      theta = 1e7 on dims 0..63) runs over the selected blocks only.
+ *
+ * Conventions (all calls):
+ *   - Every pointer argument is a DEVICE pointer unless marked "host", 16-byte
+ *     aligned, to a contiguous row-major array with the layout given.  bf16
+ *     values travel as uint16_t bit patterns.
+ *   - The caller owns every buffer, the workspace included; the library
+ *     allocates no device memory.  Its only global state is the one-time
+ *     kernel attribute setup per device.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  Arguments are validated on the host before any launch; on an
+ *     argument error nothing is launched.
+ *   - Errors come back as a qsa_status; nothing aborts or throws.  Errors
+ *     detected on the device (a bounded wait that timed out) are recorded in
+ *     the workspace's error word and read back by qsa_check_device_error.
+ *   - Positions: token t of a prefill sits at position pos0 + t.
+ */
+#ifndef QSA_H_
+#define QSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QSA_OK = 0,
+  QSA_ERR_INVALID_ARG = 1,         /* null pointer, negative size, bad range */
+  QSA_ERR_UNSUPPORTED = 2,         /* shape other than the one this library implements */
+  QSA_ERR_MISALIGNED = 3,          /* a pointer is not 16-byte aligned */
+  QSA_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes below the *_workspace_size minimum */
+  QSA_ERR_CUDA = 5,                /* a CUDA runtime / driver call failed */
+  QSA_ERR_DEVICE_TIMEOUT = 6,      /* a device-side bounded wait gave up */
+  QSA_ERR_DEVICE_BOUNDS = 7,       /* a device-side index check failed */
+  QSA_ERR_ARCH = 8                 /* the current device is not sm_100 */
+} qsa_status;
+
+/* Layer shape.  The implemented (and only accepted) values are the ones of
+ * [PT] spec table ("Qwen Sparse Attention", "QSA 인덱서", "QSA 예산") and of the
+ * rope_parameters listing in [PT] section "100만 토큰까지 늘리기":
+ * n_q_heads 24, n_kv_heads 2, head_dim 256, rope_dim 64, rope_theta 1e7,
+ * idx_heads 4, idx_dim 128, block_size 4; budget_blocks is free in [2, 4096]
+ * (default 512).  softmax_scale 0 means 1/sqrt(head_dim). */
+typedef struct {
+  int32_t n_q_heads;
+  int32_t n_kv_heads;
+  int32_t head_dim;
+  int32_t rope_dim;
+  double rope_theta;
+  int32_t idx_heads;
+  int32_t idx_dim;
+  int32_t block_size;
+  int32_t budget_blocks;
+  float softmax_scale;
+} qsa_params;
+
+/* Fills *p with the values above (budget 512). */
+void qsa_default_params(qsa_params* p);
+
+/* Human-readable name of a status code (static storage). */
+const char* qsa_status_string(qsa_status s);
+
+/* Stage 1 -- indexer block scores ([PT §QSA], eq. I_ib, with the head
+ * weights and causal block-max of this library's reading):
+ *   s(t, j)   = sum_h w[t][h] * ReLU(q_idx[t][h] . k_idx[j]) / sqrt(idx_dim)
+ *   S(qb, kb) = max over tokens t of block qb (t < T) and j of block kb with
+ *               j <= t of s(t, j),   for kb <= qb.
+ * q_idx [T][4][128] bf16, w [T][4] bf16, k_idx [T][128] bf16.
+ * Writes scores[(qb - qb_begin) * ld + kb] (fp32) for qb in [qb_begin, qb_end)
+ * and kb <= qb; entries with kb > qb are not written.
+ * Requires 0 <= qb_begin <= qb_end <= ceil(T/4), ld >= qb_end, ld % 4 == 0.
+ * ws (nullable, >= 256 bytes) receives the device error word; with ws NULL a
+ * device-side timeout is not reported (the kernel still exits). */
+qsa_status qsa_index_scores(const qsa_params* p, int64_t T, const uint16_t* q_idx, const uint16_t* w,
+                            const uint16_t* k_idx, int64_t qb_begin, int64_t qb_end, float* scores, int64_t ld,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* Stage 2 -- block selection ([PT §QSA]: token budget K = 2048, r = 4, so
+ * 512 blocks; the tail of the own block is always included).  For query
+ * block qb (row qb - qb_begin of `scores`, entries kb <= qb valid):
+ *   qb + 1 <= budget: all blocks 0..qb;
+ *   otherwise: qb and qb-1, plus the (budget-2) blocks of [0, qb-2] with the
+ *   highest score (ties to the lower block index; -0.0 counts as +0.0).
+ * sel [qb_end-qb_begin][budget] int32 ascending, padded with -1; cnt [..] int32.
+ * ws: at least qsa_select_workspace_size() bytes (holds the error word). */
+qsa_status qsa_select_blocks(const qsa_params* p, const float* scores, int64_t ld, int64_t qb_begin,
+                             int64_t qb_end, int32_t* sel, int32_t* cnt, void* ws, size_t ws_bytes, void* stream);
+qsa_status qsa_select_workspace_size(const qsa_params* p, size_t* bytes);
+
+/* Whole prefill: RoPE on Q and K, stage 1, stage 2 and stage 3 (sparse GQA
+ * attention over the selected blocks, causal inside the own block):
+ *   out[t][h] = sum_j softmax_j(q_rot[t][h] . k_rot[j][h/12] * scale) v[j][h/12]
+ *   over j in the selected blocks of block t/4 with j <= t;
+ *   lse[t][h] = log sum_j exp(logit_j).
+ * q [T][24][256], k [T][2][256] (not rotated), v [T][2][256], q_idx [T][4][128],
+ * w [T][4], k_idx [T][128]: bf16.  out [T][24][256] bf16.
+ * Optional (NULL to skip): lse [T][24] fp32; sel_out [ceil(T/4)][budget] and
+ * cnt_out [ceil(T/4)] int32; k_rot_out [T][2][256] bf16 (the rotated keys, to
+ * seed a decode cache).
+ * ws: at least the minimum of qsa_prefill_workspace_size; a larger workspace
+ * lets the call score more query blocks per pass (fewer, larger launches). */
+qsa_status qsa_prefill(const qsa_params* p, int64_t T, int64_t pos0, const uint16_t* q, const uint16_t* k,
+                       const uint16_t* v, const uint16_t* q_idx, const uint16_t* w, const uint16_t* k_idx,
+                       uint16_t* out, float* lse, int32_t* sel_out, int32_t* cnt_out, uint16_t* k_rot_out, void* ws,
+                       size_t ws_bytes, void* stream);
+/* min_bytes: smallest workspace qsa_prefill accepts; pref_bytes: the size
+ * that scores every query block in one pass, capped at 16 GiB (either
+ * pointer may be NULL). */
+qsa_status qsa_prefill_workspace_size(const qsa_params* p, int64_t T, size_t* min_bytes, size_t* pref_bytes);
+
+/* One decode step for B sequences.  Sequence b has cache_len[b] (host array)
+ * tokens already in its caches; the new token sits at position
+ * L = cache_len[b] and is appended: k_cache[b][L] = RoPE(k_new[b], L),
+ * v_cache[b][L] = v_new[b], kidx_cache[b][L] = k_idx_new[b],
+ * qidx_ring[b][L % 4] = q_idx_new[b], w_ring[b][L % 4] = w_new[b].
+ * The new token's query block qb = L / 4 is scored over the present
+ * block-mates 4*qb .. L (their indexer queries come from the ring, which the
+ * caller seeds for tokens 4*qb .. L-1 when the decode starts mid-block), the
+ * blocks are selected as in stage 2, and attention for the new token runs over
+ * them -- by construction what a prefill of L+1 tokens gives for its last
+ * token ([PT §QSA]; the full KV cache is kept).  The caller increments
+ * cache_len afterwards.
+ * k_cache, v_cache [B][max_len][2][256] bf16 (keys rotated); kidx_cache
+ * [B][max_len][128]; qidx_ring [B][4][4][128]; w_ring [B][4][4];
+ * q_new [B][24][256]; k_new, v_new [B][2][256]; q_idx_new [B][4][128];
+ * k_idx_new [B][128]; w_new [B][4]  ->  out [B][24][256] bf16;
+ * sel_out [B][budget] int32 (nullable), lse_out [B][24] fp32 (nullable).
+ * Requires cache_len[b] < max_len, B <= 4096. */
+qsa_status qsa_decode(const qsa_params* p, int32_t B, int64_t max_len, const int64_t* cache_len,
+                      uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* qidx_ring,
+                      uint16_t* w_ring, const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
+                      const uint16_t* q_idx_new, const uint16_t* k_idx_new, const uint16_t* w_new, uint16_t* out,
+                      int32_t* sel_out, float* lse_out, void* ws, size_t ws_bytes, void* stream);
+qsa_status qsa_decode_workspace_size(const qsa_params* p, int32_t B, int64_t max_len, size_t* bytes);
+
+/* Reads (synchronising `stream`) and clears the device error word at the
+ * start of a workspace passed to qsa_select_blocks / qsa_prefill /
+ * qsa_decode.  Returns QSA_OK or the first device-side error recorded. */
+qsa_status qsa_check_device_error(void* ws, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QSA_H_ */

@@ -1,0 +1,178 @@
+"""GPU parity of the prefill path (C ABI) against the CPU oracle."""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_long_qsa_b200 as qsa
+import oracle
+import qsa_inputs as Q
+from gpu_util import (SCORE_RTOL, check_outputs, check_selection, dev, gpu_prefill)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from block_sparse_long_qsa_b200 import _build
+    _build.build()
+    qsa.load()
+
+
+def _scores_gpu(P, host, qb_begin=0, qb_end=None, ld=None):
+    T = P.T
+    nqb = P.nqb
+    qb_end = nqb if qb_end is None else qb_end
+    ld = ld or ((qb_end + 3) // 4 * 4)
+    S = torch.full((qb_end - qb_begin, ld), float("nan"), dtype=torch.float32, device="cuda")
+    ws = qsa.workspace(256)
+    qsa.qsa_index_scores(qsa.params(), T, dev(host["q_idx"]), dev(host["w"]), dev(host["k_idx"]), qb_begin, qb_end,
+                         S, ld, ws)
+    torch.cuda.synchronize()
+    assert qsa.qsa_check_device_error(ws) == 0
+    return S.cpu().numpy().astype(np.float64)
+
+
+@pytest.mark.parametrize("T", [1, 3, 5, 64, 256, 333, 1000, 4099])
+def test_index_scores_vs_oracle(T):
+    P = Q.PrefillProblem(T=T, seed=T, n_plant=3)
+    host = P.host()
+    got = _scores_gpu(P, host)
+    want = oracle.Oracle().index_scores(T, host["q_idx"], host["w"], host["k_idx"], ld=got.shape[1])
+    causal = ~np.isnan(want)
+    assert np.isnan(got[~causal]).all(), "entries with kb > qb must not be written"
+    g, w = got[causal], want[causal]
+    err = np.abs(g - w) / np.maximum(np.abs(w), 1e-3)
+    assert err.max() <= SCORE_RTOL, f"T={T}: max rel err {err.max():.3e}"
+
+
+def test_index_scores_subrange():
+    """A chunk [qb_begin, qb_end) with its own row offset and a wide ld."""
+    T = 3000
+    P = Q.PrefillProblem(T=T, seed=7, n_plant=4)
+    host = P.host()
+    got = _scores_gpu(P, host, 301, 555, ld=1000)
+    want = oracle.Oracle().index_scores(T, host["q_idx"], host["w"], host["k_idx"], 301, 555, ld=1000)
+    m = ~np.isnan(want)
+    assert np.isnan(got[~m]).all()
+    err = np.abs(got[m] - want[m]) / np.maximum(np.abs(want[m]), 1e-3)
+    assert err.max() <= SCORE_RTOL
+
+
+def _select_exact_cpu(row32: np.ndarray, qb: int, budget: int) -> np.ndarray:
+    """Reference on the SAME fp32 values: forced qb, qb-1; top (budget-2) of
+    [0, qb-2] by (value desc, index asc), -0.0 == +0.0; ascending."""
+    if qb + 1 <= budget:
+        return np.arange(qb + 1)
+    vals = row32[:qb - 1].astype(np.float64) + 0.0
+    cand = np.arange(qb - 1)
+    order = np.lexsort((cand, -vals))
+    return np.sort(np.concatenate([cand[order[:budget - 2]], [qb - 1, qb]]))
+
+
+@pytest.mark.parametrize("budget", [2, 16, 512])
+def test_select_exact_on_given_scores(budget):
+    """Index work is bit-exact: the GPU select on fp32 rows equals the CPU
+    reference on the same values, including ties, -0.0 and long rows that
+    take the sampled-threshold path."""
+    rng = np.random.default_rng(budget)
+    qbs = np.array([0, 1, budget - 2, budget - 1, budget, budget + 1, 700, 6145, 7000, 20000, 70000])
+    qbs = qbs[qbs >= 0]
+    ld = int((qbs.max() + 1 + 3) // 4 * 4)
+    rows = np.zeros((len(qbs), ld), dtype=np.float32)
+    for i, qb in enumerate(qbs):
+        r = rng.gamma(4.0, 0.5, size=qb + 1).astype(np.float32)
+        if i % 3 == 0:
+            r = np.round(r * 8) / 8          # many exact ties
+        if i % 4 == 1:
+            r[::7] = -0.0
+        rows[i, :qb + 1] = r
+    # the select kernel takes rows for consecutive qb; run one row at a time
+    p = qsa.params(budget)
+    ws = qsa.workspace(qsa.qsa_select_workspace_size(p))
+    for i, qb in enumerate(qbs):
+        S = dev(rows[i:i + 1])
+        sel = torch.empty((1, budget), dtype=torch.int32, device="cuda")
+        cnt = torch.empty((1,), dtype=torch.int32, device="cuda")
+        qsa.qsa_select_blocks(p, S, ld, int(qb), int(qb) + 1, sel, cnt, ws)
+        torch.cuda.synchronize()
+        assert qsa.qsa_check_device_error(ws) == 0
+        want = _select_exact_cpu(rows[i], int(qb), budget)
+        c = int(cnt.item())
+        s = sel.cpu().numpy()[0]
+        assert c == len(want), (qb, c, len(want))
+        assert np.array_equal(s[:c], want), qb
+        assert np.all(s[c:] == -1)
+
+
+def test_select_all_equal_rows():
+    """Degenerate rows (all scores equal) go through the exact fallback."""
+    budget = 512
+    p = qsa.params(budget)
+    ws = qsa.workspace(qsa.qsa_select_workspace_size(p))
+    for qb in (9000, 40000):
+        ld = (qb + 1 + 3) // 4 * 4
+        S = torch.zeros((1, ld), dtype=torch.float32, device="cuda")
+        sel = torch.empty((1, budget), dtype=torch.int32, device="cuda")
+        cnt = torch.empty((1,), dtype=torch.int32, device="cuda")
+        qsa.qsa_select_blocks(p, S, ld, qb, qb + 1, sel, cnt, ws)
+        torch.cuda.synchronize()
+        want = np.concatenate([np.arange(budget - 2), [qb - 1, qb]])
+        assert np.array_equal(sel.cpu().numpy()[0], want)
+
+
+@pytest.mark.parametrize("T,budget", [(256, 16), (256, 64), (1, 16), (7, 16), (301, 16), (2053, 64)])
+def test_prefill_small_vs_oracle(T, budget):
+    P = Q.PrefillProblem(T=T, seed=100 + T, n_plant=3)
+    host, r = gpu_prefill(P, budget)
+    O = oracle.Oracle(oracle.params(budget=budget))
+    nqb = P.nqb
+    S = O.index_scores(T, host["q_idx"], host["w"], host["k_idx"])
+    osel, ocnt = O.select_rows(np.nan_to_num(S, nan=-1.0))
+    for qb in range(nqb):
+        check_selection(r["sel"][qb], int(r["cnt"][qb]), osel[qb], int(ocnt[qb]), S[qb], qb, budget, f"qb={qb}")
+    out, lse = O.attend_blocks(T, host["q"], host["k"], host["v"], np.arange(nqb), r["sel"], r["cnt"])
+    check_outputs(r["out"], out[:T], f"T={T} budget={budget}")
+    assert np.allclose(r["lse"], lse[:T], atol=1e-2, rtol=1e-3)
+    # k_rot_out: keys rotated by the oracle's RoPE, rounded to bf16
+    kr = np.stack([[O.rope(Q.bf16_to_f64(host["k"][t, g]), t) for g in range(2)] for t in range(min(T, 64))])
+    assert np.abs(Q.bf16_to_f64(r["k_rot"][:len(kr)]) - kr).max() < 0.05
+
+
+def test_prefill_dense_when_budget_covers():
+    """Budget 64 >= 64 blocks at T = 256: the selection is every causal block
+    and the output is dense causal GQA attention."""
+    T, budget = 256, 64
+    P = Q.PrefillProblem(T=T, seed=0, n_plant=3)
+    host, r = gpu_prefill(P, budget)
+    assert np.array_equal(r["cnt"], np.arange(1, 65))
+    for qb in range(64):
+        assert np.array_equal(r["sel"][qb][:qb + 1], np.arange(qb + 1))
+    from oracle_pins import _dense_causal_sdpa
+    want, want_lse = _dense_causal_sdpa(host["q"], host["k"], host["v"])
+    check_outputs(r["out"], want, "dense")
+
+
+def test_prefill_pos0_offset():
+    """Positions start at pos0: rotating with an offset changes the output
+    exactly as the oracle's RoPE does."""
+    T, budget, pos0 = 300, 16, 5000
+    P = Q.PrefillProblem(T=T, seed=3, n_plant=3)
+    host = P.host()
+    t = {k: dev(v) for k, v in host.items()}
+    rr = qsa.prefill(t["q"], t["k"], t["v"], t["q_idx"], t["w"], t["k_idx"], budget=budget, pos0=pos0)
+    torch.cuda.synchronize()
+    O = oracle.Oracle(oracle.params(budget=budget))
+    sel, cnt = rr["sel"].cpu().numpy(), rr["cnt"].cpu().numpy()
+    out, _ = O.attend_blocks(T, host["q"], host["k"], host["v"], np.arange(P.nqb), sel, cnt, pos0=pos0)
+    check_outputs(rr["out"].cpu().numpy(), out[:T], "pos0")
+
+
+def test_prefill_chunked_workspace_matches_single_pass():
+    """A workspace that forces many chunks gives the same result as one pass."""
+    T, budget = 8192, 64
+    P = Q.PrefillProblem(T=T, seed=11, n_plant=8)
+    host, r1 = gpu_prefill(P, budget)
+    mn, _ = qsa.qsa_prefill_workspace_size(qsa.params(budget), T)
+    _, r2 = gpu_prefill(P, budget, host=host, ws_bytes=mn)
+    assert np.array_equal(r1["sel"], r2["sel"]) and np.array_equal(r1["cnt"], r2["cnt"])
+    assert np.array_equal(r1["out"], r2["out"])
