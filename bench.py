@@ -1,0 +1,526 @@
+"""QSA hot-path benchmark on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One "step" is one pass of the whole hot path (RoPE, indexer, top-k select,
+sparse attention; for decode also the cache append and the split-KV combine)
+over one batch of synthetic input resident in HBM, through the C ABI.  The
+default workload is the 1M-token prefill; decode 64 x 256K and the 128K
+prefill are measured in the same run as secondary lines.  With --gpus N (one
+process per GPU under torchrun) every rank runs its own independent sequence
+(weak scaling, no collective: sequences are independent problems).
+
+--impl reference times the CPU oracle (the deliberately slow fp64 definition)
+on a bounded sample of the same workload, on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import qsa_inputs as Q  # noqa: E402
+
+L2_BYTES = 126 * (1 << 20)
+
+
+def peaks():
+    try:
+        m = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return dict(hbm=m["hbm_gbs"], bf16=m["bf16_tflops"], bf16_sus=m["bf16_tflops_sustained"], src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"], stdout=subprocess.PIPE,
+                                      stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.p = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.p is not None:
+            self.p.terminate()
+            try:
+                out, _ = self.p.communicate(timeout=5)
+            except Exception:
+                self.p.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------- distributed
+def dist_setup(n_gpus: int):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------ prefill workload
+def prefill_flops(T: int, sel_cnt: np.ndarray | None):
+    """Algorithmic tensor FLOPs: indexer 1024 * T(T+1)/2 (4 heads x 128 x 2 per
+    causal token pair); attention 4 * 24 * 256 * sum_t |J(t)| (QK^T and PV)."""
+    idx = 1024.0 * T * (T + 1) / 2
+    if sel_cnt is None:
+        keys = min(T, 2048) * T
+    else:
+        # |J(t)| = 4 * cnt - (tokens of the own block after t)
+        keys = float(4 * sel_cnt.astype(np.int64).sum() * 4) - 6.0 * len(sel_cnt)
+    attn = 4.0 * 24 * 256 * keys
+    return idx, attn
+
+
+def run_prefill(T: int, budget: int, steps: int, warmup: int, rank: int, world: int, seed: int, want_e2e=True):
+    import block_sparse_long_qsa_b200 as qsa
+    P = Q.PrefillProblem(T=T, seed=seed + 1000 * rank, n_plant=8, dist="zipf" if T >= 131072 else "uniform")
+    d = P.device()
+    torch.cuda.synchronize()
+    p = qsa.params(budget)
+    mn, pref = qsa.qsa_prefill_workspace_size(p, T)
+    ws = qsa.workspace(pref)
+    nqb = P.nqb
+    out = torch.empty((T, 24, 256), dtype=torch.uint16, device="cuda")
+    sel = torch.empty((nqb, budget), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((nqb,), dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        qsa.qsa_prefill(p, T, 0, d["q"], d["k"], d["v"], d["q_idx"], d["w"], d["k_idx"], out, None, sel, cnt, None,
+                        ws, stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if qsa.qsa_check_device_error(ws) != 0:
+        raise RuntimeError("device error during warm-up")
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk, qsa.trace(capacity=64 * steps + 64) as tr:
+        ev0.record(stream)
+        for _ in range(steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = ev0.elapsed_time(ev1)
+    ms_max = max_over_ranks(ms, world)
+    if qsa.qsa_check_device_error(ws) != 0:
+        raise RuntimeError("device error during the timed steps")
+    cnt_h = cnt.cpu().numpy()
+    fl_idx, fl_attn = prefill_flops(T, cnt_h)
+    kern = tr.by_kernel()
+    launches = sum(c for c, _ in kern.values())
+    res = dict(ms=ms_max, tokens=T * steps * world, kern=kern, launches=launches, clocks=clk.summary(),
+               flops_idx=fl_idx, flops_attn=fl_attn, steps=steps)
+
+    if want_e2e:
+        # end to end through the public call with host buffers: pinned inputs
+        # copied in, the attention output copied back, every step
+        names = ["q", "k", "v", "q_idx", "w", "k_idx"]
+        host = {k: torch.empty(d[k].shape, dtype=d[k].dtype, pin_memory=True) for k in names}
+        for k in names:
+            host[k].copy_(d[k])
+        out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        torch.cuda.synchronize()
+        bi = sum(host[k].numel() * host[k].element_size() for k in names)
+        bo = out_h.numel() * out_h.element_size()
+        e_steps = max(1, min(steps, 3))
+
+        def e2e_step():
+            for k in names:
+                d[k].copy_(host[k], non_blocking=True)
+            step()
+            out_h.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        ems = max_over_ranks(e0.elapsed_time(e1), world)
+        res["e2e"] = dict(value=T * e_steps * world / (ems / 1e3), unit="tokens/s", h2d_bytes_per_step=bi,
+                          d2h_bytes_per_step=bo, steps=e_steps)
+        del host, out_h
+    del d, ws, out, sel
+    torch.cuda.empty_cache()
+    return res
+
+
+# ------------------------------------------------------------- decode workload
+def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, world: int, seed: int,
+               want_e2e=True):
+    import block_sparse_long_qsa_b200 as qsa
+    n_total = warmup + steps + (min(steps, 3) + 1 if want_e2e else 0)
+    D = Q.DecodeProblem(B=B, L=L, steps=n_total, seed=seed + 1000 * rank, n_plant=8)
+    max_len = L + n_total + 4
+    kc = torch.empty((B, max_len, 2, 256), dtype=torch.uint16, device="cuda")
+    vc = torch.empty_like(kc)
+    ic = torch.empty((B, max_len, 128), dtype=torch.uint16, device="cuda")
+    D.fill_device_caches(kc, vc, ic)
+    ring = torch.zeros((B, 4, 4, 128), dtype=torch.uint16, device="cuda")
+    wring = torch.zeros((B, 4, 4), dtype=torch.uint16, device="cuda")
+    p = qsa.params(budget)
+    ws = qsa.workspace(qsa.qsa_decode_workspace_size(p, B, max_len))
+    out = torch.empty((B, 24, 256), dtype=torch.uint16, device="cuda")
+    # per-step inputs, generated once (host) and kept resident
+    names = ["q", "k", "v", "q_idx", "k_idx", "w"]
+    step_in = []
+    for s in range(n_total):
+        x = D.step_inputs(s)
+        t = L + s
+        x["k_idx"] = np.stack([D.tokens(b).k_idx(t, t + 1)[0] for b in range(B)])
+        step_in.append({k: torch.from_numpy(np.ascontiguousarray(x[k])).cuda() for k in names})
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    pos = [L]
+
+    def step(x):
+        qsa.qsa_decode(p, B, max_len, [pos[0]] * B, kc, vc, ic, ring, wring, x["q"], x["k"], x["v"], x["q_idx"],
+                       x["k_idx"], x["w"], out, ws=ws, stream=stream)
+        pos[0] += 1
+
+    si = 0
+    for _ in range(warmup):
+        step(step_in[si]); si += 1
+    torch.cuda.synchronize()
+    if qsa.qsa_check_device_error(ws) != 0:
+        raise RuntimeError("device error during warm-up")
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    L_first = pos[0]
+    with ClockSampler(torch.cuda.current_device()) as clk, qsa.trace(capacity=16 * steps + 16) as tr:
+        ev0.record(stream)
+        for _ in range(steps):
+            step(step_in[si]); si += 1
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_max = max_over_ranks(ev0.elapsed_time(ev1), world)
+    if qsa.qsa_check_device_error(ws) != 0:
+        raise RuntimeError("device error during the timed steps")
+    kern = tr.by_kernel()
+    # algorithmic bytes per step: every cached indexer key (256 B each) read once,
+    # the gathered K and V rows of the selected blocks, the appended token and the
+    # inputs / outputs
+    keys = B * (L_first + steps / 2 + 1)
+    gathered = B * min(budget, L_first // 4 + 1) * 4 * 2 * 2 * 256 * 2
+    bytes_step = keys * 256 + gathered + B * (24 * 256 * 2 * 2 + 2 * 2 * 256 * 2 + 128 * 2 * 2)
+    res = dict(ms=ms_max, tokens=B * steps * world, kern=kern, launches=sum(c for c, _ in kern.values()),
+               clocks=clk.summary(), bytes_step=bytes_step, bytes_indexer=keys * 256, steps=steps)
+    if want_e2e:
+        hosts = [{k: torch.empty(step_in[0][k].shape, dtype=step_in[0][k].dtype, pin_memory=True) for k in names}
+                 for _ in range(2)]
+        for h in hosts:
+            for k in names:
+                h[k].copy_(step_in[0][k])
+        out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        bi = sum(hosts[0][k].numel() * hosts[0][k].element_size() for k in names)
+        bo = out_h.numel() * out_h.element_size()
+        e_steps = max(1, min(steps, 3))
+        xdev = {k: torch.empty_like(step_in[0][k]) for k in names}
+
+        def e2e_step(i):
+            for k in names:
+                xdev[k].copy_(hosts[i % 2][k], non_blocking=True)
+            step(xdev)
+            out_h.copy_(out, non_blocking=True)
+
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(e_steps):
+            e2e_step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        ems = max_over_ranks(e0.elapsed_time(e1), world)
+        res["e2e"] = dict(value=B * e_steps * world / (ems / 1e3), unit="tokens/s", h2d_bytes_per_step=bi,
+                          d2h_bytes_per_step=bo, steps=e_steps)
+    del kc, vc, ic, ws, step_in
+    torch.cuda.empty_cache()
+    return res
+
+
+# ------------------------------------------------------------ CPU baselines
+def cpu_prefill_sample(T: int, budget: int, n_blocks: int, seed: int = 0, time_cap_s: float = 25.0):
+    """The oracle on a stratified sample of query blocks of the T-token
+    prefill (evenly spaced qb), all host cores.  Returns tokens/s of the
+    oracle extrapolated by the sample's share of the work, and a description."""
+    import oracle
+    O = oracle.Oracle(oracle.params(budget=budget))
+    P = Q.PrefillProblem(T=T, seed=seed, n_plant=8, dist="zipf" if T >= 131072 else "uniform")
+    nqb = P.nqb
+    qbs = np.unique(np.linspace(0, nqb - 1, n_blocks).astype(np.int64))
+    t_hi = int(qbs.max()) * 4 + 4
+    k_idx = P.k_idx(0, min(t_hi, T))
+    q_idx = np.zeros((T, 4, 128), np.uint16)
+    w = np.zeros((T, 4), np.uint16)
+    for qb in qbs:
+        t0, t1 = qb * 4, min(qb * 4 + 4, T)
+        q_idx[t0:t1] = P.q_idx(t0, t1)
+        w[t0:t1] = P.w(t0, t1)
+    kfull = np.zeros((T, 128), np.uint16)
+    kfull[:k_idx.shape[0]] = k_idx
+    # scores + selection (timed)
+    t_a = time.time()
+    sel, cnt = O.select_blocks_list(T, q_idx, w, kfull, qbs)
+    t_score = time.time() - t_a
+    # attention inputs for the selected blocks (untimed)
+    q = np.zeros((T, 24, 256), np.uint16)
+    k = np.zeros((T, 2, 256), np.uint16)
+    v = np.zeros((T, 2, 256), np.uint16)
+    for i, qb in enumerate(qbs):
+        t0, t1 = qb * 4, min(qb * 4 + 4, T)
+        q[t0:t1] = P.q(t0, t1)
+        for b in sel[i][:cnt[i]]:
+            a0, a1 = b * 4, min(b * 4 + 4, T)
+            k[a0:a1] = P.k(a0, a1)
+            v[a0:a1] = P.v(a0, a1)
+    t_b = time.time()
+    O.attend_blocks(T, q, k, v, qbs, sel, cnt)
+    t_attn = time.time() - t_b
+    elapsed = t_score + t_attn
+    # the sample is evenly spaced in qb, so its mean work matches the workload's
+    tokens = 4 * len(qbs)
+    return tokens / elapsed, dict(sample=f"{len(qbs)} evenly spaced query blocks of the {T}-token prefill "
+                                         f"(scores + selection + attention), {elapsed:.1f} s",
+                                  elapsed=elapsed)
+
+
+def cpu_decode_sample(B: int, L: int, budget: int, n_seq: int, seed: int = 0):
+    import oracle
+    O = oracle.Oracle(oracle.params(budget=budget))
+    D = Q.DecodeProblem(B=B, L=L, steps=1, seed=seed, n_plant=8)
+    elapsed = 0.0
+    for b in range(n_seq):
+        P = D.tokens(b)
+        kid = D.cache_kidx(b)
+        x = {k: getattr(P, k)(L, L + 1)[0] for k in ("q", "k", "v", "q_idx", "w")}
+        kidx_new = P.k_idx(L, L + 1)[0]
+        # selection first (timed) to know which cache rows attention needs
+        t0 = time.time()
+        S = O.block_scores(L // 4, x["q_idx"][None], x["w"][None],
+                           np.concatenate([kid, kidx_new[None]]))
+        sel, cnt = O.select(L // 4, S)
+        t_sel = time.time() - t0
+        kc = np.zeros((L, 2, 256), np.uint16)
+        vc = np.zeros((L, 2, 256), np.uint16)
+        for blk in sel[:cnt]:
+            a0, a1 = blk * 4, min(blk * 4 + 4, L)
+            if a1 > a0:
+                kc[a0:a1] = D.cache_k(b, a0, a1)
+                vc[a0:a1] = D.cache_v(b, a0, a1)
+        t1 = time.time()
+        O.decode(L, kc, vc, kid, np.zeros((0, 4, 128), np.uint16), np.zeros((0, 4), np.uint16), x["q"], x["k"],
+                 x["v"], x["q_idx"], kidx_new, x["w"])
+        elapsed += t_sel + (time.time() - t1)
+    return n_seq / elapsed, dict(sample=f"{n_seq} of {B} sequences, one decode token each at {L} cached tokens "
+                                        f"(scores + selection + attention), {elapsed:.1f} s", elapsed=elapsed)
+
+
+def cores_used():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count()
+
+
+# ------------------------------------------------------------------- main
+WORKLOADS = {
+    "prefill_1m": dict(kind="prefill", T=1 << 20),
+    "prefill_128k": dict(kind="prefill", T=131072),
+    "prefill_32k": dict(kind="prefill", T=32768),
+    "decode_64x256k": dict(kind="decode", B=64, L=262144),
+}
+
+
+def line_for(name, res, n_gpus, steps, warmup, pk):
+    wl = WORKLOADS[name]
+    if wl["kind"] == "prefill":
+        T = wl["T"]
+        value = res["tokens"] / (res["ms"] / 1e3)
+        idx_n, idx_ms = res["kern"].get("indexer", (1, float("nan")))
+        # achieved = algorithmic indexer FLOPs per launch / mean launch time
+        achieved = res["flops_idx"] * res["steps"] / idx_n / (idx_ms / idx_n / 1e3) / 1e12
+        roof = dict(kernel="indexer", bound="tensor", achieved=achieved, peak=pk["bf16_sus"], unit="TFLOP/s",
+                    frac=achieved / pk["bf16_sus"], traffic=None,
+                    peak_src=f"{pk['src']} bf16 dense sustained")
+        total_fl = res["flops_idx"] + res["flops_attn"]
+        whole = dict(tflops=total_fl / (res["ms"] / res["steps"] / 1e3) / 1e12)
+        whole["frac_of_tensor_roofline"] = whole["tflops"] / pk["bf16_sus"]
+        metric = f"QSA prefill tokens/s at {T // 1024}K context"
+        cfg = dict(workload=name, T=T, batch=1, budget_blocks=512, heads="24q/2kv x 256, idx 4 x 128",
+                   planted="8/query block, " + ("zipf(1.1) distance" if T >= 131072 else "uniform"),
+                   l2="inputs larger than L2 (126 MB): no flush needed")
+    else:
+        B, L = wl["B"], wl["L"]
+        value = res["tokens"] / (res["ms"] / 1e3)
+        n, t = res["kern"].get("decode_indexer", (1, float("nan")))
+        achieved = res["bytes_indexer"] / (t / n / 1e3) / 1e9
+        roof = dict(kernel="decode_indexer", bound="hbm", achieved=achieved, peak=pk["hbm"], unit="GB/s",
+                    frac=achieved / pk["hbm"], traffic=None, peak_src=f"{pk['src']} HBM copy")
+        whole = dict(gbs=res["bytes_step"] / (res["ms"] / res["steps"] / 1e3) / 1e9)
+        whole["frac_of_hbm_roofline"] = whole["gbs"] / pk["hbm"]
+        metric = "QSA decode tokens/s at 256K context, batch 64"
+        cfg = dict(workload=name, batch=B, context=L, budget_blocks=512, planted="8 per sequence",
+                   l2="4.3 GB of indexer keys streamed per step (larger than L2)")
+    return dict(metric=metric, value=value, unit="tokens/s", n_gpus=n_gpus, steps=steps, warmup=warmup,
+                ms_per_step=res["ms"] / steps, higher_is_better=True, scaling="weak", vs_baseline=None,
+                dtype="bf16", data="synthetic", config=cfg, roofline=roof, step_roofline=whole,
+                clocks=res["clocks"], gpu_launches=res["launches"], e2e=res.get("e2e"),
+                kernels_ms={k: dict(launches=c, total_ms=round(tt, 3)) for k, (c, tt) in res["kern"].items()})
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="prefill_1m", choices=list(WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        wl = WORKLOADS[args.workload]
+        ts, descs = [], []
+        for _ in range(args.warmup):
+            pass
+        for _ in range(args.steps):
+            if wl["kind"] == "prefill":
+                v, info = cpu_prefill_sample(wl["T"], 512, n_blocks=max(4, min(cores_used(), 16)))
+            else:
+                v, info = cpu_decode_sample(wl["B"], wl["L"], 512, n_seq=2)
+            ts.append(v)
+            descs.append(info["sample"])
+        value = statistics.median(ts)
+        cb = dict(value=value, unit="tokens/s", cores=cores_used(), kind="oracle", sample=descs[0])
+        metric = (f"QSA prefill tokens/s at {wl['T'] // 1024}K context" if wl["kind"] == "prefill"
+                  else "QSA decode tokens/s at 256K context, batch 64")
+        print(json.dumps(dict(impl="reference", metric=metric, value=value, unit="tokens/s", n_gpus=args.gpus,
+                              steps=args.steps, warmup=args.warmup, ms_per_step=None, higher_is_better=True,
+                              scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
+                              config=dict(workload=args.workload), cpu_baseline=cb,
+                              e2e=dict(value=value, unit="tokens/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))),
+              flush=True)
+        return
+
+    rank, world, local = dist_setup(args.gpus)
+    import block_sparse_long_qsa_b200 as qsa
+    qsa.load()
+    pk = peaks()
+    wl = WORKLOADS[args.workload]
+    if wl["kind"] == "prefill":
+        res = run_prefill(wl["T"], 512, args.steps, args.warmup, rank, world, seed=0)
+    else:
+        res = run_decode(wl["B"], wl["L"], 512, args.steps, args.warmup, rank, world, seed=0)
+    line = line_for(args.workload, res, world, args.steps, args.warmup, pk)
+
+    if not args.no_secondary:
+        sec = {}
+        for name in ("decode_64x256k", "prefill_128k"):
+            if name == args.workload:
+                continue
+            w2 = WORKLOADS[name]
+            if w2["kind"] == "prefill":
+                r2 = run_prefill(w2["T"], 512, args.steps, args.warmup, rank, world, seed=0, want_e2e=False)
+            else:
+                r2 = run_decode(w2["B"], w2["L"], 512, max(args.steps, 8), args.warmup, rank, world, seed=0,
+                                want_e2e=False)
+            l2 = line_for(name, r2, world, args.steps, args.warmup, pk)
+            sec[name] = {k: l2[k] for k in ("metric", "value", "unit", "ms_per_step", "roofline", "step_roofline",
+                                            "gpu_launches", "kernels_ms")}
+        line["secondary"] = sec
+
+    if rank == 0 and world == 1 and not args.no_cpu:
+        if wl["kind"] == "prefill":
+            v, info = cpu_prefill_sample(wl["T"], 512, n_blocks=max(4, min(cores_used(), 16)))
+        else:
+            v, info = cpu_decode_sample(wl["B"], wl["L"], 512, n_seq=2)
+        line["cpu_baseline"] = dict(value=v, unit="tokens/s", cores=cores_used(), kind="oracle",
+                                    sample=info["sample"])
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

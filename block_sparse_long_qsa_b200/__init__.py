@@ -22,15 +22,18 @@ _STATUS = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_UNSUPPORTED", 3: "
            4: "QSA_ERR_WORKSPACE_TOO_SMALL", 5: "QSA_ERR_CUDA", 6: "QSA_ERR_DEVICE_TIMEOUT",
            7: "QSA_ERR_DEVICE_BOUNDS", 8: "QSA_ERR_ARCH"}
 
-EXPORTED = ["qsa_default_params", "qsa_status_string", "qsa_index_scores", "qsa_select_blocks",
+EXPORTED = ["qsa_default_params", "qsa_status_string", "qsa_last_error", "qsa_index_scores", "qsa_select_blocks",
             "qsa_select_workspace_size", "qsa_prefill", "qsa_prefill_workspace_size", "qsa_decode",
-            "qsa_decode_workspace_size", "qsa_check_device_error"]
+            "qsa_decode_workspace_size", "qsa_check_device_error", "qsa_trace_begin", "qsa_trace_end"]
+
+KERNEL_NAMES = {1: "rope_table", 2: "rope_k", 3: "indexer", 4: "select", 5: "attention", 6: "decode_append",
+                7: "decode_indexer", 8: "decode_attention", 9: "decode_combine"}
 
 
 class QSAError(RuntimeError):
-    def __init__(self, status: int, where: str):
+    def __init__(self, status: int, where: str, detail: str = ""):
         self.status = status
-        super().__init__(f"{where}: {_STATUS.get(status, status)}")
+        super().__init__(f"{where}: {_STATUS.get(status, status)}" + (f" ({detail})" if detail else ""))
 
 
 class qsa_params(ctypes.Structure):
@@ -58,6 +61,8 @@ def load(path: str = LIB_PATH):
     L.qsa_default_params.restype = None
     L.qsa_status_string.argtypes = [ctypes.c_int]
     L.qsa_status_string.restype = ctypes.c_char_p
+    L.qsa_last_error.argtypes = []
+    L.qsa_last_error.restype = ctypes.c_char_p
     L.qsa_index_scores.argtypes = [P, i64, vp, vp, vp, i64, i64, vp, i64, vp, sz, vp]
     L.qsa_select_blocks.argtypes = [P, vp, i64, i64, i64, vp, vp, vp, sz, vp]
     L.qsa_select_workspace_size.argtypes = [P, psz]
@@ -67,8 +72,10 @@ def load(path: str = LIB_PATH):
                              vp, vp, vp, vp, sz, vp]
     L.qsa_decode_workspace_size.argtypes = [P, i32, i64, psz]
     L.qsa_check_device_error.argtypes = [vp, vp]
+    L.qsa_trace_begin.argtypes = [i32]
+    L.qsa_trace_end.argtypes = [vp, vp, i32, ctypes.POINTER(ctypes.c_int32)]
     for f in EXPORTED:
-        if f not in ("qsa_default_params", "qsa_status_string"):
+        if f not in ("qsa_default_params", "qsa_status_string", "qsa_last_error"):
             getattr(L, f).restype = ctypes.c_int
     _lib = L
     return L
@@ -98,7 +105,8 @@ def _stream(stream=None):
 
 def _check(rc: int, where: str):
     if rc != QSA_OK:
-        raise QSAError(rc, where)
+        detail = load().qsa_last_error().decode(errors="replace") if rc in (5, 8) else ""
+        raise QSAError(rc, where, detail)
 
 
 # ------------------------------------------------------------ raw entry points
@@ -157,6 +165,35 @@ def qsa_decode(p: qsa_params, B: int, max_len: int, cache_len, k_cache, v_cache,
 
 def qsa_check_device_error(ws, stream=None) -> int:
     return load().qsa_check_device_error(_ptr(ws), _stream(stream))
+
+
+class trace:
+    """Context manager: per-launch device times of this library's kernels,
+    from CUDA events recorded on each launching stream.  ``.records`` is a
+    list of (kernel name, milliseconds) in launch order."""
+
+    def __init__(self, capacity: int = 4096):
+        self.capacity = capacity
+        self.records = []
+
+    def __enter__(self):
+        _check(load().qsa_trace_begin(self.capacity), "qsa_trace_begin")
+        return self
+
+    def __exit__(self, *exc):
+        ids = (ctypes.c_int32 * self.capacity)()
+        ms = (ctypes.c_float * self.capacity)()
+        n = ctypes.c_int32()
+        _check(load().qsa_trace_end(ids, ms, self.capacity, ctypes.byref(n)), "qsa_trace_end")
+        self.records = [(KERNEL_NAMES.get(ids[i], str(ids[i])), ms[i]) for i in range(n.value)]
+        return False
+
+    def by_kernel(self) -> dict:
+        out = {}
+        for name, t in self.records:
+            c, tot = out.get(name, (0, 0.0))
+            out[name] = (c + 1, tot + t)
+        return out
 
 
 # ----------------------------------------------------- allocating conveniences

@@ -17,6 +17,14 @@ constexpr size_t ALIGN = 256;
 constexpr int DECODE_SPLIT = 16;
 constexpr int MAX_DEV = 64;
 
+// Last failure of this thread, for qsa_last_error().
+thread_local char g_last_error[256] = "";
+
+qsa_status fail(qsa_status st, const char* what, const char* detail = "") {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s%s%s", what, detail[0] ? ": " : "", detail);
+  return st;
+}
+
 size_t align_up(size_t x, size_t a = ALIGN) { return (x + a - 1) / a * a; }
 int64_t round4(int64_t x) { return (x + 3) / 4 * 4; }
 
@@ -53,8 +61,8 @@ std::mutex g_dev_mu;
 
 qsa_status device_info(DevInfo* out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return QSA_ERR_CUDA;
-  if (dev < 0 || dev >= MAX_DEV) return QSA_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaGetDevice");
+  if (dev < 0 || dev >= MAX_DEV) return fail(QSA_ERR_CUDA, "device ordinal out of range");
   std::lock_guard<std::mutex> lk(g_dev_mu);
   DevInfo& d = g_dev[dev];
   if (!d.known) {
@@ -62,13 +70,13 @@ qsa_status device_info(DevInfo* out) {
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return QSA_ERR_CUDA;
+      return fail(QSA_ERR_CUDA, "cudaDeviceGetAttribute");
     d.sm100 = (major == 10 && minor == 0);
     d.num_sms = sms;
     d.known = true;
   }
   *out = d;
-  return d.sm100 ? QSA_OK : QSA_ERR_ARCH;
+  return d.sm100 ? QSA_OK : fail(QSA_ERR_ARCH, "device is not sm_100");
 }
 
 // ---------------------------------------------------------------- tensor maps
@@ -90,42 +98,70 @@ EncodeTiledFn encode_fn() {
 }
 
 // 2D bf16 tensor [rows][cols] (row-major), box [box_rows][box_cols], 128B swizzle.
-bool make_map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
-                 uint32_t box_cols) {
+qsa_status make_map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                       uint32_t box_cols) {
   EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
+  if (!fn) return fail(QSA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found");
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-// 1D bf16 array of n elements, box of `box` elements.
-bool make_map_1d(CUtensorMap* m, const void* base, uint64_t n, uint32_t box) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[1] = {n};
-  cuuint32_t boxd[1] = {box};
-  cuuint32_t estr[1] = {1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 1, const_cast<void*>(base), dims, nullptr, boxd, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char d[64];
+    std::snprintf(d, sizeof(d), "CUresult %d", (int)r);
+    return fail(QSA_ERR_CUDA, "cuTensorMapEncodeTiled", d);
+  }
+  return QSA_OK;
 }
 
-qsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA; }
+// ----------------------------------------------------------------- tracing
+// When enabled, every kernel launch of the library is bracketed by two CUDA
+// events recorded on the launching stream.
+struct TraceState {
+  std::mutex mu;
+  bool on = false;
+  int cap = 0, n = 0;
+  std::vector<cudaEvent_t> ev;
+  std::vector<int32_t> ids;
+};
+TraceState g_trace;
+
+template <class F>
+cudaError_t traced(int32_t id, cudaStream_t s, F&& f) {
+  int slot = -1;
+  {
+    std::lock_guard<std::mutex> lk(g_trace.mu);
+    if (g_trace.on && g_trace.n < g_trace.cap) slot = g_trace.n++;
+  }
+  if (slot >= 0) cudaEventRecord(g_trace.ev[2 * slot], s);
+  cudaError_t e = f();
+  if (slot >= 0) {
+    cudaEventRecord(g_trace.ev[2 * slot + 1], s);
+    g_trace.ids[slot] = id;
+  }
+  return e;
+}
+
+qsa_status from_cuda(cudaError_t e, const char* where = "kernel launch") {
+  if (e == cudaSuccess) return QSA_OK;
+  return fail(QSA_ERR_CUDA, where, cudaGetErrorString(e));
+}
 
 // Indexer launch for query blocks [qb0, qb1) into S (ld), maps built here.
 qsa_status run_indexer(int64_t T, const uint16_t* q_idx, const uint16_t* w, const uint16_t* k_idx, int64_t qb0,
                        int64_t qb1, float* S, int64_t ld, uint32_t* err, int num_sms, cudaStream_t st) {
   if (qb1 <= qb0) return QSA_OK;
-  CUtensorMap tq, tk, tw;
-  if (!make_map_2d(&tq, q_idx, (uint64_t)T * 4, 128, 256, 64) || !make_map_2d(&tk, k_idx, (uint64_t)T, 128, 128, 64) ||
-      !make_map_1d(&tw, w, (uint64_t)T * 4, 256))
-    return QSA_ERR_CUDA;
+  CUtensorMap tq, tk;
+  qsa_status rs;
+  if ((rs = make_map_2d(&tq, q_idx, (uint64_t)T * 4, 128, 256, 64)) != QSA_OK) return rs;
+  if ((rs = make_map_2d(&tk, k_idx, (uint64_t)T, 128, 128, 64)) != QSA_OK) return rs;
   const float scale = 1.0f / std::sqrt(128.0f);
-  return from_cuda(qsa::launch_indexer_prefill(tq, tk, tw, S, ld, T, qb0, qb1, scale, err, num_sms, st));
+  return from_cuda(traced(QSA_KERNEL_INDEXER, st, [&] {
+    return qsa::launch_indexer_prefill(tq, tk, w, S, ld, T, qb0, qb1, scale, err, num_sms, st);
+  }), "indexer launch");
 }
 
 // ------------------------------------------------------------ prefill layout
@@ -175,6 +211,8 @@ void qsa_default_params(qsa_params* p) {
   p->softmax_scale = 0.f;
 }
 
+const char* qsa_last_error(void) { return g_last_error; }
+
 const char* qsa_status_string(qsa_status s) {
   switch (s) {
     case QSA_OK: return "ok";
@@ -206,7 +244,7 @@ qsa_status qsa_index_scores(const qsa_params* p, int64_t T, const uint16_t* q_id
   if ((st = device_info(&di)) != QSA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t* err = static_cast<uint32_t*>(ws);
-  if (err && cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return QSA_ERR_CUDA;
+  if (err && cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaMemsetAsync");
   return run_indexer(T, q_idx, w, k_idx, qb_begin, qb_end, scores, ld, err, di.num_sms, s);
 }
 
@@ -230,9 +268,10 @@ qsa_status qsa_select_blocks(const qsa_params* p, const float* scores, int64_t l
   if ((st = device_info(&di)) != QSA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t* err = static_cast<uint32_t*>(ws);
-  if (cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return QSA_ERR_CUDA;
-  return from_cuda(qsa::launch_select(scores, ld, qb_begin, qb_end - qb_begin, nullptr, p->budget_blocks, sel, cnt,
-                                      err, s));
+  if (cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaMemsetAsync");
+  return from_cuda(traced(QSA_KERNEL_SELECT, s, [&] {
+    return qsa::launch_select(scores, ld, qb_begin, qb_end - qb_begin, nullptr, p->budget_blocks, sel, cnt, err, s);
+  }));
 }
 
 qsa_status qsa_prefill_workspace_size(const qsa_params* p, int64_t T, size_t* min_bytes, size_t* pref_bytes) {
@@ -286,22 +325,28 @@ qsa_status qsa_prefill(const qsa_params* p, int64_t T, int64_t pos0, const uint1
   int32_t* cnt = cnt_out ? cnt_out : reinterpret_cast<int32_t*>(base + L.cnt);
   float* slab = reinterpret_cast<float*>(base + L.slab);
 
-  if (cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return QSA_ERR_CUDA;
+  if (cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaMemsetAsync");
   double f[32];
   inv_freq(p, f);
-  if ((st = from_cuda(qsa::launch_rope_table(T, pos0, f, cs, s))) != QSA_OK) return st;
-  if ((st = from_cuda(qsa::launch_rope_k(T, k, cs, k_rot, s))) != QSA_OK) return st;
+  if ((st = from_cuda(traced(QSA_KERNEL_ROPE_TABLE, s, [&] { return qsa::launch_rope_table(T, pos0, f, cs, s); }))) !=
+      QSA_OK)
+    return st;
+  if ((st = from_cuda(traced(QSA_KERNEL_ROPE_K, s, [&] { return qsa::launch_rope_k(T, k, cs, k_rot, s); }))) != QSA_OK)
+    return st;
   const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
   for (int64_t qb0 = 0; qb0 < nqb;) {
     const int64_t qb1 = chunk_end(qb0, nqb, slab_bytes);
     if (qb1 <= qb0) return QSA_ERR_WORKSPACE_TOO_SMALL;
     const int64_t ld = round4(qb1);
     if ((st = run_indexer(T, q_idx, w, k_idx, qb0, qb1, slab, ld, err, di.num_sms, s)) != QSA_OK) return st;
-    if ((st = from_cuda(qsa::launch_select(slab, ld, qb0, qb1 - qb0, nullptr, budget, sel + qb0 * budget, cnt + qb0,
-                                           err, s))) != QSA_OK)
+    if ((st = from_cuda(traced(QSA_KERNEL_SELECT, s, [&] {
+           return qsa::launch_select(slab, ld, qb0, qb1 - qb0, nullptr, budget, sel + qb0 * budget, cnt + qb0, err, s);
+         }))) != QSA_OK)
       return st;
-    if ((st = from_cuda(qsa::launch_sparse_attn_prefill(T, q, k_rot, v, cs, sel + qb0 * budget, cnt + qb0, budget,
-                                                        qb0, qb1, scale_log2, out, lse, s))) != QSA_OK)
+    if ((st = from_cuda(traced(QSA_KERNEL_ATTENTION, s, [&] {
+           return qsa::launch_sparse_attn_prefill(T, q, k_rot, v, cs, sel + qb0 * budget, cnt + qb0, budget, qb0, qb1,
+                                                  scale_log2, out, lse, s);
+         }))) != QSA_OK)
       return st;
     qb0 = qb1;
   }
@@ -379,25 +424,34 @@ qsa_status qsa_decode(const qsa_params* p, int32_t B, int64_t max_len, const int
   float* part_o = reinterpret_cast<float*>(base + L.part_o);
   float* part_lse = reinterpret_cast<float*>(base + L.part_lse);
 
-  if (cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return QSA_ERR_CUDA;
+  if (cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaMemsetAsync");
   double f[32];
   inv_freq(p, f);
   // the append kernel receives the lengths as launch parameters and stores
   // them (and L/4) in the workspace for the later kernels
-  if ((st = from_cuda(qsa::launch_decode_append(B, max_len, cache_len, Ls, qbs, f, k_cache, v_cache, kidx_cache,
-                                                qidx_ring, w_ring, q_new, k_new, v_new, q_idx_new, k_idx_new, w_new,
-                                                q_rot, s))) != QSA_OK)
+  if ((st = from_cuda(traced(QSA_KERNEL_DECODE_APPEND, s, [&] {
+         return qsa::launch_decode_append(B, max_len, cache_len, Ls, qbs, f, k_cache, v_cache, kidx_cache, qidx_ring,
+                                          w_ring, q_new, k_new, v_new, q_idx_new, k_idx_new, w_new, q_rot, s);
+       }))) != QSA_OK)
     return st;
   const float scale = 1.0f / std::sqrt(128.0f);
-  if ((st = from_cuda(qsa::launch_decode_indexer(B, max_len, max_L, Ls, kidx_cache, qidx_ring, w_ring, S, L.ld, scale,
-                                                 s))) != QSA_OK)
+  if ((st = from_cuda(traced(QSA_KERNEL_DECODE_INDEXER, s, [&] {
+         return qsa::launch_decode_indexer(B, max_len, max_L, Ls, kidx_cache, qidx_ring, w_ring, S, L.ld, scale, s);
+       }))) != QSA_OK)
     return st;
-  if ((st = from_cuda(qsa::launch_select(S, L.ld, 0, B, qbs, budget, sel, cnt, err, s))) != QSA_OK) return st;
+  if ((st = from_cuda(traced(QSA_KERNEL_SELECT, s, [&] {
+         return qsa::launch_select(S, L.ld, 0, B, qbs, budget, sel, cnt, err, s);
+       }))) != QSA_OK)
+    return st;
   const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
-  if ((st = from_cuda(qsa::launch_decode_attn(B, max_len, Ls, q_rot, k_cache, v_cache, sel, cnt, budget, DECODE_SPLIT,
-                                              scale_log2, part_o, part_lse, s))) != QSA_OK)
+  if ((st = from_cuda(traced(QSA_KERNEL_DECODE_ATTENTION, s, [&] {
+         return qsa::launch_decode_attn(B, max_len, Ls, q_rot, k_cache, v_cache, sel, cnt, budget, DECODE_SPLIT,
+                                        scale_log2, part_o, part_lse, s);
+       }))) != QSA_OK)
     return st;
-  return from_cuda(qsa::launch_decode_combine(B, DECODE_SPLIT, part_o, part_lse, out, lse_out, s));
+  return from_cuda(traced(QSA_KERNEL_DECODE_COMBINE, s, [&] {
+    return qsa::launch_decode_combine(B, DECODE_SPLIT, part_o, part_lse, out, lse_out, s);
+  }));
 }
 
 qsa_status qsa_check_device_error(void* ws, void* stream) {
@@ -409,6 +463,45 @@ qsa_status qsa_check_device_error(void* ws, void* stream) {
   if (h != 0 && cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) return QSA_ERR_CUDA;
   if (h == 0) return QSA_OK;
   return (h == QSA_ERR_DEVICE_TIMEOUT || h == QSA_ERR_DEVICE_BOUNDS) ? static_cast<qsa_status>(h) : QSA_ERR_CUDA;
+}
+
+qsa_status qsa_trace_begin(int32_t capacity) {
+  if (capacity <= 0 || capacity > (1 << 20)) return QSA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_trace.mu);
+  if (g_trace.on) return QSA_ERR_INVALID_ARG;
+  g_trace.ev.assign((size_t)2 * capacity, nullptr);
+  for (auto& e : g_trace.ev)
+    if (cudaEventCreate(&e) != cudaSuccess) return QSA_ERR_CUDA;
+  g_trace.ids.assign((size_t)capacity, 0);
+  g_trace.cap = capacity;
+  g_trace.n = 0;
+  g_trace.on = true;
+  return QSA_OK;
+}
+
+qsa_status qsa_trace_end(int32_t* kernel_ids, float* ms, int32_t capacity, int32_t* n_out) {
+  std::lock_guard<std::mutex> lk(g_trace.mu);
+  if (!g_trace.on) return QSA_ERR_INVALID_ARG;
+  qsa_status st = QSA_OK;
+  const int n = g_trace.n;
+  if (n > 0 && cudaEventSynchronize(g_trace.ev[2 * n - 1]) != cudaSuccess) st = QSA_ERR_CUDA;
+  int written = 0;
+  for (int i = 0; i < n && st == QSA_OK; ++i) {
+    if (i >= capacity || !kernel_ids || !ms) break;
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, g_trace.ev[2 * i], g_trace.ev[2 * i + 1]) != cudaSuccess) { st = QSA_ERR_CUDA; break; }
+    kernel_ids[i] = g_trace.ids[i];
+    ms[i] = t;
+    ++written;
+  }
+  for (auto e : g_trace.ev)
+    if (e) cudaEventDestroy(e);
+  g_trace.ev.clear();
+  g_trace.ids.clear();
+  g_trace.on = false;
+  g_trace.n = g_trace.cap = 0;
+  if (n_out) *n_out = written;
+  return st;
 }
 
 }  // extern "C"

@@ -20,7 +20,7 @@
 //   * Work unit = (query tile, key tile).  The causal triangle's units are
 //     split evenly across CTAs in query-major order, so every CTA gets the
 //     same number of MMAs whatever the chunk shape.
-//   * warp 0: TMA producer (3-stage key ring, Q + w tile); warp 1: TMEM
+//   * warp 0: producer (3-stage TMA key ring, TMA Q tile, head weights); warp 1: TMEM
 //     allocation and the single MMA-issuing thread; warps 2-9: epilogue
 //     (tcgen05.ld -> ReLU, head weights, block max -> fp32 scores).
 //   * Every mbarrier wait is bounded; on timeout the CTA records
@@ -39,7 +39,7 @@ constexpr uint32_t Q_SUB_BYTES = 256 * 128;              // 256 rows x 64 bf16
 constexpr uint32_t Q_BYTES = 4 * Q_SUB_BYTES;            // [half][k-chunk]
 constexpr uint32_t K_SUB_BYTES = 128 * 128;              // 128 rows x 64 bf16
 constexpr uint32_t K_STAGE_BYTES = 2 * K_SUB_BYTES;
-constexpr uint32_t W_BYTES = QT * 4 * 2;                 // bf16 [128][4]
+constexpr uint32_t W_BYTES = QT * 4 * 4;                 // fp32 [128][4]
 constexpr uint32_t OFF_K = Q_BYTES;
 constexpr uint32_t OFF_W = OFF_K + STAGES * K_STAGE_BYTES;
 constexpr uint32_t OFF_BAR = OFF_W + W_BYTES;
@@ -88,12 +88,12 @@ struct Iter {
 
 __global__ void __launch_bounds__(THREADS, 1)
 indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_w, float* __restrict__ S, int64_t ld, int64_t T,
+                       const uint16_t* __restrict__ w, float* __restrict__ S, int64_t ld, int64_t T,
                        int64_t qb_begin, int64_t qb_end, float scale, uint32_t* err) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* sQ = smem;
   uint8_t* sK = smem + OFF_K;
-  const uint16_t* sW = reinterpret_cast<const uint16_t*>(smem + OFF_W);
+  const float* sW = reinterpret_cast<const float*>(smem + OFF_W);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* full = bars;               // [STAGES]
   uint64_t* empty = bars + STAGES;     // [STAGES]
@@ -139,30 +139,53 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_w);
-      Iter it; it.begin(&sch, u0, u1);
-      int stage = 0; uint32_t ephase = 1; uint32_t qcount = 0;
-      for (; it.valid(); it.next()) {
-        if (it.first_of_tile(u0)) {
-          if (qcount > 0 && !mbar_wait(qempty, (qcount - 1) & 1, abort_flag, err)) break;
-          const int32_t t_first = (int32_t)(sch.T0 + QT * it.tile);
-          mbar_arrive_expect_tx(qfull, Q_BYTES + W_BYTES);
+    // The whole warp walks the units: at each new query tile all lanes load
+    // the tile's head weights (bf16 -> fp32 into shared memory) and lane 0
+    // issues the TMA loads; control flow stays warp-uniform so every exit is
+    // taken by all lanes together.
+    if (lane == 0) { tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); }
+    float* sWf = reinterpret_cast<float*>(smem + OFF_W);
+    Iter it; it.begin(&sch, u0, u1);
+    int stage = 0; uint32_t ephase = 1; uint32_t qcount = 0;
+    for (; it.valid(); it.next()) {
+      if (it.first_of_tile(u0)) {
+        bool ok = qcount == 0 || mbar_wait(qempty, (qcount - 1) & 1, abort_flag, err);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        const int64_t t_first = sch.T0 + QT * it.tile;
+        // lane l: tokens t_first + 4l .. +3
+        float wv[16];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t t = t_first + 4 * lane + u;
+          uint2 raw = make_uint2(0u, 0u);
+          if (t < T) raw = __ldg(reinterpret_cast<const uint2*>(w + 4 * t));
+          wv[4 * u + 0] = bf16lo(raw.x); wv[4 * u + 1] = bf16hi(raw.x);
+          wv[4 * u + 2] = bf16lo(raw.y); wv[4 * u + 3] = bf16hi(raw.y);
+        }
+        float4* dst = reinterpret_cast<float4*>(sWf + 16 * lane);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) dst[u] = make_float4(wv[4 * u], wv[4 * u + 1], wv[4 * u + 2], wv[4 * u + 3]);
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(qfull, Q_BYTES);
           for (int hf = 0; hf < 2; ++hf)
             for (int kc = 0; kc < 2; ++kc)
-              tma_load_2d(sQ + (hf * 2 + kc) * Q_SUB_BYTES, &tm_q, kc * 64, 4 * t_first + 256 * hf, qfull);
-          // w as a flat bf16 array of 4*T: two 256-element boxes (x * 2 bytes is a multiple of 16)
-          tma_load_1d(smem + OFF_W, &tm_w, 4 * t_first, qfull);
-          tma_load_1d(smem + OFF_W + W_BYTES / 2, &tm_w, 4 * t_first + 256, qfull);
-          ++qcount;
+              tma_load_2d(sQ + (hf * 2 + kc) * Q_SUB_BYTES, &tm_q, kc * 64, (int32_t)(4 * t_first + 256 * hf), qfull);
         }
-        if (!mbar_wait(&empty[stage], ephase, abort_flag, err)) break;
-        mbar_arrive_expect_tx(&full[stage], K_STAGE_BYTES);
-        for (int kc = 0; kc < 2; ++kc)
-          tma_load_2d(sK + stage * K_STAGE_BYTES + kc * K_SUB_BYTES, &tm_k, kc * 64, (int32_t)(KT * it.kt),
-                      &full[stage]);
-        if (++stage == STAGES) { stage = 0; ephase ^= 1; }
+        ++qcount;
       }
+      bool ok = true;
+      if (lane == 0) {
+        ok = mbar_wait(&empty[stage], ephase, abort_flag, err);
+        if (ok) {
+          mbar_arrive_expect_tx(&full[stage], K_STAGE_BYTES);
+          for (int kc = 0; kc < 2; ++kc)
+            tma_load_2d(sK + stage * K_STAGE_BYTES + kc * K_SUB_BYTES, &tm_k, kc * 64, (int32_t)(KT * it.kt),
+                        &full[stage]);
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+      if (++stage == STAGES) { stage = 0; ephase ^= 1; }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
@@ -242,7 +265,7 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
           __syncwarp();
           if (lane == 0) mbar_arrive(&accempty[hf]);
           const bool masked = kt_last_key > t_first;
-          const uint16_t* wrow = sW + (64 * hf + 32 * cgrp) * 4;
+          const float* wrow = sW + (64 * hf + 32 * cgrp) * 4;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
 #pragma unroll
@@ -251,12 +274,12 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
                 const int tl = 8 * c + 4 * half_blk + u;    // token index within the 32 columns
-                const uint2 wv = *reinterpret_cast<const uint2*>(wrow + 4 * tl);
+                const float4 wv = *reinterpret_cast<const float4*>(wrow + 4 * tl);
                 const float* x = &v[c][4 * (4 * half_blk + u)];
-                float s = bf16lo(wv.x) * fmaxf(x[0], 0.f);
-                s = fmaf(bf16hi(wv.x), fmaxf(x[1], 0.f), s);
-                s = fmaf(bf16lo(wv.y), fmaxf(x[2], 0.f), s);
-                s = fmaf(bf16hi(wv.y), fmaxf(x[3], 0.f), s);
+                float s = wv.x * fmaxf(x[0], 0.f);
+                s = fmaf(wv.y, fmaxf(x[1], 0.f), s);
+                s = fmaf(wv.z, fmaxf(x[2], 0.f), s);
+                s = fmaf(wv.w, fmaxf(x[3], 0.f), s);
                 if (masked) s = (j <= t_first + tl) ? s : 0.f;
                 sc[u] = s;
               }
@@ -307,7 +330,7 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 
 }  // namespace
 
-cudaError_t launch_indexer_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_w,
+cudaError_t launch_indexer_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const uint16_t* w,
                                    float* S, int64_t ld, int64_t T, int64_t qb_begin, int64_t qb_end, float scale,
                                    uint32_t* err, int num_sms, cudaStream_t stream) {
   if (qb_end <= qb_begin) return cudaSuccess;
@@ -331,7 +354,7 @@ cudaError_t launch_indexer_prefill(const CUtensorMap& tm_q, const CUtensorMap& t
     units += tl / KT + 1;
   }
   const int grid = (int)(units < num_sms ? units : num_sms);
-  indexer_prefill_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tm_q, tm_k, tm_w, S, ld, T, qb_begin, qb_end, scale,
+  indexer_prefill_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tm_q, tm_k, w, S, ld, T, qb_begin, qb_end, scale,
                                                                  err);
   return cudaGetLastError();
 }

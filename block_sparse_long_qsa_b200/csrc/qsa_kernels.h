@@ -12,7 +12,7 @@ cudaError_t launch_rope_table(int64_t T, int64_t pos0, const double* inv_freq_ho
 // k_rot[t][g] = RoPE(k[t][g]) on dims 0..63, dims 64..255 copied.
 cudaError_t launch_rope_k(int64_t T, const uint16_t* k, const float2* cs, uint16_t* k_rot, cudaStream_t s);
 
-cudaError_t launch_indexer_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_w,
+cudaError_t launch_indexer_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const uint16_t* w,
                                    float* S, int64_t ld, int64_t T, int64_t qb_begin, int64_t qb_end, float scale,
                                    uint32_t* err, int num_sms, cudaStream_t stream);
 

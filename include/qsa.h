@@ -75,6 +75,11 @@ void qsa_default_params(qsa_params* p);
 /* Human-readable name of a status code (static storage). */
 const char* qsa_status_string(qsa_status s);
 
+/* Description of the last failing CUDA step of a call made by this thread
+ * (e.g. the CUDA error string of a rejected launch); "" if none yet.  Valid
+ * until the thread's next failing call. */
+const char* qsa_last_error(void);
+
 /* Stage 1 -- indexer block scores ([PT §QSA], eq. I_ib, with the head
  * weights and causal block-max of this library's reading):
  *   s(t, j)   = sum_h w[t][h] * ReLU(q_idx[t][h] . k_idx[j]) / sqrt(idx_dim)
@@ -152,6 +157,28 @@ qsa_status qsa_decode_workspace_size(const qsa_params* p, int32_t B, int64_t max
  * start of a workspace passed to qsa_select_blocks / qsa_prefill /
  * qsa_decode.  Returns QSA_OK or the first device-side error recorded. */
 qsa_status qsa_check_device_error(void* ws, void* stream);
+
+/* Launch tracing, a measurement aid with no counterpart on the pages.
+ * Between qsa_trace_begin and qsa_trace_end every kernel this library
+ * launches (on any stream, in any call) is bracketed by two CUDA events
+ * recorded on its launching stream, for up to `capacity` launches (later
+ * launches are not traced).  qsa_trace_end waits for the last traced launch,
+ * writes up to `capacity` (kernel id, milliseconds) pairs in launch order,
+ * sets *n_out to the number written and releases the events.  Not
+ * re-entrant: one trace at a time per process.  Kernel ids: */
+enum {
+  QSA_KERNEL_ROPE_TABLE = 1,
+  QSA_KERNEL_ROPE_K = 2,
+  QSA_KERNEL_INDEXER = 3,
+  QSA_KERNEL_SELECT = 4,
+  QSA_KERNEL_ATTENTION = 5,
+  QSA_KERNEL_DECODE_APPEND = 6,
+  QSA_KERNEL_DECODE_INDEXER = 7,
+  QSA_KERNEL_DECODE_ATTENTION = 8,
+  QSA_KERNEL_DECODE_COMBINE = 9
+};
+qsa_status qsa_trace_begin(int32_t capacity);
+qsa_status qsa_trace_end(int32_t* kernel_ids, float* ms, int32_t capacity, int32_t* n_out);
 
 #ifdef __cplusplus
 }

@@ -60,6 +60,7 @@ def _bind(L):
     L.oracle_select_rows.argtypes = [P, vp, i64, i64, i64, vp, vp]
     L.oracle_attend_blocks.argtypes = [P, i64, i64, vp, vp, vp, i64, vp, vp, vp, vp, vp]
     L.oracle_prefill_blocks.argtypes = [P, i64, i64, vp, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp, vp]
+    L.oracle_select_blocks_list.argtypes = [P, i64, vp, vp, vp, i64, vp, vp, vp]
     L.oracle_decode.argtypes = [P, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp]
     return L
 
@@ -157,6 +158,17 @@ class Oracle:
         self.L.oracle_attend_blocks(ctypes.byref(self.P), T, pos0, _p(q), _p(k), _p(v), n, _p(qb_list), _p(sel),
                                     _p(cnt), _p(out), _p(lse))
         return out, lse
+
+    def select_blocks_list(self, T, q_idx, w, k_idx, qb_list):
+        """(sel [n][budget], cnt [n]) of the listed query blocks (scores + selection)."""
+        qb_list = np.ascontiguousarray(qb_list, dtype=np.int64)
+        n = len(qb_list)
+        sel = np.empty((n, self.P.budget), dtype=np.int32)
+        cnt = np.empty(n, dtype=np.int32)
+        q_idx, w, k_idx = _u16(q_idx), _u16(w), _u16(k_idx)
+        self.L.oracle_select_blocks_list(ctypes.byref(self.P), T, _p(q_idx), _p(w), _p(k_idx), n, _p(qb_list),
+                                         _p(sel), _p(cnt))
+        return sel, cnt
 
     def prefill_blocks(self, T, q, k, v, q_idx, w, k_idx, qb_list=None, pos0=0):
         """(sel [n][budget], cnt [n], out [n*r][H][d], lse [n*r][H]) for the listed query blocks."""

@@ -262,12 +262,11 @@ void oracle_attend_blocks(const oracle_params* p, int64_t T, int64_t pos0, const
   }
 }
 
-/* Whole prefill for the listed query blocks: scores, selection, attention.
- * sel_out [n][budget], cnt_out [n]; out / lse as oracle_attend_blocks. */
-void oracle_prefill_blocks(const oracle_params* p, int64_t T, int64_t pos0, const uint16_t* q, const uint16_t* k,
-                           const uint16_t* v, const uint16_t* q_idx, const uint16_t* w, const uint16_t* k_idx,
-                           int64_t n_blocks, const int64_t* qb_list, int32_t* sel_out, int32_t* cnt_out,
-                           double* out, double* lse) {
+/* Block scores and selection for the listed query blocks (stages 1 and 2).
+ * sel_out [n][budget], cnt_out [n]. */
+void oracle_select_blocks_list(const oracle_params* p, int64_t T, const uint16_t* q_idx, const uint16_t* w,
+                               const uint16_t* k_idx, int64_t n_blocks, const int64_t* qb_list, int32_t* sel_out,
+                               int32_t* cnt_out) {
   int r = p->block;
 #pragma omp parallel for schedule(dynamic, 1)
   for (int64_t b = 0; b < n_blocks; ++b) {
@@ -279,6 +278,15 @@ void oracle_prefill_blocks(const oracle_params* p, int64_t T, int64_t pos0, cons
     oracle_select(p, qb, S, sel_out + b * p->budget, cnt_out + b);
     free(S);
   }
+}
+
+/* Whole prefill for the listed query blocks: scores, selection, attention.
+ * sel_out [n][budget], cnt_out [n]; out / lse as oracle_attend_blocks. */
+void oracle_prefill_blocks(const oracle_params* p, int64_t T, int64_t pos0, const uint16_t* q, const uint16_t* k,
+                           const uint16_t* v, const uint16_t* q_idx, const uint16_t* w, const uint16_t* k_idx,
+                           int64_t n_blocks, const int64_t* qb_list, int32_t* sel_out, int32_t* cnt_out,
+                           double* out, double* lse) {
+  oracle_select_blocks_list(p, T, q_idx, w, k_idx, n_blocks, qb_list, sel_out, cnt_out);
   oracle_attend_blocks(p, T, pos0, q, k, v, n_blocks, qb_list, sel_out, cnt_out, out, lse);
 }
 
