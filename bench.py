@@ -315,7 +315,28 @@ def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, 
 
 
 # ------------------------------------------------------------ CPU baselines
-def cpu_prefill_sample(T: int, budget: int, n_blocks: int, seed: int = 0, time_cap_s: float = 25.0):
+_KIDX_CACHE: dict = {}
+
+
+def cpu_sample(wl: dict, target_s: float = 12.0):
+    """The oracle on a bounded sample of the workload sized to ~target_s of
+    CPU time: a calibration run, then one run scaled to the target."""
+    if wl["kind"] == "prefill":
+        n = max(4, cores_used())
+        v, info = cpu_prefill_sample(wl["T"], 512, n)
+        if info["elapsed"] < target_s / 3:
+            n2 = int(min((wl["T"] + 3) // 4, max(n + 1, n * target_s / max(info["elapsed"], 1e-3))))
+            v, info = cpu_prefill_sample(wl["T"], 512, n2)
+    else:
+        n = 2
+        v, info = cpu_decode_sample(wl["B"], wl["L"], 512, n)
+        if info["elapsed"] < target_s / 3:
+            n2 = int(min(wl["B"], max(n + 1, n * target_s / max(info["elapsed"], 1e-3))))
+            v, info = cpu_decode_sample(wl["B"], wl["L"], 512, n2)
+    return v, info
+
+
+def cpu_prefill_sample(T: int, budget: int, n_blocks: int, seed: int = 0):
     """The oracle on a stratified sample of query blocks of the T-token
     prefill (evenly spaced qb), all host cores.  Returns tokens/s of the
     oracle extrapolated by the sample's share of the work, and a description."""
@@ -324,8 +345,11 @@ def cpu_prefill_sample(T: int, budget: int, n_blocks: int, seed: int = 0, time_c
     P = Q.PrefillProblem(T=T, seed=seed, n_plant=8, dist="zipf" if T >= 131072 else "uniform")
     nqb = P.nqb
     qbs = np.unique(np.linspace(0, nqb - 1, n_blocks).astype(np.int64))
-    t_hi = int(qbs.max()) * 4 + 4
-    k_idx = P.k_idx(0, min(t_hi, T))
+    key = (T, seed)
+    if key not in _KIDX_CACHE:
+        _KIDX_CACHE.clear()
+        _KIDX_CACHE[key] = P.k_idx(0, T)
+    k_idx = _KIDX_CACHE[key]
     q_idx = np.zeros((T, 4, 128), np.uint16)
     w = np.zeros((T, 4), np.uint16)
     for qb in qbs:
@@ -453,6 +477,7 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
 
@@ -461,13 +486,8 @@ def main():
             return
         wl = WORKLOADS[args.workload]
         ts, descs = [], []
-        for _ in range(args.warmup):
-            pass
         for _ in range(args.steps):
-            if wl["kind"] == "prefill":
-                v, info = cpu_prefill_sample(wl["T"], 512, n_blocks=max(4, min(cores_used(), 16)))
-            else:
-                v, info = cpu_decode_sample(wl["B"], wl["L"], 512, n_seq=2)
+            v, info = cpu_sample(wl)
             ts.append(v)
             descs.append(info["sample"])
         value = statistics.median(ts)
@@ -488,9 +508,10 @@ def main():
     pk = peaks()
     wl = WORKLOADS[args.workload]
     if wl["kind"] == "prefill":
-        res = run_prefill(wl["T"], 512, args.steps, args.warmup, rank, world, seed=0)
+        res = run_prefill(wl["T"], 512, args.steps, args.warmup, rank, world, seed=0, want_e2e=not args.no_e2e)
     else:
-        res = run_decode(wl["B"], wl["L"], 512, args.steps, args.warmup, rank, world, seed=0)
+        res = run_decode(wl["B"], wl["L"], 512, args.steps, args.warmup, rank, world, seed=0,
+                         want_e2e=not args.no_e2e)
     line = line_for(args.workload, res, world, args.steps, args.warmup, pk)
 
     if not args.no_secondary:
@@ -510,10 +531,7 @@ def main():
         line["secondary"] = sec
 
     if rank == 0 and world == 1 and not args.no_cpu:
-        if wl["kind"] == "prefill":
-            v, info = cpu_prefill_sample(wl["T"], 512, n_blocks=max(4, min(cores_used(), 16)))
-        else:
-            v, info = cpu_decode_sample(wl["B"], wl["L"], 512, n_seq=2)
+        v, info = cpu_sample(wl)
         line["cpu_baseline"] = dict(value=v, unit="tokens/s", cores=cores_used(), kind="oracle",
                                     sample=info["sample"])
     if rank == 0:
