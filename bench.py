@@ -32,6 +32,7 @@ import torch  # noqa: E402
 import qsa_inputs as Q  # noqa: E402
 
 L2_BYTES = 126 * (1 << 20)
+DECODE_CALLS = 32          # decode tokens per sequence in one bench step (the workload's 32 steps)
 
 
 def peaks():
@@ -221,9 +222,11 @@ def run_prefill(T: int, budget: int, steps: int, warmup: int, rank: int, world: 
 def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, world: int, seed: int,
                want_e2e=True):
     import block_sparse_long_qsa_b200 as qsa
-    n_total = warmup + steps + (min(steps, 3) + 1 if want_e2e else 0)
-    D = Q.DecodeProblem(B=B, L=L, steps=n_total, seed=seed + 1000 * rank, n_plant=8)
-    max_len = L + n_total + 4
+    # one bench step = DECODE_CALLS consecutive decode tokens per sequence
+    e_steps = max(1, min(steps, 3)) if want_e2e else 0
+    n_calls = (warmup + steps + e_steps) * DECODE_CALLS
+    D = Q.DecodeProblem(B=B, L=L, steps=n_calls, seed=seed + 1000 * rank, n_plant=8)
+    max_len = L + n_calls + 4
     kc = torch.empty((B, max_len, 2, 256), dtype=torch.uint16, device="cuda")
     vc = torch.empty_like(kc)
     ic = torch.empty((B, max_len, 128), dtype=torch.uint16, device="cuda")
@@ -233,26 +236,35 @@ def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, 
     p = qsa.params(budget)
     ws = qsa.workspace(qsa.qsa_decode_workspace_size(p, B, max_len))
     out = torch.empty((B, 24, 256), dtype=torch.uint16, device="cuda")
-    # per-step inputs, generated once (host) and kept resident
+    # decode-token inputs of every call, generated once per sequence and kept resident: [call][B][...]
     names = ["q", "k", "v", "q_idx", "k_idx", "w"]
-    step_in = []
-    for s in range(n_total):
-        x = D.step_inputs(s)
-        t = L + s
-        x["k_idx"] = np.stack([D.tokens(b).k_idx(t, t + 1)[0] for b in range(B)])
-        step_in.append({k: torch.from_numpy(np.ascontiguousarray(x[k])).cuda() for k in names})
+    per_seq = [D.tokens(b) for b in range(B)]
+    allin = {}
+    for k in names:
+        arr = np.stack([getattr(per_seq[b], k)(L, L + n_calls) for b in range(B)], axis=1)
+        allin[k] = torch.from_numpy(np.ascontiguousarray(arr)).cuda()
+    step_in = [{k: allin[k][s] for k in names} for s in range(n_calls)]
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     pos = [L]
 
-    def step(x):
+    def call(x):
         qsa.qsa_decode(p, B, max_len, [pos[0]] * B, kc, vc, ic, ring, wring, x["q"], x["k"], x["v"], x["q_idx"],
                        x["k_idx"], x["w"], out, ws=ws, stream=stream)
         pos[0] += 1
 
     si = 0
+
+    def step():
+        nonlocal si
+        for _ in range(DECODE_CALLS):
+            call(step_in[si]); si += 1
+
+    # the clock sampler starts before the warm-up so that its start-up does not
+    # overlap the (short) timed region
+    clk = ClockSampler(torch.cuda.current_device()).__enter__()
     for _ in range(warmup):
-        step(step_in[si]); si += 1
+        step()
     torch.cuda.synchronize()
     if qsa.qsa_check_device_error(ws) != 0:
         raise RuntimeError("device error during warm-up")
@@ -260,56 +272,62 @@ def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, 
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     L_first = pos[0]
-    with ClockSampler(torch.cuda.current_device()) as clk, qsa.trace(capacity=16 * steps + 16) as tr:
+    with qsa.trace(capacity=16 * steps * DECODE_CALLS + 16) as tr:
         ev0.record(stream)
         for _ in range(steps):
-            step(step_in[si]); si += 1
+            step()
         ev1.record(stream)
         torch.cuda.synchronize()
+    clk.__exit__(None, None, None)
     barrier(world)
     ms_max = max_over_ranks(ev0.elapsed_time(ev1), world)
     if qsa.qsa_check_device_error(ws) != 0:
         raise RuntimeError("device error during the timed steps")
     kern = tr.by_kernel()
-    # algorithmic bytes per step: every cached indexer key (256 B each) read once,
-    # the gathered K and V rows of the selected blocks, the appended token and the
-    # inputs / outputs
-    keys = B * (L_first + steps / 2 + 1)
+    # algorithmic bytes per decode call: every cached indexer key (256 B) read
+    # once, the gathered K and V rows of the selected blocks, the appended token
+    # and the inputs / outputs
+    n_timed = steps * DECODE_CALLS
+    keys = B * (L_first + n_timed / 2 + 1)
     gathered = B * min(budget, L_first // 4 + 1) * 4 * 2 * 2 * 256 * 2
-    bytes_step = keys * 256 + gathered + B * (24 * 256 * 2 * 2 + 2 * 2 * 256 * 2 + 128 * 2 * 2)
-    res = dict(ms=ms_max, tokens=B * steps * world, kern=kern, launches=sum(c for c, _ in kern.values()),
-               clocks=clk.summary(), bytes_step=bytes_step, bytes_indexer=keys * 256, steps=steps)
+    bytes_call = keys * 256 + gathered + B * (24 * 256 * 2 * 2 + 2 * 2 * 256 * 2 + 128 * 2 * 2)
+    res = dict(ms=ms_max, tokens=B * n_timed * world, kern=kern, launches=sum(c for c, _ in kern.values()),
+               clocks=clk.summary(), bytes_step=bytes_call * DECODE_CALLS, bytes_indexer=keys * 256,
+               steps=steps, calls=n_timed)
     if want_e2e:
-        hosts = [{k: torch.empty(step_in[0][k].shape, dtype=step_in[0][k].dtype, pin_memory=True) for k in names}
-                 for _ in range(2)]
-        for h in hosts:
-            for k in names:
-                h[k].copy_(step_in[0][k])
+        # every call: that call's inputs copied in from pinned host memory, the
+        # output copied back
+        hosts = {k: torch.empty(allin[k].shape, dtype=allin[k].dtype, pin_memory=True) for k in names}
+        for k in names:
+            hosts[k].copy_(allin[k])
         out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-        bi = sum(hosts[0][k].numel() * hosts[0][k].element_size() for k in names)
-        bo = out_h.numel() * out_h.element_size()
-        e_steps = max(1, min(steps, 3))
+        bi = sum(step_in[0][k].numel() * step_in[0][k].element_size() for k in names) * DECODE_CALLS
+        bo = out_h.numel() * out_h.element_size() * DECODE_CALLS
         xdev = {k: torch.empty_like(step_in[0][k]) for k in names}
 
-        def e2e_step(i):
-            for k in names:
-                xdev[k].copy_(hosts[i % 2][k], non_blocking=True)
-            step(xdev)
-            out_h.copy_(out, non_blocking=True)
+        def e2e_step():
+            nonlocal si
+            for _ in range(DECODE_CALLS):
+                for k in names:
+                    xdev[k].copy_(hosts[k][si], non_blocking=True)
+                call(xdev)
+                si += 1
+                out_h.copy_(out, non_blocking=True)
 
         barrier(world)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for i in range(e_steps):
-            e2e_step(i)
+        for _ in range(e_steps):
+            e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
         ems = max_over_ranks(e0.elapsed_time(e1), world)
-        res["e2e"] = dict(value=B * e_steps * world / (ems / 1e3), unit="tokens/s", h2d_bytes_per_step=bi,
-                          d2h_bytes_per_step=bo, steps=e_steps)
-    del kc, vc, ic, ws, step_in
+        res["e2e"] = dict(value=B * DECODE_CALLS * e_steps * world / (ems / 1e3), unit="tokens/s",
+                          h2d_bytes_per_step=bi, d2h_bytes_per_step=bo, steps=e_steps)
+        del hosts, out_h
+    del kc, vc, ic, ws, step_in, allin
     torch.cuda.empty_cache()
     return res
 
@@ -460,12 +478,49 @@ def line_for(name, res, n_gpus, steps, warmup, pk):
         whole["frac_of_hbm_roofline"] = whole["gbs"] / pk["hbm"]
         metric = "QSA decode tokens/s at 256K context, batch 64"
         cfg = dict(workload=name, batch=B, context=L, budget_blocks=512, planted="8 per sequence",
-                   l2="4.3 GB of indexer keys streamed per step (larger than L2)")
+                   decode_tokens_per_step=DECODE_CALLS,
+                   l2="4.3 GB of indexer keys streamed per decode token (larger than L2)")
     return dict(metric=metric, value=value, unit="tokens/s", n_gpus=n_gpus, steps=steps, warmup=warmup,
                 ms_per_step=res["ms"] / steps, higher_is_better=True, scaling="weak", vs_baseline=None,
                 dtype="bf16", data="synthetic", config=cfg, roofline=roof, step_roofline=whole,
                 clocks=res["clocks"], gpu_launches=res["launches"], e2e=res.get("e2e"),
                 kernels_ms={k: dict(launches=c, total_ms=round(tt, 3)) for k, (c, tt) in res["kern"].items()})
+
+
+def ncu_case(spec: str):
+    """A small case of the hot path for profiler captures (not a benchmark)."""
+    import block_sparse_long_qsa_b200 as qsa
+    torch.cuda.set_device(0)
+    parts = spec.split(":")
+    if parts[0] == "prefill":
+        T = int(parts[1])
+        P = Q.PrefillProblem(T=T, seed=0, n_plant=8, dist="uniform")
+        d = P.device()
+        for _ in range(2):
+            r = qsa.prefill(d["q"], d["k"], d["v"], d["q_idx"], d["w"], d["k_idx"], budget=512, want_lse=False)
+        torch.cuda.synchronize()
+        assert qsa.qsa_check_device_error(r["ws"]) == 0
+    else:
+        B, L = int(parts[1]), int(parts[2])
+        D = Q.DecodeProblem(B=B, L=L, steps=2, seed=0, n_plant=8)
+        max_len = L + 8
+        kc = torch.empty((B, max_len, 2, 256), dtype=torch.uint16, device="cuda")
+        vc = torch.empty_like(kc)
+        ic = torch.empty((B, max_len, 128), dtype=torch.uint16, device="cuda")
+        D.fill_device_caches(kc, vc, ic)
+        ring = torch.zeros((B, 4, 4, 128), dtype=torch.uint16, device="cuda")
+        wring = torch.zeros((B, 4, 4), dtype=torch.uint16, device="cuda")
+        p = qsa.params(512)
+        ws = qsa.workspace(qsa.qsa_decode_workspace_size(p, B, max_len))
+        out = torch.empty((B, 24, 256), dtype=torch.uint16, device="cuda")
+        for s in range(2):
+            x = {k: torch.from_numpy(v).cuda() for k, v in D.step_inputs(s).items()}
+            kn = torch.zeros((B, 128), dtype=torch.uint16, device="cuda")
+            qsa.qsa_decode(p, B, max_len, [L + s] * B, kc, vc, ic, ring, wring, x["q"], x["k"], x["v"], x["q_idx"],
+                           kn, x["w"], out, ws=ws)
+        torch.cuda.synchronize()
+        assert qsa.qsa_check_device_error(ws) == 0
+    print("ncu case done", spec)
 
 
 def main():
@@ -478,8 +533,13 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--ncu-case", default=None,
+                    help="prefill:T or decode:B:L -- one warm-up and one call of a small case (for ncu captures)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
+    if args.ncu_case:
+        ncu_case(args.ncu_case)
+        return
 
     if args.impl == "reference":
         if rank != 0:
@@ -523,7 +583,7 @@ def main():
             if w2["kind"] == "prefill":
                 r2 = run_prefill(w2["T"], 512, args.steps, args.warmup, rank, world, seed=0, want_e2e=False)
             else:
-                r2 = run_decode(w2["B"], w2["L"], 512, max(args.steps, 8), args.warmup, rank, world, seed=0,
+                r2 = run_decode(w2["B"], w2["L"], 512, args.steps, args.warmup, rank, world, seed=0,
                                 want_e2e=False)
             l2 = line_for(name, r2, world, args.steps, args.warmup, pk)
             sec[name] = {k: l2[k] for k in ("metric", "value", "unit", "ms_per_step", "roofline", "step_roofline",

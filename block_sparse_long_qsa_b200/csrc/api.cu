@@ -344,8 +344,8 @@ qsa_status qsa_prefill(const qsa_params* p, int64_t T, int64_t pos0, const uint1
          }))) != QSA_OK)
       return st;
     if ((st = from_cuda(traced(QSA_KERNEL_ATTENTION, s, [&] {
-           return qsa::launch_sparse_attn_prefill(T, q, k_rot, v, cs, sel + qb0 * budget, cnt + qb0, budget, qb0, qb1,
-                                                  scale_log2, out, lse, s);
+           return qsa::launch_sparse_attn_prefill_tc(T, q, k_rot, v, cs, sel + qb0 * budget, cnt + qb0, budget, qb0,
+                                                     qb1, scale_log2, out, lse, err, di.num_sms, s);
          }))) != QSA_OK)
       return st;
     qb0 = qb1;

@@ -1,0 +1,451 @@
+// Stage 3 (prefill) on the 5th-generation tensor cores: sparse GQA attention
+// over the selected micro-blocks ("sparse core attention", page "Qwen3.8-
+// Flash-Next, 1/9의 학습 비용으로 Qwen3.7-Plus(397B-A17B) 수준에 도달한 125B-A6B
+// 모델", section "QSA: 인덱서 자체의 비용을 줄이는 희소 어텐션"; shapes from its
+// spec table).
+//
+//   out[t][h] = sum_j softmax_j(q_rot[t][h] . k_rot[j][g] / 16) v[j][g],
+//   g = h / 12, j over the selected blocks of block t/4 with j <= t.
+//
+// Work item = (query block, KV head): 48 query rows (4 tokens x 12 heads)
+// against up to budget x 4 keys.  Persistent CTAs (one per SM) walk the items.
+//   * warps 0-3 (loaders): Q tile with RoPE applied on the fly, then the
+//     selected K and V rows, 64 keys (16 blocks) per stage, gathered with
+//     cp.async into the canonical 128-byte-swizzled K-major layout (8 KB per
+//     64-dim chunk); 3 stages of 64 KB.
+//   * warp 6 (MMA, one thread): S = Q K^T with M = 128 (rows 48..127 are
+//     padding whose results are never read), N = 64, K = 256 into one of two
+//     TMEM S buffers; O += P V with P taken from TMEM (A operand) and V as an
+//     MN-major shared-memory operand, M = 128, N = 256, fp32 in TMEM.
+//   * warps 4-5 (softmax): one thread per query row (TMEM lanes 0..63):
+//     mask, running max in base 2 (raised only when a tile's max exceeds it by
+//     more than 8, so the O rescale is rare), exp2, row sum, P packed to bf16
+//     and stored back into the S buffer's first 32 columns; at the end of an
+//     item O is read, normalised and written as bf16 with the row's lse.
+//   * every mbarrier wait is bounded (timeout -> error word, clean exit).
+#include <cfloat>
+
+#include "qsa_device.cuh"
+#include "qsa_kernels.h"
+
+namespace qsa {
+namespace {
+
+constexpr int KT = 64;                              // keys per stage
+constexpr int NSTAGE = 3;
+constexpr int THREADS = 256;
+constexpr int LOADERS = 128;
+constexpr uint32_t QROWS = 48;
+constexpr uint32_t CHUNK_Q = QROWS * 128;           // 6 KB: 48 rows x 64 dims
+constexpr uint32_t CHUNK_KV = KT * 128;             // 8 KB: 64 keys x 64 dims
+constexpr uint32_t KV_BYTES = 4 * CHUNK_KV;         // 32 KB per K (or V) tile
+constexpr uint32_t STAGE_BYTES = 2 * KV_BYTES;      // K + V
+constexpr uint32_t OFF_STAGE = 32768;               // Q region (24 KB) padded to 32 KB
+constexpr uint32_t OFF_BAR = OFF_STAGE + NSTAGE * STAGE_BYTES;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
+static_assert(SMEM_BYTES <= 232448, "attention smem");
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TM_S0 = 0, TM_O = 256;           // S buffers at columns 0 and 64; O at 256
+
+__device__ __forceinline__ uint32_t swz128(uint32_t row, uint32_t c16) {
+  return row * 128u + ((c16 ^ (row & 7u)) << 4);
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// MN-major operand descriptor (128-byte swizzle): LBO = distance between
+// 64-element atoms along N, SBO = distance between 8-row groups along K.
+__device__ __forceinline__ uint64_t umma_desc_mn_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+// O[tmem] (+)= A[tmem] * B[smem]
+__device__ __forceinline__ void umma_ts_bf16(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+struct TcArgs {
+  int64_t T;
+  const uint16_t* q;        // [T][24][256] unrotated
+  const uint16_t* k_rot;    // [T][2][256]
+  const uint16_t* v;        // [T][2][256]
+  const float2* cs;         // [T][32] RoPE table
+  const int32_t* sel;       // [rows][budget], rows relative to qb_begin
+  const int32_t* cnt;       // [rows]
+  int budget;
+  int64_t qb_begin, n_qb;
+  float scale_log2;
+  uint16_t* out;            // [T][24][256]
+  float* lse;               // [T][24] or null
+  uint32_t* err;
+};
+
+__global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kv_full = bars + 2;             // [NSTAGE]
+  uint64_t* kv_empty = bars + 2 + NSTAGE;   // [NSTAGE]
+  uint64_t* s_full = bars + 2 + 2 * NSTAGE; // [2]
+  uint64_t* p_full = s_full + 2;            // [2]
+  uint64_t* pv_done = s_full + 4;
+  uint64_t* o_full = s_full + 5;
+  uint64_t* o_empty = s_full + 6;
+  uint64_t* mma_done = s_full + 7;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if ((smem_u32(smem) & 1023u) != 0u) {
+    if (tid == 0) report_error(a.err, QSA_ERR_DEVICE_BOUNDS);
+    return;
+  }
+  if (tid == 0) {
+    mbar_init(q_full, LOADERS);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < NSTAGE; ++s) { mbar_init(&kv_full[s], LOADERS); mbar_init(&kv_empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&s_full[b], 1); mbar_init(&p_full[b], 2); }
+    mbar_init(pv_done, 1);
+    mbar_init(o_full, 1);
+    mbar_init(o_empty, 2);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 6) { tmem_alloc(tmem_slot, TMEM_COLS); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int64_t n_items = 2 * a.n_qb;
+
+  if (warp < 4) {
+    // ---------------------------------------------------------------- loaders
+    int stage = 0;
+    uint32_t ephase = 1;
+    uint32_t items_done = 0;
+    bool ok = true;
+    for (int64_t w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++items_done) {
+      const int64_t row = w >> 1;
+      const int g = (int)(w & 1);
+      const int64_t qb = a.qb_begin + row;
+      const int cnt = a.cnt[row];
+      const int32_t* sel = a.sel + row * a.budget;
+      // Q tile, RoPE on dims 0..63 (pairs i, i+32)
+      if (items_done > 0 && !mbar_wait(q_empty, (items_done - 1) & 1, abort_flag, a.err)) { ok = false; break; }
+      for (int e = tid; e < (int)QROWS * 28; e += LOADERS) {
+        const int r = e / 28, slot = e % 28;
+        const int64_t t = 4 * qb + r / 12;
+        const int h = 12 * g + r % 12;
+        uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
+        const int q16 = slot < 4 ? slot : slot + 4;          // 16-byte chunk of the 512-byte row
+        if (t < a.T) {
+          const uint4* src = reinterpret_cast<const uint4*>(a.q + (t * 24 + h) * 256);
+          lo = __ldg(src + q16);
+          if (slot < 4) {
+            hi = __ldg(src + slot + 4);
+            const float2* c8 = a.cs + t * 32 + 8 * slot;
+            const uint32_t* x = reinterpret_cast<const uint32_t*>(&lo);
+            const uint32_t* y = reinterpret_cast<const uint32_t*>(&hi);
+            uint4 olo, ohi;
+            uint32_t* ox = reinterpret_cast<uint32_t*>(&olo);
+            uint32_t* oy = reinterpret_cast<uint32_t*>(&ohi);
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              const float2 c0 = c8[2 * p], c1 = c8[2 * p + 1];
+              const float x0 = bf16lo(x[p]), x1 = bf16hi(x[p]), y0 = bf16lo(y[p]), y1 = bf16hi(y[p]);
+              ox[p] = pack_bf16x2(x0 * c0.x - y0 * c0.y, x1 * c1.x - y1 * c1.y);
+              oy[p] = pack_bf16x2(y0 * c0.x + x0 * c0.y, y1 * c1.x + x1 * c1.y);
+            }
+            lo = olo;
+            hi = ohi;
+          }
+        }
+        *reinterpret_cast<uint4*>(smem + (q16 >> 3) * CHUNK_Q + swz128(r, q16 & 7)) = lo;
+        if (slot < 4) *reinterpret_cast<uint4*>(smem + swz128(r, slot + 4)) = hi;
+      }
+      fence_proxy_async();
+      mbar_arrive(q_full);
+      // K / V tiles
+      const int n_tiles = (cnt + 15) / 16;
+      const int64_t t_last = 4 * qb + 3;
+      int prev_stage = -1;
+      for (int i = 0; i < n_tiles; ++i) {
+        if (!mbar_wait(&kv_empty[stage], ephase, abort_flag, a.err)) { ok = false; break; }
+        const uint32_t base = smem_u32(smem + OFF_STAGE + stage * STAGE_BYTES);
+#pragma unroll 4
+        for (int e = tid; e < 2 * KT * 32; e += LOADERS) {
+          const int isv = e >> 11;
+          const int n = (e >> 5) & 63;          // key slot
+          const int c32 = e & 31;               // 16-byte chunk of the 512-byte row
+          const int blk = 16 * i + (n >> 2);
+          bool valid = blk < cnt;
+          int64_t j = 0;
+          if (valid) {
+            j = 4 * (int64_t)__ldg(sel + blk) + (n & 3);
+            valid = j <= t_last && j < a.T;
+          }
+          const uint16_t* src = (isv ? a.v : a.k_rot) + (valid ? ((j * 2 + g) * 256 + c32 * 8) : 0);
+          const uint32_t dst = base + isv * KV_BYTES + (c32 >> 3) * CHUNK_KV + swz128(n, c32 & 7);
+          cp_async16(dst, src, valid);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        if (prev_stage >= 0) {
+          asm volatile("cp.async.wait_group 1;" ::: "memory");
+          fence_proxy_async();
+          mbar_arrive(&kv_full[prev_stage]);
+        }
+        prev_stage = stage;
+        if (++stage == NSTAGE) { stage = 0; ephase ^= 1; }
+      }
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      if (prev_stage >= 0) {
+        fence_proxy_async();
+        mbar_arrive(&kv_full[prev_stage]);
+      }
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+  } else if (warp == 6) {
+    // -------------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = umma_idesc_bf16_f32(128, KT);
+      constexpr uint32_t idesc_pv = umma_idesc_bf16_f32(128, 256) | (1u << 16);   // B (V) MN-major
+      int stage = 0;
+      uint32_t fphase = 0;
+      uint32_t items_done = 0, s_count = 0, p_count = 0;
+      bool ok = true;
+      const uint32_t q_base = smem_u32(smem);
+      for (int64_t w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++items_done) {
+        const int64_t row = w >> 1;
+        const int cnt = a.cnt[row];
+        const int n_tiles = (cnt + 15) / 16;
+        if (!mbar_wait(q_full, items_done & 1, abort_flag, a.err)) { ok = false; break; }
+        tc_fence_after();
+        int pv_stage = stage;           // stage of the tile whose PV is next
+        auto issue_pv = [&](int j, bool last) -> bool {
+          const uint32_t b = p_count & 1;
+          if (!mbar_wait(&p_full[b], (p_count >> 1) & 1, abort_flag, a.err)) return false;
+          if (j == 0 && items_done > 0 && !mbar_wait(o_empty, (items_done - 1) & 1, abort_flag, a.err)) return false;
+          tc_fence_after();
+          const uint32_t v_base = smem_u32(smem + OFF_STAGE + pv_stage * STAGE_BYTES + KV_BYTES);
+#pragma unroll
+          for (int ks = 0; ks < KT / 16; ++ks) {
+            const uint64_t bd = umma_desc_mn_sw128(v_base + ks * 2048, CHUNK_KV, 1024);
+            umma_ts_bf16(tmem + TM_O, tmem + TM_S0 + 64 * b + 8 * ks, bd, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
+          }
+          tc_commit(&kv_empty[pv_stage]);
+          tc_commit(pv_done);
+          if (last) tc_commit(o_full);
+          ++p_count;
+          if (++pv_stage == NSTAGE) pv_stage = 0;
+          return true;
+        };
+        for (int i = 0; i < n_tiles && ok; ++i) {
+          if (!mbar_wait(&kv_full[stage], fphase, abort_flag, a.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t b = s_count & 1;
+          const uint32_t k_base = smem_u32(smem + OFF_STAGE + stage * STAGE_BYTES);
+#pragma unroll
+          for (int ks = 0; ks < 16; ++ks) {
+            const uint32_t c = ks >> 2, koff = (ks & 3) * 32;
+            const uint64_t ad = umma_desc_k_sw128(q_base + c * CHUNK_Q + koff);
+            const uint64_t bd = umma_desc_k_sw128(k_base + c * CHUNK_KV + koff);
+            umma_bf16(tmem + TM_S0 + 64 * b, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+          }
+          tc_commit(&s_full[b]);
+          if (i == n_tiles - 1) tc_commit(q_empty);
+          ++s_count;
+          if (++stage == NSTAGE) { stage = 0; fphase ^= 1; }
+          if (i >= 1 && !issue_pv(i - 1, false)) { ok = false; break; }
+        }
+        if (ok && n_tiles > 0 && !issue_pv(n_tiles - 1, true)) ok = false;
+      }
+      tc_commit(mma_done);
+      mbar_wait(mma_done, 0, abort_flag, a.err);
+    }
+  } else if (warp == 4 || warp == 5) {
+    // ---------------------------------------------------------------- softmax
+    const int r = 32 * (warp - 4) + lane;           // query row = TMEM lane
+    const bool row_ok = r < (int)QROWS;
+    const int tok = row_ok ? r / 12 : 0, hh = row_ok ? r % 12 : 0;
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    uint32_t items_done = 0, s_count = 0, pv_count = 0;
+    bool ok = true;
+    for (int64_t w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++items_done) {
+      const int64_t row = w >> 1;
+      const int g = (int)(w & 1);
+      const int64_t qb = a.qb_begin + row;
+      const int cnt = a.cnt[row];
+      const int32_t* sel = a.sel + row * a.budget;
+      const int n_tiles = (cnt + 15) / 16;
+      const int64_t t = 4 * qb + tok;
+      float m_run = -FLT_MAX, l_run = 0.f;
+      for (int i = 0; i < n_tiles; ++i) {
+        const uint32_t b = s_count & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&s_full[b], (s_count >> 1) & 1, abort_flag, a.err))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float s[64];
+        {
+          float tmp[32];
+          tmem_ld32(tmem + lane_off + TM_S0 + 64 * b, tmp);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) s[c] = tmp[c];
+          tmem_ld32(tmem + lane_off + TM_S0 + 64 * b + 32, tmp);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) s[32 + c] = tmp[c];
+          tmem_ld_wait();
+        }
+        // selected blocks of this tile (4 x 16 bytes of the selection row)
+        int32_t kb[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) kb[q] = 16 * i + q < cnt ? __ldg(sel + 16 * i + q) : -1;
+        float mt = -FLT_MAX;
+#pragma unroll
+        for (int n = 0; n < 64; ++n) {
+          const int blk = 16 * i + (n >> 2);
+          const int64_t j = 4 * (int64_t)kb[n >> 2] + (n & 3);
+          const bool valid = row_ok && blk < cnt && j <= t;
+          s[n] = valid ? s[n] * a.scale_log2 : -FLT_MAX;
+          mt = fmaxf(mt, s[n]);
+        }
+        if (i >= 1) {   // PV(i-1) complete before O may be rescaled (and keeps phases in step)
+          if (!__all_sync(0xffffffffu, mbar_wait(pv_done, pv_count & 1, abort_flag, a.err))) { ok = false; break; }
+          ++pv_count;
+        }
+        const bool need = mt > m_run + 8.f;
+        if (__any_sync(0xffffffffu, need)) {
+          const float m_new = need ? fmaxf(m_run, mt) : m_run;
+          const float corr = ex2(m_run - m_new);
+          l_run *= corr;
+          m_run = m_new;
+          if (i >= 1) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < 8; ++c) {
+              float o[32];
+              tmem_ld32(tmem + lane_off + TM_O + 32 * c, o);
+              tmem_ld_wait();
+              uint32_t u[32];
+#pragma unroll
+              for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(o[e] * corr);
+              tmem_st32(tmem + lane_off + TM_O + 32 * c, u);
+            }
+            tmem_st_wait();
+          }
+        }
+        uint32_t pk[32];
+        float lsum = 0.f;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float p0 = s[2 * e] == -FLT_MAX ? 0.f : ex2(s[2 * e] - m_run);
+          const float p1 = s[2 * e + 1] == -FLT_MAX ? 0.f : ex2(s[2 * e + 1] - m_run);
+          lsum += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        l_run += lsum;
+        tmem_st32(tmem + lane_off + TM_S0 + 64 * b, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[b]);
+        ++s_count;
+      }
+      if (!ok) break;
+      // item end: O / l -> bf16
+      if (!__all_sync(0xffffffffu, mbar_wait(o_full, items_done & 1, abort_flag, a.err))) { ok = false; break; }
+      ++pv_count;   // the last PV of the item also completed
+      tc_fence_after();
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      const bool write = row_ok && t < a.T && n_tiles > 0;
+      uint16_t* orow = a.out + (t * 24 + 12 * g + hh) * 256;
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        float o[32];
+        tmem_ld32(tmem + lane_off + TM_O + 32 * c, o);
+        tmem_ld_wait();
+        if (write) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(pack_bf16x2(o[8 * q] * inv, o[8 * q + 1] * inv),
+                                pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
+                                pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
+                                pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+        }
+      }
+      if (write && a.lse) a.lse[t * 24 + 12 * g + hh] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_empty);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 6) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_sparse_attn_prefill_tc(int64_t T, const uint16_t* q, const uint16_t* k_rot, const uint16_t* v,
+                                          const float2* cs, const int32_t* sel, const int32_t* cnt, int budget,
+                                          int64_t qb_begin, int64_t qb_end, float scale_log2, uint16_t* out,
+                                          float* lse, uint32_t* err, int num_sms, cudaStream_t stream) {
+  if (qb_end <= qb_begin) return cudaSuccess;
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = true;
+  }
+  TcArgs a;
+  a.T = T; a.q = q; a.k_rot = k_rot; a.v = v; a.cs = cs; a.sel = sel; a.cnt = cnt; a.budget = budget;
+  a.qb_begin = qb_begin; a.n_qb = qb_end - qb_begin; a.scale_log2 = scale_log2; a.out = out; a.lse = lse;
+  a.err = err;
+  const int64_t items = 2 * (qb_end - qb_begin);
+  const int grid = (int)(items < num_sms ? items : num_sms);
+  sparse_attn_tc_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace qsa

@@ -237,7 +237,7 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     uint32_t acc_use[2] = {0, 0};
     for (; it.valid(); it.next()) {
       if (it.first_of_tile(u0)) {
-        if (!mbar_wait(qfull, qcount & 1, abort_flag, err)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(qfull, qcount & 1, abort_flag, err))) break;
         ++qcount;
       }
       const int64_t t_tile = sch.T0 + QT * it.tile;
@@ -246,7 +246,10 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
       const int64_t kb = j >> 2;
       bool ok = true;
       for (int hf = 0; hf < 2; ++hf) {
-        if (!mbar_wait(&accfull[hf], acc_use[hf] & 1, abort_flag, err)) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(&accfull[hf], acc_use[hf] & 1, abort_flag, err))) {
+          ok = false;
+          break;
+        }
         ++acc_use[hf];
         tc_fence_after();
         const int64_t t_first = t_tile + 64 * hf + 32 * cgrp;  // first token of this thread's columns

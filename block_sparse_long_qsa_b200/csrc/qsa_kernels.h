@@ -22,7 +22,13 @@ size_t select_smem_bytes(int budget);
 cudaError_t launch_select(const float* S, int64_t ld, int64_t qb_begin, int64_t n_rows, const int64_t* row_qb,
                           int budget, int32_t* sel, int32_t* cnt, uint32_t* err, cudaStream_t stream);
 
-// Sparse GQA attention for query blocks [qb_begin, qb_end) given their selections.
+// Sparse GQA attention for query blocks [qb_begin, qb_end) given their
+// selections (sel/cnt indexed from qb_begin): tcgen05 kernel, persistent.
+cudaError_t launch_sparse_attn_prefill_tc(int64_t T, const uint16_t* q, const uint16_t* k_rot, const uint16_t* v,
+                                          const float2* cs, const int32_t* sel, const int32_t* cnt, int budget,
+                                          int64_t qb_begin, int64_t qb_end, float scale_log2, uint16_t* out,
+                                          float* lse, uint32_t* err, int num_sms, cudaStream_t stream);
+// Same, on mma.sync (used for comparison in tests only through the decode path's template).
 cudaError_t launch_sparse_attn_prefill(int64_t T, const uint16_t* q, const uint16_t* k_rot, const uint16_t* v,
                                        const float2* cs, const int32_t* sel, const int32_t* cnt, int budget,
                                        int64_t qb_begin, int64_t qb_end, float scale_log2, uint16_t* out, float* lse,
