@@ -24,7 +24,8 @@ _STATUS = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_UNSUPPORTED", 3: "
 
 EXPORTED = ["qsa_default_params", "qsa_status_string", "qsa_last_error", "qsa_index_scores", "qsa_select_blocks",
             "qsa_select_workspace_size", "qsa_prefill", "qsa_prefill_workspace_size", "qsa_decode",
-            "qsa_decode_workspace_size", "qsa_check_device_error", "qsa_trace_begin", "qsa_trace_end"]
+            "qsa_decode_workspace_size", "qsa_check_device_error", "qsa_trace_begin", "qsa_trace_end",
+            "qsa_decode_noalloc"]
 
 KERNEL_NAMES = {1: "rope_table", 2: "rope_k", 3: "indexer", 4: "select", 5: "attention", 6: "decode_append",
                 7: "decode_indexer", 8: "decode_attention", 9: "decode_combine"}
@@ -71,6 +72,8 @@ def load(path: str = LIB_PATH):
     L.qsa_decode.argtypes = [P, i32, i64, ctypes.POINTER(ctypes.c_int64), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                              vp, vp, vp, vp, sz, vp]
     L.qsa_decode_workspace_size.argtypes = [P, i32, i64, psz]
+    L.qsa_decode_noalloc.argtypes = [P, i32, i64, ctypes.POINTER(ctypes.c_int64), vp, vp, vp, vp, vp, vp, vp, vp,
+                                     vp, vp, vp, vp, vp, vp, vp]
     L.qsa_check_device_error.argtypes = [vp, vp]
     L.qsa_trace_begin.argtypes = [i32]
     L.qsa_trace_end.argtypes = [vp, vp, i32, ctypes.POINTER(ctypes.c_int32)]
@@ -161,6 +164,17 @@ def qsa_decode(p: qsa_params, B: int, max_len: int, cache_len, k_cache, v_cache,
                              _ptr(qidx_ring), _ptr(w_ring), _ptr(q_new), _ptr(k_new), _ptr(v_new), _ptr(q_idx_new),
                              _ptr(k_idx_new), _ptr(w_new), _ptr(out), _ptr(sel_out), _ptr(lse_out), _ptr(ws),
                              ws.numel() * ws.element_size(), _stream(stream)), "qsa_decode")
+
+
+def qsa_decode_noalloc(p: qsa_params, B: int, max_len: int, cache_len, k_cache, v_cache, kidx_cache, qidx_ring,
+                       w_ring, q_new, k_new, v_new, q_idx_new, k_idx_new, w_new, out, sel_out=None, lse_out=None,
+                       stream=None):
+    """qsa_decode on the library's fixed scratch array (no workspace, no allocation)."""
+    lens = (ctypes.c_int64 * B)(*[int(x) for x in cache_len])
+    _check(load().qsa_decode_noalloc(ctypes.byref(p), B, max_len, lens, _ptr(k_cache), _ptr(v_cache),
+                                     _ptr(kidx_cache), _ptr(qidx_ring), _ptr(w_ring), _ptr(q_new), _ptr(k_new),
+                                     _ptr(v_new), _ptr(q_idx_new), _ptr(k_idx_new), _ptr(w_new), _ptr(out),
+                                     _ptr(sel_out), _ptr(lse_out), _stream(stream)), "qsa_decode_noalloc")
 
 
 def qsa_check_device_error(ws, stream=None) -> int:

@@ -153,6 +153,31 @@ qsa_status qsa_decode(const qsa_params* p, int32_t B, int64_t max_len, const int
                       int32_t* sel_out, float* lse_out, void* ws, size_t ws_bytes, void* stream);
 qsa_status qsa_decode_workspace_size(const qsa_params* p, int32_t B, int64_t max_len, size_t* bytes);
 
+/* qsa_decode without a workspace argument; the pages have no counterpart:
+ * this exists for callers that cannot allocate device memory where they run
+ * a decode step (their device memory belongs to another runtime's budget, or
+ * cudaMalloc is not allowed on their request path).  The caller still owns
+ * and passes every input, output and cache, exactly as for qsa_decode; the
+ * decode scratch instead lives in a 64 MiB array inside this library, which
+ * is reserved on each GPU where the library's decode code is loaded and kept
+ * until the process exits.  Nothing is allocated by this call.
+ *   - Sizes whose qsa_decode_workspace_size exceeds 64 MiB are rejected with
+ *     QSA_ERR_WORKSPACE_TOO_SMALL before any launch (64 sequences at 256K
+ *     context need about 43 MiB).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) for that device; make that first call before
+ *     any stream capture.
+ *   - All calls share the one array per device: calls whose executions
+ *     overlap on the GPU (different streams, or different host threads on the
+ *     same device) race on it and must be serialised by the caller.
+ *   - Device-side errors are recorded in the shared array, which the caller
+ *     cannot read; they end the kernels cleanly but are not reported. */
+qsa_status qsa_decode_noalloc(const qsa_params* p, int32_t B, int64_t max_len, const int64_t* cache_len,
+                              uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* qidx_ring,
+                              uint16_t* w_ring, const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
+                              const uint16_t* q_idx_new, const uint16_t* k_idx_new, const uint16_t* w_new,
+                              uint16_t* out, int32_t* sel_out, float* lse_out, void* stream);
+
 /* Reads (synchronising `stream`) and clears the device error word at the
  * start of a workspace passed to qsa_select_blocks / qsa_prefill /
  * qsa_decode.  Returns QSA_OK or the first device-side error recorded. */
