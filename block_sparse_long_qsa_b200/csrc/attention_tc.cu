@@ -55,6 +55,12 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
                : "memory");
 }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// Two floats to packed bf16 (round to nearest even): lo in bits 0..15.
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -204,21 +210,23 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
       for (int i = 0; i < n_tiles; ++i) {
         if (!mbar_wait(&kv_empty[stage], ephase, abort_flag, a.err)) { ok = false; break; }
         const uint32_t base = smem_u32(smem + OFF_STAGE + stage * STAGE_BYTES);
-#pragma unroll 4
-        for (int e = tid; e < 2 * KT * 32; e += LOADERS) {
-          const int isv = e >> 11;
-          const int n = (e >> 5) & 63;          // key slot
-          const int c32 = e & 31;               // 16-byte chunk of the 512-byte row
-          const int blk = 16 * i + (n >> 2);
-          bool valid = blk < cnt;
-          int64_t j = 0;
-          if (valid) {
-            j = 4 * (int64_t)__ldg(sel + blk) + (n & 3);
-            valid = j <= t_last && j < a.T;
-          }
-          const uint16_t* src = (isv ? a.v : a.k_rot) + (valid ? ((j * 2 + g) * 256 + c32 * 8) : 0);
-          const uint32_t dst = base + isv * KV_BYTES + (c32 >> 3) * CHUNK_KV + swz128(n, c32 & 7);
-          cp_async16(dst, src, valid);
+        // Thread (warp w, lane c32) copies 16-byte chunk c32 of token w of each
+        // of the tile's 16 blocks, for K and for V: key slot n = 4k + w.  The
+        // 16 block indices are loaded up front (independent, L1-broadcast).
+        const int w4 = tid >> 5, c32 = tid & 31;
+        int32_t kbv[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) kbv[k] = 16 * i + k < cnt ? __ldg(sel + 16 * i + k) : -1;
+        const uint32_t dst0 = base + (c32 >> 3) * CHUNK_KV;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int n = 4 * k + w4;
+          const int64_t j = 4 * (int64_t)kbv[k] + w4;
+          const bool valid = kbv[k] >= 0 && j <= t_last && j < a.T;
+          const int64_t off = valid ? (j * 2 + g) * 256 + c32 * 8 : 0;
+          const uint32_t dst = dst0 + swz128(n, c32 & 7);
+          cp_async16(dst, a.k_rot + off, valid);
+          cp_async16(dst + KV_BYTES, a.v + off, valid);
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
         if (prev_stage >= 0) {
@@ -307,7 +315,6 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
       const int g = (int)(w & 1);
       const int64_t qb = a.qb_begin + row;
       const int cnt = a.cnt[row];
-      const int32_t* sel = a.sel + row * a.budget;
       const int n_tiles = (cnt + 15) / 16;
       const int64_t t = 4 * qb + tok;
       float m_run = -FLT_MAX, l_run = 0.f;
@@ -329,19 +336,24 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
           for (int c = 0; c < 32; ++c) s[32 + c] = tmp[c];
           tmem_ld_wait();
         }
-        // selected blocks of this tile (4 x 16 bytes of the selection row)
-        int32_t kb[16];
+        // Masking.  The selection is ascending and always ends with the own
+        // block, so every key of a tile before the last one is visible to
+        // every row; in the last tile, slots past cnt and the own block's
+        // tokens after the row's token are masked.
+        const bool last = i == n_tiles - 1;
+        if (last) {
 #pragma unroll
-        for (int q = 0; q < 16; ++q) kb[q] = 16 * i + q < cnt ? __ldg(sel + 16 * i + q) : -1;
+          for (int n = 0; n < 64; ++n) {
+            const int blk = 16 * i + (n >> 2);
+            const bool valid = blk < cnt && (blk < cnt - 1 || (n & 3) <= tok);
+            s[n] = valid ? s[n] : -FLT_MAX;
+          }
+        }
         float mt = -FLT_MAX;
 #pragma unroll
-        for (int n = 0; n < 64; ++n) {
-          const int blk = 16 * i + (n >> 2);
-          const int64_t j = 4 * (int64_t)kb[n >> 2] + (n & 3);
-          const bool valid = row_ok && blk < cnt && j <= t;
-          s[n] = valid ? s[n] * a.scale_log2 : -FLT_MAX;
-          mt = fmaxf(mt, s[n]);
-        }
+        for (int n = 0; n < 63; n += 3) mt = fmaxf(mt, max3f(s[n], s[n + 1], s[n + 2]));
+        mt = fmaxf(mt, s[63]);
+        mt = row_ok ? mt * a.scale_log2 : -FLT_MAX;   // raw max, then the (positive) scale
         if (i >= 1) {   // PV(i-1) complete before O may be rescaled (and keeps phases in step)
           if (!__all_sync(0xffffffffu, mbar_wait(pv_done, pv_count & 1, abort_flag, a.err))) { ok = false; break; }
           ++pv_count;
@@ -367,15 +379,19 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
             tmem_st_wait();
           }
         }
+        // p = 2^(s*scale - m); masked slots (-FLT_MAX) underflow to exactly 0
         uint32_t pk[32];
-        float lsum = 0.f;
+        float lsum0 = 0.f, lsum1 = 0.f;
+        const float neg_m = -m_run;
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const float p0 = s[2 * e] == -FLT_MAX ? 0.f : ex2(s[2 * e] - m_run);
-          const float p1 = s[2 * e + 1] == -FLT_MAX ? 0.f : ex2(s[2 * e + 1] - m_run);
-          lsum += p0 + p1;
-          pk[e] = pack_bf16x2(p0, p1);
+          const float p0 = ex2(fmaf(s[2 * e], a.scale_log2, neg_m));
+          const float p1 = ex2(fmaf(s[2 * e + 1], a.scale_log2, neg_m));
+          lsum0 += p0;
+          lsum1 += p1;
+          pk[e] = cvt_bf16x2(p0, p1);
         }
+        const float lsum = lsum0 + lsum1;
         l_run += lsum;
         tmem_st32(tmem + lane_off + TM_S0 + 64 * b, pk);
         tmem_st_wait();
@@ -401,10 +417,10 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            dst[q] = make_uint4(pack_bf16x2(o[8 * q] * inv, o[8 * q + 1] * inv),
-                                pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
-                                pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
-                                pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+            dst[q] = make_uint4(cvt_bf16x2(o[8 * q] * inv, o[8 * q + 1] * inv),
+                                cvt_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
+                                cvt_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
+                                cvt_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
         }
       }
       if (write && a.lse) a.lse[t * 24 + 12 * g + hh] = (m_run + log2f(l_run)) * 0.69314718055994531f;
