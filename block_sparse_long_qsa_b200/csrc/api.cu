@@ -14,7 +14,6 @@ namespace {
 
 constexpr size_t HEADER_BYTES = 256;            // device error word + padding
 constexpr size_t ALIGN = 256;
-constexpr int DECODE_SPLIT = 16;
 constexpr int MAX_DEV = 64;
 
 // Last failure of this thread, for qsa_last_error().
@@ -356,7 +355,7 @@ qsa_status qsa_prefill(const qsa_params* p, int64_t T, int64_t pos0, const uint1
 // ------------------------------------------------------------------ decode
 namespace {
 struct DecodeLayout {
-  size_t Ls, qbs, S, sel, cnt, q_rot, part_o, part_lse, total;
+  size_t Ls, qbs, S, sel, cnt, q_rot, total;
   int64_t ld;
 };
 DecodeLayout decode_layout(int B, int64_t max_len, int budget) {
@@ -369,8 +368,6 @@ DecodeLayout decode_layout(int B, int64_t max_len, int budget) {
   L.sel = off; off = align_up(off + (size_t)B * budget * 4);
   L.cnt = off; off = align_up(off + (size_t)B * 4);
   L.q_rot = off; off = align_up(off + (size_t)B * 24 * 256 * 2);
-  L.part_o = off; off = align_up(off + (size_t)B * DECODE_SPLIT * 24 * 256 * 4);
-  L.part_lse = off; off = align_up(off + (size_t)B * DECODE_SPLIT * 24 * 4);
   L.total = off;
   return L;
 }
@@ -421,8 +418,6 @@ qsa_status qsa_decode(const qsa_params* p, int32_t B, int64_t max_len, const int
   int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(base + L.sel);
   int32_t* cnt = reinterpret_cast<int32_t*>(base + L.cnt);
   uint16_t* q_rot = reinterpret_cast<uint16_t*>(base + L.q_rot);
-  float* part_o = reinterpret_cast<float*>(base + L.part_o);
-  float* part_lse = reinterpret_cast<float*>(base + L.part_lse);
 
   if (cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaMemsetAsync");
   double f[32];
@@ -444,13 +439,9 @@ qsa_status qsa_decode(const qsa_params* p, int32_t B, int64_t max_len, const int
        }))) != QSA_OK)
     return st;
   const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
-  if ((st = from_cuda(traced(QSA_KERNEL_DECODE_ATTENTION, s, [&] {
-         return qsa::launch_decode_attn(B, max_len, Ls, q_rot, k_cache, v_cache, sel, cnt, budget, DECODE_SPLIT,
-                                        scale_log2, part_o, part_lse, s);
-       }))) != QSA_OK)
-    return st;
-  return from_cuda(traced(QSA_KERNEL_DECODE_COMBINE, s, [&] {
-    return qsa::launch_decode_combine(B, DECODE_SPLIT, part_o, part_lse, out, lse_out, s);
+  return from_cuda(traced(QSA_KERNEL_DECODE_ATTENTION, s, [&] {
+    return qsa::launch_decode_attn_tc(B, max_len, Ls, q_rot, k_cache, v_cache, sel, cnt, budget, scale_log2, out,
+                                      lse_out, err, di.num_sms, s);
   }));
 }
 

@@ -114,9 +114,45 @@ struct TcArgs {
   uint16_t* out;            // [T][24][256]
   float* lse;               // [T][24] or null
   uint32_t* err;
+  // decode: q = rotated new-token queries [B][24][256], k_rot / v = caches
+  // [B][max_len][2][256], out / lse [B][24][...], one query token per sequence
+  const int64_t* Ls;        // [B] position of the new token
+  int64_t max_len;
 };
 
+// One work item = (query block, KV head) for prefill, (sequence, KV head) for decode.
+template <bool DEC>
+struct Item {
+  int64_t row;              // selection row
+  int g;                    // KV head
+  int64_t qb;               // query block
+  int64_t t0;               // position of the item's first query token
+  int64_t t_last;           // last key position any of its rows may read
+  const uint16_t* kb;       // rotated keys of this sequence
+  const uint16_t* vb;
+  __device__ __forceinline__ Item(const TcArgs& a, int64_t w) {
+    row = w >> 1;
+    g = (int)(w & 1);
+    if (DEC) {
+      const int64_t L = a.Ls[row];
+      qb = L >> 2;
+      t0 = L;
+      t_last = L;
+      kb = a.k_rot + row * a.max_len * 512;
+      vb = a.v + row * a.max_len * 512;
+    } else {
+      qb = a.qb_begin + row;
+      t0 = 4 * qb;
+      t_last = 4 * qb + 3 < a.T - 1 ? 4 * qb + 3 : a.T - 1;
+      kb = a.k_rot;
+      vb = a.v;
+    }
+  }
+};
+
+template <bool DEC>
 __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs a) {
+  constexpr int QR = DEC ? 12 : (int)QROWS;   // valid query rows per item
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* q_full = bars + 0;
@@ -163,24 +199,24 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
     uint32_t items_done = 0;
     bool ok = true;
     for (int64_t w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++items_done) {
-      const int64_t row = w >> 1;
-      const int g = (int)(w & 1);
-      const int64_t qb = a.qb_begin + row;
-      const int cnt = a.cnt[row];
-      const int32_t* sel = a.sel + row * a.budget;
-      // Q tile, RoPE on dims 0..63 (pairs i, i+32)
+      const Item<DEC> it(a, w);
+      const int g = it.g;
+      const int cnt = a.cnt[it.row];
+      const int32_t* sel = a.sel + it.row * a.budget;
+      // Q tile; prefill rotates dims 0..63 (pairs i, i+32) on the way in,
+      // decode queries arrive rotated
       if (items_done > 0 && !mbar_wait(q_empty, (items_done - 1) & 1, abort_flag, a.err)) { ok = false; break; }
-      for (int e = tid; e < (int)QROWS * 28; e += LOADERS) {
+      for (int e = tid; e < QR * 28; e += LOADERS) {
         const int r = e / 28, slot = e % 28;
-        const int64_t t = 4 * qb + r / 12;
+        const int64_t t = it.t0 + r / 12;
         const int h = 12 * g + r % 12;
         uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
         const int q16 = slot < 4 ? slot : slot + 4;          // 16-byte chunk of the 512-byte row
-        if (t < a.T) {
-          const uint4* src = reinterpret_cast<const uint4*>(a.q + (t * 24 + h) * 256);
+        if (DEC || t < a.T) {
+          const uint4* src = reinterpret_cast<const uint4*>(a.q + ((DEC ? it.row : t) * 24 + h) * 256);
           lo = __ldg(src + q16);
-          if (slot < 4) {
-            hi = __ldg(src + slot + 4);
+          if (slot < 4) hi = __ldg(src + slot + 4);
+          if (!DEC && slot < 4) {
             const float2* c8 = a.cs + t * 32 + 8 * slot;
             const uint32_t* x = reinterpret_cast<const uint32_t*>(&lo);
             const uint32_t* y = reinterpret_cast<const uint32_t*>(&hi);
@@ -205,8 +241,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
       mbar_arrive(q_full);
       // K / V tiles
       const int n_tiles = (cnt + 15) / 16;
-      const int64_t t_last = 4 * qb + 3;
-      int prev_stage = -1;
+      const int64_t t_last = it.t_last;
       for (int i = 0; i < n_tiles; ++i) {
         if (!mbar_wait(&kv_empty[stage], ephase, abort_flag, a.err)) { ok = false; break; }
         const uint32_t base = smem_u32(smem + OFF_STAGE + stage * STAGE_BYTES);
@@ -222,28 +257,20 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
         for (int k = 0; k < 16; ++k) {
           const int n = 4 * k + w4;
           const int64_t j = 4 * (int64_t)kbv[k] + w4;
-          const bool valid = kbv[k] >= 0 && j <= t_last && j < a.T;
+          const bool valid = kbv[k] >= 0 && j <= t_last;
           const int64_t off = valid ? (j * 2 + g) * 256 + c32 * 8 : 0;
           const uint32_t dst = dst0 + swz128(n, c32 & 7);
-          cp_async16(dst, a.k_rot + off, valid);
-          cp_async16(dst + KV_BYTES, a.v + off, valid);
+          cp_async16(dst, it.kb + off, valid);
+          cp_async16(dst + KV_BYTES, it.vb + off, valid);
         }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-        if (prev_stage >= 0) {
-          asm volatile("cp.async.wait_group 1;" ::: "memory");
-          fence_proxy_async();
-          mbar_arrive(&kv_full[prev_stage]);
-        }
-        prev_stage = stage;
+        // this thread's arrival on the stage's barrier fires when all its
+        // copies so far have landed: no blocking wait, all stages in flight
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&kv_full[stage]))
+                     : "memory");
         if (++stage == NSTAGE) { stage = 0; ephase ^= 1; }
       }
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-      if (prev_stage >= 0) {
-        fence_proxy_async();
-        mbar_arrive(&kv_full[prev_stage]);
-      }
     }
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == 6) {
     // -------------------------------------------------------------------- MMA
     if (lane == 0) {
@@ -281,6 +308,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
         };
         for (int i = 0; i < n_tiles && ok; ++i) {
           if (!mbar_wait(&kv_full[stage], fphase, abort_flag, a.err)) { ok = false; break; }
+          fence_proxy_async();    // the stage was written by cp.async; the MMA reads it
           tc_fence_after();
           const uint32_t b = s_count & 1;
           const uint32_t k_base = smem_u32(smem + OFF_STAGE + stage * STAGE_BYTES);
@@ -305,18 +333,18 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
   } else if (warp == 4 || warp == 5) {
     // ---------------------------------------------------------------- softmax
     const int r = 32 * (warp - 4) + lane;           // query row = TMEM lane
-    const bool row_ok = r < (int)QROWS;
+    const bool row_ok = r < QR;
     const int tok = row_ok ? r / 12 : 0, hh = row_ok ? r % 12 : 0;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     uint32_t items_done = 0, s_count = 0, pv_count = 0;
     bool ok = true;
     for (int64_t w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++items_done) {
-      const int64_t row = w >> 1;
-      const int g = (int)(w & 1);
-      const int64_t qb = a.qb_begin + row;
-      const int cnt = a.cnt[row];
+      const Item<DEC> it(a, w);
+      const int g = it.g;
+      const int cnt = a.cnt[it.row];
       const int n_tiles = (cnt + 15) / 16;
-      const int64_t t = 4 * qb + tok;
+      const int64_t t = it.t0 + tok;                  // this row's token position
+      const int own_lim = (int)(t & 3);               // last visible token of the own block
       float m_run = -FLT_MAX, l_run = 0.f;
       for (int i = 0; i < n_tiles; ++i) {
         const uint32_t b = s_count & 1;
@@ -345,7 +373,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
 #pragma unroll
           for (int n = 0; n < 64; ++n) {
             const int blk = 16 * i + (n >> 2);
-            const bool valid = blk < cnt && (blk < cnt - 1 || (n & 3) <= tok);
+            const bool valid = blk < cnt && (blk < cnt - 1 || (n & 3) <= own_lim);
             s[n] = valid ? s[n] : -FLT_MAX;
           }
         }
@@ -406,8 +434,9 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
       ++pv_count;   // the last PV of the item also completed
       tc_fence_after();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      const bool write = row_ok && t < a.T && n_tiles > 0;
-      uint16_t* orow = a.out + (t * 24 + 12 * g + hh) * 256;
+      const bool write = row_ok && (DEC || t < a.T) && n_tiles > 0;
+      const int64_t orow_idx = (DEC ? it.row : t) * 24 + 12 * g + hh;   // [token or sequence][head]
+      uint16_t* orow = a.out + orow_idx * 256;
 #pragma unroll 1
       for (int c = 0; c < 8; ++c) {
         float o[32];
@@ -423,7 +452,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
                                 cvt_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
         }
       }
-      if (write && a.lse) a.lse[t * 24 + 12 * g + hh] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+      if (write && a.lse) a.lse[orow_idx] = (m_run + log2f(l_run)) * 0.69314718055994531f;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(o_empty);
@@ -438,6 +467,22 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
   }
 }
 
+template <bool DEC>
+cudaError_t launch_tc(const TcArgs& a, int64_t items, int num_sms, cudaStream_t stream) {
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel<DEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = true;
+  }
+  const int grid = (int)(items < num_sms ? items : num_sms);
+  sparse_attn_tc_kernel<DEC><<<grid, THREADS, SMEM_BYTES, stream>>>(a);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_sparse_attn_prefill_tc(int64_t T, const uint16_t* q, const uint16_t* k_rot, const uint16_t* v,
@@ -445,23 +490,23 @@ cudaError_t launch_sparse_attn_prefill_tc(int64_t T, const uint16_t* q, const ui
                                           int64_t qb_begin, int64_t qb_end, float scale_log2, uint16_t* out,
                                           float* lse, uint32_t* err, int num_sms, cudaStream_t stream) {
   if (qb_end <= qb_begin) return cudaSuccess;
-  static bool attr_done[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_done[dev] = true;
-  }
-  TcArgs a;
+  TcArgs a{};
   a.T = T; a.q = q; a.k_rot = k_rot; a.v = v; a.cs = cs; a.sel = sel; a.cnt = cnt; a.budget = budget;
   a.qb_begin = qb_begin; a.n_qb = qb_end - qb_begin; a.scale_log2 = scale_log2; a.out = out; a.lse = lse;
   a.err = err;
-  const int64_t items = 2 * (qb_end - qb_begin);
-  const int grid = (int)(items < num_sms ? items : num_sms);
-  sparse_attn_tc_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(a);
-  return cudaGetLastError();
+  return launch_tc<false>(a, 2 * (qb_end - qb_begin), num_sms, stream);
+}
+
+cudaError_t launch_decode_attn_tc(int B, int64_t max_len, const int64_t* L_dev, const uint16_t* q_rot,
+                                  const uint16_t* k_cache, const uint16_t* v_cache, const int32_t* sel,
+                                  const int32_t* cnt, int budget, float scale_log2, uint16_t* out, float* lse,
+                                  uint32_t* err, int num_sms, cudaStream_t stream) {
+  if (B <= 0) return cudaSuccess;
+  TcArgs a{};
+  a.T = INT64_MAX; a.q = q_rot; a.k_rot = k_cache; a.v = v_cache; a.sel = sel; a.cnt = cnt; a.budget = budget;
+  a.qb_begin = 0; a.n_qb = B; a.scale_log2 = scale_log2; a.out = out; a.lse = lse; a.err = err;
+  a.Ls = L_dev; a.max_len = max_len;
+  return launch_tc<true>(a, 2 * (int64_t)B, num_sms, stream);
 }
 
 }  // namespace qsa

@@ -28,11 +28,6 @@ cudaError_t launch_sparse_attn_prefill_tc(int64_t T, const uint16_t* q, const ui
                                           const float2* cs, const int32_t* sel, const int32_t* cnt, int budget,
                                           int64_t qb_begin, int64_t qb_end, float scale_log2, uint16_t* out,
                                           float* lse, uint32_t* err, int num_sms, cudaStream_t stream);
-// Same, on mma.sync (used for comparison in tests only through the decode path's template).
-cudaError_t launch_sparse_attn_prefill(int64_t T, const uint16_t* q, const uint16_t* k_rot, const uint16_t* v,
-                                       const float2* cs, const int32_t* sel, const int32_t* cnt, int budget,
-                                       int64_t qb_begin, int64_t qb_end, float scale_log2, uint16_t* out, float* lse,
-                                       cudaStream_t stream);
 
 // ---------------------------------------------------------------- decode
 // Lengths come from the host array L_host (passed to the kernel as launch
@@ -46,11 +41,11 @@ cudaError_t launch_decode_append(int B, int64_t max_len, const int64_t* L_host, 
 cudaError_t launch_decode_indexer(int B, int64_t max_len, int64_t max_L, const int64_t* L_dev,
                                   const uint16_t* kidx_cache, const uint16_t* qidx_ring, const uint16_t* w_ring,
                                   float* S, int64_t ld, float scale, cudaStream_t s);
-cudaError_t launch_decode_attn(int B, int64_t max_len, const int64_t* L_dev, const uint16_t* q_rot,
-                               const uint16_t* k_cache, const uint16_t* v_cache, const int32_t* sel,
-                               const int32_t* cnt, int budget, int n_split, float scale_log2, float* part_o,
-                               float* part_lse, cudaStream_t s);
-cudaError_t launch_decode_combine(int B, int n_split, const float* part_o, const float* part_lse, uint16_t* out,
-                                  float* lse, cudaStream_t s);
+// Decode attention for B sequences (one new token each, rotated queries
+// q_rot [B][24][256]): the tcgen05 attention kernel over the cached K / V.
+cudaError_t launch_decode_attn_tc(int B, int64_t max_len, const int64_t* L_dev, const uint16_t* q_rot,
+                                  const uint16_t* k_cache, const uint16_t* v_cache, const int32_t* sel,
+                                  const int32_t* cnt, int budget, float scale_log2, uint16_t* out, float* lse,
+                                  uint32_t* err, int num_sms, cudaStream_t stream);
 
 }  // namespace qsa

@@ -163,7 +163,7 @@ qsa_status qsa_decode_workspace_size(const qsa_params* p, int32_t B, int64_t max
  * until the process exits.  Nothing is allocated by this call.
  *   - Sizes whose qsa_decode_workspace_size exceeds 64 MiB are rejected with
  *     QSA_ERR_WORKSPACE_TOO_SMALL before any launch (64 sequences at 256K
- *     context need about 43 MiB).
+ *     context need about 17 MiB).
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) for that device; make that first call before
  *     any stream capture.
@@ -199,8 +199,7 @@ enum {
   QSA_KERNEL_ATTENTION = 5,
   QSA_KERNEL_DECODE_APPEND = 6,
   QSA_KERNEL_DECODE_INDEXER = 7,
-  QSA_KERNEL_DECODE_ATTENTION = 8,
-  QSA_KERNEL_DECODE_COMBINE = 9
+  QSA_KERNEL_DECODE_ATTENTION = 8
 };
 qsa_status qsa_trace_begin(int32_t capacity);
 qsa_status qsa_trace_end(int32_t* kernel_ids, float* ms, int32_t capacity, int32_t* n_out);
