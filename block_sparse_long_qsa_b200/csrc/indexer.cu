@@ -162,9 +162,15 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
           wv[4 * u + 0] = bf16lo(raw.x); wv[4 * u + 1] = bf16hi(raw.x);
           wv[4 * u + 2] = bf16lo(raw.y); wv[4 * u + 3] = bf16hi(raw.y);
         }
+        // stored as token pairs: pair p holds {w(2p, h), w(2p+1, h)} for h = 0..3
         float4* dst = reinterpret_cast<float4*>(sWf + 16 * lane);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) dst[u] = make_float4(wv[4 * u], wv[4 * u + 1], wv[4 * u + 2], wv[4 * u + 3]);
+        for (int pr = 0; pr < 2; ++pr) {
+          const float* a0 = wv + 8 * pr;        // token 4*lane + 2*pr
+          const float* a1 = a0 + 4;             // token 4*lane + 2*pr + 1
+          dst[2 * pr] = make_float4(a0[0], a1[0], a0[1], a1[1]);
+          dst[2 * pr + 1] = make_float4(a0[2], a1[2], a0[3], a1[3]);
+        }
         __syncwarp();
         if (lane == 0) {
           mbar_arrive_expect_tx(qfull, Q_BYTES);
@@ -275,16 +281,25 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             for (int half_blk = 0; half_blk < 2; ++half_blk) {
               float sc[4];
 #pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const int tl = 8 * c + 4 * half_blk + u;    // token index within the 32 columns
-                const float4 wv = *reinterpret_cast<const float4*>(wrow + 4 * tl);
-                const float* x = &v[c][4 * (4 * half_blk + u)];
-                float s = wv.x * fmaxf(x[0], 0.f);
-                s = fmaf(wv.y, fmaxf(x[1], 0.f), s);
-                s = fmaf(wv.z, fmaxf(x[2], 0.f), s);
-                s = fmaf(wv.w, fmaxf(x[3], 0.f), s);
-                if (masked) s = (j <= t_first + tl) ? s : 0.f;
-                sc[u] = s;
+              for (int pr = 0; pr < 2; ++pr) {
+                // tokens tl and tl+1 at once: packed f32x2 multiply-adds over the 4 heads
+                const int tl = 8 * c + 4 * half_blk + 2 * pr;   // token index within the 32 columns
+                const float* x0 = &v[c][4 * (tl & 7)];
+                const float* x1 = x0 + 4;
+                const float4 wa = *reinterpret_cast<const float4*>(wrow + 4 * tl);       // heads 0, 1
+                const float4 wb = *reinterpret_cast<const float4*>(wrow + 4 * tl + 4);   // heads 2, 3
+                uint64_t acc = mul2(pk2(fmaxf(x0[0], 0.f), fmaxf(x1[0], 0.f)), pk2(wa.x, wa.y));
+                acc = fma2(pk2(fmaxf(x0[1], 0.f), fmaxf(x1[1], 0.f)), pk2(wa.z, wa.w), acc);
+                acc = fma2(pk2(fmaxf(x0[2], 0.f), fmaxf(x1[2], 0.f)), pk2(wb.x, wb.y), acc);
+                acc = fma2(pk2(fmaxf(x0[3], 0.f), fmaxf(x1[3], 0.f)), pk2(wb.z, wb.w), acc);
+                float s0, s1;
+                upk2(acc, s0, s1);
+                if (masked) {
+                  s0 = (j <= t_first + tl) ? s0 : 0.f;
+                  s1 = (j <= t_first + tl + 1) ? s1 : 0.f;
+                }
+                sc[2 * pr] = s0;
+                sc[2 * pr + 1] = s1;
               }
               m[2 * c + half_blk] = fmaxf(max3f(sc[0], sc[1], sc[2]), sc[3]);
             }

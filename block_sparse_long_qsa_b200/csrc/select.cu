@@ -126,7 +126,7 @@ __device__ __forceinline__ uint32_t block_excl_count(bool flag, const SelSmem& s
   return before + in_warp;
 }
 
-__global__ void __launch_bounds__(THREADS)
+__global__ void __launch_bounds__(THREADS, 3)
 select_kernel(const float* __restrict__ S, int64_t ld, int64_t qb_begin, int64_t n_rows,
               const int64_t* __restrict__ row_qb, int budget, int32_t* __restrict__ sel, int32_t* __restrict__ cnt,
               uint32_t* err) {
@@ -180,21 +180,37 @@ select_kernel(const float* __restrict__ S, int64_t ld, int64_t qb_begin, int64_t
       // 2. filter pass: keep key >= tau0 (row start is 16-byte aligned: ld % 4 == 0)
       const float4* row4 = reinterpret_cast<const float4*>(row);
       const int64_t m4 = (m + 3) >> 2;
-      for (int64_t i4 = tid; i4 - tid < m4; i4 += blockDim.x) {
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (i4 < m4) v = row4[i4];
-        const float vals[4] = {v.x, v.y, v.z, v.w};
+      // UNROLL independent 16-byte loads per thread per iteration keep enough
+      // bytes in flight to stream the row at HBM speed
+      constexpr int UNROLL = 4;
+      const int64_t stride4 = (int64_t)blockDim.x * UNROLL;
+      for (int64_t base4 = 0; base4 < m4; base4 += stride4) {
+        float4 v[UNROLL];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int64_t idx = 4 * i4 + q;
-          const bool pass = idx < m && key_of(vals[q]) >= tau0;
-          const uint32_t ball = __ballot_sync(0xffffffffu, pass);
-          if (ball) {
-            uint32_t base = 0;
-            if (lane == 0) base = atomicAdd(&sm.misc[2], (uint32_t)__popc(ball));
-            base = __shfl_sync(0xffffffffu, base, 0);
-            const uint32_t pos = base + __popc(ball & ((1u << lane) - 1u));
-            if (pass && pos < (uint32_t)cap) { sm.ckey[pos] = key_of(vals[q]); sm.cidx[pos] = (int32_t)idx; }
+        for (int u = 0; u < UNROLL; ++u) {
+          const int64_t i4 = base4 + (int64_t)u * blockDim.x + tid;
+          v[u] = i4 < m4 ? __ldcs(row4 + i4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+          const int64_t i4 = base4 + (int64_t)u * blockDim.x + tid;
+          const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+          bool any = false;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) any |= (4 * i4 + q < m) && key_of(vals[q]) >= tau0;
+          if (!__any_sync(0xffffffffu, any)) continue;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int64_t idx = 4 * i4 + q;
+            const bool pass = idx < m && key_of(vals[q]) >= tau0;
+            const uint32_t ball = __ballot_sync(0xffffffffu, pass);
+            if (ball) {
+              uint32_t base = 0;
+              if (lane == 0) base = atomicAdd(&sm.misc[2], (uint32_t)__popc(ball));
+              base = __shfl_sync(0xffffffffu, base, 0);
+              const uint32_t pos = base + __popc(ball & ((1u << lane) - 1u));
+              if (pass && pos < (uint32_t)cap) { sm.ckey[pos] = key_of(vals[q]); sm.cidx[pos] = (int32_t)idx; }
+            }
           }
         }
       }
