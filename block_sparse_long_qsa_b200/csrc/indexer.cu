@@ -8,7 +8,7 @@
 // 어텐션", eq. I_ib: ReLU of the per-head similarity, summed over the 4
 // indexer heads; block-causal scoring of r = 4 token micro-blocks.)
 //
-// Design (one persistent CTA per SM, 320 threads):
+// Design (one persistent CTA per SM, 576 threads):
 //   * A = 128 keys x 128 dims (K-major, TMA, 128B swizzle), B = 64 query tokens
 //     x 4 heads = 256 rows x 128 dims; D = A B^T is 128 x 256 fp32 in TMEM, so a
 //     TMEM lane is one key and the 4 head values of one token sit in 4
@@ -21,8 +21,9 @@
 //     split evenly across CTAs in query-major order, so every CTA gets the
 //     same number of MMAs whatever the chunk shape.
 //   * warp 0: producer (3-stage TMA key ring, TMA Q tile, head weights); warp 1: TMEM
-//     allocation and the single MMA-issuing thread; warps 2-9: epilogue
-//     (tcgen05.ld -> ReLU, head weights, block max -> fp32 scores).
+//     allocation and the single MMA-issuing thread; warps 2-17: epilogue,
+//     8 warps per TMEM accumulator (tcgen05.ld -> ReLU, head weights, block
+//     max -> fp32 scores), each 32-column load in flight behind the previous chunk.
 //   * Every mbarrier wait is bounded; on timeout the CTA records
 //     QSA_ERR_DEVICE_TIMEOUT, drains and exits.
 #include "qsa_device.cuh"
@@ -34,7 +35,7 @@ namespace {
 constexpr int QT = 128;                 // query tokens per tile
 constexpr int KT = 128;                 // keys per tile
 constexpr int STAGES = 3;
-constexpr int THREADS = 320;
+constexpr int THREADS = 576;
 constexpr uint32_t Q_SUB_BYTES = 256 * 128;              // 256 rows x 64 bf16
 constexpr uint32_t Q_BYTES = 4 * Q_SUB_BYTES;            // [half][k-chunk]
 constexpr uint32_t K_SUB_BYTES = 128 * 128;              // 128 rows x 64 bf16
@@ -125,7 +126,7 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     mbar_init(qfull, 1);
-    mbar_init(qempty, 1 + 8);
+    mbar_init(qempty, 1 + 16);
     for (int h = 0; h < 2; ++h) { mbar_init(&accfull[h], 1); mbar_init(&accempty[h], 8); }
     mbar_init(done, 1);
     *abort_flag = 0;
@@ -234,13 +235,17 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     }
   } else {
     // ----------------------------------------------------------- epilogue
-    const int e = warp - 2;                 // 0..7
+    // Two groups of 8 warps, one per TMEM accumulator: group hf drains half hf
+    // of every unit while the tensor core fills the other half.
+    const int e = warp - 2;                 // 0..15
+    const int hf = e >> 3;                  // accumulator this warp drains
     const int quad = warp & 3;              // TMEM lanes 32*quad .. +31
-    const int cgrp = e >> 2;                // column group: tokens [32*cgrp, +32) of a half
+    const int cgrp = (e >> 2) & 1;          // column group: tokens [32*cgrp, +32) of a half
     const uint32_t lane_addr = (uint32_t)(32 * quad) << 16;
     Iter it; it.begin(&sch, u0, u1);
     uint32_t qcount = 0;
-    uint32_t acc_use[2] = {0, 0};
+    uint32_t acc_use = 0;
+    const float* wrow = sW + (64 * hf + 32 * cgrp) * 4;
     for (; it.valid(); it.next()) {
       if (it.first_of_tile(u0)) {
         if (!__all_sync(0xffffffffu, mbar_wait(qfull, qcount & 1, abort_flag, err))) break;
@@ -250,87 +255,85 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
       const int64_t qb_tile = qb_begin + (QT / 4) * it.tile;
       const int64_t j = KT * it.kt + 32 * quad + lane;       // this thread's key
       const int64_t kb = j >> 2;
-      bool ok = true;
-      for (int hf = 0; hf < 2; ++hf) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&accfull[hf], acc_use[hf] & 1, abort_flag, err))) {
-          ok = false;
-          break;
-        }
-        ++acc_use[hf];
-        tc_fence_after();
-        const int64_t t_first = t_tile + 64 * hf + 32 * cgrp;  // first token of this thread's columns
-        const int64_t qb_first = qb_tile + 16 * hf + 8 * cgrp;
-        const int64_t kt_last_key = KT * it.kt + KT - 1;
-        // skip when every key block of this warp lies after every query block of its columns
-        const bool live = (KT * it.kt + 32 * quad) <= (t_first + 31) && qb_first < qb_end;
+      if (!__all_sync(0xffffffffu, mbar_wait(&accfull[hf], acc_use & 1, abort_flag, err))) break;
+      ++acc_use;
+      tc_fence_after();
+      const int64_t t_first = t_tile + 64 * hf + 32 * cgrp;  // first token of this thread's columns
+      const int64_t qb_first = qb_tile + 16 * hf + 8 * cgrp;
+      const int64_t kt_last_key = KT * it.kt + KT - 1;
+      // skip when every key block of this warp lies after every query block of its columns
+      const bool live = (KT * it.kt + 32 * quad) <= (t_first + 31) && qb_first < qb_end;
+      if (live) {
+        const bool masked = kt_last_key > t_first;
         float m[8];
-        if (live) {
-          float v[4][32];
-          const uint32_t base = tmem + lane_addr + hf * 256 + 128 * cgrp;
+        // 8 tokens (32 columns) of this key's row -> the maxima of query blocks 2c, 2c+1
+        auto chunk = [&](const float (&v)[32], int c) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld32(base + 32 * c, v[c]);
-          tmem_ld_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&accempty[hf]);
-          const bool masked = kt_last_key > t_first;
-          const float* wrow = sW + (64 * hf + 32 * cgrp) * 4;
+          for (int half_blk = 0; half_blk < 2; ++half_blk) {
+            float sc[4];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-#pragma unroll
-            for (int half_blk = 0; half_blk < 2; ++half_blk) {
-              float sc[4];
-#pragma unroll
-              for (int pr = 0; pr < 2; ++pr) {
-                // tokens tl and tl+1 at once: packed f32x2 multiply-adds over the 4 heads
-                const int tl = 8 * c + 4 * half_blk + 2 * pr;   // token index within the 32 columns
-                const float* x0 = &v[c][4 * (tl & 7)];
-                const float* x1 = x0 + 4;
-                const float4 wa = *reinterpret_cast<const float4*>(wrow + 4 * tl);       // heads 0, 1
-                const float4 wb = *reinterpret_cast<const float4*>(wrow + 4 * tl + 4);   // heads 2, 3
-                uint64_t acc = mul2(pk2(fmaxf(x0[0], 0.f), fmaxf(x1[0], 0.f)), pk2(wa.x, wa.y));
-                acc = fma2(pk2(fmaxf(x0[1], 0.f), fmaxf(x1[1], 0.f)), pk2(wa.z, wa.w), acc);
-                acc = fma2(pk2(fmaxf(x0[2], 0.f), fmaxf(x1[2], 0.f)), pk2(wb.x, wb.y), acc);
-                acc = fma2(pk2(fmaxf(x0[3], 0.f), fmaxf(x1[3], 0.f)), pk2(wb.z, wb.w), acc);
-                float s0, s1;
-                upk2(acc, s0, s1);
-                if (masked) {
-                  s0 = (j <= t_first + tl) ? s0 : 0.f;
-                  s1 = (j <= t_first + tl + 1) ? s1 : 0.f;
-                }
-                sc[2 * pr] = s0;
-                sc[2 * pr + 1] = s1;
+            for (int pr = 0; pr < 2; ++pr) {
+              // tokens tl and tl+1 at once: packed f32x2 multiply-adds over the 4 heads
+              const int tl = 8 * c + 4 * half_blk + 2 * pr;   // token index within the 32 columns
+              const float* x0 = &v[4 * (tl & 7)];
+              const float* x1 = x0 + 4;
+              const float4 wa = *reinterpret_cast<const float4*>(wrow + 4 * tl);       // heads 0, 1
+              const float4 wb = *reinterpret_cast<const float4*>(wrow + 4 * tl + 4);   // heads 2, 3
+              uint64_t acc = mul2(pk2(fmaxf(x0[0], 0.f), fmaxf(x1[0], 0.f)), pk2(wa.x, wa.y));
+              acc = fma2(pk2(fmaxf(x0[1], 0.f), fmaxf(x1[1], 0.f)), pk2(wa.z, wa.w), acc);
+              acc = fma2(pk2(fmaxf(x0[2], 0.f), fmaxf(x1[2], 0.f)), pk2(wb.x, wb.y), acc);
+              acc = fma2(pk2(fmaxf(x0[3], 0.f), fmaxf(x1[3], 0.f)), pk2(wb.z, wb.w), acc);
+              float s0, s1;
+              upk2(acc, s0, s1);
+              if (masked) {
+                s0 = (j <= t_first + tl) ? s0 : 0.f;
+                s1 = (j <= t_first + tl + 1) ? s1 : 0.f;
               }
-              m[2 * c + half_blk] = fmaxf(max3f(sc[0], sc[1], sc[2]), sc[3]);
+              sc[2 * pr] = s0;
+              sc[2 * pr + 1] = s1;
             }
+            m[2 * c + half_blk] = fmaxf(max3f(sc[0], sc[1], sc[2]), sc[3]);
           }
-        } else {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&accempty[hf]);
+        };
+        // four 32-column loads, each in flight while the previous chunk is scored
+        const uint32_t base = tmem + lane_addr + hf * 256 + 128 * cgrp;
+        float va[32], vb[32];
+        tmem_ld32(base, va);
+        tmem_ld_wait(va);
+        tmem_ld32(base + 32, vb);
+        chunk(va, 0);
+        tmem_ld_wait(vb);
+        tmem_ld32(base + 64, va);
+        chunk(vb, 1);
+        tmem_ld_wait(va);
+        tmem_ld32(base + 96, vb);
+        chunk(va, 2);
+        tmem_ld_wait(vb);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&accempty[hf]);
+        chunk(vb, 3);
 #pragma unroll
-          for (int b = 0; b < 8; ++b) m[b] = 0.f;
+        for (int b = 0; b < 8; ++b) {
+          m[b] = fmaxf(m[b], __shfl_xor_sync(0xffffffffu, m[b], 1));
+          m[b] = fmaxf(m[b], __shfl_xor_sync(0xffffffffu, m[b], 2));
         }
-        if (live) {
+        const int r = lane & 3;
 #pragma unroll
-          for (int b = 0; b < 8; ++b) {
-            m[b] = fmaxf(m[b], __shfl_xor_sync(0xffffffffu, m[b], 1));
-            m[b] = fmaxf(m[b], __shfl_xor_sync(0xffffffffu, m[b], 2));
-          }
-          const int r = lane & 3;
+        for (int rr = 0; rr < 2; ++rr) {
+          const int b = r + 4 * rr;
+          const int64_t qb = qb_first + b;
+          // select m[b] without dynamic register indexing
+          float val = m[0];
 #pragma unroll
-          for (int rr = 0; rr < 2; ++rr) {
-            const int b = r + 4 * rr;
-            const int64_t qb = qb_first + b;
-            // select m[b] without dynamic register indexing
-            float val = m[0];
-#pragma unroll
-            for (int bb = 1; bb < 8; ++bb) val = (bb == b) ? m[bb] : val;
-            if (qb < qb_end && kb <= qb) S[(qb - qb_begin) * ld + kb] = val * scale;
-          }
+          for (int bb = 1; bb < 8; ++bb) val = (bb == b) ? m[bb] : val;
+          if (qb < qb_end && kb <= qb) S[(qb - qb_begin) * ld + kb] = val * scale;
         }
+      } else {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&accempty[hf]);
       }
-      if (!ok) break;
       if (it.tile_ends_here()) {
         __syncwarp();
         if (lane == 0) mbar_arrive(qempty);
