@@ -163,14 +163,16 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
           wv[4 * u + 0] = bf16lo(raw.x); wv[4 * u + 1] = bf16hi(raw.x);
           wv[4 * u + 2] = bf16lo(raw.y); wv[4 * u + 3] = bf16hi(raw.y);
         }
-        // stored as token pairs: pair p holds {w(2p, h), w(2p+1, h)} for h = 0..3
+        // stored as token pairs: pair p holds {w(2p, h), w(2p+1, h)} for h = 0..3;
+        // heads 2 and 3 are scaled by 2^64 to pair with relu_scaled() in the epilogue
         float4* dst = reinterpret_cast<float4*>(sWf + 16 * lane);
 #pragma unroll
         for (int pr = 0; pr < 2; ++pr) {
           const float* a0 = wv + 8 * pr;        // token 4*lane + 2*pr
           const float* a1 = a0 + 4;             // token 4*lane + 2*pr + 1
           dst[2 * pr] = make_float4(a0[0], a1[0], a0[1], a1[1]);
-          dst[2 * pr + 1] = make_float4(a0[2], a1[2], a0[3], a1[3]);
+          dst[2 * pr + 1] = make_float4(a0[2] * kReluSatScale, a1[2] * kReluSatScale, a0[3] * kReluSatScale,
+                                        a1[3] * kReluSatScale);
         }
         __syncwarp();
         if (lane == 0) {
@@ -273,16 +275,18 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             float sc[4];
 #pragma unroll
             for (int pr = 0; pr < 2; ++pr) {
-              // tokens tl and tl+1 at once: packed f32x2 multiply-adds over the 4 heads
+              // tokens tl and tl+1 at once: packed f32x2 multiply-adds over the 4 heads.
+              // The ReLU of heads 0, 1 runs on the ALU (max), that of heads 2, 3 on the
+              // FMA pipe (saturating multiply by 2^-64, undone by the scaled weights).
               const int tl = 8 * c + 4 * half_blk + 2 * pr;   // token index within the 32 columns
               const float* x0 = &v[4 * (tl & 7)];
               const float* x1 = x0 + 4;
               const float4 wa = *reinterpret_cast<const float4*>(wrow + 4 * tl);       // heads 0, 1
-              const float4 wb = *reinterpret_cast<const float4*>(wrow + 4 * tl + 4);   // heads 2, 3
+              const float4 wb = *reinterpret_cast<const float4*>(wrow + 4 * tl + 4);   // heads 2, 3 (x 2^64)
               uint64_t acc = mul2(pk2(fmaxf(x0[0], 0.f), fmaxf(x1[0], 0.f)), pk2(wa.x, wa.y));
               acc = fma2(pk2(fmaxf(x0[1], 0.f), fmaxf(x1[1], 0.f)), pk2(wa.z, wa.w), acc);
-              acc = fma2(pk2(fmaxf(x0[2], 0.f), fmaxf(x1[2], 0.f)), pk2(wb.x, wb.y), acc);
-              acc = fma2(pk2(fmaxf(x0[3], 0.f), fmaxf(x1[3], 0.f)), pk2(wb.z, wb.w), acc);
+              acc = fma2(pk2(relu_scaled(x0[2]), relu_scaled(x1[2])), pk2(wb.x, wb.y), acc);
+              acc = fma2(pk2(relu_scaled(x0[3]), relu_scaled(x1[3])), pk2(wb.z, wb.w), acc);
               float s0, s1;
               upk2(acc, s0, s1);
               if (masked) {
@@ -313,20 +317,23 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         __syncwarp();
         if (lane == 0) mbar_arrive(&accempty[hf]);
         chunk(vb, 3);
+        // max over the 4 keys of the key block (lanes 4k .. 4k+3) as a transposing
+        // butterfly: after the two steps lane (a = bit 0, b = bit 1) holds the
+        // maxima of query blocks 4a + 2b and 4a + 2b + 1.
+        const bool la = (lane & 1) != 0, lb = (lane & 2) != 0;
+        float n4[4];
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {
-          m[b] = fmaxf(m[b], __shfl_xor_sync(0xffffffffu, m[b], 1));
-          m[b] = fmaxf(m[b], __shfl_xor_sync(0xffffffffu, m[b], 2));
+        for (int i = 0; i < 4; ++i) {
+          const float send = la ? m[i] : m[i + 4];
+          const float keep = la ? m[i + 4] : m[i];
+          n4[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 1));
         }
-        const int r = lane & 3;
 #pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          const int b = r + 4 * rr;
-          const int64_t qb = qb_first + b;
-          // select m[b] without dynamic register indexing
-          float val = m[0];
-#pragma unroll
-          for (int bb = 1; bb < 8; ++bb) val = (bb == b) ? m[bb] : val;
+        for (int i = 0; i < 2; ++i) {
+          const float send = lb ? n4[i] : n4[i + 2];
+          const float keep = lb ? n4[i + 2] : n4[i];
+          const float val = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
+          const int64_t qb = qb_first + (la ? 4 : 0) + (lb ? 2 : 0) + i;
           if (qb < qb_end && kb <= qb) S[(qb - qb_begin) * ld + kb] = val * scale;
         }
       } else {

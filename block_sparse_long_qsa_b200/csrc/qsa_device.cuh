@@ -221,6 +221,17 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
+// ReLU on the FMA pipe instead of the ALU: min(max(x * 2^-64, 0), 1).  For
+// x <= 2^64 this is ReLU(x) * 2^-64, exact whenever x * 2^-64 is a normal float
+// (x >= 2^-62; below that the subnormal result carries an absolute error under
+// 2^-149).  A weight scaled by 2^64 (also exact) undoes the factor inside a
+// fused multiply-add, so w * ReLU(x) keeps fp32 FMA rounding.
+constexpr float kReluSatScale = 18446744073709551616.0f;   // 2^64
+__device__ __forceinline__ float relu_scaled(float x) {
+  float r;
+  asm("mul.rn.sat.f32 %0, %1, 0f1F800000;" : "=f"(r) : "f"(x));   // 0f1F800000 = 2^-64
+  return r;
+}
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float m;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
