@@ -173,15 +173,14 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 // Same wait, with the 32 registers of one tcgen05.ld as in/out operands, so no use
 // of them can be scheduled above the wait (lets a load be in flight behind other work).
+// No memory clobber: shared / global accesses may move across it.
 __device__ __forceinline__ void tmem_ld_wait(float (&v)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;"
                : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]), "+f"(v[7]),
                  "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]), "+f"(v[14]),
                  "+f"(v[15]), "+f"(v[16]), "+f"(v[17]), "+f"(v[18]), "+f"(v[19]), "+f"(v[20]), "+f"(v[21]),
                  "+f"(v[22]), "+f"(v[23]), "+f"(v[24]), "+f"(v[25]), "+f"(v[26]), "+f"(v[27]), "+f"(v[28]),
-                 "+f"(v[29]), "+f"(v[30]), "+f"(v[31])
-               :
-               : "memory");
+                 "+f"(v[29]), "+f"(v[30]), "+f"(v[31]));
 }
 
 // Named barrier among `nthreads` threads (multiple of 32).
