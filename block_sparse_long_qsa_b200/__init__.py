@@ -28,7 +28,7 @@ EXPORTED = ["qsa_default_params", "qsa_status_string", "qsa_last_error", "qsa_in
             "qsa_decode_noalloc"]
 
 KERNEL_NAMES = {1: "rope_table", 2: "rope_k", 3: "indexer", 4: "select", 5: "attention", 6: "decode_append",
-                7: "decode_indexer", 8: "decode_attention"}
+                7: "decode_indexer", 8: "decode_attention", 9: "decode_combine"}
 
 
 class QSAError(RuntimeError):

@@ -3,6 +3,7 @@
 // validates on the host before launching anything and returns a qsa_status.
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -355,9 +356,11 @@ qsa_status qsa_prefill(const qsa_params* p, int64_t T, int64_t pos0, const uint1
 // ------------------------------------------------------------------ decode
 namespace {
 struct DecodeLayout {
-  size_t Ls, qbs, S, sel, cnt, q_rot, total;
+  size_t Ls, qbs, S, sel, cnt, q_rot, part_o, part_lse, total;
   int64_t ld;
 };
+// Split-KV ranges per (sequence, KV head): at most this many.
+constexpr int DECODE_MAX_SPLIT = 16;
 DecodeLayout decode_layout(int B, int64_t max_len, int budget) {
   DecodeLayout L;
   L.ld = round4(max_len / 4 + 1);
@@ -368,8 +371,34 @@ DecodeLayout decode_layout(int B, int64_t max_len, int budget) {
   L.sel = off; off = align_up(off + (size_t)B * budget * 4);
   L.cnt = off; off = align_up(off + (size_t)B * 4);
   L.q_rot = off; off = align_up(off + (size_t)B * 24 * 256 * 2);
+  L.part_o = off; off = align_up(off + (size_t)B * 2 * DECODE_MAX_SPLIT * 12 * 256 * 4);
+  L.part_lse = off; off = align_up(off + (size_t)B * 2 * DECODE_MAX_SPLIT * 12 * 4);
   L.total = off;
   return L;
+}
+// Number of split-KV ranges: the one that minimises the most work any SM
+// does, in tiles: (items it runs) x (tiles per item + 1.5 for the per-item
+// overhead), plus 1 for the combine when there is more than one range, given
+// the largest selection of the batch (measured on B200: at 64 sequences x 32
+// tiles one range per (sequence, KV head) is best).  The environment variable
+// QSA_DECODE_SPLITS (1 .. 16) overrides the choice.
+int decode_splits(int B, int64_t max_L, int budget, int num_sms) {
+  if (const char* e = std::getenv("QSA_DECODE_SPLITS")) {
+    const int v = std::atoi(e);
+    if (v >= 1 && v <= DECODE_MAX_SPLIT) return v;
+  }
+  int64_t cnt = max_L / 4 + 1;
+  if (cnt > budget) cnt = budget;
+  const int nt = (int)((cnt + 15) / 16);
+  int best = 1;
+  double best_cost = 1e300;
+  for (int sp = 1; sp <= DECODE_MAX_SPLIT && sp <= nt; ++sp) {
+    const int64_t items = 2 * (int64_t)B * sp;
+    const double waves = (double)((items + num_sms - 1) / num_sms);
+    const double cost = waves * ((nt + sp - 1) / sp + 1.5) + (sp > 1 ? 1.0 : 0.0);
+    if (cost < best_cost - 1e-9) { best_cost = cost; best = sp; }
+  }
+  return best;
 }
 }  // namespace
 
@@ -439,9 +468,17 @@ qsa_status qsa_decode(const qsa_params* p, int32_t B, int64_t max_len, const int
        }))) != QSA_OK)
     return st;
   const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
-  return from_cuda(traced(QSA_KERNEL_DECODE_ATTENTION, s, [&] {
-    return qsa::launch_decode_attn_tc(B, max_len, Ls, q_rot, k_cache, v_cache, sel, cnt, budget, scale_log2, out,
-                                      lse_out, err, di.num_sms, s);
+  const int n_split = decode_splits(B, max_L, budget, di.num_sms);
+  float* part_o = reinterpret_cast<float*>(base + L.part_o);
+  float* part_lse = reinterpret_cast<float*>(base + L.part_lse);
+  if ((st = from_cuda(traced(QSA_KERNEL_DECODE_ATTENTION, s, [&] {
+         return qsa::launch_decode_attn_tc(B, max_len, Ls, q_rot, k_cache, v_cache, sel, cnt, budget, scale_log2,
+                                           n_split, part_o, part_lse, out, lse_out, err, di.num_sms, s);
+       }))) != QSA_OK)
+    return st;
+  if (n_split == 1) return QSA_OK;
+  return from_cuda(traced(QSA_KERNEL_DECODE_COMBINE, s, [&] {
+    return qsa::launch_decode_combine(B, part_o, part_lse, cnt, n_split, out, lse_out, s);
   }));
 }
 

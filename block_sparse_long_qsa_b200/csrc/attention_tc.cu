@@ -118,21 +118,42 @@ struct TcArgs {
   // [B][max_len][2][256], out / lse [B][24][...], one query token per sequence
   const int64_t* Ls;        // [B] position of the new token
   int64_t max_len;
+  // split-KV decode: each (sequence, KV head) is cut into n_split ranges of
+  // whole tiles; with n_split > 1 every range writes its normalised O (fp32)
+  // and its lse in base 2 to part_o [B][2][n_split][12][256] and
+  // part_lse [B][2][n_split][12], merged afterwards by the combine kernel
+  int n_split;
+  float* part_o;
+  float* part_lse;
 };
 
-// One work item = (query block, KV head) for prefill, (sequence, KV head) for decode.
+// One work item = (query block, KV head) for prefill, (sequence, KV head,
+// split) for decode: the tiles [tile0, tile0 + n_tiles) of the row's selection
+// (16 blocks per tile, nt_total tiles in all).  Items with no tile are skipped
+// by every role alike.
 template <bool DEC>
 struct Item {
   int64_t row;              // selection row
   int g;                    // KV head
+  int split;
+  int cnt;                  // selected blocks of the row
+  int nt_total, tile0, n_tiles;
   int64_t qb;               // query block
   int64_t t0;               // position of the item's first query token
   int64_t t_last;           // last key position any of its rows may read
   const uint16_t* kb;       // rotated keys of this sequence
   const uint16_t* vb;
   __device__ __forceinline__ Item(const TcArgs& a, int64_t w) {
-    row = w >> 1;
+    const int64_t rs = w >> 1;
     g = (int)(w & 1);
+    row = DEC ? rs / a.n_split : rs;
+    split = DEC ? (int)(rs % a.n_split) : 0;
+    cnt = a.cnt[row];
+    nt_total = (cnt + 15) / 16;
+    const int per = DEC ? (nt_total + a.n_split - 1) / a.n_split : nt_total;
+    tile0 = split * per;
+    const int rest = nt_total - tile0;
+    n_tiles = rest < 0 ? 0 : (rest < per ? rest : per);
     if (DEC) {
       const int64_t L = a.Ls[row];
       qb = L >> 2;
@@ -190,7 +211,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int64_t n_items = 2 * a.n_qb;
+  const int64_t n_items = 2 * a.n_qb * (DEC ? a.n_split : 1);
 
   if (warp < 4) {
     // ---------------------------------------------------------------- loaders
@@ -198,11 +219,11 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
     uint32_t ephase = 1;
     uint32_t items_done = 0;
     bool ok = true;
-    for (int64_t w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++items_done) {
+    for (int64_t w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
       const Item<DEC> it(a, w);
+      if (it.n_tiles == 0) continue;
       const int g = it.g;
-      const int cnt = a.cnt[it.row];
-      const int32_t* sel = a.sel + it.row * a.budget;
+      const int32_t* sel = a.sel + it.row * a.budget + 16 * it.tile0;
       // Q tile; prefill rotates dims 0..63 (pairs i, i+32) on the way in,
       // decode queries arrive rotated
       if (items_done > 0 && !mbar_wait(q_empty, (items_done - 1) & 1, abort_flag, a.err)) { ok = false; break; }
@@ -240,7 +261,8 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
       fence_proxy_async();
       mbar_arrive(q_full);
       // K / V tiles
-      const int n_tiles = (cnt + 15) / 16;
+      const int n_tiles = it.n_tiles;
+      const int nsel = it.cnt - 16 * it.tile0;     // selected blocks from this item's first tile on
       const int64_t t_last = it.t_last;
       for (int i = 0; i < n_tiles; ++i) {
         if (!mbar_wait(&kv_empty[stage], ephase, abort_flag, a.err)) { ok = false; break; }
@@ -251,7 +273,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
         const int w4 = tid >> 5, c32 = tid & 31;
         int32_t kbv[16];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) kbv[k] = 16 * i + k < cnt ? __ldg(sel + 16 * i + k) : -1;
+        for (int k = 0; k < 16; ++k) kbv[k] = 16 * i + k < nsel ? __ldg(sel + 16 * i + k) : -1;
         const uint32_t dst0 = base + (c32 >> 3) * CHUNK_KV;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
@@ -269,6 +291,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
                      : "memory");
         if (++stage == NSTAGE) { stage = 0; ephase ^= 1; }
       }
+      ++items_done;
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == 6) {
@@ -281,10 +304,10 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
       uint32_t items_done = 0, s_count = 0, p_count = 0;
       bool ok = true;
       const uint32_t q_base = smem_u32(smem);
-      for (int64_t w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++items_done) {
-        const int64_t row = w >> 1;
-        const int cnt = a.cnt[row];
-        const int n_tiles = (cnt + 15) / 16;
+      for (int64_t w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
+        const Item<DEC> it(a, w);
+        const int n_tiles = it.n_tiles;
+        if (n_tiles == 0) continue;
         if (!mbar_wait(q_full, items_done & 1, abort_flag, a.err)) { ok = false; break; }
         tc_fence_after();
         int pv_stage = stage;           // stage of the tile whose PV is next
@@ -325,7 +348,8 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
           if (++stage == NSTAGE) { stage = 0; fphase ^= 1; }
           if (i >= 1 && !issue_pv(i - 1, false)) { ok = false; break; }
         }
-        if (ok && n_tiles > 0 && !issue_pv(n_tiles - 1, true)) ok = false;
+        if (ok && !issue_pv(n_tiles - 1, true)) ok = false;
+        ++items_done;
       }
       tc_commit(mma_done);
       mbar_wait(mma_done, 0, abort_flag, a.err);
@@ -338,11 +362,12 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     uint32_t items_done = 0, s_count = 0, pv_count = 0;
     bool ok = true;
-    for (int64_t w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++items_done) {
+    for (int64_t w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
       const Item<DEC> it(a, w);
+      const int n_tiles = it.n_tiles;
+      if (n_tiles == 0) continue;
       const int g = it.g;
-      const int cnt = a.cnt[it.row];
-      const int n_tiles = (cnt + 15) / 16;
+      const int cnt = it.cnt;
       const int64_t t = it.t0 + tok;                  // this row's token position
       const int own_lim = (int)(t & 3);               // last visible token of the own block
       float m_run = -FLT_MAX, l_run = 0.f;
@@ -368,11 +393,12 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
         // block, so every key of a tile before the last one is visible to
         // every row; in the last tile, slots past cnt and the own block's
         // tokens after the row's token are masked.
-        const bool last = i == n_tiles - 1;
+        const int gi = it.tile0 + i;                  // tile index within the row's selection
+        const bool last = gi == it.nt_total - 1;
         if (last) {
 #pragma unroll
           for (int n = 0; n < 64; ++n) {
-            const int blk = 16 * i + (n >> 2);
+            const int blk = 16 * gi + (n >> 2);
             const bool valid = blk < cnt && (blk < cnt - 1 || (n & 3) <= own_lim);
             s[n] = valid ? s[n] : -FLT_MAX;
           }
@@ -434,15 +460,22 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
       ++pv_count;   // the last PV of the item also completed
       tc_fence_after();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      const bool write = row_ok && (DEC || t < a.T) && n_tiles > 0;
+      const bool write = row_ok && (DEC || t < a.T);
       const int64_t orow_idx = (DEC ? it.row : t) * 24 + 12 * g + hh;   // [token or sequence][head]
       uint16_t* orow = a.out + orow_idx * 256;
+      const bool partial = DEC && a.n_split > 1;
+      const int64_t prow = ((it.row * 2 + g) * (int64_t)a.n_split + it.split) * 12 + hh;
 #pragma unroll 1
       for (int c = 0; c < 8; ++c) {
         float o[32];
         tmem_ld32(tmem + lane_off + TM_O + 32 * c, o);
         tmem_ld_wait();
-        if (write) {
+        if (write && partial) {
+          float4* dst = reinterpret_cast<float4*>(a.part_o + prow * 256 + 32 * c);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_float4(o[4 * q] * inv, o[4 * q + 1] * inv, o[4 * q + 2] * inv, o[4 * q + 3] * inv);
+        } else if (write) {
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
           for (int q = 0; q < 4; ++q)
@@ -452,10 +485,12 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
                                 cvt_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
         }
       }
-      if (write && a.lse) a.lse[orow_idx] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+      if (write && partial) a.part_lse[prow] = m_run + log2f(l_run);
+      else if (write && a.lse) a.lse[orow_idx] = (m_run + log2f(l_run)) * 0.69314718055994531f;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(o_empty);
+      ++items_done;
     }
   }
 
@@ -465,6 +500,47 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
+}
+
+constexpr int MAX_SPLIT = 16;
+
+// Split-KV merge, one CTA per (sequence, query head), one thread per dim:
+// the ranges' normalised O weighted by 2^(lse_s - max) and renormalised, and
+// lse = (max + log2 sum) ln 2.  Ranges without tiles are the ones the
+// attention kernel skipped.
+__global__ void __launch_bounds__(256) decode_combine_kernel(const float* __restrict__ part_o,
+                                                             const float* __restrict__ part_lse,
+                                                             const int32_t* __restrict__ cnt, int n_split,
+                                                             uint16_t* __restrict__ out, float* __restrict__ lse) {
+  const int bh = blockIdx.x;                    // sequence * 24 + head
+  const int b = bh / 24, h = bh % 24, g = h / 12, hh = h % 12;
+  const int d = threadIdx.x;
+  const int nt = (cnt[b] + 15) / 16;
+  const int per = (nt + n_split - 1) / n_split;
+  const int ns = per > 0 ? (nt + per - 1) / per : 0;
+  const int64_t row0 = ((int64_t)(b * 2 + g) * n_split) * 12 + hh;
+  // all loads issued before any use (at most MAX_SPLIT ranges)
+  float l2[MAX_SPLIT], ov[MAX_SPLIT];
+#pragma unroll
+  for (int sp = 0; sp < MAX_SPLIT; ++sp) {
+    l2[sp] = sp < ns ? part_lse[row0 + 12 * sp] : -FLT_MAX;
+    ov[sp] = sp < ns ? part_o[(row0 + 12 * sp) * 256 + d] : 0.f;
+  }
+  float mx = -FLT_MAX;
+#pragma unroll
+  for (int sp = 0; sp < MAX_SPLIT; ++sp) mx = fmaxf(mx, l2[sp]);
+  float wsum = 0.f, acc = 0.f;
+#pragma unroll
+  for (int sp = 0; sp < MAX_SPLIT; ++sp) {
+    if (sp < ns) {
+      const float wgt = exp2f(l2[sp] - mx);
+      wsum += wgt;
+      acc = fmaf(wgt, ov[sp], acc);
+    }
+  }
+  const float o = wsum > 0.f ? acc / wsum : 0.f;
+  out[(int64_t)bh * 256 + d] = (uint16_t)f32_to_bf16_bits(o);
+  if (lse && d == 0) lse[bh] = (mx + log2f(wsum)) * 0.69314718055994531f;
 }
 
 template <bool DEC>
@@ -493,20 +569,31 @@ cudaError_t launch_sparse_attn_prefill_tc(int64_t T, const uint16_t* q, const ui
   TcArgs a{};
   a.T = T; a.q = q; a.k_rot = k_rot; a.v = v; a.cs = cs; a.sel = sel; a.cnt = cnt; a.budget = budget;
   a.qb_begin = qb_begin; a.n_qb = qb_end - qb_begin; a.scale_log2 = scale_log2; a.out = out; a.lse = lse;
-  a.err = err;
+  a.err = err; a.n_split = 1;
   return launch_tc<false>(a, 2 * (qb_end - qb_begin), num_sms, stream);
 }
 
 cudaError_t launch_decode_attn_tc(int B, int64_t max_len, const int64_t* L_dev, const uint16_t* q_rot,
                                   const uint16_t* k_cache, const uint16_t* v_cache, const int32_t* sel,
-                                  const int32_t* cnt, int budget, float scale_log2, uint16_t* out, float* lse,
-                                  uint32_t* err, int num_sms, cudaStream_t stream) {
+                                  const int32_t* cnt, int budget, float scale_log2, int n_split, float* part_o,
+                                  float* part_lse, uint16_t* out, float* lse, uint32_t* err, int num_sms,
+                                  cudaStream_t stream) {
   if (B <= 0) return cudaSuccess;
+  if (n_split < 1) return cudaErrorInvalidValue;
   TcArgs a{};
   a.T = INT64_MAX; a.q = q_rot; a.k_rot = k_cache; a.v = v_cache; a.sel = sel; a.cnt = cnt; a.budget = budget;
   a.qb_begin = 0; a.n_qb = B; a.scale_log2 = scale_log2; a.out = out; a.lse = lse; a.err = err;
   a.Ls = L_dev; a.max_len = max_len;
-  return launch_tc<true>(a, 2 * (int64_t)B, num_sms, stream);
+  a.n_split = n_split; a.part_o = part_o; a.part_lse = part_lse;
+  return launch_tc<true>(a, 2 * (int64_t)B * n_split, num_sms, stream);
+}
+
+cudaError_t launch_decode_combine(int B, const float* part_o, const float* part_lse, const int32_t* cnt, int n_split,
+                                  uint16_t* out, float* lse, cudaStream_t stream) {
+  if (B <= 0) return cudaSuccess;
+  if (n_split < 1 || n_split > MAX_SPLIT) return cudaErrorInvalidValue;
+  decode_combine_kernel<<<B * 24, 256, 0, stream>>>(part_o, part_lse, cnt, n_split, out, lse);
+  return cudaGetLastError();
 }
 
 }  // namespace qsa

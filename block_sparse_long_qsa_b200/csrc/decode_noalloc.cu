@@ -21,7 +21,7 @@
 namespace {
 
 // Largest decode scratch this entry point serves (64 MiB: e.g. 64 sequences
-// at 256K context need about 17 MiB).
+// at 256K context need about 41 MiB).
 constexpr size_t NOALLOC_SCRATCH_BYTES = (size_t)64 << 20;
 constexpr int MAX_DEV = 64;
 

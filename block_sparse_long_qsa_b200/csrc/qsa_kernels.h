@@ -43,9 +43,16 @@ cudaError_t launch_decode_indexer(int B, int64_t max_len, int64_t max_L, const i
                                   float* S, int64_t ld, float scale, cudaStream_t s);
 // Decode attention for B sequences (one new token each, rotated queries
 // q_rot [B][24][256]): the tcgen05 attention kernel over the cached K / V.
+// Split-KV decode attention: each (sequence, KV head) is cut into n_split
+// ranges of 16-block tiles.  n_split == 1 writes out / lse directly; otherwise
+// the ranges write part_o [B][2][n_split][12][256] fp32 and part_lse
+// [B][2][n_split][12] (base 2) and launch_decode_combine merges them.
 cudaError_t launch_decode_attn_tc(int B, int64_t max_len, const int64_t* L_dev, const uint16_t* q_rot,
                                   const uint16_t* k_cache, const uint16_t* v_cache, const int32_t* sel,
-                                  const int32_t* cnt, int budget, float scale_log2, uint16_t* out, float* lse,
-                                  uint32_t* err, int num_sms, cudaStream_t stream);
+                                  const int32_t* cnt, int budget, float scale_log2, int n_split, float* part_o,
+                                  float* part_lse, uint16_t* out, float* lse, uint32_t* err, int num_sms,
+                                  cudaStream_t stream);
+cudaError_t launch_decode_combine(int B, const float* part_o, const float* part_lse, const int32_t* cnt, int n_split,
+                                  uint16_t* out, float* lse, cudaStream_t stream);
 
 }  // namespace qsa

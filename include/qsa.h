@@ -145,7 +145,12 @@ qsa_status qsa_prefill_workspace_size(const qsa_params* p, int64_t T, size_t* mi
  * q_new [B][24][256]; k_new, v_new [B][2][256]; q_idx_new [B][4][128];
  * k_idx_new [B][128]; w_new [B][4]  ->  out [B][24][256] bf16;
  * sel_out [B][budget] int32 (nullable), lse_out [B][24] fp32 (nullable).
- * Requires cache_len[b] < max_len, B <= 4096. */
+ * Requires cache_len[b] < max_len, B <= 4096.
+ * Attention is split-KV: each (sequence, KV head) is cut into 1..16 ranges of
+ * whole 16-block tiles, chosen so the batch fills the GPU's SMs; with more
+ * than one range a combine kernel merges the ranges' partial outputs by their
+ * log-sum-exp.  The environment variable QSA_DECODE_SPLITS (1..16) fixes the
+ * number of ranges (read at every call; a test and tuning aid). */
 qsa_status qsa_decode(const qsa_params* p, int32_t B, int64_t max_len, const int64_t* cache_len,
                       uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* qidx_ring,
                       uint16_t* w_ring, const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
@@ -163,7 +168,7 @@ qsa_status qsa_decode_workspace_size(const qsa_params* p, int32_t B, int64_t max
  * until the process exits.  Nothing is allocated by this call.
  *   - Sizes whose qsa_decode_workspace_size exceeds 64 MiB are rejected with
  *     QSA_ERR_WORKSPACE_TOO_SMALL before any launch (64 sequences at 256K
- *     context need about 17 MiB).
+ *     context need about 41 MiB).
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) for that device; make that first call before
  *     any stream capture.
@@ -199,7 +204,8 @@ enum {
   QSA_KERNEL_ATTENTION = 5,
   QSA_KERNEL_DECODE_APPEND = 6,
   QSA_KERNEL_DECODE_INDEXER = 7,
-  QSA_KERNEL_DECODE_ATTENTION = 8
+  QSA_KERNEL_DECODE_ATTENTION = 8,
+  QSA_KERNEL_DECODE_COMBINE = 9
 };
 qsa_status qsa_trace_begin(int32_t capacity);
 qsa_status qsa_trace_end(int32_t* kernel_ids, float* ms, int32_t capacity, int32_t* n_out);

@@ -120,3 +120,30 @@ def test_decode_append_writes_caches():
         assert np.array_equal(st.w_ring[b, L % 4].cpu().numpy(), h["w"][L])
         kr = np.stack([O.rope(Q.bf16_to_f64(h["k"][L, g]), L) for g in range(2)])
         assert np.abs(Q.bf16_to_f64(st.k_cache[b, L].cpu().numpy()) - kr).max() < 0.05
+
+
+@pytest.mark.parametrize("splits", [1, 2, 5, 16])
+def test_decode_split_kv_ranges(splits, monkeypatch):
+    """Split-KV decode with a fixed number of ranges, including ranges left
+    empty by a short sequence (1 tile) next to full-budget ones (32 tiles):
+    output and lse match the oracle on the kernel's own selection."""
+    monkeypatch.setenv("QSA_DECODE_SPLITS", str(splits))
+    budget = 512
+    L_list = [3001, 37, 9000]
+    probs = [Q.PrefillProblem(T=L + 1, seed=70 + b, n_plant=8) for b, L in enumerate(L_list)]
+    st = DecodeState(probs, L_list, max_len=max(L_list) + 8, budget=budget)
+    O = oracle.Oracle(oracle.params(budget=budget))
+    pos, out, sel, lse = st.step()
+    for b in range(len(L_list)):
+        L = pos[b]
+        h = st.hosts[b]
+        qb = L // 4
+        t0 = 4 * qb
+        cnt = int((sel[b] >= 0).sum())
+        assert cnt == min(qb + 1, budget)
+        kc = st.k_cache[b, :L].cpu().numpy()
+        _, _, oo, ol = O.decode(L, kc, h["v"][:L], h["k_idx"][:L], h["q_idx"][t0:L], h["w"][t0:L], h["q"][L],
+                                h["k"][L], h["v"][L], h["q_idx"][L], h["k_idx"][L], h["w"][L], sel_in=sel[b],
+                                cnt_in=cnt)
+        check_outputs(out[b], oo, f"splits={splits} b={b}")
+        assert np.allclose(lse[b], ol, atol=1e-2), f"splits={splits} b={b}"
