@@ -473,6 +473,12 @@ WORKLOADS = {
 }
 
 
+# DRAM bytes (read + write) per launch of the dominant kernel, from the one-pass
+# ncu capture summarised in profiles/launches_prefill_1m.md; None where no
+# capture of the current kernel exists.
+NCU_TRAFFIC = {"prefill_1m": 67.49e9 + 15.26e9}
+
+
 def line_for(name, res, n_gpus, steps, warmup, pk):
     wl = WORKLOADS[name]
     if wl["kind"] == "prefill":
@@ -482,7 +488,7 @@ def line_for(name, res, n_gpus, steps, warmup, pk):
         # achieved = algorithmic indexer FLOPs per launch / mean launch time
         achieved = res["flops_idx"] * res["steps"] / idx_n / (idx_ms / idx_n / 1e3) / 1e12
         roof = dict(kernel="indexer", bound="tensor", achieved=achieved, peak=pk["bf16_sus"], unit="TFLOP/s",
-                    frac=achieved / pk["bf16_sus"], traffic=None,
+                    frac=achieved / pk["bf16_sus"], traffic=NCU_TRAFFIC.get(name),
                     peak_src=f"{pk['src']} bf16 dense sustained")
         total_fl = res["flops_idx"] + res["flops_attn"]
         whole = dict(tflops=total_fl / (res["ms"] / res["steps"] / 1e3) / 1e12)
@@ -497,7 +503,7 @@ def line_for(name, res, n_gpus, steps, warmup, pk):
         n, t = res["kern"].get("decode_indexer", (1, float("nan")))
         achieved = res["bytes_indexer"] / (t / n / 1e3) / 1e9
         roof = dict(kernel="decode_indexer", bound="hbm", achieved=achieved, peak=pk["hbm"], unit="GB/s",
-                    frac=achieved / pk["hbm"], traffic=None, peak_src=f"{pk['src']} HBM copy")
+                    frac=achieved / pk["hbm"], traffic=NCU_TRAFFIC.get(name), peak_src=f"{pk['src']} HBM copy")
         whole = dict(gbs=res["bytes_step"] / (res["ms"] / res["steps"] / 1e3) / 1e9)
         whole["frac_of_hbm_roofline"] = whole["gbs"] / pk["hbm"]
         metric = "QSA decode tokens/s at 256K context, batch 64"
