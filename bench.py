@@ -473,9 +473,9 @@ WORKLOADS = {
 }
 
 
-# DRAM bytes (read + write) per launch of the dominant kernel, from the one-pass
-# ncu capture summarised in profiles/launches_prefill_1m.md; None where no
-# capture of the current kernel exists.
+# DRAM bytes per launch of the dominant kernel (dram__bytes_read.sum +
+# dram__bytes_write.sum, averaged over the launches of a one-pass ncu capture
+# of this workload with the current kernel); None where no such capture exists.
 NCU_TRAFFIC = {"prefill_1m": 67.49e9 + 15.26e9}
 
 
