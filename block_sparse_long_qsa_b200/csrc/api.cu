@@ -152,7 +152,8 @@ qsa_status from_cuda(cudaError_t e, const char* where = "kernel launch") {
 
 // Indexer launch for query blocks [qb0, qb1) into S (ld), maps built here.
 qsa_status run_indexer(int64_t T, const uint16_t* q_idx, const uint16_t* w, const uint16_t* k_idx, int64_t qb0,
-                       int64_t qb1, float* S, int64_t ld, uint32_t* err, int num_sms, cudaStream_t st) {
+                       int64_t qb1, float* S, int64_t ld, float* segmax, int64_t ld_seg, uint32_t* err, int num_sms,
+                       cudaStream_t st) {
   if (qb1 <= qb0) return QSA_OK;
   CUtensorMap tq, tk;
   qsa_status rs;
@@ -160,7 +161,7 @@ qsa_status run_indexer(int64_t T, const uint16_t* q_idx, const uint16_t* w, cons
   if ((rs = make_map_2d(&tk, k_idx, (uint64_t)T, 128, 128, 64)) != QSA_OK) return rs;
   const float scale = 1.0f / std::sqrt(128.0f);
   return from_cuda(traced(QSA_KERNEL_INDEXER, st, [&] {
-    return qsa::launch_indexer_prefill(tq, tk, w, S, ld, T, qb0, qb1, scale, err, num_sms, st);
+    return qsa::launch_indexer_prefill(tq, tk, w, S, ld, segmax, ld_seg, T, qb0, qb1, scale, err, num_sms, st);
   }), "indexer launch");
 }
 
@@ -180,13 +181,16 @@ PrefillLayout prefill_layout(int64_t T, int budget, bool need_krot, bool need_se
   L.total_fixed = off;
   return L;
 }
-// largest qb1 in (qb0, nqb] whose slab (qb1-qb0) x round4(qb1) x 4 fits
+// Slab bytes of one row of a chunk ending at query block qb1: the scores
+// (round4(qb1) floats) and the segment maxima (round4(ceil(qb1 / 8)) floats).
+size_t slab_row_bytes(int64_t qb1) { return ((size_t)round4(qb1) + (size_t)round4((qb1 + 7) / 8)) * 4; }
+// largest qb1 in (qb0, nqb] whose slab (qb1-qb0) x slab_row_bytes(qb1) fits
 int64_t chunk_end(int64_t qb0, int64_t nqb, size_t slab_bytes) {
   int64_t lo = qb0 + 1, hi = nqb;
-  if ((size_t)1 * round4(lo) * 4 > slab_bytes) return qb0;  // not even one row
+  if (slab_row_bytes(lo) > slab_bytes) return qb0;  // not even one row
   while (lo < hi) {
     const int64_t mid = (lo + hi + 1) / 2;
-    if ((size_t)(mid - qb0) * (size_t)round4(mid) * 4 <= slab_bytes) lo = mid; else hi = mid - 1;
+    if ((size_t)(mid - qb0) * slab_row_bytes(mid) <= slab_bytes) lo = mid; else hi = mid - 1;
   }
   return lo;
 }
@@ -245,7 +249,7 @@ qsa_status qsa_index_scores(const qsa_params* p, int64_t T, const uint16_t* q_id
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t* err = static_cast<uint32_t*>(ws);
   if (err && cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaMemsetAsync");
-  return run_indexer(T, q_idx, w, k_idx, qb_begin, qb_end, scores, ld, err, di.num_sms, s);
+  return run_indexer(T, q_idx, w, k_idx, qb_begin, qb_end, scores, ld, nullptr, 0, err, di.num_sms, s);
 }
 
 qsa_status qsa_select_workspace_size(const qsa_params* p, size_t* bytes) {
@@ -270,7 +274,8 @@ qsa_status qsa_select_blocks(const qsa_params* p, const float* scores, int64_t l
   uint32_t* err = static_cast<uint32_t*>(ws);
   if (cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaMemsetAsync");
   return from_cuda(traced(QSA_KERNEL_SELECT, s, [&] {
-    return qsa::launch_select(scores, ld, qb_begin, qb_end - qb_begin, nullptr, p->budget_blocks, sel, cnt, err, s);
+    return qsa::launch_select(scores, ld, nullptr, 0, qb_begin, qb_end - qb_begin, nullptr, p->budget_blocks, sel, cnt,
+                              err, s);
   }));
 }
 
@@ -283,7 +288,7 @@ qsa_status qsa_prefill_workspace_size(const qsa_params* p, int64_t T, size_t* mi
   // worst case: the library keeps k_rot, sel and cnt itself
   PrefillLayout L = prefill_layout(T, p->budget_blocks, true, true, true);
   const int64_t min_rows = nqb < MIN_ROWS ? nqb : MIN_ROWS;
-  const size_t row_bytes = (size_t)round4(nqb) * 4;
+  const size_t row_bytes = slab_row_bytes(nqb);
   if (min_bytes) *min_bytes = L.total_fixed + (size_t)min_rows * row_bytes;
   if (pref_bytes) {
     // whole triangle in one pass is nqb rows of round4(nqb); cap it
@@ -312,7 +317,7 @@ qsa_status qsa_prefill(const qsa_params* p, int64_t T, int64_t pos0, const uint1
   if (ws_bytes < L.total_fixed) return QSA_ERR_WORKSPACE_TOO_SMALL;
   const size_t slab_bytes = ws_bytes - L.total_fixed;
   const int64_t min_rows = nqb < MIN_ROWS ? nqb : MIN_ROWS;
-  if (slab_bytes < (size_t)min_rows * (size_t)round4(nqb) * 4) return QSA_ERR_WORKSPACE_TOO_SMALL;
+  if (slab_bytes < (size_t)min_rows * slab_row_bytes(nqb)) return QSA_ERR_WORKSPACE_TOO_SMALL;
   DevInfo di;
   if ((st = device_info(&di)) != QSA_OK) return st;
 
@@ -338,9 +343,13 @@ qsa_status qsa_prefill(const qsa_params* p, int64_t T, int64_t pos0, const uint1
     const int64_t qb1 = chunk_end(qb0, nqb, slab_bytes);
     if (qb1 <= qb0) return QSA_ERR_WORKSPACE_TOO_SMALL;
     const int64_t ld = round4(qb1);
-    if ((st = run_indexer(T, q_idx, w, k_idx, qb0, qb1, slab, ld, err, di.num_sms, s)) != QSA_OK) return st;
+    const int64_t ld_seg = round4((qb1 + 7) / 8);
+    float* segmax = slab + (size_t)(qb1 - qb0) * ld;
+    if ((st = run_indexer(T, q_idx, w, k_idx, qb0, qb1, slab, ld, segmax, ld_seg, err, di.num_sms, s)) != QSA_OK)
+      return st;
     if ((st = from_cuda(traced(QSA_KERNEL_SELECT, s, [&] {
-           return qsa::launch_select(slab, ld, qb0, qb1 - qb0, nullptr, budget, sel + qb0 * budget, cnt + qb0, err, s);
+           return qsa::launch_select(slab, ld, segmax, ld_seg, qb0, qb1 - qb0, nullptr, budget, sel + qb0 * budget,
+                                     cnt + qb0, err, s);
          }))) != QSA_OK)
       return st;
     if ((st = from_cuda(traced(QSA_KERNEL_ATTENTION, s, [&] {
@@ -464,7 +473,7 @@ qsa_status qsa_decode(const qsa_params* p, int32_t B, int64_t max_len, const int
        }))) != QSA_OK)
     return st;
   if ((st = from_cuda(traced(QSA_KERNEL_SELECT, s, [&] {
-         return qsa::launch_select(S, L.ld, 0, B, qbs, budget, sel, cnt, err, s);
+         return qsa::launch_select(S, L.ld, nullptr, 0, 0, B, qbs, budget, sel, cnt, err, s);
        }))) != QSA_OK)
     return st;
   const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;

@@ -89,8 +89,9 @@ struct Iter {
 
 __global__ void __launch_bounds__(THREADS, 1)
 indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const uint16_t* __restrict__ w, float* __restrict__ S, int64_t ld, int64_t T,
-                       int64_t qb_begin, int64_t qb_end, float scale, uint32_t* err) {
+                       const uint16_t* __restrict__ w, float* __restrict__ S, int64_t ld,
+                       float* __restrict__ segmax, int64_t ld_seg, int64_t T, int64_t qb_begin, int64_t qb_end,
+                       float scale, uint32_t* err) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* sQ = smem;
   uint8_t* sK = smem + OFF_K;
@@ -328,13 +329,31 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
           const float keep = la ? m[i + 4] : m[i];
           n4[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 1));
         }
+        float val[2];
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
           const float send = lb ? n4[i] : n4[i + 2];
           const float keep = lb ? n4[i + 2] : n4[i];
-          const float val = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
+          val[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
           const int64_t qb = qb_first + (la ? 4 : 0) + (lb ? 2 : 0) + i;
-          if (qb < qb_end && kb <= qb) S[(qb - qb_begin) * ld + kb] = val * scale;
+          if (qb < qb_end && kb <= qb) S[(qb - qb_begin) * ld + kb] = val[i] * scale;
+        }
+        if (segmax != nullptr) {
+          // segment maxima: max over the 8 key blocks of this warp's 32 keys
+          // (lane bits 2..4).  A transposing step on bit 2 leaves each lane one
+          // query block (4 a + 2 b + c0), then two plain steps; lanes 0..7 hold
+          // the 8 query blocks.  Key blocks after a query block were scored as
+          // 0 and scores are >= 0, so they do not raise a maximum.
+          const bool lc = (lane & 4) != 0;
+          float sm = fmaxf(lc ? val[1] : val[0], __shfl_xor_sync(0xffffffffu, lc ? val[0] : val[1], 4));
+          sm = fmaxf(sm, __shfl_xor_sync(0xffffffffu, sm, 8));
+          sm = fmaxf(sm, __shfl_xor_sync(0xffffffffu, sm, 16));
+          if (lane < 8) {
+            const int64_t seg = (KT * it.kt + 32 * quad) >> 5;
+            const int64_t qb = qb_first + (la ? 4 : 0) + (lb ? 2 : 0) + (lc ? 1 : 0);
+            // only segments starting at or before the row's own block: seg <= qb / 8 < ld_seg
+            if (qb < qb_end && seg <= (qb >> 3)) segmax[(qb - qb_begin) * ld_seg + seg] = sm * scale;
+          }
         }
       } else {
         tc_fence_before();
@@ -359,8 +378,8 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 }  // namespace
 
 cudaError_t launch_indexer_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const uint16_t* w,
-                                   float* S, int64_t ld, int64_t T, int64_t qb_begin, int64_t qb_end, float scale,
-                                   uint32_t* err, int num_sms, cudaStream_t stream) {
+                                   float* S, int64_t ld, float* segmax, int64_t ld_seg, int64_t T, int64_t qb_begin,
+                                   int64_t qb_end, float scale, uint32_t* err, int num_sms, cudaStream_t stream) {
   if (qb_end <= qb_begin) return cudaSuccess;
   static bool attr_done[64] = {false};
   int dev = 0;
@@ -382,8 +401,8 @@ cudaError_t launch_indexer_prefill(const CUtensorMap& tm_q, const CUtensorMap& t
     units += tl / KT + 1;
   }
   const int grid = (int)(units < num_sms ? units : num_sms);
-  indexer_prefill_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tm_q, tm_k, w, S, ld, T, qb_begin, qb_end, scale,
-                                                                 err);
+  indexer_prefill_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tm_q, tm_k, w, S, ld, segmax, ld_seg, T, qb_begin,
+                                                                 qb_end, scale, err);
   return cudaGetLastError();
 }
 

@@ -12,15 +12,22 @@ cudaError_t launch_rope_table(int64_t T, int64_t pos0, const double* inv_freq_ho
 // k_rot[t][g] = RoPE(k[t][g]) on dims 0..63, dims 64..255 copied.
 cudaError_t launch_rope_k(int64_t T, const uint16_t* k, const float2* cs, uint16_t* k_rot, cudaStream_t s);
 
+// Block scores of query blocks [qb_begin, qb_end) into S (row stride ld, only
+// kb <= qb written).  segmax (nullable, row stride ld_seg): per row, the max
+// over each segment of 8 key blocks (segment s = blocks 8s .. 8s+7, blocks
+// after the row's own block counting as 0).
 cudaError_t launch_indexer_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const uint16_t* w,
-                                   float* S, int64_t ld, int64_t T, int64_t qb_begin, int64_t qb_end, float scale,
-                                   uint32_t* err, int num_sms, cudaStream_t stream);
+                                   float* S, int64_t ld, float* segmax, int64_t ld_seg, int64_t T, int64_t qb_begin,
+                                   int64_t qb_end, float scale, uint32_t* err, int num_sms, cudaStream_t stream);
 
 // Top-k block selection, one row per query block.  Row r covers query block
-// row_qb ? row_qb[r] : qb_begin + r, read from S + r * ld.
+// row_qb ? row_qb[r] : qb_begin + r, read from S + r * ld.  segmax (nullable,
+// row stride ld_seg): the indexer's maxima over segments of 8 key blocks; with
+// it, long rows are filtered from the segment maxima instead of a full pass.
 size_t select_smem_bytes(int budget);
-cudaError_t launch_select(const float* S, int64_t ld, int64_t qb_begin, int64_t n_rows, const int64_t* row_qb,
-                          int budget, int32_t* sel, int32_t* cnt, uint32_t* err, cudaStream_t stream);
+cudaError_t launch_select(const float* S, int64_t ld, const float* segmax, int64_t ld_seg, int64_t qb_begin,
+                          int64_t n_rows, const int64_t* row_qb, int budget, int32_t* sel, int32_t* cnt, uint32_t* err,
+                          cudaStream_t stream);
 
 // Sparse GQA attention for query blocks [qb_begin, qb_end) given their
 // selections (sel/cnt indexed from qb_begin): tcgen05 kernel, persistent.

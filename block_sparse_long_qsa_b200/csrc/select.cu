@@ -127,9 +127,9 @@ __device__ __forceinline__ uint32_t block_excl_count(bool flag, const SelSmem& s
 }
 
 __global__ void __launch_bounds__(THREADS, 3)
-select_kernel(const float* __restrict__ S, int64_t ld, int64_t qb_begin, int64_t n_rows,
-              const int64_t* __restrict__ row_qb, int budget, int32_t* __restrict__ sel, int32_t* __restrict__ cnt,
-              uint32_t* err) {
+select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__ segmax, int64_t ld_seg,
+              int64_t qb_begin, int64_t n_rows, const int64_t* __restrict__ row_qb, int budget,
+              int32_t* __restrict__ sel, int32_t* __restrict__ cnt, uint32_t* err) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const int cap = cap_for(budget);
   const int P = pow2_at_least(budget);
@@ -167,6 +167,77 @@ select_kernel(const float* __restrict__ S, int64_t ld, int64_t qb_begin, int64_t
         sm.cidx[i] = (int32_t)i;
       }
       nc = m;
+    } else if (segmax != nullptr) {
+      // 1'. threshold from the segment maxima.  Segments 0 .. fs-1 (8 blocks
+      //     each) hold candidate blocks only; blocks 8 fs .. qb-2 form the tail.
+      //     If at least k segments reach tau0, at least k scores do, and every
+      //     score >= tau0 lies in such a segment or in the tail.
+      const int64_t fs = (qb - 1) >> 3;
+      const float* mrow = segmax + r * ld_seg;
+      for (int i = tid; i < NSAMPLE; i += blockDim.x) sm.sample[i] = key_of(mrow[(int64_t)i * fs / NSAMPLE]);
+      const float e = (float)NSAMPLE * (float)k / (float)fs;
+      int64_t rs = (int64_t)ceilf(e + 4.f * sqrtf(e) + 8.f);
+      if (rs > NSAMPLE) rs = NSAMPLE;
+      __syncthreads();
+      uint32_t tau0;
+      int64_t dummy;
+      radix_kth_largest([&](int64_t i) { return sm.sample[i]; }, NSAMPLE, rs, sm, tau0, dummy);
+      // 2'. the segments whose max reaches tau0 (listed in the sample buffer) ...
+      if (tid == 0) sm.misc[5] = 0;
+      __syncthreads();
+      for (int64_t b0 = 0; b0 < fs; b0 += blockDim.x) {
+        const int64_t sgi = b0 + tid;
+        const bool pass = sgi < fs && key_of(mrow[sgi]) >= tau0;
+        const uint32_t ball = __ballot_sync(0xffffffffu, pass);
+        if (ball) {
+          uint32_t base = 0;
+          if (lane == 0) base = atomicAdd(&sm.misc[5], (uint32_t)__popc(ball));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          const uint32_t pos = base + __popc(ball & ((1u << lane) - 1u));
+          if (pass && pos < (uint32_t)NSAMPLE) sm.sample[pos] = (uint32_t)sgi;
+        }
+      }
+      __syncthreads();
+      const int64_t nsl = sm.misc[5];
+      if (nsl > NSAMPLE) {
+        global_path = true;
+      } else {
+        // ... and their scores >= tau0 (two 16-byte loads per segment), then the tail
+        const float4* row4 = reinterpret_cast<const float4*>(row);
+        for (int64_t b0 = 0; b0 < 2 * nsl; b0 += blockDim.x) {
+          const int64_t e2 = b0 + tid;
+          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+          int64_t i0 = 0;
+          if (e2 < 2 * nsl) {
+            i0 = 8 * (int64_t)sm.sample[e2 >> 1] + 4 * (e2 & 1);
+            v = __ldcs(row4 + (i0 >> 2));
+          }
+          const float vals[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const bool pass = e2 < 2 * nsl && key_of(vals[q]) >= tau0;
+            const uint32_t ball = __ballot_sync(0xffffffffu, pass);
+            if (ball) {
+              uint32_t base = 0;
+              if (lane == 0) base = atomicAdd(&sm.misc[2], (uint32_t)__popc(ball));
+              base = __shfl_sync(0xffffffffu, base, 0);
+              const uint32_t pos = base + __popc(ball & ((1u << lane) - 1u));
+              if (pass && pos < (uint32_t)cap) { sm.ckey[pos] = key_of(vals[q]); sm.cidx[pos] = (int32_t)(i0 + q); }
+            }
+          }
+        }
+        if (tid < 8) {
+          const int64_t i = 8 * fs + tid;
+          if (i < m && key_of(row[i]) >= tau0) {
+            const uint32_t pos = atomicAdd(&sm.misc[2], 1u);
+            if (pos < (uint32_t)cap) { sm.ckey[pos] = key_of(row[i]); sm.cidx[pos] = (int32_t)i; }
+          }
+        }
+        __syncthreads();
+        nc = sm.misc[2];
+        global_path = (nc < k || nc > cap);
+      }
+      __syncthreads();
     } else {
       // 1. threshold from a strided sample
       for (int i = tid; i < NSAMPLE; i += blockDim.x) sm.sample[i] = key_of(row[(int64_t)i * m / NSAMPLE]);
@@ -307,8 +378,9 @@ size_t select_smem_bytes(int budget) {
   return (size_t)(256 + 16 + 32 + NSAMPLE) * 4 + (size_t)cap * 8 + (size_t)pow2_at_least(budget) * 4;
 }
 
-cudaError_t launch_select(const float* S, int64_t ld, int64_t qb_begin, int64_t n_rows, const int64_t* row_qb,
-                          int budget, int32_t* sel, int32_t* cnt, uint32_t* err, cudaStream_t stream) {
+cudaError_t launch_select(const float* S, int64_t ld, const float* segmax, int64_t ld_seg, int64_t qb_begin,
+                          int64_t n_rows, const int64_t* row_qb, int budget, int32_t* sel, int32_t* cnt, uint32_t* err,
+                          cudaStream_t stream) {
   if (n_rows <= 0) return cudaSuccess;
   const size_t smem = select_smem_bytes(budget);
   static size_t attr_set[64] = {0};
@@ -320,7 +392,8 @@ cudaError_t launch_select(const float* S, int64_t ld, int64_t qb_begin, int64_t 
     attr_set[dev] = smem;
   }
   const int64_t grid = n_rows < 148 * 64 ? n_rows : 148 * 64;
-  select_kernel<<<(unsigned)grid, THREADS, smem, stream>>>(S, ld, qb_begin, n_rows, row_qb, budget, sel, cnt, err);
+  select_kernel<<<(unsigned)grid, THREADS, smem, stream>>>(S, ld, segmax, ld_seg, qb_begin, n_rows, row_qb, budget,
+                                                          sel, cnt, err);
   return cudaGetLastError();
 }
 
