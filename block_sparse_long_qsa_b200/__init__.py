@@ -25,7 +25,7 @@ _STATUS = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_UNSUPPORTED", 3: "
 EXPORTED = ["qsa_default_params", "qsa_status_string", "qsa_last_error", "qsa_index_scores", "qsa_select_blocks",
             "qsa_select_workspace_size", "qsa_prefill", "qsa_prefill_workspace_size", "qsa_decode",
             "qsa_decode_workspace_size", "qsa_check_device_error", "qsa_trace_begin", "qsa_trace_end",
-            "qsa_decode_noalloc"]
+            "qsa_decode_noalloc", "qsa_prefill_cached", "qsa_prefill_cached_workspace_size"]
 
 KERNEL_NAMES = {1: "rope_table", 2: "rope_k", 3: "indexer", 4: "select", 5: "attention", 6: "decode_append",
                 7: "decode_indexer", 8: "decode_attention", 9: "decode_combine"}
@@ -69,6 +69,8 @@ def load(path: str = LIB_PATH):
     L.qsa_select_workspace_size.argtypes = [P, psz]
     L.qsa_prefill.argtypes = [P, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.qsa_prefill_workspace_size.argtypes = [P, i64, psz, psz]
+    L.qsa_prefill_cached.argtypes = [P, i64, i64] + [vp] * 16 + [sz, vp]
+    L.qsa_prefill_cached_workspace_size.argtypes = [P, i64, i64, psz, psz]
     L.qsa_decode.argtypes = [P, i32, i64, ctypes.POINTER(ctypes.c_int64), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                              vp, vp, vp, vp, sz, vp]
     L.qsa_decode_workspace_size.argtypes = [P, i32, i64, psz]
@@ -147,6 +149,21 @@ def qsa_prefill(p: qsa_params, T: int, pos0: int, q, k, v, q_idx, w, k_idx, out,
     _check(load().qsa_prefill(ctypes.byref(p), T, pos0, _ptr(q), _ptr(k), _ptr(v), _ptr(q_idx), _ptr(w), _ptr(k_idx),
                               _ptr(out), _ptr(lse), _ptr(sel_out), _ptr(cnt_out), _ptr(k_rot_out), _ptr(ws),
                               ws.numel() * ws.element_size(), _stream(stream)), "qsa_prefill")
+
+
+def qsa_prefill_cached_workspace_size(p: qsa_params, L_old: int, T_new: int) -> tuple[int, int]:
+    a, b = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(load().qsa_prefill_cached_workspace_size(ctypes.byref(p), L_old, T_new, ctypes.byref(a), ctypes.byref(b)),
+           "qsa_prefill_cached_workspace_size")
+    return a.value, b.value
+
+
+def qsa_prefill_cached(p: qsa_params, L_old: int, T_new: int, k_cache, v_cache, kidx_cache, qidx_prev, w_prev, q, k,
+                       v, q_idx, w, k_idx, out, lse=None, sel_out=None, cnt_out=None, ws=None, stream=None):
+    _check(load().qsa_prefill_cached(ctypes.byref(p), L_old, T_new, _ptr(k_cache), _ptr(v_cache), _ptr(kidx_cache),
+                                     _ptr(qidx_prev), _ptr(w_prev), _ptr(q), _ptr(k), _ptr(v), _ptr(q_idx), _ptr(w),
+                                     _ptr(k_idx), _ptr(out), _ptr(lse), _ptr(sel_out), _ptr(cnt_out), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream)), "qsa_prefill_cached")
 
 
 def qsa_decode_workspace_size(p: qsa_params, B: int, max_len: int) -> int:

@@ -151,17 +151,19 @@ qsa_status from_cuda(cudaError_t e, const char* where = "kernel launch") {
 }
 
 // Indexer launch for query blocks [qb0, qb1) into S (ld), maps built here.
-qsa_status run_indexer(int64_t T, const uint16_t* q_idx, const uint16_t* w, const uint16_t* k_idx, int64_t qb0,
-                       int64_t qb1, float* S, int64_t ld, float* segmax, int64_t ld_seg, uint32_t* err, int num_sms,
-                       cudaStream_t st) {
+// Keys: tokens [0, T) of k_idx; q_idx / w hold tokens [q_tok0, T).
+qsa_status run_indexer(int64_t T, int64_t q_tok0, const uint16_t* q_idx, const uint16_t* w, const uint16_t* k_idx,
+                       int64_t qb0, int64_t qb1, float* S, int64_t ld, float* segmax, int64_t ld_seg, uint32_t* err,
+                       int num_sms, cudaStream_t st) {
   if (qb1 <= qb0) return QSA_OK;
   CUtensorMap tq, tk;
   qsa_status rs;
-  if ((rs = make_map_2d(&tq, q_idx, (uint64_t)T * 4, 128, 256, 64)) != QSA_OK) return rs;
+  if ((rs = make_map_2d(&tq, q_idx, (uint64_t)(T - q_tok0) * 4, 128, 256, 64)) != QSA_OK) return rs;
   if ((rs = make_map_2d(&tk, k_idx, (uint64_t)T, 128, 128, 64)) != QSA_OK) return rs;
   const float scale = 1.0f / std::sqrt(128.0f);
   return from_cuda(traced(QSA_KERNEL_INDEXER, st, [&] {
-    return qsa::launch_indexer_prefill(tq, tk, w, S, ld, segmax, ld_seg, T, qb0, qb1, scale, err, num_sms, st);
+    return qsa::launch_indexer_prefill(tq, tk, w, S, ld, segmax, ld_seg, T, q_tok0, qb0, qb1, scale, err, num_sms,
+                                       st);
   }), "indexer launch");
 }
 
@@ -249,7 +251,7 @@ qsa_status qsa_index_scores(const qsa_params* p, int64_t T, const uint16_t* q_id
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t* err = static_cast<uint32_t*>(ws);
   if (err && cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaMemsetAsync");
-  return run_indexer(T, q_idx, w, k_idx, qb_begin, qb_end, scores, ld, nullptr, 0, err, di.num_sms, s);
+  return run_indexer(T, 0, q_idx, w, k_idx, qb_begin, qb_end, scores, ld, nullptr, 0, err, di.num_sms, s);
 }
 
 qsa_status qsa_select_workspace_size(const qsa_params* p, size_t* bytes) {
@@ -345,7 +347,7 @@ qsa_status qsa_prefill(const qsa_params* p, int64_t T, int64_t pos0, const uint1
     const int64_t ld = round4(qb1);
     const int64_t ld_seg = round4((qb1 + 7) / 8);
     float* segmax = slab + (size_t)(qb1 - qb0) * ld;
-    if ((st = run_indexer(T, q_idx, w, k_idx, qb0, qb1, slab, ld, segmax, ld_seg, err, di.num_sms, s)) != QSA_OK)
+    if ((st = run_indexer(T, 0, q_idx, w, k_idx, qb0, qb1, slab, ld, segmax, ld_seg, err, di.num_sms, s)) != QSA_OK)
       return st;
     if ((st = from_cuda(traced(QSA_KERNEL_SELECT, s, [&] {
            return qsa::launch_select(slab, ld, segmax, ld_seg, qb0, qb1 - qb0, nullptr, budget, sel + qb0 * budget,
@@ -354,7 +356,141 @@ qsa_status qsa_prefill(const qsa_params* p, int64_t T, int64_t pos0, const uint1
       return st;
     if ((st = from_cuda(traced(QSA_KERNEL_ATTENTION, s, [&] {
            return qsa::launch_sparse_attn_prefill_tc(T, q, k_rot, v, cs, sel + qb0 * budget, cnt + qb0, budget, qb0,
-                                                     qb1, scale_log2, out, lse, err, di.num_sms, s);
+                                                     qb1, 0, scale_log2, out, lse, err, di.num_sms, s);
+         }))) != QSA_OK)
+      return st;
+    qb0 = qb1;
+  }
+  return QSA_OK;
+}
+
+// --------------------------------------------------------- cached prefill
+namespace {
+struct CachedLayout {
+  size_t cs, qst, wst, sel, cnt, slab, total_fixed;
+};
+// r = L_old % 4 tokens of the partial block before the new ones are staged
+// in front of the new tokens' q_idx / w (nothing is staged when r == 0).
+CachedLayout cached_layout(int64_t L_old, int64_t T_new, int budget, bool need_sel, bool need_cnt) {
+  const int64_t r = L_old % 4;
+  const int64_t nq = (L_old + T_new - 1) / 4 - L_old / 4 + 1;
+  CachedLayout L;
+  size_t off = HEADER_BYTES;
+  L.cs = off; off = align_up(off + (size_t)T_new * 32 * sizeof(float2));
+  L.qst = off; off = align_up(off + (r ? (size_t)(r + T_new) * 4 * 128 * 2 : 0));
+  L.wst = off; off = align_up(off + (r ? (size_t)(r + T_new) * 4 * 2 : 0));
+  L.sel = off; off = align_up(off + (need_sel ? (size_t)nq * budget * 4 : 0));
+  L.cnt = off; off = align_up(off + (need_cnt ? (size_t)nq * 4 : 0));
+  L.slab = off;
+  L.total_fixed = off;
+  return L;
+}
+}  // namespace
+
+qsa_status qsa_prefill_cached_workspace_size(const qsa_params* p, int64_t L_old, int64_t T_new, size_t* min_bytes,
+                                             size_t* pref_bytes) {
+  qsa_status st = check_params(p);
+  if (st != QSA_OK) return st;
+  if (L_old < 0 || T_new <= 0) return QSA_ERR_INVALID_ARG;
+  if (L_old + T_new > ((int64_t)1 << 24)) return QSA_ERR_UNSUPPORTED;
+  const int64_t nkb = (L_old + T_new + 3) / 4, qbA = L_old / 4, nq = nkb - qbA;
+  CachedLayout L = cached_layout(L_old, T_new, p->budget_blocks, true, true);
+  const int64_t min_rows = nq < MIN_ROWS ? nq : MIN_ROWS;
+  const size_t row_bytes = slab_row_bytes(nkb);
+  if (min_bytes) *min_bytes = L.total_fixed + (size_t)min_rows * row_bytes;
+  if (pref_bytes) {
+    const size_t full = (size_t)nq * row_bytes;
+    const size_t cap = PREF_CAP > (size_t)min_rows * row_bytes ? PREF_CAP : (size_t)min_rows * row_bytes;
+    *pref_bytes = L.total_fixed + (full < cap ? full : cap);
+  }
+  return QSA_OK;
+}
+
+qsa_status qsa_prefill_cached(const qsa_params* p, int64_t L_old, int64_t T_new, uint16_t* k_cache, uint16_t* v_cache,
+                              uint16_t* kidx_cache, const uint16_t* qidx_prev, const uint16_t* w_prev,
+                              const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* q_idx,
+                              const uint16_t* w, const uint16_t* k_idx, uint16_t* out, float* lse, int32_t* sel_out,
+                              int32_t* cnt_out, void* ws, size_t ws_bytes, void* stream) {
+  qsa_status st = check_params(p);
+  if (st != QSA_OK) return st;
+  if (L_old < 0 || T_new <= 0) return QSA_ERR_INVALID_ARG;
+  if (L_old + T_new > ((int64_t)1 << 24)) return QSA_ERR_UNSUPPORTED;
+  const int64_t r = L_old % 4;
+  if (!k_cache || !v_cache || !kidx_cache || !q || !k || !v || !q_idx || !w || !k_idx || !out || !ws)
+    return QSA_ERR_INVALID_ARG;
+  if (r && (!qidx_prev || !w_prev)) return QSA_ERR_INVALID_ARG;
+  const void* ptrs[] = {k_cache, v_cache, kidx_cache, qidx_prev, w_prev, q, k, v, q_idx, w, k_idx, out, lse,
+                        sel_out, cnt_out, ws};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return QSA_ERR_MISALIGNED;
+  const int budget = p->budget_blocks;
+  const int64_t T = L_old + T_new;               // keys: tokens [0, T)
+  const int64_t nkb = (T + 3) / 4, qbA = L_old / 4, nq = nkb - qbA;
+  CachedLayout L = cached_layout(L_old, T_new, budget, sel_out == nullptr, cnt_out == nullptr);
+  if (ws_bytes < L.total_fixed) return QSA_ERR_WORKSPACE_TOO_SMALL;
+  const size_t slab_bytes = ws_bytes - L.total_fixed;
+  const int64_t min_rows = nq < MIN_ROWS ? nq : MIN_ROWS;
+  if (slab_bytes < (size_t)min_rows * slab_row_bytes(nkb)) return QSA_ERR_WORKSPACE_TOO_SMALL;
+  DevInfo di;
+  if ((st = device_info(&di)) != QSA_OK) return st;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint32_t* err = reinterpret_cast<uint32_t*>(base);
+  float2* cs = reinterpret_cast<float2*>(base + L.cs);
+  int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(base + L.sel);
+  int32_t* cnt = cnt_out ? cnt_out : reinterpret_cast<int32_t*>(base + L.cnt);
+  float* slab = reinterpret_cast<float*>(base + L.slab);
+
+  if (cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaMemsetAsync");
+  // new tokens into the caches: rotated keys at positions L_old .., values, indexer keys
+  double f[32];
+  inv_freq(p, f);
+  if ((st = from_cuda(traced(QSA_KERNEL_ROPE_TABLE, s, [&] {
+         return qsa::launch_rope_table(T_new, L_old, f, cs, s);
+       }))) != QSA_OK)
+    return st;
+  if ((st = from_cuda(traced(QSA_KERNEL_ROPE_K, s, [&] {
+         return qsa::launch_rope_k(T_new, k, cs, k_cache + L_old * 512, s);
+       }))) != QSA_OK)
+    return st;
+  if (cudaMemcpyAsync(v_cache + L_old * 512, v, (size_t)T_new * 1024, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(kidx_cache + L_old * 128, k_idx, (size_t)T_new * 256, cudaMemcpyDeviceToDevice, s) !=
+          cudaSuccess)
+    return fail(QSA_ERR_CUDA, "cudaMemcpyAsync (cache append)");
+  // indexer queries from the first new query block's first token on
+  const uint16_t* qi = q_idx;
+  const uint16_t* wi = w;
+  if (r) {
+    uint16_t* qst = reinterpret_cast<uint16_t*>(base + L.qst);
+    uint16_t* wst = reinterpret_cast<uint16_t*>(base + L.wst);
+    if (cudaMemcpyAsync(qst, qidx_prev, (size_t)r * 1024, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(qst + r * 512, q_idx, (size_t)T_new * 1024, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(wst, w_prev, (size_t)r * 8, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(wst + r * 4, w, (size_t)T_new * 8, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return fail(QSA_ERR_CUDA, "cudaMemcpyAsync (indexer query staging)");
+    qi = qst;
+    wi = wst;
+  }
+  const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
+  for (int64_t qb0 = qbA; qb0 < nkb;) {
+    const int64_t qb1 = chunk_end(qb0, nkb, slab_bytes);
+    if (qb1 <= qb0) return QSA_ERR_WORKSPACE_TOO_SMALL;
+    const int64_t ld = round4(qb1);
+    const int64_t ld_seg = round4((qb1 + 7) / 8);
+    float* segmax = slab + (size_t)(qb1 - qb0) * ld;
+    int32_t* sel_c = sel + (qb0 - qbA) * budget;
+    int32_t* cnt_c = cnt + (qb0 - qbA);
+    if ((st = run_indexer(T, 4 * qbA, qi, wi, kidx_cache, qb0, qb1, slab, ld, segmax, ld_seg, err, di.num_sms, s)) !=
+        QSA_OK)
+      return st;
+    if ((st = from_cuda(traced(QSA_KERNEL_SELECT, s, [&] {
+           return qsa::launch_select(slab, ld, segmax, ld_seg, qb0, qb1 - qb0, nullptr, budget, sel_c, cnt_c, err, s);
+         }))) != QSA_OK)
+      return st;
+    if ((st = from_cuda(traced(QSA_KERNEL_ATTENTION, s, [&] {
+           return qsa::launch_sparse_attn_prefill_tc(T, q, k_cache, v_cache, cs, sel_c, cnt_c, budget, qb0, qb1, L_old,
+                                                     scale_log2, out, lse, err, di.num_sms, s);
          }))) != QSA_OK)
       return st;
     qb0 = qb1;

@@ -101,8 +101,9 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 struct TcArgs {
-  int64_t T;
-  const uint16_t* q;        // [T][24][256] unrotated
+  int64_t T;                // keys are tokens [0, T)
+  int64_t q_tok0;           // prefill: q, cs, out and lse start at token q_tok0
+  const uint16_t* q;        // [T - q_tok0][24][256] unrotated
   const uint16_t* k_rot;    // [T][2][256]
   const uint16_t* v;        // [T][2][256]
   const float2* cs;         // [T][32] RoPE table
@@ -233,12 +234,12 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
         const int h = 12 * g + r % 12;
         uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
         const int q16 = slot < 4 ? slot : slot + 4;          // 16-byte chunk of the 512-byte row
-        if (DEC || t < a.T) {
-          const uint4* src = reinterpret_cast<const uint4*>(a.q + ((DEC ? it.row : t) * 24 + h) * 256);
+        if (DEC || (t < a.T && t >= a.q_tok0)) {
+          const uint4* src = reinterpret_cast<const uint4*>(a.q + ((DEC ? it.row : t - a.q_tok0) * 24 + h) * 256);
           lo = __ldg(src + q16);
           if (slot < 4) hi = __ldg(src + slot + 4);
           if (!DEC && slot < 4) {
-            const float2* c8 = a.cs + t * 32 + 8 * slot;
+            const float2* c8 = a.cs + (t - a.q_tok0) * 32 + 8 * slot;
             const uint32_t* x = reinterpret_cast<const uint32_t*>(&lo);
             const uint32_t* y = reinterpret_cast<const uint32_t*>(&hi);
             uint4 olo, ohi;
@@ -460,8 +461,8 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
       ++pv_count;   // the last PV of the item also completed
       tc_fence_after();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      const bool write = row_ok && (DEC || t < a.T);
-      const int64_t orow_idx = (DEC ? it.row : t) * 24 + 12 * g + hh;   // [token or sequence][head]
+      const bool write = row_ok && (DEC || (t < a.T && t >= a.q_tok0));
+      const int64_t orow_idx = (DEC ? it.row : t - a.q_tok0) * 24 + 12 * g + hh;   // [token or sequence][head]
       uint16_t* orow = a.out + orow_idx * 256;
       const bool partial = DEC && a.n_split > 1;
       const int64_t prow = ((it.row * 2 + g) * (int64_t)a.n_split + it.split) * 12 + hh;
@@ -563,11 +564,11 @@ cudaError_t launch_tc(const TcArgs& a, int64_t items, int num_sms, cudaStream_t 
 
 cudaError_t launch_sparse_attn_prefill_tc(int64_t T, const uint16_t* q, const uint16_t* k_rot, const uint16_t* v,
                                           const float2* cs, const int32_t* sel, const int32_t* cnt, int budget,
-                                          int64_t qb_begin, int64_t qb_end, float scale_log2, uint16_t* out,
-                                          float* lse, uint32_t* err, int num_sms, cudaStream_t stream) {
+                                          int64_t qb_begin, int64_t qb_end, int64_t q_tok0, float scale_log2,
+                                          uint16_t* out, float* lse, uint32_t* err, int num_sms, cudaStream_t stream) {
   if (qb_end <= qb_begin) return cudaSuccess;
   TcArgs a{};
-  a.T = T; a.q = q; a.k_rot = k_rot; a.v = v; a.cs = cs; a.sel = sel; a.cnt = cnt; a.budget = budget;
+  a.T = T; a.q_tok0 = q_tok0; a.q = q; a.k_rot = k_rot; a.v = v; a.cs = cs; a.sel = sel; a.cnt = cnt; a.budget = budget;
   a.qb_begin = qb_begin; a.n_qb = qb_end - qb_begin; a.scale_log2 = scale_log2; a.out = out; a.lse = lse;
   a.err = err; a.n_split = 1;
   return launch_tc<false>(a, 2 * (qb_end - qb_begin), num_sms, stream);

@@ -90,7 +90,8 @@ struct Iter {
 __global__ void __launch_bounds__(THREADS, 1)
 indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const uint16_t* __restrict__ w, float* __restrict__ S, int64_t ld,
-                       float* __restrict__ segmax, int64_t ld_seg, int64_t T, int64_t qb_begin, int64_t qb_end,
+                       float* __restrict__ segmax, int64_t ld_seg, int64_t T, int64_t q_tok0, int64_t qb_begin,
+                       int64_t qb_end,
                        float scale, uint32_t* err) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* sQ = smem;
@@ -160,7 +161,7 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         for (int u = 0; u < 4; ++u) {
           const int64_t t = t_first + 4 * lane + u;
           uint2 raw = make_uint2(0u, 0u);
-          if (t < T) raw = __ldg(reinterpret_cast<const uint2*>(w + 4 * t));
+          if (t < T) raw = __ldg(reinterpret_cast<const uint2*>(w + 4 * (t - q_tok0)));
           wv[4 * u + 0] = bf16lo(raw.x); wv[4 * u + 1] = bf16hi(raw.x);
           wv[4 * u + 2] = bf16lo(raw.y); wv[4 * u + 3] = bf16hi(raw.y);
         }
@@ -180,7 +181,8 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
           mbar_arrive_expect_tx(qfull, Q_BYTES);
           for (int hf = 0; hf < 2; ++hf)
             for (int kc = 0; kc < 2; ++kc)
-              tma_load_2d(sQ + (hf * 2 + kc) * Q_SUB_BYTES, &tm_q, kc * 64, (int32_t)(4 * t_first + 256 * hf), qfull);
+              tma_load_2d(sQ + (hf * 2 + kc) * Q_SUB_BYTES, &tm_q, kc * 64, (int32_t)(4 * (t_first - q_tok0) + 256 * hf),
+                          qfull);
         }
         ++qcount;
       }
@@ -378,8 +380,9 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 }  // namespace
 
 cudaError_t launch_indexer_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const uint16_t* w,
-                                   float* S, int64_t ld, float* segmax, int64_t ld_seg, int64_t T, int64_t qb_begin,
-                                   int64_t qb_end, float scale, uint32_t* err, int num_sms, cudaStream_t stream) {
+                                   float* S, int64_t ld, float* segmax, int64_t ld_seg, int64_t T, int64_t q_tok0,
+                                   int64_t qb_begin, int64_t qb_end, float scale, uint32_t* err, int num_sms,
+                                   cudaStream_t stream) {
   if (qb_end <= qb_begin) return cudaSuccess;
   static bool attr_done[64] = {false};
   int dev = 0;
@@ -401,8 +404,8 @@ cudaError_t launch_indexer_prefill(const CUtensorMap& tm_q, const CUtensorMap& t
     units += tl / KT + 1;
   }
   const int grid = (int)(units < num_sms ? units : num_sms);
-  indexer_prefill_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tm_q, tm_k, w, S, ld, segmax, ld_seg, T, qb_begin,
-                                                                 qb_end, scale, err);
+  indexer_prefill_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tm_q, tm_k, w, S, ld, segmax, ld_seg, T, q_tok0,
+                                                                 qb_begin, qb_end, scale, err);
   return cudaGetLastError();
 }
 

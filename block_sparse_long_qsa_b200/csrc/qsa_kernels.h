@@ -15,10 +15,12 @@ cudaError_t launch_rope_k(int64_t T, const uint16_t* k, const float2* cs, uint16
 // Block scores of query blocks [qb_begin, qb_end) into S (row stride ld, only
 // kb <= qb written).  segmax (nullable, row stride ld_seg): per row, the max
 // over each segment of 8 key blocks (segment s = blocks 8s .. 8s+7, blocks
-// after the row's own block counting as 0).
+// after the row's own block counting as 0).  Keys are tokens [0, T) of tm_k;
+// the query rows (tm_q) and w start at token q_tok0 (<= 4 * qb_begin).
 cudaError_t launch_indexer_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const uint16_t* w,
-                                   float* S, int64_t ld, float* segmax, int64_t ld_seg, int64_t T, int64_t qb_begin,
-                                   int64_t qb_end, float scale, uint32_t* err, int num_sms, cudaStream_t stream);
+                                   float* S, int64_t ld, float* segmax, int64_t ld_seg, int64_t T, int64_t q_tok0,
+                                   int64_t qb_begin, int64_t qb_end, float scale, uint32_t* err, int num_sms,
+                                   cudaStream_t stream);
 
 // Top-k block selection, one row per query block.  Row r covers query block
 // row_qb ? row_qb[r] : qb_begin + r, read from S + r * ld.  segmax (nullable,
@@ -31,10 +33,13 @@ cudaError_t launch_select(const float* S, int64_t ld, const float* segmax, int64
 
 // Sparse GQA attention for query blocks [qb_begin, qb_end) given their
 // selections (sel/cnt indexed from qb_begin): tcgen05 kernel, persistent.
+// Keys k_rot / v are tokens [0, T); q, the RoPE table cs, out and lse start at
+// token q_tok0 (tokens before it in the first block get no output).
 cudaError_t launch_sparse_attn_prefill_tc(int64_t T, const uint16_t* q, const uint16_t* k_rot, const uint16_t* v,
                                           const float2* cs, const int32_t* sel, const int32_t* cnt, int budget,
-                                          int64_t qb_begin, int64_t qb_end, float scale_log2, uint16_t* out,
-                                          float* lse, uint32_t* err, int num_sms, cudaStream_t stream);
+                                          int64_t qb_begin, int64_t qb_end, int64_t q_tok0, float scale_log2,
+                                          uint16_t* out, float* lse, uint32_t* err, int num_sms,
+                                          cudaStream_t stream);
 
 // ---------------------------------------------------------------- decode
 // Lengths come from the host array L_host (passed to the kernel as launch

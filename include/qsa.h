@@ -128,6 +128,34 @@ qsa_status qsa_prefill(const qsa_params* p, int64_t T, int64_t pos0, const uint1
  * pointer may be NULL). */
 qsa_status qsa_prefill_workspace_size(const qsa_params* p, int64_t T, size_t* min_bytes, size_t* pref_bytes);
 
+/* Prefill of T_new new tokens after L_old tokens already in a cache (the
+ * prefix-cached serving case of [PT §QSA] "100만 토큰까지 늘리기": most of a
+ * long prompt is cached and only the rest is prefilled).  Equals the last
+ * T_new rows of qsa_prefill over all L_old + T_new tokens with pos0 = 0:
+ * the new tokens' query blocks qb = L_old/4 .. (L_old+T_new-1)/4 are scored
+ * over every key block up to their own, selected as in stage 2, and attend
+ * over the selected cached and new keys.
+ * Caches (bf16, at least L_old + T_new rows, rows [0, L_old) given):
+ *   k_cache [..][2][256] rotated keys, v_cache [..][2][256], kidx_cache
+ *   [..][128]; rows [L_old, L_old + T_new) are written by this call (the new
+ *   keys rotated at positions L_old ..), as a decode append would.
+ * qidx_prev [L_old % 4][4][128], w_prev [L_old % 4][4]: indexer queries and
+ *   head weights of the tokens 4*(L_old/4) .. L_old-1 that share the first
+ *   new query block (NULL allowed when L_old % 4 == 0).
+ * New tokens [T_new]: q [..][24][256], k, v [..][2][256] (k not rotated),
+ *   q_idx [..][4][128], w [..][4], k_idx [..][128].
+ * Outputs: out [T_new][24][256] bf16; lse [T_new][24] fp32 (nullable);
+ *   sel_out [nq][budget], cnt_out [nq] (nullable) for the nq new query blocks.
+ * ws: at least the minimum of qsa_prefill_cached_workspace_size. */
+qsa_status qsa_prefill_cached(const qsa_params* p, int64_t L_old, int64_t T_new, uint16_t* k_cache,
+                              uint16_t* v_cache, uint16_t* kidx_cache, const uint16_t* qidx_prev,
+                              const uint16_t* w_prev, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                              const uint16_t* q_idx, const uint16_t* w, const uint16_t* k_idx, uint16_t* out,
+                              float* lse, int32_t* sel_out, int32_t* cnt_out, void* ws, size_t ws_bytes,
+                              void* stream);
+qsa_status qsa_prefill_cached_workspace_size(const qsa_params* p, int64_t L_old, int64_t T_new, size_t* min_bytes,
+                                             size_t* pref_bytes);
+
 /* One decode step for B sequences.  Sequence b has cache_len[b] (host array)
  * tokens already in its caches; the new token sits at position
  * L = cache_len[b] and is appended: k_cache[b][L] = RoPE(k_new[b], L),
