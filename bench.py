@@ -243,6 +243,97 @@ def run_prefill(T: int, budget: int, steps: int, warmup: int, rank: int, world: 
 
 
 # ------------------------------------------------------------- decode workload
+def run_prefill_cached(T: int, L_old: int, budget: int, steps: int, warmup: int, rank: int, world: int, seed: int,
+                       want_e2e=True):
+    """Prefix-cached prefill: the first L_old tokens are in the caches, a step
+    prefills the remaining T - L_old (qsa_prefill_cached); every step rewrites
+    the same cache rows with the same values."""
+    import block_sparse_long_qsa_b200 as qsa
+    T_new = T - L_old
+    P = Q.PrefillProblem(T=T, seed=seed + 1000 * rank, n_plant=8, dist="zipf" if T >= 131072 else "uniform")
+    d = P.device()
+    # caches: synthetic keys stand in for rotated ones (timing only)
+    kc, vc, ic = d["k"].clone(), d["v"].clone(), d["k_idx"].clone()
+    t0 = 4 * (L_old // 4)
+    qprev, wprev = d["q_idx"][t0:L_old].clone(), d["w"][t0:L_old].clone()
+    new = {k: d[k][L_old:].clone() for k in ("q", "k", "v", "q_idx", "w", "k_idx")}
+    del d
+    torch.cuda.synchronize()
+    p = qsa.params(budget)
+    _, pref = qsa.qsa_prefill_cached_workspace_size(p, L_old, T_new)
+    ws = qsa.workspace(pref)
+    nq = (T + 3) // 4 - L_old // 4
+    out = torch.empty((T_new, 24, 256), dtype=torch.uint16, device="cuda")
+    sel = torch.empty((nq, budget), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((nq,), dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(x=None, o=None):
+        x = x or new
+        qsa.qsa_prefill_cached(p, L_old, T_new, kc, vc, ic, qprev if t0 < L_old else None,
+                               wprev if t0 < L_old else None, x["q"], x["k"], x["v"], x["q_idx"], x["w"], x["k_idx"],
+                               out if o is None else o, None, sel, cnt, ws, stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if qsa.qsa_check_device_error(ws) != 0:
+        raise RuntimeError("device error during warm-up")
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk, qsa.trace(capacity=64 * steps + 64) as tr:
+        ev0.record(stream)
+        for _ in range(steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_max = max_over_ranks(ev0.elapsed_time(ev1), world)
+    if qsa.qsa_check_device_error(ws) != 0:
+        raise RuntimeError("device error during the timed steps")
+    cnt_h = cnt.cpu().numpy().astype(np.int64)
+    # indexer: every token of the new query blocks against all earlier keys;
+    # attention: the new tokens over their selected keys
+    first = 4 * (L_old // 4)
+    fl_idx = 1024.0 * (T * (T + 1) / 2 - first * (first + 1) / 2)
+    keys = float(16 * cnt_h.sum()) - 6.0 * len(cnt_h)
+    fl_attn = 4.0 * 24 * 256 * keys * T_new / (T - first)
+    kern = tr.by_kernel()
+    res = dict(ms=ms_max, tokens=T_new * steps * world, kern=kern, launches=sum(c for c, _ in kern.values()),
+               clocks=clk.summary(), flops_idx=fl_idx, flops_attn=fl_attn, steps=steps)
+    if want_e2e:
+        # new tokens' inputs copied in from pinned host memory and the output
+        # copied back every step (serial; the cached prefix stays resident)
+        names = ["q", "k", "v", "q_idx", "w", "k_idx"]
+        host = {k: torch.empty(new[k].shape, dtype=new[k].dtype, pin_memory=True) for k in names}
+        for k in names:
+            host[k].copy_(new[k])
+        out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        dx = {k: torch.empty_like(new[k]) for k in names}
+        bi = sum(host[k].numel() * host[k].element_size() for k in names)
+        bo = out_h.numel() * out_h.element_size()
+        e_steps = max(2, min(steps, 4))
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            for k in names:
+                dx[k].copy_(host[k], non_blocking=True)
+            step(dx)
+            out_h.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        ems = max_over_ranks(e0.elapsed_time(e1), world)
+        res["e2e"] = dict(value=T_new * e_steps * world / (ems / 1e3), unit="tokens/s", h2d_bytes_per_step=bi,
+                          d2h_bytes_per_step=bo, steps=e_steps, pipelined=False)
+    del ws, kc, vc, ic, new
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, world: int, seed: int,
                want_e2e=True):
     import block_sparse_long_qsa_b200 as qsa
@@ -363,12 +454,13 @@ _KIDX_CACHE: dict = {}
 def cpu_sample(wl: dict, target_s: float = 12.0):
     """The oracle on a bounded sample of the workload sized to ~target_s of
     CPU time: a calibration run, then one run scaled to the target."""
-    if wl["kind"] == "prefill":
+    if wl["kind"] in ("prefill", "prefill_cached"):
+        qb_lo = wl.get("L_old", 0) // 4
         n = max(4, cores_used())
-        v, info = cpu_prefill_sample(wl["T"], 512, n)
+        v, info = cpu_prefill_sample(wl["T"], 512, n, qb_lo=qb_lo)
         if info["elapsed"] < target_s / 3:
-            n2 = int(min((wl["T"] + 3) // 4, max(n + 1, n * target_s / max(info["elapsed"], 1e-3))))
-            v, info = cpu_prefill_sample(wl["T"], 512, n2)
+            n2 = int(min((wl["T"] + 3) // 4 - qb_lo, max(n + 1, n * target_s / max(info["elapsed"], 1e-3))))
+            v, info = cpu_prefill_sample(wl["T"], 512, n2, qb_lo=qb_lo)
     else:
         n = 2
         v, info = cpu_decode_sample(wl["B"], wl["L"], 512, n)
@@ -378,15 +470,16 @@ def cpu_sample(wl: dict, target_s: float = 12.0):
     return v, info
 
 
-def cpu_prefill_sample(T: int, budget: int, n_blocks: int, seed: int = 0):
+def cpu_prefill_sample(T: int, budget: int, n_blocks: int, seed: int = 0, qb_lo: int = 0):
     """The oracle on a stratified sample of query blocks of the T-token
-    prefill (evenly spaced qb), all host cores.  Returns tokens/s of the
-    oracle extrapolated by the sample's share of the work, and a description."""
+    prefill (evenly spaced qb in [qb_lo, nqb)), all host cores.  Returns
+    tokens/s of the oracle extrapolated by the sample's share of the work, and
+    a description."""
     import oracle
     O = oracle.Oracle(oracle.params(budget=budget))
     P = Q.PrefillProblem(T=T, seed=seed, n_plant=8, dist="zipf" if T >= 131072 else "uniform")
     nqb = P.nqb
-    qbs = np.unique(np.linspace(0, nqb - 1, n_blocks).astype(np.int64))
+    qbs = np.unique(np.linspace(qb_lo, nqb - 1, n_blocks).astype(np.int64))
     key = (T, seed)
     if key not in _KIDX_CACHE:
         _KIDX_CACHE.clear()
@@ -421,7 +514,8 @@ def cpu_prefill_sample(T: int, budget: int, n_blocks: int, seed: int = 0):
     elapsed = t_score + t_attn
     # the sample is evenly spaced in qb, so its mean work matches the workload's
     tokens = 4 * len(qbs)
-    return tokens / elapsed, dict(sample=f"{len(qbs)} evenly spaced query blocks of the {T}-token prefill "
+    span = "" if qb_lo == 0 else f" from query block {qb_lo} on"
+    return tokens / elapsed, dict(sample=f"{len(qbs)} evenly spaced query blocks{span} of the {T}-token prefill "
                                          f"(scores + selection + attention), {elapsed:.1f} s",
                                   elapsed=elapsed)
 
@@ -470,6 +564,9 @@ WORKLOADS = {
     "prefill_128k": dict(kind="prefill", T=131072),
     "prefill_32k": dict(kind="prefill", T=32768),
     "decode_64x256k": dict(kind="decode", B=64, L=262144),
+    # 90 % of a 1M-token prompt already cached (L_old % 4 = 2: the first new
+    # query block starts mid-block)
+    "prefill_1m_cached90": dict(kind="prefill_cached", T=1 << 20, L_old=943718),
 }
 
 
@@ -479,9 +576,18 @@ WORKLOADS = {
 NCU_TRAFFIC = {"prefill_1m": 67.49e9 + 15.26e9}
 
 
+def metric_name(wl: dict) -> str:
+    if wl["kind"] == "prefill":
+        return f"QSA prefill tokens/s at {wl['T'] // 1024}K context"
+    if wl["kind"] == "prefill_cached":
+        return (f"QSA prefix-cached prefill new tokens/s at {wl['T'] // 1024}K context, "
+                f"{round(100 * wl['L_old'] / wl['T'])}% cached")
+    return "QSA decode tokens/s at 256K context, batch 64"
+
+
 def line_for(name, res, n_gpus, steps, warmup, pk):
     wl = WORKLOADS[name]
-    if wl["kind"] == "prefill":
+    if wl["kind"] in ("prefill", "prefill_cached"):
         T = wl["T"]
         value = res["tokens"] / (res["ms"] / 1e3)
         idx_n, idx_ms = res["kern"].get("indexer", (1, float("nan")))
@@ -493,10 +599,12 @@ def line_for(name, res, n_gpus, steps, warmup, pk):
         total_fl = res["flops_idx"] + res["flops_attn"]
         whole = dict(tflops=total_fl / (res["ms"] / res["steps"] / 1e3) / 1e12)
         whole["frac_of_tensor_roofline"] = whole["tflops"] / pk["bf16_sus"]
-        metric = f"QSA prefill tokens/s at {T // 1024}K context"
+        metric = metric_name(wl)
         cfg = dict(workload=name, T=T, batch=1, budget_blocks=512, heads="24q/2kv x 256, idx 4 x 128",
                    planted="8/query block, " + ("zipf(1.1) distance" if T >= 131072 else "uniform"),
                    l2="inputs larger than L2 (126 MB): no flush needed")
+        if "L_old" in wl:
+            cfg.update(cached_tokens=wl["L_old"], new_tokens=T - wl["L_old"])
     else:
         B, L = wl["B"], wl["L"]
         value = res["tokens"] / (res["ms"] / 1e3)
@@ -582,8 +690,7 @@ def main():
             descs.append(info["sample"])
         value = statistics.median(ts)
         cb = dict(value=value, unit="tokens/s", cores=cores_used(), kind="oracle", sample=descs[0])
-        metric = (f"QSA prefill tokens/s at {wl['T'] // 1024}K context" if wl["kind"] == "prefill"
-                  else "QSA decode tokens/s at 256K context, batch 64")
+        metric = metric_name(wl)
         print(json.dumps(dict(impl="reference", metric=metric, value=value, unit="tokens/s", n_gpus=args.gpus,
                               steps=args.steps, warmup=args.warmup, ms_per_step=None, higher_is_better=True,
                               scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
@@ -599,6 +706,9 @@ def main():
     wl = WORKLOADS[args.workload]
     if wl["kind"] == "prefill":
         res = run_prefill(wl["T"], 512, args.steps, args.warmup, rank, world, seed=0, want_e2e=not args.no_e2e)
+    elif wl["kind"] == "prefill_cached":
+        res = run_prefill_cached(wl["T"], wl["L_old"], 512, args.steps, args.warmup, rank, world, seed=0,
+                                 want_e2e=not args.no_e2e)
     else:
         res = run_decode(wl["B"], wl["L"], 512, args.steps, args.warmup, rank, world, seed=0,
                          want_e2e=not args.no_e2e)
@@ -606,12 +716,15 @@ def main():
 
     if not args.no_secondary:
         sec = {}
-        for name in ("decode_64x256k", "prefill_128k"):
+        for name in ("decode_64x256k", "prefill_128k", "prefill_1m_cached90"):
             if name == args.workload:
                 continue
             w2 = WORKLOADS[name]
             if w2["kind"] == "prefill":
                 r2 = run_prefill(w2["T"], 512, args.steps, args.warmup, rank, world, seed=0, want_e2e=False)
+            elif w2["kind"] == "prefill_cached":
+                r2 = run_prefill_cached(w2["T"], w2["L_old"], 512, args.steps, args.warmup, rank, world, seed=0,
+                                        want_e2e=False)
             else:
                 r2 = run_decode(w2["B"], w2["L"], 512, args.steps, args.warmup, rank, world, seed=0,
                                 want_e2e=False)
