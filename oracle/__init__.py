@@ -21,13 +21,18 @@ class Params(ctypes.Structure):
     _fields_ = [("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("rope_dim", ctypes.c_int32), ("rope_theta", ctypes.c_double), ("idx_heads", ctypes.c_int32),
                 ("idx_dim", ctypes.c_int32), ("block", ctypes.c_int32), ("budget", ctypes.c_int32),
-                ("softmax_scale", ctypes.c_double)]
+                ("softmax_scale", ctypes.c_double), ("aggregation", ctypes.c_int32)]
+
+
+# block-score aggregation: max over causal token pairs, or mean-pooled block keys
+AGG_TOKEN_MAX = 0
+AGG_MEAN_POOL = 1
 
 
 def params(budget=512, block=4, n_q_heads=24, n_kv_heads=2, head_dim=256, rope_dim=64, rope_theta=1e7,
-           idx_heads=4, idx_dim=128, softmax_scale=0.0) -> Params:
+           idx_heads=4, idx_dim=128, softmax_scale=0.0, aggregation=AGG_TOKEN_MAX) -> Params:
     return Params(n_q_heads, n_kv_heads, head_dim, rope_dim, rope_theta, idx_heads, idx_dim, block, budget,
-                  softmax_scale)
+                  softmax_scale, aggregation)
 
 
 def build(force: bool = False) -> str:

@@ -47,6 +47,8 @@ typedef struct {
   int32_t block;       /* r = 4 [PT §QSA, "r = 4"] */
   int32_t budget;      /* 512 blocks = 2048 tokens [PT spec table, "QSA 예산"] */
   double softmax_scale;/* 0 => 1/sqrt(head_dim) */
+  int32_t aggregation; /* 0: max over causal token pairs (the stated block score);
+                          1: mean-pooled block keys [PT §QSA, I_ib over k-bar_b] */
 } oracle_params;
 
 static double bf16_to_f64(uint16_t h) {
@@ -87,6 +89,35 @@ double oracle_token_score(const oracle_params* p, const uint16_t* q_t, const uin
   return s / sqrt((double)p->idx_dim);
 }
 
+/* fp64 -> bf16 bit pattern, round to nearest even, subnormals included. */
+static uint16_t f64_to_bf16_rne(double x) {
+  union { double d; uint64_t u; } b;
+  b.d = x;
+  const uint16_t sign = (uint16_t)((b.u >> 48) & 0x8000u);
+  const double a = fabs(x);
+  if (a == 0.0) return sign;
+  int e;
+  frexp(a, &e);                                   /* a = m 2^e, m in [0.5, 1) */
+  const int unit = e - 8 > -133 ? e - 8 : -133;   /* weight of bf16's last bit */
+  const double v = ldexp(nearbyint(ldexp(a, -unit)), unit);
+  union { float f; uint32_t u; } c;
+  c.f = (float)v;                                 /* exact: <= 8 significant bits */
+  return (uint16_t)(sign | (c.u >> 16));
+}
+
+/* Compressed key of block kb ([PT] §QSA: the keys of a micro-block are
+ * mean-pooled into k-bar_b before any positional step; the indexer has no
+ * positional encoding here, so no block position is added).  Mean over the
+ * block's n present keys: exact fp64 sum, one fp64 division by n, one
+ * rounding to bf16 (the indexer's operands are bf16). */
+static void mean_key(const oracle_params* p, const uint16_t* k_idx, int64_t kb, int n, double* kbar) {
+  for (int c = 0; c < p->idx_dim; ++c) {
+    double sum = 0.0;
+    for (int i = 0; i < n; ++i) sum += bf16_to_f64(k_idx[(kb * p->block + i) * p->idx_dim + c]);
+    kbar[c] = bf16_to_f64(f64_to_bf16_rne(sum / (double)n));
+  }
+}
+
 /* ----------------------------------------------------------- block score --
  * S(qb, kb) for kb = 0..qb: max over present tokens t of block qb and keys
  * j of block kb with j <= t of s(t, j) ([PT] §QSA: micro-blocks of r tokens,
@@ -96,6 +127,30 @@ double oracle_token_score(const oracle_params* p, const uint16_t* q_t, const uin
 void oracle_block_scores(const oracle_params* p, int64_t qb, int n_present, const uint16_t* q_blk,
                          const uint16_t* w_blk, const uint16_t* k_idx, double* S) {
   int r = p->block;
+  if (p->aggregation == 1) {
+    /* mean pooling: S(qb, kb) = max over present t of block qb of
+     *   sum_h w_h(t) ReLU(q_idx_h(t) . k-bar_kb) / sqrt(idx_dim);
+     * k-bar of the own block averages its present keys (the own block is
+     * always selected, so this entry never decides a selection) */
+    double kbar[512];
+    for (int64_t kb = 0; kb <= qb; ++kb) {
+      mean_key(p, k_idx, kb, kb == qb ? n_present : r, kbar);
+      double best = -INFINITY;
+      for (int i = 0; i < n_present; ++i) {
+        const uint16_t* q_t = q_blk + (int64_t)i * p->idx_heads * p->idx_dim;
+        double s = 0.0;
+        for (int h = 0; h < p->idx_heads; ++h) {
+          double dot = 0.0;
+          for (int c = 0; c < p->idx_dim; ++c) dot += bf16_to_f64(q_t[h * p->idx_dim + c]) * kbar[c];
+          s += bf16_to_f64(w_blk[(int64_t)i * p->idx_heads + h]) * (dot > 0.0 ? dot : 0.0);
+        }
+        s /= sqrt((double)p->idx_dim);
+        if (s > best) best = s;
+      }
+      S[kb] = best;
+    }
+    return;
+  }
   for (int64_t kb = 0; kb <= qb; ++kb) {
     double best = -INFINITY;
     for (int i = 0; i < n_present; ++i) {

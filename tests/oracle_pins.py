@@ -154,6 +154,121 @@ def pin_identical_keys_block(O):
         assert abs(S[qb, qb] - want) < 1e-14 * (1 + want)
 
 
+# ------------------------------------------------ mean-pooled block keys (f2)
+def _bf16_rne_exact(x) -> float:
+    """Round a rational to the nearest bf16 value (ties to even), by integer
+    arithmetic on its exact value (fractions), independent of any float path."""
+    from fractions import Fraction
+    x = Fraction(x)
+    if x == 0:
+        return 0.0
+    sign = -1 if x < 0 else 1
+    a = abs(x)
+    e = a.numerator.bit_length() - a.denominator.bit_length()   # 2^e <= a < 2^(e+2)
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    unit = max(e - 7, -133)                 # 8 significant bits; bf16 subnormals below 2^-126
+    q = a / Fraction(2) ** unit
+    n = q.numerator // q.denominator
+    rem = q - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    return sign * float(Fraction(n) * Fraction(2) ** unit)
+
+
+def _mean_pool_scores(q_idx, w, k_idx, r=4):
+    """S(qb, kb) with mean-pooled block keys, all in numpy / exact rationals:
+    kbar = bf16 of the mean of the block's present keys (mean: exact sum, one
+    fp64 division), score = max over the block's tokens."""
+    from fractions import Fraction
+    T = q_idx.shape[0]
+    nb = (T + r - 1) // r
+    kf = Q.bf16_to_f64(k_idx)
+    kbar = np.zeros((nb, kf.shape[1]))
+    for b in range(nb):
+        rows = kf[b * r: min(b * r + r, T)]
+        n = rows.shape[0]
+        for c in range(kf.shape[1]):
+            exact_sum = sum(Fraction(float(v)) for v in rows[:, c])
+            mean64 = float(exact_sum) / n          # the sum is exact in fp64; one division
+            kbar[b, c] = _bf16_rne_exact(mean64)
+    qf, wf = Q.bf16_to_f64(q_idx), Q.bf16_to_f64(w)
+    dots = np.einsum("thc,bc->thb", qf, kbar)
+    s = (wf[:, :, None] * np.maximum(dots, 0.0)).sum(1) / SQRT_D   # [T][nb]
+    S = np.full((nb, nb), np.nan)
+    for qb in range(nb):
+        S[qb, :qb + 1] = s[qb * r: min(qb * r + r, T), :qb + 1].max(axis=0)
+    return S
+
+
+def _mean_pool_oracle(O):
+    import oracle as OR
+    return type(O)(OR.params(budget=O.P.budget, aggregation=OR.AGG_MEAN_POOL), O.L)
+
+
+def pin_mean_pool_brute(O):
+    """Mean-pooled scores equal an independent brute force (exact rational
+    rounding of the block means, numpy dot products), ragged tails included."""
+    Om = _mean_pool_oracle(O)
+    for T, seed in ((1, 0), (6, 1), (29, 2), (67, 3)):
+        P = Q.PrefillProblem(T=T, seed=40 + seed, n_plant=2)
+        q_idx, w, k_idx = P.q_idx(), P.w(), P.k_idx()
+        want = _mean_pool_scores(q_idx, w, k_idx)
+        got = Om.index_scores(T, q_idx, w, k_idx)
+        m = ~np.isnan(want)
+        assert np.allclose(got[m], want[m], rtol=1e-12, atol=1e-14), T
+
+
+def pin_mean_pool_relations(O):
+    """Closed forms: a block of four identical keys has that key as its mean,
+    so its mean-pool score is the token-pair score; keys k, -k, k, -k average
+    to 0 and score 0; keys 1, 2, 3, 4 times k average to 2.5 k."""
+    Om = _mean_pool_oracle(O)
+    T = 24
+    P = Q.PrefillProblem(T=T, seed=9)
+    q_idx, w, k_idx = P.q_idx(), P.w(), P.k_idx().copy()
+    k_idx[4:8] = k_idx[6]
+    base = _bf(np.full(128, 0.5, np.float32))
+    k_idx[8:12] = np.stack([base, _bf(-Q.bf16_to_f32(base)), base, _bf(-Q.bf16_to_f32(base))])
+    unit = _bf(np.full(128, 0.25, np.float32))
+    k_idx[12:16] = np.stack([_bf(Q.bf16_to_f32(unit) * m) for m in (1, 2, 3, 4)])
+    Sm = Om.index_scores(T, q_idx, w, k_idx)
+    Sp = O.index_scores(T, q_idx, w, k_idx)
+    for qb in (2, 3, 4, 5):
+        assert abs(Sm[qb, 1] - Sp[qb, 1]) < 1e-13 * (1 + Sp[qb, 1]), qb
+        assert Sm[qb, 2] == 0.0, qb
+        qf, wf = Q.bf16_to_f64(q_idx), Q.bf16_to_f64(w)
+        if qb >= 3:
+            kb3 = np.full(128, 0.625)
+            want = max((wf[t] * np.maximum(qf[t] @ kb3, 0.0)).sum() / SQRT_D for t in range(4 * qb, 4 * qb + 4))
+            assert abs(Sm[qb, 3] - want) < 1e-12 * (1 + want), qb
+
+
+def pin_bf16_rounding_of_means(O):
+    """The block mean is rounded to bf16 once, to nearest even: a mean exactly
+    half-way between two bf16 values goes to the even one, and one just above
+    half-way goes up."""
+    Om = _mean_pool_oracle(O)
+    T = 8
+    P = Q.PrefillProblem(T=T, seed=12)
+    q_idx, w = P.q_idx(), P.w()
+    q_idx[4:8] = 0
+    q_idx[4:8, 0, 0] = _bf(np.float32(1.0))       # score = w0 * ReLU(kbar[0]) / sqrt(128)
+    k_idx = np.zeros((T, 128), np.uint16)
+    # 1 + 2^-8 is half-way between 1 and 1 + 2^-7: keys 1, 1, 1 + 2^-7, 1 + 2^-7 -> ties to even = 1
+    a, b = np.float32(1.0), np.float32(1.0 + 2 ** -7)
+    k_idx[0:4, 0] = _bf(np.array([a, a, b, b]))
+    S = Om.index_scores(T, q_idx, w, k_idx)
+    wf = Q.bf16_to_f64(w)
+    assert abs(S[1, 0] - max(wf[t, 0] for t in range(4, 8)) * 1.0 / SQRT_D) < 1e-15
+    # keys 1, 1, 1 + 2^-7, 1 + 2^-6: mean 1 + 3 * 2^-9 (above half-way) -> 1 + 2^-7
+    k_idx[3, 0] = _bf(np.float32(1.0 + 2 ** -6))
+    S = Om.index_scores(T, q_idx, w, k_idx)
+    assert abs(S[1, 0] - max(wf[t, 0] for t in range(4, 8)) * (1.0 + 2 ** -7) / SQRT_D) < 1e-15
+
+
 # ---------------------------------------------------------------- selection
 def _select_lexsort(S_row, qb, budget):
     if qb + 1 <= budget:

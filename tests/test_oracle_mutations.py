@@ -32,6 +32,11 @@ MUTANTS = [
     ("causal_attn_off_by_one", "if (j <= t) js[n++] = j;", "if (j <= t + 1) js[n++] = j;"),
     ("value_head_swap", "vv[(e * G + g) * d + c] = bf16_to_f64(v[(js[e] * G + g) * d + c]);",
      "vv[(e * G + g) * d + c] = bf16_to_f64(v[(js[e] * G + (G - 1 - g)) * d + c]);"),
+    ("mean_not_divided", "f64_to_bf16_rne(sum / (double)n)", "f64_to_bf16_rne(sum)"),
+    ("mean_not_rounded_to_bf16", "kbar[c] = bf16_to_f64(f64_to_bf16_rne(sum / (double)n));", "kbar[c] = sum / (double)n;"),
+    ("mean_ties_away_from_zero", "ldexp(nearbyint(ldexp(a, -unit)), unit)", "ldexp(round(ldexp(a, -unit)), unit)"),
+    ("mean_pool_relu_dropped", "s += bf16_to_f64(w_blk[(int64_t)i * p->idx_heads + h]) * (dot > 0.0 ? dot : 0.0);",
+     "s += bf16_to_f64(w_blk[(int64_t)i * p->idx_heads + h]) * dot;"),
     ("decode_new_key_position", "oracle_rope(p, x, L, kr + (e * G + g) * d);", "oracle_rope(p, x, L - 1, kr + (e * G + g) * d);"),
 ]
 
