@@ -25,10 +25,12 @@ _STATUS = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_UNSUPPORTED", 3: "
 EXPORTED = ["qsa_default_params", "qsa_status_string", "qsa_last_error", "qsa_index_scores", "qsa_select_blocks",
             "qsa_select_workspace_size", "qsa_prefill", "qsa_prefill_workspace_size", "qsa_decode",
             "qsa_decode_workspace_size", "qsa_check_device_error", "qsa_trace_begin", "qsa_trace_end",
-            "qsa_decode_noalloc", "qsa_prefill_cached", "qsa_prefill_cached_workspace_size"]
+            "qsa_decode_noalloc", "qsa_prefill_cached", "qsa_prefill_cached_workspace_size",
+            "qsa_index_workspace_size"]
 
 KERNEL_NAMES = {1: "rope_table", 2: "rope_k", 3: "indexer", 4: "select", 5: "attention", 6: "decode_append",
-                7: "decode_indexer", 8: "decode_attention", 9: "decode_combine"}
+                7: "decode_indexer", 8: "decode_attention", 9: "decode_combine",
+                10: "mean_pool_keys"}
 
 
 class QSAError(RuntimeError):
@@ -41,8 +43,12 @@ class qsa_params(ctypes.Structure):
     _fields_ = [("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("rope_dim", ctypes.c_int32), ("rope_theta", ctypes.c_double), ("idx_heads", ctypes.c_int32),
                 ("idx_dim", ctypes.c_int32), ("block_size", ctypes.c_int32), ("budget_blocks", ctypes.c_int32),
-                ("softmax_scale", ctypes.c_float)]
+                ("softmax_scale", ctypes.c_float), ("aggregation", ctypes.c_int32)]
 
+
+# block-score aggregation (qsa_params.aggregation)
+AGG_TOKEN_MAX = 0
+AGG_MEAN_POOL = 1
 
 _lib = None
 
@@ -67,6 +73,7 @@ def load(path: str = LIB_PATH):
     L.qsa_index_scores.argtypes = [P, i64, vp, vp, vp, i64, i64, vp, i64, vp, sz, vp]
     L.qsa_select_blocks.argtypes = [P, vp, i64, i64, i64, vp, vp, vp, sz, vp]
     L.qsa_select_workspace_size.argtypes = [P, psz]
+    L.qsa_index_workspace_size.argtypes = [P, i64, psz]
     L.qsa_prefill.argtypes = [P, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.qsa_prefill_workspace_size.argtypes = [P, i64, psz, psz]
     L.qsa_prefill_cached.argtypes = [P, i64, i64] + [vp] * 16 + [sz, vp]
@@ -117,6 +124,12 @@ def _check(rc: int, where: str):
 # ------------------------------------------------------------ raw entry points
 def qsa_status_string(status: int) -> str:
     return load().qsa_status_string(status).decode()
+
+
+def qsa_index_workspace_size(p: qsa_params, T: int) -> int:
+    n = ctypes.c_size_t()
+    _check(load().qsa_index_workspace_size(ctypes.byref(p), T, ctypes.byref(n)), "qsa_index_workspace_size")
+    return n.value
 
 
 def qsa_index_scores(p: qsa_params, T: int, q_idx, w, k_idx, qb_begin: int, qb_end: int, scores, ld: int,
@@ -233,11 +246,11 @@ def workspace(nbytes: int, device="cuda") -> torch.Tensor:
 
 
 def prefill(q, k, v, q_idx, w, k_idx, budget: int = 512, pos0: int = 0, want_lse=True, want_sel=True,
-            want_krot=False, ws_bytes: int | None = None, stream=None):
+            want_krot=False, ws_bytes: int | None = None, stream=None, aggregation: int = AGG_TOKEN_MAX):
     """Allocate outputs and a workspace, run qsa_prefill; returns a dict."""
     T = q.shape[0]
     dev = q.device
-    p = params(budget)
+    p = params(budget, aggregation=aggregation)
     mn, pref = qsa_prefill_workspace_size(p, T)
     ws = workspace(pref if ws_bytes is None else max(ws_bytes, mn), dev)
     nqb = (T + 3) // 4

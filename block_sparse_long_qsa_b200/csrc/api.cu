@@ -38,8 +38,13 @@ qsa_status check_params(const qsa_params* p) {
   if (!(p->rope_theta > 1.0) || !std::isfinite(p->rope_theta)) return QSA_ERR_INVALID_ARG;
   if (p->budget_blocks < 2 || p->budget_blocks > 4096) return QSA_ERR_UNSUPPORTED;
   if (!(p->softmax_scale >= 0.f) || !std::isfinite(p->softmax_scale)) return QSA_ERR_INVALID_ARG;
+  if (p->aggregation != QSA_AGG_TOKEN_MAX && p->aggregation != QSA_AGG_MEAN_POOL) return QSA_ERR_INVALID_ARG;
   return QSA_OK;
 }
+
+bool mean_pool(const qsa_params* p) { return p->aggregation == QSA_AGG_MEAN_POOL; }
+// bytes of the mean-pooled keys of T tokens ([ceil(T/4)][128] bf16)
+size_t kbar_bytes(int64_t T) { return (size_t)((T + 3) / 4) * 256; }
 
 float softmax_scale(const qsa_params* p) {
   return p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt((float)p->head_dim);
@@ -151,27 +156,39 @@ qsa_status from_cuda(cudaError_t e, const char* where = "kernel launch") {
 }
 
 // Indexer launch for query blocks [qb0, qb1) into S (ld), maps built here.
-// Keys: tokens [0, T) of k_idx; q_idx / w hold tokens [q_tok0, T).
+// Keys: tokens [0, T) of k_idx; q_idx / w hold tokens [q_tok0, T).  With kbar
+// (mean pooling) the compressed keys [ceil(T/4)][128], already computed, are
+// scored instead.
 qsa_status run_indexer(int64_t T, int64_t q_tok0, const uint16_t* q_idx, const uint16_t* w, const uint16_t* k_idx,
-                       int64_t qb0, int64_t qb1, float* S, int64_t ld, float* segmax, int64_t ld_seg, uint32_t* err,
-                       int num_sms, cudaStream_t st) {
+                       const uint16_t* kbar, int64_t qb0, int64_t qb1, float* S, int64_t ld, float* segmax,
+                       int64_t ld_seg, uint32_t* err, int num_sms, cudaStream_t st) {
   if (qb1 <= qb0) return QSA_OK;
   CUtensorMap tq, tk;
   qsa_status rs;
   if ((rs = make_map_2d(&tq, q_idx, (uint64_t)(T - q_tok0) * 4, 128, 256, 64)) != QSA_OK) return rs;
-  if ((rs = make_map_2d(&tk, k_idx, (uint64_t)T, 128, 128, 64)) != QSA_OK) return rs;
+  if (kbar) {
+    if ((rs = make_map_2d(&tk, kbar, (uint64_t)((T + 3) / 4), 128, 128, 64)) != QSA_OK) return rs;
+  } else if ((rs = make_map_2d(&tk, k_idx, (uint64_t)T, 128, 128, 64)) != QSA_OK) {
+    return rs;
+  }
   const float scale = 1.0f / std::sqrt(128.0f);
   return from_cuda(traced(QSA_KERNEL_INDEXER, st, [&] {
-    return qsa::launch_indexer_prefill(tq, tk, w, S, ld, segmax, ld_seg, T, q_tok0, qb0, qb1, scale, err, num_sms,
-                                       st);
+    return qsa::launch_indexer_prefill(tq, tk, w, S, ld, segmax, ld_seg, T, q_tok0, qb0, qb1, kbar != nullptr, scale,
+                                       err, num_sms, st);
   }), "indexer launch");
+}
+
+// Compressed keys of tokens [0, T) into kbar (mean pooling only).
+qsa_status run_kbar(const uint16_t* k_idx, int64_t T, uint16_t* kbar, cudaStream_t st) {
+  return from_cuda(traced(QSA_KERNEL_KBAR, st, [&] { return qsa::launch_kbar(k_idx, T, kbar, st); }),
+                   "mean-pool launch");
 }
 
 // ------------------------------------------------------------ prefill layout
 struct PrefillLayout {
-  size_t cs, k_rot, sel, cnt, slab, total_fixed;
+  size_t cs, k_rot, sel, cnt, kbar, slab, total_fixed;
 };
-PrefillLayout prefill_layout(int64_t T, int budget, bool need_krot, bool need_sel, bool need_cnt) {
+PrefillLayout prefill_layout(int64_t T, int budget, bool need_krot, bool need_sel, bool need_cnt, bool mean) {
   const int64_t nqb = (T + 3) / 4;
   PrefillLayout L;
   size_t off = HEADER_BYTES;
@@ -179,6 +196,7 @@ PrefillLayout prefill_layout(int64_t T, int budget, bool need_krot, bool need_se
   L.k_rot = off; off = align_up(off + (need_krot ? (size_t)T * 1024 : 0));
   L.sel = off; off = align_up(off + (need_sel ? (size_t)nqb * budget * 4 : 0));
   L.cnt = off; off = align_up(off + (need_cnt ? (size_t)nqb * 4 : 0));
+  L.kbar = off; off = align_up(off + (mean ? kbar_bytes(T) : 0));
   L.slab = off;
   L.total_fixed = off;
   return L;
@@ -215,6 +233,7 @@ void qsa_default_params(qsa_params* p) {
   p->block_size = 4;
   p->budget_blocks = 512;
   p->softmax_scale = 0.f;
+  p->aggregation = QSA_AGG_TOKEN_MAX;
 }
 
 const char* qsa_last_error(void) { return g_last_error; }
@@ -244,14 +263,27 @@ qsa_status qsa_index_scores(const qsa_params* p, int64_t T, const uint16_t* q_id
   if (qb_begin < 0 || qb_end < qb_begin || qb_end > nqb || ld < qb_end || ld % 4 != 0) return QSA_ERR_INVALID_ARG;
   if (!q_idx || !w || !k_idx || !scores) return QSA_ERR_INVALID_ARG;
   if (!aligned16(q_idx) || !aligned16(w) || !aligned16(k_idx) || !aligned16(scores)) return QSA_ERR_MISALIGNED;
-  if (ws && ws_bytes < HEADER_BYTES) return QSA_ERR_WORKSPACE_TOO_SMALL;
+  const bool mp = mean_pool(p);
+  if (mp && !ws) return QSA_ERR_INVALID_ARG;
+  if (ws && ws_bytes < HEADER_BYTES + (mp ? kbar_bytes(T) : 0)) return QSA_ERR_WORKSPACE_TOO_SMALL;
   if (ws && !aligned16(ws)) return QSA_ERR_MISALIGNED;
   DevInfo di;
   if ((st = device_info(&di)) != QSA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t* err = static_cast<uint32_t*>(ws);
   if (err && cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaMemsetAsync");
-  return run_indexer(T, 0, q_idx, w, k_idx, qb_begin, qb_end, scores, ld, nullptr, 0, err, di.num_sms, s);
+  uint16_t* kbar = mp ? reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + HEADER_BYTES) : nullptr;
+  if (kbar && (st = run_kbar(k_idx, T, kbar, s)) != QSA_OK) return st;
+  return run_indexer(T, 0, q_idx, w, k_idx, kbar, qb_begin, qb_end, scores, ld, nullptr, 0, err, di.num_sms, s);
+}
+
+qsa_status qsa_index_workspace_size(const qsa_params* p, int64_t T, size_t* bytes) {
+  qsa_status st = check_params(p);
+  if (st != QSA_OK) return st;
+  if (T <= 0 || !bytes) return QSA_ERR_INVALID_ARG;
+  if (T > ((int64_t)1 << 24)) return QSA_ERR_UNSUPPORTED;
+  *bytes = HEADER_BYTES + (mean_pool(p) ? kbar_bytes(T) : 0);
+  return QSA_OK;
 }
 
 qsa_status qsa_select_workspace_size(const qsa_params* p, size_t* bytes) {
@@ -288,7 +320,7 @@ qsa_status qsa_prefill_workspace_size(const qsa_params* p, int64_t T, size_t* mi
   if (T > ((int64_t)1 << 24)) return QSA_ERR_UNSUPPORTED;
   const int64_t nqb = (T + 3) / 4;
   // worst case: the library keeps k_rot, sel and cnt itself
-  PrefillLayout L = prefill_layout(T, p->budget_blocks, true, true, true);
+  PrefillLayout L = prefill_layout(T, p->budget_blocks, true, true, true, mean_pool(p));
   const int64_t min_rows = nqb < MIN_ROWS ? nqb : MIN_ROWS;
   const size_t row_bytes = slab_row_bytes(nqb);
   if (min_bytes) *min_bytes = L.total_fixed + (size_t)min_rows * row_bytes;
@@ -315,7 +347,8 @@ qsa_status qsa_prefill(const qsa_params* p, int64_t T, int64_t pos0, const uint1
     if (ptr && !aligned16(ptr)) return QSA_ERR_MISALIGNED;
   const int budget = p->budget_blocks;
   const int64_t nqb = (T + 3) / 4;
-  PrefillLayout L = prefill_layout(T, budget, k_rot_out == nullptr, sel_out == nullptr, cnt_out == nullptr);
+  PrefillLayout L = prefill_layout(T, budget, k_rot_out == nullptr, sel_out == nullptr, cnt_out == nullptr,
+                                   mean_pool(p));
   if (ws_bytes < L.total_fixed) return QSA_ERR_WORKSPACE_TOO_SMALL;
   const size_t slab_bytes = ws_bytes - L.total_fixed;
   const int64_t min_rows = nqb < MIN_ROWS ? nqb : MIN_ROWS;
@@ -340,6 +373,8 @@ qsa_status qsa_prefill(const qsa_params* p, int64_t T, int64_t pos0, const uint1
     return st;
   if ((st = from_cuda(traced(QSA_KERNEL_ROPE_K, s, [&] { return qsa::launch_rope_k(T, k, cs, k_rot, s); }))) != QSA_OK)
     return st;
+  uint16_t* kbar = mean_pool(p) ? reinterpret_cast<uint16_t*>(base + L.kbar) : nullptr;
+  if (kbar && (st = run_kbar(k_idx, T, kbar, s)) != QSA_OK) return st;
   const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
   for (int64_t qb0 = 0; qb0 < nqb;) {
     const int64_t qb1 = chunk_end(qb0, nqb, slab_bytes);
@@ -347,7 +382,8 @@ qsa_status qsa_prefill(const qsa_params* p, int64_t T, int64_t pos0, const uint1
     const int64_t ld = round4(qb1);
     const int64_t ld_seg = round4((qb1 + 7) / 8);
     float* segmax = slab + (size_t)(qb1 - qb0) * ld;
-    if ((st = run_indexer(T, 0, q_idx, w, k_idx, qb0, qb1, slab, ld, segmax, ld_seg, err, di.num_sms, s)) != QSA_OK)
+    if ((st = run_indexer(T, 0, q_idx, w, k_idx, kbar, qb0, qb1, slab, ld, segmax, ld_seg, err, di.num_sms, s)) !=
+        QSA_OK)
       return st;
     if ((st = from_cuda(traced(QSA_KERNEL_SELECT, s, [&] {
            return qsa::launch_select(slab, ld, segmax, ld_seg, qb0, qb1 - qb0, nullptr, budget, sel + qb0 * budget,
@@ -367,11 +403,11 @@ qsa_status qsa_prefill(const qsa_params* p, int64_t T, int64_t pos0, const uint1
 // --------------------------------------------------------- cached prefill
 namespace {
 struct CachedLayout {
-  size_t cs, qst, wst, sel, cnt, slab, total_fixed;
+  size_t cs, qst, wst, sel, cnt, kbar, slab, total_fixed;
 };
 // r = L_old % 4 tokens of the partial block before the new ones are staged
 // in front of the new tokens' q_idx / w (nothing is staged when r == 0).
-CachedLayout cached_layout(int64_t L_old, int64_t T_new, int budget, bool need_sel, bool need_cnt) {
+CachedLayout cached_layout(int64_t L_old, int64_t T_new, int budget, bool need_sel, bool need_cnt, bool mean) {
   const int64_t r = L_old % 4;
   const int64_t nq = (L_old + T_new - 1) / 4 - L_old / 4 + 1;
   CachedLayout L;
@@ -381,6 +417,7 @@ CachedLayout cached_layout(int64_t L_old, int64_t T_new, int budget, bool need_s
   L.wst = off; off = align_up(off + (r ? (size_t)(r + T_new) * 4 * 2 : 0));
   L.sel = off; off = align_up(off + (need_sel ? (size_t)nq * budget * 4 : 0));
   L.cnt = off; off = align_up(off + (need_cnt ? (size_t)nq * 4 : 0));
+  L.kbar = off; off = align_up(off + (mean ? kbar_bytes(L_old + T_new) : 0));
   L.slab = off;
   L.total_fixed = off;
   return L;
@@ -394,7 +431,7 @@ qsa_status qsa_prefill_cached_workspace_size(const qsa_params* p, int64_t L_old,
   if (L_old < 0 || T_new <= 0) return QSA_ERR_INVALID_ARG;
   if (L_old + T_new > ((int64_t)1 << 24)) return QSA_ERR_UNSUPPORTED;
   const int64_t nkb = (L_old + T_new + 3) / 4, qbA = L_old / 4, nq = nkb - qbA;
-  CachedLayout L = cached_layout(L_old, T_new, p->budget_blocks, true, true);
+  CachedLayout L = cached_layout(L_old, T_new, p->budget_blocks, true, true, mean_pool(p));
   const int64_t min_rows = nq < MIN_ROWS ? nq : MIN_ROWS;
   const size_t row_bytes = slab_row_bytes(nkb);
   if (min_bytes) *min_bytes = L.total_fixed + (size_t)min_rows * row_bytes;
@@ -426,7 +463,7 @@ qsa_status qsa_prefill_cached(const qsa_params* p, int64_t L_old, int64_t T_new,
   const int budget = p->budget_blocks;
   const int64_t T = L_old + T_new;               // keys: tokens [0, T)
   const int64_t nkb = (T + 3) / 4, qbA = L_old / 4, nq = nkb - qbA;
-  CachedLayout L = cached_layout(L_old, T_new, budget, sel_out == nullptr, cnt_out == nullptr);
+  CachedLayout L = cached_layout(L_old, T_new, budget, sel_out == nullptr, cnt_out == nullptr, mean_pool(p));
   if (ws_bytes < L.total_fixed) return QSA_ERR_WORKSPACE_TOO_SMALL;
   const size_t slab_bytes = ws_bytes - L.total_fixed;
   const int64_t min_rows = nq < MIN_ROWS ? nq : MIN_ROWS;
@@ -472,6 +509,10 @@ qsa_status qsa_prefill_cached(const qsa_params* p, int64_t L_old, int64_t T_new,
     qi = qst;
     wi = wst;
   }
+  // compressed keys of all cached and new tokens (mean pooling; the caches
+  // now hold the new rows)
+  uint16_t* kbar = mean_pool(p) ? reinterpret_cast<uint16_t*>(base + L.kbar) : nullptr;
+  if (kbar && (st = run_kbar(kidx_cache, T, kbar, s)) != QSA_OK) return st;
   const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
   for (int64_t qb0 = qbA; qb0 < nkb;) {
     const int64_t qb1 = chunk_end(qb0, nkb, slab_bytes);
@@ -481,8 +522,8 @@ qsa_status qsa_prefill_cached(const qsa_params* p, int64_t L_old, int64_t T_new,
     float* segmax = slab + (size_t)(qb1 - qb0) * ld;
     int32_t* sel_c = sel + (qb0 - qbA) * budget;
     int32_t* cnt_c = cnt + (qb0 - qbA);
-    if ((st = run_indexer(T, 4 * qbA, qi, wi, kidx_cache, qb0, qb1, slab, ld, segmax, ld_seg, err, di.num_sms, s)) !=
-        QSA_OK)
+    if ((st = run_indexer(T, 4 * qbA, qi, wi, kidx_cache, kbar, qb0, qb1, slab, ld, segmax, ld_seg, err, di.num_sms,
+                          s)) != QSA_OK)
       return st;
     if ((st = from_cuda(traced(QSA_KERNEL_SELECT, s, [&] {
            return qsa::launch_select(slab, ld, segmax, ld_seg, qb0, qb1 - qb0, nullptr, budget, sel_c, cnt_c, err, s);
@@ -563,6 +604,7 @@ qsa_status qsa_decode(const qsa_params* p, int32_t B, int64_t max_len, const int
                       float* lse_out, void* ws, size_t ws_bytes, void* stream) {
   qsa_status st = check_params(p);
   if (st != QSA_OK) return st;
+  if (mean_pool(p)) return QSA_ERR_UNSUPPORTED;
   if (B <= 0 || max_len <= 0 || !cache_len) return QSA_ERR_INVALID_ARG;
   if (B > 4096 || max_len > ((int64_t)1 << 24)) return QSA_ERR_UNSUPPORTED;
   const void* ptrs[] = {k_cache, v_cache, kidx_cache, qidx_ring, w_ring, q_new, k_new, v_new,

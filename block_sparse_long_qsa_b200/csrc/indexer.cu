@@ -49,15 +49,23 @@ static_assert(SMEM_BYTES <= 232448, "indexer smem");
 constexpr uint32_t TMEM_COLS = 512;
 
 struct Sched {
-  int64_t T0, Tend, n_tiles, c;   // c = nkt(0)
+  int64_t T0, Tend, n_tiles;
   int64_t qb_begin;
+  int64_t R;                      // tokens per key-tile row: 1 (keys) or 4 (mean-pooled key blocks)
+  int64_t A;                      // (T0 + QT - 1) / QT
   __device__ __forceinline__ int64_t nkt(int64_t i) const {
     int64_t tl = T0 + QT * i + (QT - 1);
     if (tl > Tend - 1) tl = Tend - 1;
-    return tl / KT + 1;
+    return tl / (KT * R) + 1;
   }
-  // units before tile i (valid for i <= n_tiles - 1; tiles before the last are full)
-  __device__ __forceinline__ int64_t prefix(int64_t i) const { return c * i + i * (i - 1) / 2; }
+  // sum over m < N of floor(m / R)
+  __device__ __forceinline__ int64_t G(int64_t N) const {
+    const int64_t q = N / R, r = N % R;
+    return R * q * (q - 1) / 2 + r * q;
+  }
+  // units before tile i (valid for i <= n_tiles - 1; tiles before the last are
+  // full): sum over j < i of floor((A + j) / R) + 1, as QT = KT tokens
+  __device__ __forceinline__ int64_t prefix(int64_t i) const { return i + G(A + i) - G(A); }
   __device__ __forceinline__ int64_t total() const { return prefix(n_tiles - 1) + nkt(n_tiles - 1); }
   __device__ __forceinline__ void locate(int64_t u, int64_t& tile, int64_t& kt) const {
     int64_t lo = 0, hi = n_tiles - 1;
@@ -87,6 +95,7 @@ struct Iter {
   }
 };
 
+template <bool MEAN>
 __global__ void __launch_bounds__(THREADS, 1)
 indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const uint16_t* __restrict__ w, float* __restrict__ S, int64_t ld,
@@ -120,7 +129,8 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
   sch.T0 = qb_begin * 4;
   sch.Tend = qb_end * 4 < T ? qb_end * 4 : T;
   sch.n_tiles = (sch.Tend - sch.T0 + QT - 1) / QT;
-  sch.c = (sch.T0 + QT - 1) / KT + 1;
+  sch.R = MEAN ? 4 : 1;
+  sch.A = (sch.T0 + QT - 1) / QT;
   const int64_t W = sch.total();
   const int64_t u0 = W * (int64_t)blockIdx.x / gridDim.x;
   const int64_t u1 = W * (int64_t)(blockIdx.x + 1) / gridDim.x;
@@ -258,16 +268,20 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
       }
       const int64_t t_tile = sch.T0 + QT * it.tile;
       const int64_t qb_tile = qb_begin + (QT / 4) * it.tile;
-      const int64_t j = KT * it.kt + 32 * quad + lane;       // this thread's key
-      const int64_t kb = j >> 2;
+      // this thread's TMEM lane: one key (token-pair max) or one key block (mean pool);
+      // j is the first token it stands for, so "j <= t" is the causal test in both
+      const int64_t row = KT * it.kt + 32 * quad + lane;
+      const int64_t j = MEAN ? 4 * row : row;
+      const int64_t kb = MEAN ? row : row >> 2;
       if (!__all_sync(0xffffffffu, mbar_wait(&accfull[hf], acc_use & 1, abort_flag, err))) break;
       ++acc_use;
       tc_fence_after();
       const int64_t t_first = t_tile + 64 * hf + 32 * cgrp;  // first token of this thread's columns
       const int64_t qb_first = qb_tile + 16 * hf + 8 * cgrp;
-      const int64_t kt_last_key = KT * it.kt + KT - 1;
+      const int64_t kt_last_key = MEAN ? 4 * (KT * it.kt + KT - 1) : KT * it.kt + KT - 1;
       // skip when every key block of this warp lies after every query block of its columns
-      const bool live = (KT * it.kt + 32 * quad) <= (t_first + 31) && qb_first < qb_end;
+      const int64_t warp_first_key = MEAN ? 4 * (KT * it.kt + 32 * quad) : KT * it.kt + 32 * quad;
+      const bool live = warp_first_key <= (t_first + 31) && qb_first < qb_end;
       if (live) {
         const bool masked = kt_last_key > t_first;
         float m[8];
@@ -320,41 +334,70 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         __syncwarp();
         if (lane == 0) mbar_arrive(&accempty[hf]);
         chunk(vb, 3);
-        // max over the 4 keys of the key block (lanes 4k .. 4k+3) as a transposing
-        // butterfly: after the two steps lane (a = bit 0, b = bit 1) holds the
-        // maxima of query blocks 4a + 2b and 4a + 2b + 1.
-        const bool la = (lane & 1) != 0, lb = (lane & 2) != 0;
-        float n4[4];
+        if constexpr (MEAN) {
+          // one key block per lane: the 8 block maxima are the scores
+          // S(qb_first + b, kb), stored by the 32 lanes as 32 consecutive floats
+          float* srow = S + (qb_first - qb_begin) * ld + kb;
+          const int nb = (int)(qb_end - qb_first < 8 ? qb_end - qb_first : 8);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float send = la ? m[i] : m[i + 4];
-          const float keep = la ? m[i + 4] : m[i];
-          n4[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 1));
-        }
-        float val[2];
+          for (int b = 0; b < 8; ++b) {
+            if (b < nb && kb <= qb_first + b) srow[b * ld] = m[b] * scale;
+          }
+          if (segmax != nullptr) {
+            // segment maxima over 8 key blocks = 8 lanes (bits 0..2): three
+            // transposing steps leave lane (a, b, c) of each 8-lane group with
+            // the maximum of query block qb_first + 4 a + 2 b + c
+            const bool la = (lane & 1) != 0, lb = (lane & 2) != 0, lc = (lane & 4) != 0;
+            float n4[4], n2[2];
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const float send = lb ? n4[i] : n4[i + 2];
-          const float keep = lb ? n4[i + 2] : n4[i];
-          val[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
-          const int64_t qb = qb_first + (la ? 4 : 0) + (lb ? 2 : 0) + i;
-          if (qb < qb_end && kb <= qb) S[(qb - qb_begin) * ld + kb] = val[i] * scale;
-        }
-        if (segmax != nullptr) {
-          // segment maxima: max over the 8 key blocks of this warp's 32 keys
-          // (lane bits 2..4).  A transposing step on bit 2 leaves each lane one
-          // query block (4 a + 2 b + c0), then two plain steps; lanes 0..7 hold
-          // the 8 query blocks.  Key blocks after a query block were scored as
-          // 0 and scores are >= 0, so they do not raise a maximum.
-          const bool lc = (lane & 4) != 0;
-          float sm = fmaxf(lc ? val[1] : val[0], __shfl_xor_sync(0xffffffffu, lc ? val[0] : val[1], 4));
-          sm = fmaxf(sm, __shfl_xor_sync(0xffffffffu, sm, 8));
-          sm = fmaxf(sm, __shfl_xor_sync(0xffffffffu, sm, 16));
-          if (lane < 8) {
-            const int64_t seg = (KT * it.kt + 32 * quad) >> 5;
+            for (int i = 0; i < 4; ++i)
+              n4[i] = fmaxf(la ? m[i + 4] : m[i], __shfl_xor_sync(0xffffffffu, la ? m[i] : m[i + 4], 1));
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+              n2[i] = fmaxf(lb ? n4[i + 2] : n4[i], __shfl_xor_sync(0xffffffffu, lb ? n4[i] : n4[i + 2], 2));
+            const float sm = fmaxf(lc ? n2[1] : n2[0], __shfl_xor_sync(0xffffffffu, lc ? n2[0] : n2[1], 4));
+            const int64_t seg = (KT * it.kt + 32 * quad + (lane & ~7)) >> 3;
             const int64_t qb = qb_first + (la ? 4 : 0) + (lb ? 2 : 0) + (lc ? 1 : 0);
             // only segments starting at or before the row's own block: seg <= qb / 8 < ld_seg
             if (qb < qb_end && seg <= (qb >> 3)) segmax[(qb - qb_begin) * ld_seg + seg] = sm * scale;
+          }
+        } else {
+          // max over the 4 keys of the key block (lanes 4k .. 4k+3) as a transposing
+          // butterfly: after the two steps lane (a = bit 0, b = bit 1) holds the
+          // maxima of query blocks 4a + 2b and 4a + 2b + 1.
+          const bool la = (lane & 1) != 0, lb = (lane & 2) != 0;
+          float n4[4];
+  #pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float send = la ? m[i] : m[i + 4];
+            const float keep = la ? m[i + 4] : m[i];
+            n4[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 1));
+          }
+          float val[2];
+  #pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const float send = lb ? n4[i] : n4[i + 2];
+            const float keep = lb ? n4[i + 2] : n4[i];
+            val[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
+            const int64_t qb = qb_first + (la ? 4 : 0) + (lb ? 2 : 0) + i;
+            if (qb < qb_end && kb <= qb) S[(qb - qb_begin) * ld + kb] = val[i] * scale;
+          }
+          if (segmax != nullptr) {
+            // segment maxima: max over the 8 key blocks of this warp's 32 keys
+            // (lane bits 2..4).  A transposing step on bit 2 leaves each lane one
+            // query block (4 a + 2 b + c0), then two plain steps; lanes 0..7 hold
+            // the 8 query blocks.  Key blocks after a query block were scored as
+            // 0 and scores are >= 0, so they do not raise a maximum.
+            const bool lc = (lane & 4) != 0;
+            float sm = fmaxf(lc ? val[1] : val[0], __shfl_xor_sync(0xffffffffu, lc ? val[0] : val[1], 4));
+            sm = fmaxf(sm, __shfl_xor_sync(0xffffffffu, sm, 8));
+            sm = fmaxf(sm, __shfl_xor_sync(0xffffffffu, sm, 16));
+            if (lane < 8) {
+              const int64_t seg = (KT * it.kt + 32 * quad) >> 5;
+              const int64_t qb = qb_first + (la ? 4 : 0) + (lb ? 2 : 0) + (lc ? 1 : 0);
+              // only segments starting at or before the row's own block: seg <= qb / 8 < ld_seg
+              if (qb < qb_end && seg <= (qb >> 3)) segmax[(qb - qb_begin) * ld_seg + seg] = sm * scale;
+            }
           }
         }
       } else {
@@ -381,31 +424,74 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 
 cudaError_t launch_indexer_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const uint16_t* w,
                                    float* S, int64_t ld, float* segmax, int64_t ld_seg, int64_t T, int64_t q_tok0,
-                                   int64_t qb_begin, int64_t qb_end, float scale, uint32_t* err, int num_sms,
-                                   cudaStream_t stream) {
+                                   int64_t qb_begin, int64_t qb_end, bool mean_pool, float scale, uint32_t* err,
+                                   int num_sms, cudaStream_t stream) {
   if (qb_end <= qb_begin) return cudaSuccess;
-  static bool attr_done[64] = {false};
+  static bool attr_done[2][64] = {{false}, {false}};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(indexer_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SMEM_BYTES);
+  if (dev < 64 && !attr_done[mean_pool][dev]) {
+    cudaError_t e = mean_pool ? cudaFuncSetAttribute(indexer_prefill_kernel<true>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES)
+                              : cudaFuncSetAttribute(indexer_prefill_kernel<false>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr_done[dev] = true;
+    attr_done[mean_pool][dev] = true;
   }
   // units in this call; never more CTAs than units
   const int64_t T0 = qb_begin * 4;
   const int64_t Tend = qb_end * 4 < T ? qb_end * 4 : T;
   const int64_t n_tiles = (Tend - T0 + QT - 1) / QT;
+  const int64_t key_tokens = mean_pool ? 4 * KT : KT;   // tokens covered by one key tile
   int64_t units = 0;
   for (int64_t i = 0; i < n_tiles && units < num_sms; ++i) {
     int64_t tl = T0 + QT * i + QT - 1;
     if (tl > Tend - 1) tl = Tend - 1;
-    units += tl / KT + 1;
+    units += tl / key_tokens + 1;
   }
   const int grid = (int)(units < num_sms ? units : num_sms);
-  indexer_prefill_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tm_q, tm_k, w, S, ld, segmax, ld_seg, T, q_tok0,
-                                                                 qb_begin, qb_end, scale, err);
+  if (mean_pool)
+    indexer_prefill_kernel<true><<<grid, THREADS, SMEM_BYTES, stream>>>(tm_q, tm_k, w, S, ld, segmax, ld_seg, T,
+                                                                        q_tok0, qb_begin, qb_end, scale, err);
+  else
+    indexer_prefill_kernel<false><<<grid, THREADS, SMEM_BYTES, stream>>>(tm_q, tm_k, w, S, ld, segmax, ld_seg, T,
+                                                                         q_tok0, qb_begin, qb_end, scale, err);
+  return cudaGetLastError();
+}
+
+// Mean-pooled indexer keys: kbar[b][c] = bf16 of the mean of k_idx rows
+// 4b .. min(4b + 4, T) - 1 (exact fp64 sum, one fp64 division, round to
+// nearest even), one thread per (block, dim).
+namespace {
+__device__ __forceinline__ uint16_t f64_to_bf16_rne_dev(double x) {
+  const uint64_t u = (uint64_t)__double_as_longlong(x);
+  const uint16_t sign = (uint16_t)((u >> 48) & 0x8000u);
+  const double a = fabs(x);
+  if (a == 0.0) return sign;
+  int e;
+  frexp(a, &e);                                   // a = m 2^e, m in [0.5, 1)
+  const int unit = e - 8 > -133 ? e - 8 : -133;   // weight of bf16's last bit
+  const double v = ldexp(rint(ldexp(a, -unit)), unit);   // rint: nearest, ties to even
+  return (uint16_t)(sign | (__float_as_uint((float)v) >> 16));   // v has <= 8 significant bits
+}
+
+__global__ void kbar_kernel(const uint16_t* __restrict__ k_idx, int64_t T, int64_t nkb, uint16_t* __restrict__ kbar) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= nkb * 128) return;
+  const int64_t b = i >> 7, c = i & 127;
+  const int64_t t0 = 4 * b;
+  const int n = (int)(T - t0 < 4 ? T - t0 : 4);
+  double sum = 0.0;
+  for (int r = 0; r < n; ++r) sum += (double)__uint_as_float((uint32_t)k_idx[(t0 + r) * 128 + c] << 16);
+  kbar[i] = f64_to_bf16_rne_dev(sum / (double)n);
+}
+}  // namespace
+
+cudaError_t launch_kbar(const uint16_t* k_idx, int64_t T, uint16_t* kbar, cudaStream_t stream) {
+  const int64_t nkb = (T + 3) / 4;
+  if (nkb <= 0) return cudaSuccess;
+  const int64_t n = nkb * 128;
+  kbar_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(k_idx, T, nkb, kbar);
   return cudaGetLastError();
 }
 

@@ -17,10 +17,16 @@ cudaError_t launch_rope_k(int64_t T, const uint16_t* k, const float2* cs, uint16
 // over each segment of 8 key blocks (segment s = blocks 8s .. 8s+7, blocks
 // after the row's own block counting as 0).  Keys are tokens [0, T) of tm_k;
 // the query rows (tm_q) and w start at token q_tok0 (<= 4 * qb_begin).
+// mean_pool: tm_k holds the mean-pooled block keys [ceil(T/4)][128] (launch_kbar)
+// and S(qb, kb) = max over the present tokens t of block qb of the score of t
+// against kbar[kb]; otherwise tm_k holds the keys [T][128] and S is the max over
+// causal token pairs.
 cudaError_t launch_indexer_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const uint16_t* w,
                                    float* S, int64_t ld, float* segmax, int64_t ld_seg, int64_t T, int64_t q_tok0,
-                                   int64_t qb_begin, int64_t qb_end, float scale, uint32_t* err, int num_sms,
-                                   cudaStream_t stream);
+                                   int64_t qb_begin, int64_t qb_end, bool mean_pool, float scale, uint32_t* err,
+                                   int num_sms, cudaStream_t stream);
+// kbar[b] = bf16 round-to-nearest-even of the mean of k_idx rows 4b .. min(4b+4, T)-1.
+cudaError_t launch_kbar(const uint16_t* k_idx, int64_t T, uint16_t* kbar, cudaStream_t stream);
 
 // Top-k block selection, one row per query block.  Row r covers query block
 // row_qb ? row_qb[r] : qb_begin + r, read from S + r * ld.  segmax (nullable,

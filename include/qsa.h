@@ -55,7 +55,20 @@ typedef enum {
  * rope_parameters listing in [PT] section "100만 토큰까지 늘리기":
  * n_q_heads 24, n_kv_heads 2, head_dim 256, rope_dim 64, rope_theta 1e7,
  * idx_heads 4, idx_dim 128, block_size 4; budget_blocks is free in [2, 4096]
- * (default 512).  softmax_scale 0 means 1/sqrt(head_dim). */
+ * (default 512).  softmax_scale 0 means 1/sqrt(head_dim).
+ * aggregation picks the block score of stage 1 (default QSA_AGG_TOKEN_MAX):
+ *   QSA_AGG_TOKEN_MAX: S(qb, kb) = max over the causal token pairs (t in qb,
+ *     j in kb, j <= t) of s(t, j);
+ *   QSA_AGG_MEAN_POOL ([PT §QSA]: each micro-block's keys are mean-pooled
+ *     into one compressed key k-bar_b, and every query token scores the
+ *     compressed keys, O(n^2 / r)): k-bar_kb = bf16 (round to nearest even)
+ *     of the mean of block kb's present indexer keys (exact sum, one fp64
+ *     division); S(qb, kb) = max over the present tokens t of block qb of
+ *     sum_h w_h(t) ReLU(q_idx_h(t) . k-bar_kb) / sqrt(128), for kb <= qb (the
+ *     own block's entry uses all its present keys and never decides a
+ *     selection: the own block is always kept).  qsa_decode returns
+ *     QSA_ERR_UNSUPPORTED for it. */
+enum { QSA_AGG_TOKEN_MAX = 0, QSA_AGG_MEAN_POOL = 1 };
 typedef struct {
   int32_t n_q_heads;
   int32_t n_kv_heads;
@@ -67,6 +80,7 @@ typedef struct {
   int32_t block_size;
   int32_t budget_blocks;
   float softmax_scale;
+  int32_t aggregation;
 } qsa_params;
 
 /* Fills *p with the values above (budget 512). */
@@ -89,8 +103,13 @@ const char* qsa_last_error(void);
  * Writes scores[(qb - qb_begin) * ld + kb] (fp32) for qb in [qb_begin, qb_end)
  * and kb <= qb; entries with kb > qb are not written.
  * Requires 0 <= qb_begin <= qb_end <= ceil(T/4), ld >= qb_end, ld % 4 == 0.
- * ws (nullable, >= 256 bytes) receives the device error word; with ws NULL a
- * device-side timeout is not reported (the kernel still exits). */
+ * With p->aggregation == QSA_AGG_MEAN_POOL the scores are the mean-pooled ones
+ * (see qsa_params).
+ * ws: at least qsa_index_workspace_size bytes (the device error word, and the
+ * compressed keys for mean pooling); with the token-pair block score ws may be
+ * NULL, and a device-side timeout is then not reported (the kernel still
+ * exits). */
+qsa_status qsa_index_workspace_size(const qsa_params* p, int64_t T, size_t* bytes);
 qsa_status qsa_index_scores(const qsa_params* p, int64_t T, const uint16_t* q_idx, const uint16_t* w,
                             const uint16_t* k_idx, int64_t qb_begin, int64_t qb_end, float* scores, int64_t ld,
                             void* ws, size_t ws_bytes, void* stream);
@@ -233,7 +252,8 @@ enum {
   QSA_KERNEL_DECODE_APPEND = 6,
   QSA_KERNEL_DECODE_INDEXER = 7,
   QSA_KERNEL_DECODE_ATTENTION = 8,
-  QSA_KERNEL_DECODE_COMBINE = 9
+  QSA_KERNEL_DECODE_COMBINE = 9,
+  QSA_KERNEL_KBAR = 10
 };
 qsa_status qsa_trace_begin(int32_t capacity);
 qsa_status qsa_trace_end(int32_t* kernel_ids, float* ms, int32_t capacity, int32_t* n_out);

@@ -22,10 +22,10 @@ def _lib():
     qsa.load()
 
 
-def run_cached(h, L_old, T_new, budget, k_rot_full, ws_bytes=None):
+def run_cached(h, L_old, T_new, budget, k_rot_full, ws_bytes=None, aggregation=qsa.AGG_TOKEN_MAX):
     """Seed caches with the first L_old tokens, prefill the rest."""
     T = L_old + T_new
-    p = qsa.params(budget)
+    p = qsa.params(budget, aggregation=aggregation)
     kc = torch.zeros((T, 2, 256), dtype=torch.uint16, device="cuda")
     vc = torch.zeros_like(kc)
     ic = torch.zeros((T, 128), dtype=torch.uint16, device="cuda")
