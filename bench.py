@@ -136,12 +136,13 @@ def prefill_flops(T: int, sel_cnt: np.ndarray | None):
     return idx, attn
 
 
-def run_prefill(T: int, budget: int, steps: int, warmup: int, rank: int, world: int, seed: int, want_e2e=True):
+def run_prefill(T: int, budget: int, steps: int, warmup: int, rank: int, world: int, seed: int, want_e2e=True,
+                aggregation: int = 0):
     import block_sparse_long_qsa_b200 as qsa
     P = Q.PrefillProblem(T=T, seed=seed + 1000 * rank, n_plant=8, dist="zipf" if T >= 131072 else "uniform")
     d = P.device()
     torch.cuda.synchronize()
-    p = qsa.params(budget)
+    p = qsa.params(budget, aggregation=aggregation)
     mn, pref = qsa.qsa_prefill_workspace_size(p, T)
     ws = qsa.workspace(pref)
     nqb = P.nqb
@@ -175,6 +176,8 @@ def run_prefill(T: int, budget: int, steps: int, warmup: int, rank: int, world: 
         raise RuntimeError("device error during the timed steps")
     cnt_h = cnt.cpu().numpy()
     fl_idx, fl_attn = prefill_flops(T, cnt_h)
+    if aggregation == 1:
+        fl_idx /= 4          # one compressed key per block: a quarter of the dot products
     kern = tr.by_kernel()
     launches = sum(c for c, _ in kern.values())
     res = dict(ms=ms_max, tokens=T * steps * world, kern=kern, launches=launches, clocks=clk.summary(),
@@ -456,11 +459,12 @@ def cpu_sample(wl: dict, target_s: float = 12.0):
     CPU time: a calibration run, then one run scaled to the target."""
     if wl["kind"] in ("prefill", "prefill_cached"):
         qb_lo = wl.get("L_old", 0) // 4
+        agg = wl.get("aggregation", 0)
         n = max(4, cores_used())
-        v, info = cpu_prefill_sample(wl["T"], 512, n, qb_lo=qb_lo)
+        v, info = cpu_prefill_sample(wl["T"], 512, n, qb_lo=qb_lo, aggregation=agg)
         if info["elapsed"] < target_s / 3:
             n2 = int(min((wl["T"] + 3) // 4 - qb_lo, max(n + 1, n * target_s / max(info["elapsed"], 1e-3))))
-            v, info = cpu_prefill_sample(wl["T"], 512, n2, qb_lo=qb_lo)
+            v, info = cpu_prefill_sample(wl["T"], 512, n2, qb_lo=qb_lo, aggregation=agg)
     else:
         n = 2
         v, info = cpu_decode_sample(wl["B"], wl["L"], 512, n)
@@ -470,13 +474,13 @@ def cpu_sample(wl: dict, target_s: float = 12.0):
     return v, info
 
 
-def cpu_prefill_sample(T: int, budget: int, n_blocks: int, seed: int = 0, qb_lo: int = 0):
+def cpu_prefill_sample(T: int, budget: int, n_blocks: int, seed: int = 0, qb_lo: int = 0, aggregation: int = 0):
     """The oracle on a stratified sample of query blocks of the T-token
     prefill (evenly spaced qb in [qb_lo, nqb)), all host cores.  Returns
     tokens/s of the oracle extrapolated by the sample's share of the work, and
     a description."""
     import oracle
-    O = oracle.Oracle(oracle.params(budget=budget))
+    O = oracle.Oracle(oracle.params(budget=budget, aggregation=aggregation))
     P = Q.PrefillProblem(T=T, seed=seed, n_plant=8, dist="zipf" if T >= 131072 else "uniform")
     nqb = P.nqb
     qbs = np.unique(np.linspace(qb_lo, nqb - 1, n_blocks).astype(np.int64))
@@ -567,6 +571,8 @@ WORKLOADS = {
     # 90 % of a 1M-token prompt already cached (L_old % 4 = 2: the first new
     # query block starts mid-block)
     "prefill_1m_cached90": dict(kind="prefill_cached", T=1 << 20, L_old=943718),
+    # the pages' mean-pooled indexer (one compressed key per 4-token block)
+    "prefill_1m_meanpool": dict(kind="prefill", T=1 << 20, aggregation=1),
 }
 
 
@@ -578,7 +584,8 @@ NCU_TRAFFIC = {"prefill_1m": 67.49e9 + 15.26e9}
 
 def metric_name(wl: dict) -> str:
     if wl["kind"] == "prefill":
-        return f"QSA prefill tokens/s at {wl['T'] // 1024}K context"
+        mp = ", mean-pooled indexer" if wl.get("aggregation") == 1 else ""
+        return f"QSA prefill tokens/s at {wl['T'] // 1024}K context{mp}"
     if wl["kind"] == "prefill_cached":
         return (f"QSA prefix-cached prefill new tokens/s at {wl['T'] // 1024}K context, "
                 f"{round(100 * wl['L_old'] / wl['T'])}% cached")
@@ -705,7 +712,8 @@ def main():
     pk = peaks()
     wl = WORKLOADS[args.workload]
     if wl["kind"] == "prefill":
-        res = run_prefill(wl["T"], 512, args.steps, args.warmup, rank, world, seed=0, want_e2e=not args.no_e2e)
+        res = run_prefill(wl["T"], 512, args.steps, args.warmup, rank, world, seed=0, want_e2e=not args.no_e2e,
+                          aggregation=wl.get("aggregation", 0))
     elif wl["kind"] == "prefill_cached":
         res = run_prefill_cached(wl["T"], wl["L_old"], 512, args.steps, args.warmup, rank, world, seed=0,
                                  want_e2e=not args.no_e2e)
@@ -716,12 +724,13 @@ def main():
 
     if not args.no_secondary:
         sec = {}
-        for name in ("decode_64x256k", "prefill_128k", "prefill_1m_cached90"):
+        for name in ("decode_64x256k", "prefill_128k", "prefill_1m_cached90", "prefill_1m_meanpool"):
             if name == args.workload:
                 continue
             w2 = WORKLOADS[name]
             if w2["kind"] == "prefill":
-                r2 = run_prefill(w2["T"], 512, args.steps, args.warmup, rank, world, seed=0, want_e2e=False)
+                r2 = run_prefill(w2["T"], 512, args.steps, args.warmup, rank, world, seed=0, want_e2e=False,
+                                 aggregation=w2.get("aggregation", 0))
             elif w2["kind"] == "prefill_cached":
                 r2 = run_prefill_cached(w2["T"], w2["L_old"], 512, args.steps, args.warmup, rank, world, seed=0,
                                         want_e2e=False)
