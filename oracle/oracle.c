@@ -49,6 +49,12 @@ typedef struct {
   double softmax_scale;/* 0 => 1/sqrt(head_dim) */
   int32_t aggregation; /* 0: max over causal token pairs (the stated block score);
                           1: mean-pooled block keys [PT §QSA, I_ib over k-bar_b] */
+  /* YaRN [PT "100만 토큰까지 늘리기": rope_type yarn, factor 4.0,
+   * original_max_position_embeddings 262144]; factor <= 1 means plain RoPE */
+  double yarn_factor;
+  double yarn_original_max;
+  double yarn_beta_fast;  /* 32 (not on the pages: the method's usual value) */
+  double yarn_beta_slow;  /* 1 */
 } oracle_params;
 
 static double bf16_to_f64(uint16_t h) {
@@ -61,15 +67,47 @@ static double bf16_to_f64(uint16_t h) {
  * Rotary position embedding on dims [0, rope_dim) of one head vector
  * ([PT] spec table "RoPE 차원 64"; rope_theta and partial_rotary_factor 0.25
  * in [PT] "100만 토큰까지 늘리기").  y may not alias x. */
+/* Frequency of rotary pair i.  Plain: theta^(-2i/rope_dim).  YaRN (static,
+ * factor s > 1): "NTK-by-parts" -- a pair whose wavelength 2 pi / f_i fits
+ * more than beta_fast times into the original context keeps f_i, one fitting
+ * fewer than beta_slow times gets f_i / s, and in between the two are mixed
+ * linearly in the pair index i, from the index where the rotation count
+ * crosses beta_fast (rounded down) to where it crosses beta_slow (rounded
+ * up); the rotation count r(i) = L_orig f_i / (2 pi) crosses n at
+ * i(n) = rope_dim ln(L_orig / (2 pi n)) / (2 ln theta). */
+static double rope_freq(const oracle_params* p, int i) {
+  const double d = (double)p->rope_dim;
+  const double f = pow(p->rope_theta, -2.0 * (double)i / d);
+  const double s = p->yarn_factor;
+  if (!(s > 1.0)) return f;
+  const double two_pi = 2.0 * acos(-1.0);
+  const double i_fast = d * log(p->yarn_original_max / (two_pi * p->yarn_beta_fast)) / (2.0 * log(p->rope_theta));
+  const double i_slow = d * log(p->yarn_original_max / (two_pi * p->yarn_beta_slow)) / (2.0 * log(p->rope_theta));
+  double lo = floor(i_fast), hi = ceil(i_slow);
+  if (lo < 0.0) lo = 0.0;
+  if (hi > d - 1.0) hi = d - 1.0;
+  if (hi == lo) hi += 0.001;
+  double ramp = ((double)i - lo) / (hi - lo);   /* 0: keep f, 1: f / s */
+  if (ramp < 0.0) ramp = 0.0;
+  if (ramp > 1.0) ramp = 1.0;
+  return f / s * ramp + f * (1.0 - ramp);
+}
+
+/* YaRN's attention factor 0.1 ln s + 1 on the rotated dims (1 for plain RoPE). */
+static double rope_scale(const oracle_params* p) {
+  return p->yarn_factor > 1.0 ? 0.1 * log(p->yarn_factor) + 1.0 : 1.0;
+}
+
 void oracle_rope(const oracle_params* p, const double* x, int64_t pos, double* y) {
   int half = p->rope_dim / 2;
+  const double m = rope_scale(p);
   for (int c = 0; c < p->head_dim; ++c) y[c] = x[c];
   for (int i = 0; i < half; ++i) {
-    double inv_freq = pow(p->rope_theta, -2.0 * (double)i / (double)p->rope_dim);
+    double inv_freq = rope_freq(p, i);
     double a = (double)pos * inv_freq;
     double ca = cos(a), sa = sin(a);
-    y[i] = x[i] * ca - x[i + half] * sa;
-    y[i + half] = x[i + half] * ca + x[i] * sa;
+    y[i] = m * (x[i] * ca - x[i + half] * sa);
+    y[i + half] = m * (x[i + half] * ca + x[i] * sa);
   }
 }
 

@@ -154,6 +154,69 @@ def pin_identical_keys_block(O):
         assert abs(S[qb, qb] - want) < 1e-14 * (1 + want)
 
 
+# ------------------------------------------------------------- YaRN (f4)
+def _yarn_oracle(O, factor=4.0):
+    import oracle as OR
+    return type(O)(OR.params(budget=O.P.budget, yarn_factor=factor), O.L)
+
+
+def _pair_angles(Oy, pos):
+    """Rotation angle of every pair (i, i + 32) at position pos, and the
+    radius, read off the image of the unit vectors e_i."""
+    ang, rad = np.zeros(32), np.zeros(32)
+    for i in range(32):
+        x = np.zeros(256)
+        x[i] = 1.0
+        y = Oy.rope(x, pos)
+        ang[i] = math.atan2(y[i + 32], y[i])
+        rad[i] = math.hypot(y[i], y[i + 32])
+    return ang, rad
+
+
+def pin_yarn_attention_factor_and_tail(O):
+    """The rotated dims are scaled by 0.1 ln s + 1 (s = 4: 1.13863), the other
+    192 dims are untouched, for any position."""
+    Oy = _yarn_oracle(O)
+    m = 0.1 * math.log(4.0) + 1.0
+    rng = np.random.default_rng(1)
+    for pos in (0, 7, 262143, 1048575):
+        x = rng.standard_normal(256)
+        y = Oy.rope(x, pos)
+        assert abs(np.linalg.norm(y[:64]) - m * np.linalg.norm(x[:64])) < 1e-12 * np.linalg.norm(x[:64])
+        assert np.array_equal(y[64:], x[64:])
+
+
+def pin_yarn_relative_positions(O):
+    """<R(x, a), R(y, b)> depends on a - b only, as for plain RoPE."""
+    Oy = _yarn_oracle(O)
+    rng = np.random.default_rng(2)
+    x, y = rng.standard_normal(256), rng.standard_normal(256)
+    for a, b, shift in ((5, 3, 1000), (300000, 299000, 700000), (17, 900000, 12345)):
+        d0 = Oy.rope(x, a) @ Oy.rope(y, b)
+        d1 = Oy.rope(x, a + shift) @ Oy.rope(y, b + shift)
+        assert abs(d0 - d1) < 1e-9 * (1 + abs(d0)), (a, b)
+
+
+def pin_yarn_frequency_regimes(O):
+    """Pair 0 (wavelength 2 pi, far shorter than the 262144-token original
+    context) keeps its frequency 1; pair 31 (wavelength ~1.3e7 tokens, longer
+    than the context) is interpolated to theta^(-31/32) / 4; every pair's
+    frequency lies between f_i / 4 and f_i, and its ratio to f_i does not
+    increase with i; factor 1 is plain RoPE."""
+    Oy = _yarn_oracle(O)
+    ang, rad = _pair_angles(Oy, 1)
+    f = 1e7 ** (-np.arange(32) / 32.0)
+    assert abs(ang[0] - 1.0) < 1e-12
+    assert abs(ang[31] - f[31] / 4.0) < 1e-15
+    ratio = ang / f
+    assert np.all(ratio <= 1.0 + 1e-12) and np.all(ratio >= 0.25 - 1e-12)
+    assert np.all(np.diff(ratio) <= 1e-12)
+    assert np.any(np.abs(ratio - 1.0) < 1e-12) and np.any(np.abs(ratio - 0.25) < 1e-12)
+    O1 = _yarn_oracle(O, factor=1.0)
+    x = np.random.default_rng(3).standard_normal(256)
+    assert np.array_equal(O1.rope(x, 123456), O.rope(x, 123456))
+
+
 # ------------------------------------------------ mean-pooled block keys (f2)
 def _bf16_rne_exact(x) -> float:
     """Round a rational to the nearest bf16 value (ties to even), by integer

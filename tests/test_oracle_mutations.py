@@ -19,9 +19,13 @@ MUTANTS = [
     ("causal_off_by_one", "if (j > t) continue;", "if (j > t + 1) continue;"),
     ("block_sum_not_max", "if (s > best) best = s;", "best = (best < 0.0 ? 0.0 : best) + s;"),
     ("key_dim_dropped", "for (int c = 0; c < p->idx_dim; ++c) dot +=", "for (int c = 1; c < p->idx_dim; ++c) dot +="),
-    ("rope_sign", "y[i] = x[i] * ca - x[i + half] * sa;", "y[i] = x[i] * ca + x[i + half] * sa;"),
-    ("rope_pairing", "y[i + half] = x[i + half] * ca + x[i] * sa;", "y[i + half] = x[i + half] * ca + x[(i + 1) % half] * sa;"),
-    ("rope_freq", "pow(p->rope_theta, -2.0 * (double)i / (double)p->rope_dim)", "pow(p->rope_theta, -1.0 * (double)i / (double)p->rope_dim)"),
+    ("rope_sign", "y[i] = m * (x[i] * ca - x[i + half] * sa);", "y[i] = m * (x[i] * ca + x[i + half] * sa);"),
+    ("rope_pairing", "y[i + half] = m * (x[i + half] * ca + x[i] * sa);",
+     "y[i + half] = m * (x[i + half] * ca + x[(i + 1) % half] * sa);"),
+    ("rope_freq", "pow(p->rope_theta, -2.0 * (double)i / d)", "pow(p->rope_theta, -1.0 * (double)i / d)"),
+    ("yarn_scale_dropped", "return p->yarn_factor > 1.0 ? 0.1 * log(p->yarn_factor) + 1.0 : 1.0;", "return 1.0;"),
+    ("yarn_ramp_reversed", "return f / s * ramp + f * (1.0 - ramp);", "return f * ramp + f / s * (1.0 - ramp);"),
+    ("yarn_factor_multiplies", "return f / s * ramp + f * (1.0 - ramp);", "return f * s * ramp + f * (1.0 - ramp);"),
     ("tie_to_higher_index", "return (x->idx > y->idx) - (x->idx < y->idx);", "return (x->idx < y->idx) - (x->idx > y->idx);"),
     ("prev_block_not_forced", "for (int i = 0; i < budget - 2; ++i) sel[n++] = (int32_t)c[i].idx;\n  sel[n++] = (int32_t)(qb - 1);",
      "for (int i = 0; i < budget - 1; ++i) sel[n++] = (int32_t)c[i].idx;"),
