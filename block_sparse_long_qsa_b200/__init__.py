@@ -43,7 +43,9 @@ class qsa_params(ctypes.Structure):
     _fields_ = [("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("rope_dim", ctypes.c_int32), ("rope_theta", ctypes.c_double), ("idx_heads", ctypes.c_int32),
                 ("idx_dim", ctypes.c_int32), ("block_size", ctypes.c_int32), ("budget_blocks", ctypes.c_int32),
-                ("softmax_scale", ctypes.c_float), ("aggregation", ctypes.c_int32)]
+                ("softmax_scale", ctypes.c_float), ("aggregation", ctypes.c_int32),
+                ("yarn_factor", ctypes.c_double), ("yarn_original_max", ctypes.c_double),
+                ("yarn_beta_fast", ctypes.c_double), ("yarn_beta_slow", ctypes.c_double)]
 
 
 # block-score aggregation (qsa_params.aggregation)

@@ -39,6 +39,11 @@ qsa_status check_params(const qsa_params* p) {
   if (p->budget_blocks < 2 || p->budget_blocks > 4096) return QSA_ERR_UNSUPPORTED;
   if (!(p->softmax_scale >= 0.f) || !std::isfinite(p->softmax_scale)) return QSA_ERR_INVALID_ARG;
   if (p->aggregation != QSA_AGG_TOKEN_MAX && p->aggregation != QSA_AGG_MEAN_POOL) return QSA_ERR_INVALID_ARG;
+  if (!std::isfinite(p->yarn_factor) || p->yarn_factor < 0.0) return QSA_ERR_INVALID_ARG;
+  if (p->yarn_factor > 1.0 && !(p->yarn_original_max >= 1.0 && std::isfinite(p->yarn_original_max) &&
+                                p->yarn_beta_slow > 0.0 && p->yarn_beta_fast > p->yarn_beta_slow &&
+                                std::isfinite(p->yarn_beta_fast)))
+    return QSA_ERR_INVALID_ARG;
   return QSA_OK;
 }
 
@@ -50,9 +55,38 @@ float softmax_scale(const qsa_params* p) {
   return p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt((float)p->head_dim);
 }
 
+// Rotary frequencies of the 32 pairs, with static YaRN when yarn_factor > 1:
+// the pair index where the number of rotations over the original context,
+// L f_i / (2 pi), equals n is d ln(L / (2 pi n)) / (2 ln theta); pairs before
+// the beta_fast index (rounded down) keep f_i, pairs after the beta_slow index
+// (rounded up) take f_i / s, linear in the index in between.
 void inv_freq(const qsa_params* p, double* f) {
   const int half = p->rope_dim / 2;
-  for (int i = 0; i < half; ++i) f[i] = std::pow(p->rope_theta, -2.0 * (double)i / (double)p->rope_dim);
+  const double d = (double)p->rope_dim, s = p->yarn_factor;
+  double lo = 0.0, hi = 1.0;
+  if (s > 1.0) {
+    const double two_pi = 6.283185307179586476925286766559;
+    const double ln_theta = std::log(p->rope_theta);
+    lo = std::floor(d * std::log(p->yarn_original_max / (two_pi * p->yarn_beta_fast)) / (2.0 * ln_theta));
+    hi = std::ceil(d * std::log(p->yarn_original_max / (two_pi * p->yarn_beta_slow)) / (2.0 * ln_theta));
+    lo = std::max(lo, 0.0);
+    hi = std::min(hi, d - 1.0);
+    if (hi == lo) hi += 0.001;
+  }
+  for (int i = 0; i < half; ++i) {
+    const double base = std::pow(p->rope_theta, -2.0 * (double)i / d);
+    if (!(s > 1.0)) {
+      f[i] = base;
+      continue;
+    }
+    const double t = std::min(std::max(((double)i - lo) / (hi - lo), 0.0), 1.0);   // share of f / s
+    f[i] = base / s * t + base * (1.0 - t);
+  }
+}
+
+// YaRN's attention factor on the rotated dims (1 without YaRN).
+double rope_attn_factor(const qsa_params* p) {
+  return p->yarn_factor > 1.0 ? 0.1 * std::log(p->yarn_factor) + 1.0 : 1.0;
 }
 
 // --------------------------------------------------------------- device info
@@ -234,6 +268,10 @@ void qsa_default_params(qsa_params* p) {
   p->budget_blocks = 512;
   p->softmax_scale = 0.f;
   p->aggregation = QSA_AGG_TOKEN_MAX;
+  p->yarn_factor = 0.0;
+  p->yarn_original_max = 262144.0;
+  p->yarn_beta_fast = 32.0;
+  p->yarn_beta_slow = 1.0;
 }
 
 const char* qsa_last_error(void) { return g_last_error; }
@@ -368,8 +406,9 @@ qsa_status qsa_prefill(const qsa_params* p, int64_t T, int64_t pos0, const uint1
   if (cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaMemsetAsync");
   double f[32];
   inv_freq(p, f);
-  if ((st = from_cuda(traced(QSA_KERNEL_ROPE_TABLE, s, [&] { return qsa::launch_rope_table(T, pos0, f, cs, s); }))) !=
-      QSA_OK)
+  if ((st = from_cuda(traced(QSA_KERNEL_ROPE_TABLE, s, [&] {
+         return qsa::launch_rope_table(T, pos0, f, rope_attn_factor(p), cs, s);
+       }))) != QSA_OK)
     return st;
   if ((st = from_cuda(traced(QSA_KERNEL_ROPE_K, s, [&] { return qsa::launch_rope_k(T, k, cs, k_rot, s); }))) != QSA_OK)
     return st;
@@ -484,7 +523,7 @@ qsa_status qsa_prefill_cached(const qsa_params* p, int64_t L_old, int64_t T_new,
   double f[32];
   inv_freq(p, f);
   if ((st = from_cuda(traced(QSA_KERNEL_ROPE_TABLE, s, [&] {
-         return qsa::launch_rope_table(T_new, L_old, f, cs, s);
+         return qsa::launch_rope_table(T_new, L_old, f, rope_attn_factor(p), cs, s);
        }))) != QSA_OK)
     return st;
   if ((st = from_cuda(traced(QSA_KERNEL_ROPE_K, s, [&] {
@@ -641,8 +680,9 @@ qsa_status qsa_decode(const qsa_params* p, int32_t B, int64_t max_len, const int
   // the append kernel receives the lengths as launch parameters and stores
   // them (and L/4) in the workspace for the later kernels
   if ((st = from_cuda(traced(QSA_KERNEL_DECODE_APPEND, s, [&] {
-         return qsa::launch_decode_append(B, max_len, cache_len, Ls, qbs, f, k_cache, v_cache, kidx_cache, qidx_ring,
-                                          w_ring, q_new, k_new, v_new, q_idx_new, k_idx_new, w_new, q_rot, s);
+         return qsa::launch_decode_append(B, max_len, cache_len, Ls, qbs, f, rope_attn_factor(p), k_cache, v_cache,
+                                          kidx_cache, qidx_ring, w_ring, q_new, k_new, v_new, q_idx_new, k_idx_new,
+                                          w_new, q_rot, s);
        }))) != QSA_OK)
     return st;
   const float scale = 1.0f / std::sqrt(128.0f);

@@ -6,9 +6,10 @@
 
 namespace qsa {
 
-// RoPE angles of positions pos0 .. pos0+T-1: cs[t][i] = (cos a, sin a),
-// a = (pos0 + t) * inv_freq[i], i < 32, angle formed in fp64.
-cudaError_t launch_rope_table(int64_t T, int64_t pos0, const double* inv_freq_host, float2* cs, cudaStream_t s);
+// RoPE angles of positions pos0 .. pos0+T-1: cs[t][i] = attn_factor * (cos a,
+// sin a), a = (pos0 + t) * inv_freq[i], i < 32, angle formed in fp64.
+cudaError_t launch_rope_table(int64_t T, int64_t pos0, const double* inv_freq_host, double attn_factor, float2* cs,
+                              cudaStream_t s);
 // k_rot[t][g] = RoPE(k[t][g]) on dims 0..63, dims 64..255 copied.
 cudaError_t launch_rope_k(int64_t T, const uint16_t* k, const float2* cs, uint16_t* k_rot, cudaStream_t s);
 
@@ -51,7 +52,7 @@ cudaError_t launch_sparse_attn_prefill_tc(int64_t T, const uint16_t* q, const ui
 // Lengths come from the host array L_host (passed to the kernel as launch
 // parameters) and are stored to L_dev / qb_dev for the later kernels.
 cudaError_t launch_decode_append(int B, int64_t max_len, const int64_t* L_host, int64_t* L_dev, int64_t* qb_dev,
-                                 const double* inv_freq_host,
+                                 const double* inv_freq_host, double attn_factor,
                                  uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* qidx_ring,
                                  uint16_t* w_ring, const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
                                  const uint16_t* q_idx_new, const uint16_t* k_idx_new, const uint16_t* w_new,

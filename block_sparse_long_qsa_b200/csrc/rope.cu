@@ -4,17 +4,22 @@
 // (rope_dim 64 = partial_rotary_factor 0.25 of head_dim 256; page "Qwen3.8-
 // Flash-Next, 1/9의 학습 비용으로 Qwen3.7-Plus(397B-A17B) 수준에 도달한 125B-A6B
 // 모델", spec table and section "100만 토큰까지 늘리기").  Pairs are
-// (i, i + 32); angle a = position * theta^(-i/32), formed in fp64 so that
-// positions near 2^20 keep their phase, then rotated in fp32.
+// (i, i + 32); angle a = position * f_i with f_i = theta^(-i/32), or its
+// static-YaRN version (section "100만 토큰까지 늘리기": rope_type yarn,
+// factor 4) computed on the host, formed in fp64 so that positions near 2^20
+// keep their phase, then rotated in fp32; with YaRN the rotated dims are also
+// multiplied by the attention factor 0.1 ln(factor) + 1.
 #include "qsa_device.cuh"
 #include "qsa_kernels.h"
 
 namespace qsa {
 namespace {
 
-struct InvFreq { double f[32]; };
+// Frequencies of the 32 rotary pairs and the factor applied to the rotated
+// dims (YaRN's attention factor; 1 for plain RoPE).
+struct InvFreq { double f[32]; double scale; };
 
-// cs[t][i] = (cos a, sin a) for a = (pos0 + t) * inv_freq[i]
+// cs[t][i] = scale * (cos a, sin a) for a = (pos0 + t) * inv_freq[i]
 __global__ void rope_table_kernel(int64_t T, int64_t pos0, InvFreq inv, float2* __restrict__ cs) {
   const int64_t n = T * 32;
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
@@ -22,7 +27,7 @@ __global__ void rope_table_kernel(int64_t T, int64_t pos0, InvFreq inv, float2* 
     const int i = (int)(e & 31);
     double sa, ca;
     sincos((double)(pos0 + t) * inv.f[i], &sa, &ca);
-    cs[e] = make_float2((float)ca, (float)sa);
+    cs[e] = make_float2((float)(inv.scale * ca), (float)(inv.scale * sa));
   }
 }
 
@@ -87,7 +92,7 @@ __global__ void decode_append_kernel(int64_t max_len, LenChunk lens, int64_t* __
   if (threadIdx.x < 32) {
     double sa, ca;
     sincos((double)L * inv.f[threadIdx.x], &sa, &ca);
-    cs[threadIdx.x] = make_float2((float)ca, (float)sa);
+    cs[threadIdx.x] = make_float2((float)(inv.scale * ca), (float)(inv.scale * sa));
   }
   __syncthreads();
   // rotated rows: 2 kv heads (k) + 24 q heads, 4 rotate slots each; copies of the rest
@@ -116,9 +121,10 @@ __global__ void decode_append_kernel(int64_t max_len, LenChunk lens, int64_t* __
   if (threadIdx.x < 4) w_ring[((int64_t)b * 4 + slot) * 4 + threadIdx.x] = w_new[(int64_t)b * 4 + threadIdx.x];
 }
 
-InvFreq to_struct(const double* f) {
+InvFreq to_struct(const double* f, double scale) {
   InvFreq s;
   for (int i = 0; i < 32; ++i) s.f[i] = f[i];
+  s.scale = scale;
   return s;
 }
 
@@ -130,9 +136,10 @@ int grid_for(int64_t n, int threads) {
 
 }  // namespace
 
-cudaError_t launch_rope_table(int64_t T, int64_t pos0, const double* inv_freq_host, float2* cs, cudaStream_t s) {
+cudaError_t launch_rope_table(int64_t T, int64_t pos0, const double* inv_freq_host, double attn_factor, float2* cs,
+                              cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  rope_table_kernel<<<grid_for(T * 32, 256), 256, 0, s>>>(T, pos0, to_struct(inv_freq_host), cs);
+  rope_table_kernel<<<grid_for(T * 32, 256), 256, 0, s>>>(T, pos0, to_struct(inv_freq_host, attn_factor), cs);
   return cudaGetLastError();
 }
 
@@ -144,11 +151,12 @@ cudaError_t launch_rope_k(int64_t T, const uint16_t* k, const float2* cs, uint16
 }
 
 cudaError_t launch_decode_append(int B, int64_t max_len, const int64_t* L_host, int64_t* L_dev, int64_t* qb_dev,
-                                 const double* inv_freq_host, uint16_t* k_cache, uint16_t* v_cache,
-                                 uint16_t* kidx_cache, uint16_t* qidx_ring, uint16_t* w_ring, const uint16_t* q_new,
-                                 const uint16_t* k_new, const uint16_t* v_new, const uint16_t* q_idx_new,
-                                 const uint16_t* k_idx_new, const uint16_t* w_new, uint16_t* q_rot, cudaStream_t s) {
-  const InvFreq inv = to_struct(inv_freq_host);
+                                 const double* inv_freq_host, double attn_factor, uint16_t* k_cache,
+                                 uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* qidx_ring, uint16_t* w_ring,
+                                 const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
+                                 const uint16_t* q_idx_new, const uint16_t* k_idx_new, const uint16_t* w_new,
+                                 uint16_t* q_rot, cudaStream_t s) {
+  const InvFreq inv = to_struct(inv_freq_host, attn_factor);
   for (int b0 = 0; b0 < B; b0 += LEN_CHUNK) {
     const int n = B - b0 < LEN_CHUNK ? B - b0 : LEN_CHUNK;
     LenChunk lens;

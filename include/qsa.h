@@ -81,6 +81,19 @@ typedef struct {
   int32_t budget_blocks;
   float softmax_scale;
   int32_t aggregation;
+  /* Static YaRN on the rotary dims ([PT] "100만 토큰까지 늘리기": rope_type
+   * yarn, factor 4.0, original_max_position_embeddings 262144).  yarn_factor
+   * <= 1 (the default, 0) is plain RoPE.  With s = yarn_factor > 1 each
+   * rotary pair i keeps its frequency f_i = theta^(-i/32) if its wavelength
+   * fits more than yarn_beta_fast (default 32) times into
+   * yarn_original_max tokens, gets f_i / s if it fits fewer than
+   * yarn_beta_slow (default 1) times, and a linear mix in i in between
+   * (ends: the indices where the count crosses the two betas, rounded down /
+   * up); the rotated dims of q and k are multiplied by 0.1 ln s + 1. */
+  double yarn_factor;
+  double yarn_original_max;
+  double yarn_beta_fast;
+  double yarn_beta_slow;
 } qsa_params;
 
 /* Fills *p with the values above (budget 512). */
