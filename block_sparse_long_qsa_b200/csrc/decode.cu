@@ -83,14 +83,24 @@ decode_indexer_kernel(int64_t max_len, const int64_t* __restrict__ Ls, const uin
   const uint16_t* kb_base = kidx_cache + b * max_len * 128;
   float* Srow = S + b * ld;
 
-  for (int64_t jt = j_begin + 16 * warp; jt < j_end; jt += 16 * (THREADS / 32)) {
+  // the next tile's 16 keys are loaded while the current tile is scored
+  constexpr int64_t STEP = 16 * (THREADS / 32);
+  auto load_tile = [&](int64_t jt, uint4 (&k0)[4], uint4 (&k1)[4]) {
     const int64_t j0 = jt + g8, j1 = jt + g8 + 8;
     const int64_t r0 = j0 <= L ? j0 : L, r1 = j1 <= L ? j1 : L;
     const uint4* k0p = reinterpret_cast<const uint4*>(kb_base + r0 * 128);
     const uint4* k1p = reinterpret_cast<const uint4*>(kb_base + r1 * 128);
-    uint4 k0[4], k1[4];
 #pragma unroll
     for (int d = 0; d < 4; ++d) { k0[d] = ldg_stream(k0p + 4 * d + q4); k1[d] = ldg_stream(k1p + 4 * d + q4); }
+  };
+  uint4 n0[4], n1[4];
+  if (j_begin + 16 * warp < j_end) load_tile(j_begin + 16 * warp, n0, n1);
+  for (int64_t jt = j_begin + 16 * warp; jt < j_end; jt += STEP) {
+    const int64_t j0 = jt + g8, j1 = jt + g8 + 8;
+    uint4 k0[4], k1[4];
+#pragma unroll
+    for (int d = 0; d < 4; ++d) { k0[d] = n0[d]; k1[d] = n1[d]; }
+    if (jt + STEP < j_end) load_tile(jt + STEP, n0, n1);
     float acc[2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
