@@ -636,14 +636,14 @@ qsa_status qsa_decode_workspace_size(const qsa_params* p, int32_t B, int64_t max
   return QSA_OK;
 }
 
-qsa_status qsa_decode(const qsa_params* p, int32_t B, int64_t max_len, const int64_t* cache_len, uint16_t* k_cache,
-                      uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* qidx_ring, uint16_t* w_ring,
-                      const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new, const uint16_t* q_idx_new,
-                      const uint16_t* k_idx_new, const uint16_t* w_new, uint16_t* out, int32_t* sel_out,
-                      float* lse_out, void* ws, size_t ws_bytes, void* stream) {
-  qsa_status st = check_params(p);
-  if (st != QSA_OK) return st;
-  if (mean_pool(p)) return QSA_ERR_UNSUPPORTED;
+namespace {
+// One decode step; kbar_cache non-null only for the mean-pooled indexer.
+qsa_status decode_impl(const qsa_params* p, int32_t B, int64_t max_len, const int64_t* cache_len, uint16_t* k_cache,
+                       uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* kbar_cache, uint16_t* qidx_ring,
+                       uint16_t* w_ring, const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
+                       const uint16_t* q_idx_new, const uint16_t* k_idx_new, const uint16_t* w_new, uint16_t* out,
+                       int32_t* sel_out, float* lse_out, void* ws, size_t ws_bytes, void* stream) {
+  qsa_status st;
   if (B <= 0 || max_len <= 0 || !cache_len) return QSA_ERR_INVALID_ARG;
   if (B > 4096 || max_len > ((int64_t)1 << 24)) return QSA_ERR_UNSUPPORTED;
   const void* ptrs[] = {k_cache, v_cache, kidx_cache, qidx_ring, w_ring, q_new, k_new, v_new,
@@ -652,7 +652,9 @@ qsa_status qsa_decode(const qsa_params* p, int32_t B, int64_t max_len, const int
     if (!ptr) return QSA_ERR_INVALID_ARG;
     if (!aligned16(ptr)) return QSA_ERR_MISALIGNED;
   }
-  if ((sel_out && !aligned16(sel_out)) || (lse_out && !aligned16(lse_out))) return QSA_ERR_MISALIGNED;
+  if ((sel_out && !aligned16(sel_out)) || (lse_out && !aligned16(lse_out)) || (kbar_cache && !aligned16(kbar_cache)))
+    return QSA_ERR_MISALIGNED;
+  const int64_t kbar_len = (max_len + 3) / 4;
   int64_t max_L = 0;
   for (int b = 0; b < B; ++b) {
     if (cache_len[b] < 0 || cache_len[b] >= max_len) return QSA_ERR_INVALID_ARG;
@@ -682,12 +684,13 @@ qsa_status qsa_decode(const qsa_params* p, int32_t B, int64_t max_len, const int
   if ((st = from_cuda(traced(QSA_KERNEL_DECODE_APPEND, s, [&] {
          return qsa::launch_decode_append(B, max_len, cache_len, Ls, qbs, f, rope_attn_factor(p), k_cache, v_cache,
                                           kidx_cache, qidx_ring, w_ring, q_new, k_new, v_new, q_idx_new, k_idx_new,
-                                          w_new, q_rot, s);
+                                          w_new, q_rot, kbar_cache, kbar_len, s);
        }))) != QSA_OK)
     return st;
   const float scale = 1.0f / std::sqrt(128.0f);
   if ((st = from_cuda(traced(QSA_KERNEL_DECODE_INDEXER, s, [&] {
-         return qsa::launch_decode_indexer(B, max_len, max_L, Ls, kidx_cache, qidx_ring, w_ring, S, L.ld, scale, s);
+         return qsa::launch_decode_indexer(B, max_len, max_L, Ls, kidx_cache, kbar_cache, kbar_len, qidx_ring, w_ring,
+                                           S, L.ld, scale, s);
        }))) != QSA_OK)
     return st;
   if ((st = from_cuda(traced(QSA_KERNEL_SELECT, s, [&] {
@@ -707,6 +710,44 @@ qsa_status qsa_decode(const qsa_params* p, int32_t B, int64_t max_len, const int
   return from_cuda(traced(QSA_KERNEL_DECODE_COMBINE, s, [&] {
     return qsa::launch_decode_combine(B, part_o, part_lse, cnt, n_split, out, lse_out, s);
   }));
+}
+}  // namespace
+
+qsa_status qsa_decode(const qsa_params* p, int32_t B, int64_t max_len, const int64_t* cache_len, uint16_t* k_cache,
+                      uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* qidx_ring, uint16_t* w_ring,
+                      const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new, const uint16_t* q_idx_new,
+                      const uint16_t* k_idx_new, const uint16_t* w_new, uint16_t* out, int32_t* sel_out,
+                      float* lse_out, void* ws, size_t ws_bytes, void* stream) {
+  qsa_status st = check_params(p);
+  if (st != QSA_OK) return st;
+  if (mean_pool(p)) return QSA_ERR_UNSUPPORTED;   // needs the compressed-key cache: qsa_decode_mean_pool
+  return decode_impl(p, B, max_len, cache_len, k_cache, v_cache, kidx_cache, nullptr, qidx_ring, w_ring, q_new, k_new,
+                     v_new, q_idx_new, k_idx_new, w_new, out, sel_out, lse_out, ws, ws_bytes, stream);
+}
+
+qsa_status qsa_decode_mean_pool(const qsa_params* p, int32_t B, int64_t max_len, const int64_t* cache_len,
+                                uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* kbar_cache,
+                                uint16_t* qidx_ring, uint16_t* w_ring, const uint16_t* q_new, const uint16_t* k_new,
+                                const uint16_t* v_new, const uint16_t* q_idx_new, const uint16_t* k_idx_new,
+                                const uint16_t* w_new, uint16_t* out, int32_t* sel_out, float* lse_out, void* ws,
+                                size_t ws_bytes, void* stream) {
+  qsa_status st = check_params(p);
+  if (st != QSA_OK) return st;
+  if (!mean_pool(p)) return QSA_ERR_INVALID_ARG;
+  if (!kbar_cache) return QSA_ERR_INVALID_ARG;
+  return decode_impl(p, B, max_len, cache_len, k_cache, v_cache, kidx_cache, kbar_cache, qidx_ring, w_ring, q_new,
+                     k_new, v_new, q_idx_new, k_idx_new, w_new, out, sel_out, lse_out, ws, ws_bytes, stream);
+}
+
+qsa_status qsa_mean_pool_keys(const qsa_params* p, int64_t T, const uint16_t* k_idx, uint16_t* kbar, void* stream) {
+  qsa_status st = check_params(p);
+  if (st != QSA_OK) return st;
+  if (T <= 0 || !k_idx || !kbar) return QSA_ERR_INVALID_ARG;
+  if (T > ((int64_t)1 << 24)) return QSA_ERR_UNSUPPORTED;
+  if (!aligned16(k_idx) || !aligned16(kbar)) return QSA_ERR_MISALIGNED;
+  DevInfo di;
+  if ((st = device_info(&di)) != QSA_OK) return st;
+  return run_kbar(k_idx, T, kbar, static_cast<cudaStream_t>(stream));
 }
 
 qsa_status qsa_check_device_error(void* ws, void* stream) {

@@ -43,17 +43,25 @@ __device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
   return v;
 }
 
+// MEAN: the rows are mean-pooled key blocks (kbar_cache [B][kbar_len][128])
+// and S(qb, kb) is the max over the present block-mates of their score
+// against kbar[kb] (no per-key causal test: kb <= qb); otherwise the rows are
+// keys and S is the max over causal token pairs.
+template <bool MEAN>
 __global__ void __launch_bounds__(THREADS)
 decode_indexer_kernel(int64_t max_len, const int64_t* __restrict__ Ls, const uint16_t* __restrict__ kidx_cache,
+                      const uint16_t* __restrict__ kbar_cache, int64_t kbar_len,
                       const uint16_t* __restrict__ qidx_ring, const uint16_t* __restrict__ w_ring,
                       float* __restrict__ S, int64_t ld, float scale) {
   const int64_t b = blockIdx.y;
   const int64_t L = Ls[b];
   const int64_t qb = L >> 2;
+  const int64_t last_row = MEAN ? qb : L;              // last row with data
   const int64_t j_begin = (int64_t)blockIdx.x * KEYS_PER_CTA;
-  if (j_begin > L) return;
+  if (j_begin > last_row) return;
   int64_t j_end = j_begin + KEYS_PER_CTA;
-  if (j_end > 4 * qb + 4) j_end = 4 * qb + 4;
+  const int64_t rows_end = MEAN ? qb + 1 : 4 * qb + 4;
+  if (j_end > rows_end) j_end = rows_end;
   const int present = (int)(L - 4 * qb) + 1;        // block-mates 4qb .. L (ring slots 0 .. present-1)
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -80,14 +88,14 @@ decode_indexer_kernel(int64_t max_len, const int64_t* __restrict__ Ls, const uin
   }
   const int64_t t_tok = 4 * qb + q4;                 // this thread's query token
   const bool tok_ok = q4 < present;
-  const uint16_t* kb_base = kidx_cache + b * max_len * 128;
+  const uint16_t* kb_base = MEAN ? kbar_cache + b * kbar_len * 128 : kidx_cache + b * max_len * 128;
   float* Srow = S + b * ld;
 
   // the next tile's 16 keys are loaded while the current tile is scored
   constexpr int64_t STEP = 16 * (THREADS / 32);
   auto load_tile = [&](int64_t jt, uint4 (&k0)[4], uint4 (&k1)[4]) {
     const int64_t j0 = jt + g8, j1 = jt + g8 + 8;
-    const int64_t r0 = j0 <= L ? j0 : L, r1 = j1 <= L ? j1 : L;
+    const int64_t r0 = j0 <= last_row ? j0 : last_row, r1 = j1 <= last_row ? j1 : last_row;
     const uint4* k0p = reinterpret_cast<const uint4*>(kb_base + r0 * 128);
     const uint4* k1p = reinterpret_cast<const uint4*>(kb_base + r1 * 128);
 #pragma unroll
@@ -121,18 +129,33 @@ decode_indexer_kernel(int64_t max_len, const int64_t* __restrict__ Ls, const uin
     s1 = fmaf(w[1], fmaxf(acc[0][3], 0.f), s1);
     s1 = fmaf(w[2], fmaxf(acc[1][2], 0.f), s1);
     s1 = fmaf(w[3], fmaxf(acc[1][3], 0.f), s1);
-    s0 = (tok_ok && j0 <= t_tok) ? s0 : 0.f;
-    s1 = (tok_ok && j1 <= t_tok) ? s1 : 0.f;
-    // max over the 4 tokens (lanes q4), then over the 4 keys of a block (g8 % 4)
+    if constexpr (MEAN) {
+      s0 = (tok_ok && j0 <= qb) ? s0 : 0.f;
+      s1 = (tok_ok && j1 <= qb) ? s1 : 0.f;
+      // max over the 4 tokens (lanes q4); rows j0, j1 are key blocks
 #pragma unroll
-    for (int off = 1; off <= 8; off <<= 1) {
-      s0 = fmaxf(s0, __shfl_xor_sync(0xffffffffu, s0, off));
-      s1 = fmaxf(s1, __shfl_xor_sync(0xffffffffu, s1, off));
-    }
-    if ((lane & 15) == 0) {
-      const int64_t kb0 = (jt >> 2) + (lane >> 4);     // lane 0: blocks +0 / +2, lane 16: +1 / +3
-      if (kb0 <= qb) Srow[kb0] = s0 * scale;
-      if (kb0 + 2 <= qb) Srow[kb0 + 2] = s1 * scale;
+      for (int off = 1; off <= 2; off <<= 1) {
+        s0 = fmaxf(s0, __shfl_xor_sync(0xffffffffu, s0, off));
+        s1 = fmaxf(s1, __shfl_xor_sync(0xffffffffu, s1, off));
+      }
+      if (q4 == 0) {
+        if (j0 <= qb) Srow[j0] = s0 * scale;
+        if (j1 <= qb) Srow[j1] = s1 * scale;
+      }
+    } else {
+      s0 = (tok_ok && j0 <= t_tok) ? s0 : 0.f;
+      s1 = (tok_ok && j1 <= t_tok) ? s1 : 0.f;
+      // max over the 4 tokens (lanes q4), then over the 4 keys of a block (g8 % 4)
+#pragma unroll
+      for (int off = 1; off <= 8; off <<= 1) {
+        s0 = fmaxf(s0, __shfl_xor_sync(0xffffffffu, s0, off));
+        s1 = fmaxf(s1, __shfl_xor_sync(0xffffffffu, s1, off));
+      }
+      if ((lane & 15) == 0) {
+        const int64_t kb0 = (jt >> 2) + (lane >> 4);     // lane 0: blocks +0 / +2, lane 16: +1 / +3
+        if (kb0 <= qb) Srow[kb0] = s0 * scale;
+        if (kb0 + 2 <= qb) Srow[kb0 + 2] = s1 * scale;
+      }
     }
   }
 }
@@ -140,12 +163,19 @@ decode_indexer_kernel(int64_t max_len, const int64_t* __restrict__ Ls, const uin
 }  // namespace
 
 cudaError_t launch_decode_indexer(int B, int64_t max_len, int64_t max_L, const int64_t* L_dev,
-                                  const uint16_t* kidx_cache, const uint16_t* qidx_ring, const uint16_t* w_ring,
-                                  float* S, int64_t ld, float scale, cudaStream_t s) {
+                                  const uint16_t* kidx_cache, const uint16_t* kbar_cache, int64_t kbar_len,
+                                  const uint16_t* qidx_ring, const uint16_t* w_ring, float* S, int64_t ld,
+                                  float scale, cudaStream_t s) {
   if (B <= 0) return cudaSuccess;
-  const int64_t nx = (max_L + 4 + KEYS_PER_CTA - 1) / KEYS_PER_CTA;
+  const int64_t rows = kbar_cache ? max_L / 4 + 1 : max_L + 4;
+  const int64_t nx = (rows + KEYS_PER_CTA - 1) / KEYS_PER_CTA;
   dim3 grid((unsigned)nx, (unsigned)B);
-  decode_indexer_kernel<<<grid, THREADS, 0, s>>>(max_len, L_dev, kidx_cache, qidx_ring, w_ring, S, ld, scale);
+  if (kbar_cache)
+    decode_indexer_kernel<true><<<grid, THREADS, 0, s>>>(max_len, L_dev, kidx_cache, kbar_cache, kbar_len, qidx_ring,
+                                                         w_ring, S, ld, scale);
+  else
+    decode_indexer_kernel<false><<<grid, THREADS, 0, s>>>(max_len, L_dev, kidx_cache, nullptr, 0, qidx_ring, w_ring,
+                                                          S, ld, scale);
   return cudaGetLastError();
 }
 

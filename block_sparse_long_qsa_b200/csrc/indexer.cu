@@ -463,18 +463,6 @@ cudaError_t launch_indexer_prefill(const CUtensorMap& tm_q, const CUtensorMap& t
 // 4b .. min(4b + 4, T) - 1 (exact fp64 sum, one fp64 division, round to
 // nearest even), one thread per (block, dim).
 namespace {
-__device__ __forceinline__ uint16_t f64_to_bf16_rne_dev(double x) {
-  const uint64_t u = (uint64_t)__double_as_longlong(x);
-  const uint16_t sign = (uint16_t)((u >> 48) & 0x8000u);
-  const double a = fabs(x);
-  if (a == 0.0) return sign;
-  int e;
-  frexp(a, &e);                                   // a = m 2^e, m in [0.5, 1)
-  const int unit = e - 8 > -133 ? e - 8 : -133;   // weight of bf16's last bit
-  const double v = ldexp(rint(ldexp(a, -unit)), unit);   // rint: nearest, ties to even
-  return (uint16_t)(sign | (__float_as_uint((float)v) >> 16));   // v has <= 8 significant bits
-}
-
 __global__ void kbar_kernel(const uint16_t* __restrict__ k_idx, int64_t T, int64_t nkb, uint16_t* __restrict__ kbar) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= nkb * 128) return;
@@ -483,7 +471,7 @@ __global__ void kbar_kernel(const uint16_t* __restrict__ k_idx, int64_t T, int64
   const int n = (int)(T - t0 < 4 ? T - t0 : 4);
   double sum = 0.0;
   for (int r = 0; r < n; ++r) sum += (double)__uint_as_float((uint32_t)k_idx[(t0 + r) * 128 + c] << 16);
-  kbar[i] = f64_to_bf16_rne_dev(sum / (double)n);
+  kbar[i] = f64_to_bf16_rne(sum / (double)n);
 }
 }  // namespace
 

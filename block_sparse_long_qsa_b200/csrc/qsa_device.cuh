@@ -198,6 +198,19 @@ __device__ __forceinline__ uint32_t f32_to_bf16_bits(float f) {
   u += 0x7FFFu + ((u >> 16) & 1u);
   return u >> 16;
 }
+// fp64 -> bf16 bits, round to nearest even, subnormals included (for the
+// mean-pooled indexer keys, whose exact fp64 mean is rounded once).
+__device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
+  const uint64_t u = (uint64_t)__double_as_longlong(x);
+  const uint16_t sign = (uint16_t)((u >> 48) & 0x8000u);
+  const double a = fabs(x);
+  if (a == 0.0) return sign;
+  int e;
+  frexp(a, &e);                                   // a = m 2^e, m in [0.5, 1)
+  const int unit = e - 8 > -133 ? e - 8 : -133;   // weight of bf16's last bit
+  const double v = ldexp(rint(ldexp(a, -unit)), unit);   // rint: nearest, ties to even
+  return (uint16_t)(sign | (__float_as_uint((float)v) >> 16));   // v has <= 8 significant bits
+}
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return f32_to_bf16_bits(lo) | (f32_to_bf16_bits(hi) << 16);
 }

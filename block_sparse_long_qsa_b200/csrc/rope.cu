@@ -73,7 +73,8 @@ __global__ void rope_k_kernel(int64_t T, const uint4* __restrict__ k, const floa
 // Decode append: one CTA per sequence.
 //   k_cache[b][L] = RoPE(k_new[b], L); v_cache[b][L] = v_new[b];
 //   kidx_cache[b][L] = k_idx_new[b]; ring slot L % 4 <- (q_idx_new[b], w_new[b]);
-//   q_rot[b] = RoPE(q_new[b], L).
+//   q_rot[b] = RoPE(q_new[b], L); with kbar_cache (mean pooling, [B][kbar_len][128])
+//   the compressed key of block L/4 is recomputed from its present keys.
 constexpr int LEN_CHUNK = 1024;
 struct LenChunk { int64_t L[LEN_CHUNK]; int32_t b0; };
 
@@ -84,7 +85,8 @@ __global__ void decode_append_kernel(int64_t max_len, LenChunk lens, int64_t* __
                                      uint16_t* __restrict__ w_ring, const uint4* __restrict__ q_new,
                                      const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
                                      const uint4* __restrict__ q_idx_new, const uint4* __restrict__ k_idx_new,
-                                     const uint16_t* __restrict__ w_new, uint4* __restrict__ q_rot) {
+                                     const uint16_t* __restrict__ w_new, uint4* __restrict__ q_rot,
+                                     uint16_t* __restrict__ kbar_cache, int64_t kbar_len) {
   __shared__ float2 cs[32];
   const int b = lens.b0 + blockIdx.x;
   const int64_t L = lens.L[blockIdx.x];
@@ -119,6 +121,17 @@ __global__ void decode_append_kernel(int64_t max_len, LenChunk lens, int64_t* __
   for (int e = threadIdx.x; e < 64; e += blockDim.x)            // q_idx: 4 x 256 B
     qidx_ring[((int64_t)b * 4 + slot) * 64 + e] = q_idx_new[(int64_t)b * 64 + e];
   if (threadIdx.x < 4) w_ring[((int64_t)b * 4 + slot) * 4 + threadIdx.x] = w_new[(int64_t)b * 4 + threadIdx.x];
+  if (kbar_cache != nullptr && threadIdx.x < 128) {
+    // mean of keys 4 qb .. L: the earlier ones from the cache, the new one from k_idx_new
+    const int c = threadIdx.x;
+    const int64_t t0 = L & ~(int64_t)3;
+    const uint16_t* kc = reinterpret_cast<const uint16_t*>(kidx_cache) + (int64_t)b * max_len * 128;
+    const uint16_t* kn = reinterpret_cast<const uint16_t*>(k_idx_new) + (int64_t)b * 128;
+    double sum = 0.0;
+    for (int64_t t = t0; t < L; ++t) sum += (double)__uint_as_float((uint32_t)kc[t * 128 + c] << 16);
+    sum += (double)__uint_as_float((uint32_t)kn[c] << 16);
+    kbar_cache[((int64_t)b * kbar_len + (L >> 2)) * 128 + c] = f64_to_bf16_rne(sum / (double)(L - t0 + 1));
+  }
 }
 
 InvFreq to_struct(const double* f, double scale) {
@@ -155,7 +168,7 @@ cudaError_t launch_decode_append(int B, int64_t max_len, const int64_t* L_host, 
                                  uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* qidx_ring, uint16_t* w_ring,
                                  const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
                                  const uint16_t* q_idx_new, const uint16_t* k_idx_new, const uint16_t* w_new,
-                                 uint16_t* q_rot, cudaStream_t s) {
+                                 uint16_t* q_rot, uint16_t* kbar_cache, int64_t kbar_len, cudaStream_t s) {
   const InvFreq inv = to_struct(inv_freq_host, attn_factor);
   for (int b0 = 0; b0 < B; b0 += LEN_CHUNK) {
     const int n = B - b0 < LEN_CHUNK ? B - b0 : LEN_CHUNK;
@@ -167,7 +180,7 @@ cudaError_t launch_decode_append(int B, int64_t max_len, const int64_t* L_host, 
         reinterpret_cast<uint4*>(kidx_cache), reinterpret_cast<uint4*>(qidx_ring), w_ring,
         reinterpret_cast<const uint4*>(q_new), reinterpret_cast<const uint4*>(k_new),
         reinterpret_cast<const uint4*>(v_new), reinterpret_cast<const uint4*>(q_idx_new),
-        reinterpret_cast<const uint4*>(k_idx_new), w_new, reinterpret_cast<uint4*>(q_rot));
+        reinterpret_cast<const uint4*>(k_idx_new), w_new, reinterpret_cast<uint4*>(q_rot), kbar_cache, kbar_len);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

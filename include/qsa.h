@@ -67,7 +67,7 @@ typedef enum {
  *     sum_h w_h(t) ReLU(q_idx_h(t) . k-bar_kb) / sqrt(128), for kb <= qb (the
  *     own block's entry uses all its present keys and never decides a
  *     selection: the own block is always kept).  qsa_decode returns
- *     QSA_ERR_UNSUPPORTED for it. */
+ *     QSA_ERR_UNSUPPORTED for it; decode with it is qsa_decode_mean_pool. */
 enum { QSA_AGG_TOKEN_MAX = 0, QSA_AGG_MEAN_POOL = 1 };
 typedef struct {
   int32_t n_q_heads;
@@ -217,6 +217,24 @@ qsa_status qsa_decode(const qsa_params* p, int32_t B, int64_t max_len, const int
                       const uint16_t* q_idx_new, const uint16_t* k_idx_new, const uint16_t* w_new, uint16_t* out,
                       int32_t* sel_out, float* lse_out, void* ws, size_t ws_bytes, void* stream);
 qsa_status qsa_decode_workspace_size(const qsa_params* p, int32_t B, int64_t max_len, size_t* bytes);
+
+/* qsa_decode for p->aggregation == QSA_AGG_MEAN_POOL.  kbar_cache
+ * [B][ceil(max_len/4)][128] bf16 holds the compressed key of every block:
+ * block kb's row is bf16 (round to nearest even) of the mean of its present
+ * indexer keys (qsa_mean_pool_keys builds it from a k_idx cache).  The call
+ * appends the new token as qsa_decode does and rewrites the row of its block
+ * L/4 from the block's present keys (the cached ones and k_idx_new), then
+ * scores the compressed keys: the decode indexer reads one 256-byte row per
+ * block instead of four.  Same workspace as qsa_decode. */
+qsa_status qsa_decode_mean_pool(const qsa_params* p, int32_t B, int64_t max_len, const int64_t* cache_len,
+                                uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* kbar_cache,
+                                uint16_t* qidx_ring, uint16_t* w_ring, const uint16_t* q_new, const uint16_t* k_new,
+                                const uint16_t* v_new, const uint16_t* q_idx_new, const uint16_t* k_idx_new,
+                                const uint16_t* w_new, uint16_t* out, int32_t* sel_out, float* lse_out, void* ws,
+                                size_t ws_bytes, void* stream);
+/* kbar [ceil(T/4)][128] = the compressed keys of k_idx [T][128] (block b: bf16
+ * of the mean of rows 4b .. min(4b+4, T)-1); no workspace; asynchronous. */
+qsa_status qsa_mean_pool_keys(const qsa_params* p, int64_t T, const uint16_t* k_idx, uint16_t* kbar, void* stream);
 
 /* qsa_decode without a workspace argument; the pages have no counterpart:
  * this exists for callers that cannot allocate device memory where they run
