@@ -338,7 +338,7 @@ def run_prefill_cached(T: int, L_old: int, budget: int, steps: int, warmup: int,
 
 
 def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, world: int, seed: int,
-               want_e2e=True):
+               want_e2e=True, aggregation: int = 0):
     import block_sparse_long_qsa_b200 as qsa
     # one bench step = DECODE_CALLS consecutive decode tokens per sequence
     e_steps = max(1, min(steps, 3)) if want_e2e else 0
@@ -351,7 +351,13 @@ def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, 
     D.fill_device_caches(kc, vc, ic)
     ring = torch.zeros((B, 4, 4, 128), dtype=torch.uint16, device="cuda")
     wring = torch.zeros((B, 4, 4), dtype=torch.uint16, device="cuda")
-    p = qsa.params(budget)
+    p = qsa.params(budget, aggregation=aggregation)
+    kbar = None
+    if aggregation == 1:
+        # compressed-key cache of the cached prompt, kept up to date by each call
+        kbar = torch.zeros((B, (max_len + 3) // 4, 128), dtype=torch.uint16, device="cuda")
+        for b in range(B):
+            qsa.qsa_mean_pool_keys(p, L, ic[b], kbar[b])
     ws = qsa.workspace(qsa.qsa_decode_workspace_size(p, B, max_len))
     out = torch.empty((B, 24, 256), dtype=torch.uint16, device="cuda")
     # decode-token inputs of every call, generated once per sequence and kept resident: [call][B][...]
@@ -367,8 +373,12 @@ def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, 
     pos = [L]
 
     def call(x):
-        qsa.qsa_decode(p, B, max_len, [pos[0]] * B, kc, vc, ic, ring, wring, x["q"], x["k"], x["v"], x["q_idx"],
-                       x["k_idx"], x["w"], out, ws=ws, stream=stream)
+        if kbar is None:
+            qsa.qsa_decode(p, B, max_len, [pos[0]] * B, kc, vc, ic, ring, wring, x["q"], x["k"], x["v"], x["q_idx"],
+                           x["k_idx"], x["w"], out, ws=ws, stream=stream)
+        else:
+            qsa.qsa_decode_mean_pool(p, B, max_len, [pos[0]] * B, kc, vc, ic, kbar, ring, wring, x["q"], x["k"],
+                                     x["v"], x["q_idx"], x["k_idx"], x["w"], out, ws=ws, stream=stream)
         pos[0] += 1
 
     si = 0
@@ -407,6 +417,8 @@ def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, 
     # and the inputs / outputs
     n_timed = steps * DECODE_CALLS
     keys = B * (L_first + n_timed / 2 + 1)
+    if aggregation == 1:
+        keys /= 4            # one 256-byte compressed key per block
     gathered = B * min(budget, L_first // 4 + 1) * 4 * 2 * 2 * 256 * 2
     bytes_call = keys * 256 + gathered + B * (24 * 256 * 2 * 2 + 2 * 2 * 256 * 2 + 128 * 2 * 2)
     res = dict(ms=ms_max, tokens=B * n_timed * world, kern=kern, launches=sum(c for c, _ in kern.values()),
@@ -445,7 +457,7 @@ def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, 
         res["e2e"] = dict(value=B * DECODE_CALLS * e_steps * world / (ems / 1e3), unit="tokens/s",
                           h2d_bytes_per_step=bi, d2h_bytes_per_step=bo, steps=e_steps)
         del hosts, out_h
-    del kc, vc, ic, ws, step_in, allin
+    del kc, vc, ic, ws, step_in, allin, kbar
     torch.cuda.empty_cache()
     return res
 
@@ -467,10 +479,11 @@ def cpu_sample(wl: dict, target_s: float = 12.0):
             v, info = cpu_prefill_sample(wl["T"], 512, n2, qb_lo=qb_lo, aggregation=agg)
     else:
         n = 2
-        v, info = cpu_decode_sample(wl["B"], wl["L"], 512, n)
+        agg = wl.get("aggregation", 0)
+        v, info = cpu_decode_sample(wl["B"], wl["L"], 512, n, aggregation=agg)
         if info["elapsed"] < target_s / 3:
             n2 = int(min(wl["B"], max(n + 1, n * target_s / max(info["elapsed"], 1e-3))))
-            v, info = cpu_decode_sample(wl["B"], wl["L"], 512, n2)
+            v, info = cpu_decode_sample(wl["B"], wl["L"], 512, n2, aggregation=agg)
     return v, info
 
 
@@ -524,9 +537,9 @@ def cpu_prefill_sample(T: int, budget: int, n_blocks: int, seed: int = 0, qb_lo:
                                   elapsed=elapsed)
 
 
-def cpu_decode_sample(B: int, L: int, budget: int, n_seq: int, seed: int = 0):
+def cpu_decode_sample(B: int, L: int, budget: int, n_seq: int, seed: int = 0, aggregation: int = 0):
     import oracle
-    O = oracle.Oracle(oracle.params(budget=budget))
+    O = oracle.Oracle(oracle.params(budget=budget, aggregation=aggregation))
     D = Q.DecodeProblem(B=B, L=L, steps=1, seed=seed, n_plant=8)
     elapsed = 0.0
     for b in range(n_seq):
@@ -573,6 +586,7 @@ WORKLOADS = {
     "prefill_1m_cached90": dict(kind="prefill_cached", T=1 << 20, L_old=943718),
     # the pages' mean-pooled indexer (one compressed key per 4-token block)
     "prefill_1m_meanpool": dict(kind="prefill", T=1 << 20, aggregation=1),
+    "decode_64x256k_meanpool": dict(kind="decode", B=64, L=262144, aggregation=1),
 }
 
 
@@ -589,7 +603,8 @@ def metric_name(wl: dict) -> str:
     if wl["kind"] == "prefill_cached":
         return (f"QSA prefix-cached prefill new tokens/s at {wl['T'] // 1024}K context, "
                 f"{round(100 * wl['L_old'] / wl['T'])}% cached")
-    return "QSA decode tokens/s at 256K context, batch 64"
+    mp = ", mean-pooled indexer" if wl.get("aggregation") == 1 else ""
+    return f"QSA decode tokens/s at 256K context, batch 64{mp}"
 
 
 def line_for(name, res, n_gpus, steps, warmup, pk):
@@ -621,10 +636,11 @@ def line_for(name, res, n_gpus, steps, warmup, pk):
                     frac=achieved / pk["hbm"], traffic=NCU_TRAFFIC.get(name), peak_src=f"{pk['src']} HBM copy")
         whole = dict(gbs=res["bytes_step"] / (res["ms"] / res["steps"] / 1e3) / 1e9)
         whole["frac_of_hbm_roofline"] = whole["gbs"] / pk["hbm"]
-        metric = "QSA decode tokens/s at 256K context, batch 64"
+        metric = metric_name(wl)
         cfg = dict(workload=name, batch=B, context=L, budget_blocks=512, planted="8 per sequence",
                    decode_tokens_per_step=DECODE_CALLS,
-                   l2="4.3 GB of indexer keys streamed per decode token (larger than L2)")
+                   l2=("1.07 GB of compressed indexer keys" if wl.get("aggregation") == 1 else
+                       "4.3 GB of indexer keys") + " streamed per decode token (larger than L2)")
     return dict(metric=metric, value=value, unit="tokens/s", n_gpus=n_gpus, steps=steps, warmup=warmup,
                 ms_per_step=res["ms"] / steps, higher_is_better=True, scaling="weak", vs_baseline=None,
                 dtype="bf16", data="synthetic", config=cfg, roofline=roof, step_roofline=whole,
@@ -719,12 +735,13 @@ def main():
                                  want_e2e=not args.no_e2e)
     else:
         res = run_decode(wl["B"], wl["L"], 512, args.steps, args.warmup, rank, world, seed=0,
-                         want_e2e=not args.no_e2e)
+                         want_e2e=not args.no_e2e, aggregation=wl.get("aggregation", 0))
     line = line_for(args.workload, res, world, args.steps, args.warmup, pk)
 
     if not args.no_secondary:
         sec = {}
-        for name in ("decode_64x256k", "prefill_128k", "prefill_1m_cached90", "prefill_1m_meanpool"):
+        for name in ("decode_64x256k", "prefill_128k", "prefill_1m_cached90", "prefill_1m_meanpool",
+                     "decode_64x256k_meanpool"):
             if name == args.workload:
                 continue
             w2 = WORKLOADS[name]
@@ -736,7 +753,7 @@ def main():
                                         want_e2e=False)
             else:
                 r2 = run_decode(w2["B"], w2["L"], 512, args.steps, args.warmup, rank, world, seed=0,
-                                want_e2e=False)
+                                want_e2e=False, aggregation=w2.get("aggregation", 0))
             l2 = line_for(name, r2, world, args.steps, args.warmup, pk)
             sec[name] = {k: l2[k] for k in ("metric", "value", "unit", "ms_per_step", "roofline", "step_roofline",
                                             "gpu_launches", "kernels_ms")}
