@@ -68,6 +68,8 @@ def _bind(L):
     L.oracle_select_rows.argtypes = [P, vp, i64, i64, i64, vp, vp]
     L.oracle_attend_blocks.argtypes = [P, i64, i64, vp, vp, vp, i64, vp, vp, vp, vp, vp]
     L.oracle_prefill_blocks.argtypes = [P, i64, i64, vp, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp, vp]
+    L.oracle_reuse_selection.argtypes = [i64, vp, ctypes.c_int32, vp]
+    L.oracle_reuse_selection.restype = ctypes.c_int32
     L.oracle_select_blocks_list.argtypes = [P, i64, vp, vp, vp, i64, vp, vp, vp]
     L.oracle_decode.argtypes = [P, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp]
     return L
@@ -209,3 +211,21 @@ class Oracle:
         self.L.oracle_decode(ctypes.byref(self.P), L, *[_p(a) for a in args], _p(si), int(cnt_in), _p(sel), _p(cnt),
                              _p(out), _p(lse))
         return sel, int(cnt[0]), out, lse
+
+    def reuse_selection(self, qb, sel_in, cnt_in):
+        """Blocks a draft token of query block qb attends with a reused top-k
+        row (the row's first cnt_in entries joined with qb - 1 and qb)."""
+        si = np.ascontiguousarray(np.asarray(sel_in, dtype=np.int32)[:cnt_in])
+        out = np.empty(int(cnt_in) + 2, dtype=np.int32)
+        n = self.L.oracle_reuse_selection(int(qb), _p(si) if cnt_in else None, int(cnt_in), _p(out))
+        if n < 0:
+            raise ValueError("reused selection is not causal")
+        return out[:n], int(n)
+
+    def decode_reuse(self, L, k_cache, v_cache, kidx_cache, ring_q_idx, ring_w, q_new, k_new, v_new, q_idx_new,
+                     k_idx_new, w_new, sel_in, cnt_in):
+        """Draft decode token at position L over a reused top-k row."""
+        sel, n = self.reuse_selection(L // self.P.block, sel_in, cnt_in)
+        _, _, out, lse = self.decode(L, k_cache, v_cache, kidx_cache, ring_q_idx, ring_w, q_new, k_new, v_new,
+                                     q_idx_new, k_idx_new, w_new, sel_in=sel, cnt_in=n)
+        return sel, n, out, lse

@@ -417,10 +417,12 @@ void oracle_decode(const oracle_params* p, int64_t L, const uint16_t* k_cache, c
   if (L > 0) memcpy(keys, kidx_cache, sizeof(uint16_t) * (size_t)L * ID);
   memcpy(keys + L * ID, k_idx_new, sizeof(uint16_t) * (size_t)ID);
 
-  int32_t* sel = (int32_t*)malloc(sizeof(int32_t) * (size_t)p->budget);
+  /* a given selection may hold more than budget blocks (a reused one) */
+  int32_t cap = sel_in && cnt_in > p->budget ? cnt_in : p->budget;
+  int32_t* sel = (int32_t*)malloc(sizeof(int32_t) * (size_t)cap);
   int32_t cnt;
   if (sel_in) {
-    memcpy(sel, sel_in, sizeof(int32_t) * (size_t)p->budget);
+    for (int32_t i = 0; i < cap; ++i) sel[i] = i < cnt_in ? sel_in[i] : -1;
     cnt = cnt_in;
   } else {
     double* S = (double*)malloc(sizeof(double) * (size_t)(qb + 1));
@@ -431,7 +433,7 @@ void oracle_decode(const oracle_params* p, int64_t L, const uint16_t* k_cache, c
   if (sel_out) memcpy(sel_out, sel, sizeof(int32_t) * (size_t)p->budget);
   if (cnt_out) *cnt_out = cnt;
 
-  int64_t* js = (int64_t*)malloc(sizeof(int64_t) * (size_t)p->budget * r);
+  int64_t* js = (int64_t*)malloc(sizeof(int64_t) * (size_t)cap * r);
   int64_t n = gather_keys(p, sel, cnt, L, js);
   double* kr = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * G * d);
   double* vv = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * G * d);
@@ -456,4 +458,30 @@ void oracle_decode(const oracle_params* p, int64_t L, const uint16_t* k_cache, c
   }
   oracle_attend(p, qr, n, kr, vv, out, lse);
   free(qblk); free(wblk); free(keys); free(sel); free(js); free(kr); free(vv); free(x); free(qr);
+}
+
+/* ---------------------------------------------------------- top-k reuse --
+ * [PT] section "추측 디코딩을 위한 MTP와 그 밖에 유지된 설계": the MTP draft
+ * layer reuses the top-k indices between the steps of one speculative round
+ * (as GLM-5 does).  A later draft token at query block qb attends the reused
+ * set together with the blocks that stage 2 forces for every query block, its
+ * own block qb and qb - 1:
+ *   attended = sorted( {sel_in[i] : i < cnt_in}  U  {qb - 1, qb} ),
+ * qb - 1 only when qb >= 1.  Entries of sel_in must be causal (0 .. qb);
+ * returns -1 when one is not.  out holds at least cnt_in + 2 entries; returns
+ * the number written. */
+int32_t oracle_reuse_selection(int64_t qb, const int32_t* sel_in, int32_t cnt_in, int32_t* out) {
+  int64_t n_blocks = qb + 1;
+  unsigned char* in_set = (unsigned char*)calloc((size_t)n_blocks, 1);
+  for (int32_t i = 0; i < cnt_in; ++i) {
+    if (sel_in[i] < 0 || sel_in[i] > qb) { free(in_set); return -1; }
+    in_set[sel_in[i]] = 1;
+  }
+  in_set[qb] = 1;
+  if (qb >= 1) in_set[qb - 1] = 1;
+  int32_t n = 0;
+  for (int64_t b = 0; b < n_blocks; ++b)
+    if (in_set[b]) out[n++] = (int32_t)b;
+  free(in_set);
+  return n;
 }

@@ -474,4 +474,84 @@ def pin_decode_equals_prefill_last(O):
         assert np.linalg.norm(dout - out[i]) < 5e-3 * np.linalg.norm(out[i])
 
 
+
+# ---------------------------------------------------------------- top-k reuse
+def pin_reuse_selection_examples(O):
+    """The reused row joined with the token's forced blocks, worked by hand
+    from the rule (qb - 1 and qb always attended, the rest kept as given)."""
+    cases = [(5, [0, 2, 3], [0, 2, 3, 4, 5]),          # row of block 3 reused in block 5
+             (5, [1, 4, 5], [1, 4, 5]),                # own row: unchanged
+             (4, [0, 2, 3, 4], [0, 2, 3, 4]),
+             (4, [1, 2, 3], [1, 2, 3, 4]),             # row of block 3 reused in block 4
+             (0, [], [0]),
+             (0, [0], [0]),
+             (1, [0], [0, 1]),
+             (7, [0, 1, 2, 3], [0, 1, 2, 3, 6, 7]),
+             (9, [8], [8, 9])]
+    for qb, row, want in cases:
+        got, n = O.reuse_selection(qb, np.array(row, np.int32), len(row))
+        assert n == len(want) and list(got) == want, (qb, row, list(got))
+    for qb, row in ((3, [0, 4]), (2, [-1, 2])):
+        try:
+            O.reuse_selection(qb, np.array(row, np.int32), len(row))
+        except ValueError:
+            continue
+        raise AssertionError(f"non-causal row accepted: qb={qb} {row}")
+
+
+def pin_reuse_same_block_is_plain_decode(O):
+    """Reusing the row that the decode itself selects, at the same token or a
+    later token of the same query block (stage 2 already forced qb - 1, qb),
+    attends the same blocks: identical outputs at the same token."""
+    import oracle as OR
+    Ob = type(O)(OR.params(budget=6), O.L)
+    for L in (41, 44, 70):
+        P = Q.PrefillProblem(T=L + 1, seed=30 + L, n_plant=2)
+        h = P.host()
+        qb = L // 4
+        kf = np.stack([_rope_complex(Q.bf16_to_f64(h["k"][t]), t) for t in range(L)])
+        k_cache = Q.f32_to_bf16(kf.astype(np.float32))
+        t0 = 4 * qb
+        args = (L, k_cache, h["v"][:L], h["k_idx"][:L], h["q_idx"][t0:L], h["w"][t0:L], h["q"][L], h["k"][L],
+                h["v"][L], h["q_idx"][L], h["k_idx"][L], h["w"][L])
+        sel, cnt, out, lse = Ob.decode(*args)
+        rsel, rn, rout, rlse = Ob.decode_reuse(*args, sel_in=sel, cnt_in=cnt)
+        assert rn == cnt and np.array_equal(rsel, sel[:cnt]), L
+        assert np.array_equal(rout, out) and np.array_equal(rlse, lse), L
+        if L % 4 < 3:
+            again, n2 = Ob.reuse_selection((L + 1) // 4, sel, cnt)
+            assert n2 == cnt and np.array_equal(again, sel[:cnt])
+
+
+def pin_reuse_decode_brute(O):
+    """A draft token one block past the reused row: numpy softmax over exactly
+    the keys of the row's blocks and of qb - 1, qb up to the token."""
+    import oracle as OR
+    Ob = type(O)(OR.params(budget=4), O.L)
+    L = 50                                  # qb = 12
+    P = Q.PrefillProblem(T=L + 1, seed=77, n_plant=1)
+    h = P.host()
+    qb = L // 4
+    kf = np.stack([_rope_complex(Q.bf16_to_f64(h["k"][t]), t) for t in range(L)])
+    k_cache = Q.f32_to_bf16(kf.astype(np.float32))
+    row = np.array([2, 7, 10, 11], np.int32)   # a budget-4 row of block 11
+    t0 = 4 * qb
+    _, n, out, lse = Ob.decode_reuse(L, k_cache, h["v"][:L], h["k_idx"][:L], h["q_idx"][t0:L], h["w"][t0:L],
+                                     h["q"][L], h["k"][L], h["v"][L], h["q_idx"][L], h["k_idx"][L], h["w"][L],
+                                     sel_in=row, cnt_in=4)
+    assert n == 5
+    js = [j for b in (2, 7, 10, 11, 12) for j in range(4 * b, 4 * b + 4) if j <= L]
+    keys = np.concatenate([Q.bf16_to_f64(k_cache), _rope_complex(Q.bf16_to_f64(h["k"][L]), L)[None]])
+    vals = Q.bf16_to_f64(h["v"][:L + 1])
+    for hh in range(24):
+        g = hh // 12
+        q = _rope_complex(Q.bf16_to_f64(h["q"][L, hh]), L)
+        lg = np.array([q @ keys[j, g] for j in js]) / 16.0
+        m = lg.max()
+        e = np.exp(lg - m)
+        want = (e[:, None] * np.stack([vals[j, g] for j in js])).sum(0) / e.sum()
+        assert np.allclose(out[hh], want, rtol=1e-11, atol=1e-12), hh
+        assert abs(lse[hh] - (m + np.log(e.sum()))) < 1e-11
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -41,6 +41,9 @@ MUTANTS = [
     ("mean_ties_away_from_zero", "ldexp(nearbyint(ldexp(a, -unit)), unit)", "ldexp(round(ldexp(a, -unit)), unit)"),
     ("mean_pool_relu_dropped", "s += bf16_to_f64(w_blk[(int64_t)i * p->idx_heads + h]) * (dot > 0.0 ? dot : 0.0);",
      "s += bf16_to_f64(w_blk[(int64_t)i * p->idx_heads + h]) * dot;"),
+    ("reuse_own_block_not_forced", "  in_set[qb] = 1;\n", "\n"),
+    ("reuse_prev_block_not_forced", "  if (qb >= 1) in_set[qb - 1] = 1;\n", "\n"),
+    ("reuse_row_dropped", "    in_set[sel_in[i]] = 1;", "    in_set[sel_in[i]] = 0;"),
     ("decode_new_key_position", "oracle_rope(p, x, L, kr + (e * G + g) * d);", "oracle_rope(p, x, L - 1, kr + (e * G + g) * d);"),
 ]
 
