@@ -26,7 +26,8 @@ EXPORTED = ["qsa_default_params", "qsa_status_string", "qsa_last_error", "qsa_in
             "qsa_select_workspace_size", "qsa_prefill", "qsa_prefill_workspace_size", "qsa_decode",
             "qsa_decode_workspace_size", "qsa_check_device_error", "qsa_trace_begin", "qsa_trace_end",
             "qsa_decode_noalloc", "qsa_prefill_cached", "qsa_prefill_cached_workspace_size",
-            "qsa_index_workspace_size", "qsa_decode_mean_pool", "qsa_mean_pool_keys"]
+            "qsa_index_workspace_size", "qsa_decode_mean_pool", "qsa_mean_pool_keys",
+            "qsa_decode_reuse"]
 
 KERNEL_NAMES = {1: "rope_table", 2: "rope_k", 3: "indexer", 4: "select", 5: "attention", 6: "decode_append",
                 7: "decode_indexer", 8: "decode_attention", 9: "decode_combine",
@@ -85,6 +86,7 @@ def load(path: str = LIB_PATH):
     L.qsa_decode_workspace_size.argtypes = [P, i32, i64, psz]
     L.qsa_decode_mean_pool.argtypes = [P, i32, i64, ctypes.POINTER(ctypes.c_int64)] + [vp] * 15 + [vp, sz, vp]
     L.qsa_mean_pool_keys.argtypes = [P, i64, vp, vp, vp]
+    L.qsa_decode_reuse.argtypes = [P, i32, i64, ctypes.POINTER(ctypes.c_int64)] + [vp] * 16 + [vp, sz, vp]
     L.qsa_decode_noalloc.argtypes = [P, i32, i64, ctypes.POINTER(ctypes.c_int64), vp, vp, vp, vp, vp, vp, vp, vp,
                                      vp, vp, vp, vp, vp, vp, vp]
     L.qsa_check_device_error.argtypes = [vp, vp]
@@ -209,6 +211,19 @@ def qsa_decode_mean_pool(p: qsa_params, B: int, max_len: int, cache_len, k_cache
                                        _ptr(q_new), _ptr(k_new), _ptr(v_new), _ptr(q_idx_new), _ptr(k_idx_new),
                                        _ptr(w_new), _ptr(out), _ptr(sel_out), _ptr(lse_out), _ptr(ws),
                                        ws.numel() * ws.element_size(), _stream(stream)), "qsa_decode_mean_pool")
+
+
+def qsa_decode_reuse(p: qsa_params, B: int, max_len: int, cache_len, k_cache, v_cache, kidx_cache, kbar_cache,
+                     qidx_ring, w_ring, q_new, k_new, v_new, q_idx_new, k_idx_new, w_new, sel_in, cnt_in, out,
+                     lse_out=None, ws=None, stream=None):
+    """Draft decode step over a reused selection (``kbar_cache`` None unless
+    the parameters select mean pooling)."""
+    lens = (ctypes.c_int64 * B)(*[int(x) for x in cache_len])
+    _check(load().qsa_decode_reuse(ctypes.byref(p), B, max_len, lens, _ptr(k_cache), _ptr(v_cache), _ptr(kidx_cache),
+                                   _ptr(kbar_cache), _ptr(qidx_ring), _ptr(w_ring), _ptr(q_new), _ptr(k_new),
+                                   _ptr(v_new), _ptr(q_idx_new), _ptr(k_idx_new), _ptr(w_new), _ptr(sel_in),
+                                   _ptr(cnt_in), _ptr(out), _ptr(lse_out), _ptr(ws), ws.numel() * ws.element_size(),
+                                   _stream(stream)), "qsa_decode_reuse")
 
 
 def qsa_mean_pool_keys(p: qsa_params, T: int, k_idx, kbar, stream=None):

@@ -581,8 +581,9 @@ qsa_status qsa_prefill_cached(const qsa_params* p, int64_t L_old, int64_t T_new,
 // ------------------------------------------------------------------ decode
 namespace {
 struct DecodeLayout {
-  size_t Ls, qbs, S, sel, cnt, q_rot, part_o, part_lse, total;
+  size_t Ls, qbs, S, sel, sel_r, cnt, q_rot, part_o, part_lse, total;
   int64_t ld;
+  int sel_r_ld;   // row stride of the merged reused selections
 };
 // Split-KV ranges per (sequence, KV head): at most this many.
 constexpr int DECODE_MAX_SPLIT = 16;
@@ -594,6 +595,8 @@ DecodeLayout decode_layout(int B, int64_t max_len, int budget) {
   L.qbs = off; off = align_up(off + (size_t)B * 8);
   L.S = off; off = align_up(off + (size_t)B * L.ld * 4);
   L.sel = off; off = align_up(off + (size_t)B * budget * 4);
+  L.sel_r_ld = budget + 4;
+  L.sel_r = off; off = align_up(off + (size_t)B * L.sel_r_ld * 4);
   L.cnt = off; off = align_up(off + (size_t)B * 4);
   L.q_rot = off; off = align_up(off + (size_t)B * 24 * 256 * 2);
   L.part_o = off; off = align_up(off + (size_t)B * 2 * DECODE_MAX_SPLIT * 12 * 256 * 4);
@@ -637,12 +640,16 @@ qsa_status qsa_decode_workspace_size(const qsa_params* p, int32_t B, int64_t max
 }
 
 namespace {
-// One decode step; kbar_cache non-null only for the mean-pooled indexer.
+// One decode step; kbar_cache non-null only for the mean-pooled indexer;
+// sel_in / cnt_in non-null: stages 1 and 2 are skipped, the append kernel
+// merges each given selection with the token's forced blocks into the sel_r
+// region and the attention reads that.
 qsa_status decode_impl(const qsa_params* p, int32_t B, int64_t max_len, const int64_t* cache_len, uint16_t* k_cache,
                        uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* kbar_cache, uint16_t* qidx_ring,
                        uint16_t* w_ring, const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
                        const uint16_t* q_idx_new, const uint16_t* k_idx_new, const uint16_t* w_new, uint16_t* out,
-                       int32_t* sel_out, float* lse_out, void* ws, size_t ws_bytes, void* stream) {
+                       int32_t* sel_out, float* lse_out, void* ws, size_t ws_bytes, void* stream,
+                       const int32_t* sel_in = nullptr, const int32_t* cnt_in = nullptr) {
   qsa_status st;
   if (B <= 0 || max_len <= 0 || !cache_len) return QSA_ERR_INVALID_ARG;
   if (B > 4096 || max_len > ((int64_t)1 << 24)) return QSA_ERR_UNSUPPORTED;
@@ -672,7 +679,10 @@ qsa_status decode_impl(const qsa_params* p, int32_t B, int64_t max_len, const in
   int64_t* Ls = reinterpret_cast<int64_t*>(base + L.Ls);
   int64_t* qbs = reinterpret_cast<int64_t*>(base + L.qbs);
   float* S = reinterpret_cast<float*>(base + L.S);
-  int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(base + L.sel);
+  const bool reuse = sel_in != nullptr;
+  int32_t* sel_r = reinterpret_cast<int32_t*>(base + L.sel_r);
+  int32_t* sel = reuse ? sel_r : (sel_out ? sel_out : reinterpret_cast<int32_t*>(base + L.sel));
+  const int sel_ld = reuse ? L.sel_r_ld : budget;
   int32_t* cnt = reinterpret_cast<int32_t*>(base + L.cnt);
   uint16_t* q_rot = reinterpret_cast<uint16_t*>(base + L.q_rot);
 
@@ -684,25 +694,29 @@ qsa_status decode_impl(const qsa_params* p, int32_t B, int64_t max_len, const in
   if ((st = from_cuda(traced(QSA_KERNEL_DECODE_APPEND, s, [&] {
          return qsa::launch_decode_append(B, max_len, cache_len, Ls, qbs, f, rope_attn_factor(p), k_cache, v_cache,
                                           kidx_cache, qidx_ring, w_ring, q_new, k_new, v_new, q_idx_new, k_idx_new,
-                                          w_new, q_rot, kbar_cache, kbar_len, s);
+                                          w_new, q_rot, kbar_cache, kbar_len, sel_in, cnt_in, budget, sel_r, L.sel_r_ld,
+                                          cnt, err, s);
        }))) != QSA_OK)
     return st;
   const float scale = 1.0f / std::sqrt(128.0f);
-  if ((st = from_cuda(traced(QSA_KERNEL_DECODE_INDEXER, s, [&] {
-         return qsa::launch_decode_indexer(B, max_len, max_L, Ls, kidx_cache, kbar_cache, kbar_len, qidx_ring, w_ring,
-                                           S, L.ld, scale, s);
-       }))) != QSA_OK)
-    return st;
-  if ((st = from_cuda(traced(QSA_KERNEL_SELECT, s, [&] {
-         return qsa::launch_select(S, L.ld, nullptr, 0, 0, B, qbs, budget, sel, cnt, err, s);
-       }))) != QSA_OK)
-    return st;
+  if (!reuse) {
+    if ((st = from_cuda(traced(QSA_KERNEL_DECODE_INDEXER, s, [&] {
+           return qsa::launch_decode_indexer(B, max_len, max_L, Ls, kidx_cache, kbar_cache, kbar_len, qidx_ring,
+                                             w_ring, S, L.ld, scale, s);
+         }))) != QSA_OK)
+      return st;
+    if ((st = from_cuda(traced(QSA_KERNEL_SELECT, s, [&] {
+           return qsa::launch_select(S, L.ld, nullptr, 0, 0, B, qbs, budget, sel, cnt, err, s);
+         }))) != QSA_OK)
+      return st;
+  }
   const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
-  const int n_split = decode_splits(B, max_L, budget, di.num_sms);
+  // a merged reused selection holds at most budget + 2 blocks
+  const int n_split = decode_splits(B, max_L, reuse ? budget + 2 : budget, di.num_sms);
   float* part_o = reinterpret_cast<float*>(base + L.part_o);
   float* part_lse = reinterpret_cast<float*>(base + L.part_lse);
   if ((st = from_cuda(traced(QSA_KERNEL_DECODE_ATTENTION, s, [&] {
-         return qsa::launch_decode_attn_tc(B, max_len, Ls, q_rot, k_cache, v_cache, sel, cnt, budget, scale_log2,
+         return qsa::launch_decode_attn_tc(B, max_len, Ls, q_rot, k_cache, v_cache, sel, cnt, sel_ld, scale_log2,
                                            n_split, part_o, part_lse, out, lse_out, err, di.num_sms, s);
        }))) != QSA_OK)
     return st;
@@ -737,6 +751,21 @@ qsa_status qsa_decode_mean_pool(const qsa_params* p, int32_t B, int64_t max_len,
   if (!kbar_cache) return QSA_ERR_INVALID_ARG;
   return decode_impl(p, B, max_len, cache_len, k_cache, v_cache, kidx_cache, kbar_cache, qidx_ring, w_ring, q_new,
                      k_new, v_new, q_idx_new, k_idx_new, w_new, out, sel_out, lse_out, ws, ws_bytes, stream);
+}
+
+qsa_status qsa_decode_reuse(const qsa_params* p, int32_t B, int64_t max_len, const int64_t* cache_len,
+                            uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* kbar_cache,
+                            uint16_t* qidx_ring, uint16_t* w_ring, const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
+                            const uint16_t* q_idx_new, const uint16_t* k_idx_new, const uint16_t* w_new,
+                            const int32_t* sel_in, const int32_t* cnt_in, uint16_t* out, float* lse_out, void* ws,
+                            size_t ws_bytes, void* stream) {
+  qsa_status st = check_params(p);
+  if (st != QSA_OK) return st;
+  if (!sel_in || !cnt_in) return QSA_ERR_INVALID_ARG;
+  if (!aligned16(sel_in) || !aligned16(cnt_in)) return QSA_ERR_MISALIGNED;
+  if (mean_pool(p) != (kbar_cache != nullptr)) return QSA_ERR_INVALID_ARG;   // the cache is kept for that mode only
+  return decode_impl(p, B, max_len, cache_len, k_cache, v_cache, kidx_cache, kbar_cache, qidx_ring, w_ring, q_new, k_new,
+                     v_new, q_idx_new, k_idx_new, w_new, out, nullptr, lse_out, ws, ws_bytes, stream, sel_in, cnt_in);
 }
 
 qsa_status qsa_mean_pool_keys(const qsa_params* p, int64_t T, const uint16_t* k_idx, uint16_t* kbar, void* stream) {

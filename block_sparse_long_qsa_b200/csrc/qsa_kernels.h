@@ -56,7 +56,9 @@ cudaError_t launch_decode_append(int B, int64_t max_len, const int64_t* L_host, 
                                  uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* qidx_ring,
                                  uint16_t* w_ring, const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
                                  const uint16_t* q_idx_new, const uint16_t* k_idx_new, const uint16_t* w_new,
-                                 uint16_t* q_rot, uint16_t* kbar_cache, int64_t kbar_len, cudaStream_t s);
+                                 uint16_t* q_rot, uint16_t* kbar_cache, int64_t kbar_len, const int32_t* sel_in,
+                                 const int32_t* cnt_in, int budget, int32_t* sel_r, int sel_r_ld, int32_t* cnt_r,
+                                 uint32_t* err, cudaStream_t s);
 // kbar_cache (nullable, [B][kbar_len][128]): score the mean-pooled key blocks
 // (aggregation = mean pool) instead of the keys.
 cudaError_t launch_decode_indexer(int B, int64_t max_len, int64_t max_L, const int64_t* L_dev,

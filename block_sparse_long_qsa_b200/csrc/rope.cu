@@ -86,11 +86,47 @@ __global__ void decode_append_kernel(int64_t max_len, LenChunk lens, int64_t* __
                                      const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
                                      const uint4* __restrict__ q_idx_new, const uint4* __restrict__ k_idx_new,
                                      const uint16_t* __restrict__ w_new, uint4* __restrict__ q_rot,
-                                     uint16_t* __restrict__ kbar_cache, int64_t kbar_len) {
+                                     uint16_t* __restrict__ kbar_cache, int64_t kbar_len,
+                                     const int32_t* __restrict__ sel_in, const int32_t* __restrict__ cnt_in,
+                                     int budget, int32_t* __restrict__ sel_r, int sel_r_ld,
+                                     int32_t* __restrict__ cnt_r, uint32_t* err) {
   __shared__ float2 cs[32];
+  __shared__ int n_keep;
   const int b = lens.b0 + blockIdx.x;
   const int64_t L = lens.L[blockIdx.x];
-  if (threadIdx.x == 0) { L_dev[b] = L; qb_dev[b] = L >> 2; }
+  if (threadIdx.x == 0) {
+    L_dev[b] = L;
+    qb_dev[b] = L >> 2;
+    n_keep = 0;
+  }
+  if (sel_in != nullptr) {
+    // Reused selection (an earlier step's top-k of this sequence): its blocks
+    // below qb - 1, then the forced blocks qb - 1 and qb of this token.  The
+    // given row must be ascending, distinct and causal (<= qb); otherwise the
+    // step attends nothing and reports QSA_ERR_DEVICE_BOUNDS.
+    const int64_t qb = L >> 2;
+    const int c = cnt_in[b];
+    const bool c_ok = c >= 0 && c <= budget;
+    const int32_t* r = sel_in + (int64_t)b * budget;
+    int bad = !c_ok, keep = 0;
+    for (int i = threadIdx.x; c_ok && i < c; i += blockDim.x) {
+      const int32_t v = r[i];
+      bad |= v < 0 || v > qb || (i > 0 && v <= r[i - 1]);
+      keep += v < qb - 1;
+    }
+    __syncthreads();   // n_keep initialised
+    if (keep) atomicAdd(&n_keep, keep);
+    bad = __syncthreads_or(bad);
+    const int m = n_keep;   // entries below qb - 1 form a prefix of an ascending row
+    int32_t* o = sel_r + (int64_t)b * sel_r_ld;
+    for (int i = threadIdx.x; !bad && i < m; i += blockDim.x) o[i] = r[i];
+    if (threadIdx.x == 0) {
+      if (qb >= 1) o[m] = (int32_t)(qb - 1);
+      o[m + (qb >= 1)] = (int32_t)qb;
+      cnt_r[b] = bad ? 0 : m + 1 + (qb >= 1);
+      if (bad) report_error(err, QSA_ERR_DEVICE_BOUNDS);
+    }
+  }
   if (threadIdx.x < 32) {
     double sa, ca;
     sincos((double)L * inv.f[threadIdx.x], &sa, &ca);
@@ -168,7 +204,9 @@ cudaError_t launch_decode_append(int B, int64_t max_len, const int64_t* L_host, 
                                  uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* qidx_ring, uint16_t* w_ring,
                                  const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
                                  const uint16_t* q_idx_new, const uint16_t* k_idx_new, const uint16_t* w_new,
-                                 uint16_t* q_rot, uint16_t* kbar_cache, int64_t kbar_len, cudaStream_t s) {
+                                 uint16_t* q_rot, uint16_t* kbar_cache, int64_t kbar_len, const int32_t* sel_in,
+                                 const int32_t* cnt_in, int budget, int32_t* sel_r, int sel_r_ld, int32_t* cnt_r,
+                                 uint32_t* err, cudaStream_t s) {
   const InvFreq inv = to_struct(inv_freq_host, attn_factor);
   for (int b0 = 0; b0 < B; b0 += LEN_CHUNK) {
     const int n = B - b0 < LEN_CHUNK ? B - b0 : LEN_CHUNK;
@@ -180,7 +218,8 @@ cudaError_t launch_decode_append(int B, int64_t max_len, const int64_t* L_host, 
         reinterpret_cast<uint4*>(kidx_cache), reinterpret_cast<uint4*>(qidx_ring), w_ring,
         reinterpret_cast<const uint4*>(q_new), reinterpret_cast<const uint4*>(k_new),
         reinterpret_cast<const uint4*>(v_new), reinterpret_cast<const uint4*>(q_idx_new),
-        reinterpret_cast<const uint4*>(k_idx_new), w_new, reinterpret_cast<uint4*>(q_rot), kbar_cache, kbar_len);
+        reinterpret_cast<const uint4*>(k_idx_new), w_new, reinterpret_cast<uint4*>(q_rot), kbar_cache, kbar_len,
+        sel_in, cnt_in, budget, sel_r, sel_r_ld, cnt_r, err);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

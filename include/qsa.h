@@ -232,6 +232,30 @@ qsa_status qsa_decode_mean_pool(const qsa_params* p, int32_t B, int64_t max_len,
                                 const uint16_t* v_new, const uint16_t* q_idx_new, const uint16_t* k_idx_new,
                                 const uint16_t* w_new, uint16_t* out, int32_t* sel_out, float* lse_out, void* ws,
                                 size_t ws_bytes, void* stream);
+/* One draft decode step that reuses an earlier step's top-k ([PT] section
+ * "추측 디코딩을 위한 MTP와 그 밖에 유지된 설계": the MTP draft layer keeps the
+ * top-k indices across the steps of one speculative round, as GLM-5 does, so
+ * the later draft steps pay neither the indexer nor the top-k).  The new token
+ * is appended exactly as by qsa_decode (and, with p->aggregation ==
+ * QSA_AGG_MEAN_POOL, its block's compressed key is rewritten in kbar_cache as
+ * by qsa_decode_mean_pool; kbar_cache must be NULL otherwise).  Stages 1 and 2
+ * do not run: the attended blocks of sequence b are the blocks of
+ * sel_in[b][0 .. cnt_in[b]) below qb - 1, followed by the forced blocks
+ * qb - 1 (when qb >= 1) and qb of the new token (qb = cache_len[b] / 4), so a
+ * reused row taken in an earlier query block still attends the token's own
+ * block and the one before it; at most cnt_in[b] + 2 blocks.
+ * sel_in [B][budget] int32, cnt_in [B] int32 (device): typically sel_out of
+ * the round's first qsa_decode step and the number of its non-negative
+ * entries.  Each row must be ascending, distinct and causal (entries in
+ * 0 .. qb, 0 <= cnt_in[b] <= budget); a row that is not attends nothing and
+ * QSA_ERR_DEVICE_BOUNDS is recorded in the workspace.  Other arguments,
+ * outputs and the workspace are those of qsa_decode. */
+qsa_status qsa_decode_reuse(const qsa_params* p, int32_t B, int64_t max_len, const int64_t* cache_len,
+                            uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* kbar_cache,
+                            uint16_t* qidx_ring, uint16_t* w_ring, const uint16_t* q_new, const uint16_t* k_new,
+                            const uint16_t* v_new, const uint16_t* q_idx_new, const uint16_t* k_idx_new,
+                            const uint16_t* w_new, const int32_t* sel_in, const int32_t* cnt_in, uint16_t* out,
+                            float* lse_out, void* ws, size_t ws_bytes, void* stream);
 /* kbar [ceil(T/4)][128] = the compressed keys of k_idx [T][128] (block b: bf16
  * of the mean of rows 4b .. min(4b+4, T)-1); no workspace; asynchronous. */
 qsa_status qsa_mean_pool_keys(const qsa_params* p, int64_t T, const uint16_t* k_idx, uint16_t* kbar, void* stream);
