@@ -338,9 +338,11 @@ def run_prefill_cached(T: int, L_old: int, budget: int, steps: int, warmup: int,
 
 
 def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, world: int, seed: int,
-               want_e2e=True, aggregation: int = 0):
+               want_e2e=True, aggregation: int = 0, spec: int = 0):
     import block_sparse_long_qsa_b200 as qsa
-    # one bench step = DECODE_CALLS consecutive decode tokens per sequence
+    # one bench step = DECODE_CALLS consecutive decode tokens per sequence; with
+    # spec = n they form rounds of n draft steps: a full decode step, whose
+    # selection the next n - 1 steps reuse (qsa_decode_reuse)
     e_steps = max(1, min(steps, 3)) if want_e2e else 0
     n_calls = (warmup + steps + e_steps) * DECODE_CALLS
     D = Q.DecodeProblem(B=B, L=L, steps=n_calls, seed=seed + 1000 * rank, n_plant=8)
@@ -360,6 +362,7 @@ def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, 
             qsa.qsa_mean_pool_keys(p, L, ic[b], kbar[b])
     ws = qsa.workspace(qsa.qsa_decode_workspace_size(p, B, max_len))
     out = torch.empty((B, 24, 256), dtype=torch.uint16, device="cuda")
+    sel_round = torch.empty((B, budget), dtype=torch.int32, device="cuda") if spec > 1 else None
     # decode-token inputs of every call, generated once per sequence and kept resident: [call][B][...]
     names = ["q", "k", "v", "q_idx", "k_idx", "w"]
     per_seq = [D.tokens(b) for b in range(B)]
@@ -373,12 +376,16 @@ def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, 
     pos = [L]
 
     def call(x):
-        if kbar is None:
+        if spec > 1 and (pos[0] - L) % spec != 0:
+            qsa.qsa_decode_reuse(p, B, max_len, [pos[0]] * B, kc, vc, ic, kbar, ring, wring, x["q"], x["k"], x["v"],
+                                 x["q_idx"], x["k_idx"], x["w"], sel_round, None, out, ws=ws, stream=stream)
+        elif kbar is None:
             qsa.qsa_decode(p, B, max_len, [pos[0]] * B, kc, vc, ic, ring, wring, x["q"], x["k"], x["v"], x["q_idx"],
-                           x["k_idx"], x["w"], out, ws=ws, stream=stream)
+                           x["k_idx"], x["w"], out, sel_out=sel_round, ws=ws, stream=stream)
         else:
             qsa.qsa_decode_mean_pool(p, B, max_len, [pos[0]] * B, kc, vc, ic, kbar, ring, wring, x["q"], x["k"],
-                                     x["v"], x["q_idx"], x["k_idx"], x["w"], out, ws=ws, stream=stream)
+                                     x["v"], x["q_idx"], x["k_idx"], x["w"], out, sel_out=sel_round, ws=ws,
+                                     stream=stream)
         pos[0] += 1
 
     si = 0
@@ -420,7 +427,10 @@ def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, 
     if aggregation == 1:
         keys /= 4            # one 256-byte compressed key per block
     gathered = B * min(budget, L_first // 4 + 1) * 4 * 2 * 2 * 256 * 2
-    bytes_call = keys * 256 + gathered + B * (24 * 256 * 2 * 2 + 2 * 2 * 256 * 2 + 128 * 2 * 2)
+    io = B * (24 * 256 * 2 * 2 + 2 * 2 * 256 * 2 + 128 * 2 * 2)
+    # the indexer keys are read only by the calls that select
+    select_share = 1.0 / spec if spec > 1 else 1.0
+    bytes_call = keys * 256 * select_share + gathered + io
     res = dict(ms=ms_max, tokens=B * n_timed * world, kern=kern, launches=sum(c for c, _ in kern.values()),
                clocks=clk.summary(), bytes_step=bytes_call * DECODE_CALLS, bytes_indexer=keys * 256,
                steps=steps, calls=n_timed)
@@ -457,7 +467,7 @@ def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, 
         res["e2e"] = dict(value=B * DECODE_CALLS * e_steps * world / (ems / 1e3), unit="tokens/s",
                           h2d_bytes_per_step=bi, d2h_bytes_per_step=bo, steps=e_steps)
         del hosts, out_h
-    del kc, vc, ic, ws, step_in, allin, kbar
+    del kc, vc, ic, ws, step_in, allin, kbar, sel_round
     torch.cuda.empty_cache()
     return res
 
@@ -480,10 +490,11 @@ def cpu_sample(wl: dict, target_s: float = 12.0):
     else:
         n = 2
         agg = wl.get("aggregation", 0)
-        v, info = cpu_decode_sample(wl["B"], wl["L"], 512, n, aggregation=agg)
+        spec = wl.get("spec", 0)
+        v, info = cpu_decode_sample(wl["B"], wl["L"], 512, n, aggregation=agg, spec=spec)
         if info["elapsed"] < target_s / 3:
             n2 = int(min(wl["B"], max(n + 1, n * target_s / max(info["elapsed"], 1e-3))))
-            v, info = cpu_decode_sample(wl["B"], wl["L"], 512, n2, aggregation=agg)
+            v, info = cpu_decode_sample(wl["B"], wl["L"], 512, n2, aggregation=agg, spec=spec)
     return v, info
 
 
@@ -537,7 +548,8 @@ def cpu_prefill_sample(T: int, budget: int, n_blocks: int, seed: int = 0, qb_lo:
                                   elapsed=elapsed)
 
 
-def cpu_decode_sample(B: int, L: int, budget: int, n_seq: int, seed: int = 0, aggregation: int = 0):
+def cpu_decode_sample(B: int, L: int, budget: int, n_seq: int, seed: int = 0, aggregation: int = 0,
+                      spec: int = 0):
     import oracle
     O = oracle.Oracle(oracle.params(budget=budget, aggregation=aggregation))
     D = Q.DecodeProblem(B=B, L=L, steps=1, seed=seed, n_plant=8)
@@ -560,12 +572,21 @@ def cpu_decode_sample(B: int, L: int, budget: int, n_seq: int, seed: int = 0, ag
             if a1 > a0:
                 kc[a0:a1] = D.cache_k(b, a0, a1)
                 vc[a0:a1] = D.cache_v(b, a0, a1)
+        # attention on that selection (timed); with spec = n also the n - 1
+        # draft tokens of the round that reuse it
         t1 = time.time()
-        O.decode(L, kc, vc, kid, np.zeros((0, 4, 128), np.uint16), np.zeros((0, 4), np.uint16), x["q"], x["k"],
-                 x["v"], x["q_idx"], kidx_new, x["w"])
+        ring_q, ring_w = np.zeros((0, 4, 128), np.uint16), np.zeros((0, 4), np.uint16)
+        O.decode(L, kc, vc, kid, ring_q, ring_w, x["q"], x["k"], x["v"], x["q_idx"], kidx_new, x["w"],
+                 sel_in=sel, cnt_in=cnt)
+        for _ in range(max(spec, 1) - 1):
+            O.decode_reuse(L, kc, vc, kid, ring_q, ring_w, x["q"], x["k"], x["v"], x["q_idx"], kidx_new, x["w"],
+                           sel_in=sel, cnt_in=cnt)
         elapsed += t_sel + (time.time() - t1)
-    return n_seq / elapsed, dict(sample=f"{n_seq} of {B} sequences, one decode token each at {L} cached tokens "
-                                        f"(scores + selection + attention), {elapsed:.1f} s", elapsed=elapsed)
+    per = max(spec, 1)
+    what = ("one decode token each" if per == 1 else
+            f"a round of {per} draft tokens each (one selection, {per - 1} reusing it; all at position {L})")
+    return n_seq * per / elapsed, dict(sample=f"{n_seq} of {B} sequences, {what} at {L} cached tokens "
+                                              f"(scores + selection + attention), {elapsed:.1f} s", elapsed=elapsed)
 
 
 def cores_used():
@@ -587,6 +608,8 @@ WORKLOADS = {
     # the pages' mean-pooled indexer (one compressed key per 4-token block)
     "prefill_1m_meanpool": dict(kind="prefill", T=1 << 20, aggregation=1),
     "decode_64x256k_meanpool": dict(kind="decode", B=64, L=262144, aggregation=1),
+    # speculative rounds of 4 draft tokens: one selection, reused by the next 3
+    "decode_64x256k_spec4": dict(kind="decode", B=64, L=262144, spec=4),
 }
 
 
@@ -604,6 +627,8 @@ def metric_name(wl: dict) -> str:
         return (f"QSA prefix-cached prefill new tokens/s at {wl['T'] // 1024}K context, "
                 f"{round(100 * wl['L_old'] / wl['T'])}% cached")
     mp = ", mean-pooled indexer" if wl.get("aggregation") == 1 else ""
+    if wl.get("spec"):
+        mp += f", top-k reused across {wl['spec']}-step speculative rounds"
     return f"QSA decode tokens/s at 256K context, batch 64{mp}"
 
 
@@ -638,7 +663,7 @@ def line_for(name, res, n_gpus, steps, warmup, pk):
         whole["frac_of_hbm_roofline"] = whole["gbs"] / pk["hbm"]
         metric = metric_name(wl)
         cfg = dict(workload=name, batch=B, context=L, budget_blocks=512, planted="8 per sequence",
-                   decode_tokens_per_step=DECODE_CALLS,
+                   decode_tokens_per_step=DECODE_CALLS, speculative_round=wl.get("spec") or None,
                    l2=("1.07 GB of compressed indexer keys" if wl.get("aggregation") == 1 else
                        "4.3 GB of indexer keys") + " streamed per decode token (larger than L2)")
     return dict(metric=metric, value=value, unit="tokens/s", n_gpus=n_gpus, steps=steps, warmup=warmup,
@@ -735,13 +760,13 @@ def main():
                                  want_e2e=not args.no_e2e)
     else:
         res = run_decode(wl["B"], wl["L"], 512, args.steps, args.warmup, rank, world, seed=0,
-                         want_e2e=not args.no_e2e, aggregation=wl.get("aggregation", 0))
+                         want_e2e=not args.no_e2e, aggregation=wl.get("aggregation", 0), spec=wl.get("spec", 0))
     line = line_for(args.workload, res, world, args.steps, args.warmup, pk)
 
     if not args.no_secondary:
         sec = {}
         for name in ("decode_64x256k", "prefill_128k", "prefill_1m_cached90", "prefill_1m_meanpool",
-                     "decode_64x256k_meanpool"):
+                     "decode_64x256k_meanpool", "decode_64x256k_spec4"):
             if name == args.workload:
                 continue
             w2 = WORKLOADS[name]
@@ -753,7 +778,7 @@ def main():
                                         want_e2e=False)
             else:
                 r2 = run_decode(w2["B"], w2["L"], 512, args.steps, args.warmup, rank, world, seed=0,
-                                want_e2e=False, aggregation=w2.get("aggregation", 0))
+                                want_e2e=False, aggregation=w2.get("aggregation", 0), spec=w2.get("spec", 0))
             l2 = line_for(name, r2, world, args.steps, args.warmup, pk)
             sec[name] = {k: l2[k] for k in ("metric", "value", "unit", "ms_per_step", "roofline", "step_roofline",
                                             "gpu_launches", "kernels_ms")}

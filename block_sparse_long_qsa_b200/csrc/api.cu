@@ -761,8 +761,8 @@ qsa_status qsa_decode_reuse(const qsa_params* p, int32_t B, int64_t max_len, con
                             size_t ws_bytes, void* stream) {
   qsa_status st = check_params(p);
   if (st != QSA_OK) return st;
-  if (!sel_in || !cnt_in) return QSA_ERR_INVALID_ARG;
-  if (!aligned16(sel_in) || !aligned16(cnt_in)) return QSA_ERR_MISALIGNED;
+  if (!sel_in) return QSA_ERR_INVALID_ARG;
+  if (!aligned16(sel_in) || (cnt_in && !aligned16(cnt_in))) return QSA_ERR_MISALIGNED;
   if (mean_pool(p) != (kbar_cache != nullptr)) return QSA_ERR_INVALID_ARG;   // the cache is kept for that mode only
   return decode_impl(p, B, max_len, cache_len, k_cache, v_cache, kidx_cache, kbar_cache, qidx_ring, w_ring, q_new, k_new,
                      v_new, q_idx_new, k_idx_new, w_new, out, nullptr, lse_out, ws, ws_bytes, stream, sel_in, cnt_in);

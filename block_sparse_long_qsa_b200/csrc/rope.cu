@@ -91,30 +91,38 @@ __global__ void decode_append_kernel(int64_t max_len, LenChunk lens, int64_t* __
                                      int budget, int32_t* __restrict__ sel_r, int sel_r_ld,
                                      int32_t* __restrict__ cnt_r, uint32_t* err) {
   __shared__ float2 cs[32];
-  __shared__ int n_keep;
+  __shared__ int n_keep, first_neg;
   const int b = lens.b0 + blockIdx.x;
   const int64_t L = lens.L[blockIdx.x];
   if (threadIdx.x == 0) {
     L_dev[b] = L;
     qb_dev[b] = L >> 2;
     n_keep = 0;
+    first_neg = budget;
   }
   if (sel_in != nullptr) {
     // Reused selection (an earlier step's top-k of this sequence): its blocks
     // below qb - 1, then the forced blocks qb - 1 and qb of this token.  The
     // given row must be ascending, distinct and causal (<= qb); otherwise the
-    // step attends nothing and reports QSA_ERR_DEVICE_BOUNDS.
+    // step attends nothing and reports QSA_ERR_DEVICE_BOUNDS.  Without
+    // counts a row ends at its first negative entry (the -1 padding of
+    // sel_out).
     const int64_t qb = L >> 2;
-    const int c = cnt_in[b];
-    const bool c_ok = c >= 0 && c <= budget;
     const int32_t* r = sel_in + (int64_t)b * budget;
+    __syncthreads();   // n_keep, first_neg initialised
+    if (cnt_in == nullptr) {
+      for (int i = threadIdx.x; i < budget; i += blockDim.x)
+        if (r[i] < 0) atomicMin(&first_neg, i);
+      __syncthreads();
+    }
+    const int c = cnt_in != nullptr ? cnt_in[b] : first_neg;
+    const bool c_ok = c >= 0 && c <= budget;
     int bad = !c_ok, keep = 0;
     for (int i = threadIdx.x; c_ok && i < c; i += blockDim.x) {
       const int32_t v = r[i];
       bad |= v < 0 || v > qb || (i > 0 && v <= r[i - 1]);
       keep += v < qb - 1;
     }
-    __syncthreads();   // n_keep initialised
     if (keep) atomicAdd(&n_keep, keep);
     bad = __syncthreads_or(bad);
     const int m = n_keep;   // entries below qb - 1 form a prefix of an ascending row

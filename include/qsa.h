@@ -244,11 +244,12 @@ qsa_status qsa_decode_mean_pool(const qsa_params* p, int32_t B, int64_t max_len,
  * qb - 1 (when qb >= 1) and qb of the new token (qb = cache_len[b] / 4), so a
  * reused row taken in an earlier query block still attends the token's own
  * block and the one before it; at most cnt_in[b] + 2 blocks.
- * sel_in [B][budget] int32, cnt_in [B] int32 (device): typically sel_out of
- * the round's first qsa_decode step and the number of its non-negative
- * entries.  Each row must be ascending, distinct and causal (entries in
- * 0 .. qb, 0 <= cnt_in[b] <= budget); a row that is not attends nothing and
- * QSA_ERR_DEVICE_BOUNDS is recorded in the workspace.  Other arguments,
+ * sel_in [B][budget] int32, cnt_in [B] int32 (device; nullable): typically
+ * sel_out of the round's first qsa_decode step.  With cnt_in NULL a row ends
+ * at its first negative entry (the -1 padding of sel_out), else it holds
+ * cnt_in[b] entries.  Each row must be ascending, distinct and causal
+ * (entries in 0 .. qb, 0 <= cnt_in[b] <= budget); a row that is not attends
+ * nothing and QSA_ERR_DEVICE_BOUNDS is recorded in the workspace.  Other arguments,
  * outputs and the workspace are those of qsa_decode. */
 qsa_status qsa_decode_reuse(const qsa_params* p, int32_t B, int64_t max_len, const int64_t* cache_len,
                             uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* kbar_cache,
