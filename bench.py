@@ -96,15 +96,20 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- distributed
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, backend: str | None = None):
+    """One process per GPU (RANK / LOCAL_RANK / WORLD_SIZE / MASTER_* from the
+    launcher).  NCCL on GPUs; gloo when there is no GPU (the host-side tests)."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    cuda = torch.cuda.is_available()
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
-    else:
+        if cuda:
+            torch.cuda.set_device(local)
+        torch.distributed.init_process_group(backend or ("nccl" if cuda else "gloo"),
+                                             timeout=datetime.timedelta(seconds=600))
+    elif cuda:
         torch.cuda.set_device(0)
     return rank, world, local
 
@@ -115,11 +120,18 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The slowest rank's time: every rank's number, reduced with MAX."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Weak scaling: every rank draws its own independent sequences."""
+    return seed + 1000 * rank
 
 
 # ------------------------------------------------------------ prefill workload
@@ -139,7 +151,7 @@ def prefill_flops(T: int, sel_cnt: np.ndarray | None):
 def run_prefill(T: int, budget: int, steps: int, warmup: int, rank: int, world: int, seed: int, want_e2e=True,
                 aggregation: int = 0):
     import block_sparse_long_qsa_b200 as qsa
-    P = Q.PrefillProblem(T=T, seed=seed + 1000 * rank, n_plant=8, dist="zipf" if T >= 131072 else "uniform")
+    P = Q.PrefillProblem(T=T, seed=rank_seed(seed, rank), n_plant=8, dist="zipf" if T >= 131072 else "uniform")
     d = P.device()
     torch.cuda.synchronize()
     p = qsa.params(budget, aggregation=aggregation)
@@ -253,7 +265,7 @@ def run_prefill_cached(T: int, L_old: int, budget: int, steps: int, warmup: int,
     the same cache rows with the same values."""
     import block_sparse_long_qsa_b200 as qsa
     T_new = T - L_old
-    P = Q.PrefillProblem(T=T, seed=seed + 1000 * rank, n_plant=8, dist="zipf" if T >= 131072 else "uniform")
+    P = Q.PrefillProblem(T=T, seed=rank_seed(seed, rank), n_plant=8, dist="zipf" if T >= 131072 else "uniform")
     d = P.device()
     # caches: synthetic keys stand in for rotated ones (timing only)
     kc, vc, ic = d["k"].clone(), d["v"].clone(), d["k_idx"].clone()
@@ -345,7 +357,7 @@ def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, 
     # selection the next n - 1 steps reuse (qsa_decode_reuse)
     e_steps = max(1, min(steps, 3)) if want_e2e else 0
     n_calls = (warmup + steps + e_steps) * DECODE_CALLS
-    D = Q.DecodeProblem(B=B, L=L, steps=n_calls, seed=seed + 1000 * rank, n_plant=8)
+    D = Q.DecodeProblem(B=B, L=L, steps=n_calls, seed=rank_seed(seed, rank), n_plant=8)
     max_len = L + n_calls + 4
     kc = torch.empty((B, max_len, 2, 256), dtype=torch.uint16, device="cuda")
     vc = torch.empty_like(kc)
