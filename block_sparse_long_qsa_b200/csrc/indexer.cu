@@ -26,6 +26,8 @@
 //     max -> fp32 scores), each 32-column load in flight behind the previous chunk.
 //   * Every mbarrier wait is bounded; on timeout the CTA records
 //     QSA_ERR_DEVICE_TIMEOUT, drains and exits.
+#include <type_traits>
+
 #include "qsa_device.cuh"
 #include "qsa_kernels.h"
 
@@ -283,123 +285,135 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
       const int64_t warp_first_key = MEAN ? 4 * (KT * it.kt + 32 * quad) : KT * it.kt + 32 * quad;
       const bool live = warp_first_key <= (t_first + 31) && qb_first < qb_end;
       if (live) {
+        // The causal test is needed only where the key tile reaches past the
+        // first token of this thread's columns; the drain is compiled twice so
+        // the common (unmasked) copy carries no per-score test.
         const bool masked = kt_last_key > t_first;
-        float m[8];
-        // 8 tokens (32 columns) of this key's row -> the maxima of query blocks 2c, 2c+1
-        auto chunk = [&](const float (&v)[32], int c) {
-#pragma unroll
-          for (int half_blk = 0; half_blk < 2; ++half_blk) {
-            float sc[4];
-#pragma unroll
-            for (int pr = 0; pr < 2; ++pr) {
-              // tokens tl and tl+1 at once: packed f32x2 multiply-adds over the 4 heads.
-              // The ReLU of heads 0, 1 runs on the ALU (max), that of heads 2, 3 on the
-              // FMA pipe (saturating multiply by 2^-64, undone by the scaled weights).
-              const int tl = 8 * c + 4 * half_blk + 2 * pr;   // token index within the 32 columns
-              const float* x0 = &v[4 * (tl & 7)];
-              const float* x1 = x0 + 4;
-              const float4 wa = *reinterpret_cast<const float4*>(wrow + 4 * tl);       // heads 0, 1
-              const float4 wb = *reinterpret_cast<const float4*>(wrow + 4 * tl + 4);   // heads 2, 3 (x 2^64)
-              uint64_t acc = mul2(pk2(fmaxf(x0[0], 0.f), fmaxf(x1[0], 0.f)), pk2(wa.x, wa.y));
-              acc = fma2(pk2(fmaxf(x0[1], 0.f), fmaxf(x1[1], 0.f)), pk2(wa.z, wa.w), acc);
-              acc = fma2(pk2(relu_scaled(x0[2]), relu_scaled(x1[2])), pk2(wb.x, wb.y), acc);
-              acc = fma2(pk2(relu_scaled(x0[3]), relu_scaled(x1[3])), pk2(wb.z, wb.w), acc);
-              float s0, s1;
-              upk2(acc, s0, s1);
-              if (masked) {
-                s0 = (j <= t_first + tl) ? s0 : 0.f;
-                s1 = (j <= t_first + tl + 1) ? s1 : 0.f;
+        auto drain = [&](auto mtag) {
+          constexpr bool MASKED = decltype(mtag)::value;
+          // key position relative to the first column token: where MASKED the
+          // key tile ends after t_first and the warp's first key is at most
+          // t_first + 31, so -512 < jd < 160
+          const int jd = MASKED ? (int)(j - t_first) : 0;
+          float m[8];
+          // 8 tokens (32 columns) of this key's row -> the maxima of query blocks 2c, 2c+1
+          auto chunk = [&](const float (&v)[32], int c) {
+  #pragma unroll
+            for (int half_blk = 0; half_blk < 2; ++half_blk) {
+              float sc[4];
+  #pragma unroll
+              for (int pr = 0; pr < 2; ++pr) {
+                // tokens tl and tl+1 at once: packed f32x2 multiply-adds over the 4 heads.
+                // The ReLU of heads 0, 1 runs on the ALU (max), that of heads 2, 3 on the
+                // FMA pipe (saturating multiply by 2^-64, undone by the scaled weights).
+                const int tl = 8 * c + 4 * half_blk + 2 * pr;   // token index within the 32 columns
+                const float* x0 = &v[4 * (tl & 7)];
+                const float* x1 = x0 + 4;
+                const float4 wa = *reinterpret_cast<const float4*>(wrow + 4 * tl);       // heads 0, 1
+                const float4 wb = *reinterpret_cast<const float4*>(wrow + 4 * tl + 4);   // heads 2, 3 (x 2^64)
+                uint64_t acc = mul2(pk2(fmaxf(x0[0], 0.f), fmaxf(x1[0], 0.f)), pk2(wa.x, wa.y));
+                acc = fma2(pk2(fmaxf(x0[1], 0.f), fmaxf(x1[1], 0.f)), pk2(wa.z, wa.w), acc);
+                acc = fma2(pk2(relu_scaled(x0[2]), relu_scaled(x1[2])), pk2(wb.x, wb.y), acc);
+                acc = fma2(pk2(relu_scaled(x0[3]), relu_scaled(x1[3])), pk2(wb.z, wb.w), acc);
+                float s0, s1;
+                upk2(acc, s0, s1);
+                if constexpr (MASKED) {
+                  s0 = (jd <= tl) ? s0 : 0.f;
+                  s1 = (jd <= tl + 1) ? s1 : 0.f;
+                }
+                sc[2 * pr] = s0;
+                sc[2 * pr + 1] = s1;
               }
-              sc[2 * pr] = s0;
-              sc[2 * pr + 1] = s1;
+              m[2 * c + half_blk] = fmaxf(max3f(sc[0], sc[1], sc[2]), sc[3]);
             }
-            m[2 * c + half_blk] = fmaxf(max3f(sc[0], sc[1], sc[2]), sc[3]);
-          }
-        };
-        // four 32-column loads, each in flight while the previous chunk is scored
-        const uint32_t base = tmem + lane_addr + hf * 256 + 128 * cgrp;
-        float va[32], vb[32];
-        tmem_ld32(base, va);
-        tmem_ld_wait(va);
-        tmem_ld32(base + 32, vb);
-        chunk(va, 0);
-        tmem_ld_wait(vb);
-        tmem_ld32(base + 64, va);
-        chunk(vb, 1);
-        tmem_ld_wait(va);
-        tmem_ld32(base + 96, vb);
-        chunk(va, 2);
-        tmem_ld_wait(vb);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&accempty[hf]);
-        chunk(vb, 3);
-        if constexpr (MEAN) {
-          // one key block per lane: the 8 block maxima are the scores
-          // S(qb_first + b, kb), stored by the 32 lanes as 32 consecutive floats
-          float* srow = S + (qb_first - qb_begin) * ld + kb;
-          const int nb = (int)(qb_end - qb_first < 8 ? qb_end - qb_first : 8);
-#pragma unroll
-          for (int b = 0; b < 8; ++b) {
-            if (b < nb && kb <= qb_first + b) srow[b * ld] = m[b] * scale;
-          }
-          if (segmax != nullptr) {
-            // segment maxima over 8 key blocks = 8 lanes (bits 0..2): three
-            // transposing steps leave lane (a, b, c) of each 8-lane group with
-            // the maximum of query block qb_first + 4 a + 2 b + c
-            const bool la = (lane & 1) != 0, lb = (lane & 2) != 0, lc = (lane & 4) != 0;
-            float n4[4], n2[2];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              n4[i] = fmaxf(la ? m[i + 4] : m[i], __shfl_xor_sync(0xffffffffu, la ? m[i] : m[i + 4], 1));
-#pragma unroll
-            for (int i = 0; i < 2; ++i)
-              n2[i] = fmaxf(lb ? n4[i + 2] : n4[i], __shfl_xor_sync(0xffffffffu, lb ? n4[i] : n4[i + 2], 2));
-            const float sm = fmaxf(lc ? n2[1] : n2[0], __shfl_xor_sync(0xffffffffu, lc ? n2[0] : n2[1], 4));
-            const int64_t seg = (KT * it.kt + 32 * quad + (lane & ~7)) >> 3;
-            const int64_t qb = qb_first + (la ? 4 : 0) + (lb ? 2 : 0) + (lc ? 1 : 0);
-            // only segments starting at or before the row's own block: seg <= qb / 8 < ld_seg
-            if (qb < qb_end && seg <= (qb >> 3)) segmax[(qb - qb_begin) * ld_seg + seg] = sm * scale;
-          }
-        } else {
-          // max over the 4 keys of the key block (lanes 4k .. 4k+3) as a transposing
-          // butterfly: after the two steps lane (a = bit 0, b = bit 1) holds the
-          // maxima of query blocks 4a + 2b and 4a + 2b + 1.
-          const bool la = (lane & 1) != 0, lb = (lane & 2) != 0;
-          float n4[4];
+          };
+          // four 32-column loads, each in flight while the previous chunk is scored
+          const uint32_t base = tmem + lane_addr + hf * 256 + 128 * cgrp;
+          float va[32], vb[32];
+          tmem_ld32(base, va);
+          tmem_ld_wait(va);
+          tmem_ld32(base + 32, vb);
+          chunk(va, 0);
+          tmem_ld_wait(vb);
+          tmem_ld32(base + 64, va);
+          chunk(vb, 1);
+          tmem_ld_wait(va);
+          tmem_ld32(base + 96, vb);
+          chunk(va, 2);
+          tmem_ld_wait(vb);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&accempty[hf]);
+          chunk(vb, 3);
+          if constexpr (MEAN) {
+            // one key block per lane: the 8 block maxima are the scores
+            // S(qb_first + b, kb), stored by the 32 lanes as 32 consecutive floats
+            float* srow = S + (qb_first - qb_begin) * ld + kb;
+            const int nb = (int)(qb_end - qb_first < 8 ? qb_end - qb_first : 8);
   #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float send = la ? m[i] : m[i + 4];
-            const float keep = la ? m[i + 4] : m[i];
-            n4[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 1));
-          }
-          float val[2];
+            for (int b = 0; b < 8; ++b) {
+              if (b < nb && kb <= qb_first + b) srow[b * ld] = m[b] * scale;
+            }
+            if (segmax != nullptr) {
+              // segment maxima over 8 key blocks = 8 lanes (bits 0..2): three
+              // transposing steps leave lane (a, b, c) of each 8-lane group with
+              // the maximum of query block qb_first + 4 a + 2 b + c
+              const bool la = (lane & 1) != 0, lb = (lane & 2) != 0, lc = (lane & 4) != 0;
+              float n4[4], n2[2];
   #pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const float send = lb ? n4[i] : n4[i + 2];
-            const float keep = lb ? n4[i + 2] : n4[i];
-            val[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
-            const int64_t qb = qb_first + (la ? 4 : 0) + (lb ? 2 : 0) + i;
-            if (qb < qb_end && kb <= qb) S[(qb - qb_begin) * ld + kb] = val[i] * scale;
-          }
-          if (segmax != nullptr) {
-            // segment maxima: max over the 8 key blocks of this warp's 32 keys
-            // (lane bits 2..4).  A transposing step on bit 2 leaves each lane one
-            // query block (4 a + 2 b + c0), then two plain steps; lanes 0..7 hold
-            // the 8 query blocks.  Key blocks after a query block were scored as
-            // 0 and scores are >= 0, so they do not raise a maximum.
-            const bool lc = (lane & 4) != 0;
-            float sm = fmaxf(lc ? val[1] : val[0], __shfl_xor_sync(0xffffffffu, lc ? val[0] : val[1], 4));
-            sm = fmaxf(sm, __shfl_xor_sync(0xffffffffu, sm, 8));
-            sm = fmaxf(sm, __shfl_xor_sync(0xffffffffu, sm, 16));
-            if (lane < 8) {
-              const int64_t seg = (KT * it.kt + 32 * quad) >> 5;
+              for (int i = 0; i < 4; ++i)
+                n4[i] = fmaxf(la ? m[i + 4] : m[i], __shfl_xor_sync(0xffffffffu, la ? m[i] : m[i + 4], 1));
+  #pragma unroll
+              for (int i = 0; i < 2; ++i)
+                n2[i] = fmaxf(lb ? n4[i + 2] : n4[i], __shfl_xor_sync(0xffffffffu, lb ? n4[i] : n4[i + 2], 2));
+              const float sm = fmaxf(lc ? n2[1] : n2[0], __shfl_xor_sync(0xffffffffu, lc ? n2[0] : n2[1], 4));
+              const int64_t seg = (KT * it.kt + 32 * quad + (lane & ~7)) >> 3;
               const int64_t qb = qb_first + (la ? 4 : 0) + (lb ? 2 : 0) + (lc ? 1 : 0);
               // only segments starting at or before the row's own block: seg <= qb / 8 < ld_seg
               if (qb < qb_end && seg <= (qb >> 3)) segmax[(qb - qb_begin) * ld_seg + seg] = sm * scale;
             }
+          } else {
+            // max over the 4 keys of the key block (lanes 4k .. 4k+3) as a transposing
+            // butterfly: after the two steps lane (a = bit 0, b = bit 1) holds the
+            // maxima of query blocks 4a + 2b and 4a + 2b + 1.
+            const bool la = (lane & 1) != 0, lb = (lane & 2) != 0;
+            float n4[4];
+    #pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float send = la ? m[i] : m[i + 4];
+              const float keep = la ? m[i + 4] : m[i];
+              n4[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 1));
+            }
+            float val[2];
+    #pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const float send = lb ? n4[i] : n4[i + 2];
+              const float keep = lb ? n4[i + 2] : n4[i];
+              val[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
+              const int64_t qb = qb_first + (la ? 4 : 0) + (lb ? 2 : 0) + i;
+              if (qb < qb_end && kb <= qb) S[(qb - qb_begin) * ld + kb] = val[i] * scale;
+            }
+            if (segmax != nullptr) {
+              // segment maxima: max over the 8 key blocks of this warp's 32 keys
+              // (lane bits 2..4).  A transposing step on bit 2 leaves each lane one
+              // query block (4 a + 2 b + c0), then two plain steps; lanes 0..7 hold
+              // the 8 query blocks.  Key blocks after a query block were scored as
+              // 0 and scores are >= 0, so they do not raise a maximum.
+              const bool lc = (lane & 4) != 0;
+              float sm = fmaxf(lc ? val[1] : val[0], __shfl_xor_sync(0xffffffffu, lc ? val[0] : val[1], 4));
+              sm = fmaxf(sm, __shfl_xor_sync(0xffffffffu, sm, 8));
+              sm = fmaxf(sm, __shfl_xor_sync(0xffffffffu, sm, 16));
+              if (lane < 8) {
+                const int64_t seg = (KT * it.kt + 32 * quad) >> 5;
+                const int64_t qb = qb_first + (la ? 4 : 0) + (lb ? 2 : 0) + (lc ? 1 : 0);
+                // only segments starting at or before the row's own block: seg <= qb / 8 < ld_seg
+                if (qb < qb_end && seg <= (qb >> 3)) segmax[(qb - qb_begin) * ld_seg + seg] = sm * scale;
+              }
+            }
           }
-        }
+        };
+        if (masked) drain(std::true_type{});
+        else drain(std::false_type{});
       } else {
         tc_fence_before();
         __syncwarp();
