@@ -698,6 +698,20 @@ def ncu_case(spec: str):
             r = qsa.prefill(d["q"], d["k"], d["v"], d["q_idx"], d["w"], d["k_idx"], budget=512, want_lse=False)
         torch.cuda.synchronize()
         assert qsa.qsa_check_device_error(r["ws"]) == 0
+    elif parts[0] == "index":
+        # stage 1 alone (qsa_index_scores, no segment maxima), four launches
+        T = int(parts[1])
+        P = Q.PrefillProblem(T=T, seed=0, n_plant=8, dist="uniform")
+        d = P.device()
+        p = qsa.params(512)
+        nqb = (T + 3) // 4
+        ld = (nqb + 3) // 4 * 4
+        S = torch.empty((nqb, ld), dtype=torch.float32, device="cuda")
+        ws = qsa.workspace(qsa.qsa_index_workspace_size(p, T))
+        for _ in range(4):
+            qsa.qsa_index_scores(p, T, d["q_idx"], d["w"], d["k_idx"], 0, nqb, S, ld, ws)
+        torch.cuda.synchronize()
+        assert qsa.qsa_check_device_error(ws) == 0
     else:
         B, L = int(parts[1]), int(parts[2])
         D = Q.DecodeProblem(B=B, L=L, steps=2, seed=0, n_plant=8)
@@ -732,7 +746,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--ncu-case", default=None,
-                    help="prefill:T or decode:B:L -- one warm-up and one call of a small case (for ncu captures)")
+                    help="prefill:T, index:T or decode:B:L -- a few calls of a small case (for ncu captures)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     if args.ncu_case:
