@@ -230,42 +230,56 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
       if (it.n_tiles == 0) continue;
       const int g = it.g;
       const int32_t* sel = a.sel + it.row * a.budget + 16 * it.tile0;
-      // Q tile; prefill rotates dims 0..63 (pairs i, i+32) on the way in,
-      // decode queries arrive rotated
-      if (items_done > 0 && !mbar_wait(q_empty, (items_done - 1) & 1, abort_flag, a.err)) { ok = false; break; }
-      for (int e = tid; e < QR * 28; e += LOADERS) {
-        const int r = e / 28, slot = e % 28;
-        const int64_t t = it.t0 + r / 12;
-        const int h = 12 * g + r % 12;
-        uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
-        const int q16 = slot < 4 ? slot : slot + 4;          // 16-byte chunk of the 512-byte row
-        if (DEC || (t < a.T && t >= a.q_tok0)) {
-          const uint4* src = reinterpret_cast<const uint4*>(a.q + ((DEC ? it.row : t - a.q_tok0) * 24 + h) * 256);
-          lo = __ldg(src + q16);
-          if (slot < 4) hi = __ldg(src + slot + 4);
-          if (!DEC && slot < 4) {
-            const float2* c8 = a.cs + (t - a.q_tok0) * 32 + 8 * slot;
-            const uint32_t* x = reinterpret_cast<const uint32_t*>(&lo);
-            const uint32_t* y = reinterpret_cast<const uint32_t*>(&hi);
-            uint4 olo, ohi;
-            uint32_t* ox = reinterpret_cast<uint32_t*>(&olo);
-            uint32_t* oy = reinterpret_cast<uint32_t*>(&ohi);
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-              const float2 c0 = c8[2 * p], c1 = c8[2 * p + 1];
-              const float x0 = bf16lo(x[p]), x1 = bf16hi(x[p]), y0 = bf16lo(y[p]), y1 = bf16hi(y[p]);
-              ox[p] = pack_bf16x2(x0 * c0.x - y0 * c0.y, x1 * c1.x - y1 * c1.y);
-              oy[p] = pack_bf16x2(y0 * c0.x + x0 * c0.y, y1 * c1.x + x1 * c1.y);
-            }
-            lo = olo;
-            hi = ohi;
-          }
+      // Q tile, loaded after the item's first K / V tile is in flight (so
+      // that tile's latency overlaps the wait for the previous item's last S
+      // and the Q load).  Dims 64..255 (chunks 8..31) go by cp.async, zero-
+      // filled past the sequence; prefill rotates dims 0..63 (pairs i, i+32,
+      // chunks slot and slot + 4) in registers, decode queries arrive rotated.
+      // The q_full arrival fires when this thread's copies have landed.
+      auto load_q = [&]() -> bool {
+        if (items_done > 0 && !mbar_wait(q_empty, (items_done - 1) & 1, abort_flag, a.err)) return false;
+        for (int e = tid; e < QR * 24; e += LOADERS) {
+          const int r = e / 24, q16 = 8 + e % 24;
+          const int64_t t = it.t0 + r / 12;
+          const int h = 12 * g + r % 12;
+          const bool present = DEC || (t < a.T && t >= a.q_tok0);
+          const uint16_t* src = present ? a.q + ((DEC ? it.row : t - a.q_tok0) * 24 + h) * 256 + 8 * q16 : a.q;
+          cp_async16(smem_u32(smem + (q16 >> 3) * CHUNK_Q + swz128(r, q16 & 7)), src, present);
         }
-        *reinterpret_cast<uint4*>(smem + (q16 >> 3) * CHUNK_Q + swz128(r, q16 & 7)) = lo;
-        if (slot < 4) *reinterpret_cast<uint4*>(smem + swz128(r, slot + 4)) = hi;
-      }
-      fence_proxy_async();
-      mbar_arrive(q_full);
+        for (int e = tid; e < QR * 4; e += LOADERS) {
+          const int r = e >> 2, slot = e & 3;
+          const int64_t t = it.t0 + r / 12;
+          const int h = 12 * g + r % 12;
+          uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
+          if (DEC || (t < a.T && t >= a.q_tok0)) {
+            const uint4* src = reinterpret_cast<const uint4*>(a.q + ((DEC ? it.row : t - a.q_tok0) * 24 + h) * 256);
+            lo = __ldg(src + slot);
+            hi = __ldg(src + slot + 4);
+            if (!DEC) {
+              const float2* c8 = a.cs + (t - a.q_tok0) * 32 + 8 * slot;
+              const uint32_t* x = reinterpret_cast<const uint32_t*>(&lo);
+              const uint32_t* y = reinterpret_cast<const uint32_t*>(&hi);
+              uint4 olo, ohi;
+              uint32_t* ox = reinterpret_cast<uint32_t*>(&olo);
+              uint32_t* oy = reinterpret_cast<uint32_t*>(&ohi);
+#pragma unroll
+              for (int p = 0; p < 4; ++p) {
+                const float2 c0 = c8[2 * p], c1 = c8[2 * p + 1];
+                const float x0 = bf16lo(x[p]), x1 = bf16hi(x[p]), y0 = bf16lo(y[p]), y1 = bf16hi(y[p]);
+                ox[p] = pack_bf16x2(x0 * c0.x - y0 * c0.y, x1 * c1.x - y1 * c1.y);
+                oy[p] = pack_bf16x2(y0 * c0.x + x0 * c0.y, y1 * c1.x + x1 * c1.y);
+              }
+              lo = olo;
+              hi = ohi;
+            }
+          }
+          *reinterpret_cast<uint4*>(smem + swz128(r, slot)) = lo;
+          *reinterpret_cast<uint4*>(smem + swz128(r, slot + 4)) = hi;
+        }
+        fence_proxy_async();
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(q_full)) : "memory");
+        return true;
+      };
       // K / V tiles
       const int n_tiles = it.n_tiles;
       const int nsel = it.cnt - 16 * it.tile0;     // selected blocks from this item's first tile on
@@ -302,6 +316,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
         asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&kv_full[stage]))
                      : "memory");
         if (++stage == NSTAGE) { stage = 0; ephase ^= 1; }
+        if (i == 0 && !load_q()) { ok = false; break; }
       }
       ++items_done;
     }
