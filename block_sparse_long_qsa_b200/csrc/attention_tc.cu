@@ -59,6 +59,12 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
                : "memory");
 }
+// 32-byte global store (the address must be 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&x)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(x[0]), "r"(x[1]), "r"(x[2]),
+               "r"(x[3]), "r"(x[4]), "r"(x[5]), "r"(x[6]), "r"(x[7])
+               : "memory");
+}
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 // Two floats to packed bf16 (round to nearest even): lo in bits 0..15.
 __device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
@@ -284,21 +290,27 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
       const int n_tiles = it.n_tiles;
       const int nsel = it.cnt - 16 * it.tile0;     // selected blocks from this item's first tile on
       const int64_t t_last = it.t_last;
-      for (int i = 0; i < n_tiles; ++i) {
-        if (!mbar_wait(&kv_empty[stage], ephase, abort_flag, a.err)) { ok = false; break; }
-        const uint32_t base = smem_u32(smem + OFF_STAGE + stage * STAGE_BYTES);
-        // Thread (warp w, lane c32) copies 16-byte chunk c32 of token w % 4 of
-        // each of its KPT blocks of the tile (all 16 with 4 loader warps, half
-        // with 8), for K and for V: key slot n = 4k + w % 4.  The block indices
-        // are loaded up front (independent, L1-broadcast).
-        constexpr int KPT = 64 / LWARPS;
-        const int w4 = (tid >> 5) & 3, c32 = tid & 31, k0 = KPT * (tid >> 7);
-        int32_t kbv[KPT];
+      // Thread (warp w, lane c32) copies 16-byte chunk c32 of token w % 4 of
+      // each of its KPT blocks of a tile (all 16 with 4 loader warps, half
+      // with 8), for K and for V: key slot n = 4k + w % 4.  The block indices
+      // of tile i + 1 are loaded while tile i waits for its stage, so the
+      // index loads' latency stays off the issue path.
+      constexpr int KPT = 64 / LWARPS;
+      const int w4 = (tid >> 5) & 3, c32 = tid & 31, k0 = KPT * (tid >> 7);
+      int32_t kbv[KPT], kbn[KPT], kbm[KPT];
+      auto load_idx = [&](int ti, int32_t (&dst)[KPT]) {
 #pragma unroll
         for (int kk = 0; kk < KPT; ++kk) {
-          const int k = k0 + kk;
-          kbv[kk] = 16 * i + k < nsel ? __ldg(sel + 16 * i + k) : -1;
+          const int k = 16 * ti + k0 + kk;
+          dst[kk] = k < nsel ? __ldg(sel + k) : -1;
         }
+      };
+      load_idx(0, kbv);
+      if (n_tiles > 1) load_idx(1, kbn);
+      for (int i = 0; i < n_tiles; ++i) {
+        if (i + 2 < n_tiles) load_idx(i + 2, kbm);
+        if (!mbar_wait(&kv_empty[stage], ephase, abort_flag, a.err)) { ok = false; break; }
+        const uint32_t base = smem_u32(smem + OFF_STAGE + stage * STAGE_BYTES);
         const uint32_t dst0 = base + (c32 >> 3) * CHUNK_KV;
 #pragma unroll
         for (int kk = 0; kk < KPT; ++kk) {
@@ -316,6 +328,8 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
         asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&kv_full[stage]))
                      : "memory");
         if (++stage == NSTAGE) { stage = 0; ephase ^= 1; }
+#pragma unroll
+        for (int kk = 0; kk < KPT; ++kk) { kbv[kk] = kbn[kk]; kbn[kk] = kbm[kk]; }
         if (i == 0 && !load_q()) { ok = false; break; }
       }
       ++items_done;
@@ -491,17 +505,38 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
       const int64_t orow_idx = (DEC ? it.row : t - a.q_tok0) * 24 + 12 * g + hh;   // [token or sequence][head]
       uint16_t* orow = a.out + orow_idx * 256;
       const bool partial = DEC && a.n_split > 1;
+      const bool out32 = (reinterpret_cast<uintptr_t>(a.out) & 31) == 0;   // rows are 512 B apart
+      const bool part32 = (reinterpret_cast<uintptr_t>(a.part_o) & 31) == 0;
       const int64_t prow = ((it.row * 2 + g) * (int64_t)a.n_split + it.split) * 12 + hh;
 #pragma unroll 1
       for (int c = 0; c < 8; ++c) {
         float o[32];
         tmem_ld32(tmem + lane_off + TM_O + 32 * c, o);
         tmem_ld_wait();
-        if (write && partial) {
+        // each row is written by one thread: 32-byte stores where the output
+        // allows (full sectors, half the store instructions of 16-byte ones)
+        if (write && partial && part32) {
+          float* dst = a.part_o + prow * 256 + 32 * c;   // rows are 1 KB apart
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = __float_as_uint(o[8 * q + e] * inv);
+            st_global_v8(dst + 8 * q, x);
+          }
+        } else if (write && partial) {
           float4* dst = reinterpret_cast<float4*>(a.part_o + prow * 256 + 32 * c);
 #pragma unroll
           for (int q = 0; q < 8; ++q)
             dst[q] = make_float4(o[4 * q] * inv, o[4 * q + 1] * inv, o[4 * q + 2] * inv, o[4 * q + 3] * inv);
+        } else if (write && out32) {
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            uint32_t x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = cvt_bf16x2(o[16 * q + 2 * e] * inv, o[16 * q + 2 * e + 1] * inv);
+            st_global_v8(orow + 32 * c + 16 * q, x);
+          }
         } else if (write) {
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
