@@ -27,11 +27,11 @@ EXPORTED = ["qsa_default_params", "qsa_status_string", "qsa_last_error", "qsa_in
             "qsa_decode_workspace_size", "qsa_check_device_error", "qsa_trace_begin", "qsa_trace_end",
             "qsa_decode_noalloc", "qsa_prefill_cached", "qsa_prefill_cached_workspace_size",
             "qsa_index_workspace_size", "qsa_decode_mean_pool", "qsa_mean_pool_keys",
-            "qsa_decode_reuse"]
+            "qsa_decode_reuse", "qsa_verify", "qsa_verify_workspace_size"]
 
 KERNEL_NAMES = {1: "rope_table", 2: "rope_k", 3: "indexer", 4: "select", 5: "attention", 6: "decode_append",
                 7: "decode_indexer", 8: "decode_attention", 9: "decode_combine",
-                10: "mean_pool_keys"}
+                10: "mean_pool_keys", 11: "verify_expand"}
 
 
 class QSAError(RuntimeError):
@@ -86,6 +86,8 @@ def load(path: str = LIB_PATH):
     L.qsa_decode_workspace_size.argtypes = [P, i32, i64, psz]
     L.qsa_decode_mean_pool.argtypes = [P, i32, i64, ctypes.POINTER(ctypes.c_int64)] + [vp] * 15 + [vp, sz, vp]
     L.qsa_mean_pool_keys.argtypes = [P, i64, vp, vp, vp]
+    L.qsa_verify.argtypes = [P, i32, i32, i64, ctypes.POINTER(ctypes.c_int64)] + [vp] * 14 + [vp, sz, vp]
+    L.qsa_verify_workspace_size.argtypes = [P, i32, i32, i64, psz]
     L.qsa_decode_reuse.argtypes = [P, i32, i64, ctypes.POINTER(ctypes.c_int64)] + [vp] * 16 + [vp, sz, vp]
     L.qsa_decode_noalloc.argtypes = [P, i32, i64, ctypes.POINTER(ctypes.c_int64), vp, vp, vp, vp, vp, vp, vp, vp,
                                      vp, vp, vp, vp, vp, vp, vp]
@@ -224,6 +226,24 @@ def qsa_decode_reuse(p: qsa_params, B: int, max_len: int, cache_len, k_cache, v_
                                    _ptr(v_new), _ptr(q_idx_new), _ptr(k_idx_new), _ptr(w_new), _ptr(sel_in),
                                    _ptr(cnt_in), _ptr(out), _ptr(lse_out), _ptr(ws), ws.numel() * ws.element_size(),
                                    _stream(stream)), "qsa_decode_reuse")
+
+
+def qsa_verify_workspace_size(p: qsa_params, B: int, m: int, max_len: int) -> int:
+    n = ctypes.c_size_t()
+    _check(load().qsa_verify_workspace_size(ctypes.byref(p), B, m, max_len, ctypes.byref(n)),
+           "qsa_verify_workspace_size")
+    return n.value
+
+
+def qsa_verify(p: qsa_params, B: int, m: int, max_len: int, cache_len, k_cache, v_cache, kidx_cache, qidx_prev,
+               w_prev, q_new, k_new, v_new, q_idx_new, k_idx_new, w_new, out, sel_out=None, lse_out=None, ws=None,
+               stream=None):
+    """Verify m new tokens per sequence (``cache_len``: host sequence of B ints)."""
+    lens = (ctypes.c_int64 * B)(*[int(x) for x in cache_len])
+    _check(load().qsa_verify(ctypes.byref(p), B, m, max_len, lens, _ptr(k_cache), _ptr(v_cache), _ptr(kidx_cache),
+                             _ptr(qidx_prev), _ptr(w_prev), _ptr(q_new), _ptr(k_new), _ptr(v_new), _ptr(q_idx_new),
+                             _ptr(k_idx_new), _ptr(w_new), _ptr(out), _ptr(sel_out), _ptr(lse_out), _ptr(ws),
+                             ws.numel() * ws.element_size(), _stream(stream)), "qsa_verify")
 
 
 def qsa_mean_pool_keys(p: qsa_params, T: int, k_idx, kbar, stream=None):

@@ -830,3 +830,133 @@ qsa_status qsa_trace_end(int32_t* kernel_ids, float* ms, int32_t capacity, int32
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ verify
+namespace {
+constexpr int VERIFY_MAX_M = 16;
+struct VerifyLayout {
+  size_t Lb, Ls, rqb, S, selb, cntb, selt, cntt, q_rot, part_o, part_lse, total;
+  int64_t ld;
+  int nqv, max_split;
+};
+// Query blocks that m consecutive tokens can touch: (m + 2) / 4 + 1.
+VerifyLayout verify_layout(int B, int m, int64_t max_len, int budget) {
+  VerifyLayout L;
+  const int64_t rows = (int64_t)B * m;
+  L.nqv = (m + 2) / 4 + 1;
+  L.ld = round4(max_len / 4 + 1);
+  // split-KV ranges are worth having only while the token rows leave SMs
+  // idle: at most enough to give 296 (two per SM) items
+  int ms = (int)((296 + 2 * rows - 1) / (2 * rows));
+  L.max_split = ms < 1 ? 1 : (ms > DECODE_MAX_SPLIT ? DECODE_MAX_SPLIT : ms);
+  const int64_t nrow = (int64_t)B * L.nqv;
+  size_t off = HEADER_BYTES;
+  L.Lb = off; off = align_up(off + (size_t)B * 8);
+  L.Ls = off; off = align_up(off + (size_t)rows * 8);
+  L.rqb = off; off = align_up(off + (size_t)nrow * 8);
+  L.S = off; off = align_up(off + (size_t)nrow * L.ld * 4);
+  L.selb = off; off = align_up(off + (size_t)nrow * budget * 4);
+  L.cntb = off; off = align_up(off + (size_t)nrow * 4);
+  L.selt = off; off = align_up(off + (size_t)rows * budget * 4);
+  L.cntt = off; off = align_up(off + (size_t)rows * 4);
+  L.q_rot = off; off = align_up(off + (size_t)rows * 24 * 256 * 2);
+  L.part_o = off; off = align_up(off + (L.max_split > 1 ? (size_t)rows * 2 * L.max_split * 12 * 256 * 4 : 0));
+  L.part_lse = off; off = align_up(off + (L.max_split > 1 ? (size_t)rows * 2 * L.max_split * 12 * 4 : 0));
+  L.total = off;
+  return L;
+}
+}  // namespace
+
+qsa_status qsa_verify_workspace_size(const qsa_params* p, int32_t B, int32_t m, int64_t max_len, size_t* bytes) {
+  qsa_status st = check_params(p);
+  if (st != QSA_OK) return st;
+  if (B <= 0 || m <= 0 || max_len <= 0 || !bytes) return QSA_ERR_INVALID_ARG;
+  if (B > 4096 || m > VERIFY_MAX_M || max_len > ((int64_t)1 << 24)) return QSA_ERR_UNSUPPORTED;
+  *bytes = verify_layout(B, m, max_len, p->budget_blocks).total;
+  return QSA_OK;
+}
+
+qsa_status qsa_verify(const qsa_params* p, int32_t B, int32_t m, int64_t max_len, const int64_t* cache_len,
+                      uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, const uint16_t* qidx_prev,
+                      const uint16_t* w_prev, const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
+                      const uint16_t* q_idx_new, const uint16_t* k_idx_new, const uint16_t* w_new, uint16_t* out,
+                      int32_t* sel_out, float* lse_out, void* ws, size_t ws_bytes, void* stream) {
+  qsa_status st = check_params(p);
+  if (st != QSA_OK) return st;
+  if (mean_pool(p)) return QSA_ERR_UNSUPPORTED;   // token-pair scores only
+  if (B <= 0 || m <= 0 || max_len <= 0 || !cache_len) return QSA_ERR_INVALID_ARG;
+  if (B > 4096 || m > VERIFY_MAX_M || max_len > ((int64_t)1 << 24)) return QSA_ERR_UNSUPPORTED;
+  const void* ptrs[] = {k_cache, v_cache, kidx_cache, q_new, k_new, v_new, q_idx_new, k_idx_new, w_new, out, ws};
+  for (const void* ptr : ptrs) {
+    if (!ptr) return QSA_ERR_INVALID_ARG;
+    if (!aligned16(ptr)) return QSA_ERR_MISALIGNED;
+  }
+  if ((qidx_prev && !aligned16(qidx_prev)) || (w_prev && !aligned16(w_prev)) || (lse_out && !aligned16(lse_out)) ||
+      (sel_out && !aligned16(sel_out)))
+    return QSA_ERR_MISALIGNED;
+  int64_t max_L = 0;
+  bool any_partial = false;
+  for (int b = 0; b < B; ++b) {
+    if (cache_len[b] < 0 || cache_len[b] + m > max_len) return QSA_ERR_INVALID_ARG;
+    if (cache_len[b] > max_L) max_L = cache_len[b];
+    any_partial |= (cache_len[b] & 3) != 0;
+  }
+  // block-mates before the new tokens come from qidx_prev / w_prev
+  if (any_partial && (!qidx_prev || !w_prev)) return QSA_ERR_INVALID_ARG;
+  const int budget = p->budget_blocks;
+  VerifyLayout L = verify_layout(B, m, max_len, budget);
+  if (ws_bytes < L.total) return QSA_ERR_WORKSPACE_TOO_SMALL;
+  DevInfo di;
+  if ((st = device_info(&di)) != QSA_OK) return st;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint32_t* err = reinterpret_cast<uint32_t*>(base);
+  int64_t* Lb = reinterpret_cast<int64_t*>(base + L.Lb);
+  int64_t* Ls = reinterpret_cast<int64_t*>(base + L.Ls);
+  int64_t* rqb = reinterpret_cast<int64_t*>(base + L.rqb);
+  float* S = reinterpret_cast<float*>(base + L.S);
+  int32_t* selb = reinterpret_cast<int32_t*>(base + L.selb);
+  int32_t* cntb = reinterpret_cast<int32_t*>(base + L.cntb);
+  int32_t* selt = sel_out ? sel_out : reinterpret_cast<int32_t*>(base + L.selt);
+  int32_t* cntt = reinterpret_cast<int32_t*>(base + L.cntt);
+  uint16_t* q_rot = reinterpret_cast<uint16_t*>(base + L.q_rot);
+  float* part_o = reinterpret_cast<float*>(base + L.part_o);
+  float* part_lse = reinterpret_cast<float*>(base + L.part_lse);
+
+  if (cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaMemsetAsync");
+  double f[32];
+  inv_freq(p, f);
+  if ((st = from_cuda(traced(QSA_KERNEL_DECODE_APPEND, s, [&] {
+         return qsa::launch_verify_append(B, m, L.nqv, max_len, cache_len, Lb, Ls, rqb, f, rope_attn_factor(p),
+                                          k_cache, v_cache, kidx_cache, q_new, k_new, v_new, k_idx_new, q_rot, s);
+       }))) != QSA_OK)
+    return st;
+  const float scale = 1.0f / std::sqrt(128.0f);
+  if ((st = from_cuda(traced(QSA_KERNEL_DECODE_INDEXER, s, [&] {
+         return qsa::launch_verify_indexer(B, L.nqv, m, max_len, max_L, Lb, rqb, kidx_cache, qidx_prev, w_prev,
+                                           q_idx_new, w_new, S, L.ld, scale, s);
+       }))) != QSA_OK)
+    return st;
+  if ((st = from_cuda(traced(QSA_KERNEL_SELECT, s, [&] {
+         return qsa::launch_select(S, L.ld, nullptr, 0, 0, (int64_t)B * L.nqv, rqb, budget, selb, cntb, err, s);
+       }))) != QSA_OK)
+    return st;
+  if ((st = from_cuda(traced(QSA_KERNEL_VERIFY_EXPAND, s, [&] {
+         return qsa::launch_verify_expand(B, m, L.nqv, budget, Ls, selb, cntb, selt, cntt, s);
+       }))) != QSA_OK)
+    return st;
+  const int rows = B * m;
+  int n_split = decode_splits(rows, max_L + m - 1, budget, di.num_sms);
+  if (n_split > L.max_split) n_split = L.max_split;
+  const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
+  if ((st = from_cuda(traced(QSA_KERNEL_DECODE_ATTENTION, s, [&] {
+         return qsa::launch_decode_attn_tc(rows, max_len, Ls, q_rot, k_cache, v_cache, selt, cntt, budget, scale_log2,
+                                           n_split, part_o, part_lse, out, lse_out, err, di.num_sms, s, m);
+       }))) != QSA_OK)
+    return st;
+  if (n_split == 1) return QSA_OK;
+  return from_cuda(traced(QSA_KERNEL_DECODE_COMBINE, s, [&] {
+    return qsa::launch_decode_combine(rows, part_o, part_lse, cntt, n_split, out, lse_out, s);
+  }));
+}

@@ -128,7 +128,8 @@ struct TcArgs {
   uint32_t* err;
   // decode: q = rotated new-token queries [B][24][256], k_rot / v = caches
   // [B][max_len][2][256], out / lse [B][24][...], one query token per sequence
-  const int64_t* Ls;        // [B] position of the new token
+  const int64_t* Ls;        // [rows] position of the row's query token
+  int64_t rows_per_seq;     // decode rows per sequence (verify: the m new tokens), else 1
   int64_t max_len;
   // split-KV decode: each (sequence, KV head) is cut into n_split ranges of
   // whole tiles; with n_split > 1 every range writes its normalised O (fp32)
@@ -171,8 +172,8 @@ struct Item {
       qb = L >> 2;
       t0 = L;
       t_last = L;
-      kb = a.k_rot + row * a.max_len * 512;
-      vb = a.v + row * a.max_len * 512;
+      kb = a.k_rot + (row / a.rows_per_seq) * a.max_len * 512;
+      vb = a.v + (row / a.rows_per_seq) * a.max_len * 512;
     } else {
       qb = a.qb_begin + row;
       t0 = 4 * qb;
@@ -639,13 +640,13 @@ cudaError_t launch_decode_attn_tc(int B, int64_t max_len, const int64_t* L_dev, 
                                   const uint16_t* k_cache, const uint16_t* v_cache, const int32_t* sel,
                                   const int32_t* cnt, int budget, float scale_log2, int n_split, float* part_o,
                                   float* part_lse, uint16_t* out, float* lse, uint32_t* err, int num_sms,
-                                  cudaStream_t stream) {
+                                  cudaStream_t stream, int rows_per_seq) {
   if (B <= 0) return cudaSuccess;
-  if (n_split < 1) return cudaErrorInvalidValue;
+  if (n_split < 1 || rows_per_seq < 1) return cudaErrorInvalidValue;
   TcArgs a{};
   a.T = INT64_MAX; a.q = q_rot; a.k_rot = k_cache; a.v = v_cache; a.sel = sel; a.cnt = cnt; a.budget = budget;
   a.qb_begin = 0; a.n_qb = B; a.scale_log2 = scale_log2; a.out = out; a.lse = lse; a.err = err;
-  a.Ls = L_dev; a.max_len = max_len;
+  a.Ls = L_dev; a.max_len = max_len; a.rows_per_seq = rows_per_seq;
   a.n_split = n_split; a.part_o = part_o; a.part_lse = part_lse;
   return launch_tc<true>(a, 2 * (int64_t)B * n_split, num_sms, stream);
 }

@@ -47,22 +47,32 @@ __device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
 // and S(qb, kb) is the max over the present block-mates of their score
 // against kbar[kb] (no per-key causal test: kb <= qb); otherwise the rows are
 // keys and S is the max over causal token pairs.
-template <bool MEAN>
+// VER (verify, token-pair scores only): S row r scores query block
+// row_qb[r] of sequence r / nqv, whose m new tokens sit at L .. L + m - 1
+// (L = Ls[b], the length before them); the block's tokens before L take their
+// q_idx / w from the ring (slot = position % 4), the new ones from
+// qidx_new / w_new [B][m][...].  row_qb[r] < 0: nothing to score.
+template <bool MEAN, bool VER>
 __global__ void __launch_bounds__(THREADS)
 decode_indexer_kernel(int64_t max_len, const int64_t* __restrict__ Ls, const uint16_t* __restrict__ kidx_cache,
                       const uint16_t* __restrict__ kbar_cache, int64_t kbar_len,
                       const uint16_t* __restrict__ qidx_ring, const uint16_t* __restrict__ w_ring,
-                      float* __restrict__ S, int64_t ld, float scale) {
-  const int64_t b = blockIdx.y;
+                      float* __restrict__ S, int64_t ld, float scale, const int64_t* __restrict__ row_qb, int nqv,
+                      int m, const uint16_t* __restrict__ qidx_new, const uint16_t* __restrict__ w_new) {
+  const int64_t row = blockIdx.y;
+  const int64_t b = VER ? row / nqv : row;
   const int64_t L = Ls[b];
-  const int64_t qb = L >> 2;
-  const int64_t last_row = MEAN ? qb : L;              // last row with data
+  const int64_t qb = VER ? row_qb[row] : L >> 2;
+  if (VER && qb < 0) return;
+  const int64_t pos_end = VER ? L + m - 1 : L;        // last present token
+  const int64_t last_key = 4 * qb + 3 < pos_end ? 4 * qb + 3 : pos_end;
+  const int64_t last_row = MEAN ? qb : last_key;       // last row with data
   const int64_t j_begin = (int64_t)blockIdx.x * KEYS_PER_CTA;
   if (j_begin > last_row) return;
   int64_t j_end = j_begin + KEYS_PER_CTA;
   const int64_t rows_end = MEAN ? qb + 1 : 4 * qb + 4;
   if (j_end > rows_end) j_end = rows_end;
-  const int present = (int)(L - 4 * qb) + 1;        // block-mates 4qb .. L (ring slots 0 .. present-1)
+  const int present = (int)(last_key - 4 * qb) + 1;   // block-mates 4qb .. last_key
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g8 = lane >> 2, q4 = lane & 3;
@@ -74,7 +84,10 @@ decode_indexer_kernel(int64_t max_len, const int64_t* __restrict__ Ls, const uin
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
       const int head = 2 * nt + (g8 & 1);
-      const uint4* src = reinterpret_cast<const uint4*>(qidx_ring + ((b * 4 + tok) * 4 + head) * 128);
+      const int64_t pos = 4 * qb + tok;
+      const uint4* src = reinterpret_cast<const uint4*>(
+          VER && pos >= L ? qidx_new + ((b * m + (pos - L)) * 4 + head) * 128
+                          : qidx_ring + ((b * 4 + tok) * 4 + head) * 128);
 #pragma unroll
       for (int d = 0; d < 4; ++d) qf[nt][d] = tok < present ? src[4 * d + q4] : make_uint4(0, 0, 0, 0);
     }
@@ -84,12 +97,15 @@ decode_indexer_kernel(int64_t max_len, const int64_t* __restrict__ Ls, const uin
   {
     const bool ok = q4 < present;
 #pragma unroll
-    for (int h = 0; h < 4; ++h) w[h] = ok ? bf16_bits_to_f32(w_ring[(b * 4 + q4) * 4 + h]) : 0.f;
+    const int64_t pos = 4 * qb + q4;
+    for (int h = 0; h < 4; ++h)
+      w[h] = ok ? bf16_bits_to_f32(VER && pos >= L ? w_new[(b * m + (pos - L)) * 4 + h] : w_ring[(b * 4 + q4) * 4 + h])
+                : 0.f;
   }
   const int64_t t_tok = 4 * qb + q4;                 // this thread's query token
   const bool tok_ok = q4 < present;
   const uint16_t* kb_base = MEAN ? kbar_cache + b * kbar_len * 128 : kidx_cache + b * max_len * 128;
-  float* Srow = S + b * ld;
+  float* Srow = S + row * ld;
 
   // the next tile's 16 keys are loaded while the current tile is scored
   constexpr int64_t STEP = 16 * (THREADS / 32);
@@ -171,11 +187,45 @@ cudaError_t launch_decode_indexer(int B, int64_t max_len, int64_t max_L, const i
   const int64_t nx = (rows + KEYS_PER_CTA - 1) / KEYS_PER_CTA;
   dim3 grid((unsigned)nx, (unsigned)B);
   if (kbar_cache)
-    decode_indexer_kernel<true><<<grid, THREADS, 0, s>>>(max_len, L_dev, kidx_cache, kbar_cache, kbar_len, qidx_ring,
-                                                         w_ring, S, ld, scale);
+    decode_indexer_kernel<true, false><<<grid, THREADS, 0, s>>>(max_len, L_dev, kidx_cache, kbar_cache, kbar_len,
+                                                                qidx_ring, w_ring, S, ld, scale, nullptr, 1, 1,
+                                                                nullptr, nullptr);
   else
-    decode_indexer_kernel<false><<<grid, THREADS, 0, s>>>(max_len, L_dev, kidx_cache, nullptr, 0, qidx_ring, w_ring,
-                                                          S, ld, scale);
+    decode_indexer_kernel<false, false><<<grid, THREADS, 0, s>>>(max_len, L_dev, kidx_cache, nullptr, 0, qidx_ring,
+                                                                 w_ring, S, ld, scale, nullptr, 1, 1, nullptr, nullptr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_verify_indexer(int B, int nqv, int m, int64_t max_len, int64_t max_L, const int64_t* Lb_dev,
+                                  const int64_t* row_qb, const uint16_t* kidx_cache, const uint16_t* qidx_ring,
+                                  const uint16_t* w_ring, const uint16_t* qidx_new, const uint16_t* w_new, float* S,
+                                  int64_t ld, float scale, cudaStream_t s) {
+  if (B <= 0) return cudaSuccess;
+  const int64_t rows = max_L + m + 3;                 // keys up to the last new token's block end
+  const int64_t nx = (rows + KEYS_PER_CTA - 1) / KEYS_PER_CTA;
+  dim3 grid((unsigned)nx, (unsigned)(B * nqv));
+  decode_indexer_kernel<false, true><<<grid, THREADS, 0, s>>>(max_len, Lb_dev, kidx_cache, nullptr, 0, qidx_ring,
+                                                              w_ring, S, ld, scale, row_qb, nqv, m, qidx_new, w_new);
+  return cudaGetLastError();
+}
+
+// Token row t = (b, i) of a verify takes the selection of its query block:
+// row b * nqv + (pos / 4 - L_b / 4) of sel_blk / cnt_blk, pos = Ls_tok[t].
+__global__ void verify_expand_kernel(int m, int nqv, int budget, const int64_t* __restrict__ Ls_tok,
+                                     const int32_t* __restrict__ sel_blk, const int32_t* __restrict__ cnt_blk,
+                                     int32_t* __restrict__ sel_tok, int32_t* __restrict__ cnt_tok) {
+  const int64_t t = blockIdx.x;
+  const int64_t b = t / m;
+  const int64_t j = (Ls_tok[t] >> 2) - (Ls_tok[b * m] >> 2);
+  const int64_t r = b * nqv + j;
+  for (int e = threadIdx.x; e < budget; e += blockDim.x) sel_tok[t * budget + e] = sel_blk[r * budget + e];
+  if (threadIdx.x == 0) cnt_tok[t] = cnt_blk[r];
+}
+
+cudaError_t launch_verify_expand(int B, int m, int nqv, int budget, const int64_t* Ls_tok, const int32_t* sel_blk,
+                                 const int32_t* cnt_blk, int32_t* sel_tok, int32_t* cnt_tok, cudaStream_t s) {
+  if (B <= 0) return cudaSuccess;
+  verify_expand_kernel<<<B * m, 128, 0, s>>>(m, nqv, budget, Ls_tok, sel_blk, cnt_blk, sel_tok, cnt_tok);
   return cudaGetLastError();
 }
 

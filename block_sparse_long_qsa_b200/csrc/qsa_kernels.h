@@ -75,7 +75,22 @@ cudaError_t launch_decode_attn_tc(int B, int64_t max_len, const int64_t* L_dev, 
                                   const uint16_t* k_cache, const uint16_t* v_cache, const int32_t* sel,
                                   const int32_t* cnt, int budget, float scale_log2, int n_split, float* part_o,
                                   float* part_lse, uint16_t* out, float* lse, uint32_t* err, int num_sms,
-                                  cudaStream_t stream);
+                                  cudaStream_t stream, int rows_per_seq = 1);
+// Verify (m new tokens per sequence at L_b .. L_b + m - 1, nqv query-block
+// rows per sequence): append the tokens, score the query blocks they touch
+// (block tokens before L_b from the ring), and give each token row its
+// block's selection.
+cudaError_t launch_verify_append(int B, int m, int nqv, int64_t max_len, const int64_t* L_host, int64_t* Lb_dev,
+                                 int64_t* Ls_tok, int64_t* row_qb, const double* inv_freq_host, double attn_factor,
+                                 uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, const uint16_t* q_new,
+                                 const uint16_t* k_new, const uint16_t* v_new, const uint16_t* k_idx_new,
+                                 uint16_t* q_rot, cudaStream_t s);
+cudaError_t launch_verify_indexer(int B, int nqv, int m, int64_t max_len, int64_t max_L, const int64_t* Lb_dev,
+                                  const int64_t* row_qb, const uint16_t* kidx_cache, const uint16_t* qidx_ring,
+                                  const uint16_t* w_ring, const uint16_t* qidx_new, const uint16_t* w_new, float* S,
+                                  int64_t ld, float scale, cudaStream_t s);
+cudaError_t launch_verify_expand(int B, int m, int nqv, int budget, const int64_t* Ls_tok, const int32_t* sel_blk,
+                                 const int32_t* cnt_blk, int32_t* sel_tok, int32_t* cnt_tok, cudaStream_t s);
 cudaError_t launch_decode_combine(int B, const float* part_o, const float* part_lse, const int32_t* cnt, int n_split,
                                   uint16_t* out, float* lse, cudaStream_t stream);
 

@@ -178,6 +178,60 @@ __global__ void decode_append_kernel(int64_t max_len, LenChunk lens, int64_t* __
   }
 }
 
+// Verify append: block (sequence b, new token i) of a chunk of sequences puts
+// token i at position pos = L_b + i: its key rotated at pos into k_cache, its
+// value and indexer key into the caches, its queries rotated at pos into
+// q_rot[b][i] and pos into Ls_tok[b][i]; block i = 0 also records L_b and the
+// query blocks qb = L_b/4 + j (j < nqv; -1 past the last new token) that the
+// verify scores.  The q_idx / w ring is left as it is (read-only here).
+__global__ void verify_append_kernel(int64_t max_len, int m, int nqv, LenChunk lens, int64_t* __restrict__ Lb_dev,
+                                     int64_t* __restrict__ Ls_tok, int64_t* __restrict__ row_qb, InvFreq inv,
+                                     uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                                     uint4* __restrict__ kidx_cache, const uint4* __restrict__ q_new,
+                                     const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+                                     const uint4* __restrict__ k_idx_new, uint4* __restrict__ q_rot) {
+  __shared__ float2 cs[32];
+  const int bl = blockIdx.x / m, i = blockIdx.x % m;
+  const int64_t b = lens.b0 + bl;
+  const int64_t L = lens.L[bl];
+  const int64_t pos = L + i;
+  const int64_t tok = b * m + i;                       // token row [b][i]
+  if (threadIdx.x == 0) {
+    Ls_tok[tok] = pos;
+    if (i == 0) {
+      Lb_dev[b] = L;
+      for (int j = 0; j < nqv; ++j) {
+        const int64_t qb = (L >> 2) + j;
+        row_qb[b * nqv + j] = 4 * qb <= L + m - 1 ? qb : -1;
+      }
+    }
+  }
+  if (threadIdx.x < 32) {
+    double sa, ca;
+    sincos((double)pos * inv.f[threadIdx.x], &sa, &ca);
+    cs[threadIdx.x] = make_float2((float)(inv.scale * ca), (float)(inv.scale * sa));
+  }
+  __syncthreads();
+  // rotated rows: 2 kv heads (k) + 24 q heads, 4 rotate slots each; copies of the rest
+  for (int e = threadIdx.x; e < 26 * 28; e += blockDim.x) {
+    const int row = e / 28, slot = e % 28;
+    const uint4* src = row < 2 ? k_new + (tok * 2 + row) * 32 : q_new + (tok * 24 + row - 2) * 32;
+    uint4* dst = row < 2 ? k_cache + ((b * max_len + pos) * 2 + row) * 32 : q_rot + (tok * 24 + row - 2) * 32;
+    if (slot < 4) {
+      uint4 olo, ohi;
+      rotate8(src[slot], src[slot + 4], cs + 8 * slot, olo, ohi);
+      dst[slot] = olo;
+      dst[slot + 4] = ohi;
+    } else {
+      dst[slot + 4] = src[slot + 4];
+    }
+  }
+  for (int e = threadIdx.x; e < 64; e += blockDim.x)            // v: 2 x 512 B
+    v_cache[(b * max_len + pos) * 64 + e] = v_new[tok * 64 + e];
+  for (int e = threadIdx.x; e < 16; e += blockDim.x)            // k_idx: 256 B
+    kidx_cache[(b * max_len + pos) * 16 + e] = k_idx_new[tok * 16 + e];
+}
+
 InvFreq to_struct(const double* f, double scale) {
   InvFreq s;
   for (int i = 0; i < 32; ++i) s.f[i] = f[i];
@@ -228,6 +282,28 @@ cudaError_t launch_decode_append(int B, int64_t max_len, const int64_t* L_host, 
         reinterpret_cast<const uint4*>(v_new), reinterpret_cast<const uint4*>(q_idx_new),
         reinterpret_cast<const uint4*>(k_idx_new), w_new, reinterpret_cast<uint4*>(q_rot), kbar_cache, kbar_len,
         sel_in, cnt_in, budget, sel_r, sel_r_ld, cnt_r, err);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_verify_append(int B, int m, int nqv, int64_t max_len, const int64_t* L_host, int64_t* Lb_dev,
+                                 int64_t* Ls_tok, int64_t* row_qb, const double* inv_freq_host, double attn_factor,
+                                 uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, const uint16_t* q_new,
+                                 const uint16_t* k_new, const uint16_t* v_new, const uint16_t* k_idx_new,
+                                 uint16_t* q_rot, cudaStream_t s) {
+  const InvFreq inv = to_struct(inv_freq_host, attn_factor);
+  for (int b0 = 0; b0 < B; b0 += LEN_CHUNK) {
+    const int n = B - b0 < LEN_CHUNK ? B - b0 : LEN_CHUNK;
+    LenChunk lens;
+    lens.b0 = b0;
+    for (int i = 0; i < n; ++i) lens.L[i] = L_host[b0 + i];
+    verify_append_kernel<<<n * m, 256, 0, s>>>(
+        max_len, m, nqv, lens, Lb_dev, Ls_tok, row_qb, inv, reinterpret_cast<uint4*>(k_cache),
+        reinterpret_cast<uint4*>(v_cache), reinterpret_cast<uint4*>(kidx_cache), reinterpret_cast<const uint4*>(q_new),
+        reinterpret_cast<const uint4*>(k_new), reinterpret_cast<const uint4*>(v_new),
+        reinterpret_cast<const uint4*>(k_idx_new), reinterpret_cast<uint4*>(q_rot));
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -257,6 +257,37 @@ qsa_status qsa_decode_reuse(const qsa_params* p, int32_t B, int64_t max_len, con
                             const uint16_t* v_new, const uint16_t* q_idx_new, const uint16_t* k_idx_new,
                             const uint16_t* w_new, const int32_t* sel_in, const int32_t* cnt_in, uint16_t* out,
                             float* lse_out, void* ws, size_t ws_bytes, void* stream);
+/* Batched verify of m new tokens per sequence (the target pass of a
+ * speculative round, [PT] "추측 디코딩을 위한 MTP와 그 밖에 유지된 설계"):
+ * sequence b has cache_len[b] (host array) tokens in its caches and its new
+ * tokens sit at positions L = cache_len[b] .. L + m - 1.  The result is, for
+ * every sequence, what qsa_prefill_cached gives with L_old = L and
+ * T_new = m: each query block the new tokens touch is scored over all its
+ * present tokens (prefill semantics: a block's selection sees every present
+ * block-mate, later new tokens included), selected as in stage 2, and every
+ * new token attends its block's selection causally.
+ * The new tokens are appended to the caches at L .. L + m - 1 (k rotated),
+ * as m decode steps would; the q_idx / w ring is only read: qidx_prev
+ * [B][4][4][128] and w_prev [B][4][4] hold, in slot t % 4, the indexer
+ * queries and head weights of the block-mates 4*(L/4) .. L-1 (a decode ring
+ * can be passed as is; NULL allowed when every cache_len[b] % 4 == 0).
+ * q_new [B][m][24][256], k_new, v_new [B][m][2][256], q_idx_new
+ * [B][m][4][128], k_idx_new [B][m][128], w_new [B][m][4]  ->  out
+ * [B][m][24][256] bf16, sel_out [B][m][budget] int32 (nullable: each token's
+ * block selection, -1 padded), lse_out [B][m][24] fp32 (nullable).
+ * Requires 1 <= m <= 16, cache_len[b] + m <= max_len, B <= 4096, and
+ * p->aggregation == QSA_AGG_TOKEN_MAX (QSA_ERR_UNSUPPORTED otherwise).
+ * Kernels: the decode append (per new token), the decode indexer over up to
+ * (m + 2) / 4 + 1 query blocks per sequence, the select, a per-token copy
+ * of the block's selection, and the split-KV decode attention with one row
+ * per new token. */
+qsa_status qsa_verify(const qsa_params* p, int32_t B, int32_t m, int64_t max_len, const int64_t* cache_len,
+                      uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, const uint16_t* qidx_prev,
+                      const uint16_t* w_prev, const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
+                      const uint16_t* q_idx_new, const uint16_t* k_idx_new, const uint16_t* w_new, uint16_t* out,
+                      int32_t* sel_out, float* lse_out, void* ws, size_t ws_bytes, void* stream);
+qsa_status qsa_verify_workspace_size(const qsa_params* p, int32_t B, int32_t m, int64_t max_len, size_t* bytes);
+
 /* kbar [ceil(T/4)][128] = the compressed keys of k_idx [T][128] (block b: bf16
  * of the mean of rows 4b .. min(4b+4, T)-1); no workspace; asynchronous. */
 qsa_status qsa_mean_pool_keys(const qsa_params* p, int64_t T, const uint16_t* k_idx, uint16_t* kbar, void* stream);
@@ -309,7 +340,8 @@ enum {
   QSA_KERNEL_DECODE_INDEXER = 7,
   QSA_KERNEL_DECODE_ATTENTION = 8,
   QSA_KERNEL_DECODE_COMBINE = 9,
-  QSA_KERNEL_KBAR = 10
+  QSA_KERNEL_KBAR = 10,
+  QSA_KERNEL_VERIFY_EXPAND = 11
 };
 qsa_status qsa_trace_begin(int32_t capacity);
 qsa_status qsa_trace_end(int32_t* kernel_ids, float* ms, int32_t capacity, int32_t* n_out);

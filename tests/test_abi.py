@@ -89,3 +89,26 @@ def test_decode_validation(lib):
     assert rc == 1
     rc = L.qsa_decode(ctypes.byref(p), 2, 64, lens, *fake[:11], fake[11], None, None, fake[12], 16, None)
     assert rc == 4
+
+
+def header_arg_counts():
+    """Number of parameters of every function prototype in the header."""
+    src = open(os.path.join(ROOT, "include", "qsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for name, args in re.findall(r"\b(qsa_[a-z_]+)\s*\(([^;{]*?)\)\s*;", src, flags=re.S):
+        args = args.strip()
+        out[name] = 0 if args in ("", "void") else args.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_header(lib):
+    """Every ctypes signature the binding declares has the header's
+    parameter count (a wrong count would shift pointer arguments)."""
+    counts = header_arg_counts()
+    assert len(counts) >= 10
+    for name, n in counts.items():
+        fn = getattr(lib, name)
+        if fn.argtypes is None:
+            continue
+        assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
