@@ -350,15 +350,18 @@ def run_prefill_cached(T: int, L_old: int, budget: int, steps: int, warmup: int,
 
 
 def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, world: int, seed: int,
-               want_e2e=True, aggregation: int = 0, spec: int = 0):
+               want_e2e=True, aggregation: int = 0, spec: int = 0, verify_m: int = 0):
     import block_sparse_long_qsa_b200 as qsa
     # one bench step = DECODE_CALLS consecutive decode tokens per sequence; with
     # spec = n they form rounds of n draft steps: a full decode step, whose
     # selection the next n - 1 steps reuse (qsa_decode_reuse)
+    # with verify_m = m every call is one qsa_verify of m new tokens per
+    # sequence (all accepted: the next call starts m positions later)
+    per_call = verify_m if verify_m else 1
     e_steps = max(1, min(steps, 3)) if want_e2e else 0
     n_calls = (warmup + steps + e_steps) * DECODE_CALLS
-    D = Q.DecodeProblem(B=B, L=L, steps=n_calls, seed=rank_seed(seed, rank), n_plant=8)
-    max_len = L + n_calls + 4
+    D = Q.DecodeProblem(B=B, L=L, steps=n_calls * per_call, seed=rank_seed(seed, rank), n_plant=8)
+    max_len = L + n_calls * per_call + 4
     kc = torch.empty((B, max_len, 2, 256), dtype=torch.uint16, device="cuda")
     vc = torch.empty_like(kc)
     ic = torch.empty((B, max_len, 128), dtype=torch.uint16, device="cuda")
@@ -372,15 +375,18 @@ def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, 
         kbar = torch.zeros((B, (max_len + 3) // 4, 128), dtype=torch.uint16, device="cuda")
         for b in range(B):
             qsa.qsa_mean_pool_keys(p, L, ic[b], kbar[b])
-    ws = qsa.workspace(qsa.qsa_decode_workspace_size(p, B, max_len))
-    out = torch.empty((B, 24, 256), dtype=torch.uint16, device="cuda")
+    ws = qsa.workspace(qsa.qsa_verify_workspace_size(p, B, verify_m, max_len) if verify_m else
+                       qsa.qsa_decode_workspace_size(p, B, max_len))
+    out = torch.empty((B, per_call, 24, 256) if verify_m else (B, 24, 256), dtype=torch.uint16, device="cuda")
     sel_round = torch.empty((B, budget), dtype=torch.int32, device="cuda") if spec > 1 else None
     # decode-token inputs of every call, generated once per sequence and kept resident: [call][B][...]
     names = ["q", "k", "v", "q_idx", "k_idx", "w"]
     per_seq = [D.tokens(b) for b in range(B)]
     allin = {}
     for k in names:
-        arr = np.stack([getattr(per_seq[b], k)(L, L + n_calls) for b in range(B)], axis=1)
+        arr = np.stack([getattr(per_seq[b], k)(L, L + n_calls * per_call) for b in range(B)], axis=1)
+        if verify_m:   # [call][B][m][...]
+            arr = arr.reshape(n_calls, per_call, *arr.shape[1:]).swapaxes(1, 2)
         allin[k] = torch.from_numpy(np.ascontiguousarray(arr)).cuda()
     step_in = [{k: allin[k][s] for k in names} for s in range(n_calls)]
     torch.cuda.synchronize()
@@ -388,6 +394,11 @@ def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, 
     pos = [L]
 
     def call(x):
+        if verify_m:
+            qsa.qsa_verify(p, B, verify_m, max_len, [pos[0]] * B, kc, vc, ic, ring, wring, x["q"], x["k"], x["v"],
+                           x["q_idx"], x["k_idx"], x["w"], out, ws=ws, stream=stream)
+            pos[0] += verify_m
+            return
         if spec > 1 and (pos[0] - L) % spec != 0:
             qsa.qsa_decode_reuse(p, B, max_len, [pos[0]] * B, kc, vc, ic, kbar, ring, wring, x["q"], x["k"], x["v"],
                                  x["q_idx"], x["k_idx"], x["w"], sel_round, None, out, ws=ws, stream=stream)
@@ -435,17 +446,19 @@ def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, 
     # once, the gathered K and V rows of the selected blocks, the appended token
     # and the inputs / outputs
     n_timed = steps * DECODE_CALLS
-    keys = B * (L_first + n_timed / 2 + 1)
+    # keys: every cached indexer key read once per call (the algorithmic
+    # figure, also for a verify whose query blocks each read them)
+    keys = B * (L_first + n_timed * per_call / 2 + 1)
     if aggregation == 1:
         keys /= 4            # one 256-byte compressed key per block
-    gathered = B * min(budget, L_first // 4 + 1) * 4 * 2 * 2 * 256 * 2
-    io = B * (24 * 256 * 2 * 2 + 2 * 2 * 256 * 2 + 128 * 2 * 2)
+    gathered = per_call * B * min(budget, L_first // 4 + 1) * 4 * 2 * 2 * 256 * 2
+    io = per_call * B * (24 * 256 * 2 * 2 + 2 * 2 * 256 * 2 + 128 * 2 * 2)
     # the indexer keys are read only by the calls that select
     select_share = 1.0 / spec if spec > 1 else 1.0
     bytes_call = keys * 256 * select_share + gathered + io
-    res = dict(ms=ms_max, tokens=B * n_timed * world, kern=kern, launches=sum(c for c, _ in kern.values()),
-               clocks=clk.summary(), bytes_step=bytes_call * DECODE_CALLS, bytes_indexer=keys * 256,
-               steps=steps, calls=n_timed)
+    res = dict(ms=ms_max, tokens=B * n_timed * per_call * world, kern=kern,
+               launches=sum(c for c, _ in kern.values()), clocks=clk.summary(), bytes_step=bytes_call * DECODE_CALLS,
+               bytes_indexer=keys * 256, steps=steps, calls=n_timed)
     if want_e2e:
         # every call: that call's inputs copied in from pinned host memory, the
         # output copied back
@@ -476,7 +489,7 @@ def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, 
         torch.cuda.synchronize()
         barrier(world)
         ems = max_over_ranks(e0.elapsed_time(e1), world)
-        res["e2e"] = dict(value=B * DECODE_CALLS * e_steps * world / (ems / 1e3), unit="tokens/s",
+        res["e2e"] = dict(value=B * DECODE_CALLS * per_call * e_steps * world / (ems / 1e3), unit="tokens/s",
                           h2d_bytes_per_step=bi, d2h_bytes_per_step=bo, steps=e_steps)
         del hosts, out_h
     del kc, vc, ic, ws, step_in, allin, kbar, sel_round
@@ -503,6 +516,8 @@ def cpu_sample(wl: dict, target_s: float = 12.0):
         n = 2
         agg = wl.get("aggregation", 0)
         spec = wl.get("spec", 0)
+        if wl.get("verify_m"):
+            return cpu_verify_sample(wl["B"], wl["L"], 512, wl["verify_m"], target_s)
         v, info = cpu_decode_sample(wl["B"], wl["L"], 512, n, aggregation=agg, spec=spec)
         if info["elapsed"] < target_s / 3:
             n2 = int(min(wl["B"], max(n + 1, n * target_s / max(info["elapsed"], 1e-3))))
@@ -601,6 +616,47 @@ def cpu_decode_sample(B: int, L: int, budget: int, n_seq: int, seed: int = 0, ag
                                               f"(scores + selection + attention), {elapsed:.1f} s", elapsed=elapsed)
 
 
+def cpu_verify_sample(B: int, L: int, budget: int, m: int, target_s: float = 12.0, seed: int = 0):
+    """The oracle on sampled sequences of a verify call: each query block the
+    m new tokens touch is scored over the cached keys and selected, then each
+    new token attends its block's selection (the cached K / V rows the
+    selection needs are materialised untimed; rows of earlier new tokens are
+    left zero -- the work per token is the same)."""
+    import oracle
+    O = oracle.Oracle(oracle.params(budget=budget))
+    D = Q.DecodeProblem(B=B, L=L, steps=m, seed=seed, n_plant=8)
+    elapsed, n_seq = 0.0, 0
+    ring_q, ring_w = np.zeros((0, 4, 128), np.uint16), np.zeros((0, 4), np.uint16)
+    while n_seq < B and (elapsed < target_s / 2 or n_seq < 1):
+        b = n_seq
+        P = D.tokens(b)
+        kid = np.concatenate([D.cache_kidx(b), P.k_idx(L, L + m)])
+        x = {k: getattr(P, k)(L, L + m) for k in ("q", "k", "v", "q_idx", "w")}
+        for qb in sorted({(L + i) // 4 for i in range(m)}):
+            t0, t1 = max(4 * qb, L), min(4 * qb + 4, L + m)
+            ta = time.time()
+            S = O.block_scores(qb, x["q_idx"][t0 - L:t1 - L], x["w"][t0 - L:t1 - L], kid[:t1])
+            sel, cnt = O.select(qb, S)
+            elapsed += time.time() - ta
+            kc = np.zeros((t1, 2, 256), np.uint16)
+            vc = np.zeros((t1, 2, 256), np.uint16)
+            for blk in sel[:cnt]:
+                a0, a1 = blk * 4, min(blk * 4 + 4, L)
+                if a1 > a0:
+                    kc[a0:a1] = D.cache_k(b, a0, a1)
+                    vc[a0:a1] = D.cache_v(b, a0, a1)
+            for t in range(t0, t1):
+                i = t - L
+                tb = time.time()
+                O.decode(t, kc[:t], vc[:t], kid[:t], ring_q, ring_w, x["q"][i], x["k"][i], x["v"][i], x["q_idx"][i],
+                         kid[t], x["w"][i], sel_in=sel, cnt_in=cnt)
+                elapsed += time.time() - tb
+        n_seq += 1
+    return n_seq * m / elapsed, dict(sample=f"{n_seq} of {B} sequences, {m} verify tokens each at {L} cached tokens "
+                                            f"(scores + selection per touched block, attention per token), "
+                                            f"{elapsed:.1f} s", elapsed=elapsed)
+
+
 def cores_used():
     try:
         return len(os.sched_getaffinity(0))
@@ -622,6 +678,8 @@ WORKLOADS = {
     "decode_64x256k_meanpool": dict(kind="decode", B=64, L=262144, aggregation=1),
     # speculative rounds of 4 draft tokens: one selection, reused by the next 3
     "decode_64x256k_spec4": dict(kind="decode", B=64, L=262144, spec=4),
+    # target-model verify of 5 draft tokens per sequence per call (all accepted)
+    "verify_64x256k_m5": dict(kind="decode", B=64, L=262144, verify_m=5),
 }
 
 
@@ -641,6 +699,8 @@ def metric_name(wl: dict) -> str:
     mp = ", mean-pooled indexer" if wl.get("aggregation") == 1 else ""
     if wl.get("spec"):
         mp += f", top-k reused across {wl['spec']}-step speculative rounds"
+    if wl.get("verify_m"):
+        return f"QSA verified tokens/s at 256K context, batch 64, {wl['verify_m']} tokens per sequence per call"
     return f"QSA decode tokens/s at 256K context, batch 64{mp}"
 
 
@@ -675,7 +735,8 @@ def line_for(name, res, n_gpus, steps, warmup, pk):
         whole["frac_of_hbm_roofline"] = whole["gbs"] / pk["hbm"]
         metric = metric_name(wl)
         cfg = dict(workload=name, batch=B, context=L, budget_blocks=512, planted="8 per sequence",
-                   decode_tokens_per_step=DECODE_CALLS, speculative_round=wl.get("spec") or None,
+                   decode_tokens_per_step=DECODE_CALLS * (wl.get("verify_m") or 1),
+                   speculative_round=wl.get("spec") or None, verify_tokens_per_call=wl.get("verify_m") or None,
                    l2=("1.07 GB of compressed indexer keys" if wl.get("aggregation") == 1 else
                        "4.3 GB of indexer keys") + " streamed per decode token (larger than L2)")
     return dict(metric=metric, value=value, unit="tokens/s", n_gpus=n_gpus, steps=steps, warmup=warmup,
@@ -786,13 +847,14 @@ def main():
                                  want_e2e=not args.no_e2e)
     else:
         res = run_decode(wl["B"], wl["L"], 512, args.steps, args.warmup, rank, world, seed=0,
-                         want_e2e=not args.no_e2e, aggregation=wl.get("aggregation", 0), spec=wl.get("spec", 0))
+                         want_e2e=not args.no_e2e, aggregation=wl.get("aggregation", 0), spec=wl.get("spec", 0),
+                         verify_m=wl.get("verify_m", 0))
     line = line_for(args.workload, res, world, args.steps, args.warmup, pk)
 
     if not args.no_secondary:
         sec = {}
         for name in ("decode_64x256k", "prefill_128k", "prefill_1m_cached90", "prefill_1m_meanpool",
-                     "decode_64x256k_meanpool", "decode_64x256k_spec4"):
+                     "decode_64x256k_meanpool", "decode_64x256k_spec4", "verify_64x256k_m5"):
             if name == args.workload:
                 continue
             w2 = WORKLOADS[name]
@@ -804,7 +866,8 @@ def main():
                                         want_e2e=False)
             else:
                 r2 = run_decode(w2["B"], w2["L"], 512, args.steps, args.warmup, rank, world, seed=0,
-                                want_e2e=False, aggregation=w2.get("aggregation", 0), spec=w2.get("spec", 0))
+                                want_e2e=False, aggregation=w2.get("aggregation", 0), spec=w2.get("spec", 0),
+                                verify_m=w2.get("verify_m", 0))
             l2 = line_for(name, r2, world, args.steps, args.warmup, pk)
             sec[name] = {k: l2[k] for k in ("metric", "value", "unit", "ms_per_step", "roofline", "step_roofline",
                                             "gpu_launches", "kernels_ms")}

@@ -96,8 +96,8 @@ decode_indexer_kernel(int64_t max_len, const int64_t* __restrict__ Ls, const uin
   float w[4];
   {
     const bool ok = q4 < present;
-#pragma unroll
     const int64_t pos = 4 * qb + q4;
+#pragma unroll
     for (int h = 0; h < 4; ++h)
       w[h] = ok ? bf16_bits_to_f32(VER && pos >= L ? w_new[(b * m + (pos - L)) * 4 + h] : w_ring[(b * 4 + q4) * 4 + h])
                 : 0.f;
@@ -176,6 +176,117 @@ decode_indexer_kernel(int64_t max_len, const int64_t* __restrict__ Ls, const uin
   }
 }
 
+// Verify whose new tokens touch two query blocks per sequence (nqv == 2):
+// one CTA row per sequence scores both blocks against each key tile it
+// loads, so the key cache is read once per call.  Same scores as the
+// one-block kernel: rows b * 2 + jb of S for blocks row_qb[b * 2 + jb]
+// (row_qb[b * 2 + 1] < 0: the new tokens stay in the first block).
+__global__ void __launch_bounds__(THREADS)
+verify_indexer2_kernel(int64_t max_len, const int64_t* __restrict__ Ls, const uint16_t* __restrict__ kidx_cache,
+                       const uint16_t* __restrict__ qidx_ring, const uint16_t* __restrict__ w_ring,
+                       float* __restrict__ S, int64_t ld, float scale, const int64_t* __restrict__ row_qb, int m,
+                       const uint16_t* __restrict__ qidx_new, const uint16_t* __restrict__ w_new) {
+  const int64_t b = blockIdx.y;
+  const int64_t L = Ls[b];
+  const int64_t pos_end = L + m - 1;
+  const int64_t qbv[2] = {row_qb[2 * b], row_qb[2 * b + 1]};
+  const bool two = qbv[1] >= 0;
+  const int64_t qb_last = two ? qbv[1] : qbv[0];
+  const int64_t last_row = 4 * qb_last + 3 < pos_end ? 4 * qb_last + 3 : pos_end;
+  const int64_t j_begin = (int64_t)blockIdx.x * KEYS_PER_CTA;
+  if (j_begin > last_row) return;
+  int64_t j_end = j_begin + KEYS_PER_CTA;
+  if (j_end > 4 * qb_last + 4) j_end = 4 * qb_last + 4;
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g8 = lane >> 2, q4 = lane & 3;
+  uint4 qf[2][2][4];
+  float w[2][4];
+  int64_t t_tok[2];
+  bool tok_ok[2];
+#pragma unroll
+  for (int jb = 0; jb < 2; ++jb) {
+    const int64_t qb = qbv[jb];
+    const int64_t lk = 4 * qb + 3 < pos_end ? 4 * qb + 3 : pos_end;
+    const int present = qb < 0 ? 0 : (int)(lk - 4 * qb) + 1;
+    const int tok = g8 >> 1;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const int head = 2 * nt + (g8 & 1);
+      const int64_t pos = 4 * qb + tok;
+      const uint4* src = reinterpret_cast<const uint4*>(pos >= L ? qidx_new + ((b * m + (pos - L)) * 4 + head) * 128
+                                                                 : qidx_ring + ((b * 4 + tok) * 4 + head) * 128);
+#pragma unroll
+      for (int d = 0; d < 4; ++d) qf[jb][nt][d] = tok < present ? src[4 * d + q4] : make_uint4(0, 0, 0, 0);
+    }
+    const int64_t pos = 4 * qb + q4;
+#pragma unroll
+    for (int h = 0; h < 4; ++h)
+      w[jb][h] = q4 < present ? bf16_bits_to_f32(pos >= L ? w_new[(b * m + (pos - L)) * 4 + h]
+                                                          : w_ring[(b * 4 + q4) * 4 + h])
+                              : 0.f;
+    t_tok[jb] = pos;
+    tok_ok[jb] = q4 < present;
+  }
+  const uint16_t* kb_base = kidx_cache + b * max_len * 128;
+
+  constexpr int64_t STEP = 16 * (THREADS / 32);
+  auto load_tile = [&](int64_t jt, uint4 (&k0)[4], uint4 (&k1)[4]) {
+    const int64_t j0 = jt + g8, j1 = jt + g8 + 8;
+    const int64_t r0 = j0 <= last_row ? j0 : last_row, r1 = j1 <= last_row ? j1 : last_row;
+    const uint4* k0p = reinterpret_cast<const uint4*>(kb_base + r0 * 128);
+    const uint4* k1p = reinterpret_cast<const uint4*>(kb_base + r1 * 128);
+#pragma unroll
+    for (int d = 0; d < 4; ++d) { k0[d] = ldg_stream(k0p + 4 * d + q4); k1[d] = ldg_stream(k1p + 4 * d + q4); }
+  };
+  uint4 n0[4], n1[4];
+  if (j_begin + 16 * warp < j_end) load_tile(j_begin + 16 * warp, n0, n1);
+  for (int64_t jt = j_begin + 16 * warp; jt < j_end; jt += STEP) {
+    const int64_t j0 = jt + g8, j1 = jt + g8 + 8;
+    uint4 k0[4], k1[4];
+#pragma unroll
+    for (int d = 0; d < 4; ++d) { k0[d] = n0[d]; k1[d] = n1[d]; }
+    if (jt + STEP < j_end) load_tile(jt + STEP, n0, n1);
+#pragma unroll
+    for (int jb = 0; jb < 2; ++jb) {
+      if (jb == 1 && !two) break;
+      const int64_t qb = qbv[jb];
+      float acc[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+      for (int d = 0; d < 4; ++d) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          mma16816(acc[nt], k0[d].x, k1[d].x, k0[d].y, k1[d].y, qf[jb][nt][d].x, qf[jb][nt][d].y);
+          mma16816(acc[nt], k0[d].z, k1[d].z, k0[d].w, k1[d].w, qf[jb][nt][d].z, qf[jb][nt][d].w);
+        }
+      }
+      float s0 = w[jb][0] * fmaxf(acc[0][0], 0.f);
+      s0 = fmaf(w[jb][1], fmaxf(acc[0][1], 0.f), s0);
+      s0 = fmaf(w[jb][2], fmaxf(acc[1][0], 0.f), s0);
+      s0 = fmaf(w[jb][3], fmaxf(acc[1][1], 0.f), s0);
+      float s1 = w[jb][0] * fmaxf(acc[0][2], 0.f);
+      s1 = fmaf(w[jb][1], fmaxf(acc[0][3], 0.f), s1);
+      s1 = fmaf(w[jb][2], fmaxf(acc[1][2], 0.f), s1);
+      s1 = fmaf(w[jb][3], fmaxf(acc[1][3], 0.f), s1);
+      s0 = (tok_ok[jb] && j0 <= t_tok[jb]) ? s0 : 0.f;
+      s1 = (tok_ok[jb] && j1 <= t_tok[jb]) ? s1 : 0.f;
+#pragma unroll
+      for (int off = 1; off <= 8; off <<= 1) {
+        s0 = fmaxf(s0, __shfl_xor_sync(0xffffffffu, s0, off));
+        s1 = fmaxf(s1, __shfl_xor_sync(0xffffffffu, s1, off));
+      }
+      if ((lane & 15) == 0) {
+        float* Srow = S + (2 * b + jb) * ld;
+        const int64_t kb0 = (jt >> 2) + (lane >> 4);
+        if (kb0 <= qb) Srow[kb0] = s0 * scale;
+        if (kb0 + 2 <= qb) Srow[kb0 + 2] = s1 * scale;
+      }
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_decode_indexer(int B, int64_t max_len, int64_t max_L, const int64_t* L_dev,
@@ -203,6 +314,12 @@ cudaError_t launch_verify_indexer(int B, int nqv, int m, int64_t max_len, int64_
   if (B <= 0) return cudaSuccess;
   const int64_t rows = max_L + m + 3;                 // keys up to the last new token's block end
   const int64_t nx = (rows + KEYS_PER_CTA - 1) / KEYS_PER_CTA;
+  if (nqv == 2) {
+    verify_indexer2_kernel<<<dim3((unsigned)nx, (unsigned)B), THREADS, 0, s>>>(max_len, Lb_dev, kidx_cache, qidx_ring,
+                                                                               w_ring, S, ld, scale, row_qb, m,
+                                                                               qidx_new, w_new);
+    return cudaGetLastError();
+  }
   dim3 grid((unsigned)nx, (unsigned)(B * nqv));
   decode_indexer_kernel<false, true><<<grid, THREADS, 0, s>>>(max_len, Lb_dev, kidx_cache, nullptr, 0, qidx_ring,
                                                               w_ring, S, ld, scale, row_qb, nqv, m, qidx_new, w_new);
