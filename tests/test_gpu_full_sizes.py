@@ -293,3 +293,52 @@ def test_decode_mean_pool_and_reuse_full_size_sampled():
                                       in1["k"][b], in1["v"][b], in1["q_idx"][b], kin1, in1["w"][b], sel_in=g,
                                       cnt_in=gc)
         check_outputs(outs[1][b], oo1, f"reuse draft step b={b}")
+
+
+@pytest.mark.timeout(1800)
+def test_verify_full_size_sampled():
+    """64 sequences x 256K cached tokens, 5 new tokens each (as the benchmark's
+    verify calls): sampled sequences against the oracle -- selection of both
+    touched query blocks, and every new token's output on its selection."""
+    B, L, m = 64, 262144, 5
+    st = _decode_full_setup(B, L)
+    D, p = st["D"], st["p"]
+    new = {k: [] for k in ("q", "k", "v", "q_idx", "k_idx", "w")}
+    for b in range(B):
+        P = D.tokens(b)
+        for k in new:
+            new[k].append(getattr(P, k)(L, L + m))
+    x = {k: torch.from_numpy(np.ascontiguousarray(np.stack(v))).cuda() for k, v in new.items()}
+    ws = qsa.workspace(qsa.qsa_verify_workspace_size(p, B, m, st["max_len"]))
+    out = torch.empty((B, m, 24, 256), dtype=torch.uint16, device="cuda")
+    sel = torch.empty((B, m, BUDGET), dtype=torch.int32, device="cuda")
+    lse = torch.empty((B, m, 24), dtype=torch.float32, device="cuda")
+    qsa.qsa_verify(p, B, m, st["max_len"], [L] * B, st["kc"], st["vc"], st["ic"], st["ring"], st["wring"], x["q"],
+                   x["k"], x["v"], x["q_idx"], x["k_idx"], x["w"], out, sel, lse, ws)
+    torch.cuda.synchronize()
+    assert qsa.qsa_check_device_error(ws) == 0
+    out, sel, lse = out.cpu().numpy(), sel.cpu().numpy(), lse.cpu().numpy()
+    new_krot = st["kc"][:, L:L + m].cpu().numpy()
+    del st, ws
+    O = oracle.Oracle(oracle.params(budget=BUDGET))
+    ring_q, ring_w = np.zeros((0, 4, 128), np.uint16), np.zeros((0, 4), np.uint16)
+    for b in (0, 33, 63):
+        nb = {k: v[b] for k, v in new.items()}
+        kid = np.concatenate([D.cache_kidx(b), nb["k_idx"]])
+        kc_full, vc_full = D.cache_k(b), D.cache_v(b)
+        for qb in sorted({(L + i) // 4 for i in range(m)}):
+            t0, t1 = max(4 * qb, L), min(4 * qb + 4, L + m)
+            S = O.block_scores(qb, nb["q_idx"][t0 - L:t1 - L], nb["w"][t0 - L:t1 - L], kid[:t1])
+            osel, ocnt = O.select(qb, S)
+            g = sel[b, t0 - L]
+            gc = int((g >= 0).sum())
+            check_selection(g, gc, osel, ocnt, S, qb, BUDGET, f"verify b={b} qb={qb}")
+            for t in range(t0, t1):
+                i = t - L
+                assert np.array_equal(sel[b, i], g)
+                kc = np.concatenate([kc_full, new_krot[b, :i]])
+                vc = np.concatenate([vc_full, nb["v"][:i]])
+                _, _, oo, ol = O.decode(t, kc, vc, kid[:t], ring_q, ring_w, nb["q"][i], nb["k"][i], nb["v"][i],
+                                        nb["q_idx"][i], kid[t], nb["w"][i], sel_in=g, cnt_in=gc)
+                check_outputs(out[b, i], oo, f"verify b={b} t={t}")
+                assert np.allclose(lse[b, i], ol, atol=1e-2), f"verify b={b} t={t} lse"
