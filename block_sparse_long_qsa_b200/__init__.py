@@ -86,7 +86,7 @@ def load(path: str = LIB_PATH):
     L.qsa_decode_workspace_size.argtypes = [P, i32, i64, psz]
     L.qsa_decode_mean_pool.argtypes = [P, i32, i64, ctypes.POINTER(ctypes.c_int64)] + [vp] * 15 + [vp, sz, vp]
     L.qsa_mean_pool_keys.argtypes = [P, i64, vp, vp, vp]
-    L.qsa_verify.argtypes = [P, i32, i32, i64, ctypes.POINTER(ctypes.c_int64)] + [vp] * 14 + [vp, sz, vp]
+    L.qsa_verify.argtypes = [P, i32, i32, i64, ctypes.POINTER(ctypes.c_int64)] + [vp] * 15 + [vp, sz, vp]
     L.qsa_verify_workspace_size.argtypes = [P, i32, i32, i64, psz]
     L.qsa_decode_reuse.argtypes = [P, i32, i64, ctypes.POINTER(ctypes.c_int64)] + [vp] * 16 + [vp, sz, vp]
     L.qsa_decode_noalloc.argtypes = [P, i32, i64, ctypes.POINTER(ctypes.c_int64), vp, vp, vp, vp, vp, vp, vp, vp,
@@ -237,11 +237,12 @@ def qsa_verify_workspace_size(p: qsa_params, B: int, m: int, max_len: int) -> in
 
 def qsa_verify(p: qsa_params, B: int, m: int, max_len: int, cache_len, k_cache, v_cache, kidx_cache, qidx_prev,
                w_prev, q_new, k_new, v_new, q_idx_new, k_idx_new, w_new, out, sel_out=None, lse_out=None, ws=None,
-               stream=None):
-    """Verify m new tokens per sequence (``cache_len``: host sequence of B ints)."""
+               stream=None, kbar_cache=None):
+    """Verify m new tokens per sequence (``cache_len``: host sequence of B
+    ints; ``kbar_cache`` only with mean-pooled parameters)."""
     lens = (ctypes.c_int64 * B)(*[int(x) for x in cache_len])
     _check(load().qsa_verify(ctypes.byref(p), B, m, max_len, lens, _ptr(k_cache), _ptr(v_cache), _ptr(kidx_cache),
-                             _ptr(qidx_prev), _ptr(w_prev), _ptr(q_new), _ptr(k_new), _ptr(v_new), _ptr(q_idx_new),
+                             _ptr(kbar_cache), _ptr(qidx_prev), _ptr(w_prev), _ptr(q_new), _ptr(k_new), _ptr(v_new), _ptr(q_idx_new),
                              _ptr(k_idx_new), _ptr(w_new), _ptr(out), _ptr(sel_out), _ptr(lse_out), _ptr(ws),
                              ws.numel() * ws.element_size(), _stream(stream)), "qsa_verify")
 

@@ -877,14 +877,16 @@ qsa_status qsa_verify_workspace_size(const qsa_params* p, int32_t B, int32_t m, 
 }
 
 qsa_status qsa_verify(const qsa_params* p, int32_t B, int32_t m, int64_t max_len, const int64_t* cache_len,
-                      uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, const uint16_t* qidx_prev,
+                      uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* kbar_cache,
+                      const uint16_t* qidx_prev,
                       const uint16_t* w_prev, const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
                       const uint16_t* q_idx_new, const uint16_t* k_idx_new, const uint16_t* w_new, uint16_t* out,
                       int32_t* sel_out, float* lse_out, void* ws, size_t ws_bytes, void* stream) {
   qsa_status st = check_params(p);
   if (st != QSA_OK) return st;
-  if (mean_pool(p)) return QSA_ERR_UNSUPPORTED;   // token-pair scores only
   if (B <= 0 || m <= 0 || max_len <= 0 || !cache_len) return QSA_ERR_INVALID_ARG;
+  if (mean_pool(p) != (kbar_cache != nullptr)) return QSA_ERR_INVALID_ARG;   // the compressed keys go with mean pool
+  if (kbar_cache && !aligned16(kbar_cache)) return QSA_ERR_MISALIGNED;
   if (B > 4096 || m > VERIFY_MAX_M || max_len > ((int64_t)1 << 24)) return QSA_ERR_UNSUPPORTED;
   const void* ptrs[] = {k_cache, v_cache, kidx_cache, q_new, k_new, v_new, q_idx_new, k_idx_new, w_new, out, ws};
   for (const void* ptr : ptrs) {
@@ -932,10 +934,16 @@ qsa_status qsa_verify(const qsa_params* p, int32_t B, int32_t m, int64_t max_len
                                           k_cache, v_cache, kidx_cache, q_new, k_new, v_new, k_idx_new, q_rot, s);
        }))) != QSA_OK)
     return st;
+  const int64_t kbar_len = (max_len + 3) / 4;
+  if (kbar_cache && (st = from_cuda(traced(QSA_KERNEL_KBAR, s, [&] {
+                       return qsa::launch_verify_kbar(B, m, L.nqv, max_len, kbar_len, Lb, rqb, kidx_cache,
+                                                      kbar_cache, s);
+                     }))) != QSA_OK)
+    return st;
   const float scale = 1.0f / std::sqrt(128.0f);
   if ((st = from_cuda(traced(QSA_KERNEL_DECODE_INDEXER, s, [&] {
-         return qsa::launch_verify_indexer(B, L.nqv, m, max_len, max_L, Lb, rqb, kidx_cache, qidx_prev, w_prev,
-                                           q_idx_new, w_new, S, L.ld, scale, s);
+         return qsa::launch_verify_indexer(B, L.nqv, m, max_len, max_L, Lb, rqb, kidx_cache, kbar_cache, kbar_len,
+                                           qidx_prev, w_prev, q_idx_new, w_new, S, L.ld, scale, s);
        }))) != QSA_OK)
     return st;
   if ((st = from_cuda(traced(QSA_KERNEL_SELECT, s, [&] {

@@ -308,10 +308,19 @@ cudaError_t launch_decode_indexer(int B, int64_t max_len, int64_t max_L, const i
 }
 
 cudaError_t launch_verify_indexer(int B, int nqv, int m, int64_t max_len, int64_t max_L, const int64_t* Lb_dev,
-                                  const int64_t* row_qb, const uint16_t* kidx_cache, const uint16_t* qidx_ring,
-                                  const uint16_t* w_ring, const uint16_t* qidx_new, const uint16_t* w_new, float* S,
-                                  int64_t ld, float scale, cudaStream_t s) {
+                                  const int64_t* row_qb, const uint16_t* kidx_cache, const uint16_t* kbar_cache,
+                                  int64_t kbar_len, const uint16_t* qidx_ring, const uint16_t* w_ring,
+                                  const uint16_t* qidx_new, const uint16_t* w_new, float* S, int64_t ld, float scale,
+                                  cudaStream_t s) {
   if (B <= 0) return cudaSuccess;
+  if (kbar_cache) {   // mean pool: rows are the compressed key blocks 0 .. qb
+    const int64_t nkb = (max_L + m + 3) / 4 + 1;
+    const int64_t nxb = (nkb + KEYS_PER_CTA - 1) / KEYS_PER_CTA;
+    decode_indexer_kernel<true, true><<<dim3((unsigned)nxb, (unsigned)(B * nqv)), THREADS, 0, s>>>(
+        max_len, Lb_dev, kidx_cache, kbar_cache, kbar_len, qidx_ring, w_ring, S, ld, scale, row_qb, nqv, m, qidx_new,
+        w_new);
+    return cudaGetLastError();
+  }
   const int64_t rows = max_L + m + 3;                 // keys up to the last new token's block end
   const int64_t nx = (rows + KEYS_PER_CTA - 1) / KEYS_PER_CTA;
   if (nqv == 2) {
@@ -323,6 +332,32 @@ cudaError_t launch_verify_indexer(int B, int nqv, int m, int64_t max_len, int64_
   dim3 grid((unsigned)nx, (unsigned)(B * nqv));
   decode_indexer_kernel<false, true><<<grid, THREADS, 0, s>>>(max_len, Lb_dev, kidx_cache, nullptr, 0, qidx_ring,
                                                               w_ring, S, ld, scale, row_qb, nqv, m, qidx_new, w_new);
+  return cudaGetLastError();
+}
+
+// Compressed keys of the query blocks a verify touches, from the caches after
+// the append: row r = (b, j) rewrites kbar[b][row_qb[r]] as the bf16 (round
+// to nearest even) of the exact mean of the block's present keys.
+__global__ void verify_kbar_kernel(int m, int nqv, int64_t max_len, int64_t kbar_len, const int64_t* __restrict__ Lb,
+                                   const int64_t* __restrict__ row_qb, const uint16_t* __restrict__ kidx_cache,
+                                   uint16_t* __restrict__ kbar_cache) {
+  const int64_t r = blockIdx.x, b = r / nqv;
+  const int64_t qb = row_qb[r];
+  if (qb < 0) return;
+  const int64_t t0 = 4 * qb, t_end = Lb[b] + m;     // present keys t0 .. t_end - 1 (at most 4)
+  const int n = (int)(t_end - t0 < 4 ? t_end - t0 : 4);
+  const int c = threadIdx.x;
+  const uint16_t* kc = kidx_cache + b * max_len * 128;
+  double sum = 0.0;
+  for (int i = 0; i < n; ++i) sum += (double)__uint_as_float((uint32_t)kc[(t0 + i) * 128 + c] << 16);
+  kbar_cache[(b * kbar_len + qb) * 128 + c] = f64_to_bf16_rne(sum / (double)n);
+}
+
+cudaError_t launch_verify_kbar(int B, int m, int nqv, int64_t max_len, int64_t kbar_len, const int64_t* Lb,
+                               const int64_t* row_qb, const uint16_t* kidx_cache, uint16_t* kbar_cache,
+                               cudaStream_t s) {
+  if (B <= 0) return cudaSuccess;
+  verify_kbar_kernel<<<B * nqv, 128, 0, s>>>(m, nqv, max_len, kbar_len, Lb, row_qb, kidx_cache, kbar_cache);
   return cudaGetLastError();
 }
 

@@ -85,10 +85,15 @@ cudaError_t launch_verify_append(int B, int m, int nqv, int64_t max_len, const i
                                  uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, const uint16_t* q_new,
                                  const uint16_t* k_new, const uint16_t* v_new, const uint16_t* k_idx_new,
                                  uint16_t* q_rot, cudaStream_t s);
+// kbar_cache non-null: mean-pooled scores over the compressed keys.
 cudaError_t launch_verify_indexer(int B, int nqv, int m, int64_t max_len, int64_t max_L, const int64_t* Lb_dev,
-                                  const int64_t* row_qb, const uint16_t* kidx_cache, const uint16_t* qidx_ring,
-                                  const uint16_t* w_ring, const uint16_t* qidx_new, const uint16_t* w_new, float* S,
-                                  int64_t ld, float scale, cudaStream_t s);
+                                  const int64_t* row_qb, const uint16_t* kidx_cache, const uint16_t* kbar_cache,
+                                  int64_t kbar_len, const uint16_t* qidx_ring, const uint16_t* w_ring,
+                                  const uint16_t* qidx_new, const uint16_t* w_new, float* S, int64_t ld, float scale,
+                                  cudaStream_t s);
+cudaError_t launch_verify_kbar(int B, int m, int nqv, int64_t max_len, int64_t kbar_len, const int64_t* Lb,
+                               const int64_t* row_qb, const uint16_t* kidx_cache, uint16_t* kbar_cache,
+                               cudaStream_t s);
 cudaError_t launch_verify_expand(int B, int m, int nqv, int budget, const int64_t* Ls_tok, const int32_t* sel_blk,
                                  const int32_t* cnt_blk, int32_t* sel_tok, int32_t* cnt_tok, cudaStream_t s);
 cudaError_t launch_decode_combine(int B, const float* part_o, const float* part_lse, const int32_t* cnt, int n_split,

@@ -275,14 +275,19 @@ qsa_status qsa_decode_reuse(const qsa_params* p, int32_t B, int64_t max_len, con
  * [B][m][4][128], k_idx_new [B][m][128], w_new [B][m][4]  ->  out
  * [B][m][24][256] bf16, sel_out [B][m][budget] int32 (nullable: each token's
  * block selection, -1 padded), lse_out [B][m][24] fp32 (nullable).
- * Requires 1 <= m <= 16, cache_len[b] + m <= max_len, B <= 4096, and
- * p->aggregation == QSA_AGG_TOKEN_MAX (QSA_ERR_UNSUPPORTED otherwise).
+ * Requires 1 <= m <= 16, cache_len[b] + m <= max_len, B <= 4096.
+ * With p->aggregation == QSA_AGG_MEAN_POOL, kbar_cache [B][ceil(max_len/4)]
+ * [128] is the compressed-key cache (as for qsa_decode_mean_pool): the rows
+ * of the blocks the new tokens touch are rewritten from their present keys
+ * and the blocks are scored over the compressed keys; kbar_cache must be
+ * NULL otherwise.
  * Kernels: the decode append (per new token), the decode indexer over up to
  * (m + 2) / 4 + 1 query blocks per sequence, the select, a per-token copy
  * of the block's selection, and the split-KV decode attention with one row
  * per new token. */
 qsa_status qsa_verify(const qsa_params* p, int32_t B, int32_t m, int64_t max_len, const int64_t* cache_len,
-                      uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, const uint16_t* qidx_prev,
+                      uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* kbar_cache,
+                      const uint16_t* qidx_prev,
                       const uint16_t* w_prev, const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
                       const uint16_t* q_idx_new, const uint16_t* k_idx_new, const uint16_t* w_new, uint16_t* out,
                       int32_t* sel_out, float* lse_out, void* ws, size_t ws_bytes, void* stream);

@@ -23,7 +23,7 @@ def _lib():
     qsa.load()
 
 
-def run_verify(st, m, ws=None):
+def run_verify(st, m, ws=None, kbar=None):
     """qsa_verify of the next m tokens of every sequence of a DecodeState."""
     B = st.B
     new = {k: np.stack([st.hosts[b][k][st.lens[b]:st.lens[b] + m] for b in range(B)]) for k in
@@ -35,7 +35,7 @@ def run_verify(st, m, ws=None):
         ws = qsa.workspace(qsa.qsa_verify_workspace_size(st.p, B, m, st.max_len))
     qsa.qsa_verify(st.p, B, m, st.max_len, st.lens, st.k_cache, st.v_cache, st.kidx_cache, st.qidx_ring, st.w_ring,
                    dev(new["q"]), dev(new["k"]), dev(new["v"]), dev(new["q_idx"]), dev(new["k_idx"]), dev(new["w"]),
-                   out, sel, lse, ws)
+                   out, sel, lse, ws, kbar_cache=kbar)
     torch.cuda.synchronize()
     assert qsa.qsa_check_device_error(ws) == 0
     return out.cpu().numpy(), sel.cpu().numpy(), lse.cpu().numpy()
@@ -102,6 +102,43 @@ def test_verify_checks():
         qsa.qsa_verify_workspace_size(st.p, 1, 17, 40)
     assert "UNSUPPORTED" in str(e.value)
     st.p = qsa.params(budget, aggregation=qsa.AGG_MEAN_POOL)
-    with pytest.raises(qsa.QSAError) as e:
+    with pytest.raises(qsa.QSAError) as e:          # mean pool needs the compressed-key cache
         run_verify(st, 2, ws=qsa.workspace(1 << 20))
-    assert "UNSUPPORTED" in str(e.value)
+    assert "INVALID_ARG" in str(e.value)
+
+
+@pytest.mark.parametrize("budget,m", [(16, 5), (512, 5), (512, 9)])
+def test_verify_mean_pool_equals_prefill(budget, m):
+    """Mean-pooled verify: the compressed keys of the touched blocks are
+    rewritten (equal to qsa_mean_pool_keys over the extended cache) and every
+    token matches the mean-pool prefill of the whole sequence."""
+    L_list = [2048 + 4 * budget, 2302, 4099] if budget == 512 else [64, 129, 303]
+    probs = [Q.PrefillProblem(T=L + m, seed=700 + b + m, n_plant=8) for b, L in enumerate(L_list)]
+    st = DecodeState(probs, L_list, max_len=max(L_list) + m + 8, budget=budget)
+    st.p = qsa.params(budget, aggregation=qsa.AGG_MEAN_POOL)
+    kbar = torch.zeros((st.B, (st.max_len + 3) // 4, 128), dtype=torch.uint16, device="cuda")
+    for b, L in enumerate(L_list):
+        qsa.qsa_mean_pool_keys(st.p, L, st.kidx_cache[b], kbar[b])
+    out, sel, lse = run_verify(st, m, kbar=kbar)
+    O = oracle.Oracle(oracle.params(budget=budget, aggregation=oracle.AGG_MEAN_POOL))
+    for b, L in enumerate(L_list):
+        T = L + m
+        want = torch.zeros_like(kbar[b])
+        qsa.qsa_mean_pool_keys(st.p, T, st.kidx_cache[b], want)
+        torch.cuda.synchronize()
+        nb = (T + 3) // 4
+        assert torch.equal(kbar[b, :nb], want[:nb]), f"b={b} compressed keys"
+        h = st.hosts[b]
+        t_in = {k: dev(v[:T]) for k, v in h.items()}
+        full = qsa.prefill(t_in["q"], t_in["k"], t_in["v"], t_in["q_idx"], t_in["w"], t_in["k_idx"], budget=budget,
+                           aggregation=qsa.AGG_MEAN_POOL)
+        torch.cuda.synchronize()
+        fsel, fcnt, fout = full["sel"].cpu().numpy(), full["cnt"].cpu().numpy(), full["out"].cpu().numpy()
+        for i in range(m):
+            t = L + i
+            qb = t // 4
+            g = sel[b, i]
+            S = O.block_scores(qb, h["q_idx"][4 * qb:min(4 * qb + 4, T)], h["w"][4 * qb:min(4 * qb + 4, T)],
+                               h["k_idx"][:T])
+            check_selection(g, int((g >= 0).sum()), fsel[qb], int(fcnt[qb]), S, qb, budget, f"b={b} t={t}")
+            check_outputs(out[b, i], Q.bf16_to_f64(fout[t]), f"mean-pool verify vs prefill b={b} t={t}")
