@@ -69,7 +69,7 @@ def _select_exact_cpu(row32: np.ndarray, qb: int, budget: int) -> np.ndarray:
     return np.sort(np.concatenate([cand[order[:budget - 2]], [qb - 1, qb]]))
 
 
-@pytest.mark.parametrize("budget", [2, 16, 512])
+@pytest.mark.parametrize("budget", [2, 16, 512, 1000, 4096])
 def test_select_exact_on_given_scores(budget):
     """Index work is bit-exact: the GPU select on fp32 rows equals the CPU
     reference on the same values, including ties, -0.0 and long rows that
@@ -176,3 +176,28 @@ def test_prefill_chunked_workspace_matches_single_pass():
     _, r2 = gpu_prefill(P, budget, host=host, ws_bytes=mn)
     assert np.array_equal(r1["sel"], r2["sel"]) and np.array_equal(r1["cnt"], r2["cnt"])
     assert np.array_equal(r1["out"], r2["out"])
+
+
+@pytest.mark.parametrize("budget", [1000, 4096])
+def test_prefill_large_budget_sampled(budget):
+    """Budgets up to the largest the library accepts (4096 blocks = 16K keys
+    per query block): sampled query blocks against the oracle, the rest
+    checked for structure."""
+    T = 40001
+    P = Q.PrefillProblem(T=T, seed=77, n_plant=8)
+    host, r = gpu_prefill(P, budget)
+    O = oracle.Oracle(oracle.params(budget=budget))
+    nqb = P.nqb
+    cnt = r["cnt"]
+    assert np.array_equal(cnt, np.minimum(np.arange(nqb) + 1, budget)), "counts"
+    qbs = np.array([0, 1, budget - 2, budget - 1, budget, budget + 1, nqb // 2, nqb - 2, nqb - 1])
+    qbs = np.unique(qbs[(qbs >= 0) & (qbs < nqb)])
+    for qb in qbs:
+        t0, t1 = 4 * qb, min(4 * qb + 4, T)
+        S = O.block_scores(int(qb), host["q_idx"][t0:t1], host["w"][t0:t1], host["k_idx"][:t1])
+        osel, ocnt = O.select(int(qb), S)
+        check_selection(r["sel"][qb], int(cnt[qb]), osel, ocnt, S, int(qb), budget, f"qb={qb}")
+    out, lse = O.attend_blocks(T, host["q"], host["k"], host["v"], qbs, r["sel"][qbs], cnt[qbs])
+    for i, qb in enumerate(qbs):
+        for t in range(4 * qb, min(4 * qb + 4, T)):
+            check_outputs(r["out"][t], out[4 * i + t - 4 * qb], f"budget={budget} t={t}")
