@@ -292,10 +292,11 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
       const int nsel = it.cnt - 16 * it.tile0;     // selected blocks from this item's first tile on
       const int64_t t_last = it.t_last;
       // Thread (warp w, lane c32) copies 16-byte chunk c32 of token w % 4 of
-      // each of its KPT blocks of a tile (all 16 with 4 loader warps, half
-      // with 8), for K and for V: key slot n = 4k + w % 4.  The block indices
-      // of tile i + 1 are loaded while tile i waits for its stage, so the
-      // index loads' latency stays off the issue path.
+      // each of its KPT blocks of a tile (blocks k0 .. k0 + KPT - 1: warps
+      // 0-3 the first 8 of the 16, warps 4-7 the last 8), for K and for V:
+      // key slot n = 4k + w % 4.  The block indices of tiles i + 1 and i + 2
+      // are loaded while tile i waits for its stage, so the index loads'
+      // latency stays off the issue path.
       constexpr int KPT = 64 / LWARPS;
       const int w4 = (tid >> 5) & 3, c32 = tid & 31, k0 = KPT * (tid >> 7);
       int32_t kbv[KPT], kbn[KPT], kbm[KPT];
