@@ -147,3 +147,29 @@ def test_decode_split_kv_ranges(splits, monkeypatch):
                                 cnt_in=cnt)
         check_outputs(out[b], oo, f"splits={splits} b={b}")
         assert np.allclose(lse[b], ol, atol=1e-2), f"splits={splits} b={b}"
+
+
+def test_decode_largest_budget():
+    """Budget 4096 (the largest accepted): the selection binds only past
+    16K keys; decode against the prefill's last token and the oracle."""
+    budget = 4096
+    L_list = [20001, 16390]
+    probs = [Q.PrefillProblem(T=L + 1, seed=90 + b, n_plant=8) for b, L in enumerate(L_list)]
+    st = DecodeState(probs, L_list, max_len=max(L_list) + 8, budget=budget)
+    pos, out, sel, lse = st.step()
+    O = oracle.Oracle(oracle.params(budget=budget))
+    for b, L in enumerate(pos):
+        h = st.hosts[b]
+        T = L + 1
+        _, r = gpu_prefill(Q.PrefillProblem(T=T, seed=probs[b].seed), budget, host={k: v[:T] for k, v in h.items()})
+        qb = L // 4
+        cnt = int((sel[b] >= 0).sum())
+        assert cnt == min(qb + 1, budget)
+        S = O.block_scores(qb, h["q_idx"][4 * qb:T], h["w"][4 * qb:T], h["k_idx"][:T])
+        check_selection(sel[b], cnt, r["sel"][qb], int(r["cnt"][qb]), S, qb, budget, f"b={b}")
+        check_outputs(out[b], Q.bf16_to_f64(r["out"][L]), f"budget 4096 decode b={b}")
+        kc = st.k_cache[b, :L].cpu().numpy()
+        t0 = 4 * qb
+        _, _, oo, _ = O.decode(L, kc, h["v"][:L], h["k_idx"][:L], h["q_idx"][t0:L], h["w"][t0:L], h["q"][L], h["k"][L],
+                               h["v"][L], h["q_idx"][L], h["k_idx"][L], h["w"][L], sel_in=sel[b], cnt_in=cnt)
+        check_outputs(out[b], oo, f"budget 4096 decode vs oracle b={b}")
