@@ -195,11 +195,13 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
   uint64_t* kv_empty = bars + 2 + NSTAGE;   // [NSTAGE]
   uint64_t* s_full = bars + 2 + 2 * NSTAGE; // [2]
   uint64_t* p_full = s_full + 2;            // [2]
+  // [2]: P V number j completes pv_done[j & 1], so a waiter for P V j needs
+  // only P V j - 2 to have completed (not j - 1) for the parity to be exact
   uint64_t* pv_done = s_full + 4;
-  uint64_t* o_full = s_full + 5;
-  uint64_t* o_empty = s_full + 6;
-  uint64_t* mma_done = s_full + 7;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 8);
+  uint64_t* o_full = s_full + 6;
+  uint64_t* o_empty = s_full + 7;
+  uint64_t* mma_done = s_full + 8;           // [2]: the S and the P V issuer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 10);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -212,10 +214,12 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
     mbar_init(q_empty, 1);
     for (int s = 0; s < NSTAGE; ++s) { mbar_init(&kv_full[s], LOADERS); mbar_init(&kv_empty[s], 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(&s_full[b], 1); mbar_init(&p_full[b], 2); }
-    mbar_init(pv_done, 1);
+    mbar_init(&pv_done[0], 1);
+    mbar_init(&pv_done[1], 1);
     mbar_init(o_full, 1);
     mbar_init(o_empty, 2);
-    mbar_init(mma_done, 1);
+    mbar_init(&mma_done[0], 1);
+    mbar_init(&mma_done[1], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -337,9 +341,15 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
       ++items_done;
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
-  } else if (warp == W_MMA) {
+  } else if (warp == W_MMA || warp == W_MMA + 1) {
     // -------------------------------------------------------------------- MMA
+    // Two issuing threads: warp W_MMA issues every S, warp W_MMA + 1 every
+    // P V, so a P V whose P is ready is not held behind the issue of the next
+    // S (which waits for its K / V and for room in the tensor pipe); the
+    // stage a P V frees is refilled that much sooner.  S(i) overwrites the
+    // TMEM buffer P(i - 2) was read from, so it waits for P V(i - 2).
     if (lane == 0) {
+      const bool s_role = warp == W_MMA;
       constexpr uint32_t idesc_s = umma_idesc_bf16_f32(128, KT);
       constexpr uint32_t idesc_pv = umma_idesc_bf16_f32(128, 256) | (1u << 16);   // B (V) MN-major
       int stage = 0;
@@ -351,51 +361,62 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
         const Item<DEC> it(a, w);
         const int n_tiles = it.n_tiles;
         if (n_tiles == 0) continue;
-        if (!mbar_wait(q_full, items_done & 1, abort_flag, a.err)) { ok = false; break; }
-        tc_fence_after();
-        int pv_stage = stage;           // stage of the tile whose PV is next
-        auto issue_pv = [&](int j, bool last) -> bool {
-          const uint32_t b = p_count & 1;
-          if (!mbar_wait(&p_full[b], (p_count >> 1) & 1, abort_flag, a.err)) return false;
-          if (j == 0 && items_done > 0 && !mbar_wait(o_empty, (items_done - 1) & 1, abort_flag, a.err)) return false;
+        if (s_role) {
+          if (!mbar_wait(q_full, items_done & 1, abort_flag, a.err)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t v_base = smem_u32(smem + OFF_STAGE + pv_stage * STAGE_BYTES + KV_BYTES);
+          for (int i = 0; i < n_tiles; ++i) {
+            if (!mbar_wait(&kv_full[stage], fphase, abort_flag, a.err)) { ok = false; break; }
+            // P V number s_count - 2 read the buffer S(i) writes; P V s_count - 4
+            // has completed (waited before S(i - 2)) and P V s_count cannot
+            // yet (it needs this S), so the parity of pv_done[(s_count - 2) & 1]
+            // is exact even when P V s_count - 1 already completed
+            if (s_count >= 2) {
+              const uint32_t g = s_count - 2;
+              if (!mbar_wait(&pv_done[g & 1], (g >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
+            }
+            fence_proxy_async();    // the stage was written by cp.async; the MMA reads it
+            tc_fence_after();
+            const uint32_t b = s_count & 1;
+            const uint32_t k_base = smem_u32(smem + OFF_STAGE + stage * STAGE_BYTES);
 #pragma unroll
-          for (int ks = 0; ks < KT / 16; ++ks) {
-            const uint64_t bd = umma_desc_mn_sw128(v_base + ks * 2048, CHUNK_KV, 1024);
-            umma_ts_bf16(tmem + TM_O, tmem + TM_S0 + 64 * b + 8 * ks, bd, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
+            for (int ks = 0; ks < 16; ++ks) {
+              const uint32_t c = ks >> 2, koff = (ks & 3) * 32;
+              const uint64_t ad = umma_desc_k_sw128(q_base + c * CHUNK_Q + koff);
+              const uint64_t bd = umma_desc_k_sw128(k_base + c * CHUNK_KV + koff);
+              umma_bf16(tmem + TM_S0 + 64 * b, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+            }
+            tc_commit(&s_full[b]);
+            if (i == n_tiles - 1) tc_commit(q_empty);
+            ++s_count;
+            if (++stage == NSTAGE) { stage = 0; fphase ^= 1; }
           }
-          tc_commit(&kv_empty[pv_stage]);
-          tc_commit(pv_done);
-          if (last) tc_commit(o_full);
-          ++p_count;
-          if (++pv_stage == NSTAGE) pv_stage = 0;
-          return true;
-        };
-        for (int i = 0; i < n_tiles && ok; ++i) {
-          if (!mbar_wait(&kv_full[stage], fphase, abort_flag, a.err)) { ok = false; break; }
-          fence_proxy_async();    // the stage was written by cp.async; the MMA reads it
-          tc_fence_after();
-          const uint32_t b = s_count & 1;
-          const uint32_t k_base = smem_u32(smem + OFF_STAGE + stage * STAGE_BYTES);
+        } else {
+          for (int j = 0; j < n_tiles; ++j) {
+            const uint32_t b = p_count & 1;
+            if (!mbar_wait(&p_full[b], (p_count >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
+            if (j == 0 && items_done > 0 && !mbar_wait(o_empty, (items_done - 1) & 1, abort_flag, a.err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t v_base = smem_u32(smem + OFF_STAGE + stage * STAGE_BYTES + KV_BYTES);
 #pragma unroll
-          for (int ks = 0; ks < 16; ++ks) {
-            const uint32_t c = ks >> 2, koff = (ks & 3) * 32;
-            const uint64_t ad = umma_desc_k_sw128(q_base + c * CHUNK_Q + koff);
-            const uint64_t bd = umma_desc_k_sw128(k_base + c * CHUNK_KV + koff);
-            umma_bf16(tmem + TM_S0 + 64 * b, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+            for (int ks = 0; ks < KT / 16; ++ks) {
+              const uint64_t bd = umma_desc_mn_sw128(v_base + ks * 2048, CHUNK_KV, 1024);
+              umma_ts_bf16(tmem + TM_O, tmem + TM_S0 + 64 * b + 8 * ks, bd, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
+            }
+            tc_commit(&kv_empty[stage]);
+            tc_commit(&pv_done[p_count & 1]);
+            if (j == n_tiles - 1) tc_commit(o_full);
+            ++p_count;
+            if (++stage == NSTAGE) stage = 0;
           }
-          tc_commit(&s_full[b]);
-          if (i == n_tiles - 1) tc_commit(q_empty);
-          ++s_count;
-          if (++stage == NSTAGE) { stage = 0; fphase ^= 1; }
-          if (i >= 1 && !issue_pv(i - 1, false)) { ok = false; break; }
         }
-        if (ok && !issue_pv(n_tiles - 1, true)) ok = false;
         ++items_done;
       }
-      tc_commit(mma_done);
-      mbar_wait(mma_done, 0, abort_flag, a.err);
+      uint64_t* done = &mma_done[s_role ? 0 : 1];
+      tc_commit(done);
+      mbar_wait(done, 0, abort_flag, a.err);
     }
   } else if (warp == W_SOFT || warp == W_SOFT + 1) {
     // ---------------------------------------------------------------- softmax
@@ -452,7 +473,11 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
         mt = fmaxf(mt, s[63]);
         mt = row_ok ? mt * a.scale_log2 : -FLT_MAX;   // raw max, then the (positive) scale
         if (i >= 1) {   // PV(i-1) complete before O may be rescaled (and keeps phases in step)
-          if (!__all_sync(0xffffffffu, mbar_wait(pv_done, pv_count & 1, abort_flag, a.err))) { ok = false; break; }
+          if (!__all_sync(0xffffffffu,
+                          mbar_wait(&pv_done[pv_count & 1], (pv_count >> 1) & 1, abort_flag, a.err))) {
+            ok = false;
+            break;
+          }
           ++pv_count;
         }
         const bool need = mt > m_run + 8.f;
