@@ -424,7 +424,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
     const bool row_ok = r < QR;
     const int tok = row_ok ? r / 12 : 0, hh = row_ok ? r % 12 : 0;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-    uint32_t items_done = 0, s_count = 0, pv_count = 0;
+    uint32_t items_done = 0, s_count = 0, pv_seq = 0;
     bool ok = true;
     for (int64_t w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
       const Item<DEC> it(a, w);
@@ -472,14 +472,6 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
         for (int n = 0; n < 63; n += 3) mt = fmaxf(mt, max3f(s[n], s[n + 1], s[n + 2]));
         mt = fmaxf(mt, s[63]);
         mt = row_ok ? mt * a.scale_log2 : -FLT_MAX;   // raw max, then the (positive) scale
-        if (i >= 1) {   // PV(i-1) complete before O may be rescaled (and keeps phases in step)
-          if (!__all_sync(0xffffffffu,
-                          mbar_wait(&pv_done[pv_count & 1], (pv_count >> 1) & 1, abort_flag, a.err))) {
-            ok = false;
-            break;
-          }
-          ++pv_count;
-        }
         const bool need = mt > m_run + 8.f;
         if (__any_sync(0xffffffffu, need)) {
           const float m_new = need ? fmaxf(m_run, mt) : m_run;
@@ -487,6 +479,16 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
           l_run *= corr;
           m_run = m_new;
           if (i >= 1) {
+            // O may be rescaled only once P V(i - 1), number g = pv_seq + i - 1,
+            // has accumulated into it.  S(i) has completed and was issued after
+            // P V(i - 2) completed, and P V(i + 1) cannot have (it needs P(i + 1)),
+            // so the parity of pv_done[g & 1] is exact.  Only this rare path
+            // waits, so the softmax of tile i overlaps P V(i - 1).
+            const uint32_t g = pv_seq + (uint32_t)i - 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[g & 1], (g >> 1) & 1, abort_flag, a.err))) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
 #pragma unroll 1
             for (int c = 0; c < 8; ++c) {
@@ -525,7 +527,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
       if (!ok) break;
       // item end: O / l -> bf16
       if (!__all_sync(0xffffffffu, mbar_wait(o_full, items_done & 1, abort_flag, a.err))) { ok = false; break; }
-      ++pv_count;   // the last PV of the item also completed
+      pv_seq += (uint32_t)n_tiles;   // every P V of the item has completed
       tc_fence_after();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
       const bool write = row_ok && (DEC || (t < a.T && t >= a.q_tok0));
