@@ -253,37 +253,50 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
   } else {
     // ----------------------------------------------------------- epilogue
     // Two groups of 8 warps, one per TMEM accumulator: group hf drains half hf
-    // of every unit while the tensor core fills the other half.
+    // of every unit while the tensor core fills the other half.  Token, key and
+    // block numbers fit in 32 bits (T <= 2^24), so the per-unit bookkeeping is
+    // 32-bit; only the score addresses are formed in 64 bits, once per tile.
     const int e = warp - 2;                 // 0..15
     const int hf = e >> 3;                  // accumulator this warp drains
     const int quad = warp & 3;              // TMEM lanes 32*quad .. +31
     const int cgrp = (e >> 2) & 1;          // column group: tokens [32*cgrp, +32) of a half
     const uint32_t lane_addr = (uint32_t)(32 * quad) << 16;
+    const float* wrow = sW + (64 * hf + 32 * cgrp) * 4;
+    const bool la = (lane & 1) != 0, lb = (lane & 2) != 0, lc = (lane & 4) != 0;
+    // query blocks (after the first of the warp's 8) this lane ends up holding:
+    // qs, qs + 1 after the key-block butterfly, qs_seg after the segment step
+    const int qs = (la ? 4 : 0) + (lb ? 2 : 0);
+    const int qs_seg = qs + (lc ? 1 : 0);
+    const int qb0 = (int)qb_begin, qe = (int)qb_end;
     Iter it; it.begin(&sch, u0, u1);
     uint32_t qcount = 0;
     uint32_t acc_use = 0;
-    const float* wrow = sW + (64 * hf + 32 * cgrp) * 4;
+    int t_first = 0;              // first token of this thread's columns (per tile)
+    int qbf = 0;                  // first query block of those columns (per tile)
+    float* s_rows = nullptr;      // score row of query block qbf (+ qs unless MEAN)
+    float* g_row = nullptr;       // segment-maxima row of query block qbf + qs_seg
     for (; it.valid(); it.next()) {
       if (it.first_of_tile(u0)) {
         if (!__all_sync(0xffffffffu, mbar_wait(qfull, qcount & 1, abort_flag, err))) break;
         ++qcount;
+        t_first = (int)(sch.T0 + QT * it.tile) + 64 * hf + 32 * cgrp;
+        qbf = qb0 + (QT / 4) * (int)it.tile + 16 * hf + 8 * cgrp;
+        s_rows = S + (int64_t)(qbf - qb0 + (MEAN ? 0 : qs)) * ld;
+        if (segmax != nullptr) g_row = segmax + (int64_t)(qbf - qb0 + qs_seg) * ld_seg;
       }
-      const int64_t t_tile = sch.T0 + QT * it.tile;
-      const int64_t qb_tile = qb_begin + (QT / 4) * it.tile;
       // this thread's TMEM lane: one key (token-pair max) or one key block (mean pool);
       // j is the first token it stands for, so "j <= t" is the causal test in both
-      const int64_t row = KT * it.kt + 32 * quad + lane;
-      const int64_t j = MEAN ? 4 * row : row;
-      const int64_t kb = MEAN ? row : row >> 2;
+      const int key0 = KT * (int)it.kt + 32 * quad;   // the warp's first TMEM row
+      const int row = key0 + lane;
+      const int j = MEAN ? 4 * row : row;
+      const int kb = MEAN ? row : row >> 2;
       if (!__all_sync(0xffffffffu, mbar_wait(&accfull[hf], acc_use & 1, abort_flag, err))) break;
       ++acc_use;
       tc_fence_after();
-      const int64_t t_first = t_tile + 64 * hf + 32 * cgrp;  // first token of this thread's columns
-      const int64_t qb_first = qb_tile + 16 * hf + 8 * cgrp;
-      const int64_t kt_last_key = MEAN ? 4 * (KT * it.kt + KT - 1) : KT * it.kt + KT - 1;
+      const int kt_last_key = MEAN ? 4 * (KT * (int)it.kt + KT - 1) : KT * (int)it.kt + KT - 1;
       // skip when every key block of this warp lies after every query block of its columns
-      const int64_t warp_first_key = MEAN ? 4 * (KT * it.kt + 32 * quad) : KT * it.kt + 32 * quad;
-      const bool live = warp_first_key <= (t_first + 31) && qb_first < qb_end;
+      const int warp_first_key = MEAN ? 4 * key0 : key0;
+      const bool live = warp_first_key <= t_first + 31 && qbf < qe;
       if (live) {
         // The causal test is needed only where the key tile reaches past the
         // first token of this thread's columns; the drain is compiled twice so
@@ -294,7 +307,7 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
           // key position relative to the first column token: where MASKED the
           // key tile ends after t_first and the warp's first key is at most
           // t_first + 31, so -512 < jd < 160
-          const int jd = MASKED ? (int)(j - t_first) : 0;
+          const int jd = MASKED ? j - t_first : 0;
           float m[8];
           // 8 tokens (32 columns) of this key's row -> the maxima of query blocks 2c, 2c+1
           auto chunk = [&](const float (&v)[32], int c) {
@@ -347,18 +360,17 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
           chunk(vb, 3);
           if constexpr (MEAN) {
             // one key block per lane: the 8 block maxima are the scores
-            // S(qb_first + b, kb), stored by the 32 lanes as 32 consecutive floats
-            float* srow = S + (qb_first - qb_begin) * ld + kb;
-            const int nb = (int)(qb_end - qb_first < 8 ? qb_end - qb_first : 8);
+            // S(qbf + b, kb), stored by the 32 lanes as 32 consecutive floats
+            float* srow = s_rows + kb;
+            const int nb = qe - qbf < 8 ? qe - qbf : 8;
   #pragma unroll
             for (int b = 0; b < 8; ++b) {
-              if (b < nb && kb <= qb_first + b) srow[b * ld] = m[b] * scale;
+              if (b < nb && kb <= qbf + b) srow[b * ld] = m[b] * scale;
             }
             if (segmax != nullptr) {
               // segment maxima over 8 key blocks = 8 lanes (bits 0..2): three
               // transposing steps leave lane (a, b, c) of each 8-lane group with
-              // the maximum of query block qb_first + 4 a + 2 b + c
-              const bool la = (lane & 1) != 0, lb = (lane & 2) != 0, lc = (lane & 4) != 0;
+              // the maximum of query block qbf + 4 a + 2 b + c
               float n4[4], n2[2];
   #pragma unroll
               for (int i = 0; i < 4; ++i)
@@ -367,16 +379,15 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
               for (int i = 0; i < 2; ++i)
                 n2[i] = fmaxf(lb ? n4[i + 2] : n4[i], __shfl_xor_sync(0xffffffffu, lb ? n4[i] : n4[i + 2], 2));
               const float sm = fmaxf(lc ? n2[1] : n2[0], __shfl_xor_sync(0xffffffffu, lc ? n2[0] : n2[1], 4));
-              const int64_t seg = (KT * it.kt + 32 * quad + (lane & ~7)) >> 3;
-              const int64_t qb = qb_first + (la ? 4 : 0) + (lb ? 2 : 0) + (lc ? 1 : 0);
+              const int seg = (key0 + (lane & ~7)) >> 3;
+              const int qb = qbf + qs_seg;
               // only segments starting at or before the row's own block: seg <= qb / 8 < ld_seg
-              if (qb < qb_end && seg <= (qb >> 3)) segmax[(qb - qb_begin) * ld_seg + seg] = sm * scale;
+              if (qb < qe && seg <= (qb >> 3)) g_row[seg] = sm * scale;
             }
           } else {
             // max over the 4 keys of the key block (lanes 4k .. 4k+3) as a transposing
             // butterfly: after the two steps lane (a = bit 0, b = bit 1) holds the
             // maxima of query blocks 4a + 2b and 4a + 2b + 1.
-            const bool la = (lane & 1) != 0, lb = (lane & 2) != 0;
             float n4[4];
     #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -390,8 +401,8 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
               const float send = lb ? n4[i] : n4[i + 2];
               const float keep = lb ? n4[i + 2] : n4[i];
               val[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
-              const int64_t qb = qb_first + (la ? 4 : 0) + (lb ? 2 : 0) + i;
-              if (qb < qb_end && kb <= qb) S[(qb - qb_begin) * ld + kb] = val[i] * scale;
+              const int qb = qbf + qs + i;
+              if (qb < qe && kb <= qb) s_rows[i * ld + kb] = val[i] * scale;
             }
             if (segmax != nullptr) {
               // segment maxima: max over the 8 key blocks of this warp's 32 keys
@@ -399,15 +410,14 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
               // query block (4 a + 2 b + c0), then two plain steps; lanes 0..7 hold
               // the 8 query blocks.  Key blocks after a query block were scored as
               // 0 and scores are >= 0, so they do not raise a maximum.
-              const bool lc = (lane & 4) != 0;
               float sm = fmaxf(lc ? val[1] : val[0], __shfl_xor_sync(0xffffffffu, lc ? val[0] : val[1], 4));
               sm = fmaxf(sm, __shfl_xor_sync(0xffffffffu, sm, 8));
               sm = fmaxf(sm, __shfl_xor_sync(0xffffffffu, sm, 16));
               if (lane < 8) {
-                const int64_t seg = (KT * it.kt + 32 * quad) >> 5;
-                const int64_t qb = qb_first + (la ? 4 : 0) + (lb ? 2 : 0) + (lc ? 1 : 0);
+                const int seg = key0 >> 5;
+                const int qb = qbf + qs_seg;
                 // only segments starting at or before the row's own block: seg <= qb / 8 < ld_seg
-                if (qb < qb_end && seg <= (qb >> 3)) segmax[(qb - qb_begin) * ld_seg + seg] = sm * scale;
+                if (qb < qe && seg <= (qb >> 3)) g_row[seg] = sm * scale;
               }
             }
           }
