@@ -303,6 +303,12 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
       // latency stays off the issue path.
       constexpr int KPT = 64 / LWARPS;
       const int w4 = (tid >> 5) & 3, c32 = tid & 31, k0 = KPT * (tid >> 7);
+      // key positions fit in 32 bits (sequences are at most 2^24 tokens); a
+      // key row holds both KV heads (512 elements), so the source of key j is
+      // this lane's chunk of head g plus j * 512 elements, one wide multiply-add
+      const int t_last32 = (int)t_last;
+      const uint16_t* k_lane = it.kb + g * 256 + c32 * 8;
+      const uint16_t* v_lane = it.vb + g * 256 + c32 * 8;
       int32_t kbv[KPT], kbn[KPT], kbm[KPT];
       auto load_idx = [&](int ti, int32_t (&dst)[KPT]) {
 #pragma unroll
@@ -322,12 +328,12 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
         for (int kk = 0; kk < KPT; ++kk) {
           const int k = k0 + kk;
           const int n = 4 * k + w4;
-          const int64_t j = 4 * (int64_t)kbv[kk] + w4;
-          const bool valid = kbv[kk] >= 0 && j <= t_last;
-          const int64_t off = valid ? (j * 2 + g) * 256 + c32 * 8 : 0;
+          const int j = 4 * kbv[kk] + w4;
+          const bool valid = kbv[kk] >= 0 && j <= t_last32;
+          const size_t off = valid ? (size_t)(uint32_t)j * 512u : 0;
           const uint32_t dst = dst0 + swz128(n, c32 & 7);
-          cp_async16(dst, it.kb + off, valid);
-          cp_async16(dst + KV_BYTES, it.vb + off, valid);
+          cp_async16(dst, k_lane + off, valid);
+          cp_async16(dst + KV_BYTES, v_lane + off, valid);
         }
         // this thread's arrival on the stage's barrier fires when all its
         // copies so far have landed: no blocking wait, all stages in flight
