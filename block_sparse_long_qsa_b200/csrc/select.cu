@@ -185,16 +185,28 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
       // 2'. the segments whose max reaches tau0 (listed in the sample buffer) ...
       if (tid == 0) sm.misc[5] = 0;
       __syncthreads();
-      for (int64_t b0 = 0; b0 < fs; b0 += blockDim.x) {
-        const int64_t sgi = b0 + tid;
-        const bool pass = sgi < fs && key_of(mrow[sgi]) >= tau0;
-        const uint32_t ball = __ballot_sync(0xffffffffu, pass);
-        if (ball) {
-          uint32_t base = 0;
-          if (lane == 0) base = atomicAdd(&sm.misc[5], (uint32_t)__popc(ball));
-          base = __shfl_sync(0xffffffffu, base, 0);
-          const uint32_t pos = base + __popc(ball & ((1u << lane) - 1u));
-          if (pass && pos < (uint32_t)NSAMPLE) sm.sample[pos] = (uint32_t)sgi;
+      // SEG_UNROLL loads per thread in flight before any is tested: the scan is
+      // one row of up to 32K maxima per CTA, bound by load latency otherwise
+      constexpr int SEG_UNROLL = 8;
+      for (int64_t b0 = 0; b0 < fs; b0 += (int64_t)blockDim.x * SEG_UNROLL) {
+        uint32_t kv[SEG_UNROLL];
+#pragma unroll
+        for (int u = 0; u < SEG_UNROLL; ++u) {
+          const int64_t sgi = b0 + (int64_t)u * blockDim.x + tid;
+          kv[u] = sgi < fs ? key_of(__ldcs(mrow + sgi)) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < SEG_UNROLL; ++u) {
+          const int64_t sgi = b0 + (int64_t)u * blockDim.x + tid;
+          const bool pass = sgi < fs && kv[u] >= tau0;
+          const uint32_t ball = __ballot_sync(0xffffffffu, pass);
+          if (ball) {
+            uint32_t base = 0;
+            if (lane == 0) base = atomicAdd(&sm.misc[5], (uint32_t)__popc(ball));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            const uint32_t pos = base + __popc(ball & ((1u << lane) - 1u));
+            if (pass && pos < (uint32_t)NSAMPLE) sm.sample[pos] = (uint32_t)sgi;
+          }
         }
       }
       __syncthreads();
@@ -204,25 +216,38 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
       } else {
         // ... and their scores >= tau0 (two 16-byte loads per segment), then the tail
         const float4* row4 = reinterpret_cast<const float4*>(row);
-        for (int64_t b0 = 0; b0 < 2 * nsl; b0 += blockDim.x) {
-          const int64_t e2 = b0 + tid;
-          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-          int64_t i0 = 0;
-          if (e2 < 2 * nsl) {
-            i0 = 8 * (int64_t)sm.sample[e2 >> 1] + 4 * (e2 & 1);
-            v = __ldcs(row4 + (i0 >> 2));
-          }
-          const float vals[4] = {v.x, v.y, v.z, v.w};
+        constexpr int CAND_UNROLL = 4;
+        for (int64_t b0 = 0; b0 < 2 * nsl; b0 += (int64_t)blockDim.x * CAND_UNROLL) {
+          float4 v[CAND_UNROLL];
+          int64_t i0[CAND_UNROLL];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const bool pass = e2 < 2 * nsl && key_of(vals[q]) >= tau0;
-            const uint32_t ball = __ballot_sync(0xffffffffu, pass);
-            if (ball) {
-              uint32_t base = 0;
-              if (lane == 0) base = atomicAdd(&sm.misc[2], (uint32_t)__popc(ball));
-              base = __shfl_sync(0xffffffffu, base, 0);
-              const uint32_t pos = base + __popc(ball & ((1u << lane) - 1u));
-              if (pass && pos < (uint32_t)cap) { sm.ckey[pos] = key_of(vals[q]); sm.cidx[pos] = (int32_t)(i0 + q); }
+          for (int u = 0; u < CAND_UNROLL; ++u) {
+            const int64_t e2 = b0 + (int64_t)u * blockDim.x + tid;
+            v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            i0[u] = 0;
+            if (e2 < 2 * nsl) {
+              i0[u] = 8 * (int64_t)sm.sample[e2 >> 1] + 4 * (e2 & 1);
+              v[u] = __ldcs(row4 + (i0[u] >> 2));
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < CAND_UNROLL; ++u) {
+            const int64_t e2 = b0 + (int64_t)u * blockDim.x + tid;
+            const float vals[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const bool pass = e2 < 2 * nsl && key_of(vals[q]) >= tau0;
+              const uint32_t ball = __ballot_sync(0xffffffffu, pass);
+              if (ball) {
+                uint32_t base = 0;
+                if (lane == 0) base = atomicAdd(&sm.misc[2], (uint32_t)__popc(ball));
+                base = __shfl_sync(0xffffffffu, base, 0);
+                const uint32_t pos = base + __popc(ball & ((1u << lane) - 1u));
+                if (pass && pos < (uint32_t)cap) {
+                  sm.ckey[pos] = key_of(vals[q]);
+                  sm.cidx[pos] = (int32_t)(i0[u] + q);
+                }
+              }
             }
           }
         }
@@ -353,6 +378,36 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
     if (tid == 0) { sm.out[k] = (int32_t)(qb - 1); sm.out[k + 1] = (int32_t)qb; }
     for (int i = budget + tid; i < P; i += blockDim.x) sm.out[i] = INT_MAX;
     __syncthreads();
+    if (P <= THREADS) {
+      // one entry per thread: compare-exchange steps with a partner in the
+      // same warp by shuffle, wider ones through two alternating shared
+      // buffers (sm.out and the spent candidate keys), one barrier each
+      int32_t v = tid < P ? sm.out[tid] : INT_MAX;
+      int32_t* const buf0 = sm.out;
+      int32_t* const buf1 = reinterpret_cast<int32_t*>(sm.ckey);
+      int nb = 0;
+      for (int size = 2; size <= P; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          int32_t o;
+          if (stride >= 32) {
+            nb ^= 1;
+            int32_t* const b = nb ? buf1 : buf0;
+            if (tid < P) b[tid] = v;
+            __syncthreads();
+            o = tid < P ? b[tid ^ stride] : v;
+          } else {
+            o = __shfl_xor_sync(0xffffffffu, v, stride);
+          }
+          // the lower slot of an ascending pair keeps the minimum
+          const bool up = (tid & size) == 0, lower = (tid & stride) == 0;
+          v = (lower == up) ? min(v, o) : max(v, o);
+        }
+      }
+      if (tid < budget) srow[tid] = v;
+      if (tid == 0) cnt[r] = budget;
+      __syncthreads();
+      continue;
+    }
     for (int size = 2; size <= P; size <<= 1) {
       for (int stride = size >> 1; stride > 0; stride >>= 1) {
         for (int i = tid; i < P / 2; i += blockDim.x) {
