@@ -10,13 +10,15 @@
 // Work item = (query block, KV head): 48 query rows (4 tokens x 12 heads)
 // against up to budget x 4 keys.  Persistent CTAs (one per SM) walk the items.
 //   * warps 0-7 (loaders): Q tile with RoPE applied on the fly, then the
-//     selected K and V rows, 64 keys (16 blocks) per stage, gathered with
+//     selected K and V rows, 64 keys (16 blocks) per tile, gathered with
 //     cp.async into the canonical 128-byte-swizzled K-major layout (8 KB per
-//     64-dim chunk); 3 stages of 64 KB.
-//   * warp 10 (MMA, one thread): S = Q K^T with M = 128 (rows 48..127 are
-//     padding whose results are never read), N = 64, K = 256 into one of two
-//     TMEM S buffers; O += P V with P taken from TMEM (A operand) and V as an
-//     MN-major shared-memory operand, M = 128, N = 256, fp32 in TMEM.
+//     64-dim chunk); a ring of three 32 KB K slots and one of three V slots.
+//   * warp 10 (one thread): S = Q K^T with M = 128 (rows 48..127 are
+//     padding whose results are never read), N = 64, K = 256 into one of
+//     three TMEM S buffers; it frees the K slot.  Warp 11 (one thread):
+//     O += P V with P taken from TMEM (A operand) and V as an MN-major
+//     shared-memory operand, M = 128, N = 256, fp32 in TMEM; it frees the
+//     V slot.
 //   * warps 8-9 (softmax): one thread per query row (TMEM lanes 0..63):
 //     mask, running max in base 2 (raised only when a tile's max exceeds it by
 //     more than 8, so the O rescale is rare), exp2, row sum, P packed to bf16
@@ -31,10 +33,9 @@
 namespace qsa {
 namespace {
 
-constexpr int KT = 64;                              // keys per stage
-constexpr int NSTAGE = 3;
-// 8 loader warps issue a 64 KB stage in about half the time 4 take (the
-// gathers are issue-bound between stage releases): 5 % faster at 1M tokens.
+constexpr int KT = 64;                              // keys per tile
+// 8 loader warps issue a 64 KB tile in about half the time 4 take (the
+// gathers are issue-bound between slot releases): 5 % faster at 1M tokens.
 constexpr int LWARPS = 8;                            // loader warps (4 or 8)
 constexpr int LOADERS = 32 * LWARPS;
 constexpr int W_SOFT = LWARPS;                       // softmax warps W_SOFT, W_SOFT + 1
@@ -44,13 +45,21 @@ constexpr uint32_t QROWS = 48;
 constexpr uint32_t CHUNK_Q = QROWS * 128;           // 6 KB: 48 rows x 64 dims
 constexpr uint32_t CHUNK_KV = KT * 128;             // 8 KB: 64 keys x 64 dims
 constexpr uint32_t KV_BYTES = 4 * CHUNK_KV;         // 32 KB per K (or V) tile
-constexpr uint32_t STAGE_BYTES = 2 * KV_BYTES;      // K + V
 constexpr uint32_t OFF_STAGE = 32768;               // Q region (24 KB) padded to 32 KB
-constexpr uint32_t OFF_BAR = OFF_STAGE + NSTAGE * STAGE_BYTES;
+// Separate K and V rings in the same 192 KB: a K slot is freed once S has
+// read it, a V slot once P V has, so the next K tile lands while the
+// softmax and P V of the current one run.  Three S / P buffers in TMEM let
+// S run a tile further ahead of P V.  (2 K + 4 V slots, 4 K + 2 V slots or
+// four S buffers were no faster; one ring of three K + V stages with two S
+// buffers was 4 % slower at 1M tokens.)
+constexpr int NK = 3, NV = 3;
+constexpr int NSB = 3;                               // S / P buffers in TMEM
+constexpr uint32_t OFF_V = OFF_STAGE + NK * KV_BYTES;
+constexpr uint32_t OFF_BAR = OFF_V + NV * KV_BYTES;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
 static_assert(SMEM_BYTES <= 232448, "attention smem");
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TM_S0 = 0, TM_O = 256;           // S buffers at columns 0 and 64; O at 256
+constexpr uint32_t TM_S0 = 0, TM_O = 256;           // S buffers at columns 0, 64, 128; O at 256
 
 __device__ __forceinline__ uint32_t swz128(uint32_t row, uint32_t c16) {
   return row * 128u + ((c16 ^ (row & 7u)) << 4);
@@ -191,17 +200,18 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* kv_full = bars + 2;             // [NSTAGE]
-  uint64_t* kv_empty = bars + 2 + NSTAGE;   // [NSTAGE]
-  uint64_t* s_full = bars + 2 + 2 * NSTAGE; // [2]
-  uint64_t* p_full = s_full + 2;            // [2]
-  // [2]: P V number j completes pv_done[j & 1], so a waiter for P V j needs
-  // only P V j - 2 to have completed (not j - 1) for the parity to be exact
-  uint64_t* pv_done = s_full + 4;
-  uint64_t* o_full = s_full + 6;
-  uint64_t* o_empty = s_full + 7;
-  uint64_t* mma_done = s_full + 8;           // [2]: the S and the P V issuer
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 10);
+  uint64_t* k_full = bars + 2;              // [NK]
+  uint64_t* k_empty = k_full + NK;          // [NK]
+  uint64_t* v_full = k_empty + NK;          // [NV]
+  uint64_t* v_empty = v_full + NV;          // [NV]
+  uint64_t* s_full = v_empty + NV;          // [NSB]
+  uint64_t* p_full = s_full + NSB;          // [NSB]
+  // [NSB]: P V number j completes pv_done[j % NSB]
+  uint64_t* pv_done = p_full + NSB;
+  uint64_t* o_full = pv_done + NSB;
+  uint64_t* o_empty = o_full + 1;
+  uint64_t* mma_done = o_empty + 1;          // [2]: the S and the P V issuer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -212,10 +222,9 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
   if (tid == 0) {
     mbar_init(q_full, LOADERS);
     mbar_init(q_empty, 1);
-    for (int s = 0; s < NSTAGE; ++s) { mbar_init(&kv_full[s], LOADERS); mbar_init(&kv_empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&s_full[b], 1); mbar_init(&p_full[b], 2); }
-    mbar_init(&pv_done[0], 1);
-    mbar_init(&pv_done[1], 1);
+    for (int s = 0; s < NK; ++s) { mbar_init(&k_full[s], LOADERS); mbar_init(&k_empty[s], 1); }
+    for (int s = 0; s < NV; ++s) { mbar_init(&v_full[s], LOADERS); mbar_init(&v_empty[s], 1); }
+    for (int b = 0; b < NSB; ++b) { mbar_init(&s_full[b], 1); mbar_init(&p_full[b], 2); mbar_init(&pv_done[b], 1); }
     mbar_init(o_full, 1);
     mbar_init(o_empty, 2);
     mbar_init(&mma_done[0], 1);
@@ -232,8 +241,8 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
 
   if (warp < LWARPS) {
     // ---------------------------------------------------------------- loaders
-    int stage = 0;
-    uint32_t ephase = 1;
+    int kst = 0, vst = 0;
+    uint32_t keph = 1, veph = 1;
     uint32_t items_done = 0;
     bool ok = true;
     for (int64_t w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
@@ -299,7 +308,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
       // each of its KPT blocks of a tile (blocks k0 .. k0 + KPT - 1: warps
       // 0-3 the first 8 of the 16, warps 4-7 the last 8), for K and for V:
       // key slot n = 4k + w % 4.  The block indices of tiles i + 1 and i + 2
-      // are loaded while tile i waits for its stage, so the index loads'
+      // are loaded while tile i waits for its slots, so the index loads'
       // latency stays off the issue path.
       constexpr int KPT = 64 / LWARPS;
       const int w4 = (tid >> 5) & 3, c32 = tid & 31, k0 = KPT * (tid >> 7);
@@ -321,25 +330,37 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
       if (n_tiles > 1) load_idx(1, kbn);
       for (int i = 0; i < n_tiles; ++i) {
         if (i + 2 < n_tiles) load_idx(i + 2, kbm);
-        if (!mbar_wait(&kv_empty[stage], ephase, abort_flag, a.err)) { ok = false; break; }
-        const uint32_t base = smem_u32(smem + OFF_STAGE + stage * STAGE_BYTES);
-        const uint32_t dst0 = base + (c32 >> 3) * CHUNK_KV;
+        if (!mbar_wait(&k_empty[kst], keph, abort_flag, a.err)) { ok = false; break; }
+        size_t off[KPT];
+        bool valid[KPT];
+        {
+          const uint32_t dst0 = smem_u32(smem + OFF_STAGE + kst * KV_BYTES) + (c32 >> 3) * CHUNK_KV;
 #pragma unroll
-        for (int kk = 0; kk < KPT; ++kk) {
-          const int k = k0 + kk;
-          const int n = 4 * k + w4;
-          const int j = 4 * kbv[kk] + w4;
-          const bool valid = kbv[kk] >= 0 && j <= t_last32;
-          const size_t off = valid ? (size_t)(uint32_t)j * 512u : 0;
-          const uint32_t dst = dst0 + swz128(n, c32 & 7);
-          cp_async16(dst, k_lane + off, valid);
-          cp_async16(dst + KV_BYTES, v_lane + off, valid);
+          for (int kk = 0; kk < KPT; ++kk) {
+            const int n = 4 * (k0 + kk) + w4;
+            const int j = 4 * kbv[kk] + w4;
+            valid[kk] = kbv[kk] >= 0 && j <= t_last32;
+            off[kk] = valid[kk] ? (size_t)(uint32_t)j * 512u : 0;
+            cp_async16(dst0 + swz128(n, c32 & 7), k_lane + off[kk], valid[kk]);
+          }
         }
-        // this thread's arrival on the stage's barrier fires when all its
-        // copies so far have landed: no blocking wait, all stages in flight
-        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&kv_full[stage]))
+        // this thread's arrival fires when all its copies so far have landed:
+        // no blocking wait, every slot in flight
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&k_full[kst]))
                      : "memory");
-        if (++stage == NSTAGE) { stage = 0; ephase ^= 1; }
+        if (!mbar_wait(&v_empty[vst], veph, abort_flag, a.err)) { ok = false; break; }
+        {
+          const uint32_t dst0 = smem_u32(smem + OFF_V + vst * KV_BYTES) + (c32 >> 3) * CHUNK_KV;
+#pragma unroll
+          for (int kk = 0; kk < KPT; ++kk) {
+            const int n = 4 * (k0 + kk) + w4;
+            cp_async16(dst0 + swz128(n, c32 & 7), v_lane + off[kk], valid[kk]);
+          }
+        }
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&v_full[vst]))
+                     : "memory");
+        if (++kst == NK) { kst = 0; keph ^= 1; }
+        if (++vst == NV) { vst = 0; veph ^= 1; }
 #pragma unroll
         for (int kk = 0; kk < KPT; ++kk) { kbv[kk] = kbn[kk]; kbn[kk] = kbm[kk]; }
         if (i == 0 && !load_q()) { ok = false; break; }
@@ -351,14 +372,14 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
     // -------------------------------------------------------------------- MMA
     // Two issuing threads: warp W_MMA issues every S, warp W_MMA + 1 every
     // P V, so a P V whose P is ready is not held behind the issue of the next
-    // S (which waits for its K / V and for room in the tensor pipe); the
-    // stage a P V frees is refilled that much sooner.  S(i) overwrites the
-    // TMEM buffer P(i - 2) was read from, so it waits for P V(i - 2).
+    // S (which waits for its K tile and for room in the tensor pipe); the
+    // V slot a P V frees is refilled that much sooner.  S(i) overwrites the
+    // TMEM buffer P(i - NSB) was read from, so it waits for P V(i - NSB).
     if (lane == 0) {
       const bool s_role = warp == W_MMA;
       constexpr uint32_t idesc_s = umma_idesc_bf16_f32(128, KT);
       constexpr uint32_t idesc_pv = umma_idesc_bf16_f32(128, 256) | (1u << 16);   // B (V) MN-major
-      int stage = 0;
+      int stage = 0;                 // K slot (S issuer) or V slot (P V issuer)
       uint32_t fphase = 0;
       uint32_t items_done = 0, s_count = 0, p_count = 0;
       bool ok = true;
@@ -371,19 +392,19 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
           if (!mbar_wait(q_full, items_done & 1, abort_flag, a.err)) { ok = false; break; }
           tc_fence_after();
           for (int i = 0; i < n_tiles; ++i) {
-            if (!mbar_wait(&kv_full[stage], fphase, abort_flag, a.err)) { ok = false; break; }
-            // P V number s_count - 2 read the buffer S(i) writes; P V s_count - 4
-            // has completed (waited before S(i - 2)) and P V s_count cannot
-            // yet (it needs this S), so the parity of pv_done[(s_count - 2) & 1]
-            // is exact even when P V s_count - 1 already completed
-            if (s_count >= 2) {
-              const uint32_t g = s_count - 2;
-              if (!mbar_wait(&pv_done[g & 1], (g >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
+            if (!mbar_wait(&k_full[stage], fphase, abort_flag, a.err)) { ok = false; break; }
+            // P V number s_count - NSB read the buffer S(i) writes.  Its
+            // barrier pv_done[(s_count - NSB) % NSB] is next completed by P V
+            // s_count, which needs this S, and P V s_count - 2 NSB was waited
+            // for before S(i - NSB), so the parity wait is exact
+            if (s_count >= NSB) {
+              const uint32_t g = s_count - NSB;
+              if (!mbar_wait(&pv_done[g % NSB], (g / NSB) & 1, abort_flag, a.err)) { ok = false; break; }
             }
-            fence_proxy_async();    // the stage was written by cp.async; the MMA reads it
+            fence_proxy_async();    // the slot was written by cp.async; the MMA reads it
             tc_fence_after();
-            const uint32_t b = s_count & 1;
-            const uint32_t k_base = smem_u32(smem + OFF_STAGE + stage * STAGE_BYTES);
+            const uint32_t b = s_count % NSB;
+            const uint32_t k_base = smem_u32(smem + OFF_STAGE + stage * KV_BYTES);
 #pragma unroll
             for (int ks = 0; ks < 16; ++ks) {
               const uint32_t c = ks >> 2, koff = (ks & 3) * 32;
@@ -392,30 +413,33 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
               umma_bf16(tmem + TM_S0 + 64 * b, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
             }
             tc_commit(&s_full[b]);
+            tc_commit(&k_empty[stage]);
             if (i == n_tiles - 1) tc_commit(q_empty);
             ++s_count;
-            if (++stage == NSTAGE) { stage = 0; fphase ^= 1; }
+            if (++stage == NK) { stage = 0; fphase ^= 1; }
           }
         } else {
           for (int j = 0; j < n_tiles; ++j) {
-            const uint32_t b = p_count & 1;
-            if (!mbar_wait(&p_full[b], (p_count >> 1) & 1, abort_flag, a.err)) { ok = false; break; }
+            const uint32_t b = p_count % NSB;
+            if (!mbar_wait(&p_full[b], (p_count / NSB) & 1, abort_flag, a.err)) { ok = false; break; }
             if (j == 0 && items_done > 0 && !mbar_wait(o_empty, (items_done - 1) & 1, abort_flag, a.err)) {
               ok = false;
               break;
             }
+            if (!mbar_wait(&v_full[stage], fphase, abort_flag, a.err)) { ok = false; break; }
+            fence_proxy_async();    // the slot was written by cp.async; the MMA reads it
             tc_fence_after();
-            const uint32_t v_base = smem_u32(smem + OFF_STAGE + stage * STAGE_BYTES + KV_BYTES);
+            const uint32_t v_base = smem_u32(smem + OFF_V + stage * KV_BYTES);
 #pragma unroll
             for (int ks = 0; ks < KT / 16; ++ks) {
               const uint64_t bd = umma_desc_mn_sw128(v_base + ks * 2048, CHUNK_KV, 1024);
               umma_ts_bf16(tmem + TM_O, tmem + TM_S0 + 64 * b + 8 * ks, bd, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
             }
-            tc_commit(&kv_empty[stage]);
-            tc_commit(&pv_done[p_count & 1]);
+            tc_commit(&v_empty[stage]);
+            tc_commit(&pv_done[p_count % NSB]);
             if (j == n_tiles - 1) tc_commit(o_full);
             ++p_count;
-            if (++stage == NSTAGE) stage = 0;
+            if (++stage == NV) { stage = 0; fphase ^= 1; }
           }
         }
         ++items_done;
@@ -442,8 +466,8 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
       const int own_lim = (int)(t & 3);               // last visible token of the own block
       float m_run = -FLT_MAX, l_run = 0.f;
       for (int i = 0; i < n_tiles; ++i) {
-        const uint32_t b = s_count & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&s_full[b], (s_count >> 1) & 1, abort_flag, a.err))) {
+        const uint32_t b = s_count % NSB;
+        if (!__all_sync(0xffffffffu, mbar_wait(&s_full[b], (s_count / NSB) & 1, abort_flag, a.err))) {
           ok = false;
           break;
         }
@@ -487,11 +511,12 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
           if (i >= 1) {
             // O may be rescaled only once P V(i - 1), number g = pv_seq + i - 1,
             // has accumulated into it.  S(i) has completed and was issued after
-            // P V(i - 2) completed, and P V(i + 1) cannot have (it needs P(i + 1)),
-            // so the parity of pv_done[g & 1] is exact.  Only this rare path
-            // waits, so the softmax of tile i overlaps P V(i - 1).
+            // P V(i - NSB) completed, and P V(g + NSB) cannot have (it needs
+            // P(i + 1) at least), so the parity of pv_done[g % NSB] is exact.
+            // Only this rare path waits, so the softmax of tile i overlaps
+            // P V(i - 1).
             const uint32_t g = pv_seq + (uint32_t)i - 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[g & 1], (g >> 1) & 1, abort_flag, a.err))) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[g % NSB], (g / NSB) & 1, abort_flag, a.err))) {
               ok = false;
               break;
             }
