@@ -19,11 +19,13 @@
 //     O += P V with P taken from TMEM (A operand) and V as an MN-major
 //     shared-memory operand, M = 128, N = 256, fp32 in TMEM; it frees the
 //     V slot.
-//   * warps 8-9 (softmax): one thread per query row (TMEM lanes 0..63):
-//     mask, running max in base 2 (raised only when a tile's max exceeds it by
-//     more than 8, so the O rescale is rare), exp2, row sum, P packed to bf16
-//     and stored back into the S buffer's first 32 columns; at the end of an
-//     item O is read, normalised and written as bf16 with the row's lse.
+//   * warps 8-9 and 12-13 (softmax): two threads per query row (TMEM lanes
+//     0..63), each with half of a tile's 64 columns: mask, running max in
+//     base 2 (the two halves swap their tile maxima; the max is raised only
+//     when a tile's max exceeds it by more than 8, so the O rescale is rare),
+//     exp2, row sum, P packed to bf16 and stored back into the S buffer's
+//     first 32 columns; at the end of an item each thread normalises and
+//     writes its 128 of the row's 256 dims, bf16, with the row's lse.
 //   * every mbarrier wait is bounded (timeout -> error word, clean exit).
 #include <cfloat>
 
@@ -38,14 +40,17 @@ constexpr int KT = 64;                              // keys per tile
 // gathers are issue-bound between slot releases): 5 % faster at 1M tokens.
 constexpr int LWARPS = 8;                            // loader warps (4 or 8)
 constexpr int LOADERS = 32 * LWARPS;
-constexpr int W_SOFT = LWARPS;                       // softmax warps W_SOFT, W_SOFT + 1
+constexpr int W_SOFT = LWARPS;                       // softmax warps W_SOFT, W_SOFT + 1 (columns 0..31)
 constexpr int W_MMA = LWARPS + 2;
-constexpr int THREADS = 32 * (LWARPS + 4);
+constexpr int W_SOFT2 = LWARPS + 4;                  // softmax warps W_SOFT2, W_SOFT2 + 1 (columns 32..63)
+constexpr int THREADS = 32 * (LWARPS + 6);
 constexpr uint32_t QROWS = 48;
 constexpr uint32_t CHUNK_Q = QROWS * 128;           // 6 KB: 48 rows x 64 dims
 constexpr uint32_t CHUNK_KV = KT * 128;             // 8 KB: 64 keys x 64 dims
 constexpr uint32_t KV_BYTES = 4 * CHUNK_KV;         // 32 KB per K (or V) tile
 constexpr uint32_t OFF_STAGE = 32768;               // Q region (24 KB) padded to 32 KB
+constexpr uint32_t OFF_XCH = 4 * CHUNK_Q;           // softmax exchange (1 KB) in the Q region's padding
+static_assert(OFF_XCH + 1024 <= OFF_STAGE, "exchange buffer");
 // Separate K and V rings in the same 192 KB: a K slot is freed once S has
 // read it, a V slot once P V has, so the next K tile lands while the
 // softmax and P V of the current one run.  Three S / P buffers in TMEM let
@@ -116,6 +121,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
         "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
         "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
@@ -211,7 +224,8 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
   uint64_t* o_full = pv_done + NSB;
   uint64_t* o_empty = o_full + 1;
   uint64_t* mma_done = o_empty + 1;          // [2]: the S and the P V issuer
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 2);
+  uint64_t* xbar = mma_done + 2;             // [2]: softmax row groups 0..31, 32..63
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xbar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -224,9 +238,11 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
     mbar_init(q_empty, 1);
     for (int s = 0; s < NK; ++s) { mbar_init(&k_full[s], LOADERS); mbar_init(&k_empty[s], 1); }
     for (int s = 0; s < NV; ++s) { mbar_init(&v_full[s], LOADERS); mbar_init(&v_empty[s], 1); }
-    for (int b = 0; b < NSB; ++b) { mbar_init(&s_full[b], 1); mbar_init(&p_full[b], 2); mbar_init(&pv_done[b], 1); }
+    for (int b = 0; b < NSB; ++b) { mbar_init(&s_full[b], 1); mbar_init(&p_full[b], 4); mbar_init(&pv_done[b], 1); }
+    mbar_init(&xbar[0], 64);
+    mbar_init(&xbar[1], 64);
     mbar_init(o_full, 1);
-    mbar_init(o_empty, 2);
+    mbar_init(o_empty, 4);
     mbar_init(&mma_done[0], 1);
     mbar_init(&mma_done[1], 1);
     *abort_flag = 0;
@@ -448,12 +464,34 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
       tc_commit(done);
       mbar_wait(done, 0, abort_flag, a.err);
     }
-  } else if (warp == W_SOFT || warp == W_SOFT + 1) {
+  } else if (warp == W_SOFT || warp == W_SOFT + 1 || warp == W_SOFT2 || warp == W_SOFT2 + 1) {
     // ---------------------------------------------------------------- softmax
-    const int r = 32 * (warp - W_SOFT) + lane;      // query row = TMEM lane
+    // Four warps: warps W_SOFT, W_SOFT + 1 take columns 0..31 of each tile's
+    // S for query rows 0..31 and 32..63, warps W_SOFT2, W_SOFT2 + 1 columns
+    // 32..63 of the same rows (a warp reaches TMEM lanes 32 (warp % 4) ..).
+    // The two threads of a row swap their tile maxima (and at the end of an
+    // item their row sums) through shared memory and a per-row-group
+    // mbarrier, so both use the same running max; each rescales, normalises
+    // and writes its own 128 of the row's 256 output dims.
+    const int half = warp >= W_SOFT2 ? 1 : 0;
+    const int quad = warp & 3;                      // 0 or 1: TMEM lanes 32 quad ..
+    const int r = 32 * quad + lane;                 // query row = TMEM lane
     const bool row_ok = r < QR;
     const int tok = row_ok ? r / 12 : 0, hh = row_ok ? r % 12 : 0;
-    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
+    float* xch = reinterpret_cast<float*>(smem + OFF_XCH);   // [2 slots][2 halves][64 rows]
+    uint64_t* xb = &xbar[quad];
+    uint32_t xc = 0;                                // exchanges so far (slot and parity)
+    // swap a value with the other thread of this row; false on abort / timeout
+    auto exchange = [&](float mine, float& other) -> bool {
+      const uint32_t slot = xc & 1;
+      xch[(slot * 2 + half) * 64 + r] = mine;
+      mbar_arrive(xb);                              // every lane: releases its own store
+      const bool okx = __all_sync(0xffffffffu, mbar_wait(xb, xc & 1, abort_flag, a.err));
+      other = xch[(slot * 2 + (half ^ 1)) * 64 + r];
+      ++xc;
+      return okx;
+    };
     uint32_t items_done = 0, s_count = 0, pv_seq = 0;
     bool ok = true;
     for (int64_t w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
@@ -472,17 +510,9 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
           break;
         }
         tc_fence_after();
-        float s[64];
-        {
-          float tmp[32];
-          tmem_ld32(tmem + lane_off + TM_S0 + 64 * b, tmp);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) s[c] = tmp[c];
-          tmem_ld32(tmem + lane_off + TM_S0 + 64 * b + 32, tmp);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) s[32 + c] = tmp[c];
-          tmem_ld_wait();
-        }
+        float s[32];
+        tmem_ld32(tmem + lane_off + TM_S0 + 64 * b + 32 * half, s);
+        tmem_ld_wait(s);
         // Masking.  The selection is ascending and always ends with the own
         // block, so every key of a tile before the last one is visible to
         // every row; in the last tile, slots past cnt and the own block's
@@ -491,17 +521,22 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
         const bool last = gi == it.nt_total - 1;
         if (last) {
 #pragma unroll
-          for (int n = 0; n < 64; ++n) {
-            const int blk = 16 * gi + (n >> 2);
-            const bool valid = blk < cnt && (blk < cnt - 1 || (n & 3) <= own_lim);
-            s[n] = valid ? s[n] : -FLT_MAX;
+          for (int c = 0; c < 32; ++c) {
+            const int blk = 16 * gi + 8 * half + (c >> 2);
+            const bool valid = blk < cnt && (blk < cnt - 1 || (c & 3) <= own_lim);
+            s[c] = valid ? s[c] : -FLT_MAX;
           }
         }
         float mt = -FLT_MAX;
 #pragma unroll
-        for (int n = 0; n < 63; n += 3) mt = fmaxf(mt, max3f(s[n], s[n + 1], s[n + 2]));
-        mt = fmaxf(mt, s[63]);
+        for (int c = 0; c < 30; c += 3) mt = fmaxf(mt, max3f(s[c], s[c + 1], s[c + 2]));
+        mt = fmaxf(mt, fmaxf(s[30], s[31]));
         mt = row_ok ? mt * a.scale_log2 : -FLT_MAX;   // raw max, then the (positive) scale
+        // both threads of the row have read their S columns before either
+        // writes P over them
+        float mt_other;
+        if (!exchange(mt, mt_other)) { ok = false; break; }
+        mt = fmaxf(mt, mt_other);
         const bool need = mt > m_run + 8.f;
         if (__any_sync(0xffffffffu, need)) {
           const float m_new = need ? fmaxf(m_run, mt) : m_run;
@@ -522,33 +557,33 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
             }
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 0; c < 4; ++c) {
               float o[32];
-              tmem_ld32(tmem + lane_off + TM_O + 32 * c, o);
-              tmem_ld_wait();
+              tmem_ld32(tmem + lane_off + TM_O + 128 * half + 32 * c, o);
+              tmem_ld_wait(o);
               uint32_t u[32];
 #pragma unroll
               for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(o[e] * corr);
-              tmem_st32(tmem + lane_off + TM_O + 32 * c, u);
+              tmem_st32(tmem + lane_off + TM_O + 128 * half + 32 * c, u);
             }
             tmem_st_wait();
           }
         }
         // p = 2^(s*scale - m); masked slots (-FLT_MAX) underflow to exactly 0
-        uint32_t pk[32];
+        uint32_t pk[16];
         float lsum0 = 0.f, lsum1 = 0.f;
         const float neg_m = -m_run;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
+        for (int e = 0; e < 16; ++e) {
           const float p0 = ex2(fmaf(s[2 * e], a.scale_log2, neg_m));
           const float p1 = ex2(fmaf(s[2 * e + 1], a.scale_log2, neg_m));
           lsum0 += p0;
           lsum1 += p1;
           pk[e] = cvt_bf16x2(p0, p1);
         }
-        const float lsum = lsum0 + lsum1;
-        l_run += lsum;
-        tmem_st32(tmem + lane_off + TM_S0 + 64 * b, pk);
+        l_run += lsum0 + lsum1;
+        // keys 32 half .. +31 of the tile, packed two per column
+        tmem_st16(tmem + lane_off + TM_S0 + 64 * b + 16 * half, pk);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -560,23 +595,26 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
       if (!__all_sync(0xffffffffu, mbar_wait(o_full, items_done & 1, abort_flag, a.err))) { ok = false; break; }
       pv_seq += (uint32_t)n_tiles;   // every P V of the item has completed
       tc_fence_after();
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      float l_other;
+      if (!exchange(l_run, l_other)) { ok = false; break; }
+      const float l_row = l_run + l_other;
+      const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
       const bool write = row_ok && (DEC || (t < a.T && t >= a.q_tok0));
       const int64_t orow_idx = (DEC ? it.row : t - a.q_tok0) * 24 + 12 * g + hh;   // [token or sequence][head]
-      uint16_t* orow = a.out + orow_idx * 256;
+      uint16_t* orow = a.out + orow_idx * 256 + 128 * half;
       const bool partial = DEC && a.n_split > 1;
       const bool out32 = (reinterpret_cast<uintptr_t>(a.out) & 31) == 0;   // rows are 512 B apart
       const bool part32 = (reinterpret_cast<uintptr_t>(a.part_o) & 31) == 0;
       const int64_t prow = ((it.row * 2 + g) * (int64_t)a.n_split + it.split) * 12 + hh;
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < 4; ++c) {
         float o[32];
-        tmem_ld32(tmem + lane_off + TM_O + 32 * c, o);
-        tmem_ld_wait();
-        // each row is written by one thread: 32-byte stores where the output
-        // allows (full sectors, half the store instructions of 16-byte ones)
+        tmem_ld32(tmem + lane_off + TM_O + 128 * half + 32 * c, o);
+        tmem_ld_wait(o);
+        // 32-byte stores where the output allows (full sectors, half the
+        // store instructions of 16-byte ones)
         if (write && partial && part32) {
-          float* dst = a.part_o + prow * 256 + 32 * c;   // rows are 1 KB apart
+          float* dst = a.part_o + prow * 256 + 128 * half + 32 * c;   // rows are 1 KB apart
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             uint32_t x[8];
@@ -585,7 +623,7 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
             st_global_v8(dst + 8 * q, x);
           }
         } else if (write && partial) {
-          float4* dst = reinterpret_cast<float4*>(a.part_o + prow * 256 + 32 * c);
+          float4* dst = reinterpret_cast<float4*>(a.part_o + prow * 256 + 128 * half + 32 * c);
 #pragma unroll
           for (int q = 0; q < 8; ++q)
             dst[q] = make_float4(o[4 * q] * inv, o[4 * q + 1] * inv, o[4 * q + 2] * inv, o[4 * q + 3] * inv);
@@ -607,15 +645,16 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
                                 cvt_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
         }
       }
-      if (write && partial) a.part_lse[prow] = m_run + log2f(l_run);
-      else if (write && a.lse) a.lse[orow_idx] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+      if (half == 0) {
+        if (write && partial) a.part_lse[prow] = m_run + log2f(l_row);
+        else if (write && a.lse) a.lse[orow_idx] = (m_run + log2f(l_row)) * 0.69314718055994531f;
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(o_empty);
       ++items_done;
     }
   }
-
   tc_fence_before();
   __syncthreads();
   if (warp == W_MMA) {
