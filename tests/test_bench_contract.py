@@ -80,5 +80,6 @@ def test_reference_arm_line(tmp_path):
     assert p.returncode == 0, p.stderr
     line = json.loads(p.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] == 12.5
+    assert line["ms_per_step"] == 1000.0 and line["warmup"] == 3   # one sampled step's wall time
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
