@@ -501,9 +501,13 @@ def run_decode(B: int, L: int, budget: int, steps: int, warmup: int, rank: int, 
 _KIDX_CACHE: dict = {}
 
 
-def cpu_sample(wl: dict, target_s: float = 12.0):
+def cpu_sample(wl: dict, target_s: float = 12.0, stratified: int = 0):
     """The oracle on a bounded sample of the workload sized to ~target_s of
-    CPU time: a calibration run, then one run scaled to the target."""
+    CPU time: a calibration run, then one run scaled to the target.  With
+    stratified = n (prefill only) the sample is instead the n stratified query
+    blocks the parity checks use."""
+    if stratified and wl["kind"] == "prefill":
+        return cpu_prefill_sample(wl["T"], 512, stratified, aggregation=wl.get("aggregation", 0), stratified=True)
     if wl["kind"] in ("prefill", "prefill_cached"):
         qb_lo = wl.get("L_old", 0) // 4
         agg = wl.get("aggregation", 0)
@@ -525,16 +529,32 @@ def cpu_sample(wl: dict, target_s: float = 12.0):
     return v, info
 
 
-def cpu_prefill_sample(T: int, budget: int, n_blocks: int, seed: int = 0, qb_lo: int = 0, aggregation: int = 0):
-    """The oracle on a stratified sample of query blocks of the T-token
-    prefill (evenly spaced qb in [qb_lo, nqb)), all host cores.  Returns
-    tokens/s of the oracle extrapolated by the sample's share of the work, and
-    a description."""
+def _oracle_work(qbs: np.ndarray, T: int, budget: int) -> np.ndarray:
+    """Multiply-adds the oracle spends on query block qb: scores (16 token
+    pairs x 4 heads x 128 dims per causal key block) plus attention (4 tokens
+    x 24 heads x 2 x 256 per attended key)."""
+    qbs = np.asarray(qbs, dtype=np.float64)
+    n_tok = np.minimum(4.0, T - 4.0 * qbs)
+    keys = np.minimum(4.0 * (qbs + 1), 4.0 * budget)
+    return 16 * 512 * (qbs + 1) + n_tok * 24 * 512 * keys
+
+
+def cpu_prefill_sample(T: int, budget: int, n_blocks: int, seed: int = 0, qb_lo: int = 0, aggregation: int = 0,
+                       stratified: bool = False):
+    """The oracle on a sample of query blocks of the T-token prefill (evenly
+    spaced in [qb_lo, nqb), or the stratified sample of the parity checks),
+    all host cores.  Returns tokens/s of the oracle extrapolated to the whole
+    workload by the sample's share of the oracle's multiply-adds, and a
+    description."""
     import oracle
     O = oracle.Oracle(oracle.params(budget=budget, aggregation=aggregation))
     P = Q.PrefillProblem(T=T, seed=seed, n_plant=8, dist="zipf" if T >= 131072 else "uniform")
     nqb = P.nqb
-    qbs = np.unique(np.linspace(qb_lo, nqb - 1, n_blocks).astype(np.int64))
+    if stratified:
+        qbs = Q.stratified_query_blocks(nqb, n=n_blocks, budget=budget, seed=T)
+        qbs = qbs[qbs >= qb_lo]
+    else:
+        qbs = np.unique(np.linspace(qb_lo, nqb - 1, n_blocks).astype(np.int64))
     key = (T, seed)
     if key not in _KIDX_CACHE:
         _KIDX_CACHE.clear()
@@ -567,12 +587,15 @@ def cpu_prefill_sample(T: int, budget: int, n_blocks: int, seed: int = 0, qb_lo:
     O.attend_blocks(T, q, k, v, qbs, sel, cnt)
     t_attn = time.time() - t_b
     elapsed = t_score + t_attn
-    # the sample is evenly spaced in qb, so its mean work matches the workload's
-    tokens = 4 * len(qbs)
+    all_q = np.arange(qb_lo, nqb)
+    share = _oracle_work(qbs, T, budget).sum() / _oracle_work(all_q, T, budget).sum()
+    tokens = T - 4 * qb_lo
     span = "" if qb_lo == 0 else f" from query block {qb_lo} on"
-    return tokens / elapsed, dict(sample=f"{len(qbs)} evenly spaced query blocks{span} of the {T}-token prefill "
-                                         f"(scores + selection + attention), {elapsed:.1f} s",
-                                  elapsed=elapsed)
+    kind = "stratified (first, last, around the budget boundary, evenly spaced)" if stratified else "evenly spaced"
+    return tokens * share / elapsed, dict(
+        sample=f"{len(qbs)} {kind} query blocks{span} of the {T}-token prefill (scores + selection + attention), "
+               f"{elapsed:.1f} s, extrapolated by their {100 * share:.3f} % share of the oracle's multiply-adds",
+        elapsed=elapsed)
 
 
 def cpu_decode_sample(B: int, L: int, budget: int, n_seq: int, seed: int = 0, aggregation: int = 0,
@@ -602,7 +625,8 @@ def cpu_decode_sample(B: int, L: int, budget: int, n_seq: int, seed: int = 0, ag
         # attention on that selection (timed); with spec = n also the n - 1
         # draft tokens of the round that reuse it
         t1 = time.time()
-        ring_q, ring_w = np.zeros((0, 4, 128), np.uint16), np.zeros((0, 4), np.uint16)
+        # no block-mates before token L: the workload's L is a multiple of 4
+        ring_q, ring_w = P.q_idx(4 * (L // 4), L), P.w(4 * (L // 4), L)
         O.decode(L, kc, vc, kid, ring_q, ring_w, x["q"], x["k"], x["v"], x["q_idx"], kidx_new, x["w"],
                  sel_in=sel, cnt_in=cnt)
         for _ in range(max(spec, 1) - 1):
@@ -626,7 +650,6 @@ def cpu_verify_sample(B: int, L: int, budget: int, m: int, target_s: float = 12.
     O = oracle.Oracle(oracle.params(budget=budget))
     D = Q.DecodeProblem(B=B, L=L, steps=m, seed=seed, n_plant=8)
     elapsed, n_seq = 0.0, 0
-    ring_q, ring_w = np.zeros((0, 4, 128), np.uint16), np.zeros((0, 4), np.uint16)
     while n_seq < B and (elapsed < target_s / 2 or n_seq < 1):
         b = n_seq
         P = D.tokens(b)
@@ -648,8 +671,12 @@ def cpu_verify_sample(B: int, L: int, budget: int, m: int, target_s: float = 12.
             for t in range(t0, t1):
                 i = t - L
                 tb = time.time()
-                O.decode(t, kc[:t], vc[:t], kid[:t], ring_q, ring_w, x["q"][i], x["k"][i], x["v"][i], x["q_idx"][i],
-                         kid[t], x["w"][i], sel_in=sel, cnt_in=cnt)
+                # block-mates 4 qb .. t - 1: cached tokens before L, new tokens from L on
+                c1 = max(4 * qb, min(L, t))
+                mates_q = np.concatenate([P.q_idx(4 * qb, c1), x["q_idx"][max(4 * qb, L) - L:i]])
+                mates_w = np.concatenate([P.w(4 * qb, c1), x["w"][max(4 * qb, L) - L:i]])
+                O.decode(t, kc[:t], vc[:t], kid[:t], mates_q, mates_w, x["q"][i], x["k"][i], x["v"][i],
+                         x["q_idx"][i], kid[t], x["w"][i], sel_in=sel, cnt_in=cnt)
                 elapsed += time.time() - tb
         n_seq += 1
     return n_seq * m / elapsed, dict(sample=f"{n_seq} of {B} sequences, {m} verify tokens each at {L} cached tokens "
@@ -857,10 +884,18 @@ def main():
                          verify_m=wl.get("verify_m", 0))
     line = line_for(args.workload, res, world, args.steps, args.warmup, pk)
 
+    if rank == 0 and world == 1 and not args.no_cpu:
+        # 256 stratified query blocks at 1M (about half a minute on 16 cores)
+        v, info = cpu_sample(wl, stratified=256 if wl.get("T", 0) >= 1 << 20 else 0)
+        line["cpu_baseline"] = dict(value=v, unit="tokens/s", cores=cores_used(), kind="oracle",
+                                    sample=info["sample"])
+
     if not args.no_secondary:
+        # the other workloads, compact (the line's end is what a log tail
+        # keeps, so the plain decode and the 128K / 32K prefill come last)
         sec = {}
-        for name in ("decode_64x256k", "prefill_128k", "prefill_1m_cached90", "prefill_1m_meanpool",
-                     "decode_64x256k_meanpool", "decode_64x256k_spec4", "verify_64x256k_m5"):
+        for name in ("prefill_1m_cached90", "prefill_1m_meanpool", "decode_64x256k_meanpool", "decode_64x256k_spec4",
+                     "verify_64x256k_m5", "prefill_32k", "prefill_128k", "decode_64x256k"):
             if name == args.workload:
                 continue
             w2 = WORKLOADS[name]
@@ -875,14 +910,16 @@ def main():
                                 want_e2e=False, aggregation=w2.get("aggregation", 0), spec=w2.get("spec", 0),
                                 verify_m=w2.get("verify_m", 0))
             l2 = line_for(name, r2, world, args.steps, args.warmup, pk)
-            sec[name] = {k: l2[k] for k in ("metric", "value", "unit", "ms_per_step", "roofline", "step_roofline",
-                                            "gpu_launches", "kernels_ms")}
+            sr = l2["step_roofline"]
+            sec[name] = dict(metric=l2["metric"], value=round(l2["value"], 1), ms_per_step=round(l2["ms_per_step"], 3),
+                             kernel=l2["roofline"]["kernel"], kernel_frac=round(l2["roofline"]["frac"], 4),
+                             step_frac=round(sr.get("frac_of_tensor_roofline", sr.get("frac_of_hbm_roofline")), 4))
+            km = l2["kernels_ms"]
+            for kname in ("attention", "decode_attention"):
+                if kname in km:   # the attention's share of the step
+                    sec[name][kname + "_ms_per_step"] = round(km[kname]["total_ms"] / args.steps, 3)
         line["secondary"] = sec
 
-    if rank == 0 and world == 1 and not args.no_cpu:
-        v, info = cpu_sample(wl)
-        line["cpu_baseline"] = dict(value=v, unit="tokens/s", cores=cores_used(), kind="oracle",
-                                    sample=info["sample"])
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

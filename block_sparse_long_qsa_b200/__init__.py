@@ -27,7 +27,8 @@ EXPORTED = ["qsa_default_params", "qsa_status_string", "qsa_last_error", "qsa_in
             "qsa_decode_workspace_size", "qsa_check_device_error", "qsa_trace_begin", "qsa_trace_end",
             "qsa_decode_noalloc", "qsa_prefill_cached", "qsa_prefill_cached_workspace_size",
             "qsa_index_workspace_size", "qsa_decode_mean_pool", "qsa_mean_pool_keys",
-            "qsa_decode_reuse", "qsa_verify", "qsa_verify_workspace_size"]
+            "qsa_decode_reuse", "qsa_verify", "qsa_verify_workspace_size", "qsa_set_decode_splits",
+            "qsa_decode_noalloc_check_error"]
 
 KERNEL_NAMES = {1: "rope_table", 2: "rope_k", 3: "indexer", 4: "select", 5: "attention", 6: "decode_append",
                 7: "decode_indexer", 8: "decode_attention", 9: "decode_combine",
@@ -92,6 +93,8 @@ def load(path: str = LIB_PATH):
     L.qsa_decode_noalloc.argtypes = [P, i32, i64, ctypes.POINTER(ctypes.c_int64), vp, vp, vp, vp, vp, vp, vp, vp,
                                      vp, vp, vp, vp, vp, vp, vp]
     L.qsa_check_device_error.argtypes = [vp, vp]
+    L.qsa_decode_noalloc_check_error.argtypes = [vp]
+    L.qsa_set_decode_splits.argtypes = [i32]
     L.qsa_trace_begin.argtypes = [i32]
     L.qsa_trace_end.argtypes = [vp, vp, i32, ctypes.POINTER(ctypes.c_int32)]
     for f in EXPORTED:
@@ -265,6 +268,16 @@ def qsa_decode_noalloc(p: qsa_params, B: int, max_len: int, cache_len, k_cache, 
 
 def qsa_check_device_error(ws, stream=None) -> int:
     return load().qsa_check_device_error(_ptr(ws), _stream(stream))
+
+
+def qsa_decode_noalloc_check_error(stream=None) -> int:
+    """Device error word of qsa_decode_noalloc's fixed array (synchronises)."""
+    return load().qsa_decode_noalloc_check_error(_stream(stream))
+
+
+def qsa_set_decode_splits(n: int):
+    """Fix the number of split-KV decode ranges (1..16) for this process; 0 = automatic."""
+    _check(load().qsa_set_decode_splits(int(n)), "qsa_set_decode_splits")
 
 
 class trace:

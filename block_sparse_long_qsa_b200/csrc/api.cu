@@ -5,6 +5,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -608,13 +609,12 @@ DecodeLayout decode_layout(int B, int64_t max_len, int budget) {
 // does, in tiles: (items it runs) x (tiles per item + 1.5 for the per-item
 // overhead), plus 1 for the combine when there is more than one range, given
 // the largest selection of the batch (measured on B200: at 64 sequences x 32
-// tiles one range per (sequence, KV head) is best).  The environment variable
-// QSA_DECODE_SPLITS (1 .. 16) overrides the choice.
+// tiles one range per (sequence, KV head) is best).  qsa_set_decode_splits
+// (1 .. 16) overrides the choice for the whole process.
+std::atomic<int> g_forced_splits{0};
 int decode_splits(int B, int64_t max_L, int budget, int num_sms) {
-  if (const char* e = std::getenv("QSA_DECODE_SPLITS")) {
-    const int v = std::atoi(e);
-    if (v >= 1 && v <= DECODE_MAX_SPLIT) return v;
-  }
+  const int forced = g_forced_splits.load(std::memory_order_relaxed);
+  if (forced >= 1 && forced <= DECODE_MAX_SPLIT) return forced;
   int64_t cnt = max_L / 4 + 1;
   if (cnt > budget) cnt = budget;
   const int nt = (int)((cnt + 15) / 16);
@@ -629,6 +629,12 @@ int decode_splits(int B, int64_t max_L, int budget, int num_sms) {
   return best;
 }
 }  // namespace
+
+qsa_status qsa_set_decode_splits(int32_t n) {
+  if (n < 0 || n > DECODE_MAX_SPLIT) return QSA_ERR_INVALID_ARG;
+  g_forced_splits.store(n, std::memory_order_relaxed);
+  return QSA_OK;
+}
 
 qsa_status qsa_decode_workspace_size(const qsa_params* p, int32_t B, int64_t max_len, size_t* bytes) {
   qsa_status st = check_params(p);

@@ -13,8 +13,6 @@
 // The array below is reserved on every GPU on which this file's device code
 // is loaded (with CUDA's default lazy module loading: at the first call of
 // this entry point on that GPU) and stays reserved until the process exits.
-#include <mutex>
-
 #include "qsa.h"
 #include "qsa_kernels.h"
 
@@ -23,26 +21,18 @@ namespace {
 // Largest decode scratch this entry point serves (64 MiB: e.g. 64 sequences
 // at 256K context need about 41 MiB).
 constexpr size_t NOALLOC_SCRATCH_BYTES = (size_t)64 << 20;
-constexpr int MAX_DEV = 64;
 
 static __device__ __align__(256) unsigned char g_decode_scratch[NOALLOC_SCRATCH_BYTES];
 
-// Device address of g_decode_scratch, looked up once per device.  In host
-// code the symbol name is only a host-side handle; kernels must be given the
-// address returned by cudaGetSymbolAddress for the current device.
-void* g_scratch_addr[MAX_DEV] = {nullptr};
-std::mutex g_scratch_mu;
-
+// Device address of g_decode_scratch on the current device.  In host code
+// the symbol name is only a host-side handle; kernels must be given the
+// address cudaGetSymbolAddress returns.  It is looked up on every call (a
+// host-side lookup once the module is loaded), so a context that was torn
+// down and created again never gets a stale address.
 qsa_status scratch_for_current_device(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEV) return QSA_ERR_CUDA;
-  std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return QSA_ERR_CUDA;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return QSA_ERR_CUDA;
+  *out = p;
   return QSA_OK;
 }
 
@@ -60,8 +50,16 @@ extern "C" qsa_status qsa_decode_noalloc(const qsa_params* p, int32_t B, int64_t
   if (need > NOALLOC_SCRATCH_BYTES) return QSA_ERR_WORKSPACE_TOO_SMALL;   // beyond the fixed scratch size
   void* scratch = nullptr;
   if ((st = scratch_for_current_device(&scratch)) != QSA_OK) return st;
-  // The regular decode step on the fixed scratch; it clears the error word
-  // at its start, and everything else it writes before reading.
+  // The regular decode step on the fixed scratch.  It clears the error word
+  // at its start and writes everything else before reading it, so nothing of
+  // an earlier call's contents is used.
   return qsa_decode(p, B, max_len, cache_len, k_cache, v_cache, kidx_cache, qidx_ring, w_ring, q_new, k_new, v_new,
                     q_idx_new, k_idx_new, w_new, out, sel_out, lse_out, scratch, NOALLOC_SCRATCH_BYTES, stream);
+}
+
+extern "C" qsa_status qsa_decode_noalloc_check_error(void* stream) {
+  void* scratch = nullptr;
+  qsa_status st = scratch_for_current_device(&scratch);
+  if (st != QSA_OK) return st;
+  return qsa_check_device_error(scratch, stream);
 }

@@ -19,7 +19,8 @@
  *     values travel as uint16_t bit patterns.
  *   - The caller owns every buffer, the workspace included; the library
  *     allocates no device memory.  Its only global state is the one-time
- *     kernel attribute setup per device.
+ *     kernel attribute setup per device and the fixed 64 MiB scratch array
+ *     of qsa_decode_noalloc (reserved where that code is loaded).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream).  Arguments are validated on the host before any launch; on an
  *     argument error nothing is launched.
@@ -209,14 +210,20 @@ qsa_status qsa_prefill_cached_workspace_size(const qsa_params* p, int64_t L_old,
  * Attention is split-KV: each (sequence, KV head) is cut into 1..16 ranges of
  * whole 16-block tiles, chosen so the batch fills the GPU's SMs; with more
  * than one range a combine kernel merges the ranges' partial outputs by their
- * log-sum-exp.  The environment variable QSA_DECODE_SPLITS (1..16) fixes the
- * number of ranges (read at every call; a test and tuning aid). */
+ * log-sum-exp (qsa_set_decode_splits fixes the number of ranges). */
 qsa_status qsa_decode(const qsa_params* p, int32_t B, int64_t max_len, const int64_t* cache_len,
                       uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* qidx_ring,
                       uint16_t* w_ring, const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
                       const uint16_t* q_idx_new, const uint16_t* k_idx_new, const uint16_t* w_new, uint16_t* out,
                       int32_t* sel_out, float* lse_out, void* ws, size_t ws_bytes, void* stream);
 qsa_status qsa_decode_workspace_size(const qsa_params* p, int32_t B, int64_t max_len, size_t* bytes);
+
+/* A tuning and test aid with no counterpart on the pages: n in 1..16 fixes
+ * the number of split-KV ranges of every later decode-attention launch of
+ * this process (all decode calls, verify included); n = 0 restores the
+ * automatic choice.  Returns QSA_ERR_INVALID_ARG outside 0..16.  Takes
+ * effect at the next call; calls already enqueued keep their split. */
+qsa_status qsa_set_decode_splits(int32_t n);
 
 /* qsa_decode for p->aggregation == QSA_AGG_MEAN_POOL.  kbar_cache
  * [B][ceil(max_len/4)][128] bf16 holds the compressed key of every block:
@@ -302,25 +309,34 @@ qsa_status qsa_mean_pool_keys(const qsa_params* p, int64_t T, const uint16_t* k_
  * a decode step (their device memory belongs to another runtime's budget, or
  * cudaMalloc is not allowed on their request path).  The caller still owns
  * and passes every input, output and cache, exactly as for qsa_decode; the
- * decode scratch instead lives in a 64 MiB array inside this library, which
- * is reserved on each GPU where the library's decode code is loaded and kept
- * until the process exits.  Nothing is allocated by this call.
+ * decode scratch instead lives in a 64 MiB array inside this library.
+ *   - The array is reserved on a device when the library's decode code is
+ *     loaded there: with CUDA's default lazy module loading, at the first
+ *     call of this entry point on that device.  That first call maps the
+ *     64 MiB (it can fail under memory pressure and can synchronise), so
+ *     make it once at initialisation, outside the request path and outside
+ *     any stream capture.  Later calls allocate nothing; the array stays
+ *     reserved until the process exits.
  *   - Sizes whose qsa_decode_workspace_size exceeds 64 MiB are rejected with
  *     QSA_ERR_WORKSPACE_TOO_SMALL before any launch (64 sequences at 256K
  *     context need about 41 MiB).
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) for that device; make that first call before
- *     any stream capture.
+ *   - Every call looks up the array's device address for the current device
+ *     (cudaGetSymbolAddress, a host-side lookup once the code is loaded).
  *   - All calls share the one array per device: calls whose executions
  *     overlap on the GPU (different streams, or different host threads on the
  *     same device) race on it and must be serialised by the caller.
- *   - Device-side errors are recorded in the shared array, which the caller
- *     cannot read; they end the kernels cleanly but are not reported. */
+ *   - Device-side errors are recorded in the array's error word; read them
+ *     with qsa_decode_noalloc_check_error. */
 qsa_status qsa_decode_noalloc(const qsa_params* p, int32_t B, int64_t max_len, const int64_t* cache_len,
                               uint16_t* k_cache, uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* qidx_ring,
                               uint16_t* w_ring, const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new,
                               const uint16_t* q_idx_new, const uint16_t* k_idx_new, const uint16_t* w_new,
                               uint16_t* out, int32_t* sel_out, float* lse_out, void* stream);
+/* The device error word of qsa_decode_noalloc's array on the current device:
+ * synchronises `stream` and returns QSA_OK or the device-side error that the
+ * most recent qsa_decode_noalloc call on this device recorded (each call
+ * clears the word when it starts), then clears it. */
+qsa_status qsa_decode_noalloc_check_error(void* stream);
 
 /* Reads (synchronising `stream`) and clears the device error word at the
  * start of a workspace passed to qsa_select_blocks / qsa_prefill /

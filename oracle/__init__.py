@@ -71,7 +71,9 @@ def _bind(L):
     L.oracle_reuse_selection.argtypes = [i64, vp, ctypes.c_int32, vp]
     L.oracle_reuse_selection.restype = ctypes.c_int32
     L.oracle_select_blocks_list.argtypes = [P, i64, vp, vp, vp, i64, vp, vp, vp]
-    L.oracle_decode.argtypes = [P, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp]
+    L.oracle_attend_gathered.argtypes = [P, i64, vp, i64, vp, vp, vp, vp, vp]
+    L.oracle_decode.argtypes = [P, i64, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp]
+    L.oracle_decode.restype = i32
     return L
 
 
@@ -169,6 +171,20 @@ class Oracle:
                                     _p(cnt), _p(out), _p(lse))
         return out, lse
 
+    def attend_gathered(self, pos_t, q_t, pos_j, k_rows, v_rows):
+        """One token at position pos_t (unrotated q_t [24][256]) over the
+        candidate keys at positions pos_j (unrotated k_rows, v_rows
+        [n][2][256]); keys after pos_t are skipped.  -> (out [24][256], lse [24])."""
+        H, d = self.P.n_q_heads, self.P.head_dim
+        pos_j = np.ascontiguousarray(pos_j, dtype=np.int64)
+        q_t, k_rows, v_rows = _u16(q_t), _u16(k_rows), _u16(v_rows)
+        assert k_rows.shape[0] == v_rows.shape[0] == pos_j.shape[0]
+        out = np.empty((H, d))
+        lse = np.empty(H)
+        self.L.oracle_attend_gathered(ctypes.byref(self.P), int(pos_t), _p(q_t), len(pos_j), _p(pos_j), _p(k_rows),
+                                      _p(v_rows), _p(out), _p(lse))
+        return out, lse
+
     def select_blocks_list(self, T, q_idx, w, k_idx, qb_list):
         """(sel [n][budget], cnt [n]) of the listed query blocks (scores + selection)."""
         qb_list = np.ascontiguousarray(qb_list, dtype=np.int64)
@@ -199,7 +215,9 @@ class Oracle:
 
     def decode(self, L, k_cache, v_cache, kidx_cache, ring_q_idx, ring_w, q_new, k_new, v_new, q_idx_new, k_idx_new,
                w_new, sel_in=None, cnt_in=0):
-        """One decode token at position L; caches hold rows [0, L)."""
+        """One decode token at position L; caches hold rows [0, L).  ring_q_idx
+        [n][4][128] / ring_w [n][4] are the block-mates 4*(L//4) .. L-1, in
+        order (n = L % 4 rows exactly; anything else raises)."""
         H, d = self.P.n_q_heads, self.P.head_dim
         out = np.empty((H, d))
         lse = np.empty(H)
@@ -207,9 +225,15 @@ class Oracle:
         cnt = np.zeros(1, dtype=np.int32)
         args = [_u16(a) for a in (k_cache, v_cache, kidx_cache, ring_q_idx, ring_w, q_new, k_new, v_new, q_idx_new,
                                   k_idx_new, w_new)]
+        n_ring = args[3].shape[0]
+        if args[4].shape[0] != n_ring:
+            raise ValueError("ring_q_idx and ring_w hold different numbers of block-mates")
         si = None if sel_in is None else np.ascontiguousarray(sel_in, dtype=np.int32)
-        self.L.oracle_decode(ctypes.byref(self.P), L, *[_p(a) for a in args], _p(si), int(cnt_in), _p(sel), _p(cnt),
-                             _p(out), _p(lse))
+        ptrs = [_p(a) for a in args]
+        rc = self.L.oracle_decode(ctypes.byref(self.P), L, *ptrs[:5], int(n_ring), *ptrs[5:], _p(si), int(cnt_in),
+                                  _p(sel), _p(cnt), _p(out), _p(lse))
+        if rc != 0:
+            raise ValueError(f"oracle_decode: {n_ring} ring rows given, token {L} has {L % self.P.block} block-mates")
         return sel, int(cnt[0]), out, lse
 
     def reuse_selection(self, qb, sel_in, cnt_in):

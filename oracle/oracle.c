@@ -289,6 +289,39 @@ static int64_t gather_keys(const oracle_params* p, const int32_t* sel, int32_t c
   return n;
 }
 
+/* Attention of one query token over an explicit list of candidate keys
+ * (the same definition as oracle_attend_blocks, for callers that hold only
+ * the rows a token can read): token at position pos_t with unrotated q_t
+ * [H][d]; n keys at positions pos_j[n] with unrotated k_rows, v_rows
+ * [n][G][d].  Keys with pos_j > pos_t are skipped (causality); the rest are
+ * rotated at their positions and attended as by oracle_attend.
+ * out [H][d], lse [H]. */
+void oracle_attend_gathered(const oracle_params* p, int64_t pos_t, const uint16_t* q_t, int64_t n,
+                            const int64_t* pos_j, const uint16_t* k_rows, const uint16_t* v_rows, double* out,
+                            double* lse) {
+  int H = p->n_q_heads, G = p->n_kv_heads, d = p->head_dim;
+  double* kr = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * G * d);
+  double* vv = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * G * d);
+  double* x = (double*)malloc(sizeof(double) * (size_t)d);
+  double* qr = (double*)malloc(sizeof(double) * (size_t)H * d);
+  int64_t m = 0;
+  for (int64_t e = 0; e < n; ++e) {
+    if (pos_j[e] > pos_t) continue;
+    for (int g = 0; g < G; ++g) {
+      for (int c = 0; c < d; ++c) x[c] = bf16_to_f64(k_rows[(e * G + g) * d + c]);
+      oracle_rope(p, x, pos_j[e], kr + (m * G + g) * d);
+      for (int c = 0; c < d; ++c) vv[(m * G + g) * d + c] = bf16_to_f64(v_rows[(e * G + g) * d + c]);
+    }
+    ++m;
+  }
+  for (int h = 0; h < H; ++h) {
+    for (int c = 0; c < d; ++c) x[c] = bf16_to_f64(q_t[h * d + c]);
+    oracle_rope(p, x, pos_t, qr + h * d);
+  }
+  oracle_attend(p, qr, m, kr, vv, out, lse);
+  free(kr); free(vv); free(x); free(qr);
+}
+
 /* ---------------------------------------------------------------- prefill --
  * Scores for query blocks [qb_begin, qb_end) into S[(qb-qb_begin)*ld + kb],
  * kb <= qb (other entries untouched).  T tokens in total. */
@@ -392,18 +425,23 @@ void oracle_prefill_blocks(const oracle_params* p, int64_t T, int64_t pos0, cons
  * ring_w for tokens qb*r .. L-1 followed by the new token's.  The result is by
  * definition that of a prefill's token L over the same keys.
  * If sel_in is non-NULL it replaces the oracle's own selection.
- * k_cache, v_cache [L][G][d]; kidx_cache [L][idx_dim]; q_new [H][d];
+ * k_cache, v_cache [L][G][d]; kidx_cache [L][idx_dim]; ring_q_idx
+ * [n_ring][idx_heads][idx_dim] and ring_w [n_ring][idx_heads] hold the block-mates
+ * qb*r .. L-1 in order (n_ring must equal L - qb*r); q_new [H][d];
  * k_new, v_new [G][d]; q_idx_new [idx_heads][idx_dim]; k_idx_new [idx_dim];
- * w_new [idx_heads]  ->  out [H][d], lse [H], sel_out [budget], cnt_out. */
-void oracle_decode(const oracle_params* p, int64_t L, const uint16_t* k_cache, const uint16_t* v_cache,
-                   const uint16_t* kidx_cache, const uint16_t* ring_q_idx, const uint16_t* ring_w,
-                   const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new, const uint16_t* q_idx_new,
-                   const uint16_t* k_idx_new, const uint16_t* w_new, const int32_t* sel_in, int32_t cnt_in,
-                   int32_t* sel_out, int32_t* cnt_out, double* out, double* lse) {
+ * w_new [idx_heads]  ->  out [H][d], lse [H], sel_out [budget], cnt_out.
+ * Returns 0, or -1 (nothing computed) when n_ring is not the number of
+ * block-mates before the new token. */
+int32_t oracle_decode(const oracle_params* p, int64_t L, const uint16_t* k_cache, const uint16_t* v_cache,
+                      const uint16_t* kidx_cache, const uint16_t* ring_q_idx, const uint16_t* ring_w, int32_t n_ring,
+                      const uint16_t* q_new, const uint16_t* k_new, const uint16_t* v_new, const uint16_t* q_idx_new,
+                      const uint16_t* k_idx_new, const uint16_t* w_new, const int32_t* sel_in, int32_t cnt_in,
+                      int32_t* sel_out, int32_t* cnt_out, double* out, double* lse) {
   int H = p->n_q_heads, G = p->n_kv_heads, d = p->head_dim, r = p->block;
   int IH = p->idx_heads, ID = p->idx_dim;
   int64_t qb = L / r;
   int n_prev = (int)(L - qb * r);            /* block-mates before the new token */
+  if (n_ring != n_prev) return -1;
   int n_present = n_prev + 1;
   uint16_t* qblk = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)n_present * IH * ID);
   uint16_t* wblk = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)n_present * IH);
@@ -458,6 +496,7 @@ void oracle_decode(const oracle_params* p, int64_t L, const uint16_t* k_cache, c
   }
   oracle_attend(p, qr, n, kr, vv, out, lse);
   free(qblk); free(wblk); free(keys); free(sel); free(js); free(kr); free(vv); free(x); free(qr);
+  return 0;
 }
 
 /* ---------------------------------------------------------- top-k reuse --

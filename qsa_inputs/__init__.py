@@ -231,6 +231,32 @@ def planter_map(seed: int, nqb: int, n_plant: int, dist: str) -> np.ndarray:
     return planter
 
 
+def stratified_query_blocks(nqb: int, n: int = 256, budget: int = 512, seed: int = 0) -> np.ndarray:
+    """A stratified sample of min(n, nqb) query-block indices of a prefill
+    with nqb blocks (a sampling recipe for the checks and the CPU baseline,
+    not part of the method): the first three, the last three, the six around
+    the budget boundary (budget - 3 .. budget + 2, where selection starts to
+    drop blocks), four seeded random ones, and the rest evenly spaced over
+    [0, nqb); sorted and distinct."""
+    n = min(n, nqb)
+    fixed = [0, 1, 2, nqb - 3, nqb - 2, nqb - 1] + list(range(budget - 3, budget + 3))
+    rng = np.random.default_rng(seed)
+    fixed += rng.integers(0, max(nqb, 1), size=4).tolist()
+    picked = sorted({int(q) for q in fixed if 0 <= q < nqb})[:n]
+    chosen = set(picked)
+    # evenly spaced fill: walk a fine grid and take every point not yet chosen
+    need = n - len(chosen)
+    if need > 0:
+        free = np.setdiff1d(np.arange(nqb, dtype=np.int64), np.fromiter(chosen, np.int64, len(chosen)))
+        idx = np.linspace(0, len(free) - 1, need).round().astype(np.int64)
+        chosen.update(int(q) for q in free[np.unique(idx)])
+        extra = need - len(np.unique(idx))
+        if extra > 0:
+            rest = np.setdiff1d(free, np.fromiter(chosen, np.int64, len(chosen)))
+            chosen.update(int(q) for q in rest[:extra])
+    return np.array(sorted(chosen), dtype=np.int64)
+
+
 # ------------------------------------------------------------------ prefill
 @dataclass
 class PrefillProblem:

@@ -82,3 +82,31 @@ def gpu_prefill(P: Q.PrefillProblem, budget: int, host=None, ws_bytes=None, on_d
     out = {k: (v.cpu().numpy() if isinstance(v, torch.Tensor) and k != "ws" else v) for k, v in r.items()}
     del r, t
     return host, out
+
+
+def pmap(fn, items):
+    """fn over items on a thread pool (the oracle's C calls release the GIL),
+    results in order; exceptions re-raised in the caller."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    items = list(items)
+    try:
+        n = len(os.sched_getaffinity(0))
+    except Exception:
+        n = os.cpu_count() or 4
+    with ThreadPoolExecutor(max_workers=max(1, min(n, len(items)))) as ex:
+        return list(ex.map(fn, items))
+
+
+def gather_rows(blocks, T, k_fn, v_fn):
+    """Positions and unrotated K / V rows of the listed key blocks (tokens
+    4b .. min(4b + 4, T) - 1), from row generators k_fn(j0, j1), v_fn(j0, j1)."""
+    pos, ks, vs = [], [], []
+    for b in blocks:
+        j0, j1 = 4 * int(b), min(4 * int(b) + 4, T)
+        if j1 <= j0:
+            continue
+        pos.extend(range(j0, j1))
+        ks.append(k_fn(j0, j1))
+        vs.append(v_fn(j0, j1))
+    return np.asarray(pos, np.int64), np.concatenate(ks), np.concatenate(vs)

@@ -404,6 +404,21 @@ def pin_attention_dense_when_budget_covers(O):
         assert np.allclose(lse[:T], want_l, rtol=1e-10, atol=1e-12), T
 
 
+def pin_attend_gathered_dense(O):
+    """The explicit-key-list entry: every token of a short sequence over all
+    its keys (given in shuffled order, later keys included so that the causal
+    skip matters) equals dense causal GQA attention (torch SDPA, fp64)."""
+    T = 23
+    P = Q.PrefillProblem(T=T, seed=41, n_plant=0)
+    h = P.host()
+    want, want_lse = _dense_causal_sdpa(h["q"], h["k"], h["v"])
+    perm = np.random.default_rng(5).permutation(T)
+    for t in (0, 1, 7, 22):
+        out, lse = O.attend_gathered(t, h["q"][t], perm, h["k"][perm], h["v"][perm])
+        assert np.abs(out - want[t]).max() < 1e-10, t
+        assert np.abs(lse - want_lse[t]).max() < 1e-10, t
+
+
 def pin_attention_constant_v_and_single_key(O):
     T = 12
     P = Q.PrefillProblem(T=T, seed=10)

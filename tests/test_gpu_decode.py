@@ -19,6 +19,13 @@ def _lib():
     qsa.load()
 
 
+@pytest.fixture
+def automatic_splits_after():
+    """Back to the automatic split-KV choice once the test is done."""
+    yield
+    qsa.qsa_set_decode_splits(0)
+
+
 class DecodeState:
     """Caches [B][max_len] seeded from a prefill of each sequence's first L tokens."""
 
@@ -123,11 +130,11 @@ def test_decode_append_writes_caches():
 
 
 @pytest.mark.parametrize("splits", [1, 2, 5, 16])
-def test_decode_split_kv_ranges(splits, monkeypatch):
+def test_decode_split_kv_ranges(splits, automatic_splits_after):
     """Split-KV decode with a fixed number of ranges, including ranges left
     empty by a short sequence (1 tile) next to full-budget ones (32 tiles):
     output and lse match the oracle on the kernel's own selection."""
-    monkeypatch.setenv("QSA_DECODE_SPLITS", str(splits))
+    qsa.qsa_set_decode_splits(splits)
     budget = 512
     L_list = [3001, 37, 9000]
     probs = [Q.PrefillProblem(T=L + 1, seed=70 + b, n_plant=8) for b, L in enumerate(L_list)]

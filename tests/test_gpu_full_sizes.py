@@ -1,7 +1,9 @@
-"""GPU parity at the full workload sizes (32K, 128K and 1M prefill; decode of
-64 sequences x 256K), run as the benchmark runs them (same workspace, so the
-same chunking), checked on sampled query blocks / sequences that the fp64
-oracle computes one by one, plus structural checks of every selection row."""
+"""GPU parity at the full workload sizes (32K, 128K and 1M prefill; the
+mean-pool, reuse and verify paths at 64 sequences x 256K), run as the
+benchmark runs them (same workspace, so the same chunking), checked on
+stratified query blocks / sampled sequences that the fp64 oracle computes one
+by one, plus structural checks of every selection row.  The plain decode of
+config 3 (all 32 appending steps) is in test_gpu_decode_config3.py."""
 import numpy as np
 import pytest
 import torch
@@ -9,7 +11,7 @@ import torch
 import block_sparse_long_qsa_b200 as qsa
 import oracle
 import qsa_inputs as Q
-from gpu_util import check_outputs, check_selection
+from gpu_util import check_outputs, check_selection, gather_rows, pmap
 
 pytestmark = pytest.mark.gpu
 
@@ -23,11 +25,10 @@ def _lib():
     qsa.load()
 
 
-def _sample_blocks(nqb: int, seed: int) -> list[int]:
-    fixed = [0, 1, 2, 509, 510, 511, 512, 513, 2047, nqb // 3, nqb // 2, (2 * nqb) // 3, nqb - 2, nqb - 1]
-    rng = np.random.default_rng(seed)
-    extra = rng.integers(0, nqb, size=4).tolist()
-    return sorted({int(q) for q in fixed + extra if 0 <= q < nqb})
+def _sample_blocks(nqb: int, seed: int, n: int = 18) -> list[int]:
+    """n stratified query blocks: the first and last, those around the budget
+    boundary, seeded random ones and evenly spaced ones."""
+    return [int(q) for q in Q.stratified_query_blocks(nqb, n=n, budget=BUDGET, seed=seed)]
 
 
 def _check_selection_structure(sel: torch.Tensor, cnt: torch.Tensor):
@@ -53,25 +54,46 @@ def _check_selection_structure(sel: torch.Tensor, cnt: torch.Tensor):
 def _oracle_block_outputs(O, P, qb, sel_row, cnt):
     """fp64 attention of the tokens of block qb over the given selection."""
     T = P.T
+    pos, ks, vs = gather_rows(sel_row[:cnt], T, P.k, P.v)
     t0, t1 = 4 * qb, min(4 * qb + 4, T)
-    blocks = sel_row[:cnt]
-    ks, vs, js = [], [], []
-    for b in blocks:
-        j0, j1 = 4 * int(b), min(4 * int(b) + 4, T)
-        k = Q.bf16_to_f64(P.k(j0, j1))
-        v = Q.bf16_to_f64(P.v(j0, j1))
-        for j in range(j0, j1):
-            ks.append(np.stack([O.rope(k[j - j0, g], j) for g in range(2)]))
-            vs.append(v[j - j0])
-            js.append(j)
-    ks, vs, js = np.stack(ks), np.stack(vs), np.asarray(js)
-    q = Q.bf16_to_f64(P.q(t0, t1))
-    res = []
-    for t in range(t0, t1):
-        q_rot = np.stack([O.rope(q[t - t0, h], t) for h in range(24)])
-        m = js <= t
-        res.append(O.attend(q_rot, ks[m], vs[m]))
-    return res
+    q = P.q(t0, t1)
+    return [O.attend_gathered(t, q[t - t0], pos, ks, vs) for t in range(t0, t1)]
+
+
+def _check_sampled_blocks(O, P, qbs, sel, cnt, out, lse, what, k_idx=None):
+    """Oracle scores, selection and attention of the sampled query blocks (a
+    thread pool over blocks), compared by the acceptance criteria; returns the
+    number of near-tie selection differences."""
+    T = P.T
+    k_idx = P.k_idx() if k_idx is None else k_idx
+    sel_h = sel[torch.tensor(qbs, device=sel.device)].cpu().numpy()
+    cnt_h = cnt[torch.tensor(qbs, device=cnt.device)].cpu().numpy()
+    rows = torch.cat([torch.arange(4 * q, min(4 * q + 4, T)) for q in qbs]).to(out.device)
+    out_h = out[rows].cpu().numpy()
+    lse_h = lse[rows].cpu().numpy() if lse is not None else None
+    first = {}
+    n = 0
+    for q in qbs:
+        first[q] = n
+        n += min(4 * q + 4, T) - 4 * q
+
+    def one(i):
+        qb = qbs[i]
+        t0, t1 = 4 * qb, min(4 * qb + 4, T)
+        S = O.block_scores(qb, P.q_idx(t0, t1), P.w(t0, t1), k_idx[:t1])
+        osel, ocnt = O.select(qb, S)
+        return S, osel, ocnt, _oracle_block_outputs(O, P, qb, sel_h[i], int(cnt_h[i]))
+
+    n_diff = 0
+    for i, (S, osel, ocnt, want) in enumerate(pmap(one, range(len(qbs)))):
+        qb = qbs[i]
+        n_diff += check_selection(sel_h[i], int(cnt_h[i]), osel, ocnt, S, qb, BUDGET, f"{what} qb={qb}")
+        for k, (o, l) in enumerate(want):
+            r = first[qb] + k
+            check_outputs(out_h[r], o, f"{what} t={4 * qb + k}")
+            if lse_h is not None:
+                assert np.allclose(lse_h[r], l, atol=1e-2), f"{what} t={4 * qb + k} lse"
+    return n_diff
 
 
 @pytest.mark.timeout(1800)
@@ -94,64 +116,10 @@ def test_prefill_full_size_sampled(T, dist):
     _check_selection_structure(sel, cnt)
 
     O = oracle.Oracle(oracle.params(budget=BUDGET))
-    k_idx = P.k_idx()
-    n_diff = 0
-    for qb in _sample_blocks(nqb, seed=T):
-        t0, t1 = 4 * qb, min(4 * qb + 4, T)
-        S = O.block_scores(qb, P.q_idx(t0, t1), P.w(t0, t1), k_idx[:t1])
-        osel, ocnt = O.select(qb, S)
-        g = sel[qb].cpu().numpy()
-        gc = int(cnt[qb])
-        n_diff += check_selection(g, gc, osel, ocnt, S, qb, BUDGET, f"T={T} qb={qb}")
-        want = _oracle_block_outputs(O, P, qb, g, gc)
-        got = out[t0:t1].cpu().numpy()
-        got_lse = lse[t0:t1].cpu().numpy()
-        for i, (o, l) in enumerate(want):
-            check_outputs(got[i], o, f"T={T} t={t0 + i}")
-            assert np.allclose(got_lse[i], l, atol=1e-2), f"T={T} t={t0 + i} lse"
-    print(f"T={T}: sampled rows differ from the oracle selection in {n_diff} near-tie blocks")
-
-
-@pytest.mark.timeout(1800)
-def test_decode_full_size_sampled():
-    B, L = 64, 262144
-    D = Q.DecodeProblem(B=B, L=L, steps=1, seed=0, n_plant=8)
-    max_len = L + 8
-    kc = torch.empty((B, max_len, 2, 256), dtype=torch.uint16, device="cuda")
-    vc = torch.empty_like(kc)
-    ic = torch.empty((B, max_len, 128), dtype=torch.uint16, device="cuda")
-    D.fill_device_caches(kc, vc, ic)
-    ring = torch.zeros((B, 4, 4, 128), dtype=torch.uint16, device="cuda")
-    wring = torch.zeros((B, 4, 4), dtype=torch.uint16, device="cuda")
-    p = qsa.params(BUDGET)
-    ws = qsa.workspace(qsa.qsa_decode_workspace_size(p, B, max_len))
-    x = {k: torch.from_numpy(np.ascontiguousarray(v)).cuda() for k, v in D.step_inputs(0).items()}
-    kin = np.stack([D.tokens(b).k_idx(L, L + 1)[0] for b in range(B)])
-    out = torch.empty((B, 24, 256), dtype=torch.uint16, device="cuda")
-    sel = torch.empty((B, BUDGET), dtype=torch.int32, device="cuda")
-    lse = torch.empty((B, 24), dtype=torch.float32, device="cuda")
-    qsa.qsa_decode(p, B, max_len, [L] * B, kc, vc, ic, ring, wring, x["q"], x["k"], x["v"], x["q_idx"],
-                   torch.from_numpy(kin).cuda(), x["w"], out, sel, lse, ws)
-    torch.cuda.synchronize()
-    assert qsa.qsa_check_device_error(ws) == 0
-    del kc, vc, ic
-    O = oracle.Oracle(oracle.params(budget=BUDGET))
-    inp = D.step_inputs(0)
-    qb = L // 4
-    for b in (0, 1, 31, 63):
-        kcache, vcache, icache = D.cache_k(b), D.cache_v(b), D.cache_kidx(b)
-        ring_q = np.zeros((0, 4, 128), np.uint16)
-        ring_w = np.zeros((0, 4), np.uint16)
-        S = O.block_scores(qb, inp["q_idx"][b][None], inp["w"][b][None], np.concatenate([icache, kin[b][None]]))
-        osel, ocnt, _, _ = O.decode(L, kcache, vcache, icache, ring_q, ring_w, inp["q"][b], inp["k"][b], inp["v"][b],
-                                    inp["q_idx"][b], kin[b], inp["w"][b])
-        g = sel[b].cpu().numpy()
-        gc = int((g >= 0).sum())
-        check_selection(g, gc, osel, ocnt, S, qb, BUDGET, f"decode b={b}")
-        _, _, oo, ol = O.decode(L, kcache, vcache, icache, ring_q, ring_w, inp["q"][b], inp["k"][b], inp["v"][b],
-                                inp["q_idx"][b], kin[b], inp["w"][b], sel_in=g, cnt_in=gc)
-        check_outputs(out[b].cpu().numpy(), oo, f"decode b={b}")
-        assert np.allclose(lse[b].cpu().numpy(), ol, atol=1e-2), f"decode b={b} lse"
+    # 256 stratified query blocks at 1M (the survey's sample), 64 below
+    qbs = _sample_blocks(nqb, seed=T, n=256 if T >= 1 << 20 else 64)
+    n_diff = _check_sampled_blocks(O, P, qbs, sel, cnt, out, lse, f"T={T}")
+    print(f"T={T}: {len(qbs)} sampled query blocks, {n_diff} near-tie selection differences")
 
 
 @pytest.mark.timeout(600)
@@ -195,20 +163,9 @@ def test_prefill_mean_pool_1m_sampled():
     del d, ws
     _check_selection_structure(sel, cnt)
     O = oracle.Oracle(oracle.params(budget=BUDGET, aggregation=oracle.AGG_MEAN_POOL))
-    k_idx = P.k_idx()
-    n_diff = 0
-    for qb in _sample_blocks(nqb, seed=7)[::2]:
-        t0, t1 = 4 * qb, min(4 * qb + 4, T)
-        S = O.block_scores(qb, P.q_idx(t0, t1), P.w(t0, t1), k_idx[:t1])
-        osel, ocnt = O.select(qb, S)
-        g = sel[qb].cpu().numpy()
-        gc = int(cnt[qb])
-        n_diff += check_selection(g, gc, osel, ocnt, S, qb, BUDGET, f"mean pool qb={qb}")
-        want = _oracle_block_outputs(O, P, qb, g, gc)
-        got = out[t0:t1].cpu().numpy()
-        for i, (o, l) in enumerate(want):
-            check_outputs(got[i], o, f"mean pool t={t0 + i}")
-    print(f"mean pool 1M: sampled rows differ from the oracle selection in {n_diff} near-tie blocks")
+    qbs = _sample_blocks(nqb, seed=7, n=64)
+    n_diff = _check_sampled_blocks(O, P, qbs, sel, cnt, out, None, "mean pool 1M")
+    print(f"mean pool 1M: {len(qbs)} sampled query blocks, {n_diff} near-tie selection differences")
 
 
 def _decode_full_setup(B, L, aggregation=0):
@@ -320,8 +277,8 @@ def test_verify_full_size_sampled():
     out, sel, lse = out.cpu().numpy(), sel.cpu().numpy(), lse.cpu().numpy()
     new_krot = st["kc"][:, L:L + m].cpu().numpy()
     del st, ws
+    assert L % 4 == 0
     O = oracle.Oracle(oracle.params(budget=BUDGET))
-    ring_q, ring_w = np.zeros((0, 4, 128), np.uint16), np.zeros((0, 4), np.uint16)
     for b in (0, 33, 63):
         nb = {k: v[b] for k, v in new.items()}
         kid = np.concatenate([D.cache_kidx(b), nb["k_idx"]])
@@ -338,7 +295,9 @@ def test_verify_full_size_sampled():
                 assert np.array_equal(sel[b, i], g)
                 kc = np.concatenate([kc_full, new_krot[b, :i]])
                 vc = np.concatenate([vc_full, nb["v"][:i]])
-                _, _, oo, ol = O.decode(t, kc, vc, kid[:t], ring_q, ring_w, nb["q"][i], nb["k"][i], nb["v"][i],
-                                        nb["q_idx"][i], kid[t], nb["w"][i], sel_in=g, cnt_in=gc)
+                # block-mates 4 qb .. t - 1 (new tokens, as L % 4 == 0)
+                m0 = 4 * qb - L
+                _, _, oo, ol = O.decode(t, kc, vc, kid[:t], nb["q_idx"][m0:i], nb["w"][m0:i], nb["q"][i], nb["k"][i],
+                                        nb["v"][i], nb["q_idx"][i], kid[t], nb["w"][i], sel_in=g, cnt_in=gc)
                 check_outputs(out[b, i], oo, f"verify b={b} t={t}")
                 assert np.allclose(lse[b, i], ol, atol=1e-2), f"verify b={b} t={t} lse"

@@ -24,6 +24,13 @@ def _lib():
     qsa.load()
 
 
+@pytest.fixture
+def automatic_splits_after():
+    """Back to the automatic split-KV choice once the test is done."""
+    yield
+    qsa.qsa_set_decode_splits(0)
+
+
 def _new(st):
     return {k: np.stack([st.hosts[b][k][st.lens[b]] for b in range(st.B)]) for k in
             ("q", "k", "v", "q_idx", "k_idx", "w")}
@@ -81,11 +88,11 @@ def test_speculative_round_vs_oracle(budget):
             assert np.allclose(lse[b], ol, atol=1e-2), f"b={b} step={s} lse"
 
 
-def test_reuse_at_same_token_equals_decode(monkeypatch):
+def test_reuse_at_same_token_equals_decode(automatic_splits_after):
     """Reusing the row a decode step selected, at that same token, attends the
     same blocks in the same order: bit-identical output and lse (one KV range,
     so both take the same summation order)."""
-    monkeypatch.setenv("QSA_DECODE_SPLITS", "1")
+    qsa.qsa_set_decode_splits(1)
     budget = 64
     L_list = [1001, 2048, 4093]
     probs = [Q.PrefillProblem(T=L + 1, seed=520 + b, n_plant=4) for b, L in enumerate(L_list)]

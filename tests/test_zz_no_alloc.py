@@ -36,26 +36,47 @@ def test_decode_noalloc_matches_workspace_decode():
     b = [t.clone() for t in a]                 # identical caches for the no-alloc path
     ws = qsa.workspace(qsa.qsa_decode_workspace_size(p, B, max_len))
     seqs = [D.tokens(i) for i in range(B)]
+    # every tensor of both calls exists before the first no-alloc call, so
+    # nothing in between can allocate device memory
+    xs, outs = [], []
+    for s in range(2):
+        t = L + s
+        xs.append({k: torch.from_numpy(np.ascontiguousarray(np.stack([getattr(seqs[i], k)(t, t + 1)[0]
+                                                                       for i in range(B)]))).cuda()
+                   for k in ("q", "k", "v", "q_idx", "k_idx", "w")})
+        outs.append(dict(out_ws=torch.empty((B, 24, 256), dtype=torch.uint16, device="cuda"),
+                         out_na=torch.empty((B, 24, 256), dtype=torch.uint16, device="cuda"),
+                         sel_ws=torch.empty((B, budget), dtype=torch.int32, device="cuda"),
+                         sel_na=torch.empty((B, budget), dtype=torch.int32, device="cuda"),
+                         lse_ws=torch.empty((B, 24), dtype=torch.float32, device="cuda"),
+                         lse_na=torch.empty((B, 24), dtype=torch.float32, device="cuda")))
+    torch.cuda.synchronize()
+    free_after_first = None
     for s in range(2):                         # two calls in a row
         t = L + s
-        x = {k: torch.from_numpy(np.ascontiguousarray(np.stack([getattr(seqs[i], k)(t, t + 1)[0]
-                                                                 for i in range(B)]))).cuda()
-             for k in ("q", "k", "v", "q_idx", "k_idx", "w")}
-        out_ws = torch.empty((B, 24, 256), dtype=torch.uint16, device="cuda")
-        out_na = torch.empty_like(out_ws)
-        sel_ws = torch.empty((B, budget), dtype=torch.int32, device="cuda")
-        sel_na = torch.empty_like(sel_ws)
-        qsa.qsa_decode(p, B, max_len, [t] * B, *a, x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], x["w"], out_ws,
-                       sel_ws, None, ws)
+        x, o = xs[s], outs[s]
+        qsa.qsa_decode(p, B, max_len, [t] * B, *a, x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], x["w"],
+                       o["out_ws"], o["sel_ws"], o["lse_ws"], ws)
         qsa.qsa_decode_noalloc(p, B, max_len, [t] * B, *b, x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], x["w"],
-                               out_na, sel_na, None)
+                               o["out_na"], o["sel_na"], o["lse_na"])
         torch.cuda.synchronize()
+        free_now, _ = torch.cuda.mem_get_info()
+        if s == 0:
+            free_after_first = free_now          # the first call may map the fixed array
+        else:
+            assert free_now == free_after_first, "the second no-alloc call changed free device memory"
         assert qsa.qsa_check_device_error(ws) == 0
-        assert torch.equal(sel_ws, sel_na)
-        g = Q.bf16_to_f64(out_na.cpu().numpy())
-        w = Q.bf16_to_f64(out_ws.cpu().numpy())
+        assert qsa.qsa_decode_noalloc_check_error() == 0
+        # the same kernels with the same split on the same inputs: identical
+        assert torch.equal(o["sel_ws"], o["sel_na"])
+        assert torch.equal(o["out_ws"], o["out_na"])
+        assert torch.equal(o["lse_ws"], o["lse_na"])
+        # and within the tolerance the other tests use (a non-empty output)
+        g = Q.bf16_to_f64(o["out_na"].cpu().numpy())
+        w = Q.bf16_to_f64(o["out_ws"].cpu().numpy())
         assert np.abs(g - w).max() <= OUT_MAX_ABS
         assert np.linalg.norm(g - w) <= OUT_REL_L2 * np.linalg.norm(w)
+        assert np.linalg.norm(w) > 0
     for ta, tb in zip(a, b):                   # both paths appended the same tokens
         assert torch.equal(ta, tb)
 
