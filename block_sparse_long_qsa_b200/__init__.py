@@ -16,6 +16,7 @@ import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libqsa.so")
+LIB_DEBUG_PATH = os.path.join(_PKG, "libqsa_debug.so")   # the debug build (tests of the failure handling)
 
 QSA_OK = 0
 _STATUS = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_UNSUPPORTED", 3: "QSA_ERR_MISALIGNED",
@@ -57,11 +58,35 @@ AGG_MEAN_POOL = 1
 _lib = None
 
 
+_libs: dict = {}
+_lib_path = None
+
+
 def load(path: str = LIB_PATH):
-    """Load libqsa.so and declare its signatures (raises if it is not built)."""
-    global _lib
+    """Load libqsa.so and declare its signatures (raises if it is not built).
+    The first library loaded serves every call of this module (see
+    use_library)."""
+    global _lib, _lib_path
     if _lib is not None:
         return _lib
+    _lib = _open(path)
+    _lib_path = path
+    return _lib
+
+
+def use_library(path: str) -> str | None:
+    """Route this module's calls to the library at ``path`` (e.g. the debug
+    build, libqsa_debug.so); returns the path that served them before."""
+    global _lib, _lib_path
+    prev = _lib_path
+    _lib = _open(path)
+    _lib_path = path
+    return prev
+
+
+def _open(path: str):
+    if path in _libs:
+        return _libs[path]
     if not os.path.exists(path):
         raise ImportError(f"{path} is missing: build it with `python -m block_sparse_long_qsa_b200._build` "
                           "(the QSA path has no non-CUDA fallback)")
@@ -100,7 +125,10 @@ def load(path: str = LIB_PATH):
     for f in EXPORTED:
         if f not in ("qsa_default_params", "qsa_status_string", "qsa_last_error"):
             getattr(L, f).restype = ctypes.c_int
-    _lib = L
+    if hasattr(L, "qsa_debug_inject"):        # the debug build only
+        L.qsa_debug_inject.argtypes = [i32]
+        L.qsa_debug_inject.restype = ctypes.c_int
+    _libs[path] = L
     return L
 
 
@@ -273,6 +301,21 @@ def qsa_check_device_error(ws, stream=None) -> int:
 def qsa_decode_noalloc_check_error(stream=None) -> int:
     """Device error word of qsa_decode_noalloc's fixed array (synchronises)."""
     return load().qsa_decode_noalloc_check_error(_stream(stream))
+
+
+# fault-injection codes of the debug build (include/qsa_debug.h)
+INJECT_INDEXER_STALL = 1
+INJECT_ATTENTION_STALL = 2
+INJECT_ATTENTION_BAD_BLOCK = 3
+
+
+def qsa_debug_inject(code: int):
+    """Arm a test fault for the next launch of the kernel it names (the debug
+    build, libqsa_debug.so, only)."""
+    L = load()
+    if not hasattr(L, "qsa_debug_inject"):
+        raise RuntimeError("qsa_debug_inject exists only in the debug build (use_library(LIB_DEBUG_PATH))")
+    _check(L.qsa_debug_inject(int(code)), "qsa_debug_inject")
 
 
 def qsa_set_decode_splits(n: int):

@@ -12,6 +12,12 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libqsa.so")
 BUILD_DIR = os.path.join(PKG, "_build")
+# the debug build (tests of the failure handling): the same sources with the
+# device bounds checks, the fault-injection hooks of include/qsa_debug.h and
+# a 20 ms limit on every device-side wait
+LIB_DEBUG = os.path.join(PKG, "libqsa_debug.so")
+BUILD_DIR_DEBUG = os.path.join(PKG, "_build_debug")
+DEBUG_FLAGS = ["-DQSA_DEBUG_BOUNDS", "-DQSA_DEBUG_HOOKS", "-DQSA_WAIT_TIMEOUT_NS=20000000ull"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -25,25 +31,28 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) + \
         glob.glob(os.path.join(INCLUDE, "*.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every csrc/*.cu to an object (in parallel) and link libqsa.so."""
-    if not force and not _stale():
-        return LIB
-    os.makedirs(BUILD_DIR, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Compile every csrc/*.cu to an object (in parallel) and link libqsa.so
+    (debug=True: libqsa_debug.so with the debug flags)."""
+    lib = LIB_DEBUG if debug else LIB
+    bdir = BUILD_DIR_DEBUG if debug else BUILD_DIR
+    if not force and not _stale(lib):
+        return lib
+    os.makedirs(bdir, exist_ok=True)
     procs, objs = [], []
     for src in sources():
-        obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
+        obj = os.path.join(bdir, os.path.basename(src) + ".o")
         objs.append(obj)
-        cmd = ["nvcc", *NVCC_FLAGS, "-c", src, "-o", obj]
+        cmd = ["nvcc", *NVCC_FLAGS, *(DEBUG_FLAGS if debug else []), "-c", src, "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         procs.append((src, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)))
@@ -56,11 +65,15 @@ def build(force: bool = False, verbose: bool = False) -> str:
             failed.append(src)
     if failed:
         raise RuntimeError(f"nvcc failed for: {failed}")
-    subprocess.run(["nvcc", "-shared", "-gencode", "arch=compute_100a,code=sm_100a", *objs, "-o", LIB],
+    subprocess.run(["nvcc", "-shared", "-gencode", "arch=compute_100a,code=sm_100a", *objs, "-o", lib],
                    check=True)
-    return LIB
+    return lib
+
+
+def build_all(force: bool = False) -> tuple[str, str]:
+    """The release library and the debug build."""
+    return build(force), build(force, debug=True)
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="-v" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug="--debug" in sys.argv))

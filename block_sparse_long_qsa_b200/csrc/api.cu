@@ -11,6 +11,7 @@
 
 #include "qsa.h"
 #include "qsa_kernels.h"
+#include "qsa_debug.h"
 
 namespace {
 
@@ -836,6 +837,26 @@ qsa_status qsa_trace_end(int32_t* kernel_ids, float* ms, int32_t capacity, int32
 }
 
 }  // extern "C"
+
+// Test hooks of the debug build (include/qsa_debug.h).
+#ifdef QSA_DEBUG_HOOKS
+namespace qsa {
+namespace {
+std::atomic<int> g_debug_inject{0};
+}  // namespace
+int take_debug_injection(int code) {
+  int expected = code;
+  return g_debug_inject.compare_exchange_strong(expected, 0) ? code : 0;
+}
+}  // namespace qsa
+
+extern "C" qsa_status qsa_debug_inject(int32_t code) {
+  if (code < QSA_INJECT_NONE || code > QSA_INJECT_ATTENTION_BAD_BLOCK) return QSA_ERR_INVALID_ARG;
+  qsa::g_debug_inject.store(code);
+  return QSA_OK;
+}
+#endif
+
 
 // ------------------------------------------------------------------ verify
 namespace {

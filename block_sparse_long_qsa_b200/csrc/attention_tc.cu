@@ -26,7 +26,10 @@
 //     exp2, row sum, P packed to bf16 and stored back into the S buffer's
 //     first 32 columns; at the end of an item each thread normalises and
 //     writes its 128 of the row's 256 dims, bf16, with the row's lse.
-//   * every mbarrier wait is bounded (timeout -> error word, clean exit).
+//   * every mbarrier wait is bounded (timeout -> error word, clean exit): on
+//     an abort every role leaves its loop, the loaders wait for their own
+//     cp.async copies and each MMA issuer for its last commit (a wait that
+//     ignores the abort) before TMEM is released.
 #include <cfloat>
 
 #include "qsa_device.cuh"
@@ -160,6 +163,7 @@ struct TcArgs {
   int n_split;
   float* part_o;
   float* part_lse;
+  int inject;               // debug build: fault-injection code (QSA_INJECT_*), else 0
 };
 
 // One work item = (query block, KV head) for prefill, (sequence, KV head,
@@ -354,8 +358,17 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
 #pragma unroll
           for (int kk = 0; kk < KPT; ++kk) {
             const int n = 4 * (k0 + kk) + w4;
+#ifdef QSA_DEBUG_HOOKS
+            // test hook: CTA 0's first tile names a block after the query
+            // block (never read: the causal test below masks it too)
+            if (a.inject == QSA_INJECT_ATTENTION_BAD_BLOCK && blockIdx.x == 0 && items_done == 0 && i == 0 &&
+                k0 + kk == 0)
+              kbv[kk] = (int)it.qb + 1;
+#endif
+            // a selected block is causal: -1 (padding) or 0 .. qb
+            const bool in_range = kbv[kk] == -1 || QSA_BOUNDS_OK(kbv[kk] >= 0 && kbv[kk] <= it.qb, a.err);
             const int j = 4 * kbv[kk] + w4;
-            valid[kk] = kbv[kk] >= 0 && j <= t_last32;
+            valid[kk] = in_range && kbv[kk] >= 0 && j <= t_last32;
             off[kk] = valid[kk] ? (size_t)(uint32_t)j * 512u : 0;
             cp_async16(dst0 + swz128(n, c32 & 7), k_lane + off[kk], valid[kk]);
           }
@@ -428,6 +441,11 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
               const uint64_t bd = umma_desc_k_sw128(k_base + c * CHUNK_KV + koff);
               umma_bf16(tmem + TM_S0 + 64 * b, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
             }
+#ifdef QSA_DEBUG_HOOKS
+            // test hook: CTA 0 never signals its first S, so the softmax warps
+            // time out and the CTA aborts
+            if (!(a.inject == QSA_INJECT_ATTENTION_STALL && blockIdx.x == 0 && s_count == 0))
+#endif
             tc_commit(&s_full[b]);
             tc_commit(&k_empty[stage]);
             if (i == n_tiles - 1) tc_commit(q_empty);
@@ -460,9 +478,11 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
         }
         ++items_done;
       }
+      // every MMA this thread issued has retired before TMEM is released
+      // (also after an abort: a wait that ignores the abort flag)
       uint64_t* done = &mma_done[s_role ? 0 : 1];
       tc_commit(done);
-      mbar_wait(done, 0, abort_flag, a.err);
+      mbar_wait_drain(done, 0, a.err);
     }
   } else if (warp == W_SOFT || warp == W_SOFT + 1 || warp == W_SOFT2 || warp == W_SOFT2 + 1) {
     // ---------------------------------------------------------------- softmax
@@ -731,6 +751,8 @@ cudaError_t launch_sparse_attn_prefill_tc(int64_t T, const uint16_t* q, const ui
   a.T = T; a.q_tok0 = q_tok0; a.q = q; a.k_rot = k_rot; a.v = v; a.cs = cs; a.sel = sel; a.cnt = cnt; a.budget = budget;
   a.qb_begin = qb_begin; a.n_qb = qb_end - qb_begin; a.scale_log2 = scale_log2; a.out = out; a.lse = lse;
   a.err = err; a.n_split = 1;
+  a.inject = take_debug_injection(QSA_INJECT_ATTENTION_STALL);
+  if (a.inject == 0) a.inject = take_debug_injection(QSA_INJECT_ATTENTION_BAD_BLOCK);
   return launch_tc<false>(a, 2 * (qb_end - qb_begin), num_sms, stream);
 }
 

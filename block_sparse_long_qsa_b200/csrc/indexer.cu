@@ -25,7 +25,10 @@
 //     8 warps per TMEM accumulator (tcgen05.ld -> ReLU, head weights, block
 //     max -> fp32 scores), each 32-column load in flight behind the previous chunk.
 //   * Every mbarrier wait is bounded; on timeout the CTA records
-//     QSA_ERR_DEVICE_TIMEOUT, drains and exits.
+//     QSA_ERR_DEVICE_TIMEOUT and every role leaves its loop; before TMEM is
+//     released the MMA thread waits for its last commit and the producer for
+//     its last TMA loads (waits that ignore the abort), so nothing is in
+//     flight when the CTA exits.
 #include <type_traits>
 
 #include "qsa_device.cuh"
@@ -103,7 +106,7 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                        const uint16_t* __restrict__ w, float* __restrict__ S, int64_t ld,
                        float* __restrict__ segmax, int64_t ld_seg, int64_t T, int64_t q_tok0, int64_t qb_begin,
                        int64_t qb_end,
-                       float scale, uint32_t* err) {
+                       float scale, uint32_t* err, int inject) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* sQ = smem;
   uint8_t* sK = smem + OFF_K;
@@ -162,6 +165,11 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     float* sWf = reinterpret_cast<float*>(smem + OFF_W);
     Iter it; it.begin(&sch, u0, u1);
     int stage = 0; uint32_t ephase = 1; uint32_t qcount = 0;
+    // for the drain at exit: bit s of `issued` / `par` = a load was issued into
+    // stage s / the full-barrier phase parity of the last one; the same for
+    // the Q tile (bit 31 of last_qpar: none issued)
+    uint32_t issued = 0, par = 0;
+    uint32_t last_qpar = 1u << 31;
     for (; it.valid(); it.next()) {
       if (it.first_of_tile(u0)) {
         bool ok = qcount == 0 || mbar_wait(qempty, (qcount - 1) & 1, abort_flag, err);
@@ -190,6 +198,7 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         }
         __syncwarp();
         if (lane == 0) {
+          last_qpar = qcount & 1;
           mbar_arrive_expect_tx(qfull, Q_BYTES);
           for (int hf = 0; hf < 2; ++hf)
             for (int kc = 0; kc < 2; ++kc)
@@ -202,6 +211,9 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
       if (lane == 0) {
         ok = mbar_wait(&empty[stage], ephase, abort_flag, err);
         if (ok) {
+          // the load completes phase (wraps of this stage) of full[stage]
+          issued |= 1u << stage;
+          par = (par & ~(1u << stage)) | ((ephase ^ 1u) << stage);
           mbar_arrive_expect_tx(&full[stage], K_STAGE_BYTES);
           for (int kc = 0; kc < 2; ++kc)
             tma_load_2d(sK + stage * K_STAGE_BYTES + kc * K_SUB_BYTES, &tm_k, kc * 64, (int32_t)(KT * it.kt),
@@ -211,6 +223,16 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
       if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
       if (++stage == STAGES) { stage = 0; ephase ^= 1; }
     }
+    // Drain: every TMA load this warp issued has landed before the CTA exits
+    // (after an abort some were never consumed).  A stage's full barrier
+    // cannot move past its last issued load, so the parity test is exact.
+    if (lane == 0) {
+#pragma unroll
+      for (int s = 0; s < STAGES; ++s)
+        if ((issued >> s) & 1u) mbar_wait_drain(&full[s], (par >> s) & 1u, err);
+      if (last_qpar <= 1u) mbar_wait_drain(qfull, last_qpar, err);
+    }
+    __syncwarp();
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
     if (lane == 0) {
@@ -238,6 +260,11 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             const uint64_t bd = umma_desc_k_sw128(b_base + (k >> 2) * Q_SUB_BYTES + koff);
             umma_bf16(tmem + hf * 256, ad, bd, idesc, k > 0 ? 1u : 0u);
           }
+#ifdef QSA_DEBUG_HOOKS
+          // test hook: CTA 0 never signals its first accumulator, so that
+          // accumulator's epilogue warps time out and the CTA aborts
+          if (!(inject == QSA_INJECT_INDEXER_STALL && blockIdx.x == 0 && acc_use[0] == 0 && hf == 0))
+#endif
           tc_commit(&accfull[hf]);
           ++acc_use[hf];
         }
@@ -246,9 +273,9 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         if (it.tile_ends_here()) tc_commit(qempty);
         if (++stage == STAGES) { stage = 0; fphase ^= 1; }
       }
-      // all issued MMAs retired before TMEM is released
+      // all issued MMAs retired before TMEM is released (also after an abort)
       tc_commit(done);
-      mbar_wait(done, 0, abort_flag, err);
+      mbar_wait_drain(done, 0, err);
     }
   } else {
     // ----------------------------------------------------------- epilogue
@@ -365,7 +392,7 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             const int nb = qe - qbf < 8 ? qe - qbf : 8;
   #pragma unroll
             for (int b = 0; b < 8; ++b) {
-              if (b < nb && kb <= qbf + b) srow[b * ld] = m[b] * scale;
+              if (b < nb && kb <= qbf + b && QSA_BOUNDS_OK(kb < ld && qbf + b >= qb0, err)) srow[b * ld] = m[b] * scale;
             }
             if (segmax != nullptr) {
               // segment maxima over 8 key blocks = 8 lanes (bits 0..2): three
@@ -382,7 +409,7 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
               const int seg = (key0 + (lane & ~7)) >> 3;
               const int qb = qbf + qs_seg;
               // only segments starting at or before the row's own block: seg <= qb / 8 < ld_seg
-              if (qb < qe && seg <= (qb >> 3)) g_row[seg] = sm * scale;
+              if (qb < qe && seg <= (qb >> 3) && QSA_BOUNDS_OK(seg < ld_seg && qb >= qb0, err)) g_row[seg] = sm * scale;
             }
           } else {
             // max over the 4 keys of the key block (lanes 4k .. 4k+3) as a transposing
@@ -402,7 +429,7 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
               const float keep = lb ? n4[i + 2] : n4[i];
               val[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
               const int qb = qbf + qs + i;
-              if (qb < qe && kb <= qb) s_rows[i * ld + kb] = val[i] * scale;
+              if (qb < qe && kb <= qb && QSA_BOUNDS_OK(kb < ld && qb >= qb0, err)) s_rows[i * ld + kb] = val[i] * scale;
             }
             if (segmax != nullptr) {
               // segment maxima: max over the 8 key blocks of this warp's 32 keys
@@ -417,7 +444,8 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 const int seg = key0 >> 5;
                 const int qb = qbf + qs_seg;
                 // only segments starting at or before the row's own block: seg <= qb / 8 < ld_seg
-                if (qb < qe && seg <= (qb >> 3)) g_row[seg] = sm * scale;
+                if (qb < qe && seg <= (qb >> 3) && QSA_BOUNDS_OK(seg < ld_seg && qb >= qb0, err))
+                  g_row[seg] = sm * scale;
               }
             }
           }
@@ -474,12 +502,13 @@ cudaError_t launch_indexer_prefill(const CUtensorMap& tm_q, const CUtensorMap& t
     units += tl / key_tokens + 1;
   }
   const int grid = (int)(units < num_sms ? units : num_sms);
+  const int inject = take_debug_injection(QSA_INJECT_INDEXER_STALL);
   if (mean_pool)
     indexer_prefill_kernel<true><<<grid, THREADS, SMEM_BYTES, stream>>>(tm_q, tm_k, w, S, ld, segmax, ld_seg, T,
-                                                                        q_tok0, qb_begin, qb_end, scale, err);
+                                                                        q_tok0, qb_begin, qb_end, scale, err, inject);
   else
     indexer_prefill_kernel<false><<<grid, THREADS, SMEM_BYTES, stream>>>(tm_q, tm_k, w, S, ld, segmax, ld_seg, T,
-                                                                         q_tok0, qb_begin, qb_end, scale, err);
+                                                                         q_tok0, qb_begin, qb_end, scale, err, inject);
   return cudaGetLastError();
 }
 

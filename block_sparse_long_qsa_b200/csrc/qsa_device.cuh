@@ -77,6 +77,35 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Wait used on the way out of a kernel for work this thread already issued
+// (MMAs behind a tcgen05.commit, TMA copies behind an expect_tx).  That work
+// completes on its own, so the wait ignores the abort flag; it gives up only
+// after QSA_WAIT_TIMEOUT_NS (recording a timeout).  A CTA drains this way
+// before it releases TMEM or exits, so nothing it issued is still writing
+// TMEM or its shared memory when the SM is handed to the next CTA.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint32_t* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0u && globaltimer() - t0 > QSA_WAIT_TIMEOUT_NS) {
+      report_error(err, QSA_ERR_DEVICE_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// ------------------------------------------------------------ debug build --
+// QSA_DEBUG_BOUNDS (debug build only): index-range checks on the attention
+// gathers and the indexer's score stores.  A failed check records
+// QSA_ERR_DEVICE_BOUNDS and the access is skipped.  Release builds compile
+// no check.
+#ifdef QSA_DEBUG_BOUNDS
+#define QSA_BOUNDS_OK(cond, err) ((cond) ? true : (report_error((err), QSA_ERR_DEVICE_BOUNDS), false))
+#else
+#define QSA_BOUNDS_OK(cond, err) true
+#endif
+
 // -------------------------------------------------------------------- TMA --
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

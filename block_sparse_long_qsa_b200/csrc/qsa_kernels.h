@@ -4,7 +4,19 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "qsa_debug.h"   // the fault-injection codes of the debug build's tests
+
 namespace qsa {
+
+// Debug build (QSA_DEBUG_HOOKS) only: returns `code` (a QSA_INJECT_* of
+// qsa_debug.h) if the fault injection that qsa_debug_inject armed is `code`,
+// disarming it (so it applies to one launch); otherwise 0.  Release builds
+// return 0 and compile no injection code.
+#ifdef QSA_DEBUG_HOOKS
+int take_debug_injection(int code);
+#else
+inline int take_debug_injection(int) { return 0; }
+#endif
 
 // RoPE angles of positions pos0 .. pos0+T-1: cs[t][i] = attn_factor * (cos a,
 // sin a), a = (pos0 + t) * inv_freq[i], i < 32, angle formed in fp64.

@@ -18,8 +18,8 @@ def lib():
     return qsa.load()
 
 
-def header_functions():
-    src = open(os.path.join(ROOT, "include", "qsa.h")).read()
+def header_functions(name="qsa.h"):
+    src = open(os.path.join(ROOT, "include", name)).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(qsa_[a-z_]+)\s*\(", src)))
 
@@ -30,6 +30,18 @@ def test_exports_every_declared_symbol(lib):
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(qsa.EXPORTED)
+
+
+def test_debug_build_exports_the_hooks():
+    """The debug build (libqsa_debug.so) exports every symbol of qsa.h and
+    the test hooks of qsa_debug.h; the release library has no hook."""
+    path = _build.build(debug=True)
+    D = ctypes.CDLL(path)
+    for n in header_functions() + header_functions("qsa_debug.h"):
+        assert hasattr(D, n), n
+    R = ctypes.CDLL(_build.build())
+    for n in header_functions("qsa_debug.h"):
+        assert not hasattr(R, n), n
 
 
 def test_status_strings(lib):

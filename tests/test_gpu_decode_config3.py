@@ -62,7 +62,8 @@ def test_decode_32_appending_steps_64x256k():
         qsa.qsa_decode(p, B, max_len, [L + s] * B, kc, vc, ic, ring, wring, x["q"], x["k"], x["v"], x["q_idx"],
                        x["k_idx"], x["w"], out, sel, lse, ws)
         if s in CHECK_STEPS:
-            got[s] = (out[idx].cpu().numpy(), sel[idx].cpu().numpy(), lse[idx].cpu().numpy())
+            got[s] = (out.view(torch.int16)[idx].cpu().numpy().view(np.uint16), sel[idx].cpu().numpy(),
+                      lse[idx].cpu().numpy())
     torch.cuda.synchronize()
     assert qsa.qsa_check_device_error(ws) == 0
     # every sequence appended all 32 tokens: the last appended indexer key

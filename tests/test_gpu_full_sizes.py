@@ -69,7 +69,7 @@ def _check_sampled_blocks(O, P, qbs, sel, cnt, out, lse, what, k_idx=None):
     sel_h = sel[torch.tensor(qbs, device=sel.device)].cpu().numpy()
     cnt_h = cnt[torch.tensor(qbs, device=cnt.device)].cpu().numpy()
     rows = torch.cat([torch.arange(4 * q, min(4 * q + 4, T)) for q in qbs]).to(out.device)
-    out_h = out[rows].cpu().numpy()
+    out_h = out.view(torch.int16)[rows].cpu().numpy().view(np.uint16)   # no uint16 gather on CUDA
     lse_h = lse[rows].cpu().numpy() if lse is not None else None
     first = {}
     n = 0
