@@ -23,7 +23,8 @@ class Params(ctypes.Structure):
                 ("idx_dim", ctypes.c_int32), ("block", ctypes.c_int32), ("budget", ctypes.c_int32),
                 ("softmax_scale", ctypes.c_double), ("aggregation", ctypes.c_int32),
                 ("yarn_factor", ctypes.c_double), ("yarn_original_max", ctypes.c_double),
-                ("yarn_beta_fast", ctypes.c_double), ("yarn_beta_slow", ctypes.c_double)]
+                ("yarn_beta_fast", ctypes.c_double), ("yarn_beta_slow", ctypes.c_double),
+                ("idx_rope", ctypes.c_int32), ("idx_exact", ctypes.c_int32), ("idx_pos0", ctypes.c_int64)]
 
 
 # block-score aggregation: max over causal token pairs, or mean-pooled block keys
@@ -33,9 +34,11 @@ AGG_MEAN_POOL = 1
 
 def params(budget=512, block=4, n_q_heads=24, n_kv_heads=2, head_dim=256, rope_dim=64, rope_theta=1e7,
            idx_heads=4, idx_dim=128, softmax_scale=0.0, aggregation=AGG_TOKEN_MAX, yarn_factor=0.0,
-           yarn_original_max=262144.0, yarn_beta_fast=32.0, yarn_beta_slow=1.0) -> Params:
+           yarn_original_max=262144.0, yarn_beta_fast=32.0, yarn_beta_slow=1.0, idx_rope=0, idx_exact=0,
+           idx_pos0=0) -> Params:
     return Params(n_q_heads, n_kv_heads, head_dim, rope_dim, rope_theta, idx_heads, idx_dim, block, budget,
-                  softmax_scale, aggregation, yarn_factor, yarn_original_max, yarn_beta_fast, yarn_beta_slow)
+                  softmax_scale, aggregation, yarn_factor, yarn_original_max, yarn_beta_fast, yarn_beta_slow,
+                  idx_rope, idx_exact, idx_pos0)
 
 
 def build(force: bool = False) -> str:

@@ -55,6 +55,18 @@ typedef struct {
   double yarn_original_max;
   double yarn_beta_fast;  /* 32 (not on the pages: the method's usual value) */
   double yarn_beta_slow;  /* 1 */
+  /* Mean-pooled indexer only ([PT] §QSA: the block's keys are compressed
+   * before the positional step and the compressed key gets one block-start
+   * position).  idx_rope = 1: the indexer queries are rotated at their token
+   * positions and the compressed key of block b at its start position
+   * 4b, with the layer's RoPE (dims [0, rope_dim), as for Q and K); token t
+   * sits at position idx_pos0 + t.  idx_exact = 1: the compressed and rotated
+   * indexer operands are kept in fp64 instead of being rounded to bf16 (a
+   * diagnostic reading; the default rounds them, as the model's tensors are
+   * bf16). */
+  int32_t idx_rope;
+  int32_t idx_exact;
+  int64_t idx_pos0;
 } oracle_params;
 
 static double bf16_to_f64(uint16_t h) {
@@ -127,32 +139,65 @@ double oracle_token_score(const oracle_params* p, const uint16_t* q_t, const uin
   return s / sqrt((double)p->idx_dim);
 }
 
-/* fp64 -> bf16 bit pattern, round to nearest even, subnormals included. */
-static uint16_t f64_to_bf16_rne(double x) {
-  union { double d; uint64_t u; } b;
-  b.d = x;
-  const uint16_t sign = (uint16_t)((b.u >> 48) & 0x8000u);
+/* fp64 -> bf16 bit pattern, rounded to the nearest bf16 value, ties to the
+ * one with an even last bit (IEEE round-to-nearest-even), subnormals
+ * included.  The bf16 values next to |x| are the multiples of the spacing
+ * u = 2^(e - 8) around it (|x| in [2^(e-1), 2^e); u = 2^-133 below the
+ * normal range): lo = floor(|x| / u) u and lo + u.  Both divisions by u and
+ * the products are exact in fp64 (powers of two). */
+static uint16_t bf16_round_nearest_even(double x) {
   const double a = fabs(x);
+  const uint16_t sign = signbit(x) ? 0x8000u : 0u;
   if (a == 0.0) return sign;
   int e;
-  frexp(a, &e);                                   /* a = m 2^e, m in [0.5, 1) */
-  const int unit = e - 8 > -133 ? e - 8 : -133;   /* weight of bf16's last bit */
-  const double v = ldexp(nearbyint(ldexp(a, -unit)), unit);
-  union { float f; uint32_t u; } c;
-  c.f = (float)v;                                 /* exact: <= 8 significant bits */
-  return (uint16_t)(sign | (c.u >> 16));
+  (void)frexp(a, &e);
+  const double u = ldexp(1.0, e - 8 > -133 ? e - 8 : -133);
+  const double n_lo = floor(a / u);                 /* lo = n_lo u, exact */
+  const double below = a - n_lo * u, above = (n_lo + 1.0) * u - a;
+  double n = n_lo;
+  if (above < below || (above == below && fmod(n_lo, 2.0) != 0.0)) n = n_lo + 1.0;
+  union { float f; uint32_t u32; } c;
+  c.f = (float)(n * u);                             /* exact: a bf16 value */
+  return (uint16_t)(sign | (c.u32 >> 16));
+}
+
+/* RoPE of the first rope_dim dims of an n-dim vector at position pos (the
+ * same rotation as oracle_rope, for the indexer's 128-dim vectors). */
+static void rope_vec(const oracle_params* p, const double* x, int n, int64_t pos, double* y) {
+  const int half = p->rope_dim / 2;
+  const double m = rope_scale(p);
+  for (int c = 0; c < n; ++c) y[c] = x[c];
+  for (int i = 0; i < half; ++i) {
+    const double a = (double)pos * rope_freq(p, i);
+    const double ca = cos(a), sa = sin(a);
+    y[i] = m * (x[i] * ca - x[i + half] * sa);
+    y[i + half] = m * (x[i + half] * ca + x[i] * sa);
+  }
+}
+
+/* The value an indexer operand takes: rounded to bf16 unless idx_exact. */
+static double idx_operand(const oracle_params* p, double v) {
+  return p->idx_exact ? v : bf16_to_f64(bf16_round_nearest_even(v));
 }
 
 /* Compressed key of block kb ([PT] §QSA: the keys of a micro-block are
- * mean-pooled into k-bar_b before any positional step; the indexer has no
- * positional encoding here, so no block position is added).  Mean over the
+ * mean-pooled into k-bar_b before the positional step).  Mean over the
  * block's n present keys: exact fp64 sum, one fp64 division by n, one
- * rounding to bf16 (the indexer's operands are bf16). */
+ * rounding to bf16 (the model's tensors are bf16; not with idx_exact).  With
+ * idx_rope the compressed key then gets the block's start position
+ * idx_pos0 + kb r (rotated, then rounded to bf16 unless idx_exact). */
 static void mean_key(const oracle_params* p, const uint16_t* k_idx, int64_t kb, int n, double* kbar) {
+  double mean[512];
   for (int c = 0; c < p->idx_dim; ++c) {
     double sum = 0.0;
     for (int i = 0; i < n; ++i) sum += bf16_to_f64(k_idx[(kb * p->block + i) * p->idx_dim + c]);
-    kbar[c] = bf16_to_f64(f64_to_bf16_rne(sum / (double)n));
+    mean[c] = idx_operand(p, sum / (double)n);
+  }
+  if (p->idx_rope) {
+    rope_vec(p, mean, p->idx_dim, p->idx_pos0 + kb * p->block, kbar);
+    for (int c = 0; c < p->idx_dim; ++c) kbar[c] = idx_operand(p, kbar[c]);
+  } else {
+    for (int c = 0; c < p->idx_dim; ++c) kbar[c] = mean[c];
   }
 }
 
@@ -171,15 +216,31 @@ void oracle_block_scores(const oracle_params* p, int64_t qb, int n_present, cons
      * k-bar of the own block averages its present keys (the own block is
      * always selected, so this entry never decides a selection) */
     double kbar[512];
+    /* the indexer queries of the block's present tokens, rotated at their
+     * positions with idx_rope (rounded to bf16 unless idx_exact) */
+    double* qv = (double*)malloc(sizeof(double) * (size_t)n_present * p->idx_heads * p->idx_dim);
+    double x[512];
+    for (int i = 0; i < n_present; ++i)
+      for (int h = 0; h < p->idx_heads; ++h) {
+        const uint16_t* q_th = q_blk + ((int64_t)i * p->idx_heads + h) * p->idx_dim;
+        double* dst = qv + ((int64_t)i * p->idx_heads + h) * p->idx_dim;
+        for (int c = 0; c < p->idx_dim; ++c) x[c] = bf16_to_f64(q_th[c]);
+        if (p->idx_rope) {
+          rope_vec(p, x, p->idx_dim, p->idx_pos0 + qb * r + i, dst);
+          for (int c = 0; c < p->idx_dim; ++c) dst[c] = idx_operand(p, dst[c]);
+        } else {
+          for (int c = 0; c < p->idx_dim; ++c) dst[c] = x[c];
+        }
+      }
     for (int64_t kb = 0; kb <= qb; ++kb) {
       mean_key(p, k_idx, kb, kb == qb ? n_present : r, kbar);
       double best = -INFINITY;
       for (int i = 0; i < n_present; ++i) {
-        const uint16_t* q_t = q_blk + (int64_t)i * p->idx_heads * p->idx_dim;
+        const double* q_t = qv + (int64_t)i * p->idx_heads * p->idx_dim;
         double s = 0.0;
         for (int h = 0; h < p->idx_heads; ++h) {
           double dot = 0.0;
-          for (int c = 0; c < p->idx_dim; ++c) dot += bf16_to_f64(q_t[h * p->idx_dim + c]) * kbar[c];
+          for (int c = 0; c < p->idx_dim; ++c) dot += q_t[h * p->idx_dim + c] * kbar[c];
           s += bf16_to_f64(w_blk[(int64_t)i * p->idx_heads + h]) * (dot > 0.0 ? dot : 0.0);
         }
         s /= sqrt((double)p->idx_dim);
@@ -187,6 +248,7 @@ void oracle_block_scores(const oracle_params* p, int64_t qb, int n_present, cons
       }
       S[kb] = best;
     }
+    free(qv);
     return;
   }
   for (int64_t kb = 0; kb <= qb; ++kb) {

@@ -332,6 +332,77 @@ def pin_bf16_rounding_of_means(O):
     assert abs(S[1, 0] - max(wf[t, 0] for t in range(4, 8)) * (1.0 + 2 ** -7) / SQRT_D) < 1e-15
 
 
+def _rope_exact_rounded(x, pos, exact):
+    """Complex-form RoPE of a 128-dim indexer vector at pos (dims 0..63),
+    rounded to bf16 by exact rationals unless exact."""
+    y = _rope_complex(x, pos)
+    return y if exact else np.array([_bf16_rne_exact(v) for v in y])
+
+
+def _mean_pool_rope_scores(q_idx, w, k_idx, pos0, exact, r=4):
+    """Brute force of the block-start-position reading: block means (rounded
+    to bf16 unless exact) rotated at 4b + pos0 and queries rotated at t + pos0
+    (each rounded to bf16 unless exact), numpy dot products."""
+    from fractions import Fraction
+    T = q_idx.shape[0]
+    nb = (T + r - 1) // r
+    kf = Q.bf16_to_f64(k_idx)
+    kbar = np.zeros((nb, kf.shape[1]))
+    for b in range(nb):
+        rows = kf[b * r: min(b * r + r, T)]
+        mean = np.array([float(sum(Fraction(float(v)) for v in rows[:, c])) / rows.shape[0]
+                         for c in range(kf.shape[1])])
+        if not exact:
+            mean = np.array([_bf16_rne_exact(v) for v in mean])
+        kbar[b] = _rope_exact_rounded(mean, pos0 + r * b, exact)
+    qf = Q.bf16_to_f64(q_idx)
+    qr = np.stack([[_rope_exact_rounded(qf[t, h], pos0 + t, exact) for h in range(qf.shape[1])] for t in range(T)])
+    wf = Q.bf16_to_f64(w)
+    dots = np.einsum("thc,bc->thb", qr, kbar)
+    s = (wf[:, :, None] * np.maximum(dots, 0.0)).sum(1) / SQRT_D
+    S = np.full((nb, nb), np.nan)
+    for qb in range(nb):
+        S[qb, :qb + 1] = s[qb * r: min(qb * r + r, T), :qb + 1].max(axis=0)
+    return S
+
+
+def _idx_rope_oracle(O, exact=0, pos0=0):
+    import oracle as OR
+    return type(O)(OR.params(budget=O.P.budget, aggregation=OR.AGG_MEAN_POOL, idx_rope=1, idx_exact=exact,
+                             idx_pos0=pos0), O.L)
+
+
+def pin_idx_rope_brute(O):
+    """Mean pooling with the block-start position ([PT] §QSA): scores equal a
+    brute force on complex-form RoPE (key of block b at 4b, query of token t
+    at t, both offset by pos0), with and without the bf16 rounding of the
+    operands, ragged tails included."""
+    for T, seed, pos0 in ((7, 0, 0), (29, 1, 0), (41, 2, 1000), (13, 3, 262140)):
+        P = Q.PrefillProblem(T=T, seed=60 + seed, n_plant=2)
+        q_idx, w, k_idx = P.q_idx(), P.w(), P.k_idx()
+        for exact in (0, 1):
+            want = _mean_pool_rope_scores(q_idx, w, k_idx, pos0, exact)
+            got = _idx_rope_oracle(O, exact, pos0).index_scores(T, q_idx, w, k_idx)
+            m = ~np.isnan(want)
+            assert np.allclose(got[m], want[m], rtol=1e-9, atol=1e-12), (T, exact)
+
+
+def pin_idx_rope_relative_positions(O):
+    """With exact operands the scores depend on positions only through the
+    distance between the query token and the key block's start: a common
+    offset of every position leaves them unchanged, while the rotation itself
+    changes them (a key block scored at distance 0 and at distance 40 differ)."""
+    T = 48
+    P = Q.PrefillProblem(T=T, seed=71, n_plant=3)
+    q_idx, w, k_idx = P.q_idx(), P.w(), P.k_idx()
+    S0 = _idx_rope_oracle(O, 1, 0).index_scores(T, q_idx, w, k_idx)
+    S1 = _idx_rope_oracle(O, 1, 123457).index_scores(T, q_idx, w, k_idx)
+    m = ~np.isnan(S0)
+    assert np.allclose(S0[m], S1[m], rtol=1e-8, atol=1e-12)
+    Sp = _mean_pool_oracle(O).index_scores(T, q_idx, w, k_idx)
+    assert not np.allclose(S0[m], Sp[m], rtol=1e-3), "the rotation must change the scores"
+
+
 # ---------------------------------------------------------------- selection
 def _select_lexsort(S_row, qb, budget):
     if qb + 1 <= budget:

@@ -36,9 +36,16 @@ MUTANTS = [
     ("causal_attn_off_by_one", "if (j <= t) js[n++] = j;", "if (j <= t + 1) js[n++] = j;"),
     ("value_head_swap", "vv[(e * G + g) * d + c] = bf16_to_f64(v[(js[e] * G + g) * d + c]);",
      "vv[(e * G + g) * d + c] = bf16_to_f64(v[(js[e] * G + (G - 1 - g)) * d + c]);"),
-    ("mean_not_divided", "f64_to_bf16_rne(sum / (double)n)", "f64_to_bf16_rne(sum)"),
-    ("mean_not_rounded_to_bf16", "kbar[c] = bf16_to_f64(f64_to_bf16_rne(sum / (double)n));", "kbar[c] = sum / (double)n;"),
-    ("mean_ties_away_from_zero", "ldexp(nearbyint(ldexp(a, -unit)), unit)", "ldexp(round(ldexp(a, -unit)), unit)"),
+    ("mean_not_divided", "mean[c] = idx_operand(p, sum / (double)n);", "mean[c] = idx_operand(p, sum);"),
+    ("operands_not_rounded_to_bf16", "return p->idx_exact ? v : bf16_to_f64(bf16_round_nearest_even(v));",
+     "return v;"),
+    ("mean_ties_away_from_zero", "(above == below && fmod(n_lo, 2.0) != 0.0)", "(above == below)"),
+    ("idx_rope_key_at_block_end", "rope_vec(p, mean, p->idx_dim, p->idx_pos0 + kb * p->block, kbar);",
+     "rope_vec(p, mean, p->idx_dim, p->idx_pos0 + kb * p->block + p->block - 1, kbar);"),
+    ("idx_rope_query_not_rotated", "rope_vec(p, x, p->idx_dim, p->idx_pos0 + qb * r + i, dst);",
+     "rope_vec(p, x, p->idx_dim, 0, dst);"),
+    ("idx_rope_frequency", "const double a = (double)pos * rope_freq(p, i);",
+     "const double a = (double)pos * rope_freq(p, i + 1);"),
     ("mean_pool_relu_dropped", "s += bf16_to_f64(w_blk[(int64_t)i * p->idx_heads + h]) * (dot > 0.0 ? dot : 0.0);",
      "s += bf16_to_f64(w_blk[(int64_t)i * p->idx_heads + h]) * dot;"),
     ("reuse_own_block_not_forced", "  in_set[qb] = 1;\n", "\n"),
