@@ -33,7 +33,7 @@ EXPORTED = ["qsa_default_params", "qsa_status_string", "qsa_last_error", "qsa_in
 
 KERNEL_NAMES = {1: "rope_table", 2: "rope_k", 3: "indexer", 4: "select", 5: "attention", 6: "decode_append",
                 7: "decode_indexer", 8: "decode_attention", 9: "decode_combine",
-                10: "mean_pool_keys", 11: "verify_expand"}
+                10: "mean_pool_keys", 11: "verify_expand", 12: "idx_rope"}
 
 
 class QSAError(RuntimeError):
@@ -48,7 +48,8 @@ class qsa_params(ctypes.Structure):
                 ("idx_dim", ctypes.c_int32), ("block_size", ctypes.c_int32), ("budget_blocks", ctypes.c_int32),
                 ("softmax_scale", ctypes.c_float), ("aggregation", ctypes.c_int32),
                 ("yarn_factor", ctypes.c_double), ("yarn_original_max", ctypes.c_double),
-                ("yarn_beta_fast", ctypes.c_double), ("yarn_beta_slow", ctypes.c_double)]
+                ("yarn_beta_fast", ctypes.c_double), ("yarn_beta_slow", ctypes.c_double),
+                ("idx_rope", ctypes.c_int32)]
 
 
 # block-score aggregation (qsa_params.aggregation)
@@ -358,11 +359,12 @@ def workspace(nbytes: int, device="cuda") -> torch.Tensor:
 
 
 def prefill(q, k, v, q_idx, w, k_idx, budget: int = 512, pos0: int = 0, want_lse=True, want_sel=True,
-            want_krot=False, ws_bytes: int | None = None, stream=None, aggregation: int = AGG_TOKEN_MAX):
+            want_krot=False, ws_bytes: int | None = None, stream=None, aggregation: int = AGG_TOKEN_MAX,
+            idx_rope: int = 0):
     """Allocate outputs and a workspace, run qsa_prefill; returns a dict."""
     T = q.shape[0]
     dev = q.device
-    p = params(budget, aggregation=aggregation)
+    p = params(budget, aggregation=aggregation, idx_rope=idx_rope)
     mn, pref = qsa_prefill_workspace_size(p, T)
     ws = workspace(pref if ws_bytes is None else max(ws_bytes, mn), dev)
     nqb = (T + 3) // 4

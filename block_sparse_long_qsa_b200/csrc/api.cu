@@ -46,10 +46,14 @@ qsa_status check_params(const qsa_params* p) {
                                 p->yarn_beta_slow > 0.0 && p->yarn_beta_fast > p->yarn_beta_slow &&
                                 std::isfinite(p->yarn_beta_fast)))
     return QSA_ERR_INVALID_ARG;
+  if (p->idx_rope != 0 && p->idx_rope != 1) return QSA_ERR_INVALID_ARG;
+  if (p->idx_rope && p->aggregation != QSA_AGG_MEAN_POOL) return QSA_ERR_INVALID_ARG;
   return QSA_OK;
 }
 
 bool mean_pool(const qsa_params* p) { return p->aggregation == QSA_AGG_MEAN_POOL; }
+// the mean-pooled indexer with its block-start positions
+bool idx_rope(const qsa_params* p) { return p->idx_rope == 1; }
 // bytes of the mean-pooled keys of T tokens ([ceil(T/4)][128] bf16)
 size_t kbar_bytes(int64_t T) { return (size_t)((T + 3) / 4) * 256; }
 
@@ -215,16 +219,38 @@ qsa_status run_indexer(int64_t T, int64_t q_tok0, const uint16_t* q_idx, const u
 }
 
 // Compressed keys of tokens [0, T) into kbar (mean pooling only).
-qsa_status run_kbar(const uint16_t* k_idx, int64_t T, uint16_t* kbar, cudaStream_t st) {
+// With block-start positions (p->idx_rope) each compressed key is also
+// rotated at the position of its block's first token, pos0 + 4b.
+qsa_status run_kbar(const qsa_params* p, const uint16_t* k_idx, int64_t T, int64_t pos0, uint16_t* kbar,
+                    cudaStream_t st) {
+  if (idx_rope(p)) {
+    double f[32];
+    inv_freq(p, f);
+    return from_cuda(traced(QSA_KERNEL_KBAR, st, [&] {
+      return qsa::launch_kbar_rope(k_idx, T, pos0, f, rope_attn_factor(p), kbar, st);
+    }), "mean-pool launch");
+  }
   return from_cuda(traced(QSA_KERNEL_KBAR, st, [&] { return qsa::launch_kbar(k_idx, T, kbar, st); }),
                    "mean-pool launch");
 }
+// Indexer queries rotated at positions pos0 + t (block-start positions only).
+qsa_status run_idx_rope_q(const qsa_params* p, int64_t T, int64_t pos0, const uint16_t* q_idx, uint16_t* out,
+                          cudaStream_t st) {
+  double f[32];
+  inv_freq(p, f);
+  return from_cuda(traced(QSA_KERNEL_IDX_ROPE, st, [&] {
+    return qsa::launch_idx_rope_q(T, pos0, f, rope_attn_factor(p), q_idx, out, st);
+  }), "indexer RoPE launch");
+}
+// bytes of the rotated indexer queries of T tokens ([T][4][128] bf16)
+size_t qrot_bytes(int64_t T) { return (size_t)T * 1024; }
 
 // ------------------------------------------------------------ prefill layout
 struct PrefillLayout {
-  size_t cs, k_rot, sel, cnt, kbar, slab, total_fixed;
+  size_t cs, k_rot, sel, cnt, kbar, qrot, slab, total_fixed;
 };
-PrefillLayout prefill_layout(int64_t T, int budget, bool need_krot, bool need_sel, bool need_cnt, bool mean) {
+PrefillLayout prefill_layout(int64_t T, int budget, bool need_krot, bool need_sel, bool need_cnt, bool mean,
+                             bool rope_idx = false) {
   const int64_t nqb = (T + 3) / 4;
   PrefillLayout L;
   size_t off = HEADER_BYTES;
@@ -233,6 +259,7 @@ PrefillLayout prefill_layout(int64_t T, int budget, bool need_krot, bool need_se
   L.sel = off; off = align_up(off + (need_sel ? (size_t)nqb * budget * 4 : 0));
   L.cnt = off; off = align_up(off + (need_cnt ? (size_t)nqb * 4 : 0));
   L.kbar = off; off = align_up(off + (mean ? kbar_bytes(T) : 0));
+  L.qrot = off; off = align_up(off + (rope_idx ? qrot_bytes(T) : 0));
   L.slab = off;
   L.total_fixed = off;
   return L;
@@ -274,6 +301,7 @@ void qsa_default_params(qsa_params* p) {
   p->yarn_original_max = 262144.0;
   p->yarn_beta_fast = 32.0;
   p->yarn_beta_slow = 1.0;
+  p->idx_rope = 0;
 }
 
 const char* qsa_last_error(void) { return g_last_error; }
@@ -303,18 +331,25 @@ qsa_status qsa_index_scores(const qsa_params* p, int64_t T, const uint16_t* q_id
   if (qb_begin < 0 || qb_end < qb_begin || qb_end > nqb || ld < qb_end || ld % 4 != 0) return QSA_ERR_INVALID_ARG;
   if (!q_idx || !w || !k_idx || !scores) return QSA_ERR_INVALID_ARG;
   if (!aligned16(q_idx) || !aligned16(w) || !aligned16(k_idx) || !aligned16(scores)) return QSA_ERR_MISALIGNED;
-  const bool mp = mean_pool(p);
+  const bool mp = mean_pool(p), rope = idx_rope(p);
   if (mp && !ws) return QSA_ERR_INVALID_ARG;
-  if (ws && ws_bytes < HEADER_BYTES + (mp ? kbar_bytes(T) : 0)) return QSA_ERR_WORKSPACE_TOO_SMALL;
+  const size_t kbar_off = HEADER_BYTES, qrot_off = align_up(kbar_off + (mp ? kbar_bytes(T) : 0));
+  if (ws && ws_bytes < qrot_off + (rope ? qrot_bytes(T) : 0)) return QSA_ERR_WORKSPACE_TOO_SMALL;
   if (ws && !aligned16(ws)) return QSA_ERR_MISALIGNED;
   DevInfo di;
   if ((st = device_info(&di)) != QSA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t* err = static_cast<uint32_t*>(ws);
   if (err && cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaMemsetAsync");
-  uint16_t* kbar = mp ? reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + HEADER_BYTES) : nullptr;
-  if (kbar && (st = run_kbar(k_idx, T, kbar, s)) != QSA_OK) return st;
-  return run_indexer(T, 0, q_idx, w, k_idx, kbar, qb_begin, qb_end, scores, ld, nullptr, 0, err, di.num_sms, s);
+  uint16_t* kbar = mp ? reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + kbar_off) : nullptr;
+  if (kbar && (st = run_kbar(p, k_idx, T, 0, kbar, s)) != QSA_OK) return st;
+  const uint16_t* qi = q_idx;
+  if (rope) {   // token t at position t
+    uint16_t* qr = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + qrot_off);
+    if ((st = run_idx_rope_q(p, T, 0, q_idx, qr, s)) != QSA_OK) return st;
+    qi = qr;
+  }
+  return run_indexer(T, 0, qi, w, k_idx, kbar, qb_begin, qb_end, scores, ld, nullptr, 0, err, di.num_sms, s);
 }
 
 qsa_status qsa_index_workspace_size(const qsa_params* p, int64_t T, size_t* bytes) {
@@ -322,7 +357,7 @@ qsa_status qsa_index_workspace_size(const qsa_params* p, int64_t T, size_t* byte
   if (st != QSA_OK) return st;
   if (T <= 0 || !bytes) return QSA_ERR_INVALID_ARG;
   if (T > ((int64_t)1 << 24)) return QSA_ERR_UNSUPPORTED;
-  *bytes = HEADER_BYTES + (mean_pool(p) ? kbar_bytes(T) : 0);
+  *bytes = align_up(HEADER_BYTES + (mean_pool(p) ? kbar_bytes(T) : 0)) + (idx_rope(p) ? qrot_bytes(T) : 0);
   return QSA_OK;
 }
 
@@ -360,7 +395,7 @@ qsa_status qsa_prefill_workspace_size(const qsa_params* p, int64_t T, size_t* mi
   if (T > ((int64_t)1 << 24)) return QSA_ERR_UNSUPPORTED;
   const int64_t nqb = (T + 3) / 4;
   // worst case: the library keeps k_rot, sel and cnt itself
-  PrefillLayout L = prefill_layout(T, p->budget_blocks, true, true, true, mean_pool(p));
+  PrefillLayout L = prefill_layout(T, p->budget_blocks, true, true, true, mean_pool(p), idx_rope(p));
   const int64_t min_rows = nqb < MIN_ROWS ? nqb : MIN_ROWS;
   const size_t row_bytes = slab_row_bytes(nqb);
   if (min_bytes) *min_bytes = L.total_fixed + (size_t)min_rows * row_bytes;
@@ -388,7 +423,7 @@ qsa_status qsa_prefill(const qsa_params* p, int64_t T, int64_t pos0, const uint1
   const int budget = p->budget_blocks;
   const int64_t nqb = (T + 3) / 4;
   PrefillLayout L = prefill_layout(T, budget, k_rot_out == nullptr, sel_out == nullptr, cnt_out == nullptr,
-                                   mean_pool(p));
+                                   mean_pool(p), idx_rope(p));
   if (ws_bytes < L.total_fixed) return QSA_ERR_WORKSPACE_TOO_SMALL;
   const size_t slab_bytes = ws_bytes - L.total_fixed;
   const int64_t min_rows = nqb < MIN_ROWS ? nqb : MIN_ROWS;
@@ -415,7 +450,13 @@ qsa_status qsa_prefill(const qsa_params* p, int64_t T, int64_t pos0, const uint1
   if ((st = from_cuda(traced(QSA_KERNEL_ROPE_K, s, [&] { return qsa::launch_rope_k(T, k, cs, k_rot, s); }))) != QSA_OK)
     return st;
   uint16_t* kbar = mean_pool(p) ? reinterpret_cast<uint16_t*>(base + L.kbar) : nullptr;
-  if (kbar && (st = run_kbar(k_idx, T, kbar, s)) != QSA_OK) return st;
+  if (kbar && (st = run_kbar(p, k_idx, T, pos0, kbar, s)) != QSA_OK) return st;
+  const uint16_t* qi = q_idx;
+  if (idx_rope(p)) {   // the indexer queries rotated at their positions pos0 + t
+    uint16_t* qr = reinterpret_cast<uint16_t*>(base + L.qrot);
+    if ((st = run_idx_rope_q(p, T, pos0, q_idx, qr, s)) != QSA_OK) return st;
+    qi = qr;
+  }
   const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
   for (int64_t qb0 = 0; qb0 < nqb;) {
     const int64_t qb1 = chunk_end(qb0, nqb, slab_bytes);
@@ -423,7 +464,7 @@ qsa_status qsa_prefill(const qsa_params* p, int64_t T, int64_t pos0, const uint1
     const int64_t ld = round4(qb1);
     const int64_t ld_seg = round4((qb1 + 7) / 8);
     float* segmax = slab + (size_t)(qb1 - qb0) * ld;
-    if ((st = run_indexer(T, 0, q_idx, w, k_idx, kbar, qb0, qb1, slab, ld, segmax, ld_seg, err, di.num_sms, s)) !=
+    if ((st = run_indexer(T, 0, qi, w, k_idx, kbar, qb0, qb1, slab, ld, segmax, ld_seg, err, di.num_sms, s)) !=
         QSA_OK)
       return st;
     if ((st = from_cuda(traced(QSA_KERNEL_SELECT, s, [&] {
@@ -469,6 +510,7 @@ qsa_status qsa_prefill_cached_workspace_size(const qsa_params* p, int64_t L_old,
                                              size_t* pref_bytes) {
   qsa_status st = check_params(p);
   if (st != QSA_OK) return st;
+  if (idx_rope(p)) return QSA_ERR_UNSUPPORTED;   // block-start positions: prefill and decode only
   if (L_old < 0 || T_new <= 0) return QSA_ERR_INVALID_ARG;
   if (L_old + T_new > ((int64_t)1 << 24)) return QSA_ERR_UNSUPPORTED;
   const int64_t nkb = (L_old + T_new + 3) / 4, qbA = L_old / 4, nq = nkb - qbA;
@@ -491,6 +533,7 @@ qsa_status qsa_prefill_cached(const qsa_params* p, int64_t L_old, int64_t T_new,
                               int32_t* cnt_out, void* ws, size_t ws_bytes, void* stream) {
   qsa_status st = check_params(p);
   if (st != QSA_OK) return st;
+  if (idx_rope(p)) return QSA_ERR_UNSUPPORTED;   // block-start positions: prefill and decode only
   if (L_old < 0 || T_new <= 0) return QSA_ERR_INVALID_ARG;
   if (L_old + T_new > ((int64_t)1 << 24)) return QSA_ERR_UNSUPPORTED;
   const int64_t r = L_old % 4;
@@ -553,7 +596,7 @@ qsa_status qsa_prefill_cached(const qsa_params* p, int64_t L_old, int64_t T_new,
   // compressed keys of all cached and new tokens (mean pooling; the caches
   // now hold the new rows)
   uint16_t* kbar = mean_pool(p) ? reinterpret_cast<uint16_t*>(base + L.kbar) : nullptr;
-  if (kbar && (st = run_kbar(kidx_cache, T, kbar, s)) != QSA_OK) return st;
+  if (kbar && (st = run_kbar(p, kidx_cache, T, 0, kbar, s)) != QSA_OK) return st;
   const float scale_log2 = softmax_scale(p) * 1.4426950408889634f;
   for (int64_t qb0 = qbA; qb0 < nkb;) {
     const int64_t qb1 = chunk_end(qb0, nkb, slab_bytes);
@@ -583,7 +626,7 @@ qsa_status qsa_prefill_cached(const qsa_params* p, int64_t L_old, int64_t T_new,
 // ------------------------------------------------------------------ decode
 namespace {
 struct DecodeLayout {
-  size_t Ls, qbs, S, sel, sel_r, cnt, q_rot, part_o, part_lse, total;
+  size_t Ls, qbs, S, sel, sel_r, cnt, q_rot, part_o, part_lse, ring_rot, total;
   int64_t ld;
   int sel_r_ld;   // row stride of the merged reused selections
 };
@@ -603,6 +646,7 @@ DecodeLayout decode_layout(int B, int64_t max_len, int budget) {
   L.q_rot = off; off = align_up(off + (size_t)B * 24 * 256 * 2);
   L.part_o = off; off = align_up(off + (size_t)B * 2 * DECODE_MAX_SPLIT * 12 * 256 * 4);
   L.part_lse = off; off = align_up(off + (size_t)B * 2 * DECODE_MAX_SPLIT * 12 * 4);
+  L.ring_rot = off; off = align_up(off + (size_t)B * 4 * 4 * 128 * 2);
   L.total = off;
   return L;
 }
@@ -692,6 +736,9 @@ qsa_status decode_impl(const qsa_params* p, int32_t B, int64_t max_len, const in
   const int sel_ld = reuse ? L.sel_r_ld : budget;
   int32_t* cnt = reinterpret_cast<int32_t*>(base + L.cnt);
   uint16_t* q_rot = reinterpret_cast<uint16_t*>(base + L.q_rot);
+  // block-start positions: the append kernel writes the block-mates' indexer
+  // queries rotated at their positions here, and the decode indexer reads them
+  uint16_t* ring_rot = idx_rope(p) ? reinterpret_cast<uint16_t*>(base + L.ring_rot) : nullptr;
 
   if (cudaMemsetAsync(err, 0, 4, s) != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaMemsetAsync");
   double f[32];
@@ -702,14 +749,14 @@ qsa_status decode_impl(const qsa_params* p, int32_t B, int64_t max_len, const in
          return qsa::launch_decode_append(B, max_len, cache_len, Ls, qbs, f, rope_attn_factor(p), k_cache, v_cache,
                                           kidx_cache, qidx_ring, w_ring, q_new, k_new, v_new, q_idx_new, k_idx_new,
                                           w_new, q_rot, kbar_cache, kbar_len, sel_in, cnt_in, budget, sel_r, L.sel_r_ld,
-                                          cnt, err, s);
+                                          cnt, err, s, idx_rope(p), ring_rot);
        }))) != QSA_OK)
     return st;
   const float scale = 1.0f / std::sqrt(128.0f);
   if (!reuse) {
     if ((st = from_cuda(traced(QSA_KERNEL_DECODE_INDEXER, s, [&] {
-           return qsa::launch_decode_indexer(B, max_len, max_L, Ls, kidx_cache, kbar_cache, kbar_len, qidx_ring,
-                                             w_ring, S, L.ld, scale, s);
+           return qsa::launch_decode_indexer(B, max_len, max_L, Ls, kidx_cache, kbar_cache, kbar_len,
+                                             ring_rot ? ring_rot : qidx_ring, w_ring, S, L.ld, scale, s);
          }))) != QSA_OK)
       return st;
     if ((st = from_cuda(traced(QSA_KERNEL_SELECT, s, [&] {
@@ -783,7 +830,7 @@ qsa_status qsa_mean_pool_keys(const qsa_params* p, int64_t T, const uint16_t* k_
   if (!aligned16(k_idx) || !aligned16(kbar)) return QSA_ERR_MISALIGNED;
   DevInfo di;
   if ((st = device_info(&di)) != QSA_OK) return st;
-  return run_kbar(k_idx, T, kbar, static_cast<cudaStream_t>(stream));
+  return run_kbar(p, k_idx, T, 0, kbar, static_cast<cudaStream_t>(stream));
 }
 
 qsa_status qsa_check_device_error(void* ws, void* stream) {
@@ -897,6 +944,7 @@ VerifyLayout verify_layout(int B, int m, int64_t max_len, int budget) {
 qsa_status qsa_verify_workspace_size(const qsa_params* p, int32_t B, int32_t m, int64_t max_len, size_t* bytes) {
   qsa_status st = check_params(p);
   if (st != QSA_OK) return st;
+  if (idx_rope(p)) return QSA_ERR_UNSUPPORTED;   // block-start positions: prefill and decode only
   if (B <= 0 || m <= 0 || max_len <= 0 || !bytes) return QSA_ERR_INVALID_ARG;
   if (B > 4096 || m > VERIFY_MAX_M || max_len > ((int64_t)1 << 24)) return QSA_ERR_UNSUPPORTED;
   *bytes = verify_layout(B, m, max_len, p->budget_blocks).total;
@@ -911,6 +959,7 @@ qsa_status qsa_verify(const qsa_params* p, int32_t B, int32_t m, int64_t max_len
                       int32_t* sel_out, float* lse_out, void* ws, size_t ws_bytes, void* stream) {
   qsa_status st = check_params(p);
   if (st != QSA_OK) return st;
+  if (idx_rope(p)) return QSA_ERR_UNSUPPORTED;   // block-start positions: prefill and decode only
   if (B <= 0 || m <= 0 || max_len <= 0 || !cache_len) return QSA_ERR_INVALID_ARG;
   if (mean_pool(p) != (kbar_cache != nullptr)) return QSA_ERR_INVALID_ARG;   // the compressed keys go with mean pool
   if (kbar_cache && !aligned16(kbar_cache)) return QSA_ERR_MISALIGNED;

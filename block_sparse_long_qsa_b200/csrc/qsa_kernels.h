@@ -40,6 +40,14 @@ cudaError_t launch_indexer_prefill(const CUtensorMap& tm_q, const CUtensorMap& t
                                    int num_sms, cudaStream_t stream);
 // kbar[b] = bf16 round-to-nearest-even of the mean of k_idx rows 4b .. min(4b+4, T)-1.
 cudaError_t launch_kbar(const uint16_t* k_idx, int64_t T, uint16_t* kbar, cudaStream_t stream);
+// The mean-pooled indexer with block-start positions: kbar as launch_kbar,
+// then dims 0..63 rotated at position pos0 + 4b (fp64, rounded to bf16).
+cudaError_t launch_kbar_rope(const uint16_t* k_idx, int64_t T, int64_t pos0, const double* inv_freq_host,
+                             double attn_factor, uint16_t* kbar, cudaStream_t stream);
+// out[t] = q_idx[t] ([T][4][128]) with dims 0..63 of every head rotated at
+// position pos0 + t (fp64, rounded to bf16), dims 64..127 copied.
+cudaError_t launch_idx_rope_q(int64_t T, int64_t pos0, const double* inv_freq_host, double attn_factor,
+                              const uint16_t* q_idx, uint16_t* out, cudaStream_t stream);
 
 // Top-k block selection, one row per query block.  Row r covers query block
 // row_qb ? row_qb[r] : qb_begin + r, read from S + r * ld.  segmax (nullable,
@@ -70,7 +78,7 @@ cudaError_t launch_decode_append(int B, int64_t max_len, const int64_t* L_host, 
                                  const uint16_t* q_idx_new, const uint16_t* k_idx_new, const uint16_t* w_new,
                                  uint16_t* q_rot, uint16_t* kbar_cache, int64_t kbar_len, const int32_t* sel_in,
                                  const int32_t* cnt_in, int budget, int32_t* sel_r, int sel_r_ld, int32_t* cnt_r,
-                                 uint32_t* err, cudaStream_t s);
+                                 uint32_t* err, cudaStream_t s, bool idx_rope = false, uint16_t* ring_rot = nullptr);
 // kbar_cache (nullable, [B][kbar_len][128]): score the mean-pooled key blocks
 // (aggregation = mean pool) instead of the keys.
 cudaError_t launch_decode_indexer(int B, int64_t max_len, int64_t max_L, const int64_t* L_dev,

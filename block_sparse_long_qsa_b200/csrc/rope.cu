@@ -70,6 +70,68 @@ __global__ void rope_k_kernel(int64_t T, const uint4* __restrict__ k, const floa
   }
 }
 
+// Indexer queries of the mean-pooled indexer with block-start positions:
+// out[t][h] = q_idx[t][h] with dims 0..63 rotated at position pos0 + t
+// (pairs (i, i + 32); fp64 angle and rotation, rounded to bf16 once) and
+// dims 64..127 copied.  One thread per (token, pair i): the pair's angle
+// serves the 4 heads, and the thread copies one of the token's 32 16-byte
+// chunks of unrotated dims (head i / 8, chunk i % 8).
+__global__ void idx_rope_q_kernel(int64_t T, int64_t pos0, InvFreq inv, const uint16_t* __restrict__ q,
+                                  uint16_t* __restrict__ out) {
+  const int64_t n = T * 32;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = e >> 5;
+    const int i = (int)(e & 31);
+    double sa, ca;
+    sincos((double)(pos0 + t) * inv.f[i], &sa, &ca);
+    ca *= inv.scale;
+    sa *= inv.scale;
+    const uint16_t* src = q + t * 512;
+    uint16_t* dst = out + t * 512;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const double x = (double)bf16_bits_to_f32(src[h * 128 + i]), y = (double)bf16_bits_to_f32(src[h * 128 + i + 32]);
+      dst[h * 128 + i] = f64_to_bf16_rne(x * ca - y * sa);
+      dst[h * 128 + i + 32] = f64_to_bf16_rne(y * ca + x * sa);
+    }
+    const int h = i >> 3, c = i & 7;
+    reinterpret_cast<uint4*>(dst + h * 128 + 64)[c] = reinterpret_cast<const uint4*>(src + h * 128 + 64)[c];
+  }
+}
+
+// Compressed keys with block-start positions: kbar[b] = bf16 of the mean of
+// k_idx rows 4b .. min(4b + 4, T) - 1 (exact fp64 sum, one division), then
+// dims 0..63 rotated at position pos0 + 4b (fp64, rounded to bf16 once
+// more).  One thread per (block, j < 96): the pair (j, j + 32) for j < 32,
+// else the unrotated dim j + 32.
+__device__ __forceinline__ double kbar_mean_bf16(const uint16_t* __restrict__ rows, int n, int c) {
+  double sum = 0.0;
+  for (int r = 0; r < n; ++r) sum += (double)bf16_bits_to_f32(rows[r * 128 + c]);
+  return (double)bf16_bits_to_f32(f64_to_bf16_rne(sum / (double)n));
+}
+__global__ void kbar_rope_kernel(const uint16_t* __restrict__ k_idx, int64_t T, int64_t nkb, int64_t pos0, InvFreq inv,
+                                 uint16_t* __restrict__ kbar) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= nkb * 96) return;
+  const int64_t b = e / 96;
+  const int j = (int)(e - b * 96);
+  const int64_t t0 = 4 * b;
+  const int n = (int)(T - t0 < 4 ? T - t0 : 4);
+  const uint16_t* rows = k_idx + t0 * 128;
+  uint16_t* dst = kbar + b * 128;
+  if (j < 32) {
+    const double x = kbar_mean_bf16(rows, n, j), y = kbar_mean_bf16(rows, n, j + 32);
+    double sa, ca;
+    sincos((double)(pos0 + t0) * inv.f[j], &sa, &ca);
+    ca *= inv.scale;
+    sa *= inv.scale;
+    dst[j] = f64_to_bf16_rne(x * ca - y * sa);
+    dst[j + 32] = f64_to_bf16_rne(y * ca + x * sa);
+  } else {
+    dst[j + 32] = f64_to_bf16_rne(kbar_mean_bf16(rows, n, j + 32));
+  }
+}
+
 // Decode append: one CTA per sequence.
 //   k_cache[b][L] = RoPE(k_new[b], L); v_cache[b][L] = v_new[b];
 //   kidx_cache[b][L] = k_idx_new[b]; ring slot L % 4 <- (q_idx_new[b], w_new[b]);
@@ -89,8 +151,10 @@ __global__ void decode_append_kernel(int64_t max_len, LenChunk lens, int64_t* __
                                      uint16_t* __restrict__ kbar_cache, int64_t kbar_len,
                                      const int32_t* __restrict__ sel_in, const int32_t* __restrict__ cnt_in,
                                      int budget, int32_t* __restrict__ sel_r, int sel_r_ld,
-                                     int32_t* __restrict__ cnt_r, uint32_t* err) {
+                                     int32_t* __restrict__ cnt_r, uint32_t* err, int idx_rope,
+                                     uint16_t* __restrict__ ring_rot) {
   __shared__ float2 cs[32];
+  __shared__ double kmean[128];
   __shared__ int n_keep, first_neg;
   const int b = lens.b0 + blockIdx.x;
   const int64_t L = lens.L[blockIdx.x];
@@ -165,16 +229,62 @@ __global__ void decode_append_kernel(int64_t max_len, LenChunk lens, int64_t* __
   for (int e = threadIdx.x; e < 64; e += blockDim.x)            // q_idx: 4 x 256 B
     qidx_ring[((int64_t)b * 4 + slot) * 64 + e] = q_idx_new[(int64_t)b * 64 + e];
   if (threadIdx.x < 4) w_ring[((int64_t)b * 4 + slot) * 4 + threadIdx.x] = w_new[(int64_t)b * 4 + threadIdx.x];
-  if (kbar_cache != nullptr && threadIdx.x < 128) {
+  const int64_t t0 = L & ~(int64_t)3;     // first token of the new token's block
+  if (kbar_cache != nullptr) {
     // mean of keys 4 qb .. L: the earlier ones from the cache, the new one from k_idx_new
-    const int c = threadIdx.x;
-    const int64_t t0 = L & ~(int64_t)3;
-    const uint16_t* kc = reinterpret_cast<const uint16_t*>(kidx_cache) + (int64_t)b * max_len * 128;
-    const uint16_t* kn = reinterpret_cast<const uint16_t*>(k_idx_new) + (int64_t)b * 128;
-    double sum = 0.0;
-    for (int64_t t = t0; t < L; ++t) sum += (double)__uint_as_float((uint32_t)kc[t * 128 + c] << 16);
-    sum += (double)__uint_as_float((uint32_t)kn[c] << 16);
-    kbar_cache[((int64_t)b * kbar_len + (L >> 2)) * 128 + c] = f64_to_bf16_rne(sum / (double)(L - t0 + 1));
+    uint16_t* krow = kbar_cache + ((int64_t)b * kbar_len + (L >> 2)) * 128;
+    if (threadIdx.x < 128) {
+      const int c = threadIdx.x;
+      const uint16_t* kc = reinterpret_cast<const uint16_t*>(kidx_cache) + (int64_t)b * max_len * 128;
+      const uint16_t* kn = reinterpret_cast<const uint16_t*>(k_idx_new) + (int64_t)b * 128;
+      double sum = 0.0;
+      for (int64_t t = t0; t < L; ++t) sum += (double)__uint_as_float((uint32_t)kc[t * 128 + c] << 16);
+      sum += (double)__uint_as_float((uint32_t)kn[c] << 16);
+      const uint16_t m = f64_to_bf16_rne(sum / (double)(L - t0 + 1));
+      if (idx_rope) kmean[c] = (double)bf16_bits_to_f32(m);
+      else krow[c] = m;
+    }
+    if (idx_rope) {
+      // the block's start position 4 qb: dims 0..63 rotated (fp64, one more rounding)
+      __syncthreads();
+      if (threadIdx.x < 32) {
+        const int i = threadIdx.x;
+        double sa, ca;
+        sincos((double)t0 * inv.f[i], &sa, &ca);
+        ca *= inv.scale;
+        sa *= inv.scale;
+        krow[i] = f64_to_bf16_rne(kmean[i] * ca - kmean[i + 32] * sa);
+        krow[i + 32] = f64_to_bf16_rne(kmean[i + 32] * ca + kmean[i] * sa);
+      } else if (threadIdx.x >= 64 && threadIdx.x < 128) {
+        krow[threadIdx.x] = f64_to_bf16_rne(kmean[threadIdx.x]);
+      }
+    }
+  }
+  if (ring_rot != nullptr) {
+    // indexer queries of the block-mates 4 qb .. L rotated at their positions
+    // (the mean-pooled indexer with block-start positions): ring slot j holds
+    // token 4 qb + j; the new token's own q_idx is read from q_idx_new
+    const int present = (int)(L - t0) + 1;
+    const uint16_t* ring16 = reinterpret_cast<const uint16_t*>(qidx_ring);
+    const uint16_t* new16 = reinterpret_cast<const uint16_t*>(q_idx_new) + (int64_t)b * 512;
+    for (int e = threadIdx.x; e < present * 32; e += blockDim.x) {
+      const int tok = e >> 5, i = e & 31;
+      const uint16_t* src = tok == slot ? new16 : ring16 + ((int64_t)b * 4 + tok) * 512;
+      uint16_t* dst = ring_rot + ((int64_t)b * 4 + tok) * 512;
+      double sa, ca;
+      sincos((double)(t0 + tok) * inv.f[i], &sa, &ca);
+      ca *= inv.scale;
+      sa *= inv.scale;
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const double x = (double)bf16_bits_to_f32(src[h * 128 + i]);
+        const double y = (double)bf16_bits_to_f32(src[h * 128 + i + 32]);
+        dst[h * 128 + i] = f64_to_bf16_rne(x * ca - y * sa);
+        dst[h * 128 + i + 32] = f64_to_bf16_rne(y * ca + x * sa);
+      }
+      const int h = i >> 3, c = i & 7;
+      reinterpret_cast<uint4*>(dst + h * 128 + 64)[c] = reinterpret_cast<const uint4*>(src + h * 128 + 64)[c];
+    }
   }
 }
 
@@ -261,6 +371,23 @@ cudaError_t launch_rope_k(int64_t T, const uint16_t* k, const float2* cs, uint16
   return cudaGetLastError();
 }
 
+cudaError_t launch_idx_rope_q(int64_t T, int64_t pos0, const double* inv_freq_host, double attn_factor,
+                              const uint16_t* q_idx, uint16_t* out, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  idx_rope_q_kernel<<<grid_for(T * 32, 256), 256, 0, s>>>(T, pos0, to_struct(inv_freq_host, attn_factor), q_idx, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kbar_rope(const uint16_t* k_idx, int64_t T, int64_t pos0, const double* inv_freq_host,
+                             double attn_factor, uint16_t* kbar, cudaStream_t s) {
+  const int64_t nkb = (T + 3) / 4;
+  if (nkb <= 0) return cudaSuccess;
+  const int64_t n = nkb * 96;
+  kbar_rope_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(k_idx, T, nkb, pos0, to_struct(inv_freq_host, attn_factor),
+                                                                kbar);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_decode_append(int B, int64_t max_len, const int64_t* L_host, int64_t* L_dev, int64_t* qb_dev,
                                  const double* inv_freq_host, double attn_factor, uint16_t* k_cache,
                                  uint16_t* v_cache, uint16_t* kidx_cache, uint16_t* qidx_ring, uint16_t* w_ring,
@@ -268,7 +395,7 @@ cudaError_t launch_decode_append(int B, int64_t max_len, const int64_t* L_host, 
                                  const uint16_t* q_idx_new, const uint16_t* k_idx_new, const uint16_t* w_new,
                                  uint16_t* q_rot, uint16_t* kbar_cache, int64_t kbar_len, const int32_t* sel_in,
                                  const int32_t* cnt_in, int budget, int32_t* sel_r, int sel_r_ld, int32_t* cnt_r,
-                                 uint32_t* err, cudaStream_t s) {
+                                 uint32_t* err, cudaStream_t s, bool idx_rope, uint16_t* ring_rot) {
   const InvFreq inv = to_struct(inv_freq_host, attn_factor);
   for (int b0 = 0; b0 < B; b0 += LEN_CHUNK) {
     const int n = B - b0 < LEN_CHUNK ? B - b0 : LEN_CHUNK;
@@ -281,7 +408,7 @@ cudaError_t launch_decode_append(int B, int64_t max_len, const int64_t* L_host, 
         reinterpret_cast<const uint4*>(q_new), reinterpret_cast<const uint4*>(k_new),
         reinterpret_cast<const uint4*>(v_new), reinterpret_cast<const uint4*>(q_idx_new),
         reinterpret_cast<const uint4*>(k_idx_new), w_new, reinterpret_cast<uint4*>(q_rot), kbar_cache, kbar_len,
-        sel_in, cnt_in, budget, sel_r, sel_r_ld, cnt_r, err);
+        sel_in, cnt_in, budget, sel_r, sel_r_ld, cnt_r, err, idx_rope ? 1 : 0, ring_rot);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -95,6 +95,19 @@ typedef struct {
   double yarn_original_max;
   double yarn_beta_fast;
   double yarn_beta_slow;
+  /* Block-start position of the mean-pooled indexer ([PT §QSA]: the keys of
+   * a micro-block are compressed before the positional step and the
+   * compressed key gets one block-start position).  0 (default): the indexer
+   * has no positional encoding.  1 (only with QSA_AGG_MEAN_POOL): the
+   * indexer queries of token t are rotated at t's position and the compressed
+   * key of block b at the position of its first token, 4b, with this layer's
+   * RoPE (dims 0..63 of the 128, pairs (i, i + 32), theta and YaRN as above);
+   * the rotation is computed in fp64 and each rotated operand is rounded to
+   * bf16 once (the compressed key after its mean was rounded to bf16).
+   * Positions: pos0 + t in qsa_prefill, t in qsa_index_scores and
+   * qsa_mean_pool_keys, the cache position in the decode calls.
+   * qsa_prefill_cached and qsa_verify return QSA_ERR_UNSUPPORTED with it. */
+  int32_t idx_rope;
 } qsa_params;
 
 /* Fills *p with the values above (budget 512). */
@@ -362,7 +375,8 @@ enum {
   QSA_KERNEL_DECODE_ATTENTION = 8,
   QSA_KERNEL_DECODE_COMBINE = 9,
   QSA_KERNEL_KBAR = 10,
-  QSA_KERNEL_VERIFY_EXPAND = 11
+  QSA_KERNEL_VERIFY_EXPAND = 11,
+  QSA_KERNEL_IDX_ROPE = 12
 };
 qsa_status qsa_trace_begin(int32_t capacity);
 qsa_status qsa_trace_end(int32_t* kernel_ids, float* ms, int32_t capacity, int32_t* n_out);
