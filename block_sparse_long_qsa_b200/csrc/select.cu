@@ -46,7 +46,7 @@ __host__ __device__ inline int pow2_at_least(int x) {
 }
 
 struct SelSmem {
-  uint32_t* hist;   // [256]
+  uint32_t* hist;   // [2][256]: the radix passes alternate between the two
   uint32_t* misc;   // [16]
   uint32_t* warp_tot;  // [32]
   uint32_t* sample; // [NSAMPLE]
@@ -64,18 +64,26 @@ __device__ void radix_kth_largest(Get get, int64_t n, int64_t k, const SelSmem& 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t prefix = 0, mask = 0;
   int64_t kk = k;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += blockDim.x) sm.hist[i] = 0;
-    __syncthreads();
+  // Two histograms: pass p counts into hist[p % 2] while the other one is
+  // cleared for pass p + 1, and the chosen digit goes to misc[2 (p % 2)], so
+  // a pass needs two barriers (after the counts, after the scan).
+  for (int i = tid; i < 256; i += blockDim.x) sm.hist[i] = 0;
+  __syncthreads();
+  int pass = 0;
+  for (int shift = 24; shift >= 0; shift -= 8, ++pass) {
+    uint32_t* hist = sm.hist + 256 * (pass & 1);
+    uint32_t* next = sm.hist + 256 * ((pass + 1) & 1);
+    for (int i = tid; i < 256; i += blockDim.x) next[i] = 0;
     for (int64_t i = tid; i < n; i += blockDim.x) {
       const uint32_t key = get(i);
-      if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 255u], 1u);
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
     }
     __syncthreads();
+    uint32_t* out2 = sm.misc + 2 * (pass & 1);
     if (warp == 0) {
       uint32_t c[8], s = 0;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) { c[q] = sm.hist[255 - 8 * lane - q]; s += c[q]; }
+      for (int q = 0; q < 8; ++q) { c[q] = hist[255 - 8 * lane - q]; s += c[q]; }
       uint32_t incl = s;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -88,8 +96,8 @@ __device__ void radix_kth_largest(Get get, int64_t n, int64_t k, const SelSmem& 
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           if (cum + c[q] >= kk) {
-            sm.misc[0] = (uint32_t)(255 - 8 * lane - q);
-            sm.misc[1] = (uint32_t)(kk - cum);
+            out2[0] = (uint32_t)(255 - 8 * lane - q);
+            out2[1] = (uint32_t)(kk - cum);
             break;
           }
           cum += c[q];
@@ -97,12 +105,12 @@ __device__ void radix_kth_largest(Get get, int64_t n, int64_t k, const SelSmem& 
       }
     }
     __syncthreads();
-    const uint32_t bin = sm.misc[0];
-    kk = sm.misc[1];
+    const uint32_t bin = out2[0];
+    kk = out2[1];
     prefix |= bin << shift;
     mask |= 0xFFu << shift;
-    __syncthreads();
   }
+  __syncthreads();   // every thread has read the last digit before the caller reuses misc / hist
   tau = prefix;
   n_gt = k - kk;
 }
@@ -135,7 +143,7 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
   const int P = pow2_at_least(budget);
   SelSmem sm;
   sm.hist = reinterpret_cast<uint32_t*>(smem_raw);
-  sm.misc = sm.hist + 256;
+  sm.misc = sm.hist + 512;
   sm.warp_tot = sm.misc + 16;
   sm.sample = sm.warp_tot + 32;
   sm.ckey = sm.sample + NSAMPLE;
@@ -154,7 +162,7 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
     }
     const int64_t m = qb - 1;          // candidates 0 .. qb-2
     const int64_t k = budget - 2;
-    if (tid == 0) { sm.misc[2] = 0; sm.misc[3] = 0; }
+    if (tid == 0) { sm.misc[8] = 0; sm.misc[9] = 0; }
     __syncthreads();
 
     bool global_path = false;
@@ -174,7 +182,16 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
       //     score >= tau0 lies in such a segment or in the tail.
       const int64_t fs = (qb - 1) >> 3;
       const float* mrow = segmax + r * ld_seg;
-      for (int i = tid; i < NSAMPLE; i += blockDim.x) sm.sample[i] = key_of(mrow[(int64_t)i * fs / NSAMPLE]);
+      // NSAMPLE / 4 evenly spaced 16-byte groups of 4 consecutive maxima (the
+      // row is 16-byte aligned: ld_seg % 4 == 0; fs > cap / 8 >= 4 x groups)
+      {
+        const float4* mrow4 = reinterpret_cast<const float4*>(mrow);
+        const int64_t fs4 = fs >> 2;
+        for (int i = tid; i < NSAMPLE / 4; i += blockDim.x) {
+          const float4 g = __ldcs(mrow4 + (int64_t)i * fs4 / (NSAMPLE / 4));
+          reinterpret_cast<uint4*>(sm.sample)[i] = make_uint4(key_of(g.x), key_of(g.y), key_of(g.z), key_of(g.w));
+        }
+      }
       const float e = (float)NSAMPLE * (float)k / (float)fs;
       int64_t rs = (int64_t)ceilf(e + 4.f * sqrtf(e) + 8.f);
       if (rs > NSAMPLE) rs = NSAMPLE;
@@ -183,34 +200,47 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
       int64_t dummy;
       radix_kth_largest([&](int64_t i) { return sm.sample[i]; }, NSAMPLE, rs, sm, tau0, dummy);
       // 2'. the segments whose max reaches tau0 (listed in the sample buffer) ...
-      if (tid == 0) sm.misc[5] = 0;
+      if (tid == 0) sm.misc[11] = 0;
       __syncthreads();
-      // SEG_UNROLL loads per thread in flight before any is tested: the scan is
-      // one row of up to 32K maxima per CTA, bound by load latency otherwise
-      constexpr int SEG_UNROLL = 8;
-      for (int64_t b0 = 0; b0 < fs; b0 += (int64_t)blockDim.x * SEG_UNROLL) {
-        uint32_t kv[SEG_UNROLL];
+      // SEG_UNROLL 16-byte loads (4 maxima each) per thread in flight before
+      // any is tested: the scan is one row of up to 32K maxima per CTA, bound
+      // by load latency otherwise; most groups have no maximum reaching tau0
+      // and skip the compaction
+      constexpr int SEG_UNROLL = 4;
+      const float4* mrow4 = reinterpret_cast<const float4*>(mrow);
+      const int64_t fs4 = (fs + 3) >> 2;     // rows are padded to a multiple of 4 (ld_seg)
+      for (int64_t b0 = 0; b0 < fs4; b0 += (int64_t)blockDim.x * SEG_UNROLL) {
+        float4 kv[SEG_UNROLL];
 #pragma unroll
         for (int u = 0; u < SEG_UNROLL; ++u) {
-          const int64_t sgi = b0 + (int64_t)u * blockDim.x + tid;
-          kv[u] = sgi < fs ? key_of(__ldcs(mrow + sgi)) : 0u;
+          const int64_t g = b0 + (int64_t)u * blockDim.x + tid;
+          kv[u] = g < fs4 ? __ldcs(mrow4 + g) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
         for (int u = 0; u < SEG_UNROLL; ++u) {
-          const int64_t sgi = b0 + (int64_t)u * blockDim.x + tid;
-          const bool pass = sgi < fs && kv[u] >= tau0;
-          const uint32_t ball = __ballot_sync(0xffffffffu, pass);
-          if (ball) {
-            uint32_t base = 0;
-            if (lane == 0) base = atomicAdd(&sm.misc[5], (uint32_t)__popc(ball));
-            base = __shfl_sync(0xffffffffu, base, 0);
-            const uint32_t pos = base + __popc(ball & ((1u << lane) - 1u));
-            if (pass && pos < (uint32_t)NSAMPLE) sm.sample[pos] = (uint32_t)sgi;
+          const int64_t g = b0 + (int64_t)u * blockDim.x + tid;
+          const float vals[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
+          bool any = false;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) any |= (4 * g + q < fs) && key_of(vals[q]) >= tau0;
+          if (!__any_sync(0xffffffffu, any)) continue;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int64_t sgi = 4 * g + q;
+            const bool pass = sgi < fs && key_of(vals[q]) >= tau0;
+            const uint32_t ball = __ballot_sync(0xffffffffu, pass);
+            if (ball) {
+              uint32_t base = 0;
+              if (lane == 0) base = atomicAdd(&sm.misc[11], (uint32_t)__popc(ball));
+              base = __shfl_sync(0xffffffffu, base, 0);
+              const uint32_t pos = base + __popc(ball & ((1u << lane) - 1u));
+              if (pass && pos < (uint32_t)NSAMPLE) sm.sample[pos] = (uint32_t)sgi;
+            }
           }
         }
       }
       __syncthreads();
-      const int64_t nsl = sm.misc[5];
+      const int64_t nsl = sm.misc[11];
       if (nsl > NSAMPLE) {
         global_path = true;
       } else {
@@ -240,7 +270,7 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
               const uint32_t ball = __ballot_sync(0xffffffffu, pass);
               if (ball) {
                 uint32_t base = 0;
-                if (lane == 0) base = atomicAdd(&sm.misc[2], (uint32_t)__popc(ball));
+                if (lane == 0) base = atomicAdd(&sm.misc[8], (uint32_t)__popc(ball));
                 base = __shfl_sync(0xffffffffu, base, 0);
                 const uint32_t pos = base + __popc(ball & ((1u << lane) - 1u));
                 if (pass && pos < (uint32_t)cap) {
@@ -254,12 +284,12 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
         if (tid < 8) {
           const int64_t i = 8 * fs + tid;
           if (i < m && key_of(row[i]) >= tau0) {
-            const uint32_t pos = atomicAdd(&sm.misc[2], 1u);
+            const uint32_t pos = atomicAdd(&sm.misc[8], 1u);
             if (pos < (uint32_t)cap) { sm.ckey[pos] = key_of(row[i]); sm.cidx[pos] = (int32_t)i; }
           }
         }
         __syncthreads();
-        nc = sm.misc[2];
+        nc = sm.misc[8];
         global_path = (nc < k || nc > cap);
       }
       __syncthreads();
@@ -302,7 +332,7 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
             const uint32_t ball = __ballot_sync(0xffffffffu, pass);
             if (ball) {
               uint32_t base = 0;
-              if (lane == 0) base = atomicAdd(&sm.misc[2], (uint32_t)__popc(ball));
+              if (lane == 0) base = atomicAdd(&sm.misc[8], (uint32_t)__popc(ball));
               base = __shfl_sync(0xffffffffu, base, 0);
               const uint32_t pos = base + __popc(ball & ((1u << lane) - 1u));
               if (pass && pos < (uint32_t)cap) { sm.ckey[pos] = key_of(vals[q]); sm.cidx[pos] = (int32_t)idx; }
@@ -311,13 +341,13 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
         }
       }
       __syncthreads();
-      nc = sm.misc[2];
+      nc = sm.misc[8];
       global_path = (nc < k || nc > cap);
       __syncthreads();
     }
 
     if (k == 0) {
-      if (tid == 0) sm.misc[2] = 0;
+      if (tid == 0) sm.misc[8] = 0;
       __syncthreads();
     } else if (!global_path) {
       __syncthreads();
@@ -326,12 +356,12 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
       radix_kth_largest([&](int64_t i) { return sm.ckey[i]; }, nc, k, sm, tau, n_gt);
       const int64_t need = k - n_gt;
       // count ties
-      if (tid == 0) { sm.misc[2] = 0; sm.misc[4] = 0; }
+      if (tid == 0) { sm.misc[8] = 0; sm.misc[10] = 0; }
       __syncthreads();
       for (int64_t i = tid; i < nc; i += blockDim.x)
-        if (sm.ckey[i] == tau) atomicAdd(&sm.misc[4], 1u);
+        if (sm.ckey[i] == tau) atomicAdd(&sm.misc[10], 1u);
       __syncthreads();
-      const int64_t n_eq = sm.misc[4];
+      const int64_t n_eq = sm.misc[10];
       uint32_t idx_cut = 0xFFFFFFFFu;   // take ties with index <= idx_cut
       if (n_eq > need) {
         uint32_t ntau;
@@ -344,7 +374,7 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
         const uint32_t key = sm.ckey[i];
         const bool take = key > tau || (key == tau && (uint32_t)sm.cidx[i] <= idx_cut);
         if (take) {
-          const uint32_t pos = atomicAdd(&sm.misc[2], 1u);
+          const uint32_t pos = atomicAdd(&sm.misc[8], 1u);
           if (pos < (uint32_t)k) sm.out[pos] = sm.cidx[i];
         }
       }
@@ -355,7 +385,7 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
       int64_t n_gt;
       radix_kth_largest([&](int64_t i) { return key_of(row[i]); }, m, k, sm, tau, n_gt);
       const int64_t need = k - n_gt;
-      if (tid == 0) sm.misc[2] = 0;
+      if (tid == 0) sm.misc[8] = 0;
       __syncthreads();
       int64_t eq_taken = 0;
       for (int64_t base = 0; base < m; base += blockDim.x) {
@@ -366,14 +396,14 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
         uint32_t tot;
         const uint32_t rank = block_excl_count(eq, sm, &tot);
         if (gt || (eq && eq_taken + (int64_t)rank < need)) {
-          const uint32_t pos = atomicAdd(&sm.misc[2], 1u);
+          const uint32_t pos = atomicAdd(&sm.misc[8], 1u);
           if (pos < (uint32_t)k) sm.out[pos] = (int32_t)i;
         }
         eq_taken += tot;
       }
       __syncthreads();
     }
-    if (tid == 0 && sm.misc[2] != (uint32_t)k) report_error(err, QSA_ERR_DEVICE_BOUNDS);
+    if (tid == 0 && sm.misc[8] != (uint32_t)k) report_error(err, QSA_ERR_DEVICE_BOUNDS);
     // 4. forced blocks, then ascending sort of the budget entries
     if (tid == 0) { sm.out[k] = (int32_t)(qb - 1); sm.out[k + 1] = (int32_t)qb; }
     for (int i = budget + tid; i < P; i += blockDim.x) sm.out[i] = INT_MAX;
@@ -430,7 +460,7 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
 
 size_t select_smem_bytes(int budget) {
   const int cap = cap_for(budget);
-  return (size_t)(256 + 16 + 32 + NSAMPLE) * 4 + (size_t)cap * 8 + (size_t)pow2_at_least(budget) * 4;
+  return (size_t)(512 + 16 + 32 + NSAMPLE) * 4 + (size_t)cap * 8 + (size_t)pow2_at_least(budget) * 4;
 }
 
 cudaError_t launch_select(const float* S, int64_t ld, const float* segmax, int64_t ld_seg, int64_t qb_begin,
