@@ -711,9 +711,14 @@ WORKLOADS = {
 
 
 # DRAM bytes per launch of the dominant kernel (dram__bytes_read.sum +
-# dram__bytes_write.sum, averaged over the launches of a one-pass ncu capture
-# of this workload with the current kernel); None where no such capture exists.
-NCU_TRAFFIC = {"prefill_1m": 60.84e9 + 15.46e9, "decode_64x256k": 4.2954e9 + 0.0093e9,
+# dram__bytes_write.sum) with the current kernels; None where no capture exists.
+# prefill_1m: from a small-case capture of the indexer (the last 2,048 query
+# blocks of the 1M-token problem: 522K units, 0.357 GB read, 2.09 GB written),
+# the reads scaled to the mean launch of the 1M prefill by units (3.36M, an
+# upper bound: key bands are read once per band) and the writes (the score
+# slab and segment maxima, in proportion to the causal entries) 15.46 GB.
+# The decode figures are averaged launches of one-pass captures.
+NCU_TRAFFIC = {"prefill_1m": 0.357e9 * 3.36 / 0.522 + 15.46e9, "decode_64x256k": 4.2954e9 + 0.0093e9,
                "decode_64x256k_spec4": 4.2957e9 + 0.0085e9, "verify_64x256k_m5": 4.2982e9 + 0.0084e9}
 
 

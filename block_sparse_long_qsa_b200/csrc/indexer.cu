@@ -53,11 +53,23 @@ constexpr uint32_t SMEM_BYTES = OFF_BAR + 128;
 static_assert(SMEM_BYTES <= 232448, "indexer smem");
 constexpr uint32_t TMEM_COLS = 512;
 
+// Key bands of BAND key tiles (32 MB of indexer keys): every band's units
+// (query tile ascending, then key tile) are split evenly across the CTAs and
+// the CTAs take the bands in order, so at any time they all read the same
+// band of keys, which L2 serves to all of them, instead of sweeping the whole
+// key range at unrelated offsets.  A query tile's Q operand is loaded once per
+// (band, query tile) segment of a CTA.  Measured on B200 (1M tokens): DRAM
+// reads of the indexer 37x lower than with one query-major split, and the 1M
+// prefill 3-4 % faster (the power the reads drew goes to the clock); bands
+// of 64 key tiles were slower (more Q reloads), 256 and 1024 alike.
+constexpr int64_t BAND = 1024;
+
 struct Sched {
   int64_t T0, Tend, n_tiles;
   int64_t qb_begin;
   int64_t R;                      // tokens per key-tile row: 1 (keys) or 4 (mean-pooled key blocks)
   int64_t A;                      // (T0 + QT - 1) / QT
+  int64_t n_bands;
   __device__ __forceinline__ int64_t nkt(int64_t i) const {
     int64_t tl = T0 + QT * i + (QT - 1);
     if (tl > Tend - 1) tl = Tend - 1;
@@ -68,31 +80,123 @@ struct Sched {
     const int64_t q = N / R, r = N % R;
     return R * q * (q - 1) / 2 + r * q;
   }
-  // units before tile i (valid for i <= n_tiles - 1; tiles before the last are
-  // full): sum over j < i of floor((A + j) / R) + 1, as QT = KT tokens
+  // units before tile i in query-major order (valid for i <= n_tiles - 1;
+  // tiles before the last are full): sum over j < i of floor((A + j) / R) + 1
   __device__ __forceinline__ int64_t prefix(int64_t i) const { return i + G(A + i) - G(A); }
   __device__ __forceinline__ int64_t total() const { return prefix(n_tiles - 1) + nkt(n_tiles - 1); }
-  __device__ __forceinline__ void locate(int64_t u, int64_t& tile, int64_t& kt) const {
-    int64_t lo = 0, hi = n_tiles - 1;
+  // sum over j < i of nkt(j), 0 <= i <= n_tiles
+  __device__ __forceinline__ int64_t sum_nkt(int64_t i) const { return i < n_tiles ? prefix(i) : total(); }
+  // first tile j in [0, i) with nkt(j) >= x (nkt is non-decreasing), or i
+  __device__ __forceinline__ int64_t first_reaching(int64_t i, int64_t x) const {
+    int64_t lo = 0, hi = i;
     while (lo < hi) {
-      int64_t mid = (lo + hi + 1) >> 1;
-      if (prefix(mid) <= u) lo = mid; else hi = mid - 1;
+      const int64_t mid = (lo + hi) >> 1;
+      if (nkt(mid) >= x) hi = mid; else lo = mid + 1;
     }
-    tile = lo;
-    kt = u - prefix(lo);
+    return lo;
+  }
+  // sum over j < i of min(nkt(j), x): the units of tiles [0, i) with key tile < x
+  __device__ __forceinline__ int64_t cmin(int64_t i, int64_t x) const {
+    const int64_t f = first_reaching(i, x);
+    return sum_nkt(f) + (i - f) * x;
+  }
+  // units before band b (key tiles < BAND b of every tile)
+  __device__ __forceinline__ int64_t band_start(int64_t b) const { return cmin(n_tiles, BAND * b); }
+  // units of band b in tiles [0, i)
+  __device__ __forceinline__ int64_t in_band(int64_t b, int64_t i) const {
+    return cmin(i, BAND * (b + 1)) - cmin(i, BAND * b);
   }
 };
 
-struct Iter {
+// A CTA's units: in every band, its even share (CTA c of G takes band
+// positions [U_b c / G, U_b (c + 1) / G) of the band's U_b units), band after
+// band, so all CTAs sweep the same band at the same time.
+struct IterBand {
+  const Sched* s;
+  int64_t v, v_begin, v_end;   // position in the band's unit order; this CTA's range in the band
+  int64_t tile, kt;
+  int64_t left;                // units this CTA has left, this one included
+  int band, seg_end;           // band; one past the last key tile of this (band, tile) segment
+  int64_t cta, ncta;
+  __device__ __forceinline__ void range(int b, int64_t& lo, int64_t& hi) const {
+    const int64_t n = s->band_start(b + 1) - s->band_start(b);
+    lo = n * cta / ncta;
+    hi = n * (cta + 1) / ncta;
+  }
+  __device__ __forceinline__ void set_seg_end() {
+    const int64_t n = s->nkt(tile), e = BAND * (band + 1);
+    seg_end = (int)(n < e ? n : e);
+  }
+  // next band with units for this CTA, positioned at its first one
+  __device__ __forceinline__ void advance_band() {
+    for (++band; band < s->n_bands; ++band) {
+      range(band, v_begin, v_end);
+      if (v_end > v_begin) break;
+    }
+    if (band >= s->n_bands) return;
+    v = v_begin;
+    int64_t tl = 0, th = s->n_tiles - 1;         // largest tile whose in-band offset <= v
+    while (tl < th) {
+      const int64_t mid = (tl + th + 1) >> 1;
+      if (s->in_band(band, mid) <= v) tl = mid; else th = mid - 1;
+    }
+    tile = tl;
+    kt = BAND * band + (v - s->in_band(band, tile));
+    set_seg_end();
+  }
+  // (u0, u1: the query-major split, unused by this schedule)
+  __device__ __forceinline__ void begin(const Sched* sch, int64_t, int64_t) {
+    s = sch; cta = blockIdx.x; ncta = gridDim.x;
+    left = 0;
+    for (int b = 0; b < s->n_bands; ++b) {
+      int64_t lo, hi;
+      range(b, lo, hi);
+      left += hi - lo;
+    }
+    band = -1;
+    if (left > 0) advance_band();
+  }
+  __device__ __forceinline__ bool valid() const { return left > 0; }
+  // a new segment starts (a new query tile, or this CTA's first unit of a
+  // band): the Q tile is (re)loaded
+  __device__ __forceinline__ bool first_of_tile(int64_t) const { return kt == BAND * band || v == v_begin; }
+  // the next unit of this CTA belongs to another segment
+  __device__ __forceinline__ bool tile_ends_here() const {
+    return (kt == seg_end - 1 || v + 1 == v_end) && left > 1;
+  }
+  __device__ __forceinline__ void next() {
+    --left; ++v; ++kt;
+    if (left <= 0) return;
+    if (v == v_end) { advance_band(); return; }
+    if (kt < seg_end) return;
+    ++tile;                       // the next tile of the band (it reaches into the band too)
+    kt = BAND * band;
+    set_seg_end();
+  }
+};
+
+// The units split evenly across CTAs in query-major order (the schedule of
+// the mean-pooled indexer, whose compressed keys are a quarter of the size;
+// its epilogue is at the register limit and the band bookkeeping spills).
+struct IterQuery {
   const Sched* s;
   int64_t u, u_end, tile, kt, nkt;
+  // units [u0, u1) of the query-major order
   __device__ __forceinline__ void begin(const Sched* sch, int64_t u0, int64_t u1) {
     s = sch; u = u0; u_end = u1;
-    if (u < u_end) { s->locate(u, tile, kt); nkt = s->nkt(tile); }
+    if (u < u_end) {
+      int64_t lo = 0, hi = s->n_tiles - 1;
+      while (lo < hi) {
+        const int64_t mid = (lo + hi + 1) >> 1;
+        if (s->prefix(mid) <= u) lo = mid; else hi = mid - 1;
+      }
+      tile = lo;
+      kt = u - s->prefix(lo);
+      nkt = s->nkt(tile);
+    }
   }
   __device__ __forceinline__ bool valid() const { return u < u_end; }
   __device__ __forceinline__ bool first_of_tile(int64_t u0) const { return kt == 0 || u == u0; }
-  // next unit in range belongs to another tile
   __device__ __forceinline__ bool tile_ends_here() const { return kt == nkt - 1 && u + 1 < u_end; }
   __device__ __forceinline__ void next() {
     ++u; ++kt;
@@ -123,6 +227,7 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  using It = std::conditional_t<MEAN, IterQuery, IterBand>;
 
   if ((smem_u32(smem) & 1023u) != 0u) {  // the swizzled operand layout needs 1 KB alignment
     if (threadIdx.x == 0) report_error(err, QSA_ERR_DEVICE_BOUNDS);
@@ -136,6 +241,7 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
   sch.n_tiles = (sch.Tend - sch.T0 + QT - 1) / QT;
   sch.R = MEAN ? 4 : 1;
   sch.A = (sch.T0 + QT - 1) / QT;
+  sch.n_bands = MEAN ? 1 : (sch.nkt(sch.n_tiles - 1) + BAND - 1) / BAND;
   const int64_t W = sch.total();
   const int64_t u0 = W * (int64_t)blockIdx.x / gridDim.x;
   const int64_t u1 = W * (int64_t)(blockIdx.x + 1) / gridDim.x;
@@ -163,7 +269,7 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     // taken by all lanes together.
     if (lane == 0) { tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); }
     float* sWf = reinterpret_cast<float*>(smem + OFF_W);
-    Iter it; it.begin(&sch, u0, u1);
+    It it; it.begin(&sch, u0, u1);
     int stage = 0; uint32_t ephase = 1; uint32_t qcount = 0;
     // for the drain at exit: bit s of `issued` / `par` = a load was issued into
     // stage s / the full-barrier phase parity of the last one; the same for
@@ -237,7 +343,7 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     // ---------------------------------------------------------------- MMA
     if (lane == 0) {
       constexpr uint32_t idesc = umma_idesc_bf16_f32(128, 256);
-      Iter it; it.begin(&sch, u0, u1);
+      It it; it.begin(&sch, u0, u1);
       int stage = 0; uint32_t fphase = 0; uint32_t qcount = 0;
       uint32_t acc_use[2] = {0, 0};
       bool ok = true;
@@ -295,7 +401,7 @@ indexer_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     const int qs = (la ? 4 : 0) + (lb ? 2 : 0);
     const int qs_seg = qs + (lc ? 1 : 0);
     const int qb0 = (int)qb_begin, qe = (int)qb_end;
-    Iter it; it.begin(&sch, u0, u1);
+    It it; it.begin(&sch, u0, u1);
     uint32_t qcount = 0;
     uint32_t acc_use = 0;
     int t_first = 0;              // first token of this thread's columns (per tile)
