@@ -792,6 +792,21 @@ def ncu_case(spec: str):
             r = qsa.prefill(d["q"], d["k"], d["v"], d["q_idx"], d["w"], d["k_idx"], budget=512, want_lse=False)
         torch.cuda.synchronize()
         assert qsa.qsa_check_device_error(r["ws"]) == 0
+    elif parts[0] == "indextail":
+        # stage 1 alone over the last `rows` query blocks of a T-token problem
+        # (keys larger than L2, a few GB on the device), three launches
+        T, rows = int(parts[1]), int(parts[2])
+        P = Q.PrefillProblem(T=T, seed=0, n_plant=8, dist="zipf")
+        d = P.device()
+        p = qsa.params(512)
+        nqb = (T + 3) // 4
+        ld = (nqb + 3) // 4 * 4
+        S = torch.empty((rows, ld), dtype=torch.float32, device="cuda")
+        ws = qsa.workspace(qsa.qsa_index_workspace_size(p, T))
+        for _ in range(3):
+            qsa.qsa_index_scores(p, T, d["q_idx"], d["w"], d["k_idx"], nqb - rows, nqb, S, ld, ws)
+        torch.cuda.synchronize()
+        assert qsa.qsa_check_device_error(ws) == 0
     elif parts[0] == "index":
         # stage 1 alone (qsa_index_scores, no segment maxima), four launches
         T = int(parts[1])
@@ -840,7 +855,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--ncu-case", default=None,
-                    help="prefill:T, index:T or decode:B:L -- a few calls of a small case (for ncu captures)")
+                    help="prefill:T, index:T, indextail:T:rows or decode:B:L -- a few calls of a small case "
+                         "(for ncu captures)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     if args.ncu_case:
