@@ -9,6 +9,8 @@
 #include <mutex>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "qsa.h"
 #include "qsa_kernels.h"
 #include "qsa_debug.h"
@@ -163,8 +165,28 @@ qsa_status make_map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t
 }
 
 // ----------------------------------------------------------------- tracing
-// When enabled, every kernel launch of the library is bracketed by two CUDA
-// events recorded on the launching stream.
+// Every kernel launch of the library is wrapped in an NVTX range named
+// "qsa/<kernel>" (free when no tool is attached; lets ncu --nvtx filter one
+// stage of a step).  When tracing is enabled, each launch is also bracketed
+// by two CUDA events recorded on the launching stream.
+const char* nvtx_name(int32_t id) {
+  switch (id) {
+    case QSA_KERNEL_ROPE_TABLE: return "qsa/rope_table";
+    case QSA_KERNEL_ROPE_K: return "qsa/rope_k";
+    case QSA_KERNEL_INDEXER: return "qsa/indexer";
+    case QSA_KERNEL_SELECT: return "qsa/select";
+    case QSA_KERNEL_ATTENTION: return "qsa/attention";
+    case QSA_KERNEL_DECODE_APPEND: return "qsa/decode_append";
+    case QSA_KERNEL_DECODE_INDEXER: return "qsa/decode_indexer";
+    case QSA_KERNEL_DECODE_ATTENTION: return "qsa/decode_attention";
+    case QSA_KERNEL_DECODE_COMBINE: return "qsa/decode_combine";
+    case QSA_KERNEL_KBAR: return "qsa/kbar";
+    case QSA_KERNEL_VERIFY_EXPAND: return "qsa/verify_expand";
+    case QSA_KERNEL_IDX_ROPE: return "qsa/idx_rope";
+    default: return "qsa/other";
+  }
+}
+
 struct TraceState {
   std::mutex mu;
   bool on = false;
@@ -182,7 +204,9 @@ cudaError_t traced(int32_t id, cudaStream_t s, F&& f) {
     if (g_trace.on && g_trace.n < g_trace.cap) slot = g_trace.n++;
   }
   if (slot >= 0) cudaEventRecord(g_trace.ev[2 * slot], s);
+  nvtxRangePushA(nvtx_name(id));
   cudaError_t e = f();
+  nvtxRangePop();
   if (slot >= 0) {
     cudaEventRecord(g_trace.ev[2 * slot + 1], s);
     g_trace.ids[slot] = id;
