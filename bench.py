@@ -149,12 +149,12 @@ def prefill_flops(T: int, sel_cnt: np.ndarray | None):
 
 
 def run_prefill(T: int, budget: int, steps: int, warmup: int, rank: int, world: int, seed: int, want_e2e=True,
-                aggregation: int = 0):
+                aggregation: int = 0, idx_rope: int = 0):
     import block_sparse_long_qsa_b200 as qsa
     P = Q.PrefillProblem(T=T, seed=rank_seed(seed, rank), n_plant=8, dist="zipf" if T >= 131072 else "uniform")
     d = P.device()
     torch.cuda.synchronize()
-    p = qsa.params(budget, aggregation=aggregation)
+    p = qsa.params(budget, aggregation=aggregation, idx_rope=idx_rope)
     mn, pref = qsa.qsa_prefill_workspace_size(p, T)
     ws = qsa.workspace(pref)
     nqb = P.nqb
@@ -507,15 +507,17 @@ def cpu_sample(wl: dict, target_s: float = 12.0, stratified: int = 0):
     stratified = n (prefill only) the sample is instead the n stratified query
     blocks the parity checks use."""
     if stratified and wl["kind"] == "prefill":
-        return cpu_prefill_sample(wl["T"], 512, stratified, aggregation=wl.get("aggregation", 0), stratified=True)
+        return cpu_prefill_sample(wl["T"], 512, stratified, aggregation=wl.get("aggregation", 0), stratified=True,
+                                  idx_rope=wl.get("idx_rope", 0))
     if wl["kind"] in ("prefill", "prefill_cached"):
         qb_lo = wl.get("L_old", 0) // 4
         agg = wl.get("aggregation", 0)
         n = max(4, cores_used())
-        v, info = cpu_prefill_sample(wl["T"], 512, n, qb_lo=qb_lo, aggregation=agg)
+        rope = wl.get("idx_rope", 0)
+        v, info = cpu_prefill_sample(wl["T"], 512, n, qb_lo=qb_lo, aggregation=agg, idx_rope=rope)
         if info["elapsed"] < target_s / 3:
             n2 = int(min((wl["T"] + 3) // 4 - qb_lo, max(n + 1, n * target_s / max(info["elapsed"], 1e-3))))
-            v, info = cpu_prefill_sample(wl["T"], 512, n2, qb_lo=qb_lo, aggregation=agg)
+            v, info = cpu_prefill_sample(wl["T"], 512, n2, qb_lo=qb_lo, aggregation=agg, idx_rope=rope)
     else:
         n = 2
         agg = wl.get("aggregation", 0)
@@ -540,14 +542,14 @@ def _oracle_work(qbs: np.ndarray, T: int, budget: int) -> np.ndarray:
 
 
 def cpu_prefill_sample(T: int, budget: int, n_blocks: int, seed: int = 0, qb_lo: int = 0, aggregation: int = 0,
-                       stratified: bool = False):
+                       stratified: bool = False, idx_rope: int = 0):
     """The oracle on a sample of query blocks of the T-token prefill (evenly
     spaced in [qb_lo, nqb), or the stratified sample of the parity checks),
     all host cores.  Returns tokens/s of the oracle extrapolated to the whole
     workload by the sample's share of the oracle's multiply-adds, and a
     description."""
     import oracle
-    O = oracle.Oracle(oracle.params(budget=budget, aggregation=aggregation))
+    O = oracle.Oracle(oracle.params(budget=budget, aggregation=aggregation, idx_rope=idx_rope))
     P = Q.PrefillProblem(T=T, seed=seed, n_plant=8, dist="zipf" if T >= 131072 else "uniform")
     nqb = P.nqb
     if stratified:
@@ -702,6 +704,9 @@ WORKLOADS = {
     "prefill_1m_cached90": dict(kind="prefill_cached", T=1 << 20, L_old=943718),
     # the pages' mean-pooled indexer (one compressed key per 4-token block)
     "prefill_1m_meanpool": dict(kind="prefill", T=1 << 20, aggregation=1),
+    # the same with the indexer's RoPE: queries rotated at their token, each
+    # compressed key at its block's first token
+    "prefill_1m_meanpool_rope": dict(kind="prefill", T=1 << 20, aggregation=1, idx_rope=1),
     "decode_64x256k_meanpool": dict(kind="decode", B=64, L=262144, aggregation=1),
     # speculative rounds of 4 draft tokens: one selection, reused by the next 3
     "decode_64x256k_spec4": dict(kind="decode", B=64, L=262144, spec=4),
@@ -725,6 +730,8 @@ NCU_TRAFFIC = {"prefill_1m": 0.357e9 * 3.36 / 0.522 + 15.46e9, "decode_64x256k":
 def metric_name(wl: dict) -> str:
     if wl["kind"] == "prefill":
         mp = ", mean-pooled indexer" if wl.get("aggregation") == 1 else ""
+        if wl.get("idx_rope"):
+            mp += " with block-start RoPE"
         return f"QSA prefill tokens/s at {wl['T'] // 1024}K context{mp}"
     if wl["kind"] == "prefill_cached":
         return (f"QSA prefix-cached prefill new tokens/s at {wl['T'] // 1024}K context, "
@@ -895,7 +902,7 @@ def main():
     wl = WORKLOADS[args.workload]
     if wl["kind"] == "prefill":
         res = run_prefill(wl["T"], 512, args.steps, args.warmup, rank, world, seed=0, want_e2e=not args.no_e2e,
-                          aggregation=wl.get("aggregation", 0))
+                          aggregation=wl.get("aggregation", 0), idx_rope=wl.get("idx_rope", 0))
     elif wl["kind"] == "prefill_cached":
         res = run_prefill_cached(wl["T"], wl["L_old"], 512, args.steps, args.warmup, rank, world, seed=0,
                                  want_e2e=not args.no_e2e)
@@ -915,14 +922,15 @@ def main():
         # the other workloads, compact (the line's end is what a log tail
         # keeps, so the plain decode and the 128K / 32K prefill come last)
         sec = {}
-        for name in ("prefill_1m_cached90", "prefill_1m_meanpool", "decode_64x256k_meanpool", "decode_64x256k_spec4",
+        for name in ("prefill_1m_cached90", "prefill_1m_meanpool", "prefill_1m_meanpool_rope",
+                     "decode_64x256k_meanpool", "decode_64x256k_spec4",
                      "verify_64x256k_m5", "prefill_32k", "prefill_128k", "decode_64x256k"):
             if name == args.workload:
                 continue
             w2 = WORKLOADS[name]
             if w2["kind"] == "prefill":
                 r2 = run_prefill(w2["T"], 512, args.steps, args.warmup, rank, world, seed=0, want_e2e=False,
-                                 aggregation=w2.get("aggregation", 0))
+                                 aggregation=w2.get("aggregation", 0), idx_rope=w2.get("idx_rope", 0))
             elif w2["kind"] == "prefill_cached":
                 r2 = run_prefill_cached(w2["T"], w2["L_old"], 512, args.steps, args.warmup, rank, world, seed=0,
                                         want_e2e=False)
