@@ -12,12 +12,15 @@
 // as unsigned integers.  One CTA per row:
 //   1. rows with at most CAP candidates are loaded whole into shared memory;
 //      longer rows draw a strided sample of 2048 scores whose order statistic
-//      at a safely conservative rank gives a threshold, and one coalesced
+//      at a safely conservative rank, its low 16 bits cleared (two radix
+//      passes), gives a threshold, and one coalesced
 //      pass keeps the scores at or above it (ballot-compacted) -- a few
 //      thousand candidates out of up to 262,143;
 //   2. an exact MSB-first radix select (8-bit digits, shared histograms)
-//      finds the k-th largest key among the candidates; ties at the threshold
-//      are resolved by a second radix select on the block indices;
+//      finds the k-th largest key among the candidates, starting at the
+//      first digit where the smallest and largest candidate differ; ties at
+//      the threshold are resolved by a second radix select on the block
+//      indices;
 //   3. if the sample's threshold left fewer than k or more than CAP
 //      candidates (rare), the same radix select runs over the whole row in
 //      global memory and an index-ordered pass collects the winners;
@@ -59,10 +62,16 @@ __device__ __forceinline__ uint32_t key_of(float x) { return __float_as_uint(x) 
 
 // k-th largest (1-based k, 1 <= k <= n) of get(0..n-1) by MSB-first radix
 // select.  Returns the key and the number of elements strictly greater.
+// Every key may be known to share its bits above digit hi_shift with
+// `common` (hi_shift < 24 skips those digits' passes; hi_shift < 0: all keys
+// equal `common`); with lo_shift > 0 the select stops after that digit and
+// returns the k-th largest key with its lower bits cleared (a lower bound).
 template <class Get>
-__device__ void radix_kth_largest(Get get, int64_t n, int64_t k, const SelSmem& sm, uint32_t& tau, int64_t& n_gt) {
+__device__ void radix_kth_largest(Get get, int64_t n, int64_t k, const SelSmem& sm, uint32_t& tau, int64_t& n_gt,
+                                  uint32_t common = 0, int hi_shift = 24, int lo_shift = 0) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  uint32_t prefix = 0, mask = 0;
+  uint32_t mask = hi_shift >= 24 ? 0u : ~0u << (hi_shift + 8);
+  uint32_t prefix = common & mask;
   int64_t kk = k;
   // Two histograms: pass p counts into hist[p % 2] while the other one is
   // cleared for pass p + 1, and the chosen digit goes to misc[2 (p % 2)], so
@@ -70,7 +79,7 @@ __device__ void radix_kth_largest(Get get, int64_t n, int64_t k, const SelSmem& 
   for (int i = tid; i < 256; i += blockDim.x) sm.hist[i] = 0;
   __syncthreads();
   int pass = 0;
-  for (int shift = 24; shift >= 0; shift -= 8, ++pass) {
+  for (int shift = hi_shift; shift >= lo_shift; shift -= 8, ++pass) {
     uint32_t* hist = sm.hist + 256 * (pass & 1);
     uint32_t* next = sm.hist + 256 * ((pass + 1) & 1);
     for (int i = tid; i < 256; i += blockDim.x) next[i] = 0;
@@ -162,8 +171,10 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
     }
     const int64_t m = qb - 1;          // candidates 0 .. qb-2
     const int64_t k = budget - 2;
-    if (tid == 0) { sm.misc[8] = 0; sm.misc[9] = 0; }
+    if (tid == 0) { sm.misc[8] = 0; sm.misc[9] = 0; sm.misc[12] = 0xFFFFFFFFu; sm.misc[13] = 0u; }
     __syncthreads();
+    // range of the candidates' keys (the exact select skips the digits they share)
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
 
     bool global_path = false;
     int64_t nc = 0;
@@ -171,8 +182,11 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
       // budget 2: only the forced blocks
     } else if (m <= cap) {
       for (int64_t i = tid; i < m; i += blockDim.x) {
-        sm.ckey[i] = key_of(row[i]);
+        const uint32_t key = key_of(row[i]);
+        sm.ckey[i] = key;
         sm.cidx[i] = (int32_t)i;
+        kmin = min(kmin, key);
+        kmax = max(kmax, key);
       }
       nc = m;
     } else if (segmax != nullptr) {
@@ -196,9 +210,11 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
       int64_t rs = (int64_t)ceilf(e + 4.f * sqrtf(e) + 8.f);
       if (rs > NSAMPLE) rs = NSAMPLE;
       __syncthreads();
+      // tau0 = the rs-th largest sampled maximum with its low 16 bits cleared
+      // (two radix passes; a slightly lower, still conservative threshold)
       uint32_t tau0;
       int64_t dummy;
-      radix_kth_largest([&](int64_t i) { return sm.sample[i]; }, NSAMPLE, rs, sm, tau0, dummy);
+      radix_kth_largest([&](int64_t i) { return sm.sample[i]; }, NSAMPLE, rs, sm, tau0, dummy, 0u, 24, 16);
       // 2'. the segments whose max reaches tau0 (listed in the sample buffer) ...
       if (tid == 0) sm.misc[11] = 0;
       __syncthreads();
@@ -277,6 +293,7 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
                   sm.ckey[pos] = key_of(vals[q]);
                   sm.cidx[pos] = (int32_t)(i0[u] + q);
                 }
+                if (pass) kmax = max(kmax, key_of(vals[q]));
               }
             }
           }
@@ -286,8 +303,10 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
           if (i < m && key_of(row[i]) >= tau0) {
             const uint32_t pos = atomicAdd(&sm.misc[8], 1u);
             if (pos < (uint32_t)cap) { sm.ckey[pos] = key_of(row[i]); sm.cidx[pos] = (int32_t)i; }
+            kmax = max(kmax, key_of(row[i]));
           }
         }
+        kmin = tau0;
         __syncthreads();
         nc = sm.misc[8];
         global_path = (nc < k || nc > cap);
@@ -302,7 +321,7 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
       __syncthreads();
       uint32_t tau0;
       int64_t dummy;
-      radix_kth_largest([&](int64_t i) { return sm.sample[i]; }, NSAMPLE, rs, sm, tau0, dummy);
+      radix_kth_largest([&](int64_t i) { return sm.sample[i]; }, NSAMPLE, rs, sm, tau0, dummy, 0u, 24, 16);
       // 2. filter pass: keep key >= tau0 (row start is 16-byte aligned: ld % 4 == 0)
       const float4* row4 = reinterpret_cast<const float4*>(row);
       const int64_t m4 = (m + 3) >> 2;
@@ -336,10 +355,12 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
               base = __shfl_sync(0xffffffffu, base, 0);
               const uint32_t pos = base + __popc(ball & ((1u << lane) - 1u));
               if (pass && pos < (uint32_t)cap) { sm.ckey[pos] = key_of(vals[q]); sm.cidx[pos] = (int32_t)idx; }
+              if (pass) kmax = max(kmax, key_of(vals[q]));
             }
           }
         }
       }
+      kmin = tau0;
       __syncthreads();
       nc = sm.misc[8];
       global_path = (nc < k || nc > cap);
@@ -350,10 +371,18 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
       if (tid == 0) sm.misc[8] = 0;
       __syncthreads();
     } else if (!global_path) {
+      {
+        const uint32_t wmin = __reduce_min_sync(0xffffffffu, kmin), wmax = __reduce_max_sync(0xffffffffu, kmax);
+        if (lane == 0) { atomicMin(&sm.misc[12], wmin); atomicMax(&sm.misc[13], wmax); }
+      }
       __syncthreads();
+      const uint32_t lo = sm.misc[12], hi = sm.misc[13];
+      // digits above the first bit where the smallest and largest candidate
+      // keys differ are the same for every candidate
+      const int same = lo == hi ? 32 : __clz(lo ^ hi);
       uint32_t tau;
       int64_t n_gt;
-      radix_kth_largest([&](int64_t i) { return sm.ckey[i]; }, nc, k, sm, tau, n_gt);
+      radix_kth_largest([&](int64_t i) { return sm.ckey[i]; }, nc, k, sm, tau, n_gt, lo, 24 - 8 * (same >> 3));
       const int64_t need = k - n_gt;
       // count ties
       if (tid == 0) { sm.misc[8] = 0; sm.misc[10] = 0; }
@@ -370,12 +399,22 @@ select_kernel(const float* __restrict__ S, int64_t ld, const float* __restrict__
                           ntau, d2);
         idx_cut = ~ntau;
       }
-      for (int64_t i = tid; i < nc; i += blockDim.x) {
-        const uint32_t key = sm.ckey[i];
-        const bool take = key > tau || (key == tau && (uint32_t)sm.cidx[i] <= idx_cut);
-        if (take) {
-          const uint32_t pos = atomicAdd(&sm.misc[8], 1u);
-          if (pos < (uint32_t)k) sm.out[pos] = sm.cidx[i];
+      for (int64_t b = 0; b < nc; b += blockDim.x) {
+        const int64_t i = b + tid;
+        bool take = false;
+        int32_t ci = 0;
+        if (i < nc) {
+          const uint32_t key = sm.ckey[i];
+          ci = sm.cidx[i];
+          take = key > tau || (key == tau && (uint32_t)ci <= idx_cut);
+        }
+        const uint32_t ball = __ballot_sync(0xffffffffu, take);
+        if (ball) {
+          uint32_t base = 0;
+          if (lane == 0) base = atomicAdd(&sm.misc[8], (uint32_t)__popc(ball));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          const uint32_t pos = base + __popc(ball & ((1u << lane) - 1u));
+          if (take && pos < (uint32_t)k) sm.out[pos] = ci;
         }
       }
       __syncthreads();
