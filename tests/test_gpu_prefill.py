@@ -105,19 +105,37 @@ def test_select_exact_on_given_scores(budget):
 
 
 def test_select_all_equal_rows():
-    """Degenerate rows (all scores equal) go through the exact fallback."""
+    """Degenerate rows: all scores equal (a row loaded whole, whose exact
+    select then has no digit to resolve, and longer rows that take the exact
+    fallback), and rows of two values one unit in the last place apart (only
+    the last digit differs)."""
     budget = 512
     p = qsa.params(budget)
     ws = qsa.workspace(qsa.qsa_select_workspace_size(p))
-    for qb in (9000, 40000):
+    for qb in (3000, 9000, 40000):
         ld = (qb + 1 + 3) // 4 * 4
         S = torch.zeros((1, ld), dtype=torch.float32, device="cuda")
         sel = torch.empty((1, budget), dtype=torch.int32, device="cuda")
         cnt = torch.empty((1,), dtype=torch.int32, device="cuda")
         qsa.qsa_select_blocks(p, S, ld, qb, qb + 1, sel, cnt, ws)
         torch.cuda.synchronize()
+        assert qsa.qsa_check_device_error(ws) == 0
         want = np.concatenate([np.arange(budget - 2), [qb - 1, qb]])
         assert np.array_equal(sel.cpu().numpy()[0], want)
+    rng = np.random.default_rng(7)
+    lo = np.float32(1.5)
+    hi = np.nextafter(lo, np.float32(2.0))
+    for qb in (3000, 40000):
+        ld = (qb + 1 + 3) // 4 * 4
+        row = np.zeros(ld, dtype=np.float32)
+        row[:qb + 1] = np.where(rng.random(qb + 1) < 0.05, hi, lo)
+        S = dev(row[None, :])
+        sel = torch.empty((1, budget), dtype=torch.int32, device="cuda")
+        cnt = torch.empty((1,), dtype=torch.int32, device="cuda")
+        qsa.qsa_select_blocks(p, S, ld, qb, qb + 1, sel, cnt, ws)
+        torch.cuda.synchronize()
+        assert qsa.qsa_check_device_error(ws) == 0
+        assert np.array_equal(sel.cpu().numpy()[0], _select_exact_cpu(row, qb, budget))
 
 
 @pytest.mark.parametrize("T,budget", [(256, 16), (256, 64), (1, 16), (7, 16), (301, 16), (2053, 64)])
