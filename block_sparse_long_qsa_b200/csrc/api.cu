@@ -166,24 +166,24 @@ qsa_status make_map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t
 
 // ----------------------------------------------------------------- tracing
 // Every kernel launch of the library is wrapped in an NVTX range named
-// "qsa/<kernel>" (free when no tool is attached; lets ncu --nvtx filter one
+// "qsa.<kernel>" (free when no tool is attached; lets ncu --nvtx filter one
 // stage of a step).  When tracing is enabled, each launch is also bracketed
 // by two CUDA events recorded on the launching stream.
 const char* nvtx_name(int32_t id) {
   switch (id) {
-    case QSA_KERNEL_ROPE_TABLE: return "qsa/rope_table";
-    case QSA_KERNEL_ROPE_K: return "qsa/rope_k";
-    case QSA_KERNEL_INDEXER: return "qsa/indexer";
-    case QSA_KERNEL_SELECT: return "qsa/select";
-    case QSA_KERNEL_ATTENTION: return "qsa/attention";
-    case QSA_KERNEL_DECODE_APPEND: return "qsa/decode_append";
-    case QSA_KERNEL_DECODE_INDEXER: return "qsa/decode_indexer";
-    case QSA_KERNEL_DECODE_ATTENTION: return "qsa/decode_attention";
-    case QSA_KERNEL_DECODE_COMBINE: return "qsa/decode_combine";
-    case QSA_KERNEL_KBAR: return "qsa/kbar";
-    case QSA_KERNEL_VERIFY_EXPAND: return "qsa/verify_expand";
-    case QSA_KERNEL_IDX_ROPE: return "qsa/idx_rope";
-    default: return "qsa/other";
+    case QSA_KERNEL_ROPE_TABLE: return "qsa.rope_table";
+    case QSA_KERNEL_ROPE_K: return "qsa.rope_k";
+    case QSA_KERNEL_INDEXER: return "qsa.indexer";
+    case QSA_KERNEL_SELECT: return "qsa.select";
+    case QSA_KERNEL_ATTENTION: return "qsa.attention";
+    case QSA_KERNEL_DECODE_APPEND: return "qsa.decode_append";
+    case QSA_KERNEL_DECODE_INDEXER: return "qsa.decode_indexer";
+    case QSA_KERNEL_DECODE_ATTENTION: return "qsa.decode_attention";
+    case QSA_KERNEL_DECODE_COMBINE: return "qsa.decode_combine";
+    case QSA_KERNEL_KBAR: return "qsa.kbar";
+    case QSA_KERNEL_VERIFY_EXPAND: return "qsa.verify_expand";
+    case QSA_KERNEL_IDX_ROPE: return "qsa.idx_rope";
+    default: return "qsa.other";
   }
 }
 
