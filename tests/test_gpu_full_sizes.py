@@ -144,12 +144,15 @@ def test_prefill_all_scores_tied_32k():
 
 
 @pytest.mark.timeout(1800)
-def test_prefill_mean_pool_1m_sampled():
-    """The mean-pooled indexer at 1M tokens, run as the benchmark runs it."""
+@pytest.mark.parametrize("rope", [0, 1])
+def test_prefill_mean_pool_1m_sampled(rope):
+    """The mean-pooled indexer at 1M tokens, run as the benchmark runs it;
+    rope = 1: with the indexer's RoPE (queries at their token, each compressed
+    key at its block's first token)."""
     T = 1048576
     P = Q.PrefillProblem(T=T, seed=0, n_plant=8, dist="zipf")
     d = P.device()
-    p = qsa.params(BUDGET, aggregation=qsa.AGG_MEAN_POOL)
+    p = qsa.params(BUDGET, aggregation=qsa.AGG_MEAN_POOL, idx_rope=rope)
     _, pref = qsa.qsa_prefill_workspace_size(p, T)
     ws = qsa.workspace(pref)
     nqb = P.nqb
@@ -162,10 +165,11 @@ def test_prefill_mean_pool_1m_sampled():
     assert qsa.qsa_check_device_error(ws) == 0
     del d, ws
     _check_selection_structure(sel, cnt)
-    O = oracle.Oracle(oracle.params(budget=BUDGET, aggregation=oracle.AGG_MEAN_POOL))
+    O = oracle.Oracle(oracle.params(budget=BUDGET, aggregation=oracle.AGG_MEAN_POOL, idx_rope=rope))
     qbs = _sample_blocks(nqb, seed=7, n=64)
-    n_diff = _check_sampled_blocks(O, P, qbs, sel, cnt, out, None, "mean pool 1M")
-    print(f"mean pool 1M: {len(qbs)} sampled query blocks, {n_diff} near-tie selection differences")
+    what = "mean pool 1M" + (" with RoPE" if rope else "")
+    n_diff = _check_sampled_blocks(O, P, qbs, sel, cnt, out, None, what)
+    print(f"{what}: {len(qbs)} sampled query blocks, {n_diff} near-tie selection differences")
 
 
 def _decode_full_setup(B, L, aggregation=0):
