@@ -116,7 +116,7 @@ def test_prefill_full_size_sampled(T, dist):
     _check_selection_structure(sel, cnt)
 
     O = oracle.Oracle(oracle.params(budget=BUDGET))
-    # 256 stratified query blocks at 1M (the survey's sample), 64 below
+    # 256 stratified query blocks at 1M (the stratified sample the CPU baseline times too), 64 below
     qbs = _sample_blocks(nqb, seed=T, n=256 if T >= 1 << 20 else 64)
     n_diff = _check_sampled_blocks(O, P, qbs, sel, cnt, out, lse, f"T={T}")
     print(f"T={T}: {len(qbs)} sampled query blocks, {n_diff} near-tie selection differences")
