@@ -193,7 +193,9 @@ def run_prefill(T: int, budget: int, steps: int, warmup: int, rank: int, world: 
     kern = tr.by_kernel()
     launches = sum(c for c, _ in kern.values())
     res = dict(ms=ms_max, tokens=T * steps * world, kern=kern, launches=launches, clocks=clk.summary(),
-               flops_idx=fl_idx, flops_attn=fl_attn, steps=steps)
+               flops_idx=fl_idx, flops_attn=fl_attn, steps=steps,
+               # K and V rows the attention gathers per step: 4 keys x 2 KV heads x 2 x 512 B per selected block
+               gather_bytes=float(cnt_h.astype(np.int64).sum()) * 8192.0)
 
     if want_e2e:
         # end to end through the public call with host buffers: pinned inputs
@@ -759,6 +761,14 @@ def line_for(name, res, n_gpus, steps, warmup, pk):
                     peak_src=f"{pk['src']} bf16 dense sustained")
         total_fl = res["flops_idx"] + res["flops_attn"]
         whole = dict(tflops=total_fl / (res["ms"] / res["steps"] / 1e3) / 1e12)
+        if "gather_bytes" in res and "attention" in res["kern"]:
+            # the attention against its own bound: gathered K / V bytes (L2 hits
+            # included) per second against the HBM copy bandwidth
+            att_s = res["kern"]["attention"][1] / res["steps"] / 1e3
+            gbs = res["gather_bytes"] / att_s / 1e9
+            whole["attention"] = dict(bound="hbm", gathered_gb_per_step=round(res["gather_bytes"] / 1e9, 2),
+                                      achieved_gbs=round(gbs, 1), frac_of_hbm=round(gbs / pk["hbm"], 4),
+                                      tflops=round(res["flops_attn"] / att_s / 1e12, 1))
         whole["frac_of_tensor_roofline"] = whole["tflops"] / pk["bf16_sus"]
         metric = metric_name(wl)
         cfg = dict(workload=name, T=T, batch=1, budget_blocks=512, heads="24q/2kv x 256, idx 4 x 128",
