@@ -308,6 +308,7 @@ def qsa_decode_noalloc_check_error(stream=None) -> int:
 INJECT_INDEXER_STALL = 1
 INJECT_ATTENTION_STALL = 2
 INJECT_ATTENTION_BAD_BLOCK = 3
+INJECT_ATTENTION_RESCALE_ALL = 4
 
 
 def qsa_debug_inject(code: int):

@@ -922,7 +922,7 @@ int take_debug_injection(int code) {
 }  // namespace qsa
 
 extern "C" qsa_status qsa_debug_inject(int32_t code) {
-  if (code < QSA_INJECT_NONE || code > QSA_INJECT_ATTENTION_BAD_BLOCK) return QSA_ERR_INVALID_ARG;
+  if (code < QSA_INJECT_NONE || code > QSA_INJECT_ATTENTION_RESCALE_ALL) return QSA_ERR_INVALID_ARG;
   qsa::g_debug_inject.store(code);
   return QSA_OK;
 }

@@ -557,7 +557,13 @@ __global__ void __launch_bounds__(THREADS, 1) sparse_attn_tc_kernel(const TcArgs
         float mt_other;
         if (!exchange(mt, mt_other)) { ok = false; break; }
         mt = fmaxf(mt, mt_other);
+#ifdef QSA_DEBUG_HOOKS
+        // test hook: no lazy margin, every tile takes the new maximum and
+        // rescales O (corr = 1 where the maximum did not grow)
+        const bool need = a.inject == QSA_INJECT_ATTENTION_RESCALE_ALL || mt > m_run + 8.f;
+#else
         const bool need = mt > m_run + 8.f;
+#endif
         if (__any_sync(0xffffffffu, need)) {
           const float m_new = need ? fmaxf(m_run, mt) : m_run;
           const float corr = ex2(m_run - m_new);
@@ -753,6 +759,7 @@ cudaError_t launch_sparse_attn_prefill_tc(int64_t T, const uint16_t* q, const ui
   a.err = err; a.n_split = 1;
   a.inject = take_debug_injection(QSA_INJECT_ATTENTION_STALL);
   if (a.inject == 0) a.inject = take_debug_injection(QSA_INJECT_ATTENTION_BAD_BLOCK);
+  if (a.inject == 0) a.inject = take_debug_injection(QSA_INJECT_ATTENTION_RESCALE_ALL);
   return launch_tc<false>(a, 2 * (qb_end - qb_begin), num_sms, stream);
 }
 
@@ -768,6 +775,7 @@ cudaError_t launch_decode_attn_tc(int B, int64_t max_len, const int64_t* L_dev, 
   a.qb_begin = 0; a.n_qb = B; a.scale_log2 = scale_log2; a.out = out; a.lse = lse; a.err = err;
   a.Ls = L_dev; a.max_len = max_len; a.rows_per_seq = rows_per_seq;
   a.n_split = n_split; a.part_o = part_o; a.part_lse = part_lse;
+  a.inject = take_debug_injection(QSA_INJECT_ATTENTION_RESCALE_ALL);
   return launch_tc<true>(a, 2 * (int64_t)B * n_split, num_sms, stream);
 }
 

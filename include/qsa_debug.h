@@ -13,8 +13,9 @@
  *     output's row range and leading dimension; a failed check records
  *     QSA_ERR_DEVICE_BOUNDS (read with qsa_check_device_error) and the access
  *     is skipped;
- *   - qsa_debug_inject arms one fault for the next launch of the kernel it
- *     names.  The faults make no out-of-range access and leave no wait
+ *   - qsa_debug_inject arms one fault (or, for QSA_INJECT_ATTENTION_RESCALE_ALL,
+ *     one change of schedule that leaves the result within rounding of the
+ *     normal one) for the next launch of the kernel it names.  The faults make no out-of-range access and leave no wait
  *     unbounded: a stall withholds one completion signal, so a waiting role
  *     times out, records QSA_ERR_DEVICE_TIMEOUT and the CTA drains what it
  *     issued and exits; a bad block names a block after the query block,
@@ -35,7 +36,10 @@ enum {
   QSA_INJECT_NONE = 0,
   QSA_INJECT_INDEXER_STALL = 1,        /* next indexer launch: CTA 0 never signals its first accumulator */
   QSA_INJECT_ATTENTION_STALL = 2,      /* next prefill attention launch: CTA 0 never signals its first S tile */
-  QSA_INJECT_ATTENTION_BAD_BLOCK = 3   /* next prefill attention launch: CTA 0's first gathered block is qb + 1 */
+  QSA_INJECT_ATTENTION_BAD_BLOCK = 3,  /* next prefill attention launch: CTA 0's first gathered block is qb + 1 */
+  QSA_INJECT_ATTENTION_RESCALE_ALL = 4 /* next attention launch (prefill or decode): the online softmax takes a
+                                          new running maximum, and rescales the accumulated output, on every tile
+                                          (no lazy margin), so that path runs on ordinary inputs */
 };
 
 /* Arms `code` for the next launch of the kernel it names (one launch; a new

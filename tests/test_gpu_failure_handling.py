@@ -120,6 +120,49 @@ def test_bounds_check_reports_non_causal_block(libs, problem):
     assert torch.equal(got["out"], want["out"])
 
 
+def test_attention_rescale_on_every_tile(libs):
+    """The online softmax's rescale of the accumulated output (taken only when
+    a tile's maximum exceeds the running one by more than 2^8, which unit-scale
+    inputs almost never reach) forced on every tile by the debug hook, in a
+    prefill with 32-tile rows and in a decode step: the outputs stay within the
+    acceptance bounds of the oracle (prefill, on the GPU's own selection) and
+    of the normal run (decode)."""
+    import oracle
+    from gpu_util import check_outputs
+    from test_gpu_decode import DecodeState
+    T, budget = 4096, 512
+    P = Q.PrefillProblem(T=T, seed=93, n_plant=8)
+    host = P.host()
+    t = {k: dev(v) for k, v in host.items()}
+
+    def run():
+        qsa.qsa_debug_inject(qsa.INJECT_ATTENTION_RESCALE_ALL)
+        return _prefill(t, budget)
+    rc, got = _with(qsa.LIB_DEBUG_PATH, run)
+    assert rc == 0
+    out, sel, cnt = got["out"].numpy(), got["sel"].numpy(), got["cnt"].numpy()
+    nqb = P.nqb
+    qbs = np.array(sorted({0, 1, budget - 1, budget, nqb - 1} | set(range(530, nqb, 41))), dtype=np.int64)
+    O = oracle.Oracle(oracle.params(budget=budget))
+    want, _ = O.attend_blocks(T, host["q"], host["k"], host["v"], qbs, sel[qbs], cnt[qbs])
+    rows = np.concatenate([np.arange(4 * q, min(4 * q + 4, T)) for q in qbs])
+    check_outputs(out[rows], want[:len(rows)], "prefill, rescale on every tile")
+
+    L_list = [2301, 4097]
+    probs = [Q.PrefillProblem(T=L + 1, seed=95 + b, n_plant=8) for b, L in enumerate(L_list)]
+
+    def step(inject):
+        st = DecodeState(probs, L_list, max_len=max(L_list) + 8, budget=budget)
+        if inject:
+            qsa.qsa_debug_inject(qsa.INJECT_ATTENTION_RESCALE_ALL)
+        return st.step()
+    _, o_ref, s_ref, _ = step(False)
+    _, o_dbg, s_dbg, _ = _with(qsa.LIB_DEBUG_PATH, lambda: step(True))
+    assert np.array_equal(s_ref, s_dbg)
+    for b in range(len(L_list)):
+        check_outputs(o_dbg[b], Q.bf16_to_f64(o_ref[b]), f"decode b={b}, rescale on every tile")
+
+
 def test_release_library_has_no_hooks(libs):
     with pytest.raises(RuntimeError):
         qsa.qsa_debug_inject(qsa.INJECT_INDEXER_STALL)
