@@ -826,6 +826,28 @@ def ncu_case(spec: str):
             qsa.qsa_index_scores(p, T, d["q_idx"], d["w"], d["k_idx"], nqb - rows, nqb, S, ld, ws)
         torch.cuda.synchronize()
         assert qsa.qsa_check_device_error(ws) == 0
+    elif parts[0] == "attntail":
+        # the prefill of the last `rows` query blocks of a T-token problem over
+        # the cached first T - 4 rows tokens (qsa_prefill_cached): the
+        # attention gathers from a T-token cache larger than L2, a few GB on
+        # the device; the full q is never generated (indexer keys unplanted)
+        T, rows = int(parts[1]), int(parts[2])
+        T_new = 4 * rows
+        L_old = T - T_new
+        P = Q.PrefillProblem(T=T, seed=0, n_plant=0, dist="zipf")
+        kc, vc, ic = (P.device_rows(n, 0, T) for n in ("k", "v", "k_idx"))
+        new = {n: P.device_rows(n, L_old, T) for n in ("q", "k", "v", "q_idx", "w", "k_idx")}
+        p = qsa.params(512)
+        _, pref = qsa.qsa_prefill_cached_workspace_size(p, L_old, T_new)
+        ws = qsa.workspace(pref)
+        out = torch.empty((T_new, 24, 256), dtype=torch.uint16, device="cuda")
+        sel = torch.empty((rows, 512), dtype=torch.int32, device="cuda")
+        cnt = torch.empty((rows,), dtype=torch.int32, device="cuda")
+        for _ in range(2):
+            qsa.qsa_prefill_cached(p, L_old, T_new, kc, vc, ic, None, None, new["q"], new["k"], new["v"],
+                                   new["q_idx"], new["w"], new["k_idx"], out, None, sel, cnt, ws)
+        torch.cuda.synchronize()
+        assert qsa.qsa_check_device_error(ws) == 0
     elif parts[0] == "index":
         # stage 1 alone (qsa_index_scores, no segment maxima), four launches
         T = int(parts[1])
@@ -874,7 +896,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--ncu-case", default=None,
-                    help="prefill:T, index:T, indextail:T:rows or decode:B:L -- a few calls of a small case "
+                    help="prefill:T, index:T, indextail:T:rows, attntail:T:rows or decode:B:L -- a few calls of a small case "
                          "(for ncu captures)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))

@@ -334,6 +334,26 @@ class PrefillProblem:
     def host(self) -> dict:
         return dict(q=self.q(), k=self.k(), v=self.v(), q_idx=self.q_idx(), w=self.w(), k_idx=self.k_idx())
 
+    def device_rows(self, name: str, t0: int, t1: int, device="cuda"):
+        """Rows [t0, t1) of one input generated on the GPU, bit-identical to the
+        host generator's rows -- except k_idx, whose planted blocks are not
+        applied here (use ``device()`` or ``k_idx()`` for those)."""
+        import torch
+        shapes = dict(q=(N_Q_HEADS, HEAD_DIM, S_Q), k=(N_KV_HEADS, HEAD_DIM, S_K), v=(N_KV_HEADS, HEAD_DIM, S_V),
+                      q_idx=(IDX_HEADS, IDX_DIM, S_QIDX), k_idx=(IDX_DIM, S_KIDX))
+        cs = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+        L = lib()
+        n = t1 - t0
+        if name == "w":
+            t = torch.empty((n, IDX_HEADS), dtype=torch.uint16, device=device)
+            _chk(L.qsagen_softmax4_bf16_dev(self.seed & MASK64, S_W, t0, n, t.data_ptr(), cs))
+            return t
+        *dims, st = shapes[name]
+        per = int(np.prod(dims))
+        t = torch.empty((n, *dims), dtype=torch.uint16, device=device)
+        _chk(L.qsagen_normal_bf16_dev(self.seed & MASK64, st, t0 * per, n * per, t.data_ptr(), cs))
+        return t
+
     def device(self, device="cuda", stream=None) -> dict:
         """Full tensors generated on the GPU (bit-identical to ``host()``)."""
         import torch
