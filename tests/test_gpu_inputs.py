@@ -30,3 +30,15 @@ def test_decode_caches_device_equals_host():
         assert np.array_equal(kc[b, :1000].cpu().numpy(), D.cache_k(b))
         assert np.array_equal(vc[b, :1000].cpu().numpy(), D.cache_v(b))
         assert np.array_equal(ic[b, :1000].cpu().numpy(), D.cache_kidx(b))
+
+
+def test_device_rows_equal_host_rows():
+    """Row ranges generated on the device (the profiling cases that never
+    build the whole query tensor) equal the host generator's rows; the
+    indexer keys there are the unplanted ones."""
+    P = Q.PrefillProblem(T=9000, seed=6, n_plant=0)
+    for name, (t0, t1) in (("q", (8000, 9000)), ("k", (0, 9000)), ("v", (123, 4567)), ("q_idx", (8192, 9000)),
+                           ("w", (7, 8999)), ("k_idx", (0, 9000))):
+        got = P.device_rows(name, t0, t1).cpu().numpy()
+        want = getattr(P, name)(t0, t1)
+        assert np.array_equal(got, want), name
